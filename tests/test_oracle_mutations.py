@@ -1,0 +1,77 @@
+"""Plant plausible mistakes in the oracle (CPU only) and check a pin catches each.
+
+This is evidence that the pins in ``test_oracle_pins`` are strong enough: a
+dropped term, a flipped sign, a transposed operand, a missing shift or a wrong
+damping convention must each make some pin fail.
+"""
+import numpy as np
+import pytest
+
+from oracle import cells, elk, newton, scan
+import tests.test_oracle_pins as pins
+
+
+def _fails(fn, *args):
+    with pytest.raises(AssertionError):
+        fn(*args)
+
+
+def test_flipped_sign_in_jacobian(monkeypatch):
+    orig = cells.GRU._row_scales
+
+    def bad(self, h, r, z, g, n):
+        cz, cn, cr = orig(self, h, r, z, g, n)
+        return -cz, cn, cr
+    monkeypatch.setattr(cells.GRU, "_row_scales", bad)
+    _fails(pins.test_jacobian_central_differences, "dense")
+
+
+def test_dropped_reset_gate_term(monkeypatch):
+    orig = cells.GRU._row_scales
+
+    def bad(self, h, r, z, g, n):
+        cz, cn, cr = orig(self, h, r, z, g, n)
+        return cz, cn, 0.0 * cr
+    monkeypatch.setattr(cells.GRU, "_row_scales", bad)
+    _fails(pins.test_jacobian_central_differences, "dense")
+    _fails(pins.test_jacobian_central_differences, "diag")
+
+
+def test_transposed_recurrent_block(monkeypatch):
+    orig = cells.GRU.U
+    monkeypatch.setattr(cells.GRU, "U", lambda self, gate: orig(self, gate).T)
+    _fails(pins.test_jacobian_central_differences, "dense")
+
+
+def test_reset_gate_before_bias(monkeypatch):
+    def bad(self, h, p):
+        d = self.d
+        q = self.recurrent(h) - self.b_hh
+        r = cells.sigmoid(p[..., 0:d] + q[..., 0:d] + self.b_hh[0:d])
+        z = cells.sigmoid(p[..., d:2 * d] + q[..., d:2 * d] + self.b_hh[d:2 * d])
+        g = q[..., 2 * d:]
+        n = np.tanh(p[..., 2 * d:] + r * g + self.b_hh[2 * d:])
+        return r, z, g, n, (1 - z) * n + z * h
+    monkeypatch.setattr(cells.GRU, "gates", bad)
+    _fails(pins.test_cell_equals_torch_grucell, "dense")
+
+
+def test_missing_shift(monkeypatch):
+    monkeypatch.setattr(newton, "shifted", lambda h, h0: h)
+    _fails(pins.test_undamped_newton_recovers_one_state_per_iteration, "QUASI")
+
+
+def test_transposed_dense_scan(monkeypatch):
+    orig = scan.affine_scan
+
+    def bad(A, b, h0):
+        A = np.asarray(A)
+        return orig(np.swapaxes(A, -1, -2) if A.ndim == 4 else A, b, h0)
+    monkeypatch.setattr(pins, "affine_scan", bad)
+    _fails(pins.test_scan_closed_forms_dense)
+
+
+def test_inverted_damping_convention(monkeypatch):
+    orig = elk.lm_step_normal
+    monkeypatch.setattr(elk, "lm_step_normal", lambda A, b, y, h0, lam: orig(A, b, y, h0, 1.0 / lam))
+    _fails(pins.test_lm_limits, False)
