@@ -1,0 +1,257 @@
+/*
+ * pararnn.h -- C ABI of the parallel-Newton GRU evaluator for NVIDIA B200 (sm_100a).
+ *
+ * The library evaluates a nonlinear recurrence h_t = f(h_{t-1}, x_t) (a GRU
+ * cell) over a whole sequence at once.  All T states are treated as the
+ * unknowns of one system of nonlinear equations, one per step, and solved
+ * with Newton iterations; each iteration solves the linearised, block
+ * bidiagonal system h_t = A_t h_{t-1} + b_t with a parallel scan over t.
+ *   - "ParaRNN: A Revolutionary Framework for Parallel Training of Nonlinear
+ *     RNNs", sections "Core Idea" and "Newton's Iteration";
+ *   - "Towards Scalable and Stable Parallelization of Nonlinear RNNs",
+ *     abstract (DEER as a fixed-point problem, quasi-Newton, ELK) and the atlas
+ *     summary, "Approach" (diagonal Jacobian; Levenberg-Marquardt step as a
+ *     parallel Kalman filter/smoother);
+ *   - "Parallelizing non-linear sequential models over the sequence length",
+ *     abstract (DEER).
+ *
+ * Conventions for every entry point
+ *   - Device pointers are CUDA device addresses of the current device; host
+ *     pointers are ordinary host memory.  Each argument says which it is.
+ *   - Arrays are dense, row-major and contiguous; device arrays start on a
+ *     16-byte boundary.
+ *   - The caller owns all memory, including the workspace.  The library
+ *     allocates no device or host memory and keeps no state between calls.
+ *   - Work is enqueued on `stream` (NULL means the legacy default stream).
+ *   - Return value: a pararnn_status code; pararnn_status_string() names it.
+ *     On PARARNN_INVALID_ARG nothing was enqueued.
+ */
+#ifndef PARARNN_H
+#define PARARNN_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define PARARNN_API __attribute__((visibility("default")))
+#else
+#define PARARNN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t.  Declared here so that the header needs no CUDA include. */
+struct CUstream_st;
+typedef struct CUstream_st *pararnn_stream;
+
+/* Solver modes ("Towards Scalable and Stable Parallelization of Nonlinear
+ * RNNs": abstract; atlas summary "Approach").
+ *   DEER      Newton with the full D x D Jacobian of the cell.
+ *   QUASI     quasi-DEER: the Jacobian replaced by its diagonal.
+ *   ELK       Newton with a Levenberg-Marquardt trust region, the damped step
+ *             computed as a Kalman filter + smoother (full Jacobian).
+ *   QUASI_ELK ELK with the diagonal Jacobian. */
+typedef enum {
+    PARARNN_DEER = 0,
+    PARARNN_QUASI = 1,
+    PARARNN_ELK = 2,
+    PARARNN_QUASI_ELK = 3
+} pararnn_mode;
+
+/* Cell kinds.  DENSE: the GRU with full recurrent matrices U_r, U_z, U_n.
+ * DIAG: the recurrent weights are elementwise vectors u_r, u_z, u_n, so the
+ * Jacobian is exactly diagonal and QUASI is exact Newton (the "adapted" GRU of
+ * the ParaRNN abstract). */
+typedef enum { PARARNN_GRU_DENSE = 0, PARARNN_GRU_DIAG = 1 } pararnn_cell_kind;
+
+typedef enum { PARARNN_F32 = 0, PARARNN_BF16 = 1 } pararnn_dtype;
+
+typedef enum {
+    PARARNN_OK = 0,             /* converged: max |h^(i+1) - h^(i)| <= tol        */
+    PARARNN_NOT_CONVERGED = 1,  /* max_iters reached; h holds the last iterate    */
+    PARARNN_DIVERGED = 2,       /* a non-finite value appeared; h holds that iterate */
+    PARARNN_INVALID_ARG = 3,    /* bad pointer, size, alignment, mode or workspace */
+    PARARNN_CUDA_ERROR = 4,     /* a CUDA runtime call failed                      */
+    PARARNN_TIMEOUT = 5         /* a bounded device-side wait expired (h unreliable) */
+} pararnn_status;
+
+/* The GRU cell.
+ *   din, d     input and state widths.  d must be a multiple of 4.
+ *   x_dtype    element type of x; w_dtype that of w_ih.  Both F32, or both BF16.
+ * Gates (rows of every [3D, .] array in the order r, z, n):
+ *   r = sigmoid(W_r x + b_ir + U_r h + b_hr),  z = sigmoid(W_z x + b_iz + U_z h + b_hz),
+ *   n = tanh(W_n x + b_in + r * (U_n h + b_hn)),  f = (1 - z) * n + z * h.          */
+typedef struct {
+    int kind;     /* pararnn_cell_kind */
+    int din;
+    int d;
+    int x_dtype;  /* pararnn_dtype */
+    int w_dtype;  /* pararnn_dtype */
+} pararnn_cell;
+
+/* Cell parameters, all DEVICE pointers.
+ *   w_ih  [3D, Din]  of w_dtype
+ *   b_ih  [3D]       float
+ *   w_hh  DENSE: [3D, D] float (U_r; U_z; U_n stacked by rows)
+ *         DIAG:  [3D]    float (u_r, u_z, u_n)
+ *   b_hh  [3D]       float                                                    */
+typedef struct {
+    const void *w_ih;
+    const float *b_ih;
+    const float *w_hh;
+    const float *b_hh;
+} pararnn_params;
+
+/* Per-solve report, written to DEVICE memory by pararnn_newton_solve_async
+ * (and copied to the host by pararnn_newton_solve). */
+typedef struct {
+    int iters;          /* linear solves performed                                */
+    int status;         /* PARARNN_OK / NOT_CONVERGED / DIVERGED / TIMEOUT        */
+    float delta;        /* max |h^(iters) - h^(iters-1)|                           */
+    float residual;     /* max |h_t - f(h_{t-1}, x_t)| at the last linearisation   */
+} pararnn_info;
+
+/*
+ * pararnn_workspace_size -- bytes of device workspace pararnn_newton_solve needs.
+ * Returns 0 for arguments pararnn_newton_solve would reject.
+ */
+PARARNN_API size_t pararnn_workspace_size(const pararnn_cell *cell, int B, int T, int mode);
+
+/*
+ * pararnn_newton_solve -- evaluate the GRU over B sequences of length T by
+ * (quasi-)Newton / (quasi-)ELK iterations, and wait for the result.
+ *
+ * Method ("ParaRNN" summary, "Core Idea" and "Newton's Iteration";
+ * "Towards Scalable and Stable Parallelization of Nonlinear RNNs", abstract
+ * and atlas summary "Approach"):
+ *   unknowns h_1..h_T per sequence, residual r_t = h_t - f(h_{t-1}, x_t),
+ *   h_0 = h0 fixed; initial guess h^(0) = 0.
+ *   Iteration i linearises f at the shifted guess h^(i)_{t-1}:
+ *     A_t = df/dh (DEER, ELK) or its diagonal (QUASI, QUASI_ELK),
+ *     b_t = f(h^(i)_{t-1}, x_t) - A_t h^(i)_{t-1};
+ *   DEER / QUASI:   h^(i+1) solves h_t = A_t h_{t-1} + b_t (parallel scan);
+ *   ELK / QUASI_ELK: h^(i+1) minimises
+ *       sum_t |h_t - A_t h_{t-1} - b_t|^2 + lambda sum_t |h_t - h^(i)_t|^2
+ *     (Kalman filter + RTS smoother with process noise I, observation noise
+ *     I / lambda, observations h^(i)).
+ *   Stop when delta = max_{b,t,d} |h^(i+1) - h^(i)| <= tol (iters = i + 1),
+ *   when a value is non-finite (DIVERGED), or after max_iters iterations.
+ *
+ * Arguments
+ *   cell, params   the GRU (host struct; params holds device pointers).
+ *   x              DEVICE [B, T, Din] of cell->x_dtype; x[:, 0] is x_1.
+ *   h0             DEVICE [B, D] float.
+ *   B, T           batch and sequence length, B >= 1, T >= 1.
+ *   mode           pararnn_mode.  The DIAG cell has a diagonal Jacobian, so
+ *                  DEER equals QUASI and ELK equals QUASI_ELK for it.
+ *   lambda         LM damping (> 0) for ELK / QUASI_ELK; ignored otherwise.
+ *   tol            convergence threshold on max |dh| (>= 0).
+ *   max_iters      iteration cap; <= 0 means T.
+ *   h              DEVICE [B, T, D] float, output (the final iterate; h[:, t]
+ *                  is h_{t+1}).  Must not alias any input or the workspace.
+ *   info           HOST pararnn_info, output; may be NULL.
+ *   workspace      DEVICE, at least pararnn_workspace_size(cell, B, T, mode)
+ *                  bytes, 256-byte aligned, not used by anything else while the
+ *                  solve runs.  Its contents on entry do not matter.
+ *   stream         stream to enqueue on.  The call synchronises this stream
+ *                  once, at the end, to read the report.
+ * Returns pararnn_status (the solve's own status, or INVALID_ARG / CUDA_ERROR).
+ * Limits: DENSE cells need d <= 64 (recurrent matrices are kept on chip).
+ */
+PARARNN_API int pararnn_newton_solve(const pararnn_cell *cell, const pararnn_params *params,
+                         const void *x, const float *h0, int B, int T, int mode,
+                         float lambda, float tol, int max_iters, float *h,
+                         pararnn_info *info, void *workspace, size_t ws_bytes,
+                         pararnn_stream stream);
+
+/*
+ * pararnn_newton_solve_async -- the same solve without any host synchronisation.
+ * The report is written to `info_dev` (DEVICE pararnn_info) when the last
+ * kernel finishes.  Returns PARARNN_OK if everything was enqueued (the solve's
+ * own status is info_dev->status), else INVALID_ARG / CUDA_ERROR.
+ */
+PARARNN_API int pararnn_newton_solve_async(const pararnn_cell *cell, const pararnn_params *params,
+                               const void *x, const float *h0, int B, int T, int mode,
+                               float lambda, float tol, int max_iters, float *h,
+                               pararnn_info *info_dev, void *workspace, size_t ws_bytes,
+                               pararnn_stream stream);
+
+/*
+ * pararnn_input_projection -- P = x W_ih^T + b_ih for every (b, t): the input
+ * pre-activations, which do not depend on the state and so are computed once
+ * per solve (as one GEMM [B*T, Din] x [Din, 3D]).  pararnn_newton_solve runs
+ * this first; calling it separately lets a caller reuse P across solves (for
+ * example a sweep over the ELK damping lambda, which the quasi-ELK method
+ * needs: "Towards Scalable and Stable Parallelization of Nonlinear RNNs",
+ * atlas summary "Limitations").
+ *   x   DEVICE [B, T, Din] of cell->x_dtype;  params->w_ih, params->b_ih used.
+ *   P   DEVICE float [B, T, 3D] output, gate-major rows (r, z, n).
+ * Asynchronous.  Returns PARARNN_OK, INVALID_ARG or CUDA_ERROR.
+ */
+PARARNN_API int pararnn_input_projection(const pararnn_cell *cell, const pararnn_params *params,
+                                         const void *x, int B, int T, float *P,
+                                         pararnn_stream stream);
+
+/*
+ * pararnn_newton_iterate_async -- the Newton loop of pararnn_newton_solve_async
+ * on precomputed pre-activations P (from pararnn_input_projection): every
+ * iteration, the cell and its Jacobian at the shifted guess, the parallel
+ * linear solve, and the on-device convergence test, until it stops.
+ *   P           DEVICE float [B, T, 3D]; not modified.
+ *   other arguments as pararnn_newton_solve_async; params->w_ih is not read.
+ *   workspace   pararnn_workspace_size(cell, B, T, mode) bytes (its
+ *               projection section is left unused).
+ * Asynchronous; the report goes to info_dev.
+ */
+PARARNN_API int pararnn_newton_iterate_async(const pararnn_cell *cell,
+                                             const pararnn_params *params, const float *P,
+                                             const float *h0, int B, int T, int mode,
+                                             float lambda, float tol, int max_iters, float *h,
+                                             pararnn_info *info_dev, void *workspace,
+                                             size_t ws_bytes, pararnn_stream stream);
+
+/*
+ * pararnn_affine_scan_workspace_size -- bytes of device workspace that
+ * pararnn_affine_scan needs for these sizes (0 if they would be rejected).
+ */
+PARARNN_API size_t pararnn_affine_scan_workspace_size(int B, int T, int D, int dense);
+
+/*
+ * pararnn_affine_scan -- solve the linear recurrence h_t = A_t h_{t-1} + b_t,
+ * t = 1..T, h_0 = h0, for B independent sequences, as a single-pass parallel
+ * scan over t (the linear solve inside each Newton iteration; "ParaRNN"
+ * summary, "Newton's Iteration"; "Towards Scalable and Stable Parallelization
+ * of Nonlinear RNNs", atlas summary "Builds on": parallel associative scan).
+ *
+ *   A      DEVICE float.  dense == 0: [B, T, D], A_t acts elementwise.
+ *                         dense != 0: [B, T, D, D], row-major matrices.
+ *   b      DEVICE float [B, T, D].
+ *   h0     DEVICE float [B, D].
+ *   h      DEVICE float [B, T, D], output.  May alias b (not A or h0).
+ *   workspace  DEVICE, >= pararnn_affine_scan_workspace_size(B, T, D, dense)
+ *              bytes, 256-byte aligned.  Contents on entry do not matter.
+ *   D must be a multiple of 4; dense needs D <= 64.
+ * Fully asynchronous.  Returns PARARNN_OK, INVALID_ARG or CUDA_ERROR; a
+ * bounded device wait that expired is reported through the next call of
+ * pararnn_affine_scan_status().
+ */
+PARARNN_API int pararnn_affine_scan(const float *A, const float *b, const float *h0, int B, int T,
+                        int D, int dense, float *h, void *workspace, size_t ws_bytes,
+                        pararnn_stream stream);
+
+/*
+ * pararnn_affine_scan_status -- read (and wait for) the device status word the
+ * last pararnn_affine_scan using `workspace` wrote: PARARNN_OK or
+ * PARARNN_TIMEOUT.  Synchronises `stream`.
+ */
+PARARNN_API int pararnn_affine_scan_status(const void *workspace, pararnn_stream stream);
+
+/* pararnn_status_string -- a static, human-readable name of a status code. */
+PARARNN_API const char *pararnn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PARARNN_H */

@@ -1,0 +1,243 @@
+"""Thin ctypes binding of ``libpararnn.so`` (the C ABI in ``include/pararnn.h``).
+
+Argument marshalling only: every step of the solve runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current stream.  There is no
+CPU path: if the library is missing or a tensor is not on a CUDA device, the
+call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpararnn.so")
+
+DEER, QUASI, ELK, QUASI_ELK = 0, 1, 2, 3
+MODES = {"DEER": DEER, "QUASI": QUASI, "ELK": ELK, "QUASI_ELK": QUASI_ELK}
+GRU_DENSE, GRU_DIAG = 0, 1
+F32, BF16 = 0, 1
+STATUS = {0: "OK", 1: "NOT_CONVERGED", 2: "DIVERGED", 3: "INVALID_ARG", 4: "CUDA_ERROR",
+          5: "TIMEOUT"}
+EXPORTS = ("pararnn_workspace_size", "pararnn_newton_solve", "pararnn_newton_solve_async",
+           "pararnn_input_projection", "pararnn_newton_iterate_async",
+           "pararnn_affine_scan_workspace_size", "pararnn_affine_scan",
+           "pararnn_affine_scan_status", "pararnn_status_string")
+
+
+class Cell(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int), ("din", ctypes.c_int), ("d", ctypes.c_int),
+                ("x_dtype", ctypes.c_int), ("w_dtype", ctypes.c_int)]
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("w_ih", ctypes.c_void_p), ("b_ih", ctypes.c_void_p),
+                ("w_hh", ctypes.c_void_p), ("b_hh", ctypes.c_void_p)]
+
+
+class Info(ctypes.Structure):
+    _fields_ = [("iters", ctypes.c_int), ("status", ctypes.c_int),
+                ("delta", ctypes.c_float), ("residual", ctypes.c_float)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library once; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"{_LIB_PATH} is missing: build it with `python -m newton_solve_nonlinear_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, ci, cf, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.pararnn_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci, ci]
+        L.pararnn_workspace_size.restype = sz
+        solve_args = [ctypes.POINTER(Cell), ctypes.POINTER(Params), vp, vp, ci, ci, ci, cf, cf, ci,
+                      vp, vp, vp, sz, vp]
+        L.pararnn_newton_solve.argtypes = solve_args
+        L.pararnn_newton_solve.restype = ci
+        L.pararnn_newton_solve_async.argtypes = solve_args
+        L.pararnn_newton_solve_async.restype = ci
+        L.pararnn_input_projection.argtypes = [ctypes.POINTER(Cell), ctypes.POINTER(Params), vp, ci,
+                                               ci, vp, vp]
+        L.pararnn_input_projection.restype = ci
+        L.pararnn_newton_iterate_async.argtypes = solve_args
+        L.pararnn_newton_iterate_async.restype = ci
+        L.pararnn_affine_scan_workspace_size.argtypes = [ci, ci, ci, ci]
+        L.pararnn_affine_scan_workspace_size.restype = sz
+        L.pararnn_affine_scan.argtypes = [vp, vp, vp, ci, ci, ci, ci, vp, vp, sz, vp]
+        L.pararnn_affine_scan.restype = ci
+        L.pararnn_affine_scan_status.argtypes = [vp, vp]
+        L.pararnn_affine_scan_status.restype = ci
+        L.pararnn_status_string.argtypes = [ci]
+        L.pararnn_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return F32
+    if t == torch.bfloat16:
+        return BF16
+    raise TypeError(f"unsupported dtype {t}")
+
+
+def _dev(t: torch.Tensor, name: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def make_cell(kind: str, din: int, d: int, dtype: torch.dtype) -> Cell:
+    return Cell(GRU_DENSE if kind == "dense" else GRU_DIAG, din, d, _dtype_code(dtype),
+                _dtype_code(dtype))
+
+
+def workspace_size(kind: str, din: int, d: int, B: int, T: int, mode: str,
+                   dtype: torch.dtype = torch.float32) -> int:
+    cell = make_cell(kind, din, d, dtype)
+    return int(lib().pararnn_workspace_size(ctypes.byref(cell), B, T, MODES[mode]))
+
+
+def alloc_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A 256-byte aligned device buffer of at least ``nbytes`` bytes."""
+    buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device or "cuda")
+    off = (-buf.data_ptr()) % 256
+    return buf[off:off + nbytes]
+
+
+@dataclass
+class SolveResult:
+    h: torch.Tensor
+    iters: int
+    status: str
+    delta: float
+    residual: float
+
+
+def newton_solve(w_ih, b_ih, w_hh, b_hh, x, h0, *, kind: str, mode: str, tol: float,
+                 lam: float = 0.0, max_iters: int = 0, out=None, workspace=None,
+                 stream=None, sync: bool = True, info_dev=None):
+    """Evaluate the GRU over x [B, T, Din] with the chosen Newton mode.
+
+    All tensors must be contiguous CUDA tensors (x and w_ih fp32 or bf16, the
+    rest fp32).  With ``sync`` the call waits and returns a SolveResult; with
+    ``sync=False`` it only enqueues, writing the report into ``info_dev`` (an
+    int32 CUDA tensor of 4 elements) and returns ``out``."""
+    B, T, din = x.shape
+    d = h0.shape[1]
+    cell = make_cell(kind, din, d, x.dtype)
+    if w_ih.dtype != x.dtype:
+        raise TypeError("x and w_ih must have the same dtype")
+    L = lib()
+    m = MODES[mode]
+    need = int(L.pararnn_workspace_size(ctypes.byref(cell), B, T, m))
+    if need == 0:
+        raise ValueError("arguments rejected by pararnn_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, x.device)
+    if out is None:
+        out = torch.empty(B, T, d, dtype=torch.float32, device=x.device)
+    params = Params(_dev(w_ih, "w_ih"), _dev(b_ih, "b_ih"), _dev(w_hh, "w_hh"), _dev(b_hh, "b_hh"))
+    args = (ctypes.byref(cell), ctypes.byref(params), _dev(x, "x"), _dev(h0, "h0"), B, T, m,
+            float(lam), float(tol), int(max_iters), _dev(out, "out"))
+    if sync:
+        info = Info()
+        rc = L.pararnn_newton_solve(*args, ctypes.byref(info), _dev(workspace, "workspace"),
+                                    workspace.numel(), _stream(stream))
+        if rc in (3, 4):
+            raise RuntimeError(f"pararnn_newton_solve: {L.pararnn_status_string(rc).decode()}")
+        return SolveResult(out, info.iters, STATUS[info.status], info.delta, info.residual)
+    if info_dev is None:
+        raise ValueError("sync=False needs info_dev (int32 CUDA tensor with 4 elements)")
+    rc = L.pararnn_newton_solve_async(*args, _dev(info_dev, "info_dev"),
+                                      _dev(workspace, "workspace"), workspace.numel(),
+                                      _stream(stream))
+    if rc != 0:
+        raise RuntimeError(f"pararnn_newton_solve_async: {L.pararnn_status_string(rc).decode()}")
+    return out
+
+
+def input_projection(x, w_ih, b_ih, *, d: int, kind: str = "dense", out=None, stream=None):
+    """P = x W_ih^T + b_ih for every step: x [B,T,Din] -> P [B,T,3D] fp32."""
+    B, T, din = x.shape
+    cell = make_cell(kind, din, d, x.dtype)
+    if out is None:
+        out = torch.empty(B, T, 3 * d, dtype=torch.float32, device=x.device)
+    params = Params(_dev(w_ih, "w_ih"), _dev(b_ih, "b_ih"), 0, 0)
+    rc = lib().pararnn_input_projection(ctypes.byref(cell), ctypes.byref(params), _dev(x, "x"),
+                                        B, T, _dev(out, "out"), _stream(stream))
+    if rc != 0:
+        raise RuntimeError(f"pararnn_input_projection: {STATUS.get(rc, rc)}")
+    return out
+
+
+def newton_iterate(P, w_hh, b_hh, h0, *, kind: str, din: int, mode: str, tol: float,
+                   info_dev, lam: float = 0.0, max_iters: int = 0, out=None, workspace=None,
+                   dtype=torch.float32, stream=None):
+    """Enqueue the Newton loop on precomputed P [B,T,3D]; report into info_dev."""
+    B, T, _ = P.shape
+    d = h0.shape[1]
+    cell = make_cell(kind, din, d, dtype)
+    L = lib()
+    m = MODES[mode]
+    if workspace is None:
+        workspace = alloc_workspace(int(L.pararnn_workspace_size(ctypes.byref(cell), B, T, m)),
+                                    P.device)
+    if out is None:
+        out = torch.empty(B, T, d, dtype=torch.float32, device=P.device)
+    params = Params(0, 0, _dev(w_hh, "w_hh"), _dev(b_hh, "b_hh"))
+    rc = L.pararnn_newton_iterate_async(ctypes.byref(cell), ctypes.byref(params), _dev(P, "P"),
+                                        _dev(h0, "h0"), B, T, m, float(lam), float(tol),
+                                        int(max_iters), _dev(out, "out"), _dev(info_dev, "info"),
+                                        _dev(workspace, "workspace"), workspace.numel(),
+                                        _stream(stream))
+    if rc != 0:
+        raise RuntimeError(f"pararnn_newton_iterate_async: {STATUS.get(rc, rc)}")
+    return out
+
+
+def solve_workload(w, mode: str, *, lam: float = 0.0, tol=None, max_iters: int = 0,
+                   device="cuda", **kw) -> SolveResult:
+    """Move a ``inputs.Workload`` to the device and solve it."""
+    dev = lambda t: t.to(device).contiguous()
+    return newton_solve(dev(w.w_ih), dev(w.b_ih), dev(w.w_hh), dev(w.b_hh), dev(w.x), dev(w.h0),
+                        kind=w.kind, mode=mode, tol=w.tol if tol is None else tol, lam=lam,
+                        max_iters=max_iters, **kw)
+
+
+def affine_scan(A, b, h0, *, out=None, workspace=None, stream=None, check: bool = False):
+    """h_t = A_t h_{t-1} + b_t over t for every sequence.  A is [B,T,D]
+    (diagonal) or [B,T,D,D] (dense); b [B,T,D]; h0 [B,D]; all fp32 CUDA."""
+    B, T, D = b.shape
+    dense = 1 if A.dim() == 4 else 0
+    L = lib()
+    need = int(L.pararnn_affine_scan_workspace_size(B, T, D, dense))
+    if need == 0:
+        raise ValueError("arguments rejected by pararnn_affine_scan_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, b.device)
+    if out is None:
+        out = torch.empty_like(b)
+    rc = L.pararnn_affine_scan(_dev(A, "A"), _dev(b, "b"), _dev(h0, "h0"), B, T, D, dense,
+                               _dev(out, "out"), _dev(workspace, "workspace"), workspace.numel(),
+                               _stream(stream))
+    if rc != 0:
+        raise RuntimeError(f"pararnn_affine_scan: {L.pararnn_status_string(rc).decode()}")
+    if check:
+        st = L.pararnn_affine_scan_status(_dev(workspace, "workspace"), _stream(stream))
+        if st != 0:
+            raise RuntimeError(f"pararnn_affine_scan: {STATUS.get(st, st)}")
+    return out

@@ -1,0 +1,662 @@
+// newton_diag.cu -- persistent solver for the diagonal-Jacobian family:
+//   quasi-DEER on the dense GRU, exact Newton (DEER == quasi-DEER) on the
+//   diagonal-recurrence GRU, and quasi-ELK on either cell.
+//
+// Method: "Towards Scalable and Stable Parallelization of Nonlinear RNNs"
+// (abstract; atlas summary "Approach": diagonal Jacobian, O(TD) work and
+// memory per iteration; LM damping solved as a parallel Kalman filter and
+// smoother) on the unrolled system of the ParaRNN summary ("Core Idea",
+// "Newton's Iteration").
+//
+// One cooperative launch runs the whole Newton loop.  Per iteration every CTA
+// walks its share of tiles; a tile is (sequence b, a group of DG state lanes,
+// a chunk of L time steps).  Inside a tile each thread owns TK consecutive
+// steps of 4 adjacent lanes (float4 accesses along D, coalesced across the
+// warp), so:
+//   1. the cell is evaluated at the shifted guess for all of the tile's states
+//      at once (the guess is known, so this part has no sequential dependence);
+//      for the dense cell the recurrent product U h_{t-1} is computed from a
+//      shared-memory copy of the tile's guess rows and of U, in fp32 FMAs so
+//      the fixed point is the fp32 rollout's;
+//   2. each thread composes its TK affine maps (a_t, b_t) per lane in
+//      registers, a shared-memory pass turns these into exclusive prefixes
+//      across the tile's thread rows, and one thread per lane resolves the
+//      tile's carry-in with a decoupled look-back over earlier chunks of the
+//      same lanes (single pass over HBM);
+//   3. the states are re-swept from the carry, written once, and the max of
+//      |h^(i+1) - h^(i)| (and of the residual) is reduced to one atomicMax per
+//      CTA.
+// A bounded grid barrier closes the iteration; every CTA reads the same
+// reduced delta and stops together.  quasi-ELK runs a forward pass (scalar
+// Kalman covariance as a 2x2 Mobius scan, then the filtered mean as an affine
+// scan) and a backward pass (RTS smoother as a reverse affine scan), each
+// single-pass with look-back, separated by a grid barrier.
+#include <cstdio>
+
+#include "common.cuh"
+#include "lookback.cuh"
+#include "solver.cuh"
+
+namespace pararnn {
+
+Tiling make_tiling(int B, int T, int D, bool dense_cell) {
+    Tiling t{};
+    t.DG = dense_cell ? D : (D < 64 ? D : 64);
+    t.DB = t.DG / 4;
+    t.NTB = kThreads / t.DB;
+    t.TK = 4;
+    t.L = t.NTB * t.TK;
+    t.n_dgroups = (D + t.DG - 1) / t.DG;
+    t.n_groups = B * t.n_dgroups;
+    t.n_chunks = (T + t.L - 1) / t.L;
+    t.n_tiles = static_cast<long long>(t.n_groups) * t.n_chunks;
+    return t;
+}
+
+namespace {
+
+constexpr int TK = 4;
+
+struct TileCoord {
+    long long tile;
+    int chunk, b, dg, db, tb, lane0, d0, t0, tile_t0;
+    bool active, dvalid;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(const DiagArgs &A, long long tile) {
+    TileCoord c;
+    const Tiling &tl = A.tl;
+    c.tile = tile;
+    c.chunk = static_cast<int>(tile / tl.n_groups);
+    const int grp = static_cast<int>(tile % tl.n_groups);
+    c.b = grp / tl.n_dgroups;
+    c.dg = grp % tl.n_dgroups;
+    c.db = threadIdx.x % tl.DB;
+    c.tb = threadIdx.x / tl.DB;
+    c.active = c.tb < tl.NTB;
+    c.lane0 = c.db * 4;
+    c.d0 = c.dg * tl.DG + c.lane0;
+    c.dvalid = c.active && c.d0 < A.D;
+    c.tile_t0 = c.chunk * tl.L;
+    c.t0 = c.tile_t0 + c.tb * TK;
+    return c;
+}
+
+// Shared memory carve-up (floats).
+struct Smem {
+    float *Us;    // dense: [D][3][DG]
+    float *hs;    // dense: [L+1][D]   guess rows tile_t0-1 .. tile_t0+L-1
+    float *s0, *s1, *s2, *s3;  // [NTB][DG] scan scratch
+    float *c0, *c1;            // [DG] carries
+    unsigned *red;             // [32]
+};
+
+__host__ __device__ inline size_t smem_floats(const Tiling &tl, int D, bool dense) {
+    size_t n = 0;
+    if (dense) n += static_cast<size_t>(D) * 3 * tl.DG + static_cast<size_t>(tl.L + 1) * D;
+    n += 4 * static_cast<size_t>(tl.NTB) * tl.DG + 2 * tl.DG + 32;
+    return n;
+}
+
+__device__ __forceinline__ Smem carve(float *base, const Tiling &tl, int D, bool dense) {
+    Smem s;
+    float *p = base;
+    s.Us = p;
+    s.hs = p;
+    if (dense) {
+        s.Us = p;
+        p += static_cast<size_t>(D) * 3 * tl.DG;
+        s.hs = p;
+        p += static_cast<size_t>(tl.L + 1) * D;
+    }
+    const size_t n = static_cast<size_t>(tl.NTB) * tl.DG;
+    s.s0 = p; p += n;
+    s.s1 = p; p += n;
+    s.s2 = p; p += n;
+    s.s3 = p; p += n;
+    s.c0 = p; p += tl.DG;
+    s.c1 = p; p += tl.DG;
+    s.red = reinterpret_cast<unsigned *>(p);
+    return s;
+}
+
+// ---------------------------------------------------------------------------
+// 1. linearisation at the shifted guess
+// ---------------------------------------------------------------------------
+// Produces, for the thread's TK x 4 states: a (diag of the Jacobian), bb
+// (f - a h_{t-1}) and y (the guess at t).  Steps past T or lanes past D get
+// the identity map (a = 1, bb = 0).
+template <bool DENSE>
+__device__ __forceinline__ void linearise(const DiagArgs &A, const TileCoord &c, const Smem &sm,
+                                          const float *hold, bool zero_guess, float (&a)[TK][4],
+                                          float (&bb)[TK][4], float (&y)[TK][4], unsigned &rmax) {
+    const int D = A.D, T = A.T;
+    const size_t rowP = 3 * static_cast<size_t>(D);
+    float hp[TK + 1][4];
+    float G[3][TK][4];
+    if (DENSE) {
+        // guess rows tile_t0-1 .. tile_t0+L-1 into shared memory (row 0 may be h0)
+        const int L = A.tl.L, nq = D / 4, nvec = (L + 1) * nq;
+        for (int i = threadIdx.x; i < nvec; i += kThreads) {
+            const int r = i / nq, col = (i % nq) * 4;
+            const int t = c.tile_t0 - 1 + r;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (t < 0)
+                v = __ldg(reinterpret_cast<const float4 *>(A.h0 + static_cast<size_t>(c.b) * D + col));
+            else if (!zero_guess && t < T)
+                v = ldcg4(hold + (static_cast<size_t>(c.b) * T + t) * D + col);
+            *reinterpret_cast<float4 *>(sm.hs + static_cast<size_t>(r) * D + col) = v;
+        }
+        __syncthreads();
+        if (c.active) {
+#pragma unroll
+            for (int k = 0; k <= TK; ++k) {
+                const float4 v = *reinterpret_cast<const float4 *>(sm.hs + static_cast<size_t>(c.tb * TK + k) * D + c.d0);
+                hp[k][0] = v.x; hp[k][1] = v.y; hp[k][2] = v.z; hp[k][3] = v.w;
+            }
+#pragma unroll
+            for (int g = 0; g < 3; ++g)
+#pragma unroll
+                for (int k = 0; k < TK; ++k)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) G[g][k][j] = 0.f;
+            const int DG = A.tl.DG;
+            for (int m = 0; m < D; m += 4) {
+                float4 hv[TK];
+#pragma unroll
+                for (int k = 0; k < TK; ++k)
+                    hv[k] = *reinterpret_cast<const float4 *>(sm.hs + static_cast<size_t>(c.tb * TK + k) * D + m);
+#pragma unroll
+                for (int mm = 0; mm < 4; ++mm) {
+                    const float4 u0 = *reinterpret_cast<const float4 *>(sm.Us + ((m + mm) * 3 + 0) * DG + c.lane0);
+                    const float4 u1 = *reinterpret_cast<const float4 *>(sm.Us + ((m + mm) * 3 + 1) * DG + c.lane0);
+                    const float4 u2 = *reinterpret_cast<const float4 *>(sm.Us + ((m + mm) * 3 + 2) * DG + c.lane0);
+#pragma unroll
+                    for (int k = 0; k < TK; ++k) {
+                        const float h = get(hv[k], mm);
+                        G[0][k][0] = fmaf(u0.x, h, G[0][k][0]);
+                        G[0][k][1] = fmaf(u0.y, h, G[0][k][1]);
+                        G[0][k][2] = fmaf(u0.z, h, G[0][k][2]);
+                        G[0][k][3] = fmaf(u0.w, h, G[0][k][3]);
+                        G[1][k][0] = fmaf(u1.x, h, G[1][k][0]);
+                        G[1][k][1] = fmaf(u1.y, h, G[1][k][1]);
+                        G[1][k][2] = fmaf(u1.z, h, G[1][k][2]);
+                        G[1][k][3] = fmaf(u1.w, h, G[1][k][3]);
+                        G[2][k][0] = fmaf(u2.x, h, G[2][k][0]);
+                        G[2][k][1] = fmaf(u2.y, h, G[2][k][1]);
+                        G[2][k][2] = fmaf(u2.z, h, G[2][k][2]);
+                        G[2][k][3] = fmaf(u2.w, h, G[2][k][3]);
+                    }
+                }
+            }
+        }
+    } else if (c.dvalid) {
+#pragma unroll
+        for (int k = 0; k <= TK; ++k) {
+            const int t = c.t0 - 1 + k;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (t < 0)
+                v = __ldg(reinterpret_cast<const float4 *>(A.h0 + static_cast<size_t>(c.b) * D + c.d0));
+            else if (!zero_guess && t < T)
+                v = ldcg4(hold + (static_cast<size_t>(c.b) * T + t) * D + c.d0);
+            hp[k][0] = v.x; hp[k][1] = v.y; hp[k][2] = v.z; hp[k][3] = v.w;
+        }
+    }
+
+    // per-lane constants: recurrent biases and the diagonal of each U_g
+    float bh[3][4], ud[3][4];
+    if (c.dvalid) {
+#pragma unroll
+        for (int g = 0; g < 3; ++g) {
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(A.b_hh + g * D + c.d0));
+            bh[g][0] = v.x; bh[g][1] = v.y; bh[g][2] = v.z; bh[g][3] = v.w;
+            if (DENSE) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    ud[g][j] = sm.Us[((c.d0 + j) * 3 + g) * A.tl.DG + c.lane0 + j];
+            } else {
+                const float4 u = __ldg(reinterpret_cast<const float4 *>(A.w_hh + g * D + c.d0));
+                ud[g][0] = u.x; ud[g][1] = u.y; ud[g][2] = u.z; ud[g][3] = u.w;
+            }
+        }
+    }
+
+#pragma unroll
+    for (int k = 0; k < TK; ++k) {
+        const int t = c.t0 + k;
+        const bool valid = c.dvalid && t < T;
+        float4 pv[3];
+        if (valid) {
+            const float *prow = A.P + (static_cast<size_t>(c.b) * T + t) * rowP + c.d0;
+#pragma unroll
+            for (int g = 0; g < 3; ++g) pv[g] = __ldg(reinterpret_cast<const float4 *>(prow + g * D));
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (!valid) {
+                a[k][j] = 1.f;
+                bb[k][j] = 0.f;
+                y[k][j] = 0.f;
+                continue;
+            }
+            const float h = hp[k][j];
+            const float gr = DENSE ? G[0][k][j] : ud[0][j] * h;
+            const float gz = DENSE ? G[1][k][j] : ud[1][j] * h;
+            const float gnh = DENSE ? G[2][k][j] : ud[2][j] * h;
+            const float r = sigmoidf_(get(pv[0], j) + gr + bh[0][j]);
+            const float z = sigmoidf_(get(pv[1], j) + gz + bh[1][j]);
+            const float gn = gnh + bh[2][j];
+            const float n = tanhf_(get(pv[2], j) + r * gn);
+            const float f = n + z * (h - n);
+            const float omz = 1.f - z;
+            const float cz = (h - n) * z * omz;
+            const float cn = omz * (1.f - n * n) * r;
+            const float cr = cn * gn * (1.f - r);
+            const float aa = z + cz * ud[1][j] + cn * ud[2][j] + cr * ud[0][j];
+            a[k][j] = aa;
+            bb[k][j] = f - aa * h;
+            y[k][j] = hp[k + 1][j];
+            rmax = max(rmax, abs_bits(hp[k + 1][j] - f));
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 3. tile passes
+// ---------------------------------------------------------------------------
+// Forward affine scan of (a, bb) with the carry from the previous chunk; writes
+// out[k][j] = state at step t0+k.  All threads of the CTA must call it.
+__device__ __forceinline__ void scan_forward(const DiagArgs &A, const TileCoord &c, const Smem &sm,
+                                             unsigned long long *desc, unsigned epoch,
+                                             const float (&a)[TK][4], const float (&bb)[TK][4],
+                                             const float *carry0 /*[DG] for chunk 0*/,
+                                             float (&out)[TK][4]) {
+    const Tiling &tl = A.tl;
+    float cA[4], cB[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) { cA[j] = 1.f; cB[j] = 0.f; }
+#pragma unroll
+    for (int k = 0; k < TK; ++k)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            cB[j] = fmaf(a[k][j], cB[j], bb[k][j]);
+            cA[j] = a[k][j] * cA[j];
+        }
+    if (c.active)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            sm.s0[c.tb * tl.DG + c.lane0 + j] = cA[j];
+            sm.s1[c.tb * tl.DG + c.lane0 + j] = cB[j];
+        }
+    __syncthreads();
+    if (threadIdx.x < tl.DG) {
+        const int lane = threadIdx.x;
+        float EA = 1.f, EB = 0.f;
+        for (int q = 0; q < tl.NTB; ++q) {
+            const float qa = sm.s0[q * tl.DG + lane], qb = sm.s1[q * tl.DG + lane];
+            sm.s0[q * tl.DG + lane] = EA;
+            sm.s1[q * tl.DG + lane] = EB;
+            EB = fmaf(qa, EB, qb);
+            EA = qa * EA;
+        }
+        sm.c0[lane] = lookback_affine(desc, c.tile, tl.n_groups, tl.DG, lane, epoch, EA, EB,
+                                      c.chunk == 0, carry0[lane], &A.hdr->status);
+    }
+    __syncthreads();
+    if (c.active) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int l = c.lane0 + j;
+            float h = fmaf(sm.s0[c.tb * tl.DG + l], sm.c0[l], sm.s1[c.tb * tl.DG + l]);
+#pragma unroll
+            for (int k = 0; k < TK; ++k) {
+                h = fmaf(a[k][j], h, bb[k][j]);
+                out[k][j] = h;
+            }
+        }
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ void store_states(const DiagArgs &A, const TileCoord &c, float *dst,
+                                             const float (&v)[TK][4]) {
+    if (!c.dvalid) return;
+#pragma unroll
+    for (int k = 0; k < TK; ++k) {
+        const int t = c.t0 + k;
+        if (t < A.T)
+            stcg4(dst + (static_cast<size_t>(c.b) * A.T + t) * A.D + c.d0,
+                  make_float4(v[k][0], v[k][1], v[k][2], v[k][3]));
+    }
+}
+
+__device__ __forceinline__ void load_states(const DiagArgs &A, const TileCoord &c, const float *src,
+                                            int shift, float (&v)[TK][4], float fill) {
+#pragma unroll
+    for (int k = 0; k < TK; ++k) {
+        const int t = c.t0 + k + shift;
+        float4 x = make_float4(fill, fill, fill, fill);
+        if (c.dvalid && t < A.T) x = ldcg4(src + (static_cast<size_t>(c.b) * A.T + t) * A.D + c.d0);
+        v[k][0] = x.x; v[k][1] = x.y; v[k][2] = x.z; v[k][3] = x.w;
+    }
+}
+
+// carries of chunk 0 for this tile's lanes: h0 (mean) into sm.c1
+__device__ __forceinline__ void load_h0_carry(const DiagArgs &A, const TileCoord &c, const Smem &sm) {
+    if (threadIdx.x < A.tl.DG) {
+        const int d = c.dg * A.tl.DG + threadIdx.x;
+        sm.c1[threadIdx.x] = d < A.D ? __ldg(A.h0 + static_cast<size_t>(c.b) * A.D + d) : 0.f;
+    }
+    __syncthreads();
+}
+
+// --- quasi-DEER tile: linearise, scan, write, reduce ------------------------
+template <bool DENSE>
+__device__ void quasi_tile(const DiagArgs &A, long long tile, const Smem &sm, const float *hold,
+                           float *hnew, bool zero_guess, unsigned epoch, unsigned &dmax,
+                           unsigned &rmax) {
+    const TileCoord c = tile_coord(A, tile);
+    float a[TK][4], bb[TK][4], y[TK][4], out[TK][4];
+    load_h0_carry(A, c, sm);
+    linearise<DENSE>(A, c, sm, hold, zero_guess, a, bb, y, rmax);
+    scan_forward(A, c, sm, A.desc, epoch, a, bb, sm.c1, out);
+    if (c.dvalid) {
+#pragma unroll
+        for (int k = 0; k < TK; ++k)
+            if (c.t0 + k < A.T)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) dmax = max(dmax, abs_bits(out[k][j] - y[k][j]));
+    }
+    store_states(A, c, hnew, out);
+}
+
+// --- quasi-ELK forward tile: Kalman covariance (Mobius) + filtered mean -------
+template <bool DENSE>
+__device__ void elk_forward_tile(const DiagArgs &A, long long tile, const Smem &sm,
+                                 const float *hold, bool zero_guess, unsigned epoch,
+                                 unsigned &rmax) {
+    const Tiling &tl = A.tl;
+    const TileCoord c = tile_coord(A, tile);
+    const float lam = A.lambda;
+    float a[TK][4], bb[TK][4], y[TK][4];
+    load_h0_carry(A, c, sm);
+    linearise<DENSE>(A, c, sm, hold, zero_guess, a, bb, y, rmax);
+
+    unsigned long long *desc_cov = A.desc;
+    unsigned long long *desc_mean = A.desc + static_cast<size_t>(tl.n_tiles) * tl.DG * 4;
+
+    // (i) covariance: P_t = M_t * P_{t-1} with M_t = [[a^2, 1], [lam a^2, 1 + lam]], P_0 = 0
+    Mob cm[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) cm[j] = Mob{1.f, 0.f, 0.f, 1.f};
+#pragma unroll
+    for (int k = 0; k < TK; ++k)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float a2 = a[k][j] * a[k][j];
+            const bool valid = c.dvalid && c.t0 + k < A.T;
+            const Mob Mk = valid ? Mob{a2, 1.f, lam * a2, 1.f + lam} : Mob{1.f, 0.f, 0.f, 1.f};
+            cm[j] = mob_mul(Mk, cm[j]);
+        }
+    if (c.active)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int idx = c.tb * tl.DG + c.lane0 + j;
+            sm.s0[idx] = cm[j].m0; sm.s1[idx] = cm[j].m1; sm.s2[idx] = cm[j].m2; sm.s3[idx] = cm[j].m3;
+        }
+    __syncthreads();
+    if (threadIdx.x < tl.DG) {
+        const int lane = threadIdx.x;
+        Mob E{1.f, 0.f, 0.f, 1.f};
+        for (int q = 0; q < tl.NTB; ++q) {
+            const int idx = q * tl.DG + lane;
+            const Mob Q{sm.s0[idx], sm.s1[idx], sm.s2[idx], sm.s3[idx]};
+            sm.s0[idx] = E.m0; sm.s1[idx] = E.m1; sm.s2[idx] = E.m2; sm.s3[idx] = E.m3;
+            E = mob_mul(Q, E);
+        }
+        sm.c0[lane] = lookback_mobius(desc_cov, c.tile, tl.n_groups, tl.DG, lane, epoch, E,
+                                      c.chunk == 0, 0.f, &A.hdr->status);
+    }
+    __syncthreads();
+    float Pk[TK][4], al[TK][4], be[TK][4];
+    if (c.active) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int idx = c.tb * tl.DG + c.lane0 + j;
+            const Mob E{sm.s0[idx], sm.s1[idx], sm.s2[idx], sm.s3[idx]};
+            float P = mob_apply(E, sm.c0[c.lane0 + j]);
+#pragma unroll
+            for (int k = 0; k < TK; ++k) {
+                const float Pm = fmaf(a[k][j] * a[k][j], P, 1.f);  // P-_t
+                const float K = lam * Pm / (1.f + lam * Pm);       // gain; K = lam P_t
+                P = Pm / (1.f + lam * Pm);
+                Pk[k][j] = P;
+                const float omk = 1.f - K;
+                const bool valid = c.dvalid && c.t0 + k < A.T;
+                al[k][j] = valid ? omk * a[k][j] : 1.f;
+                be[k][j] = valid ? fmaf(omk, bb[k][j], K * y[k][j]) : 0.f;
+            }
+        }
+    }
+    __syncthreads();
+    // (ii) filtered mean: m_t = (1 - K_t)(a_t m_{t-1} + b_t) + K_t y_t, m_0 = h0
+    float m[TK][4];
+    scan_forward(A, c, sm, desc_mean, epoch, al, be, sm.c1, m);
+    store_states(A, c, A.elk_m, m);
+    store_states(A, c, A.elk_p, Pk);
+    store_states(A, c, A.elk_a, a);
+    store_states(A, c, A.elk_b, bb);
+}
+
+// --- quasi-ELK backward tile: RTS smoother as a reverse affine scan ----------
+__device__ void elk_backward_tile(const DiagArgs &A, long long tile, const Smem &sm,
+                                  const float *hold, float *hnew, bool zero_guess,
+                                  unsigned epoch, unsigned &dmax) {
+    const Tiling &tl = A.tl;
+    const TileCoord c = tile_coord(A, tile);
+    unsigned long long *desc_bwd = A.desc + static_cast<size_t>(tl.n_tiles) * tl.DG * 6;
+    float m[TK][4], P[TK][4], an[TK][4], bn[TK][4], y[TK][4];
+    load_states(A, c, A.elk_m, 0, m, 0.f);
+    load_states(A, c, A.elk_p, 0, P, 0.f);
+    load_states(A, c, A.elk_a, 1, an, 0.f);
+    load_states(A, c, A.elk_b, 1, bn, 0.f);
+    if (zero_guess) {
+#pragma unroll
+        for (int k = 0; k < TK; ++k)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) y[k][j] = 0.f;
+    } else {
+        load_states(A, c, hold, 0, y, 0.f);
+    }
+    // s_t = G_t s_{t+1} + c_t,  G_t = P_t a_{t+1} / (a_{t+1}^2 P_t + 1),
+    // c_t = m_t - G_t (a_{t+1} m_t + b_{t+1});  G = 0 at t = T-1; identity past T.
+    float Gk[TK][4], Ck[TK][4];
+#pragma unroll
+    for (int k = 0; k < TK; ++k) {
+        const int t = c.t0 + k;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (!c.dvalid || t >= A.T) { Gk[k][j] = 1.f; Ck[k][j] = 0.f; continue; }
+            if (t == A.T - 1) { Gk[k][j] = 0.f; Ck[k][j] = m[k][j]; continue; }
+            const float an_ = an[k][j];
+            const float G = P[k][j] * an_ / fmaf(an_ * an_, P[k][j], 1.f);
+            Gk[k][j] = G;
+            Ck[k][j] = m[k][j] - G * fmaf(an_, m[k][j], bn[k][j]);
+        }
+    }
+    // reverse composition within the thread: maps s_{t0+TK} -> s_{t0}
+    float cG[4], cC[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) { cG[j] = 1.f; cC[j] = 0.f; }
+#pragma unroll
+    for (int k = TK - 1; k >= 0; --k)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            cC[j] = fmaf(Gk[k][j], cC[j], Ck[k][j]);
+            cG[j] = Gk[k][j] * cG[j];
+        }
+    if (c.active)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            sm.s0[c.tb * tl.DG + c.lane0 + j] = cG[j];
+            sm.s1[c.tb * tl.DG + c.lane0 + j] = cC[j];
+        }
+    __syncthreads();
+    if (threadIdx.x < tl.DG) {
+        const int lane = threadIdx.x;
+        float EG = 1.f, EC = 0.f;
+        for (int q = tl.NTB - 1; q >= 0; --q) {
+            const float qg = sm.s0[q * tl.DG + lane], qc = sm.s1[q * tl.DG + lane];
+            sm.s0[q * tl.DG + lane] = EG;
+            sm.s1[q * tl.DG + lane] = EC;
+            EC = fmaf(qg, EC, qc);
+            EG = qg * EG;
+        }
+        sm.c0[lane] = lookback_affine(desc_bwd, c.tile, -static_cast<long long>(tl.n_groups),
+                                      tl.DG, lane, epoch, EG, EC, c.chunk == tl.n_chunks - 1,
+                                      0.f, &A.hdr->status);
+    }
+    __syncthreads();
+    float out[TK][4];
+    if (c.active) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int l = c.lane0 + j;
+            float s = fmaf(sm.s0[c.tb * tl.DG + l], sm.c0[l], sm.s1[c.tb * tl.DG + l]);
+#pragma unroll
+            for (int k = TK - 1; k >= 0; --k) {
+                s = fmaf(Gk[k][j], s, Ck[k][j]);
+                out[k][j] = s;
+            }
+        }
+    }
+    __syncthreads();
+    if (c.dvalid) {
+#pragma unroll
+        for (int k = 0; k < TK; ++k)
+            if (c.t0 + k < A.T)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) dmax = max(dmax, abs_bits(out[k][j] - y[k][j]));
+    }
+    store_states(A, c, hnew, out);
+}
+
+// ---------------------------------------------------------------------------
+// 4. the persistent kernel
+// ---------------------------------------------------------------------------
+template <bool DENSE, bool ELK>
+__global__ void __launch_bounds__(kThreads, 1) diag_solver_kernel(DiagArgs A) {
+    extern __shared__ float4 smem_raw[];
+    const Tiling &tl = A.tl;
+    const Smem sm = carve(reinterpret_cast<float *>(smem_raw), tl, A.D, DENSE);
+    WsHeader *hdr = A.hdr;
+    unsigned *status = &hdr->status;
+    const unsigned nblocks = gridDim.x;
+
+    if (DENSE) {
+        // U^T slices into shared memory, layout [m][g][lane]: Us = U_g[lane][m]
+        const int D = A.D, n = D * 3 * tl.DG;
+        for (int i = threadIdx.x; i < n; i += kThreads) {
+            const int lane = i % tl.DG, g = (i / tl.DG) % 3, m = i / (3 * tl.DG);
+            sm.Us[i] = __ldg(A.w_hh + (static_cast<size_t>(g) * D + lane) * D + m);
+        }
+        __syncthreads();
+    }
+
+    int it = 0;
+    int iters = 0;
+    int final_status = PARARNN_NOT_CONVERGED;
+    unsigned last_delta = 0u, last_resid = 0u;
+    for (; it < A.max_iters; ++it) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) {
+            hdr->delta_bits[(it + 1) % 3] = 0u;
+            hdr->resid_bits[(it + 1) % 3] = 0u;
+        }
+        const float *hold = A.hbuf[it & 1];
+        float *hnew = A.hbuf[(it + 1) & 1];
+        const bool zero_guess = it == 0;
+        const unsigned epoch = static_cast<unsigned>(it + 1);
+        unsigned dmax = 0u, rmax = 0u;
+        if (!ELK) {
+            for (long long tile = blockIdx.x; tile < tl.n_tiles; tile += nblocks)
+                quasi_tile<DENSE>(A, tile, sm, hold, hnew, zero_guess, epoch, dmax, rmax);
+        } else {
+            for (long long tile = blockIdx.x; tile < tl.n_tiles; tile += nblocks)
+                elk_forward_tile<DENSE>(A, tile, sm, hold, zero_guess, epoch, rmax);
+            grid_barrier(hdr->barrier, nblocks, status);
+            for (long long k = blockIdx.x; k < tl.n_tiles; k += nblocks)
+                elk_backward_tile(A, tl.n_tiles - 1 - k, sm, hold, hnew, zero_guess, epoch, dmax);
+        }
+        const unsigned bd = block_max_u32(dmax, sm.red);
+        const unsigned br = block_max_u32(rmax, sm.red);
+        if (threadIdx.x == 0) {
+            atomicMax(&hdr->delta_bits[it % 3], bd);
+            atomicMax(&hdr->resid_bits[it % 3], br);
+        }
+        grid_barrier(hdr->barrier, nblocks, status);
+        last_delta = ld_acquire_u32(&hdr->delta_bits[it % 3]);
+        last_resid = ld_acquire_u32(&hdr->resid_bits[it % 3]);
+        iters = it + 1;
+        if (timed_out(status)) { final_status = PARARNN_TIMEOUT; break; }
+        if (last_delta >= 0x7f800000u) { final_status = PARARNN_DIVERGED; break; }
+        if (__uint_as_float(last_delta) <= A.tol) { final_status = PARARNN_OK; break; }
+    }
+    // the final iterate lives in hbuf[iters & 1]; hbuf[1] is the caller's array
+    if ((iters & 1) == 0 && iters > 0) {
+        const size_t n4 = static_cast<size_t>(A.B) * A.T * A.D / 4;
+        const float4 *src = reinterpret_cast<const float4 *>(A.hbuf[0]);
+        float4 *dst = reinterpret_cast<float4 *>(A.hbuf[1]);
+        for (size_t i = static_cast<size_t>(blockIdx.x) * kThreads + threadIdx.x; i < n4;
+             i += static_cast<size_t>(nblocks) * kThreads)
+            dst[i] = __ldcg(src + i);
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        pararnn_info info;
+        info.iters = iters;
+        info.status = final_status;
+        info.delta = __uint_as_float(last_delta);
+        info.residual = __uint_as_float(last_resid);
+        *A.info_out = info;
+        hdr->info = info;
+    }
+}
+
+template <bool DENSE, bool ELK>
+cudaError_t launch_one(const DiagArgs &a, cudaStream_t s) {
+    auto kern = diag_solver_kernel<DENSE, ELK>;
+    const size_t smem = smem_floats(a.tl, a.D, DENSE) * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    int dev = 0, nsm = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem)) !=
+        cudaSuccess)
+        return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    long long grid = static_cast<long long>(per_sm) * nsm;
+    if (grid > a.tl.n_tiles) grid = a.tl.n_tiles;
+    DiagArgs args = a;
+    void *params[] = {&args};
+    return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern),
+                                       dim3(static_cast<unsigned>(grid)), dim3(kThreads), params,
+                                       smem, s);
+}
+
+}  // namespace
+
+size_t diag_solver_smem_bytes(const Tiling &tl, int D, bool dense) {
+    return smem_floats(tl, D, dense) * sizeof(float);
+}
+
+cudaError_t launch_diag_solver(const pararnn_cell &cell, int mode, const DiagArgs &a,
+                               cudaStream_t s) {
+    const bool dense = cell.kind == PARARNN_GRU_DENSE;
+    const bool elk = mode == PARARNN_ELK || mode == PARARNN_QUASI_ELK;
+    if (dense) return elk ? launch_one<true, true>(a, s) : launch_one<true, false>(a, s);
+    return elk ? launch_one<false, true>(a, s) : launch_one<false, false>(a, s);
+}
+
+}  // namespace pararnn

@@ -1,0 +1,281 @@
+// pararnn_api.cu -- the C ABI: argument checks, workspace layout, launches.
+//
+// Every entry point is declared and documented in include/pararnn.h.  Nothing
+// here allocates memory; the caller's workspace is carved into the sections
+// below (each 256-byte aligned):
+//   header  WsHeader (grid barrier, status word, delta/residual slots, report)
+//   P       [B, T, 3D] fp32 input pre-activations
+//   hbuf    [B, T, D]  fp32 second iterate buffer (the caller's h is the first)
+//   desc    look-back descriptors: tiles x lanes x (2 words, or 8 for quasi-ELK)
+//   elk     quasi-ELK forward results m, P, a, b: 4 x [B, T, D] fp32
+//   dense   block-scan scratch of the dense-Jacobian modes
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "solver.cuh"
+
+namespace pararnn {
+
+size_t scan_diag_ws_bytes(int B, int T, int D);
+size_t diag_solver_smem_bytes(const Tiling &tl, int D, bool dense);
+size_t dense_ws_bytes(const pararnn_cell &cell, int B, int T, int mode);
+cudaError_t launch_dense_solver(const pararnn_cell &cell, int mode, const DiagArgs &a,
+                                void *dense_ws, cudaStream_t s);
+cudaError_t launch_scan_dense(const float *A, const float *b, const float *h0, int B, int T,
+                              int D, float *h, void *ws, cudaStream_t s);
+size_t scan_dense_ws_bytes(int B, int T, int D);
+
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    const auto pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+    return pa < pb + nb && pb < pa + na;
+}
+
+bool diag_jacobian(const pararnn_cell &cell, int mode) {
+    return cell.kind == PARARNN_GRU_DIAG || mode == PARARNN_QUASI || mode == PARARNN_QUASI_ELK;
+}
+
+bool is_elk(int mode) { return mode == PARARNN_ELK || mode == PARARNN_QUASI_ELK; }
+
+bool cell_ok(const pararnn_cell *cell, int B, int T, int mode) {
+    if (cell == nullptr || B < 1 || T < 1) return false;
+    if (cell->kind != PARARNN_GRU_DENSE && cell->kind != PARARNN_GRU_DIAG) return false;
+    if (cell->d < 4 || cell->d % 4 != 0 || cell->din < 1) return false;
+    if (cell->x_dtype != cell->w_dtype) return false;
+    if (cell->x_dtype != PARARNN_F32 && cell->x_dtype != PARARNN_BF16) return false;
+    if (mode < PARARNN_DEER || mode > PARARNN_QUASI_ELK) return false;
+    if (cell->kind == PARARNN_GRU_DENSE && cell->d > 64) return false;
+    // the state array is indexed with 32-bit time and lane counts
+    if (static_cast<long long>(T) * 3 * cell->d > (1ll << 31)) return false;
+    return true;
+}
+
+}  // namespace
+
+WsLayout ws_layout(const pararnn_cell &cell, int B, int T, int mode) {
+    WsLayout L{};
+    const size_t states = static_cast<size_t>(B) * T * cell.d;
+    const bool diag = diag_jacobian(cell, mode);
+    const Tiling tl = make_tiling(B, T, cell.d, cell.kind == PARARNN_GRU_DENSE);
+    size_t off = 0;
+    L.header = off; off += 256;
+    L.P = off; off = align256(off + states * 3 * sizeof(float));
+    L.hbuf = off; off = align256(off + states * sizeof(float));
+    L.desc = off;
+    if (diag) off = align256(off + static_cast<size_t>(tl.n_tiles) * tl.DG * (is_elk(mode) ? 8 : 2) * 8);
+    L.elk = off;
+    if (diag && is_elk(mode)) off = align256(off + 4 * states * sizeof(float));
+    L.dense = off;
+    if (!diag) off = align256(off + dense_ws_bytes(cell, B, T, mode));
+    L.total = off;
+    return L;
+}
+
+}  // namespace pararnn
+
+using namespace pararnn;
+
+extern "C" {
+
+size_t pararnn_workspace_size(const pararnn_cell *cell, int B, int T, int mode) {
+    if (!cell_ok(cell, B, T, mode)) return 0;
+    return ws_layout(*cell, B, T, mode).total;
+}
+
+// Checks shared by every solve entry point.  `need_x`: the projection runs.
+static int check_solve(const pararnn_cell *cell, const pararnn_params *params, const void *x,
+                       const float *P, const float *h0, int B, int T, int mode, float lambda,
+                       float tol, float *h, void *workspace, size_t ws_bytes) {
+    if (!cell_ok(cell, B, T, mode) || params == nullptr) return PARARNN_INVALID_ARG;
+    if ((!x && !P) || !h0 || !h || !workspace || !params->w_hh || !params->b_hh)
+        return PARARNN_INVALID_ARG;
+    if (x && (!params->w_ih || !params->b_ih)) return PARARNN_INVALID_ARG;
+    if (!(tol >= 0.f) || !std::isfinite(tol)) return PARARNN_INVALID_ARG;
+    if (is_elk(mode) && !(lambda > 0.f && std::isfinite(lambda))) return PARARNN_INVALID_ARG;
+    if ((x && !aligned(x, 16)) || (P && !aligned(P, 16)) || !aligned(h0, 16) || !aligned(h, 16) ||
+        !aligned(params->w_hh, 16) || !aligned(params->b_hh, 16) || !aligned(workspace, 256))
+        return PARARNN_INVALID_ARG;
+    if (x && (!aligned(params->b_ih, 16) || !aligned(params->w_ih, 16))) return PARARNN_INVALID_ARG;
+    const WsLayout L = ws_layout(*cell, B, T, mode);
+    if (ws_bytes < L.total) return PARARNN_INVALID_ARG;
+    const size_t states = static_cast<size_t>(B) * T * cell->d;
+    const size_t xbytes = static_cast<size_t>(B) * T * cell->din *
+                          (cell->x_dtype == PARARNN_BF16 ? 2 : 4);
+    if (overlaps(h, states * 4, workspace, L.total) ||
+        (x && overlaps(h, states * 4, x, xbytes)) || (P && overlaps(h, states * 4, P, states * 12)) ||
+        overlaps(h, states * 4, h0, static_cast<size_t>(B) * cell->d * 4))
+        return PARARNN_INVALID_ARG;
+    if (P && overlaps(P, states * 12, workspace, L.total)) return PARARNN_INVALID_ARG;
+    return PARARNN_OK;
+}
+
+// Enqueue the Newton loop on pre-activations P (device).
+static cudaError_t enqueue_iterate(const pararnn_cell *cell, const pararnn_params *params,
+                                   const float *P, const float *h0, int B, int T, int mode,
+                                   float lambda, float tol, int max_iters, float *h,
+                                   pararnn_info *info_dev, void *workspace, cudaStream_t s) {
+    const WsLayout L = ws_layout(*cell, B, T, mode);
+    char *ws = static_cast<char *>(workspace);
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws + L.header);
+    const bool diag = diag_jacobian(*cell, mode);
+    const size_t states = static_cast<size_t>(B) * T * cell->d;
+
+    DiagArgs a{};
+    a.B = B; a.T = T; a.D = cell->d;
+    a.P = P;
+    a.w_hh = params->w_hh;
+    a.b_hh = params->b_hh;
+    a.h0 = h0;
+    a.hbuf[0] = reinterpret_cast<float *>(ws + L.hbuf);
+    a.hbuf[1] = h;
+    a.lambda = lambda;
+    a.tol = tol;
+    a.max_iters = max_iters <= 0 ? T : max_iters;
+    a.tl = make_tiling(B, T, cell->d, cell->kind == PARARNN_GRU_DENSE);
+    a.desc = reinterpret_cast<unsigned long long *>(ws + L.desc);
+    const size_t states4 = states * sizeof(float);
+    a.elk_m = reinterpret_cast<float *>(ws + L.elk);
+    a.elk_p = reinterpret_cast<float *>(ws + L.elk + states4);
+    a.elk_a = reinterpret_cast<float *>(ws + L.elk + 2 * states4);
+    a.elk_b = reinterpret_cast<float *>(ws + L.elk + 3 * states4);
+    a.hdr = hdr;
+    a.info_out = info_dev ? info_dev : &hdr->info;
+
+    cudaError_t e = cudaMemsetAsync(ws + L.header, 0, 256, s);
+    if (e == cudaSuccess && diag && L.elk > L.desc) e = cudaMemsetAsync(ws + L.desc, 0, L.elk - L.desc, s);
+    if (e != cudaSuccess) return e;
+    return diag ? launch_diag_solver(*cell, mode, a, s)
+                : launch_dense_solver(*cell, mode, a, ws + L.dense, s);
+}
+
+int pararnn_input_projection(const pararnn_cell *cell, const pararnn_params *params,
+                             const void *x, int B, int T, float *P, pararnn_stream stream) {
+    if (!cell_ok(cell, B, T, PARARNN_QUASI) || !params || !x || !P || !params->w_ih || !params->b_ih)
+        return PARARNN_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(P, 16) || !aligned(params->w_ih, 16) || !aligned(params->b_ih, 16))
+        return PARARNN_INVALID_ARG;
+    const cudaError_t e = launch_projection(*cell, x, params->w_ih, params->b_ih, P,
+                                            static_cast<long long>(B) * T,
+                                            reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
+}
+
+int pararnn_newton_iterate_async(const pararnn_cell *cell, const pararnn_params *params,
+                                 const float *P, const float *h0, int B, int T, int mode,
+                                 float lambda, float tol, int max_iters, float *h,
+                                 pararnn_info *info_dev, void *workspace, size_t ws_bytes,
+                                 pararnn_stream stream) {
+    if (!P || !info_dev || !aligned(info_dev, 4)) return PARARNN_INVALID_ARG;
+    int rc = check_solve(cell, params, nullptr, P, h0, B, T, mode, lambda, tol, h, workspace,
+                         ws_bytes);
+    if (rc != PARARNN_OK) return rc;
+    const cudaError_t e = enqueue_iterate(cell, params, P, h0, B, T, mode, lambda, tol, max_iters,
+                                          h, info_dev, workspace,
+                                          reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
+}
+
+static int solve_enqueue(const pararnn_cell *cell, const pararnn_params *params, const void *x,
+                         const float *h0, int B, int T, int mode, float lambda, float tol,
+                         int max_iters, float *h, pararnn_info *info_dev, void *workspace,
+                         size_t ws_bytes, pararnn_stream stream) {
+    int rc = check_solve(cell, params, x, nullptr, h0, B, T, mode, lambda, tol, h, workspace,
+                         ws_bytes);
+    if (rc != PARARNN_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const WsLayout L = ws_layout(*cell, B, T, mode);
+    float *P = reinterpret_cast<float *>(static_cast<char *>(workspace) + L.P);
+    cudaError_t e = launch_projection(*cell, x, params->w_ih, params->b_ih, P,
+                                      static_cast<long long>(B) * T, s);
+    if (e == cudaSuccess)
+        e = enqueue_iterate(cell, params, P, h0, B, T, mode, lambda, tol, max_iters, h, info_dev,
+                            workspace, s);
+    return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
+}
+
+int pararnn_newton_solve_async(const pararnn_cell *cell, const pararnn_params *params,
+                               const void *x, const float *h0, int B, int T, int mode,
+                               float lambda, float tol, int max_iters, float *h,
+                               pararnn_info *info_dev, void *workspace, size_t ws_bytes,
+                               pararnn_stream stream) {
+    if (info_dev == nullptr || !aligned(info_dev, 4)) return PARARNN_INVALID_ARG;
+    return solve_enqueue(cell, params, x, h0, B, T, mode, lambda, tol, max_iters, h, info_dev,
+                         workspace, ws_bytes, stream);
+}
+
+int pararnn_newton_solve(const pararnn_cell *cell, const pararnn_params *params, const void *x,
+                         const float *h0, int B, int T, int mode, float lambda, float tol,
+                         int max_iters, float *h, pararnn_info *info, void *workspace,
+                         size_t ws_bytes, pararnn_stream stream) {
+    const int rc = solve_enqueue(cell, params, x, h0, B, T, mode, lambda, tol, max_iters, h,
+                                 nullptr, workspace, ws_bytes, stream);
+    if (rc != PARARNN_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const WsLayout L = ws_layout(*cell, B, T, mode);
+    pararnn_info host{};
+    const WsHeader *hdr = reinterpret_cast<const WsHeader *>(static_cast<char *>(workspace) + L.header);
+    cudaError_t e = cudaMemcpyAsync(&host, &hdr->info, sizeof(host), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
+    if (info) *info = host;
+    return host.status;
+}
+
+size_t pararnn_affine_scan_workspace_size(int B, int T, int D, int dense) {
+    if (B < 1 || T < 1 || D < 4 || D % 4 != 0) return 0;
+    if (static_cast<long long>(T) * D > (1ll << 31)) return 0;
+    if (dense) return D <= 64 ? scan_dense_ws_bytes(B, T, D) : 0;
+    return scan_diag_ws_bytes(B, T, D);
+}
+
+int pararnn_affine_scan(const float *A, const float *b, const float *h0, int B, int T, int D,
+                        int dense, float *h, void *workspace, size_t ws_bytes,
+                        pararnn_stream stream) {
+    const size_t need = pararnn_affine_scan_workspace_size(B, T, D, dense);
+    if (need == 0 || ws_bytes < need) return PARARNN_INVALID_ARG;
+    if (!A || !b || !h0 || !h || !workspace) return PARARNN_INVALID_ARG;
+    if (!aligned(A, 16) || !aligned(b, 16) || !aligned(h0, 16) || !aligned(h, 16) ||
+        !aligned(workspace, 256))
+        return PARARNN_INVALID_ARG;
+    const size_t nA = static_cast<size_t>(B) * T * D * (dense ? D : 1) * 4;
+    const size_t nh = static_cast<size_t>(B) * T * D * 4;
+    if (overlaps(h, nh, A, nA) || overlaps(h, nh, h0, static_cast<size_t>(B) * D * 4) ||
+        overlaps(h, nh, workspace, need))
+        return PARARNN_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const cudaError_t e = dense ? launch_scan_dense(A, b, h0, B, T, D, h, workspace, s)
+                                : launch_scan_diag(A, b, h0, B, T, D, h, workspace, s);
+    return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
+}
+
+int pararnn_affine_scan_status(const void *workspace, pararnn_stream stream) {
+    if (!workspace || !aligned(workspace, 256)) return PARARNN_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned st = 0;
+    const WsHeader *hdr = static_cast<const WsHeader *>(workspace);
+    cudaError_t e = cudaMemcpyAsync(&st, &hdr->status, sizeof(st), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
+    return (st & kStatusTimeout) ? PARARNN_TIMEOUT : PARARNN_OK;
+}
+
+const char *pararnn_status_string(int status) {
+    switch (status) {
+        case PARARNN_OK: return "PARARNN_OK";
+        case PARARNN_NOT_CONVERGED: return "PARARNN_NOT_CONVERGED";
+        case PARARNN_DIVERGED: return "PARARNN_DIVERGED";
+        case PARARNN_INVALID_ARG: return "PARARNN_INVALID_ARG";
+        case PARARNN_CUDA_ERROR: return "PARARNN_CUDA_ERROR";
+        case PARARNN_TIMEOUT: return "PARARNN_TIMEOUT";
+        default: return "PARARNN_UNKNOWN_STATUS";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,137 @@
+// scan_diag.cu -- standalone diagonal affine scan h_t = a_t * h_{t-1} + b_t.
+//
+// The linear solve inside each quasi-Newton iteration, exposed on its own
+// ("Towards Scalable and Stable Parallelization of Nonlinear RNNs", atlas
+// summary "Builds on": parallel associative scan; "ParaRNN" summary,
+// "Newton's Iteration": forward substitution on a block lower-triangular
+// system).  Single pass over HBM (12 bytes per element: a, b in, h out):
+// tiles of (sequence, 64 lanes, L steps) are taken in order from a ticket
+// counter, so every tile's predecessor has already started; each thread
+// composes 4 steps x 4 lanes in registers, a shared-memory pass forms the
+// tile-local exclusive prefixes, one thread per lane resolves the carry with a
+// decoupled look-back, and the tile is re-swept and written with float4 stores.
+#include "common.cuh"
+#include "lookback.cuh"
+#include "solver.cuh"
+
+namespace pararnn {
+namespace {
+
+constexpr int TK = 4;
+
+struct ScanArgs {
+    const float *A, *b, *h0;
+    float *h;
+    int B, T, D;
+    Tiling tl;
+    unsigned long long *desc;
+    WsHeader *hdr;
+};
+
+__global__ void __launch_bounds__(kThreads) scan_diag_kernel(ScanArgs S) {
+    __shared__ float sA[kThreads * 4], sB[kThreads * 4];  // [NTB][DG] (NTB*DG <= 1024)
+    __shared__ float sC[64];
+    __shared__ long long s_tile;
+    const Tiling &tl = S.tl;
+    if (threadIdx.x == 0) s_tile = static_cast<long long>(atomicAdd(&S.hdr->ticket, 1ull));
+    __syncthreads();
+    const long long tile = s_tile;
+    const int chunk = static_cast<int>(tile / tl.n_groups);
+    const int grp = static_cast<int>(tile % tl.n_groups);
+    const int b = grp / tl.n_dgroups, dg = grp % tl.n_dgroups;
+    const int db = threadIdx.x % tl.DB, tb = threadIdx.x / tl.DB;
+    const bool active = tb < tl.NTB;
+    const int lane0 = db * 4, d0 = dg * tl.DG + lane0;
+    const bool dvalid = active && d0 < S.D;
+    const int t0 = chunk * tl.L + tb * TK;
+
+    float a[TK][4], bb[TK][4];
+#pragma unroll
+    for (int k = 0; k < TK; ++k) {
+        const int t = t0 + k;
+        float4 av = make_float4(1.f, 1.f, 1.f, 1.f), bv = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (dvalid && t < S.T) {
+            const size_t off = (static_cast<size_t>(b) * S.T + t) * S.D + d0;
+            av = __ldcs(reinterpret_cast<const float4 *>(S.A + off));
+            bv = __ldcs(reinterpret_cast<const float4 *>(S.b + off));
+        }
+        a[k][0] = av.x; a[k][1] = av.y; a[k][2] = av.z; a[k][3] = av.w;
+        bb[k][0] = bv.x; bb[k][1] = bv.y; bb[k][2] = bv.z; bb[k][3] = bv.w;
+    }
+    float cA[4], cB[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) { cA[j] = 1.f; cB[j] = 0.f; }
+#pragma unroll
+    for (int k = 0; k < TK; ++k)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            cB[j] = fmaf(a[k][j], cB[j], bb[k][j]);
+            cA[j] = a[k][j] * cA[j];
+        }
+    if (active)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            sA[tb * tl.DG + lane0 + j] = cA[j];
+            sB[tb * tl.DG + lane0 + j] = cB[j];
+        }
+    __syncthreads();
+    if (threadIdx.x < tl.DG) {
+        const int lane = threadIdx.x;
+        float EA = 1.f, EB = 0.f;
+        for (int q = 0; q < tl.NTB; ++q) {
+            const float qa = sA[q * tl.DG + lane], qb = sB[q * tl.DG + lane];
+            sA[q * tl.DG + lane] = EA;
+            sB[q * tl.DG + lane] = EB;
+            EB = fmaf(qa, EB, qb);
+            EA = qa * EA;
+        }
+        const int d = dg * tl.DG + lane;
+        const float carry0 = (chunk == 0 && d < S.D) ? __ldg(S.h0 + static_cast<size_t>(b) * S.D + d) : 0.f;
+        sC[lane] = lookback_affine(S.desc, tile, tl.n_groups, tl.DG, lane, 1u, EA, EB, chunk == 0,
+                                   carry0, &S.hdr->status);
+    }
+    __syncthreads();
+    if (!dvalid) return;
+    float out[TK][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int l = lane0 + j;
+        float hv = fmaf(sA[tb * tl.DG + l], sC[l], sB[tb * tl.DG + l]);
+#pragma unroll
+        for (int k = 0; k < TK; ++k) {
+            hv = fmaf(a[k][j], hv, bb[k][j]);
+            out[k][j] = hv;
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < TK; ++k) {
+        const int t = t0 + k;
+        if (t < S.T)
+            __stcs(reinterpret_cast<float4 *>(S.h + (static_cast<size_t>(b) * S.T + t) * S.D + d0),
+                   make_float4(out[k][0], out[k][1], out[k][2], out[k][3]));
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_scan_diag(const float *A, const float *b, const float *h0, int B, int T, int D,
+                             float *h, void *ws, cudaStream_t s) {
+    ScanArgs S;
+    S.A = A; S.b = b; S.h0 = h0; S.h = h;
+    S.B = B; S.T = T; S.D = D;
+    S.tl = make_tiling(B, T, D, false);
+    S.hdr = static_cast<WsHeader *>(ws);
+    S.desc = reinterpret_cast<unsigned long long *>(static_cast<char *>(ws) + 256);
+    const size_t desc_bytes = static_cast<size_t>(S.tl.n_tiles) * S.tl.DG * 2 * 8;
+    cudaError_t e = cudaMemsetAsync(ws, 0, 256 + desc_bytes, s);
+    if (e != cudaSuccess) return e;
+    scan_diag_kernel<<<static_cast<unsigned>(S.tl.n_tiles), kThreads, 0, s>>>(S);
+    return cudaGetLastError();
+}
+
+size_t scan_diag_ws_bytes(int B, int T, int D) {
+    const Tiling tl = make_tiling(B, T, D, false);
+    return 256 + static_cast<size_t>(tl.n_tiles) * tl.DG * 2 * 8;
+}
+
+}  // namespace pararnn

@@ -1,0 +1,71 @@
+// solver.cuh -- internal interface between the C ABI and the solver kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/pararnn.h"
+
+namespace pararnn {
+
+// Device-side header at the start of every workspace (256 bytes).
+struct WsHeader {
+    unsigned barrier[2];     // grid barrier: arrivals, generation
+    unsigned status;         // kStatusTimeout bit
+    unsigned delta_bits[3];  // per-iteration max |dh| (rotating slots)
+    unsigned resid_bits[3];  // per-iteration max |residual|
+    unsigned pad0[7];
+    pararnn_info info;       // report of the last solve
+    unsigned long long ticket;  // tile ticket of standalone (non-cooperative) scans
+    unsigned pad1[38];
+};
+static_assert(sizeof(WsHeader) <= 256, "header must fit 256 bytes");
+
+// Tiling of the [B, T, D] state array into (sequence, lane-group, chunk) tiles.
+struct Tiling {
+    int DG;         // lanes (state components) per tile, multiple of 4, <= 64
+    int DB;         // float4 columns per tile row = DG / 4
+    int NTB;        // thread rows (t-blocks) per tile = kThreads / DB
+    int TK;         // time steps per thread
+    int L;          // time steps per tile = NTB * TK
+    int n_dgroups;  // ceil(D / DG)
+    int n_groups;   // B * n_dgroups
+    int n_chunks;   // ceil(T / L)
+    long long n_tiles;
+};
+
+Tiling make_tiling(int B, int T, int D, bool dense_cell);
+
+// Arguments of the persistent diagonal-Jacobian solver kernels.
+struct DiagArgs {
+    int B, T, D;
+    const float *P;      // [B, T, 3D] input pre-activations (b_ih included)
+    const float *w_hh;   // dense [3D, D] or diag [3D]
+    const float *b_hh;   // [3D]
+    const float *h0;     // [B, D]
+    float *hbuf[2];      // iterate ping-pong; hbuf[1] is the caller's output
+    float lambda, tol;
+    int max_iters;
+    Tiling tl;
+    unsigned long long *desc;  // look-back descriptors
+    float *elk_m, *elk_p, *elk_a, *elk_b;  // quasi-ELK forward results [B, T, D]
+    WsHeader *hdr;
+    pararnn_info *info_out;  // device report destination
+};
+
+// Workspace carve-up shared by the size query and the solver.
+struct WsLayout {
+    size_t header, P, hbuf, desc, elk, dense, total;
+};
+WsLayout ws_layout(const pararnn_cell &cell, int B, int T, int mode);
+
+// Kernel launchers (return a cudaError_t).
+cudaError_t launch_projection(const pararnn_cell &cell, const void *x, const void *w_ih,
+                              const float *b_ih, float *P, long long M, cudaStream_t s);
+cudaError_t launch_diag_solver(const pararnn_cell &cell, int mode, const DiagArgs &a,
+                               cudaStream_t s);
+cudaError_t launch_scan_diag(const float *A, const float *b, const float *h0, int B, int T,
+                             int D, float *h, void *ws, cudaStream_t s);
+
+}  // namespace pararnn

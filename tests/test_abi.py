@@ -1,0 +1,79 @@
+"""The C ABI library loads and exports every entry point the header declares.
+
+CPU only: these call host-side functions of the library (size queries and
+status names), never a kernel.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from newton_solve_nonlinear_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"PARARNN_API\s+[\w\s\*]+?\b(pararnn_\w+)\s*\(", src)
+    return names
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(binding._LIB_PATH):
+        from newton_solve_nonlinear_b200 import build
+        build.build()
+    return binding.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert set(names) >= set(binding.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code, name in binding.STATUS.items():
+        assert L.pararnn_status_string(code).decode() == "PARARNN_" + name
+    assert L.pararnn_status_string(99).decode() == "PARARNN_UNKNOWN_STATUS"
+
+
+def test_workspace_sizes(L):
+    ws = lambda *a, **k: binding.workspace_size(*a, **k)
+    # valid problems need at least the projection and a second iterate buffer
+    n = ws("dense", 64, 64, 16, 1024, "QUASI")
+    assert n >= 16 * 1024 * 64 * 4 * 4
+    assert ws("diag", 2048, 2048, 8, 4096, "QUASI") >= 8 * 4096 * 2048 * 16
+    # quasi-ELK keeps its forward results
+    assert ws("dense", 64, 64, 8, 1000, "QUASI_ELK") > ws("dense", 64, 64, 8, 1000, "QUASI")
+    # rejected: D not a multiple of 4, dense D > 64, bad mode, empty sizes
+    assert ws("dense", 4, 6, 1, 10, "QUASI") == 0
+    assert ws("dense", 4, 128, 1, 10, "QUASI") == 0
+    assert ws("diag", 4, 128, 1, 10, "QUASI") > 0
+    assert ws("dense", 4, 8, 0, 10, "QUASI") == 0
+    assert ws("dense", 4, 8, 1, 0, "QUASI") == 0
+    cell = binding.make_cell("dense", 4, 8, __import__("torch").float32)
+    assert L.pararnn_workspace_size(ctypes.byref(cell), 1, 10, 7) == 0
+
+
+def test_scan_workspace_sizes(L):
+    assert L.pararnn_affine_scan_workspace_size(16, 1024, 64, 0) > 0
+    assert L.pararnn_affine_scan_workspace_size(16, 1024, 62, 0) == 0
+    assert L.pararnn_affine_scan_workspace_size(0, 1024, 64, 0) == 0
+
+
+def test_invalid_arguments_are_rejected_without_a_gpu(L):
+    """Argument checks run on the host before anything is enqueued."""
+    cell = binding.make_cell("dense", 4, 8, __import__("torch").float32)
+    params = binding.Params(0, 0, 0, 0)
+    rc = L.pararnn_newton_solve(ctypes.byref(cell), ctypes.byref(params), None, None, 1, 10, 1,
+                                0.0, 1e-5, 0, None, None, None, 0, None)
+    assert rc == 3
+    rc = L.pararnn_affine_scan(None, None, None, 1, 10, 8, 0, None, None, 0, None)
+    assert rc == 3
