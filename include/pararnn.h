@@ -147,7 +147,8 @@ PARARNN_API size_t pararnn_workspace_size(const pararnn_cell *cell, int B, int T
  *                  DEER equals QUASI and ELK equals QUASI_ELK for it.
  *   lambda         LM damping (> 0) for ELK / QUASI_ELK; ignored otherwise.
  *   tol            convergence threshold on max |dh| (>= 0).
- *   max_iters      iteration cap; <= 0 means T.
+ *   max_iters      iteration cap; <= 0 means T + 1 (undamped Newton is exact
+ *                  after T iterations; one more observes delta = 0).
  *   h              DEVICE [B, T, D] float, output (the final iterate; h[:, t]
  *                  is h_{t+1}).  Must not alias any input or the workspace.
  *   info           HOST pararnn_info, output; may be NULL.

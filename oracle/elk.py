@@ -187,7 +187,7 @@ def elk_solve(cell: GRU, x: np.ndarray, h0: np.ndarray, mode: str, lam: float, t
     x = np.asarray(x, np.float64)
     h0 = np.asarray(h0, np.float64)
     B, T, _ = x.shape
-    max_iters = T if max_iters is None or max_iters <= 0 else max_iters
+    max_iters = T + 1 if max_iters is None or max_iters <= 0 else max_iters
     dense = mode == "ELK" and cell.kind == "dense"
     p = cell.project(x)
     h = np.zeros((B, T, cell.d))

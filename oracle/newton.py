@@ -23,7 +23,9 @@ Readings of what the pages leave open (also listed in the design notes):
     the next guess is h^(i+1)_t = A_t h^(i+1)_{t-1} + b_t, h^(i+1)_0 = h0;
   * convergence: delta = max over (b, t, d) of |h^(i+1) - h^(i)|; stop with
     iters = i + 1 when delta <= tol; a non-finite value anywhere stops with
-    DIVERGED; otherwise NOT_CONVERGED after max_iters (default T) iterations.
+    DIVERGED; otherwise NOT_CONVERGED after max_iters iterations.  The default
+    cap is T + 1: undamped Newton is exact after T iterations (each iteration
+    fixes one more leading state), and one more iteration observes delta = 0.
 """
 from __future__ import annotations
 
@@ -74,7 +76,7 @@ def newton_solve(cell: GRU, x: np.ndarray, h0: np.ndarray, mode: str, tol: float
     h0 = np.asarray(h0, np.float64)
     B, T, _ = x.shape
     D = cell.d
-    max_iters = T if max_iters is None or max_iters <= 0 else max_iters
+    max_iters = T + 1 if max_iters is None or max_iters <= 0 else max_iters
     dense = mode == "DEER" and cell.kind == "dense"
     p = cell.project(x)
     h = np.zeros((B, T, D)) if h_init is None else np.array(h_init, np.float64, copy=True)

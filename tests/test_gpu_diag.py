@@ -99,27 +99,40 @@ def test_each_iteration_matches_oracle(name, over, mode, lam):
 
 
 # --------------------------------------------------------- converged ---------
-@pytest.mark.parametrize("name,over,mode,lam", [
-    ("tiny", {}, "QUASI", 0.0),
-    ("untrained", dict(T=1024), "QUASI", 0.0),
-    ("untrained", dict(B=3, T=2049, bias_std=0.2, h0_std=0.5), "QUASI", 0.0),
-    ("diag", dict(B=2, T=513, d=512, din=128), "QUASI", 0.0),
-    ("diag", dict(B=1, T=100, d=68, din=20, h0_std=1.0), "DEER", 0.0),
-    ("near_unstable", dict(B=2, T=1000), "QUASI", 0.0),
-    ("near_unstable", dict(B=2, T=1000), "QUASI_ELK", 0.01),
-    ("near_unstable", dict(B=2, T=1000), "QUASI_ELK", 0.1),
+@pytest.mark.parametrize("name,over,mode", [
+    ("tiny", {}, "QUASI"),
+    ("untrained", dict(T=1024), "QUASI"),
+    ("untrained", dict(B=3, T=2049, bias_std=0.2, h0_std=0.5), "QUASI"),
+    ("diag", dict(B=2, T=513, d=512, din=128), "QUASI"),
+    ("diag", dict(B=1, T=100, d=68, din=20, h0_std=1.0), "DEER"),
+    ("near_unstable", dict(B=2, T=1000), "QUASI"),
 ])
-def test_converged_matches_rollout_and_counts(name, over, mode, lam):
+def test_converged_matches_rollout_and_counts(name, over, mode):
     kw = {k: over[k] for k in ("bias_std", "h0_std") if k in over}
     w = make_workload(name, **{k: v for k, v in over.items() if k not in kw}, **kw)
     c, x, h0 = _oracle(w)
     want = rollout(c, x, h0)
-    r = _gpu(w, mode, lam=lam)
+    r = _gpu(w, mode)
     assert r.status == "OK"
     assert np.max(np.abs(r.h.double().cpu().numpy() - want)) <= 1e-4
-    ref = (oracle.newton_solve(c, x, h0, mode, w.tol) if mode in ("QUASI", "DEER")
-           else oracle.elk_solve(c, x, h0, mode, lam, w.tol))
+    ref = oracle.newton_solve(c, x, h0, mode, w.tol)
     assert abs(r.iters - ref["iters"]) <= 1, (r.iters, ref["iters"])
+
+
+@pytest.mark.parametrize("lam", [0.01, 0.1, 1.0])
+def test_quasi_elk_matches_oracle_iterates(lam):
+    """Damped steps converge linearly, so at tol 1e-4 both solvers stop while
+    still up to ~1e-3 from the fixed point (the oracle too).  Gate: the count
+    within +-1 of the oracle's, and -- when the counts agree -- the final
+    iterate equal to the oracle's final iterate within 1e-4."""
+    w = make_workload("near_unstable", B=2, T=1000)
+    c, x, h0 = _oracle(w)
+    r = _gpu(w, "QUASI_ELK", lam=lam)
+    ref = oracle.elk_solve(c, x, h0, "QUASI_ELK", lam, w.tol)
+    assert r.status == "OK" and ref["status"] == "OK"
+    assert abs(r.iters - ref["iters"]) <= 1, (r.iters, ref["iters"])
+    if r.iters == ref["iters"]:
+        assert np.max(np.abs(r.h.double().cpu().numpy() - ref["h"])) <= 1e-4
 
 
 def test_quasi_elk_tight_tolerance_reaches_rollout():

@@ -259,6 +259,11 @@ def test_newton_counts_and_statuses():
     x_bad[0, 50, 0] = np.nan
     r = newton.newton_solve(c, x_bad, h0, "QUASI", w.tol)
     assert r["status"] == "DIVERGED" and r["iters"] == 1
+    # default cap T + 1: T = 1 is exact after one iteration, observed by the second
+    w1 = make_workload("tiny", T=1, h0_std=1.0)
+    r1 = newton.newton_solve(GRU.from_workload(w1), w1.x.double().numpy(),
+                             w1.h0.double().numpy(), "QUASI", 1e-12)
+    assert r1["status"] == "OK" and r1["iters"] == 2 and r1["deltas"][-1] == 0.0
     # the counting rule: iters is the first i+1 with delta_i <= tol
     r = newton.newton_solve(c, x, h0, "DEER", w.tol)
     assert r["deltas"][-1] <= w.tol and all(d > w.tol for d in r["deltas"][:-1])
