@@ -248,6 +248,34 @@ PARARNN_API int pararnn_affine_scan(const float *A, const float *b, const float 
  */
 PARARNN_API int pararnn_affine_scan_status(const void *workspace, pararnn_stream stream);
 
+/*
+ * pararnn_affine_scan_noalloc -- the diagonal scan of pararnn_affine_scan
+ * (dense == 0) for callers that cannot allocate device memory: plugins handed
+ * only their input and output buffers, code running where an allocator must
+ * not be entered, or paths that forbid allocation after start-up.  The pages
+ * have no counterpart; this is an interface for such callers.
+ *
+ * The scan's scratch (status header and look-back descriptors) is a
+ * file-scope device array of 16 MiB inside this library, created when the
+ * library's device code is loaded and held by every GPU that loads it until
+ * the process exits.  No call allocates or frees anything.
+ *   A, b, h0, h   as pararnn_affine_scan with dense == 0 (h may alias b).
+ *   status_dev    DEVICE unsigned, may be NULL: receives 0, or 1 if a bounded
+ *                 device-side wait expired (result unreliable).
+ * Limits: sizes whose scratch exceeds the array, i.e. 256 + 16 * L bytes with
+ * L = (number of 64-lane, 64-step tiles) * min(D, 64) > 16 MiB (about 2^24
+ * elements of B*T*D for D >= 64), are rejected with PARARNN_INVALID_ARG.
+ * The first call on each device looks the array's device address up with
+ * that device current; make that first call before any stream capture.
+ * Every call shares the one array and overwrites it (the parts that must
+ * start at zero are cleared on the stream first), so calls that overlap on
+ * the GPU -- on different streams, or from different host threads -- race.
+ * Asynchronous.  Returns PARARNN_OK, INVALID_ARG or CUDA_ERROR.
+ */
+PARARNN_API int pararnn_affine_scan_noalloc(const float *A, const float *b, const float *h0,
+                                            int B, int T, int D, float *h,
+                                            unsigned *status_dev, pararnn_stream stream);
+
 /* pararnn_status_string -- a static, human-readable name of a status code. */
 PARARNN_API const char *pararnn_status_string(int status);
 

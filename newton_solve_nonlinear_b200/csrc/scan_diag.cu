@@ -10,6 +10,8 @@
 // composes 4 steps x 4 lanes in registers, a shared-memory pass forms the
 // tile-local exclusive prefixes, one thread per lane resolves the carry with a
 // decoupled look-back, and the tile is re-swept and written with float4 stores.
+#include <mutex>
+
 #include "common.cuh"
 #include "lookback.cuh"
 #include "solver.cuh"
@@ -135,3 +137,77 @@ size_t scan_diag_ws_bytes(int B, int T, int D) {
 }
 
 }  // namespace pararnn
+
+// ---------------------------------------------------------------------------
+// The same scan for callers that cannot allocate device memory.
+//
+// Some callers cannot call cudaMalloc at the point where they need a scan:
+// code that runs while an allocator is locked or must not grow its memory
+// footprint, plugins handed only input and output buffers by a host framework,
+// and code paths where allocation is forbidden after start-up.  For them the
+// scan's scratch (a 256-byte status header and the look-back descriptors) lives
+// in the file-scope device array below, which the CUDA runtime creates when it
+// loads this library's device code; every GPU that loads the library holds it
+// until the process exits.
+// ---------------------------------------------------------------------------
+namespace pararnn {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+constexpr int kNoAllocMaxDevices = 64;
+
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+cudaError_t noalloc_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace pararnn
+
+extern "C" PARARNN_API int pararnn_affine_scan_noalloc(const float *A, const float *b,
+                                                       const float *h0, int B, int T, int D,
+                                                       float *h, unsigned *status_dev,
+                                                       pararnn_stream stream) {
+    using namespace pararnn;
+    if (B < 1 || T < 1 || D < 4 || D % 4 != 0) return PARARNN_INVALID_ARG;
+    if (static_cast<long long>(T) * D > (1ll << 31)) return PARARNN_INVALID_ARG;
+    if (!A || !b || !h0 || !h) return PARARNN_INVALID_ARG;
+    const auto al16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    if (!al16(A) || !al16(b) || !al16(h0) || !al16(h)) return PARARNN_INVALID_ARG;
+    if (status_dev && (reinterpret_cast<uintptr_t>(status_dev) & 3u) != 0) return PARARNN_INVALID_ARG;
+    if (scan_diag_ws_bytes(B, T, D) > kNoAllocScratchBytes) return PARARNN_INVALID_ARG;
+    const size_t nh = static_cast<size_t>(B) * T * D * 4;
+    const auto over = [](const void *x, size_t nx, const void *y, size_t ny) {
+        const auto px = reinterpret_cast<uintptr_t>(x), py = reinterpret_cast<uintptr_t>(y);
+        return px < py + ny && py < px + nx;
+    };
+    if (over(h, nh, A, nh) || over(h, nh, h0, static_cast<size_t>(B) * D * 4)) return PARARNN_INVALID_ARG;
+    void *scratch = nullptr;
+    if (noalloc_scratch(&scratch) != cudaSuccess) return PARARNN_CUDA_ERROR;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // launch_scan_diag first clears the header and the descriptors it will use
+    cudaError_t e = launch_scan_diag(A, b, h0, B, T, D, h, scratch, s);
+    if (e == cudaSuccess && status_dev)
+        e = cudaMemcpyAsync(status_dev, &static_cast<WsHeader *>(scratch)->status, sizeof(unsigned),
+                            cudaMemcpyDeviceToDevice, s);
+    return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
+}
