@@ -157,6 +157,19 @@ __device__ __forceinline__ unsigned block_max_u32(unsigned v, unsigned *red /*[3
     return r;
 }
 
+// (c0, c1) += (a0, a1) * h as one packed fp32x2 FMA (sm_100 f32x2 datapath:
+// the same fp32 rounding as two FFMAs, half the issued instructions).
+__device__ __forceinline__ void ffma2(float &c0, float &c1, float a0, float a1, float h) {
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %4};\n\t"
+        "mov.b64 rc, {%0, %1};\n\t"
+        "fma.rn.f32x2 rc, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rc;\n\t}"
+        : "+f"(c0), "+f"(c1)
+        : "f"(a0), "f"(a1), "f"(h));
+}
+
 __device__ __forceinline__ float4 ldcg4(const float *p) {
     return __ldcg(reinterpret_cast<const float4 *>(p));
 }

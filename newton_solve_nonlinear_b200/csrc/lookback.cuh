@@ -13,35 +13,112 @@
 
 namespace pararnn {
 
+// Every descriptor word carries its own tag (epoch and state) next to its
+// value in one 64-bit word, and each (epoch, state) value is written once, so a
+// word whose tag matches *is* the value: no acquire/release ordering is needed
+// between words.  The look-back therefore reads predecessors with relaxed
+// loads in batches of up to kWin tiles, which resolves a chain of aggregates in
+// about one L2 round trip per batch instead of one per tile.
+constexpr int kWin = 4;
+
+__device__ __forceinline__ bool word_ready(unsigned long long w, unsigned epoch) {
+    const unsigned t = word_tag(w);
+    return (t >> 2) == epoch && (t & 3u) != 0u;
+}
+
+// Spin until the word carries this epoch in any published state; 0 on timeout.
+__device__ __forceinline__ unsigned long long wait_ready(const unsigned long long *p,
+                                                         unsigned epoch, unsigned *status) {
+    long long spins = 0;
+    while (true) {
+        const unsigned long long w = ld_relaxed(p);
+        if (word_ready(w, epoch)) return w;
+        if (++spins > 64) {
+            if ((spins & 1023) == 0 && timed_out(status)) return 0ull;
+            if (spins > kSpinBudget) {
+                flag_timeout(status);
+                return 0ull;
+            }
+            __nanosleep(32);
+        }
+    }
+}
+
+// Spin until the word carries exactly `tag`; 0 on timeout.
+__device__ __forceinline__ unsigned long long wait_tag(const unsigned long long *p, unsigned tag,
+                                                       unsigned *status) {
+    long long spins = 0;
+    while (true) {
+        const unsigned long long w = ld_relaxed(p);
+        if (word_tag(w) == tag) return w;
+        if (++spins > 64) {
+            if ((spins & 1023) == 0 && timed_out(status)) return 0ull;
+            if (spins > kSpinBudget) {
+                flag_timeout(status);
+                return 0ull;
+            }
+            __nanosleep(32);
+        }
+    }
+}
+
 // Affine maps x -> A x + B.  Descriptor slot = 2 words: [0] tag|A (or tag|INC
-// value), [1] tag|B.  `step` is the tile distance to the predecessor (+-n_groups).
+// value), [1] tag|B.  `step` is the tile distance to the predecessor
+// (+n_groups forward, -n_groups for a reverse scan); `avail` is the number of
+// predecessors (0: this tile's carry-in is `carry0`).
 __device__ __forceinline__ float lookback_affine(unsigned long long *desc, long long tile,
                                                  long long step, int DG, int lane, unsigned epoch,
-                                                 float EA, float EB, bool first, float carry0,
+                                                 float EA, float EB, int avail, float carry0,
                                                  unsigned *status) {
     unsigned long long *mine = desc + (static_cast<size_t>(tile) * DG + lane) * 2;
     float hin = carry0;
-    if (!first) {
-        st_relaxed(mine + 1, pack_word(make_tag(epoch, kStateAgg), EB));
-        st_release(mine, pack_word(make_tag(epoch, kStateAgg), EA));
+    if (avail > 0) {
+        const unsigned tag_agg = make_tag(epoch, kStateAgg);
+        st_relaxed(mine + 1, pack_word(tag_agg, EB));
+        st_relaxed(mine, pack_word(tag_agg, EA));
         float accA = 1.f, accB = 0.f;
         long long j = tile - step;
-        while (true) {
-            unsigned long long *pj = desc + (static_cast<size_t>(j) * DG + lane) * 2;
-            const unsigned long long w = wait_word(pj, epoch, status);
-            if (w == 0ull) { hin = 0.f; break; }
-            if ((word_tag(w) & 3u) == kStateInc) {
-                hin = fmaf(accA, word_val(w), accB);
-                break;
-            }
-            const unsigned long long w1 = ld_relaxed(pj + 1);
-            const float Aj = word_val(w), Bj = word_val(w1);
-            accB = fmaf(accA, Bj, accB);
-            accA = accA * Aj;
-            j -= step;
+        int left = avail;
+        bool done = false;
+        while (!done && left > 0) {
+            const int n = left < kWin ? left : kWin;
+            unsigned long long w0[kWin], w1[kWin];
+#pragma unroll
+            for (int q = 0; q < kWin; ++q)
+                if (q < n) {
+                    const unsigned long long *p = desc + (static_cast<size_t>(j - q * step) * DG + lane) * 2;
+                    w0[q] = ld_relaxed(p);
+                    w1[q] = ld_relaxed(p + 1);
+                }
+#pragma unroll
+            for (int q = 0; q < kWin; ++q)
+                if (q < n && !done) {
+                    const unsigned long long *p = desc + (static_cast<size_t>(j - q * step) * DG + lane) * 2;
+                    unsigned long long a = w0[q];
+                    if (!word_ready(a, epoch)) a = wait_ready(p, epoch, status);
+                    if (a == 0ull) {
+                        hin = 0.f;
+                        done = true;
+                    } else if ((word_tag(a) & 3u) == kStateInc) {
+                        hin = fmaf(accA, word_val(a), accB);
+                        done = true;
+                    } else {
+                        unsigned long long bw = w1[q];
+                        if (word_tag(bw) != word_tag(a)) bw = wait_tag(p + 1, word_tag(a), status);
+                        if (bw == 0ull) {
+                            hin = 0.f;
+                            done = true;
+                        } else {
+                            accB = fmaf(accA, word_val(bw), accB);
+                            accA = accA * word_val(a);
+                        }
+                    }
+                }
+            j -= static_cast<long long>(n) * step;
+            left -= n;
         }
     }
-    st_release(mine, pack_word(make_tag(epoch, kStateInc), fmaf(EA, hin, EB)));
+    st_relaxed(mine, pack_word(make_tag(epoch, kStateInc), fmaf(EA, hin, EB)));
     return hin;
 }
 
@@ -63,33 +140,66 @@ __device__ __forceinline__ float mob_apply(const Mob &x, float P) {
 
 __device__ __forceinline__ float lookback_mobius(unsigned long long *desc, long long tile,
                                                  long long step, int DG, int lane, unsigned epoch,
-                                                 const Mob &E, bool first, float carry0,
+                                                 const Mob &E, int avail, float carry0,
                                                  unsigned *status) {
+    constexpr int W = kWin;
     unsigned long long *mine = desc + (static_cast<size_t>(tile) * DG + lane) * 4;
     float pin = carry0;
-    if (!first) {
+    if (avail > 0) {
         const unsigned tg = make_tag(epoch, kStateAgg);
         st_relaxed(mine + 1, pack_word(tg, E.m1));
         st_relaxed(mine + 2, pack_word(tg, E.m2));
         st_relaxed(mine + 3, pack_word(tg, E.m3));
-        st_release(mine, pack_word(tg, E.m0));
+        st_relaxed(mine, pack_word(tg, E.m0));
         Mob acc{1.f, 0.f, 0.f, 1.f};
         long long j = tile - step;
-        while (true) {
-            unsigned long long *pj = desc + (static_cast<size_t>(j) * DG + lane) * 4;
-            const unsigned long long w = wait_word(pj, epoch, status);
-            if (w == 0ull) { pin = 0.f; break; }
-            if ((word_tag(w) & 3u) == kStateInc) {
-                pin = mob_apply(acc, word_val(w));
-                break;
-            }
-            Mob Mj{word_val(w), word_val(ld_relaxed(pj + 1)), word_val(ld_relaxed(pj + 2)),
-                   word_val(ld_relaxed(pj + 3))};
-            acc = mob_mul(acc, Mj);
-            j -= step;
+        int left = avail;
+        bool done = false;
+        while (!done && left > 0) {
+            const int n = left < W ? left : W;
+            unsigned long long w[W][4];
+#pragma unroll
+            for (int q = 0; q < W; ++q)
+                if (q < n) {
+                    const unsigned long long *p = desc + (static_cast<size_t>(j - q * step) * DG + lane) * 4;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) w[q][e] = ld_relaxed(p + e);
+                }
+#pragma unroll
+            for (int q = 0; q < W; ++q)
+                if (q < n && !done) {
+                    const unsigned long long *p = desc + (static_cast<size_t>(j - q * step) * DG + lane) * 4;
+                    unsigned long long a = w[q][0];
+                    if (!word_ready(a, epoch)) a = wait_ready(p, epoch, status);
+                    if (a == 0ull) {
+                        pin = 0.f;
+                        done = true;
+                    } else if ((word_tag(a) & 3u) == kStateInc) {
+                        pin = mob_apply(acc, word_val(a));
+                        done = true;
+                    } else {
+                        float m[3];
+                        bool ok = true;
+#pragma unroll
+                        for (int e = 1; e < 4; ++e) {
+                            unsigned long long v = w[q][e];
+                            if (word_tag(v) != word_tag(a)) v = wait_tag(p + e, word_tag(a), status);
+                            if (v == 0ull) ok = false;
+                            m[e - 1] = word_val(v);
+                        }
+                        if (!ok) {
+                            pin = 0.f;
+                            done = true;
+                        } else {
+                            acc = mob_mul(acc, Mob{word_val(a), m[0], m[1], m[2]});
+                        }
+                    }
+                }
+            j -= static_cast<long long>(n) * step;
+            left -= n;
         }
     }
-    st_release(mine, pack_word(make_tag(epoch, kStateInc), mob_apply(E, pin)));
+    st_relaxed(mine, pack_word(make_tag(epoch, kStateInc), mob_apply(E, pin)));
     return pin;
 }
 

@@ -39,12 +39,12 @@
 
 namespace pararnn {
 
-Tiling make_tiling(int B, int T, int D, bool dense_cell) {
+Tiling make_tiling(int B, int T, int D, bool dense_cell, int TK) {
     Tiling t{};
     t.DG = dense_cell ? D : (D < 64 ? D : 64);
     t.DB = t.DG / 4;
     t.NTB = kThreads / t.DB;
-    t.TK = 4;
+    t.TK = TK;
     t.L = t.NTB * t.TK;
     t.n_dgroups = (D + t.DG - 1) / t.DG;
     t.n_groups = B * t.n_dgroups;
@@ -55,14 +55,13 @@ Tiling make_tiling(int B, int T, int D, bool dense_cell) {
 
 namespace {
 
-constexpr int TK = 4;
-
 struct TileCoord {
     long long tile;
     int chunk, b, dg, db, tb, lane0, d0, t0, tile_t0;
     bool active, dvalid;
 };
 
+template <int TK>
 __device__ __forceinline__ TileCoord tile_coord(const DiagArgs &A, long long tile) {
     TileCoord c;
     const Tiling &tl = A.tl;
@@ -86,28 +85,48 @@ __device__ __forceinline__ TileCoord tile_coord(const DiagArgs &A, long long til
 struct Smem {
     float *Us;    // dense: [D][3][DG]
     float *hs;    // dense: [L+1][D]   guess rows tile_t0-1 .. tile_t0+L-1
+    float *aby;   // dense-mma: a, bb, y of the tile [3][L][D+4]
     float *s0, *s1, *s2, *s3;  // [NTB][DG] scan scratch
     float *c0, *c1;            // [DG] carries
     unsigned *red;             // [32]
 };
 
-__host__ __device__ inline size_t smem_floats(const Tiling &tl, int D, bool dense) {
+// Cell variants of the solver kernels.
+constexpr int kCellDiag = 0;      // diagonal recurrence: u_g * h, no product
+constexpr int kCellDenseFma = 1;  // dense U h in fp32 FMAs (any D multiple of 4)
+constexpr int kCellDenseMma = 2;  // dense U h on tensor cores, 3 x TF32 (D in 8,16,32,64)
+
+__host__ __device__ inline int mma_stride(int D) { return D + 4; }  // padded rows: no bank conflicts
+
+__host__ __device__ inline size_t smem_floats(const Tiling &tl, int D, int cell) {
     size_t n = 0;
-    if (dense) n += static_cast<size_t>(D) * 3 * tl.DG + static_cast<size_t>(tl.L + 1) * D;
+    if (cell == kCellDenseFma)
+        n += static_cast<size_t>(D) * 3 * tl.DG + static_cast<size_t>(tl.L + 1) * D;
+    if (cell == kCellDenseMma) {
+        const size_t S = mma_stride(D);
+        n += static_cast<size_t>(tl.L + 1) * S + 3 * static_cast<size_t>(tl.L) * S;
+    }
     n += 4 * static_cast<size_t>(tl.NTB) * tl.DG + 2 * tl.DG + 32;
     return n;
 }
 
-__device__ __forceinline__ Smem carve(float *base, const Tiling &tl, int D, bool dense) {
+__device__ __forceinline__ Smem carve(float *base, const Tiling &tl, int D, int cell) {
     Smem s;
     float *p = base;
     s.Us = p;
     s.hs = p;
-    if (dense) {
+    s.aby = p;
+    if (cell == kCellDenseFma) {
         s.Us = p;
         p += static_cast<size_t>(D) * 3 * tl.DG;
         s.hs = p;
         p += static_cast<size_t>(tl.L + 1) * D;
+    } else if (cell == kCellDenseMma) {
+        const size_t S = mma_stride(D);
+        s.hs = p;
+        p += static_cast<size_t>(tl.L + 1) * S;
+        s.aby = p;
+        p += 3 * static_cast<size_t>(tl.L) * S;
     }
     const size_t n = static_cast<size_t>(tl.NTB) * tl.DG;
     s.s0 = p; p += n;
@@ -120,16 +139,197 @@ __device__ __forceinline__ Smem carve(float *base, const Tiling &tl, int D, bool
     return s;
 }
 
+// One state of the cell and its Jacobian diagonal.  pr, pz, pn: input
+// pre-activations (b_ih included); gr, gz, gnh: recurrent sums U_g h (or
+// u_g * h); bh: b_hh; ud: diagonal entries of U_g; h: guess at t-1; hc: guess
+// at t.  Returns a = dJ_tt and bb = f - a h, and folds |hc - f| into rmax.
+__device__ __forceinline__ void cell_state(float pr, float pz, float pn, float gr, float gz,
+                                           float gnh, float bhr, float bhz, float bhn, float udr,
+                                           float udz, float udn, float h, float hc, float &a,
+                                           float &bb, unsigned &rmax) {
+    const float r = sigmoidf_(pr + gr + bhr);
+    const float z = sigmoidf_(pz + gz + bhz);
+    const float gn = gnh + bhn;
+    const float n = tanhf_(pn + r * gn);
+    const float f = n + z * (h - n);
+    const float omz = 1.f - z;
+    const float cz = (h - n) * z * omz;
+    const float cn = omz * (1.f - n * n) * r;
+    const float cr = cn * gn * (1.f - r);
+    a = z + cz * udz + cn * udn + cr * udr;
+    bb = f - a * h;
+    rmax = max(rmax, abs_bits(hc - f));
+}
+
+__device__ __forceinline__ void mma_tf32(float (&c)[4], const unsigned (&a)[4], unsigned b0,
+                                         unsigned b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// x = hi + lo with hi exactly representable in TF32 (top 10 mantissa bits) and
+// lo the exact fp32 remainder; hi*hi + hi*lo + lo*hi then carries a product to
+// ~2^-21 relative accuracy (the error-compensated 3 x TF32 split).
+__device__ __forceinline__ void split_tf32(float x, unsigned &hi, unsigned &lo) {
+    hi = __float_as_uint(x) & 0xffffe000u;
+    lo = __float_as_uint(x - __uint_as_float(hi));
+}
+
+// Dense cell with U h on the tensor cores.  Warp w owns lane block
+// lb = w % (D/8) (8 state lanes) and two 16-step row blocks of the tile; its
+// mma.sync m16n8k8 fragments hold, per thread, the three gates of the same
+// (step, lane) pairs, so the cell is evaluated straight from the accumulators.
+// a, bb, y go through shared memory to the (thread row, float4 column) layout
+// of the scan.
+template <int TK>
+__device__ __forceinline__ void linearise_mma(const DiagArgs &A, const TileCoord &c, const Smem &sm,
+                                              const float *hold, bool zero_guess, float (&a)[TK][4],
+                                              float (&bb)[TK][4], float (&y)[TK][4],
+                                              unsigned &rmax) {
+    const int D = A.D, T = A.T, L = A.tl.L;
+    const int S = mma_stride(D);
+    const int nq = D / 4, nvec = (L + 1) * nq;
+    for (int i = threadIdx.x; i < nvec; i += kThreads) {
+        const int r = i / nq, col = (i % nq) * 4;
+        const int t = c.tile_t0 - 1 + r;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (t < 0)
+            v = __ldg(reinterpret_cast<const float4 *>(A.h0 + static_cast<size_t>(c.b) * D + col));
+        else if (!zero_guess && t < T)
+            v = ldcg4(hold + (static_cast<size_t>(c.b) * T + t) * D + col);
+        *reinterpret_cast<float4 *>(sm.hs + static_cast<size_t>(r) * S + col) = v;
+    }
+    __syncthreads();
+    {
+        const int lid = threadIdx.x & 31, w = threadIdx.x >> 5;
+        const int gid = lid >> 2, tq = lid & 3;
+        const int LB = D / 8;
+        const int lb = w % LB;
+        const int row0 = (w / LB) * 32;  // first tile step of the warp's two row blocks
+        float acc[2][3][4];
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int g = 0; g < 3; ++g)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[m][g][e] = 0.f;
+        // U_g rows of this warp's 8 lanes, read through L1 (48 KB, shared by all CTAs)
+        const float *urow[3];
+#pragma unroll
+        for (int g = 0; g < 3; ++g) urow[g] = A.w_hh + static_cast<size_t>(g * D + lb * 8 + gid) * D;
+        // input pre-activations of this thread's (step, lane-pair) slots, issued
+        // before the products so that their latency overlaps the MMAs
+        const int l0 = lb * 8 + 2 * tq;  // lanes l0, l0 + 1
+        float2 pv[2][2][3];
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int t = c.tile_t0 + row0 + m * 16 + gid + hh * 8;
+                const float *prow = A.P + (static_cast<size_t>(c.b) * T + (t < T ? t : T - 1)) * 3 * D + l0;
+#pragma unroll
+                for (int g = 0; g < 3; ++g) pv[m][hh][g] = __ldg(reinterpret_cast<const float2 *>(prow + g * D));
+            }
+        for (int k0 = 0; k0 < D; k0 += 8) {
+            unsigned bh[3][2], bl[3][2];
+#pragma unroll
+            for (int g = 0; g < 3; ++g) {
+                split_tf32(__ldg(urow[g] + k0 + tq), bh[g][0], bl[g][0]);
+                split_tf32(__ldg(urow[g] + k0 + tq + 4), bh[g][1], bl[g][1]);
+            }
+            unsigned ah[2][4], al[2][4];
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const float *r0 = sm.hs + static_cast<size_t>(row0 + m * 16 + gid) * S + k0 + tq;
+                const float *r1 = r0 + 8 * S;
+                split_tf32(r0[0], ah[m][0], al[m][0]);
+                split_tf32(r1[0], ah[m][1], al[m][1]);
+                split_tf32(r0[4], ah[m][2], al[m][2]);
+                split_tf32(r1[4], ah[m][3], al[m][3]);
+            }
+            // small terms first; six independent accumulators between dependent MMAs
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+#pragma unroll
+                for (int g = 0; g < 3; ++g) mma_tf32(acc[m][g], al[m], bh[g][0], bh[g][1]);
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+#pragma unroll
+                for (int g = 0; g < 3; ++g) mma_tf32(acc[m][g], ah[m], bl[g][0], bl[g][1]);
+#pragma unroll
+            for (int m = 0; m < 2; ++m)
+#pragma unroll
+                for (int g = 0; g < 3; ++g) mma_tf32(acc[m][g], ah[m], bh[g][0], bh[g][1]);
+        }
+        // the cell for this thread's (step, lane) pairs
+        float bh2[3][2], ud2[3][2];
+#pragma unroll
+        for (int g = 0; g < 3; ++g) {
+            const float2 v = __ldg(reinterpret_cast<const float2 *>(A.b_hh + g * D + l0));
+            bh2[g][0] = v.x;
+            bh2[g][1] = v.y;
+            ud2[g][0] = __ldg(A.w_hh + static_cast<size_t>(g * D + l0) * D + l0);
+            ud2[g][1] = __ldg(A.w_hh + static_cast<size_t>(g * D + l0 + 1) * D + l0 + 1);
+        }
+        float *sa = sm.aby, *sb = sm.aby + static_cast<size_t>(L) * S, *sy = sb + static_cast<size_t>(L) * S;
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int tl_ = row0 + m * 16 + gid + hh * 8;  // tile-local step
+                const int t = c.tile_t0 + tl_;
+                float2 av = make_float2(1.f, 1.f), bv = make_float2(0.f, 0.f), yv = make_float2(0.f, 0.f);
+                if (t < T) {
+                    const float2 pr = pv[m][hh][0], pz = pv[m][hh][1], pn = pv[m][hh][2];
+                    const float2 hp = *reinterpret_cast<const float2 *>(sm.hs + static_cast<size_t>(tl_) * S + l0);
+                    yv = *reinterpret_cast<const float2 *>(sm.hs + static_cast<size_t>(tl_ + 1) * S + l0);
+                    cell_state(pr.x, pz.x, pn.x, acc[m][0][hh * 2], acc[m][1][hh * 2],
+                               acc[m][2][hh * 2], bh2[0][0], bh2[1][0], bh2[2][0], ud2[0][0],
+                               ud2[1][0], ud2[2][0], hp.x, yv.x, av.x, bv.x, rmax);
+                    cell_state(pr.y, pz.y, pn.y, acc[m][0][hh * 2 + 1], acc[m][1][hh * 2 + 1],
+                               acc[m][2][hh * 2 + 1], bh2[0][1], bh2[1][1], bh2[2][1], ud2[0][1],
+                               ud2[1][1], ud2[2][1], hp.y, yv.y, av.y, bv.y, rmax);
+                }
+                const size_t off = static_cast<size_t>(tl_) * S + l0;
+                *reinterpret_cast<float2 *>(sa + off) = av;
+                *reinterpret_cast<float2 *>(sb + off) = bv;
+                *reinterpret_cast<float2 *>(sy + off) = yv;
+            }
+    }
+    __syncthreads();
+    if (c.active) {
+        const float *sa = sm.aby, *sb = sm.aby + static_cast<size_t>(L) * S, *sy = sb + static_cast<size_t>(L) * S;
+#pragma unroll
+        for (int k = 0; k < TK; ++k) {
+            const size_t off = static_cast<size_t>(c.tb * TK + k) * S + c.d0;
+            const float4 av = *reinterpret_cast<const float4 *>(sa + off);
+            const float4 bv = *reinterpret_cast<const float4 *>(sb + off);
+            const float4 yv = *reinterpret_cast<const float4 *>(sy + off);
+            a[k][0] = av.x; a[k][1] = av.y; a[k][2] = av.z; a[k][3] = av.w;
+            bb[k][0] = bv.x; bb[k][1] = bv.y; bb[k][2] = bv.z; bb[k][3] = bv.w;
+            y[k][0] = yv.x; y[k][1] = yv.y; y[k][2] = yv.z; y[k][3] = yv.w;
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------
 // 1. linearisation at the shifted guess
 // ---------------------------------------------------------------------------
 // Produces, for the thread's TK x 4 states: a (diag of the Jacobian), bb
 // (f - a h_{t-1}) and y (the guess at t).  Steps past T or lanes past D get
 // the identity map (a = 1, bb = 0).
-template <bool DENSE>
+template <int CELL, int TK>
 __device__ __forceinline__ void linearise(const DiagArgs &A, const TileCoord &c, const Smem &sm,
                                           const float *hold, bool zero_guess, float (&a)[TK][4],
                                           float (&bb)[TK][4], float (&y)[TK][4], unsigned &rmax) {
+    if (CELL == kCellDenseMma) {
+        linearise_mma<TK>(A, c, sm, hold, zero_guess, a, bb, y, rmax);
+        return;
+    }
+    constexpr bool DENSE = CELL == kCellDenseFma;
     const int D = A.D, T = A.T;
     const size_t rowP = 3 * static_cast<size_t>(D);
     float hp[TK + 1][4];
@@ -174,18 +374,12 @@ __device__ __forceinline__ void linearise(const DiagArgs &A, const TileCoord &c,
 #pragma unroll
                     for (int k = 0; k < TK; ++k) {
                         const float h = get(hv[k], mm);
-                        G[0][k][0] = fmaf(u0.x, h, G[0][k][0]);
-                        G[0][k][1] = fmaf(u0.y, h, G[0][k][1]);
-                        G[0][k][2] = fmaf(u0.z, h, G[0][k][2]);
-                        G[0][k][3] = fmaf(u0.w, h, G[0][k][3]);
-                        G[1][k][0] = fmaf(u1.x, h, G[1][k][0]);
-                        G[1][k][1] = fmaf(u1.y, h, G[1][k][1]);
-                        G[1][k][2] = fmaf(u1.z, h, G[1][k][2]);
-                        G[1][k][3] = fmaf(u1.w, h, G[1][k][3]);
-                        G[2][k][0] = fmaf(u2.x, h, G[2][k][0]);
-                        G[2][k][1] = fmaf(u2.y, h, G[2][k][1]);
-                        G[2][k][2] = fmaf(u2.z, h, G[2][k][2]);
-                        G[2][k][3] = fmaf(u2.w, h, G[2][k][3]);
+                        ffma2(G[0][k][0], G[0][k][1], u0.x, u0.y, h);
+                        ffma2(G[0][k][2], G[0][k][3], u0.z, u0.w, h);
+                        ffma2(G[1][k][0], G[1][k][1], u1.x, u1.y, h);
+                        ffma2(G[1][k][2], G[1][k][3], u1.z, u1.w, h);
+                        ffma2(G[2][k][0], G[2][k][1], u2.x, u2.y, h);
+                        ffma2(G[2][k][2], G[2][k][3], u2.z, u2.w, h);
                     }
                 }
             }
@@ -266,6 +460,7 @@ __device__ __forceinline__ void linearise(const DiagArgs &A, const TileCoord &c,
 // ---------------------------------------------------------------------------
 // Forward affine scan of (a, bb) with the carry from the previous chunk; writes
 // out[k][j] = state at step t0+k.  All threads of the CTA must call it.
+template <int TK>
 __device__ __forceinline__ void scan_forward(const DiagArgs &A, const TileCoord &c, const Smem &sm,
                                              unsigned long long *desc, unsigned epoch,
                                              const float (&a)[TK][4], const float (&bb)[TK][4],
@@ -300,7 +495,7 @@ __device__ __forceinline__ void scan_forward(const DiagArgs &A, const TileCoord 
             EA = qa * EA;
         }
         sm.c0[lane] = lookback_affine(desc, c.tile, tl.n_groups, tl.DG, lane, epoch, EA, EB,
-                                      c.chunk == 0, carry0[lane], &A.hdr->status);
+                                      c.chunk, carry0[lane], &A.hdr->status);
     }
     __syncthreads();
     if (c.active) {
@@ -318,6 +513,7 @@ __device__ __forceinline__ void scan_forward(const DiagArgs &A, const TileCoord 
     __syncthreads();
 }
 
+template <int TK>
 __device__ __forceinline__ void store_states(const DiagArgs &A, const TileCoord &c, float *dst,
                                              const float (&v)[TK][4]) {
     if (!c.dvalid) return;
@@ -330,6 +526,7 @@ __device__ __forceinline__ void store_states(const DiagArgs &A, const TileCoord 
     }
 }
 
+template <int TK>
 __device__ __forceinline__ void load_states(const DiagArgs &A, const TileCoord &c, const float *src,
                                             int shift, float (&v)[TK][4], float fill) {
 #pragma unroll
@@ -351,14 +548,14 @@ __device__ __forceinline__ void load_h0_carry(const DiagArgs &A, const TileCoord
 }
 
 // --- quasi-DEER tile: linearise, scan, write, reduce ------------------------
-template <bool DENSE>
+template <int CELL, int TK>
 __device__ void quasi_tile(const DiagArgs &A, long long tile, const Smem &sm, const float *hold,
                            float *hnew, bool zero_guess, unsigned epoch, unsigned &dmax,
                            unsigned &rmax) {
-    const TileCoord c = tile_coord(A, tile);
+    const TileCoord c = tile_coord<TK>(A, tile);
     float a[TK][4], bb[TK][4], y[TK][4], out[TK][4];
     load_h0_carry(A, c, sm);
-    linearise<DENSE>(A, c, sm, hold, zero_guess, a, bb, y, rmax);
+    linearise<CELL, TK>(A, c, sm, hold, zero_guess, a, bb, y, rmax);
     scan_forward(A, c, sm, A.desc, epoch, a, bb, sm.c1, out);
     if (c.dvalid) {
 #pragma unroll
@@ -371,16 +568,16 @@ __device__ void quasi_tile(const DiagArgs &A, long long tile, const Smem &sm, co
 }
 
 // --- quasi-ELK forward tile: Kalman covariance (Mobius) + filtered mean -------
-template <bool DENSE>
+template <int CELL, int TK>
 __device__ void elk_forward_tile(const DiagArgs &A, long long tile, const Smem &sm,
                                  const float *hold, bool zero_guess, unsigned epoch,
                                  unsigned &rmax) {
     const Tiling &tl = A.tl;
-    const TileCoord c = tile_coord(A, tile);
+    const TileCoord c = tile_coord<TK>(A, tile);
     const float lam = A.lambda;
     float a[TK][4], bb[TK][4], y[TK][4];
     load_h0_carry(A, c, sm);
-    linearise<DENSE>(A, c, sm, hold, zero_guess, a, bb, y, rmax);
+    linearise<CELL, TK>(A, c, sm, hold, zero_guess, a, bb, y, rmax);
 
     unsigned long long *desc_cov = A.desc;
     unsigned long long *desc_mean = A.desc + static_cast<size_t>(tl.n_tiles) * tl.DG * 4;
@@ -415,7 +612,7 @@ __device__ void elk_forward_tile(const DiagArgs &A, long long tile, const Smem &
             E = mob_mul(Q, E);
         }
         sm.c0[lane] = lookback_mobius(desc_cov, c.tile, tl.n_groups, tl.DG, lane, epoch, E,
-                                      c.chunk == 0, 0.f, &A.hdr->status);
+                                      c.chunk, 0.f, &A.hdr->status);
     }
     __syncthreads();
     float Pk[TK][4], al[TK][4], be[TK][4];
@@ -449,11 +646,12 @@ __device__ void elk_forward_tile(const DiagArgs &A, long long tile, const Smem &
 }
 
 // --- quasi-ELK backward tile: RTS smoother as a reverse affine scan ----------
+template <int TK>
 __device__ void elk_backward_tile(const DiagArgs &A, long long tile, const Smem &sm,
                                   const float *hold, float *hnew, bool zero_guess,
                                   unsigned epoch, unsigned &dmax) {
     const Tiling &tl = A.tl;
-    const TileCoord c = tile_coord(A, tile);
+    const TileCoord c = tile_coord<TK>(A, tile);
     unsigned long long *desc_bwd = A.desc + static_cast<size_t>(tl.n_tiles) * tl.DG * 6;
     float m[TK][4], P[TK][4], an[TK][4], bn[TK][4], y[TK][4];
     load_states(A, c, A.elk_m, 0, m, 0.f);
@@ -513,7 +711,7 @@ __device__ void elk_backward_tile(const DiagArgs &A, long long tile, const Smem 
             EG = qg * EG;
         }
         sm.c0[lane] = lookback_affine(desc_bwd, c.tile, -static_cast<long long>(tl.n_groups),
-                                      tl.DG, lane, epoch, EG, EC, c.chunk == tl.n_chunks - 1,
+                                      tl.DG, lane, epoch, EG, EC, tl.n_chunks - 1 - c.chunk,
                                       0.f, &A.hdr->status);
     }
     __syncthreads();
@@ -544,16 +742,16 @@ __device__ void elk_backward_tile(const DiagArgs &A, long long tile, const Smem 
 // ---------------------------------------------------------------------------
 // 4. the persistent kernel
 // ---------------------------------------------------------------------------
-template <bool DENSE, bool ELK>
-__global__ void __launch_bounds__(kThreads, 1) diag_solver_kernel(DiagArgs A) {
+template <int CELL, bool ELK, int TK>
+__global__ void __launch_bounds__(kThreads, ELK ? 1 : 2) diag_solver_kernel(DiagArgs A) {
     extern __shared__ float4 smem_raw[];
     const Tiling &tl = A.tl;
-    const Smem sm = carve(reinterpret_cast<float *>(smem_raw), tl, A.D, DENSE);
+    const Smem sm = carve(reinterpret_cast<float *>(smem_raw), tl, A.D, CELL);
     WsHeader *hdr = A.hdr;
     unsigned *status = &hdr->status;
     const unsigned nblocks = gridDim.x;
 
-    if (DENSE) {
+    if (CELL == kCellDenseFma) {
         // U^T slices into shared memory, layout [m][g][lane]: Us = U_g[lane][m]
         const int D = A.D, n = D * 3 * tl.DG;
         for (int i = threadIdx.x; i < n; i += kThreads) {
@@ -579,13 +777,13 @@ __global__ void __launch_bounds__(kThreads, 1) diag_solver_kernel(DiagArgs A) {
         unsigned dmax = 0u, rmax = 0u;
         if (!ELK) {
             for (long long tile = blockIdx.x; tile < tl.n_tiles; tile += nblocks)
-                quasi_tile<DENSE>(A, tile, sm, hold, hnew, zero_guess, epoch, dmax, rmax);
+                quasi_tile<CELL, TK>(A, tile, sm, hold, hnew, zero_guess, epoch, dmax, rmax);
         } else {
             for (long long tile = blockIdx.x; tile < tl.n_tiles; tile += nblocks)
-                elk_forward_tile<DENSE>(A, tile, sm, hold, zero_guess, epoch, rmax);
+                elk_forward_tile<CELL, TK>(A, tile, sm, hold, zero_guess, epoch, rmax);
             grid_barrier(hdr->barrier, nblocks, status);
             for (long long k = blockIdx.x; k < tl.n_tiles; k += nblocks)
-                elk_backward_tile(A, tl.n_tiles - 1 - k, sm, hold, hnew, zero_guess, epoch, dmax);
+                elk_backward_tile<TK>(A, tl.n_tiles - 1 - k, sm, hold, hnew, zero_guess, epoch, dmax);
         }
         const unsigned bd = block_max_u32(dmax, sm.red);
         const unsigned br = block_max_u32(rmax, sm.red);
@@ -621,10 +819,10 @@ __global__ void __launch_bounds__(kThreads, 1) diag_solver_kernel(DiagArgs A) {
     }
 }
 
-template <bool DENSE, bool ELK>
+template <int CELL, bool ELK, int TK>
 cudaError_t launch_one(const DiagArgs &a, cudaStream_t s) {
-    auto kern = diag_solver_kernel<DENSE, ELK>;
-    const size_t smem = smem_floats(a.tl, a.D, DENSE) * sizeof(float);
+    auto kern = diag_solver_kernel<CELL, ELK, TK>;
+    const size_t smem = smem_floats(a.tl, a.D, CELL) * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -647,16 +845,27 @@ cudaError_t launch_one(const DiagArgs &a, cudaStream_t s) {
 
 }  // namespace
 
-size_t diag_solver_smem_bytes(const Tiling &tl, int D, bool dense) {
-    return smem_floats(tl, D, dense) * sizeof(float);
+static int cell_variant(const pararnn_cell &cell) {
+    if (cell.kind != PARARNN_GRU_DENSE) return kCellDiag;
+    const int D = cell.d;
+    return (D == 8 || D == 16 || D == 32 || D == 64) ? kCellDenseMma : kCellDenseFma;
 }
 
 cudaError_t launch_diag_solver(const pararnn_cell &cell, int mode, const DiagArgs &a,
                                cudaStream_t s) {
-    const bool dense = cell.kind == PARARNN_GRU_DENSE;
     const bool elk = mode == PARARNN_ELK || mode == PARARNN_QUASI_ELK;
-    if (dense) return elk ? launch_one<true, true>(a, s) : launch_one<true, false>(a, s);
-    return elk ? launch_one<false, true>(a, s) : launch_one<false, false>(a, s);
+    if (a.tl.TK != kSolverTK) return cudaErrorInvalidValue;
+    switch (cell_variant(cell)) {
+        case kCellDenseMma:
+            return elk ? launch_one<kCellDenseMma, true, kSolverTK>(a, s)
+                       : launch_one<kCellDenseMma, false, kSolverTK>(a, s);
+        case kCellDenseFma:
+            return elk ? launch_one<kCellDenseFma, true, kSolverTK>(a, s)
+                       : launch_one<kCellDenseFma, false, kSolverTK>(a, s);
+        default:
+            return elk ? launch_one<kCellDiag, true, kSolverTK>(a, s)
+                       : launch_one<kCellDiag, false, kSolverTK>(a, s);
+    }
 }
 
 }  // namespace pararnn

@@ -19,7 +19,6 @@
 namespace pararnn {
 
 size_t scan_diag_ws_bytes(int B, int T, int D);
-size_t diag_solver_smem_bytes(const Tiling &tl, int D, bool dense);
 size_t dense_ws_bytes(const pararnn_cell &cell, int B, int T, int mode);
 cudaError_t launch_dense_solver(const pararnn_cell &cell, int mode, const DiagArgs &a,
                                 void *dense_ws, cudaStream_t s);
@@ -65,7 +64,7 @@ WsLayout ws_layout(const pararnn_cell &cell, int B, int T, int mode) {
     WsLayout L{};
     const size_t states = static_cast<size_t>(B) * T * cell.d;
     const bool diag = diag_jacobian(cell, mode);
-    const Tiling tl = make_tiling(B, T, cell.d, cell.kind == PARARNN_GRU_DENSE);
+    const Tiling tl = make_tiling(B, T, cell.d, cell.kind == PARARNN_GRU_DENSE, kSolverTK);
     size_t off = 0;
     L.header = off; off += 256;
     L.P = off; off = align256(off + states * 3 * sizeof(float));
@@ -140,7 +139,7 @@ static cudaError_t enqueue_iterate(const pararnn_cell *cell, const pararnn_param
     a.lambda = lambda;
     a.tol = tol;
     a.max_iters = max_iters <= 0 ? T + 1 : max_iters;
-    a.tl = make_tiling(B, T, cell->d, cell->kind == PARARNN_GRU_DENSE);
+    a.tl = make_tiling(B, T, cell->d, cell->kind == PARARNN_GRU_DENSE, kSolverTK);
     a.desc = reinterpret_cast<unsigned long long *>(ws + L.desc);
     const size_t states4 = states * sizeof(float);
     a.elk_m = reinterpret_cast<float *>(ws + L.elk);

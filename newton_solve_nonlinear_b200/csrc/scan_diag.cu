@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(kThreads) scan_diag_kernel(ScanArgs S) {
         }
         const int d = dg * tl.DG + lane;
         const float carry0 = (chunk == 0 && d < S.D) ? __ldg(S.h0 + static_cast<size_t>(b) * S.D + d) : 0.f;
-        sC[lane] = lookback_affine(S.desc, tile, tl.n_groups, tl.DG, lane, 1u, EA, EB, chunk == 0,
+        sC[lane] = lookback_affine(S.desc, tile, tl.n_groups, tl.DG, lane, 1u, EA, EB, chunk,
                                    carry0, &S.hdr->status);
     }
     __syncthreads();
@@ -121,7 +121,7 @@ cudaError_t launch_scan_diag(const float *A, const float *b, const float *h0, in
     ScanArgs S;
     S.A = A; S.b = b; S.h0 = h0; S.h = h;
     S.B = B; S.T = T; S.D = D;
-    S.tl = make_tiling(B, T, D, false);
+    S.tl = make_tiling(B, T, D, false, TK);
     S.hdr = static_cast<WsHeader *>(ws);
     S.desc = reinterpret_cast<unsigned long long *>(static_cast<char *>(ws) + 256);
     const size_t desc_bytes = static_cast<size_t>(S.tl.n_tiles) * S.tl.DG * 2 * 8;
@@ -132,7 +132,7 @@ cudaError_t launch_scan_diag(const float *A, const float *b, const float *h0, in
 }
 
 size_t scan_diag_ws_bytes(int B, int T, int D) {
-    const Tiling tl = make_tiling(B, T, D, false);
+    const Tiling tl = make_tiling(B, T, D, false, TK);
     return 256 + static_cast<size_t>(tl.n_tiles) * tl.DG * 2 * 8;
 }
 

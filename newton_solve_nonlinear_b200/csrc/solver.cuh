@@ -35,7 +35,12 @@ struct Tiling {
     long long n_tiles;
 };
 
-Tiling make_tiling(int B, int T, int D, bool dense_cell);
+// Tiling of the state array.  The solver kernels take two steps per thread
+// (kSolverTK): that keeps the per-thread state -- 3 x TK x 4 recurrent sums for
+// the dense cell, the TK x 4 scan operands -- inside the register budget of
+// two CTAs per SM.  The standalone scan holds only a and b and takes four.
+constexpr int kSolverTK = 2;
+Tiling make_tiling(int B, int T, int D, bool dense_cell, int TK);
 
 // Arguments of the persistent diagonal-Jacobian solver kernels.
 struct DiagArgs {

@@ -81,6 +81,10 @@ def test_affine_scan_closed_forms():
     ("near_unstable", dict(B=2, T=600), "QUASI_ELK", 0.1),
     ("near_unstable", dict(B=2, T=333, d=32, din=16, h0_std=0.5), "QUASI_ELK", 1.0),
     ("diag", dict(B=2, T=260, d=64, din=64), "QUASI_ELK", 0.01),
+    ("untrained", dict(B=2, T=500, d=16, din=16, bias_std=0.3), "QUASI", 0.0),
+    ("untrained", dict(B=2, T=333, d=8, din=8, h0_std=0.5), "QUASI", 0.0),
+    ("untrained", dict(B=2, T=200, d=12, din=12), "QUASI", 0.0),
+    ("untrained", dict(B=1, T=301, d=32, din=32, bias_std=0.3), "QUASI_ELK", 0.1),
 ])
 def test_each_iteration_matches_oracle(name, over, mode, lam):
     kw = {k: over[k] for k in ("bias_std", "h0_std") if k in over}
