@@ -158,8 +158,12 @@ static cudaError_t enqueue_iterate(const pararnn_cell *cell, const pararnn_param
 
 int pararnn_input_projection(const pararnn_cell *cell, const pararnn_params *params,
                              const void *x, int B, int T, float *P, pararnn_stream stream) {
-    if (!cell_ok(cell, B, T, PARARNN_QUASI) || !params || !x || !P || !params->w_ih || !params->b_ih)
+    // the projection does not involve the recurrence: only the widths and dtypes matter
+    if (!cell || B < 1 || T < 1 || cell->d < 1 || cell->din < 1) return PARARNN_INVALID_ARG;
+    if (cell->x_dtype != cell->w_dtype ||
+        (cell->x_dtype != PARARNN_F32 && cell->x_dtype != PARARNN_BF16))
         return PARARNN_INVALID_ARG;
+    if (!params || !x || !P || !params->w_ih || !params->b_ih) return PARARNN_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(P, 16) || !aligned(params->w_ih, 16) || !aligned(params->b_ih, 16))
         return PARARNN_INVALID_ARG;
     const cudaError_t e = launch_projection(*cell, x, params->w_ih, params->b_ih, P,

@@ -1,0 +1,312 @@
+// proj_tcgen05.cu -- the input projection P = x W_ih^T + b_ih on the 5th-generation
+// tensor cores (tcgen05, sm_100a), for bf16 operands.
+//
+// The input projection does not depend on the state, so one GEMM
+// [B*T, Din] x [Din, 3D] serves every Newton iteration.  For the bf16 layer
+// (Din = D = 2048) it is the one tensor-bound step of the solve (2*M*N*K flop).
+//
+// One CTA computes a 128 x 256 fp32 tile of P:
+//   * TMA brings 128 x 64 tiles of x and 256 x 64 tiles of W_ih (bf16, 128-byte
+//     swizzle) into a 4-stage shared-memory ring, signalled by mbarriers;
+//   * one thread issues tcgen05.mma kind::f16 (bf16 x bf16 -> fp32, M=128,
+//     N=256, K=16 per instruction) into a 256-column TMEM accumulator and
+//     frees each stage with tcgen05.commit;
+//   * after the last k-block, the four warps read the accumulator rows with
+//     tcgen05.ld (thread = row), add the bias, stage 32-column blocks in
+//     shared memory with the 128-byte swizzle, and TMA stores them.
+// Every wait is bounded; a wait that runs out marks the tile and the epilogue
+// writes NaN, which the solver reports as DIVERGED.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "solver.cuh"
+
+namespace pararnn {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;        // 16 KB
+constexpr int B_BYTES = BN * BK * 2;        // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;  // + alignment + barriers
+constexpr long long kWaitBudget = 1ll << 22;
+
+__device__ __forceinline__ unsigned smem_u32(const void *p) {
+    return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(unsigned bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(unsigned bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(unsigned bar, unsigned parity) {
+    unsigned done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+// Bounded wait that ignores the error flag (used to drain work in flight).
+__device__ __forceinline__ void mbar_drain(unsigned bar, unsigned parity) {
+    for (long long n = 0; n < kWaitBudget && !mbar_try_wait(bar, parity); ++n) {
+    }
+}
+// Bounded wait; returns false (and sets *err) when the budget runs out.
+__device__ __forceinline__ bool mbar_wait(unsigned bar, unsigned parity, volatile int *err) {
+    long long n = 0;
+    while (!mbar_try_wait(bar, parity)) {
+        if (*err) return false;
+        if (++n > kWaitBudget) {
+            *err = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(unsigned dst, const CUtensorMap *map, int c0, int c1,
+                                            unsigned bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<unsigned long long>(map)), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int c0, int c1, unsigned src) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<unsigned long long>(map)),
+                 "r"(c0), "r"(c1), "r"(src)
+                 : "memory");
+}
+
+// K-major operand tile with 128-byte swizzle: rows of 128 bytes, 8-row groups
+// 1024 bytes apart (SBO), descriptor version 1, layout type 2 (SWIZZLE_128B).
+__device__ __forceinline__ unsigned long long sw128_desc(unsigned addr) {
+    unsigned long long d = 0;
+    d |= static_cast<unsigned long long>((addr >> 4) & 0x3fffu);
+    d |= static_cast<unsigned long long>(1u) << 16;           // LBO (unused with swizzle)
+    d |= static_cast<unsigned long long>(1024u >> 4) << 32;   // SBO
+    d |= static_cast<unsigned long long>(1u) << 46;           // version
+    d |= static_cast<unsigned long long>(2u) << 61;           // SWIZZLE_128B
+    return d;
+}
+
+// kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, both K-major.
+constexpr unsigned kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) |
+                                (static_cast<unsigned>(BN >> 3) << 17) |
+                                (static_cast<unsigned>(BM >> 4) << 24);
+
+__global__ void __launch_bounds__(128, 1)
+proj_tcgen05_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
+                    const __grid_constant__ CUtensorMap map_p, const float *__restrict__ bias, int K,
+                    float *__restrict__ Pout, long long M, int N) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    unsigned long long *bars = reinterpret_cast<unsigned long long *>(smem + STAGES * STAGE_BYTES);
+    // bars[0..3] full, bars[4..7] empty, bars[8] done; then TMEM base address and error flag
+    unsigned *tmem_slot = reinterpret_cast<unsigned *>(bars + 2 * STAGES + 1);
+    volatile int *err = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *issued = reinterpret_cast<volatile int *>(tmem_slot + 2);    // TMA k-blocks issued
+    volatile int *consumed = reinterpret_cast<volatile int *>(tmem_slot + 3);  // k-blocks given to MMA
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
+    const int nk = K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&bars[s]), 1);
+            mbar_init(smem_u32(&bars[STAGES + s]), 1);
+        }
+        mbar_init(smem_u32(&bars[2 * STAGES]), 1);
+        *err = 0;
+        *issued = 0;
+        *consumed = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 2) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(BN));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;");
+    const unsigned tmem = *tmem_slot;
+
+    if (threadIdx.x == 0) {
+        // TMA producer
+        for (int kb = 0; kb < nk; ++kb) {
+            const int s = kb % STAGES;
+            const unsigned ph = (kb / STAGES) & 1u;
+            if (!mbar_wait(smem_u32(&bars[STAGES + s]), ph ^ 1u, err)) break;
+            const unsigned full = smem_u32(&bars[s]);
+            mbar_expect_tx(full, STAGE_BYTES);
+            unsigned char *sa = smem + s * STAGE_BYTES;
+            tma_load_2d(smem_u32(sa), &map_x, kb * BK, m0, full);
+            tma_load_2d(smem_u32(sa + A_BYTES), &map_w, kb * BK, n0, full);
+            *issued = kb + 1;
+        }
+    } else if (threadIdx.x == 32) {
+        // MMA issuer
+        for (int kb = 0; kb < nk; ++kb) {
+            const int s = kb % STAGES;
+            const unsigned ph = (kb / STAGES) & 1u;
+            if (!mbar_wait(smem_u32(&bars[s]), ph, err)) break;
+            asm volatile("tcgen05.fence::after_thread_sync;");
+            const unsigned sa = smem_u32(smem + s * STAGE_BYTES);
+            const unsigned sb = sa + A_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+                const unsigned long long da = sw128_desc(sa + kk * 32);
+                const unsigned long long db = sw128_desc(sb + kk * 32);
+                const unsigned acc = (kb > 0 || kk > 0) ? 1u : 0u;
+                asm volatile(
+                    "{\n\t.reg .pred p;\n\t"
+                    "setp.ne.b32 p, %4, 0;\n\t"
+                    "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem),
+                    "l"(da), "l"(db), "r"(kIdescBf16), "r"(acc));
+            }
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                smem_u32(&bars[STAGES + s])));
+            *consumed = kb + 1;
+        }
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_u32(&bars[2 * STAGES])));
+    }
+    __syncwarp();
+
+    // epilogue: thread = accumulator row
+    const bool ok = mbar_wait(smem_u32(&bars[2 * STAGES]), 0u, err);
+    asm volatile("tcgen05.fence::after_thread_sync;");
+    __syncthreads();  // every stage is free now: reuse the ring as the output staging area
+    const bool good = ok && !*err;
+    const int row = threadIdx.x;
+    if (!good) {
+        // a wait ran out: drain the copies and products still in flight, then
+        // mark this tile with NaN (no TMA store from a ring that may still change)
+        if (threadIdx.x == 0) {
+            for (int kb = *consumed; kb < *issued; ++kb)
+                mbar_drain(smem_u32(&bars[kb % STAGES]), (kb / STAGES) & 1u);
+            mbar_drain(smem_u32(&bars[2 * STAGES]), 0u);
+        }
+        __syncthreads();
+        if (m0 + row < M)
+            for (int n = n0; n < n0 + BN; ++n) Pout[(m0 + row) * static_cast<long long>(N) + n] = __int_as_float(0x7fc00000);
+        asm volatile("tcgen05.fence::before_thread_sync;");
+        __syncthreads();
+        if (warp == 2) {
+            asm volatile("tcgen05.fence::after_thread_sync;");
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BN));
+        }
+        return;
+    }
+    unsigned char *stage = smem;  // 8 blocks of [128 rows x 128 B]
+#pragma unroll 1
+    for (int cb = 0; cb < BN / 32; ++cb) {
+        unsigned v[32];
+        const unsigned taddr = tmem + (static_cast<unsigned>(warp * 32) << 16) + cb * 32;
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+            "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+              "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+              "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+              "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+              "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+              "=r"(v[31])
+            : "r"(taddr));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        unsigned char *blk = stage + cb * (BM * 128) + row * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {  // 16-byte chunk j of this row, swizzled
+            float4 o;
+            const int n = n0 + cb * 32 + j * 4;
+            o.x = __uint_as_float(v[4 * j + 0]) + __ldg(bias + n + 0);
+            o.y = __uint_as_float(v[4 * j + 1]) + __ldg(bias + n + 1);
+            o.z = __uint_as_float(v[4 * j + 2]) + __ldg(bias + n + 2);
+            o.w = __uint_as_float(v[4 * j + 3]) + __ldg(bias + n + 3);
+            *reinterpret_cast<float4 *>(blk + ((j ^ (row & 7)) << 4)) = o;
+        }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("tcgen05.fence::before_thread_sync;");
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int cb = 0; cb < BN / 32; ++cb)
+            tma_store_2d(&map_p, n0 + cb * 32, m0, smem_u32(stage + cb * (BM * 128)));
+        asm volatile("cp.async.bulk.commit_group;");
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+    }
+    __syncthreads();
+    if (warp == 2) {
+        asm volatile("tcgen05.fence::after_thread_sync;");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BN));
+    }
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+bool make_map(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, long long rows,
+              int cols, int box_cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * esize};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool proj_tcgen05_supported(const pararnn_cell &cell) {
+    return cell.x_dtype == PARARNN_BF16 && cell.din % BK == 0 && (3 * cell.d) % BN == 0 &&
+           encode_fn() != nullptr;
+}
+
+cudaError_t launch_proj_tcgen05(const pararnn_cell &cell, const void *x, const void *w_ih,
+                                const float *b_ih, float *P, long long M, cudaStream_t s) {
+    const int N = 3 * cell.d, K = cell.din;
+    CUtensorMap mx, mw, mp;
+    if (!make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, M, K, BK, BM) ||
+        !make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w_ih, N, K, BK, BN) ||
+        !make_map(&mp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, P, M, N, 32, BM))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(proj_tcgen05_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(static_cast<unsigned>((M + BM - 1) / BM), static_cast<unsigned>(N / BN));
+    proj_tcgen05_kernel<<<grid, 128, SMEM_BYTES, s>>>(mx, mw, mp, b_ih, K, P, M, N);
+    return cudaGetLastError();
+}
+
+}  // namespace pararnn

@@ -85,8 +85,15 @@ __global__ void __launch_bounds__(256) proj_gemm_kernel(const Tin *__restrict__ 
 
 }  // namespace
 
+bool proj_tcgen05_supported(const pararnn_cell &cell);
+cudaError_t launch_proj_tcgen05(const pararnn_cell &cell, const void *x, const void *w_ih,
+                                const float *b_ih, float *P, long long M, cudaStream_t s);
+
+// bf16 operands with Din a multiple of 64 and 3D a multiple of 256 take the
+// tcgen05 kernel (proj_tcgen05.cu); everything else this CUDA-core kernel.
 cudaError_t launch_projection(const pararnn_cell &cell, const void *x, const void *w_ih,
                               const float *b_ih, float *P, long long M, cudaStream_t s) {
+    if (proj_tcgen05_supported(cell)) return launch_proj_tcgen05(cell, x, w_ih, b_ih, P, M, s);
     const int N = 3 * cell.d, K = cell.din;
     const dim3 grid(static_cast<unsigned>((M + BM - 1) / BM), (N + BN - 1) / BN);
     if (cell.x_dtype == PARARNN_BF16)
