@@ -129,6 +129,32 @@ __device__ __forceinline__ float tanhf_(float v) {
     return 1.0f - __fdividef(2.0f, __expf(2.0f * v) + 1.0f);
 }
 
+// One GRU state (gate order r, z, n; reset gate applied after the recurrent
+// bias) and the diagonal of its Jacobian with respect to the previous state.
+//   pr, pz, pn   input pre-activations (W x + b_ih) of the lane
+//   gr, gz, gnh  recurrent sums U_g h (or u_g * h for the diagonal cell)
+//   bh*          recurrent biases b_hh;  ud*: diagonal entries of U_g
+//   h            the previous state h_{t-1}
+// Returns f = f(h, x), a = df/dh (diagonal entry) and bb = f - a h.
+//   a = z + (h - n) z (1 - z) U_z + (1 - z)(1 - n^2) r U_n
+//         + (1 - z)(1 - n^2) g r (1 - r) U_r          (diagonal entries)
+__device__ __forceinline__ void gru_cell_diag(float pr, float pz, float pn, float gr, float gz,
+                                              float gnh, float bhr, float bhz, float bhn, float udr,
+                                              float udz, float udn, float h, float &f, float &a,
+                                              float &bb) {
+    const float r = sigmoidf_(pr + gr + bhr);
+    const float z = sigmoidf_(pz + gz + bhz);
+    const float gn = gnh + bhn;
+    const float n = tanhf_(pn + r * gn);
+    f = n + z * (h - n);
+    const float omz = 1.f - z;
+    const float cz = (h - n) * z * omz;
+    const float cn = omz * (1.f - n * n) * r;
+    const float cr = cn * gn * (1.f - r);
+    a = z + cz * udz + cn * udn + cr * udr;
+    bb = f - a * h;
+}
+
 // |x| as an unsigned bit pattern: ordered like the float for x >= 0, and any
 // NaN or Inf maps above every finite value (0x7f800000 and up), so an integer
 // max over patterns both finds the largest |dh| and flags non-finite values.

@@ -147,17 +147,8 @@ __device__ __forceinline__ void cell_state(float pr, float pz, float pn, float g
                                            float gnh, float bhr, float bhz, float bhn, float udr,
                                            float udz, float udn, float h, float hc, float &a,
                                            float &bb, unsigned &rmax) {
-    const float r = sigmoidf_(pr + gr + bhr);
-    const float z = sigmoidf_(pz + gz + bhz);
-    const float gn = gnh + bhn;
-    const float n = tanhf_(pn + r * gn);
-    const float f = n + z * (h - n);
-    const float omz = 1.f - z;
-    const float cz = (h - n) * z * omz;
-    const float cn = omz * (1.f - n * n) * r;
-    const float cr = cn * gn * (1.f - r);
-    a = z + cz * udz + cn * udn + cr * udr;
-    bb = f - a * h;
+    float f;
+    gru_cell_diag(pr, pz, pn, gr, gz, gnh, bhr, bhz, bhn, udr, udz, udn, h, f, a, bb);
     rmax = max(rmax, abs_bits(hc - f));
 }
 
@@ -437,18 +428,11 @@ __device__ __forceinline__ void linearise(const DiagArgs &A, const TileCoord &c,
             const float gr = DENSE ? G[0][k][j] : ud[0][j] * h;
             const float gz = DENSE ? G[1][k][j] : ud[1][j] * h;
             const float gnh = DENSE ? G[2][k][j] : ud[2][j] * h;
-            const float r = sigmoidf_(get(pv[0], j) + gr + bh[0][j]);
-            const float z = sigmoidf_(get(pv[1], j) + gz + bh[1][j]);
-            const float gn = gnh + bh[2][j];
-            const float n = tanhf_(get(pv[2], j) + r * gn);
-            const float f = n + z * (h - n);
-            const float omz = 1.f - z;
-            const float cz = (h - n) * z * omz;
-            const float cn = omz * (1.f - n * n) * r;
-            const float cr = cn * gn * (1.f - r);
-            const float aa = z + cz * ud[1][j] + cn * ud[2][j] + cr * ud[0][j];
+            float f, aa, bv;
+            gru_cell_diag(get(pv[0], j), get(pv[1], j), get(pv[2], j), gr, gz, gnh, bh[0][j], bh[1][j],
+                          bh[2][j], ud[0][j], ud[1][j], ud[2][j], h, f, aa, bv);
             a[k][j] = aa;
-            bb[k][j] = f - aa * h;
+            bb[k][j] = bv;
             y[k][j] = hp[k + 1][j];
             rmax = max(rmax, abs_bits(hp[k + 1][j] - f));
         }

@@ -22,6 +22,9 @@ size_t scan_diag_ws_bytes(int B, int T, int D);
 size_t dense_ws_bytes(const pararnn_cell &cell, int B, int T, int mode);
 cudaError_t launch_dense_solver(const pararnn_cell &cell, int mode, const DiagArgs &a,
                                 void *dense_ws, cudaStream_t s);
+size_t quasi_tc_desc_bytes(int B, int T, int D);
+bool quasi_tc_supported(const pararnn_cell &cell, int B, int T);
+cudaError_t launch_quasi_tc(const DiagArgs &a, cudaStream_t s);
 cudaError_t launch_scan_dense(const float *A, const float *b, const float *h0, int B, int T,
                               int D, float *h, void *ws, cudaStream_t s);
 size_t scan_dense_ws_bytes(int B, int T, int D);
@@ -70,7 +73,16 @@ WsLayout ws_layout(const pararnn_cell &cell, int B, int T, int mode) {
     L.P = off; off = align256(off + states * 3 * sizeof(float));
     L.hbuf = off; off = align256(off + states * sizeof(float));
     L.desc = off;
-    if (diag) off = align256(off + static_cast<size_t>(tl.n_tiles) * tl.DG * (is_elk(mode) ? 8 : 2) * 8);
+    if (diag) {
+        size_t desc = static_cast<size_t>(tl.n_tiles) * tl.DG * (is_elk(mode) ? 8 : 2) * 8;
+        // the tensor-core dense-cell path tiles by 128 steps x all lanes
+        if (cell.kind == PARARNN_GRU_DENSE && mode == PARARNN_QUASI &&
+            (cell.d == 32 || cell.d == 64)) {
+            const size_t tc = quasi_tc_desc_bytes(B, T, cell.d);
+            if (tc > desc) desc = tc;
+        }
+        off = align256(off + desc);
+    }
     L.elk = off;
     if (diag && is_elk(mode)) off = align256(off + 4 * states * sizeof(float));
     L.dense = off;
@@ -152,6 +164,12 @@ static cudaError_t enqueue_iterate(const pararnn_cell *cell, const pararnn_param
     cudaError_t e = cudaMemsetAsync(ws + L.header, 0, 256, s);
     if (e == cudaSuccess && diag && L.elk > L.desc) e = cudaMemsetAsync(ws + L.desc, 0, L.elk - L.desc, s);
     if (e != cudaSuccess) return e;
+    if (mode == PARARNN_QUASI && quasi_tc_supported(*cell, B, T)) {
+        // the tensor-core path reads the initial guess (zero) from memory
+        e = cudaMemsetAsync(a.hbuf[0], 0, states * sizeof(float), s);
+        if (e != cudaSuccess) return e;
+        return launch_quasi_tc(a, s);
+    }
     return diag ? launch_diag_solver(*cell, mode, a, s)
                 : launch_dense_solver(*cell, mode, a, ws + L.dense, s);
 }
