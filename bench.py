@@ -37,9 +37,13 @@ WORKLOAD = "untrained dense GRU Din=D=64, B=16/GPU, T={T}, fp32, quasi-DEER tol 
 # bytes each state moves per Newton iteration in a fused single pass:
 # P (3 fp32 pre-activations) + previous guess + new guess
 BYTES_PER_STATE_ITER = 20
-# ncu DRAM traffic of the solver kernel (bytes per launch) and the hash of the
-# kernel source it was measured on; reported only while the source is unchanged.
-NCU_TRAFFIC = {"bytes_per_launch": None, "source_sha1": None}
+# ncu DRAM traffic of the solver kernel (read + write bytes of one launch,
+# captured at T = 16384: 4.812 GB over 14 iterations x 16.78 M states) and the
+# hash of the kernel source it was measured on.  Traffic grows with states x
+# iterations, so the full launch's is scaled from it; reported only while the
+# source is unchanged.
+NCU_TRAFFIC = {"bytes_per_state_iter": 4.812e9 / (14 * 16 * 16384 * 64),
+               "source_sha1": "6cb957761e3f"}
 
 
 def log(*a):
@@ -55,7 +59,7 @@ def peaks():
 
 
 def kernel_sha():
-    src = os.path.join(ROOT, "newton_solve_nonlinear_b200", "csrc", "newton_diag.cu")
+    src = os.path.join(ROOT, "newton_solve_nonlinear_b200", "csrc", "newton_dense_tc.cu")
     return hashlib.sha1(open(src, "rb").read()).hexdigest()[:12]
 
 
@@ -246,7 +250,7 @@ def run_ours(args):
     solver_avg_s = statistics.mean(solver_ms) / 1e3
     algo_bytes = iters * states * BYTES_PER_STATE_ITER
     achieved = algo_bytes / solver_avg_s / 1e9
-    traffic = (NCU_TRAFFIC["bytes_per_launch"]
+    traffic = (NCU_TRAFFIC["bytes_per_state_iter"] * iters * states
                if NCU_TRAFFIC["source_sha1"] == kernel_sha() else None)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -255,13 +259,14 @@ def run_ours(args):
         "config": {"workload": WORKLOAD.format(T=T), "B": B, "T": T, "D": D, "din": din,
                    "mode": "QUASI", "tol": w.tol, "iters": iters,
                    "status": binding.STATUS.get(status),
-                   "l2": "inputs larger than L2: x 268 MB, P 805 MB, h 268 MB per solve",
+                   "l2": (f"inputs larger than L2 (126 MB): x {x.numel() * 4 / 1e6:.0f} MB, "
+                          f"P {P.numel() * 4 / 1e6:.0f} MB, h {out.numel() * 4 / 1e6:.0f} MB per solve"),
                    "parallelism": f"replicas over sequences x{world}",
                    "projection_ms": statistics.mean(proj_ms),
                    "solver_ms": statistics.mean(solver_ms)},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "diag_solver_kernel<dense,quasi> (persistent, all iterations)",
+                     "kernel": "quasi_tc_kernel<64> (persistent, all iterations)",
                      "algorithmic_bytes": f"{BYTES_PER_STATE_ITER} B/state/iteration x {iters} "
                                           f"iterations x {states} states",
                      "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"},
