@@ -134,7 +134,9 @@ PARARNN_API size_t pararnn_workspace_size(const pararnn_cell *cell, int B, int T
  *   ELK / QUASI_ELK: h^(i+1) minimises
  *       sum_t |h_t - A_t h_{t-1} - b_t|^2 + lambda sum_t |h_t - h^(i)_t|^2
  *     (Kalman filter + RTS smoother with process noise I, observation noise
- *     I / lambda, observations h^(i)).
+ *     I / lambda, observations h^(i)).  QUASI_ELK runs that smoother as
+ *     scans; ELK on the DENSE cell solves the same minimiser from its
+ *     block-tridiagonal normal equations by block cyclic reduction.
  *   Stop when delta = max_{b,t,d} |h^(i+1) - h^(i)| <= tol (iters = i + 1),
  *   when a value is non-finite (DIVERGED), or after max_iters iterations.
  *
@@ -159,6 +161,8 @@ PARARNN_API size_t pararnn_workspace_size(const pararnn_cell *cell, int B, int T
  *                  once, at the end, to read the report.
  * Returns pararnn_status (the solve's own status, or INVALID_ARG / CUDA_ERROR).
  * Limits: DENSE cells need d <= 64 (recurrent matrices are kept on chip).
+ * ELK on the DENSE cell keeps three D x D matrices per step in the workspace
+ * (D rounded up to 8, 16, 32 or 64): about 3 * B * T * D^2 * 4 bytes.
  */
 PARARNN_API int pararnn_newton_solve(const pararnn_cell *cell, const pararnn_params *params,
                          const void *x, const float *h0, int B, int T, int mode,

@@ -53,8 +53,12 @@ DenseGeom dense_geom(int B, int T, int D) {
 
 static size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Phi [B][NC][D][D], p [B][NC][D], carry [B][NC][D]
+size_t dense_elk_ws_bytes(int B, int T, int D);
+
+// DEER: Phi [B][NC][D][D], p [B][NC][D], carry [B][NC][D]; ELK: the cyclic
+// reduction arrays of newton_dense_elk.cu.
 size_t dense_ws_bytes(const pararnn_cell &cell, int B, int T, int mode) {
+    if (mode == PARARNN_ELK) return dense_elk_ws_bytes(B, T, cell.d);
     const DenseGeom g = dense_geom(B, T, cell.d);
     const size_t n = static_cast<size_t>(B) * g.NC;
     const size_t D = cell.d;
@@ -644,8 +648,12 @@ cudaError_t launch_dscan(const DScanArgs &S, cudaStream_t s) {
 
 }  // namespace
 
+size_t dense_elk_ws_bytes(int B, int T, int D);
+cudaError_t launch_dense_elk(const DiagArgs &a, void *ws, cudaStream_t s);
+
 cudaError_t launch_dense_solver(const pararnn_cell &cell, int mode, const DiagArgs &a,
                                 void *dense_ws, cudaStream_t s) {
+    if (mode == PARARNN_ELK) return launch_dense_elk(a, dense_ws, s);
     if (mode != PARARNN_DEER) return cudaErrorNotSupported;
     DenseArgs S;
     S.a = a;

@@ -54,8 +54,6 @@ bool cell_ok(const pararnn_cell *cell, int B, int T, int mode) {
     if (cell->x_dtype != PARARNN_F32 && cell->x_dtype != PARARNN_BF16) return false;
     if (mode < PARARNN_DEER || mode > PARARNN_QUASI_ELK) return false;
     if (cell->kind == PARARNN_GRU_DENSE && cell->d > 64) return false;
-    // full-Jacobian ELK on the dense cell is not provided by this library yet
-    if (cell->kind == PARARNN_GRU_DENSE && mode == PARARNN_ELK) return false;
     // the state array is indexed with 32-bit time and lane counts
     if (static_cast<long long>(T) * 3 * cell->d > (1ll << 31)) return false;
     return true;

@@ -52,6 +52,9 @@ def test_workspace_sizes(L):
     assert ws("diag", 2048, 2048, 8, 4096, "QUASI") >= 8 * 4096 * 2048 * 16
     # quasi-ELK keeps its forward results
     assert ws("dense", 64, 64, 8, 1000, "QUASI_ELK") > ws("dense", 64, 64, 8, 1000, "QUASI")
+    # ELK on the dense cell keeps three D x D blocks per step for the reduction
+    assert ws("dense", 64, 64, 8, 10000, "ELK") >= 3 * 8 * 10000 * 64 * 64 * 4
+    assert ws("dense", 4, 12, 2, 33, "ELK") >= 3 * 2 * 33 * 16 * 16 * 4
     # rejected: D not a multiple of 4, dense D > 64, bad mode, empty sizes
     assert ws("dense", 4, 6, 1, 10, "QUASI") == 0
     assert ws("dense", 4, 128, 1, 10, "QUASI") == 0

@@ -1,0 +1,110 @@
+"""GPU parity of ELK on the dense GRU (full-Jacobian Levenberg-Marquardt step)
+against the fp64 oracle.
+
+The GPU solves each damped step's block-tridiagonal normal equations by block
+cyclic reduction; the oracle solves the same equations by sequential block
+elimination (and is cross-checked against a Kalman filter + RTS smoother by
+the CPU pins), so the two share nothing but the problem statement.
+
+Tolerances:
+  * single iterations (max_iters = 1, 2, 3) vs the oracle's iterates:
+    max-abs <= 5e-5.  Each level of the reduction inverts and multiplies
+    fp32 D x D blocks (about log2 T levels, condition numbers up to
+    ~ (1 + |J|)^2 / lambda), so the spread is larger than the diagonal
+    path's 2e-5;
+  * iteration counts within +-1 of the oracle's, and the final iterate within
+    1e-4 of the oracle's final iterate when the counts agree (damped steps
+    converge linearly, so the stopping iterate is what both solvers share);
+  * full size: whole sampled sequences within 1e-4 of the fp64 rollout
+    (lambda = 0.01 is close to DEER and stops next to the fixed point).
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle.cells import GRU, rollout
+from newton_solve_nonlinear_b200 import binding
+from newton_solve_nonlinear_b200.inputs import make_workload
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle(w):
+    return GRU.from_workload(w), w.x.double().numpy(), w.h0.double().numpy()
+
+
+def _make(name, over):
+    kw = {k: over[k] for k in ("bias_std", "h0_std") if k in over}
+    return make_workload(name, **{k: v for k, v in over.items() if k not in kw}, **kw)
+
+
+@pytest.mark.parametrize("name,over,lam", [
+    ("near_unstable", dict(B=2, T=300), 0.1),
+    ("near_unstable", dict(B=2, T=257, d=32, din=16, h0_std=0.5), 1.0),
+    ("near_unstable", dict(B=3, T=129, d=16, din=16), 0.01),
+    ("tiny", dict(T=1000, bias_std=0.3, h0_std=0.5), 0.1),
+    ("untrained", dict(B=2, T=130, d=12, din=12, bias_std=0.3), 0.1),
+    ("near_unstable", dict(B=2, T=1, d=8, din=8, h0_std=1.0), 0.1),
+    ("near_unstable", dict(B=1, T=2, d=64, din=64, h0_std=1.0), 0.3),
+    ("near_unstable", dict(B=1, T=3, d=64, din=64, h0_std=1.0), 0.3),
+])
+def test_each_elk_iteration_matches_oracle(name, over, lam):
+    w = _make(name, over)
+    c, x, h0 = _oracle(w)
+    ref = oracle.elk_solve(c, x, h0, "ELK", lam, 0.0, max_iters=3, record=True)
+    for n in (1, 2, 3):
+        r = binding.solve_workload(w, "ELK", lam=lam, tol=0.0, max_iters=n)
+        assert r.iters == n and r.status == "NOT_CONVERGED"
+        err = np.max(np.abs(r.h.double().cpu().numpy() - ref["iterates"][n - 1]))
+        assert err <= 5e-5, (n, err)
+        assert abs(r.delta - ref["deltas"][n - 1]) <= 5e-5 + 1e-5 * ref["deltas"][n - 1]
+
+
+@pytest.mark.parametrize("T,lam", [(1000, 0.01), (1000, 0.1), (300, 1.0)])
+def test_elk_matches_oracle_count_and_final_iterate(T, lam):
+    w = make_workload("near_unstable", B=2, T=T)
+    c, x, h0 = _oracle(w)
+    r = binding.solve_workload(w, "ELK", lam=lam)
+    ref = oracle.elk_solve(c, x, h0, "ELK", lam, w.tol)
+    assert r.status == "OK" and ref["status"] == "OK"
+    assert abs(r.iters - ref["iters"]) <= 1, (r.iters, ref["iters"])
+    if r.iters == ref["iters"]:
+        assert np.max(np.abs(r.h.double().cpu().numpy() - ref["h"])) <= 1e-4
+
+
+def test_elk_small_lambda_reaches_rollout():
+    """lambda -> 0 is DEER: at a tight tolerance ELK lands on the rollout."""
+    w = make_workload("dense_deer", B=2, T=700)
+    c, x, h0 = _oracle(w)
+    r = binding.solve_workload(w, "ELK", lam=1e-3, tol=1e-6)
+    assert r.status == "OK"
+    assert np.max(np.abs(r.h.double().cpu().numpy() - rollout(c, x, h0))) <= 1e-4
+
+
+def test_elk_full_size_sampled():
+    """The full near-unstable workload (B = 8, T = 10000, D = 64)."""
+    w = make_workload("near_unstable")
+    r = binding.solve_workload(w, "ELK", lam=0.01)
+    assert r.status == "OK"
+    c = GRU.from_workload(w)
+    h = r.h.cpu()
+    for b in (0, 5):
+        want = rollout(c, w.x[b:b + 1].double().numpy(), w.h0[b:b + 1].double().numpy())
+        assert np.max(np.abs(h[b:b + 1].double().numpy() - want)) <= 1e-4
+    p = os.path.join(os.path.dirname(__file__), "golden", "oracle_iters.json")
+    g = json.load(open(p)).get("near_unstable/ELK/0.01") if os.path.exists(p) else None
+    if g is not None:
+        assert abs(r.iters - g["iters"]) <= 1, (r.iters, g["iters"])
+
+
+def test_elk_nan_input_diverges_and_bad_lambda_rejected():
+    w = make_workload("near_unstable", B=2, T=200)
+    w.x[1, 50, 3] = float("nan")
+    r = binding.solve_workload(w, "ELK", lam=0.1)
+    assert r.status == "DIVERGED" and r.iters == 1
+    w = make_workload("near_unstable", B=1, T=50)
+    with pytest.raises(Exception):
+        binding.solve_workload(w, "ELK", lam=0.0)
