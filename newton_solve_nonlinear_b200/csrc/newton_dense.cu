@@ -54,11 +54,14 @@ DenseGeom dense_geom(int B, int T, int D) {
 static size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 size_t dense_elk_ws_bytes(int B, int T, int D);
+bool deer_mma_supported(const pararnn_cell &cell);
+size_t deer_mma_ws_bytes(int B, int T);
 
 // DEER: Phi [B][NC][D][D], p [B][NC][D], carry [B][NC][D]; ELK: the cyclic
 // reduction arrays of newton_dense_elk.cu.
 size_t dense_ws_bytes(const pararnn_cell &cell, int B, int T, int mode) {
     if (mode == PARARNN_ELK) return dense_elk_ws_bytes(B, T, cell.d);
+    if (deer_mma_supported(cell)) return deer_mma_ws_bytes(B, T);
     const DenseGeom g = dense_geom(B, T, cell.d);
     const size_t n = static_cast<size_t>(B) * g.NC;
     const size_t D = cell.d;
@@ -650,10 +653,13 @@ cudaError_t launch_dscan(const DScanArgs &S, cudaStream_t s) {
 
 size_t dense_elk_ws_bytes(int B, int T, int D);
 cudaError_t launch_dense_elk(const DiagArgs &a, void *ws, cudaStream_t s);
+bool deer_mma_supported(const pararnn_cell &cell);
+cudaError_t launch_deer_mma(const DiagArgs &a, void *ws, cudaStream_t s);
 
 cudaError_t launch_dense_solver(const pararnn_cell &cell, int mode, const DiagArgs &a,
                                 void *dense_ws, cudaStream_t s) {
     if (mode == PARARNN_ELK) return launch_dense_elk(a, dense_ws, s);
+    if (mode == PARARNN_DEER && deer_mma_supported(cell)) return launch_deer_mma(a, dense_ws, s);
     if (mode != PARARNN_DEER) return cudaErrorNotSupported;
     DenseArgs S;
     S.a = a;
