@@ -1,14 +1,19 @@
 #!/usr/bin/env python
 """Benchmark: converged GRU states per second by parallel Newton on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--T T]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--T T]
 
-A step is one whole solve of the untrained dense GRU workload (Din = D = 64,
-B = 16 sequences per GPU, T = 65536, fp32, weights N(0, 1/D), inputs N(0, 1),
-quasi-DEER to tol 1e-5): the input projection, then every Newton iteration
-(fused cell + diagonal Jacobian + single-pass scan + convergence reduction)
-until the on-device test stops it.  value = B*T*D states x steps x ranks /
-(max over ranks of the device time of the K timed steps).
+A step is one whole solve: the input projection, then every Newton iteration
+until the on-device test stops it.  The default workload is the untrained
+dense GRU (Din = D = 64, B = 16 sequences per GPU, T = 65536, fp32, weights
+N(0, 1/D), inputs N(0, 1), quasi-DEER to tol 1e-5: fused cell + diagonal
+Jacobian + single-pass scan + convergence reduction per iteration).
+``--workload`` selects another solver family with the same line format:
+diag (diagonal-recurrence GRU, exact Newton), dense_deer (full-Jacobian DEER
+on tensor cores), quasi_elk and elk (damped steps on the near-unstable GRU).
+value = B*T*D states x steps x ranks / (max over ranks of the device time of
+the K timed steps).
 
 Sequences are independent, so N GPUs run N replicas of the per-GPU batch
 (weak scaling, no data-path collective); the launcher is torchrun, one rank
@@ -33,10 +38,50 @@ sys.path.insert(0, ROOT)
 
 METRIC = "converged states/sec (B*T*D per s, Newton to tol)"
 UNIT = "states/s"
-WORKLOAD = "untrained dense GRU Din=D=64, B=16/GPU, T={T}, fp32, quasi-DEER tol 1e-5"
-# bytes each state moves per Newton iteration in a fused single pass:
-# P (3 fp32 pre-activations) + previous guess + new guess
-BYTES_PER_STATE_ITER = 20
+# The benchmarked solves, one per row family of the hot path.  "untrained"
+# (the default) is the headline; the others measure the other solver kernels
+# with the same JSON line.  Roofline units per state and Newton iteration:
+#   hbm    algorithmic bytes a fused single pass moves: P (3 fp32
+#          pre-activations) + previous guess + new guess = 20 B; quasi-ELK
+#          forward (P + guess, writes m, P, a, b) + backward (reads 16, guess 4,
+#          writes 4) = 56 B;
+#   tensor D x D Jacobian products, 2 D^3 flop per step = 2 D^2 per state;
+#   alu    dense ELK cyclic reduction, about 14 D^3 flop per step (J^T J 2 D^3,
+#          each step eliminated once: inverse + two products 6 D^3, folded once:
+#          three products 6 D^3) = 14 D^2 per state.
+BENCHES = {
+    "untrained": dict(
+        workload="untrained", mode="QUASI", lam=0.0, bound="hbm", per_state=20,
+        kernel="quasi_tc_kernel<64> (persistent, all iterations)",
+        desc="untrained dense GRU Din=D=64, B={B}/GPU, T={T}, fp32, quasi-DEER tol 1e-5",
+        cpu_sample=dict(B=16, T=1024), ref_sample=dict(B=4, T=256)),
+    "diag": dict(
+        workload="diag", mode="QUASI", lam=0.0, bound="hbm", per_state=20,
+        kernel="diag_solver_kernel<diag cell, quasi> (persistent, all iterations)",
+        desc="diagonal-recurrence GRU Din=D=2048, B={B}/GPU, T={T}, bf16 x and W_ih, fp32 state, "
+             "quasi-DEER (exact Newton) tol 1e-4",
+        cpu_sample=dict(B=1, T=1024), ref_sample=dict(B=1, T=128)),
+    "dense_deer": dict(
+        workload="dense_deer", mode="DEER", lam=0.0, bound="tensor", per_state=None,
+        kernel="deer_mma_kernel (persistent, all iterations)",
+        desc="dense GRU Din=16, D=32, B={B}/GPU, T={T}, fp32 cell, TF32 Jacobian products, DEER tol 1e-5",
+        cpu_sample=dict(B=1, T=4096), ref_sample=dict(B=1, T=512)),
+    "quasi_elk": dict(
+        workload="near_unstable", mode="QUASI_ELK", lam=0.1, bound="hbm", per_state=56,
+        kernel="diag_solver_kernel<dense cell, quasi-ELK> (persistent, all iterations)",
+        desc="near-unstable dense GRU Din=D=64 (spectral radius 1.5), B={B}/GPU, T={T}, fp32, "
+             "quasi-ELK lambda 0.1, tol 1e-4",
+        cpu_sample=dict(B=1, T=2000), ref_sample=dict(B=1, T=250)),
+    "elk": dict(
+        workload="near_unstable", mode="ELK", lam=0.01, bound="alu", per_state=None,
+        kernel="dense_elk_kernel<64> (persistent, all iterations)",
+        desc="near-unstable dense GRU Din=D=64 (spectral radius 1.5), B={B}/GPU, T={T}, fp32, "
+             "ELK lambda 0.01, tol 1e-4",
+        cpu_sample=dict(B=1, T=1000), ref_sample=dict(B=1, T=150)),
+}
+# fp32 FMA peak for the ALU-bound row: 148 SMs x 128 fp32 lanes x 2 flop x
+# 1965 MHz (the part's maximum SM clock), in TFLOP/s.
+ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # ncu DRAM traffic of the solver kernel (read + write bytes of one launch,
 # captured at T = 16384: 4.812 GB over 14 iterations x 16.78 M states) and the
 # hash of the kernel source it was measured on.  Traffic grows with states x
@@ -56,6 +101,14 @@ def peaks():
         d = json.load(open(p))
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def tf32_peak():
+    """Dense TF32 TFLOP/s: the measured bf16 burst peak x 1/2 (nominal ratio)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return float(json.load(open(p))["bf16_tflops"]) / 2
+    return 1590.0 / 2
 
 
 def kernel_sha():
@@ -109,9 +162,9 @@ class Clocks:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def cpu_baseline_oracle(T_sample: int = 1024, B_sample: int = 16):
-    """Time the fp64 oracle (as it stands) on a bounded sample of the workload."""
-    import numpy as np
+def cpu_baseline_oracle(spec: dict, sample: dict):
+    """Time the fp64 oracle (as it stands) on a bounded sample of the workload:
+    the same generator and distributions, fewer sequences and steps."""
     import oracle
     from oracle.cells import GRU
     from newton_solve_nonlinear_b200.inputs import make_workload
@@ -120,35 +173,43 @@ def cpu_baseline_oracle(T_sample: int = 1024, B_sample: int = 16):
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:  # pragma: no cover
         cores = 1
-    w = make_workload("untrained", B=B_sample, T=T_sample)
+    w = make_workload(spec["workload"], **sample)
     c = GRU.from_workload(w)
     x, h0 = w.x.double().numpy(), w.h0.double().numpy()
+    mode = spec["mode"]
     t0 = time.perf_counter()
-    r = oracle.newton_solve(c, x, h0, "QUASI", w.tol)
+    if mode in ("ELK", "QUASI_ELK"):
+        r = oracle.elk_solve(c, x, h0, mode, spec["lam"], w.tol)
+    else:
+        r = oracle.newton_solve(c, x, h0, mode, w.tol)
     secs = time.perf_counter() - t0
     states = w.B * w.T * w.d
     return {"value": states / secs, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"fp64 numpy oracle quasi-DEER to tol 1e-5 on B={w.B}, T={w.T}, D=64 "
-                      f"({r['iters']} iterations, {secs:.1f} s); same distributions"}
+            "sample": f"fp64 numpy oracle, {mode} to tol {w.tol:g} on B={w.B}, T={w.T}, "
+                      f"D={w.d} ({r['iters']} iterations, {secs:.1f} s); same distributions"}
 
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    spec = BENCHES[args.workload]
     steps = []
     base = None
     for i in range(args.warmup + args.steps):
-        cb = cpu_baseline_oracle(T_sample=256, B_sample=4)
+        cb = cpu_baseline_oracle(spec, spec["ref_sample"])
         if i >= args.warmup:
             steps.append(cb["value"])
         base = cb
     v = statistics.median(steps)
+    from newton_solve_nonlinear_b200.inputs import WORKLOADS
+    full = WORKLOADS[spec["workload"]]
+    T = args.T or full["T"]
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD.format(T=args.T), "sample": base["sample"]},
+            "config": {"workload": spec["desc"].format(B=full["B"], T=T), "sample": base["sample"]},
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": base["cores"], "kind": "oracle",
                              "sample": base["sample"]},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -175,24 +236,27 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    w = make_workload("untrained", T=args.T, seed=rank)
-    B, T, D, din = w.B, w.T, w.d, w.din
+    spec = BENCHES[args.workload]
+    mode, lam = spec["mode"], spec["lam"]
+    over = {"T": args.T} if args.T else {}
+    w = make_workload(spec["workload"], seed=rank, **over)
+    B, T, D, din, kind = w.B, w.T, w.d, w.din, w.kind
     states = B * T * D
     g = lambda t: t.to(dev).contiguous()
     w_ih, b_ih, w_hh, b_hh, x, h0 = map(g, (w.w_ih, w.b_ih, w.w_hh, w.b_hh, w.x, w.h0))
-    cell = binding.make_cell("dense", din, D, torch.float32)
-    ws = binding.alloc_workspace(binding.workspace_size("dense", din, D, B, T, "QUASI"), dev)
+    ws = binding.alloc_workspace(
+        binding.workspace_size(kind, din, D, B, T, mode, w.x_dtype), dev)
     P = torch.empty(B, T, 3 * D, dtype=torch.float32, device=dev)
     out = torch.empty(B, T, D, dtype=torch.float32, device=dev)
     info = torch.zeros(4, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step(ev_mid=None):
-        binding.input_projection(x, w_ih, b_ih, d=D, out=P)
+        binding.input_projection(x, w_ih, b_ih, d=D, kind=kind, out=P)
         if ev_mid is not None:
             ev_mid.record(stream)
-        binding.newton_iterate(P, w_hh, b_hh, h0, kind="dense", din=din, mode="QUASI",
-                               tol=w.tol, info_dev=info, out=out, workspace=ws)
+        binding.newton_iterate(P, w_hh, b_hh, h0, kind=kind, din=din, mode=mode, lam=lam,
+                               tol=w.tol, info_dev=info, out=out, workspace=ws, dtype=w.x_dtype)
 
     for _ in range(args.warmup):
         step()
@@ -232,8 +296,8 @@ def run_ours(args):
     ea.record(stream)
     for _ in range(e2e_steps):
         x_dev.copy_(x_host, non_blocking=True)
-        r = binding.newton_solve(w_ih, b_ih, w_hh, b_hh, x_dev, h0, kind="dense", mode="QUASI",
-                                 tol=w.tol, out=out, workspace=ws)
+        binding.newton_solve(w_ih, b_ih, w_hh, b_hh, x_dev, h0, kind=kind, mode=mode, lam=lam,
+                             tol=w.tol, out=out, workspace=ws)
         h_host.copy_(out, non_blocking=True)
     eb.record(stream)
     torch.cuda.synchronize()
@@ -244,34 +308,50 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1:
-        cpu = cpu_baseline_oracle()
+        cpu = cpu_baseline_oracle(spec, spec["cpu_sample"])
 
-    peak, peak_kind = peaks()
+    hbm_peak, peak_kind = peaks()
     solver_avg_s = statistics.mean(solver_ms) / 1e3
-    algo_bytes = iters * states * BYTES_PER_STATE_ITER
-    achieved = algo_bytes / solver_avg_s / 1e9
-    traffic = (NCU_TRAFFIC["bytes_per_state_iter"] * iters * states
-               if NCU_TRAFFIC["source_sha1"] == kernel_sha() else None)
+    traffic = None
+    if spec["bound"] == "hbm":
+        per_state = spec["per_state"]
+        achieved = iters * states * per_state / solver_avg_s / 1e9
+        peak, unit = hbm_peak, "GB/s"
+        algo = f"{per_state} B/state/iteration x {iters} iterations x {states} states"
+        pk = f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+        if args.workload == "untrained" and NCU_TRAFFIC["source_sha1"] == kernel_sha():
+            traffic = NCU_TRAFFIC["bytes_per_state_iter"] * iters * states
+    elif spec["bound"] == "tensor":
+        per_state = 2 * D * D
+        achieved = iters * states * per_state / solver_avg_s / 1e12
+        peak, unit = tf32_peak(), "TFLOP/s"
+        algo = f"2 D^3 flop/step = {per_state} flop/state/iteration x {iters} x {states} states"
+        pk = "TF32 dense = MEASURED_PEAKS.json bf16_tflops x 1/2 (nominal TF32:bf16 ratio)"
+    else:
+        per_state = 14 * D * D
+        achieved = iters * states * per_state / solver_avg_s / 1e12
+        peak, unit = ALU_PEAK_TFLOPS, "TFLOP/s"
+        algo = f"14 D^3 flop/step = {per_state} flop/state/iteration x {iters} x {states} states"
+        pk = "fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1965 MHz"
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD.format(T=T), "B": B, "T": T, "D": D, "din": din,
-                   "mode": "QUASI", "tol": w.tol, "iters": iters,
-                   "status": binding.STATUS.get(status),
-                   "l2": (f"inputs larger than L2 (126 MB): x {x.numel() * 4 / 1e6:.0f} MB, "
-                          f"P {P.numel() * 4 / 1e6:.0f} MB, h {out.numel() * 4 / 1e6:.0f} MB per solve"),
+        "config": {"workload": spec["desc"].format(B=B, T=T), "name": args.workload,
+                   "B": B, "T": T, "D": D, "din": din, "cell": kind, "mode": mode,
+                   "lambda": lam if mode in ("ELK", "QUASI_ELK") else None,
+                   "tol": w.tol, "iters": iters, "status": binding.STATUS.get(status),
+                   "l2": (f"inputs larger than L2 (126 MB) summed per solve: "
+                          f"x {x.numel() * x.element_size() / 1e6:.0f} MB, "
+                          f"P {P.numel() * 4 / 1e6:.0f} MB, h {out.numel() * 4 / 1e6:.0f} MB"),
                    "parallelism": f"replicas over sequences x{world}",
                    "projection_ms": statistics.mean(proj_ms),
                    "solver_ms": statistics.mean(solver_ms)},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "quasi_tc_kernel<64> (persistent, all iterations)",
-                     "algorithmic_bytes": f"{BYTES_PER_STATE_ITER} B/state/iteration x {iters} "
-                                          f"iterations x {states} states",
-                     "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"},
+        "roofline": {"bound": spec["bound"], "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "traffic": traffic, "kernel": spec["kernel"],
+                     "algorithmic": algo, "peak_kind": pk},
         "e2e": {"value": e2e_value, "unit": UNIT,
-                "h2d_bytes_per_step": x_host.numel() * 4,
+                "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
                 "d2h_bytes_per_step": h_host.numel() * 4 + 16},
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
@@ -291,7 +371,9 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--T", type=int, default=65536)
+    ap.add_argument("--workload", default="untrained", choices=sorted(BENCHES),
+                    help="which solve to time (default: the untrained dense GRU headline)")
+    ap.add_argument("--T", type=int, default=0, help="override the sequence length")
     args = ap.parse_args()
     if args.warmup < 3:
         log("warmup raised to 3 (timing rule)")
