@@ -52,7 +52,7 @@ UNIT = "states/s"
 BENCHES = {
     "untrained": dict(
         workload="untrained", mode="QUASI", lam=0.0, bound="hbm", per_state=20,
-        kernel="quasi_tc_kernel<64> (persistent, all iterations)",
+        kernel="quasi_tc2_kernel<64> (persistent, all iterations)",
         desc="untrained dense GRU Din=D=64, B={B}/GPU, T={T}, fp32, quasi-DEER tol 1e-5",
         cpu_sample=dict(B=16, T=1024), ref_sample=dict(B=4, T=256)),
     "diag": dict(
@@ -82,13 +82,12 @@ BENCHES = {
 # fp32 FMA peak for the ALU-bound row: 148 SMs x 128 fp32 lanes x 2 flop x
 # 1965 MHz (the part's maximum SM clock), in TFLOP/s.
 ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
-# ncu DRAM traffic of the solver kernel (read + write bytes of one launch,
-# captured at T = 16384: 4.812 GB over 14 iterations x 16.78 M states) and the
+# ncu DRAM traffic of the solver kernel per state and iteration (read + write
+# bytes of one launch captured at T = 16384, / (iterations x states)) and the
 # hash of the kernel source it was measured on.  Traffic grows with states x
 # iterations, so the full launch's is scaled from it; reported only while the
 # source is unchanged.
-NCU_TRAFFIC = {"bytes_per_state_iter": 4.812e9 / (14 * 16 * 16384 * 64),
-               "source_sha1": "6cb957761e3f"}
+NCU_TRAFFIC = {"bytes_per_state_iter": None, "source_sha1": None}
 
 
 def log(*a):
@@ -112,7 +111,7 @@ def tf32_peak():
 
 
 def kernel_sha():
-    src = os.path.join(ROOT, "newton_solve_nonlinear_b200", "csrc", "newton_dense_tc.cu")
+    src = os.path.join(ROOT, "newton_solve_nonlinear_b200", "csrc", "newton_dense_tc2.cu")
     return hashlib.sha1(open(src, "rb").read()).hexdigest()[:12]
 
 

@@ -1,0 +1,637 @@
+// newton_dense_tc2.cu -- quasi-DEER on the dense GRU, software-pipelined over
+// tiles, with the recurrent product U h_{t-1} on the 5th-generation tensor
+// cores (tcgen05, sm_100a) and the time scan in registers.
+//
+// Method: "Towards Scalable and Stable Parallelization of Nonlinear RNNs"
+// (atlas summary, "Approach": quasi-DEER, the diagonal of the Jacobian, O(TD)
+// memory and work per iteration) on the unrolled system of the ParaRNN summary
+// ("Core Idea", "Newton's Iteration"), with the affine scan as a single pass
+// over time (decoupled look-back between tiles).
+//
+// One cooperative launch runs every Newton iteration; one CTA per SM walks
+// tiles of (sequence b, 128 steps, all D state lanes), chunk-major.  Each
+// tile's guess rows h_{t0-1} .. h_{t0+127} arrive by TMA in one of two
+// shared-memory slots.  While tile i is finished by all eight warps, the
+// asynchronous units already work on the next ones:
+//   * tile i+1's rows h_{t-1} are split into a TF32-exact high part and an fp32
+//     remainder and written to TMEM as the A operand; one thread then issues
+//     tcgen05.mma kind::tf32 (M = 128 steps, N = 3D gate rows, K = 8 per
+//     instruction) for lo*U_hi + hi*U_lo + hi*U_hi (the error-compensated
+//     3 x TF32 split: G = U h_{t-1} fp32-accurate) into the second of two
+//     TMEM accumulators (U_hi / U_lo stay in shared memory for the solve);
+//   * tile i+2's rows are in flight by TMA into the slot tile i frees.
+// Tile i's epilogue reads its accumulator in the 16x256b fragment layout
+// (each thread: 4 steps x 8 lanes, all three gates), evaluates the cell and
+// its Jacobian diagonal (a_t, b_t = f_t - a_t h_{t-1}), and scans over time
+// without leaving registers: Kogge-Stone over the 8 steps a quad column holds
+// (warp shuffles), a 4-group prefix inside the thread, a 4-warp prefix through
+// shared memory, and the tile's carry-in by decoupled look-back over earlier
+// chunks of the sequence.  Every state is then final and is stored with the
+// convergence maxima max |h^(i+1) - h^(i)| and max |h_t - f_t|.
+// Traffic per state and iteration: P (12 B), the guess (4 B, by TMA),
+// h^(i+1) (4 B).  A bounded grid barrier ends each iteration.
+#include "common.cuh"
+#include "lookback.cuh"
+#include "solver.cuh"
+#include "tc_utils.cuh"
+
+namespace pararnn {
+namespace {
+using namespace tc;
+
+constexpr int TM = 128;        // steps per tile (MMA M)
+constexpr int NTHREADS = 512;  // 16 warps: TMEM lane quarter x lane quarter
+constexpr int ROWS = TM + 1;   // staged guess rows t0-1 .. t0+127
+
+template <int D>
+struct Tc2Geom {
+    static constexpr int N = 3 * D;                  // MMA N: gate rows (r, z, n) x lanes
+    static constexpr int HALVES = D / 32;            // 128-byte K atoms per row
+    static constexpr int SLOT_HALF = 17 * 1024;      // one K atom of ROWS staged rows (1 KB aligned)
+    static constexpr int SLOT_BYTES = HALVES * SLOT_HALF;
+    static constexpr int SLOT_TX = HALVES * ROWS * 128;  // bytes one TMA fill delivers
+    static constexpr int B_HALF = N * 128;
+    static constexpr int B_BYTES = HALVES * B_HALF;
+    // TMEM columns: accumulators at 0 and ACC1, A operand hi / lo after them
+    static constexpr int ACC1 = (N + 63) / 64 * 64;
+    static constexpr int A_HI = 2 * ACC1;
+    static constexpr int A_LO = A_HI + 64;
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int LH = D / 4;   // lanes per warp group in the epilogue
+    static constexpr int NJ = LH / 8;  // 8-lane column groups per thread
+    static constexpr int KW = D / 4;   // K columns of the A operand each warp writes
+    static constexpr int V = 2 * NJ;   // consecutive lanes per epilogue thread
+    // The MMA's N order is permuted inside each gate so that the 16x256b
+    // fragment hands thread tq of lane group lh the lanes lh LH + V tq .. + V-1:
+    // accumulator column c = lh LH + 8 j + 2 tq + x holds lane
+    // lh LH + V tq + 2 j + x.
+    static __device__ __forceinline__ int lane_of_col(int c) {
+        const int lh = c / LH, w = c % LH, j = w >> 3, tq = (w >> 1) & 3, x = w & 1;
+        return lh * LH + V * tq + 2 * j + x;
+    }
+    static constexpr int OFF_BHI = 0;
+    static constexpr int OFF_BLO = B_BYTES;
+    static constexpr int OFF_SLOT = 2 * B_BYTES;
+    static constexpr int OFF_MISC = OFF_SLOT + 2 * SLOT_BYTES;
+    // misc floats: b_hh 3D, diag U 3D, warp-quarter totals 2 x 4D, carries D, reduction 32
+    static constexpr int MISC_FLOATS = 6 * D + 8 * D + D + 32;
+    static constexpr int SMEM_BYTES = OFF_MISC + MISC_FLOATS * 4 + 64 + 1024;
+    static_assert(D == 32 || D == 64, "tensor-core cell path takes D = 32 or 64");
+    static_assert(A_LO + 64 <= TMEM_COLS, "TMEM columns");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+struct Tc2Args {
+    DiagArgs a;
+    int n_chunks;
+    long long n_tiles;
+};
+
+// Swizzled byte offset of element (row, k) inside a K-major 128-byte-swizzle
+// tile made of K atoms of `half_bytes` each (rows of 128 bytes).
+__device__ __forceinline__ int sw_off(int row, int k, int half_bytes) {
+    const int hf = k >> 5, j = (k & 31) >> 2;
+    return hf * half_bytes + row * 128 + ((j ^ (row & 7)) << 4) + ((k & 3) << 2);
+}
+
+// V consecutive floats (V = 4 or 2; 16- resp. 8-byte aligned).
+template <int V>
+__device__ __forceinline__ void ldv(const float *p, float (&o)[V]) {
+    if constexpr (V == 4) {
+        const float4 v = *reinterpret_cast<const float4 *>(p);
+        o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+    } else {
+        const float2 v = *reinterpret_cast<const float2 *>(p);
+        o[0] = v.x; o[1] = v.y;
+    }
+}
+template <int V>
+__device__ __forceinline__ void ldgv(const float *p, float (&o)[V]) {
+    if constexpr (V == 4) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(p));
+        o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+    } else {
+        const float2 v = __ldg(reinterpret_cast<const float2 *>(p));
+        o[0] = v.x; o[1] = v.y;
+    }
+}
+template <int V>
+__device__ __forceinline__ void stv(float *p, const float (&v)[V]) {
+    if constexpr (V == 4)
+        __stcg(reinterpret_cast<float4 *>(p), make_float4(v[0], v[1], v[2], v[3]));
+    else
+        __stcg(reinterpret_cast<float2 *>(p), make_float2(v[0], v[1]));
+}
+
+// Affine map composition: apply (a1, b1) first, then (a2, b2).
+__device__ __forceinline__ void compose(float &a2, float &b2, float a1, float b1) {
+    b2 = fmaf(a2, b1, b2);
+    a2 = a2 * a1;
+}
+
+// 16 / 8 consecutive TMEM columns of this warp's lane quarter <- registers.
+__device__ __forceinline__ void tmem_st(unsigned taddr, const unsigned (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+        "%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st(unsigned taddr, const unsigned (&v)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+                 "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+
+// A operand of the tile staged in `slot`: rows r = 0..127 are h_{t0+r-1}
+// (staged row r; h0 replaces it for a sequence's first step).  Warp (quarter
+// qd, column group kq) writes TMEM lanes 32 qd .. 32 qd + 31 (its own lane
+// quarter), K columns kq KW .. kq KW + KW - 1, split into hi (A_HI) and lo (A_LO).
+template <int D>
+__device__ __forceinline__ void write_a(const unsigned char *slot, unsigned tmem, const float *h0row,
+                                        bool first_chunk, int warp, int lane) {
+    using G = Tc2Geom<D>;
+    constexpr int KW = G::KW;
+    const int qd = warp & 3, kq = warp >> 2;
+    const int r = qd * 32 + lane;
+    const int k0 = kq * KW;
+    float v[KW];
+#pragma unroll
+    for (int q = 0; q < KW / 4; ++q) {
+        const float4 x = *reinterpret_cast<const float4 *>(slot + sw_off(r, k0 + 4 * q, G::SLOT_HALF));
+        v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+    }
+    if (first_chunk && r == 0)
+#pragma unroll
+        for (int q = 0; q < KW; ++q) v[q] = __ldg(h0row + k0 + q);
+    unsigned hi[KW], lo[KW];
+#pragma unroll
+    for (int q = 0; q < KW; ++q) {
+        hi[q] = __float_as_uint(v[q]) & 0xffffe000u;
+        lo[q] = __float_as_uint(v[q] - __uint_as_float(hi[q]));
+    }
+    const unsigned lane_base = static_cast<unsigned>(qd * 32) << 16;
+    tmem_st(tmem + lane_base + G::A_HI + k0, hi);
+    tmem_st(tmem + lane_base + G::A_LO + k0, lo);
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// One thread: G = lo*U_hi + hi*U_lo + hi*U_hi into accumulator `acc`, then
+// commit to `bar`.
+template <int D>
+__device__ __forceinline__ void issue_mma(unsigned tmem, unsigned acc, unsigned b_hi, unsigned b_lo,
+                                          unsigned idesc, unsigned bar) {
+    using G = Tc2Geom<D>;
+#pragma unroll
+    for (int term = 0; term < 3; ++term) {
+        const unsigned a_col = term == 0 ? G::A_LO : G::A_HI;
+        const unsigned bs = term == 1 ? b_lo : b_hi;
+#pragma unroll
+        for (int ks = 0; ks < D / 8; ++ks) {
+            const int hf = ks >> 2, off = (ks & 3) * 32;
+            const unsigned long long db = sw128_desc(bs + hf * G::B_HALF + off);
+            const unsigned en = (term > 0 || ks > 0) ? 1u : 0u;
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "setp.ne.b32 p, %4, 0;\n\t"
+                "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(
+                    tmem + acc),
+                "r"(tmem + a_col + ks * 8), "l"(db), "r"(idesc), "r"(en), "r"(0u));
+        }
+    }
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar));
+}
+
+// Pull a tile's input pre-activations (rows t0 .. t0+127 of P, contiguous,
+// clamped to the sequence) into L2 ahead of use.
+template <int D>
+__device__ __forceinline__ void prefetch_p(const float *P, long long tile, int B, int T) {
+    const int t0 = static_cast<int>(tile / B) * TM;
+    const int n = min(TM, T - t0);
+    const float *src = P + (static_cast<size_t>(tile % B) * T + t0) * 3 * D;
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(n * 3 * D * 4) : "memory");
+}
+
+template <int D>
+__device__ __forceinline__ void issue_fill(const CUtensorMap *map, unsigned char *slot, long long row0,
+                                           unsigned bar) {
+    using G = Tc2Geom<D>;
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // after the slot's last reads
+    mbar_expect_tx(bar, G::SLOT_TX);
+#pragma unroll
+    for (int hf = 0; hf < G::HALVES; ++hf)
+        tma_load_2d(smem_u32(slot + hf * G::SLOT_HALF), map, hf * 32, static_cast<int>(row0 - 1), bar);
+}
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
+quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_constant__ CUtensorMap map_h1,
+                 Tc2Args S) {
+    using G = Tc2Geom<D>;
+    constexpr int LH = G::LH, NJ = G::NJ;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    unsigned char *bhi = smem + G::OFF_BHI, *blo = smem + G::OFF_BLO;
+    unsigned char *slots = smem + G::OFF_SLOT;
+    float *misc = reinterpret_cast<float *>(smem + G::OFF_MISC);
+    float *c_bh = misc;                   // [3D] b_hh
+    float *c_ud = c_bh + 3 * D;           // [3D] diagonal of U_g
+    float *wt_a = c_ud + 3 * D;           // [4][D] affine total of each warp quarter's 32 steps
+    float *wt_b = wt_a + 4 * D;
+    float *carry = wt_b + 4 * D;          // [D] tile carry-in
+    unsigned *red = reinterpret_cast<unsigned *>(carry + D);  // [32]
+    unsigned long long *bars = reinterpret_cast<unsigned long long *>(red + 32);  // fill[2], mma[2]
+    unsigned *tmem_slot = reinterpret_cast<unsigned *>(bars + 4);
+    volatile int *cta_err = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const DiagArgs &A = S.a;
+    const int T = A.T, B = A.B;
+    WsHeader *hdr = A.hdr;
+    unsigned *status = &hdr->status;
+    const unsigned nblocks = gridDim.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int qd = warp & 3, lh = warp >> 2, gid = lane >> 2, tq = lane & 3;
+    constexpr int V = G::V;
+    const int dbase = lh * LH + V * tq;  // this thread's lanes in the epilogue and scan
+
+    // ---- once per solve: U split into TF32 hi / lo, constants, barriers, TMEM
+    for (int i = tid; i < G::N * D; i += NTHREADS) {
+        const int n = i / D, k = i % D;
+        const int g = n / D, dl = G::lane_of_col(n % D);
+        const float v = __ldg(A.w_hh + (static_cast<size_t>(g) * D + dl) * D + k);
+        const float hi = __uint_as_float(__float_as_uint(v) & 0xffffe000u);
+        const int off = sw_off(n, k, G::B_HALF);
+        *reinterpret_cast<float *>(bhi + off) = hi;
+        *reinterpret_cast<float *>(blo + off) = v - hi;
+    }
+    for (int i = tid; i < 3 * D; i += NTHREADS) {
+        c_bh[i] = __ldg(A.b_hh + i);
+        const int g = i / D, d = i % D;
+        c_ud[i] = __ldg(A.w_hh + (static_cast<size_t>(g) * D + d) * D + d);
+    }
+    if (tid == 0) {
+        for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&bars[q]), 1);
+        *cta_err = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(G::TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("tcgen05.fence::before_thread_sync;");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;");
+    const unsigned tmem = *tmem_slot;
+    constexpr unsigned idesc = make_idesc(2u, TM, G::N);  // kind::tf32, M=128, N=3D
+    const unsigned b_hi = smem_u32(bhi), b_lo = smem_u32(blo);
+
+    // bit q: mbarrier parity of fill slot q / accumulator q; an operation in flight
+    unsigned fill_par = 0u, mma_par = 0u, fill_pending = 0u, mma_pending = 0u;
+    const long long my_n =
+        blockIdx.x < S.n_tiles ? (S.n_tiles - blockIdx.x + nblocks - 1) / nblocks : 0;
+    auto tile_of = [&](long long k) { return static_cast<long long>(blockIdx.x) + k * nblocks; };
+    auto row0_of = [&](long long tile) {
+        return static_cast<long long>(tile % B) * T + static_cast<long long>(tile / B) * TM;
+    };
+
+    int iters = 0, final_status = PARARNN_NOT_CONVERGED;
+    unsigned last_delta = 0u, last_resid = 0u;
+    for (int it = 0; it < A.max_iters; ++it) {
+        if (blockIdx.x == 0 && tid == 0) {
+            hdr->delta_bits[(it + 1) % 3] = 0u;
+            hdr->resid_bits[(it + 1) % 3] = 0u;
+        }
+        float *hnew = A.hbuf[(it + 1) & 1];
+        const CUtensorMap *map = (it & 1) ? &map_h1 : &map_h0;
+        const unsigned epoch = static_cast<unsigned>(it + 1);
+        unsigned dmax = 0u, rmax = 0u;
+
+        // prologue: fill slots 0 and 1, operand + products of the first tile
+        if (tid == 0) {
+            for (int q = 0; q < 2 && q < my_n; ++q) {
+                prefetch_p<D>(A.P, tile_of(q), B, T);
+                issue_fill<D>(map, slots + q * G::SLOT_BYTES, row0_of(tile_of(q)), smem_u32(&bars[q]));
+            }
+        }
+        fill_pending = my_n > 1 ? 3u : (my_n > 0 ? 1u : 0u);
+        if (my_n > 0) {
+            if (!mbar_wait(smem_u32(&bars[0]), fill_par & 1u, cta_err)) *cta_err = 1;
+            fill_par ^= 1u;
+            fill_pending &= ~1u;
+            const long long t0t = tile_of(0);
+            write_a<D>(slots, tmem, A.h0 + static_cast<size_t>(t0t % B) * D, t0t / B == 0, warp, lane);
+            asm volatile("tcgen05.fence::before_thread_sync;");
+            __syncthreads();
+            if (tid == 0) {
+                asm volatile("tcgen05.fence::after_thread_sync;");
+                issue_mma<D>(tmem, 0u, b_hi, b_lo, idesc, smem_u32(&bars[2]));
+            }
+            mma_pending |= 1u;
+        }
+
+        for (long long k = 0; k < my_n; ++k) {
+            const long long tile = tile_of(k);
+            const int chunk = static_cast<int>(tile / B), b = static_cast<int>(tile % B);
+            const int t0 = chunk * TM;
+            const long long row0 = static_cast<long long>(b) * T + t0;
+            const int cur = static_cast<int>(k & 1);
+            const unsigned char *slot = slots + cur * G::SLOT_BYTES;
+
+            if (tid == 0 && k + 2 < my_n) prefetch_p<D>(A.P, tile_of(k + 2), B, T);
+            // 1. this tile's input pre-activations: thread (gid, tq) of warp (qd, lh)
+            // owns steps r = 32 qd + 16 rh + 8 e + gid and lanes dbase .. dbase + V - 1
+            float pv[2][2][3][V];
+#pragma unroll
+            for (int rh = 0; rh < 2; ++rh)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int r = qd * 32 + rh * 16 + gid + 8 * e;
+                    const float *prow = A.P + (static_cast<size_t>(row0) + r) * 3 * D + dbase;
+#pragma unroll
+                    for (int g = 0; g < 3; ++g) {
+                        if (t0 + r < T)
+                            ldgv<V>(prow + g * D, pv[rh][e][g]);
+                        else
+#pragma unroll
+                            for (int v = 0; v < V; ++v) pv[rh][e][g][v] = 0.f;
+                    }
+                }
+
+            // 2. the products of tile k are done: refill A with tile k+1 and start its products
+            if (!mbar_wait(smem_u32(&bars[2 + cur]), (mma_par >> cur) & 1u, cta_err)) *cta_err = 1;
+            mma_par ^= 1u << cur;
+            mma_pending &= ~(1u << cur);
+            if (k + 1 < my_n) {
+                const int nxt = cur ^ 1;
+                if (!mbar_wait(smem_u32(&bars[nxt]), (fill_par >> nxt) & 1u, cta_err)) *cta_err = 1;
+                fill_par ^= 1u << nxt;
+                fill_pending &= ~(1u << nxt);
+                const long long tn = tile_of(k + 1);
+                write_a<D>(slots + nxt * G::SLOT_BYTES, tmem, A.h0 + static_cast<size_t>(tn % B) * D,
+                           tn / B == 0, warp, lane);
+                asm volatile("tcgen05.fence::before_thread_sync;");
+            }
+            __syncthreads();
+            if (*cta_err != 0) break;  // uniform: read after the barrier
+            asm volatile("tcgen05.fence::after_thread_sync;");
+            if (k + 1 < my_n) {
+                if (tid == 0)
+                    issue_mma<D>(tmem, (cur ^ 1) ? G::ACC1 : 0u, b_hi, b_lo, idesc,
+                                 smem_u32(&bars[2 + (cur ^ 1)]));
+                mma_pending |= 1u << (cur ^ 1);
+            }
+
+            // 3. epilogue: the cell at the guess, a_t and b_t per (step, lane);
+            // element (rh, e, j, x) is step r = 32 qd + 16 rh + 8 e + gid, lane
+            // dbase + 2 j + x
+            float av[2][2][NJ][2], bv[2][2][NJ][2];
+            const unsigned acc = cur ? G::ACC1 : 0u;
+#pragma unroll
+            for (int rh = 0; rh < 2; ++rh) {
+                const unsigned trow = tmem + acc + (static_cast<unsigned>(qd * 32 + rh * 16) << 16);
+                float hp[2][V], y[2][V];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int r = qd * 32 + rh * 16 + gid + 8 * e;
+                    ldv<V>(reinterpret_cast<const float *>(slot + sw_off(r, dbase, G::SLOT_HALF)), hp[e]);
+                    if (t0 == 0 && r == 0) ldgv<V>(A.h0 + static_cast<size_t>(b) * D + dbase, hp[e]);
+                    ldv<V>(reinterpret_cast<const float *>(slot + sw_off(r + 1, dbase, G::SLOT_HALF)), y[e]);
+                }
+#pragma unroll
+                for (int j = 0; j < NJ; ++j) {
+                    unsigned gv[3][4];
+#pragma unroll
+                    for (int g = 0; g < 3; ++g)
+                        asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];"
+                                     : "=r"(gv[g][0]), "=r"(gv[g][1]), "=r"(gv[g][2]), "=r"(gv[g][3])
+                                     : "r"(trow + g * D + lh * LH + 8 * j));
+                    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int r = qd * 32 + rh * 16 + gid + 8 * e;
+                        const bool ok = t0 + r < T;
+#pragma unroll
+                        for (int x = 0; x < 2; ++x) {
+                            const int v = 2 * j + x;
+                            float a_ = 1.f, b_ = 0.f;
+                            if (ok) {
+                                float f;
+                                const int d = dbase + v;
+                                gru_cell_diag(pv[rh][e][0][v], pv[rh][e][1][v], pv[rh][e][2][v],
+                                              __uint_as_float(gv[0][2 * e + x]),
+                                              __uint_as_float(gv[1][2 * e + x]),
+                                              __uint_as_float(gv[2][2 * e + x]), c_bh[d], c_bh[D + d],
+                                              c_bh[2 * D + d], c_ud[d], c_ud[D + d], c_ud[2 * D + d],
+                                              hp[e][v], f, a_, b_);
+                                rmax = max(rmax, abs_bits(y[e][v] - f));
+                            }
+                            av[rh][e][j][x] = a_;
+                            bv[rh][e][j][x] = b_;
+                        }
+                    }
+                }
+            }
+            asm volatile("tcgen05.fence::before_thread_sync;");
+
+            // 4. scan over the tile's steps, per lane d, in registers.  Inside a
+            // warp the steps of lane d are s = 16 rh + 8 e + gid (gid across the
+            // 8 lanes of one tq, (rh, e) inside the thread).
+            // 4a. inclusive Kogge-Stone across gid within each 8-step group
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) {
+#pragma unroll
+                for (int rh = 0; rh < 2; ++rh)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e)
+#pragma unroll
+                        for (int j = 0; j < NJ; ++j)
+#pragma unroll
+                            for (int x = 0; x < 2; ++x) {
+                                const float pa = __shfl_up_sync(0xffffffffu, av[rh][e][j][x], 4 * o);
+                                const float pb = __shfl_up_sync(0xffffffffu, bv[rh][e][j][x], 4 * o);
+                                if (gid >= o) compose(av[rh][e][j][x], bv[rh][e][j][x], pa, pb);
+                            }
+            }
+            // 4b. prefix over the four groups (group totals sit at gid = 7); the
+            // warp quarter's total goes to shared memory
+#pragma unroll
+            for (int j = 0; j < NJ; ++j)
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    float ea = 1.f, eb = 0.f;
+#pragma unroll
+                    for (int g4 = 0; g4 < 4; ++g4) {
+                        const int rh = g4 >> 1, e = g4 & 1;
+                        float ta = __shfl_sync(0xffffffffu, av[rh][e][j][x], 28 + tq);
+                        float tb = __shfl_sync(0xffffffffu, bv[rh][e][j][x], 28 + tq);
+                        if (g4 > 0) compose(av[rh][e][j][x], bv[rh][e][j][x], ea, eb);
+                        compose(ta, tb, ea, eb);
+                        ea = ta;
+                        eb = tb;
+                    }
+                    if (gid == 0) {
+                        const int d = dbase + 2 * j + x;
+                        wt_a[qd * D + d] = ea;
+                        wt_b[qd * D + d] = eb;
+                    }
+                }
+            __syncthreads();
+            // 4c. the tile's carry-in per lane by look-back over earlier chunks
+            if (tid < D) {
+                const int d = tid;
+                float EA = wt_a[d], EB = wt_b[d];
+#pragma unroll
+                for (int q = 1; q < 4; ++q) {
+                    float qa = wt_a[q * D + d], qb = wt_b[q * D + d];
+                    compose(qa, qb, EA, EB);
+                    EA = qa;
+                    EB = qb;
+                }
+                const float c0 = chunk == 0 ? __ldg(A.h0 + static_cast<size_t>(b) * D + d) : 0.f;
+                carry[d] = lookback_affine(A.desc, tile, B, D, d, epoch, EA, EB, chunk, c0, status);
+            }
+            __syncthreads();
+            // 4d. states: carry through the earlier warp quarters, then the thread's prefixes
+            {
+                float hin[V];
+#pragma unroll
+                for (int v = 0; v < V; ++v) {
+                    float h = carry[dbase + v];
+                    for (int q = 0; q < qd; ++q) h = fmaf(wt_a[q * D + dbase + v], h, wt_b[q * D + dbase + v]);
+                    hin[v] = h;
+                }
+#pragma unroll
+                for (int rh = 0; rh < 2; ++rh)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int r = qd * 32 + rh * 16 + gid + 8 * e;
+                        if (t0 + r < T) {
+                            float y[V], h[V];
+                            ldv<V>(reinterpret_cast<const float *>(slot + sw_off(r + 1, dbase, G::SLOT_HALF)), y);
+#pragma unroll
+                            for (int j = 0; j < NJ; ++j)
+#pragma unroll
+                                for (int x = 0; x < 2; ++x) {
+                                    const int v = 2 * j + x;
+                                    h[v] = fmaf(av[rh][e][j][x], hin[v], bv[rh][e][j][x]);
+                                    dmax = max(dmax, abs_bits(h[v] - y[v]));
+                                }
+                            stv<V>(hnew + (static_cast<size_t>(row0) + r) * D + dbase, h);
+                        }
+                    }
+            }
+
+            // 5. slot `cur` and accumulator `cur` are free: refill the slot with tile k+2
+            asm volatile("tcgen05.fence::before_thread_sync;");
+            __syncthreads();
+            if (k + 2 < my_n) {
+                if (tid == 0)
+                    issue_fill<D>(map, slots + cur * G::SLOT_BYTES, row0_of(tile_of(k + 2)),
+                                  smem_u32(&bars[cur]));
+                fill_pending |= 1u << cur;
+            }
+        }
+        const unsigned bd = block_max_u32(dmax, red);
+        const unsigned br = block_max_u32(rmax, red);
+        if (tid == 0) {
+            atomicMax(&hdr->delta_bits[it % 3], bd);
+            atomicMax(&hdr->resid_bits[it % 3], br);
+            if (*cta_err) flag_timeout(status);
+        }
+        grid_barrier(hdr->barrier, nblocks, status);
+        last_delta = ld_acquire_u32(&hdr->delta_bits[it % 3]);
+        last_resid = ld_acquire_u32(&hdr->resid_bits[it % 3]);
+        iters = it + 1;
+        if (*cta_err || timed_out(status)) { final_status = PARARNN_TIMEOUT; break; }
+        if (last_delta >= 0x7f800000u) { final_status = PARARNN_DIVERGED; break; }
+        if (__uint_as_float(last_delta) <= A.tol) { final_status = PARARNN_OK; break; }
+    }
+    if ((iters & 1) == 0 && iters > 0) {
+        const size_t n4 = static_cast<size_t>(A.B) * A.T * A.D / 4;
+        const float4 *src = reinterpret_cast<const float4 *>(A.hbuf[0]);
+        float4 *dst = reinterpret_cast<float4 *>(A.hbuf[1]);
+        for (size_t q = static_cast<size_t>(blockIdx.x) * NTHREADS + tid; q < n4;
+             q += static_cast<size_t>(nblocks) * NTHREADS)
+            dst[q] = __ldcg(src + q);
+    }
+    if (blockIdx.x == 0 && tid == 0) {
+        pararnn_info info;
+        info.iters = iters;
+        info.status = final_status;
+        info.delta = __uint_as_float(last_delta);
+        info.residual = __uint_as_float(last_resid);
+        *A.info_out = info;
+        hdr->info = info;
+    }
+    if (tid == 0) {  // copies and products still in flight after a failed wait finish first
+        for (int q = 0; q < 2; ++q) {
+            if ((fill_pending >> q) & 1u) mbar_drain(smem_u32(&bars[q]), (fill_par >> q) & 1u);
+            if ((mma_pending >> q) & 1u) mbar_drain(smem_u32(&bars[2 + q]), (mma_par >> q) & 1u);
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;");
+    __syncthreads();
+    if (warp == 1) {
+        asm volatile("tcgen05.fence::after_thread_sync;");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(G::TMEM_COLS));
+    }
+}
+
+template <int D>
+cudaError_t launch_tc2(const DiagArgs &a, cudaStream_t s) {
+    using G = Tc2Geom<D>;
+    Tc2Args S;
+    S.a = a;
+    S.n_chunks = (a.T + TM - 1) / TM;
+    S.n_tiles = static_cast<long long>(a.B) * S.n_chunks;
+    CUtensorMap m0, m1;
+    const long long rows = static_cast<long long>(a.B) * a.T;
+    if (!make_map(&m0, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.hbuf[0], rows, D, 32, ROWS) ||
+        !make_map(&m1, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.hbuf[1], rows, D, 32, ROWS))
+        return cudaErrorInvalidValue;
+    auto kern = quasi_tc2_kernel<D>;
+    // every CTA takes all 512 TMEM columns, so at most one may reside on an SM:
+    // the shared-memory request alone guarantees it
+    const int smem = G::SMEM_BYTES > 120 * 1024 ? G::SMEM_BYTES : 120 * 1024;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, nsm = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NTHREADS, smem)) != cudaSuccess)
+        return e;
+    if (per_sm != 1) return cudaErrorInvalidConfiguration;
+    long long grid = nsm;
+    if (grid > S.n_tiles) grid = S.n_tiles;
+    void *params[] = {&m0, &m1, &S};
+    return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kern),
+                                       dim3(static_cast<unsigned>(grid)), dim3(NTHREADS), params, smem, s);
+}
+
+}  // namespace
+
+// Look-back descriptors of the tensor-core path: tiles of 128 steps x D lanes, two words each.
+size_t quasi_tc_desc_bytes(int B, int T, int D) {
+    const long long tiles = static_cast<long long>(B) * ((T + TM - 1) / TM);
+    return static_cast<size_t>(tiles) * D * 2 * 8;
+}
+
+bool quasi_tc_supported(const pararnn_cell &cell, int B, int T) {
+    if (cell.kind != PARARNN_GRU_DENSE || (cell.d != 32 && cell.d != 64)) return false;
+    if (static_cast<long long>(B) * T >= (1ll << 31) - 1) return false;
+    return encode_fn() != nullptr;
+}
+
+cudaError_t launch_quasi_tc2(const DiagArgs &a, cudaStream_t s) {
+    return a.D == 32 ? launch_tc2<32>(a, s) : launch_tc2<64>(a, s);
+}
+
+}  // namespace pararnn

@@ -24,7 +24,7 @@ cudaError_t launch_dense_solver(const pararnn_cell &cell, int mode, const DiagAr
                                 void *dense_ws, cudaStream_t s);
 size_t quasi_tc_desc_bytes(int B, int T, int D);
 bool quasi_tc_supported(const pararnn_cell &cell, int B, int T);
-cudaError_t launch_quasi_tc(const DiagArgs &a, cudaStream_t s);
+cudaError_t launch_quasi_tc2(const DiagArgs &a, cudaStream_t s);
 cudaError_t launch_scan_dense(const float *A, const float *b, const float *h0, int B, int T,
                               int D, float *h, void *ws, cudaStream_t s);
 size_t scan_dense_ws_bytes(int B, int T, int D);
@@ -166,7 +166,7 @@ static cudaError_t enqueue_iterate(const pararnn_cell *cell, const pararnn_param
         // the tensor-core path reads the initial guess (zero) from memory
         e = cudaMemsetAsync(a.hbuf[0], 0, states * sizeof(float), s);
         if (e != cudaSuccess) return e;
-        return launch_quasi_tc(a, s);
+        return launch_quasi_tc2(a, s);
     }
     return diag ? launch_diag_solver(*cell, mode, a, s)
                 : launch_dense_solver(*cell, mode, a, ws + L.dense, s);
