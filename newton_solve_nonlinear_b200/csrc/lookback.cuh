@@ -66,6 +66,7 @@ __device__ __forceinline__ unsigned long long wait_tag(const unsigned long long 
 // value), [1] tag|B.  `step` is the tile distance to the predecessor
 // (+n_groups forward, -n_groups for a reverse scan); `avail` is the number of
 // predecessors (0: this tile's carry-in is `carry0`).
+template <int W = kWin>
 __device__ __forceinline__ float lookback_affine(unsigned long long *desc, long long tile,
                                                  long long step, int DG, int lane, unsigned epoch,
                                                  float EA, float EB, int avail, float carry0,
@@ -81,17 +82,17 @@ __device__ __forceinline__ float lookback_affine(unsigned long long *desc, long 
         int left = avail;
         bool done = false;
         while (!done && left > 0) {
-            const int n = left < kWin ? left : kWin;
-            unsigned long long w0[kWin], w1[kWin];
+            const int n = left < W ? left : W;
+            unsigned long long w0[W], w1[W];
 #pragma unroll
-            for (int q = 0; q < kWin; ++q)
+            for (int q = 0; q < W; ++q)
                 if (q < n) {
                     const unsigned long long *p = desc + (static_cast<size_t>(j - q * step) * DG + lane) * 2;
                     w0[q] = ld_relaxed(p);
                     w1[q] = ld_relaxed(p + 1);
                 }
 #pragma unroll
-            for (int q = 0; q < kWin; ++q)
+            for (int q = 0; q < W; ++q)
                 if (q < n && !done) {
                     const unsigned long long *p = desc + (static_cast<size_t>(j - q * step) * DG + lane) * 2;
                     unsigned long long a = w0[q];
