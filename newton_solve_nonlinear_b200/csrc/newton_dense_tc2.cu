@@ -225,90 +225,6 @@ __device__ __forceinline__ void issue_fill(const CUtensorMap *map, unsigned char
         tma_load_2d(smem_u32(slot + hf * G::SLOT_HALF), map, hf * 32, static_cast<int>(row0 - 1), bar);
 }
 
-// Decoupled look-back for lane d, shared by the G = NTHREADS / D threads of
-// one lane group (consecutive lanes of a warp; q = rank in the group).  The
-// group reads the descriptors of G predecessors at once (thread q: the
-// (q+1)-th tile back), finds the nearest one that holds an inclusive value,
-// and composes the aggregates in front of it with an ordered shuffle
-// reduction; windows repeat until an inclusive value is reached (the chunk-0
-// tile always publishes one).  Thread q = 0 publishes the tile's aggregate
-// first and its inclusive value last.  Returns the carry into the tile
-// (carry0 for a sequence's first chunk).  Waits are bounded: a descriptor
-// that never arrives reads as an inclusive 0 and raises the timeout flag.
-template <int G>
-__device__ __forceinline__ float coop_lookback(unsigned long long *desc, long long tile, long long step,
-                                               int D, int d, int q, unsigned epoch, float EA, float EB,
-                                               int avail, float carry0, unsigned *status) {
-    unsigned long long *mine = desc + (static_cast<size_t>(tile) * D + d) * 2;
-    const int lane = threadIdx.x & 31;
-    const int gbase = lane & ~(G - 1);
-    const unsigned gmask = G == 32 ? 0xffffffffu : (((1u << G) - 1u) << gbase);
-    float hin = carry0;
-    if (avail > 0) {  // the same for every thread of the CTA
-        if (q == 0) {
-            const unsigned tag = make_tag(epoch, kStateAgg);
-            st_relaxed(mine + 1, pack_word(tag, EB));
-            st_relaxed(mine, pack_word(tag, EA));
-        }
-        float accA = 1.f, accB = 0.f;
-        bool done = false;
-        for (int base = 0;; base += G) {
-            const int p = base + q;
-            float ma = 1.f, mb = 0.f, iv = 0.f;
-            bool inc = false;
-            if (!done && p < avail) {
-                const unsigned long long *pp = desc + (static_cast<size_t>(tile - (p + 1) * step) * D + d) * 2;
-                unsigned long long a = ld_relaxed(pp);
-                if (!word_ready(a, epoch)) a = wait_ready(pp, epoch, status);
-                if (a == 0ull) {
-                    inc = true;
-                } else if ((word_tag(a) & 3u) == kStateInc) {
-                    inc = true;
-                    iv = word_val(a);
-                } else {
-                    unsigned long long bw = ld_relaxed(pp + 1);
-                    if (word_tag(bw) != word_tag(a)) bw = wait_tag(pp + 1, word_tag(a), status);
-                    if (bw == 0ull) {
-                        inc = true;
-                    } else {
-                        ma = word_val(a);
-                        mb = word_val(bw);
-                    }
-                }
-            }
-            const unsigned incm = (__ballot_sync(0xffffffffu, inc) & gmask) >> gbase;
-            const int k = incm ? __ffs(incm) - 1 : G;  // nearest inclusive in this window
-            if (q >= k) {
-                ma = 1.f;
-                mb = 0.f;
-            }
-#pragma unroll
-            for (int o = 1; o < G; o <<= 1) {  // ordered: map_q o map_{q+1} o ...
-                const float na = __shfl_down_sync(0xffffffffu, ma, o);
-                const float nb = __shfl_down_sync(0xffffffffu, mb, o);
-                if ((q & (2 * o - 1)) == 0) {
-                    mb = fmaf(ma, nb, mb);
-                    ma = ma * na;
-                }
-            }
-            ma = __shfl_sync(0xffffffffu, ma, gbase);
-            mb = __shfl_sync(0xffffffffu, mb, gbase);
-            const float kv = __shfl_sync(0xffffffffu, iv, gbase + (k < G ? k : 0));
-            if (!done) {
-                accB = fmaf(accA, mb, accB);
-                accA = accA * ma;
-                if (k < G) {
-                    hin = fmaf(accA, kv, accB);
-                    done = true;
-                }
-            }
-            if (__all_sync(0xffffffffu, done)) break;
-        }
-    }
-    if (q == 0) st_relaxed(mine, pack_word(make_tag(epoch, kStateInc), fmaf(EA, hin, EB)));
-    return hin;
-}
-
 template <int D>
 __global__ void __launch_bounds__(NTHREADS, 1)
 quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_constant__ CUtensorMap map_h1,

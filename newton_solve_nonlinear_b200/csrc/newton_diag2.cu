@@ -1,0 +1,307 @@
+// newton_diag2.cu -- Newton on the diagonal-recurrence GRU (exact Newton: the
+// Jacobian of u_g * h is diagonal, so the quasi-DEER step is the DEER step),
+// as a software-pipelined streaming kernel.
+//
+// Method: the unrolled system of the ParaRNN summary ("Core Idea", "Newton's
+// Iteration") with the diagonal Jacobian of "Towards Scalable and Stable
+// Parallelization of Nonlinear RNNs" (atlas summary, "Approach"); the affine
+// recurrence h_t = a_t h_{t-1} + b_t is solved in one pass over time with
+// decoupled look-back between tiles.
+//
+// One cooperative launch runs every Newton iteration; one CTA of 512 threads
+// per SM walks tiles of (sequence b, 64 lanes, 64 steps), chunk-major.  A
+// tile's input pre-activations (3 gates) and guess rows h_{t0-1} .. h_{t0+63}
+// arrive by TMA in one of two shared-memory slots while the previous tile is
+// processed.  Thread (lane d, segment s) owns 8 consecutive steps of one lane:
+// it evaluates the cell and a_t, b_t (b_t = f_t - a_t h_{t-1}), composes its 8
+// maps, the 8 segments of a lane are chained through shared memory, the
+// tile's carry-in per lane comes from a cooperative look-back (8 threads per
+// lane), and every state is swept and stored with the convergence maxima
+// max |h^(i+1) - h^(i)| and max |h_t - f_t|.
+// Traffic per state and iteration: P (12 B), the guess (4 B), h^(i+1) (4 B).
+#include "common.cuh"
+#include "lookback.cuh"
+#include "solver.cuh"
+#include "tc_utils.cuh"
+
+namespace pararnn {
+namespace {
+using namespace tc;
+
+constexpr int TS = 64;          // steps per tile
+constexpr int DL = 64;          // lanes per tile
+constexpr int NT = 512;         // threads: lane x 8 segments
+constexpr int SEGS = NT / DL;   // 8 segments of 8 steps
+constexpr int SL = TS / SEGS;   // steps per thread
+constexpr int HALF = 32;        // lanes per 128-byte TMA box row
+constexpr int P_BOX = TS * 128;                // one (gate, half) box of P: 8 KB
+constexpr int H_BOX = 9 * 1024;                // one half of TS + 1 guess rows (8320 B), 1 KB aligned
+constexpr int SLOT = 6 * P_BOX + 2 * H_BOX;    // 66 KB
+constexpr int SLOT_TX = 6 * P_BOX + 2 * (TS + 1) * 128;
+constexpr int OFF_MISC = 2 * SLOT;
+// misc floats: segment maps 2 x SEGS x DL, carries DL, reduction 32
+constexpr int MISC_FLOATS = 2 * SEGS * DL + DL + 32;
+constexpr int SMEM_BYTES = OFF_MISC + MISC_FLOATS * 4 + 64 + 1024;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+
+struct Diag2Args {
+    DiagArgs a;
+    int ndg;            // lane groups per sequence (D / 64)
+    int ngroups;        // B * ndg: tiles per chunk
+    long long n_tiles;
+};
+
+// Byte offset of (row, lane k < 64) in a pair of 128-byte-swizzled boxes of
+// `box` bytes each (lanes 0..31 in the first, 32..63 in the second).
+__device__ __forceinline__ int sw_off(int row, int k, int box) {
+    const int hf = k >> 5, j = (k & 31) >> 2;
+    return hf * box + row * 128 + ((j ^ (row & 7)) << 4) + ((k & 3) << 2);
+}
+
+__device__ __forceinline__ void issue_fill(const CUtensorMap *mp, const CUtensorMap *mh,
+                                           unsigned char *slot, int D, long long row0, int lane0,
+                                           unsigned bar) {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // after the slot's last reads
+    mbar_expect_tx(bar, SLOT_TX);
+#pragma unroll
+    for (int g = 0; g < 3; ++g)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+            tma_load_2d(smem_u32(slot + (2 * g + hf) * P_BOX), mp, g * D + lane0 + hf * HALF,
+                        static_cast<int>(row0), bar);
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf)
+        tma_load_2d(smem_u32(slot + 6 * P_BOX + hf * H_BOX), mh, lane0 + hf * HALF,
+                    static_cast<int>(row0 - 1), bar);
+}
+
+__device__ __forceinline__ void tile_pos(const Diag2Args &S, long long tile, int T, int &chunk, int &b,
+                                         int &dg, long long &row0) {
+    chunk = static_cast<int>(tile / S.ngroups);
+    const int grp = static_cast<int>(tile % S.ngroups);
+    b = grp / S.ndg;
+    dg = grp % S.ndg;
+    row0 = static_cast<long long>(b) * T + static_cast<long long>(chunk) * TS;
+}
+
+__global__ void __launch_bounds__(NT, 1)
+diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ CUtensorMap map_h0,
+             const __grid_constant__ CUtensorMap map_h1, Diag2Args S) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    float *misc = reinterpret_cast<float *>(smem + OFF_MISC);
+    float *seg_a = misc;                   // [SEGS][DL] map of each 8-step segment
+    float *seg_b = seg_a + SEGS * DL;
+    float *carry = seg_b + SEGS * DL;      // [DL] tile carry-in
+    unsigned *red = reinterpret_cast<unsigned *>(carry + DL);  // [32]
+    unsigned long long *bars = reinterpret_cast<unsigned long long *>(red + 32);  // fill[2]
+    volatile int *cta_err = reinterpret_cast<volatile int *>(bars + 2);
+
+    const DiagArgs &A = S.a;
+    const int T = A.T, D = A.D;
+    WsHeader *hdr = A.hdr;
+    unsigned *status = &hdr->status;
+    const unsigned nblocks = gridDim.x;
+    const int tid = threadIdx.x;
+    const int d = tid & (DL - 1), seg = tid / DL;  // sweep role: lane, segment
+    const int ld = tid / SEGS, lq = tid % SEGS;     // look-back role: lane, rank
+
+    if (tid == 0) {
+        mbar_init(smem_u32(&bars[0]), 1);
+        mbar_init(smem_u32(&bars[1]), 1);
+        *cta_err = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    unsigned fill_par = 0u, fill_pending = 0u;
+    const long long my_n = blockIdx.x < S.n_tiles ? (S.n_tiles - blockIdx.x + nblocks - 1) / nblocks : 0;
+    int iters = 0, final_status = PARARNN_NOT_CONVERGED;
+    unsigned last_delta = 0u, last_resid = 0u;
+    for (int it = 0; it < A.max_iters; ++it) {
+        if (blockIdx.x == 0 && tid == 0) {
+            hdr->delta_bits[(it + 1) % 3] = 0u;
+            hdr->resid_bits[(it + 1) % 3] = 0u;
+        }
+        float *hnew = A.hbuf[(it + 1) & 1];
+        const CUtensorMap *mh = (it & 1) ? &map_h1 : &map_h0;
+        const unsigned epoch = static_cast<unsigned>(it + 1);
+        unsigned dmax = 0u, rmax = 0u;
+
+        if (tid == 0) {
+            for (int q = 0; q < 2 && q < my_n; ++q) {
+                int chunk, b, dg;
+                long long row0;
+                tile_pos(S, blockIdx.x + static_cast<long long>(q) * nblocks, T, chunk, b, dg, row0);
+                issue_fill(&map_p, mh, smem + q * SLOT, D, row0, dg * DL, smem_u32(&bars[q]));
+            }
+        }
+        fill_pending = my_n > 1 ? 3u : (my_n > 0 ? 1u : 0u);
+
+        for (long long k = 0; k < my_n; ++k) {
+            const long long tile = blockIdx.x + k * nblocks;
+            int chunk, b, dg;
+            long long row0;
+            tile_pos(S, tile, T, chunk, b, dg, row0);
+            const int t0 = chunk * TS, lane0 = dg * DL;
+            const int cur = static_cast<int>(k & 1);
+            const unsigned char *slot = smem + cur * SLOT;
+            const unsigned char *Hs = slot + 6 * P_BOX;
+            if (!mbar_wait(smem_u32(&bars[cur]), (fill_par >> cur) & 1u, cta_err)) *cta_err = 1;
+            fill_par ^= 1u << cur;
+            fill_pending &= ~(1u << cur);
+
+            // 1. cells of this thread's 8 steps
+            const int di = lane0 + d;
+            const float ur = __ldg(A.w_hh + di), uz = __ldg(A.w_hh + D + di), un = __ldg(A.w_hh + 2 * D + di);
+            const float br = __ldg(A.b_hh + di), bz = __ldg(A.b_hh + D + di), bn = __ldg(A.b_hh + 2 * D + di);
+            float av[SL], bv[SL], yv[SL];
+            float EA = 1.f, EB = 0.f;
+#pragma unroll
+            for (int i = 0; i < SL; ++i) {
+                const int s = seg * SL + i;
+                float hp = *reinterpret_cast<const float *>(Hs + sw_off(s, d, H_BOX));
+                if (t0 == 0 && s == 0) hp = __ldg(A.h0 + static_cast<size_t>(b) * D + di);
+                const float y = *reinterpret_cast<const float *>(Hs + sw_off(s + 1, d, H_BOX));
+                float a_ = 1.f, b_ = 0.f;
+                if (t0 + s < T) {
+                    const float pr = *reinterpret_cast<const float *>(slot + 0 * P_BOX + sw_off(s, d, P_BOX));
+                    const float pz = *reinterpret_cast<const float *>(slot + 2 * P_BOX + sw_off(s, d, P_BOX));
+                    const float pn = *reinterpret_cast<const float *>(slot + 4 * P_BOX + sw_off(s, d, P_BOX));
+                    float f;
+                    gru_cell_diag(pr, pz, pn, ur * hp, uz * hp, un * hp, br, bz, bn, ur, uz, un, hp, f, a_, b_);
+                    rmax = max(rmax, abs_bits(y - f));
+                }
+                av[i] = a_;
+                bv[i] = b_;
+                yv[i] = y;
+                EB = fmaf(a_, EB, b_);
+                EA = a_ * EA;
+            }
+            seg_a[seg * DL + d] = EA;
+            seg_b[seg * DL + d] = EB;
+            __syncthreads();
+            if (*cta_err != 0) break;  // uniform: read after the barrier
+
+            // 2. tile carry-in per lane (8 threads per lane)
+            {
+                float TA = 1.f, TB = 0.f;
+#pragma unroll
+                for (int q = 0; q < SEGS; ++q) {
+                    const float qa = seg_a[q * DL + ld], qb = seg_b[q * DL + ld];
+                    TB = fmaf(qa, TB, qb);
+                    TA = qa * TA;
+                }
+                const float c0 = chunk == 0 ? __ldg(A.h0 + static_cast<size_t>(b) * D + lane0 + ld) : 0.f;
+                const float hin =
+                    coop_lookback<SEGS>(A.desc, tile, S.ngroups, DL, ld, lq, epoch, TA, TB, chunk, c0, status);
+                if (lq == 0) carry[ld] = hin;
+            }
+            __syncthreads();
+
+            // 3. sweep: carry through the earlier segments, then this thread's steps
+            {
+                float h = carry[d];
+                for (int q = 0; q < seg; ++q) h = fmaf(seg_a[q * DL + d], h, seg_b[q * DL + d]);
+                float *out = hnew + static_cast<size_t>(row0) * D + di;
+#pragma unroll
+                for (int i = 0; i < SL; ++i) {
+                    const int s = seg * SL + i;
+                    h = fmaf(av[i], h, bv[i]);
+                    if (t0 + s < T) {
+                        __stcg(out + static_cast<size_t>(s) * D, h);
+                        dmax = max(dmax, abs_bits(h - yv[i]));
+                    }
+                }
+            }
+            __syncthreads();  // slot, segment maps and carries are rewritten next
+            if (k + 2 < my_n) {
+                if (tid == 0) {
+                    int c2, b2, dg2;
+                    long long r2;
+                    tile_pos(S, tile + 2 * static_cast<long long>(nblocks), T, c2, b2, dg2, r2);
+                    issue_fill(&map_p, mh, smem + cur * SLOT, D, r2, dg2 * DL, smem_u32(&bars[cur]));
+                }
+                fill_pending |= 1u << cur;
+            }
+        }
+        const unsigned bd = block_max_u32(dmax, red);
+        const unsigned br = block_max_u32(rmax, red);
+        if (tid == 0) {
+            atomicMax(&hdr->delta_bits[it % 3], bd);
+            atomicMax(&hdr->resid_bits[it % 3], br);
+            if (*cta_err) flag_timeout(status);
+        }
+        grid_barrier(hdr->barrier, nblocks, status);
+        last_delta = ld_acquire_u32(&hdr->delta_bits[it % 3]);
+        last_resid = ld_acquire_u32(&hdr->resid_bits[it % 3]);
+        iters = it + 1;
+        if (*cta_err || timed_out(status)) { final_status = PARARNN_TIMEOUT; break; }
+        if (last_delta >= 0x7f800000u) { final_status = PARARNN_DIVERGED; break; }
+        if (__uint_as_float(last_delta) <= A.tol) { final_status = PARARNN_OK; break; }
+    }
+    if ((iters & 1) == 0 && iters > 0) {
+        const size_t n4 = static_cast<size_t>(A.B) * A.T * A.D / 4;
+        const float4 *src = reinterpret_cast<const float4 *>(A.hbuf[0]);
+        float4 *dst = reinterpret_cast<float4 *>(A.hbuf[1]);
+        for (size_t q = static_cast<size_t>(blockIdx.x) * NT + tid; q < n4; q += static_cast<size_t>(nblocks) * NT)
+            dst[q] = __ldcg(src + q);
+    }
+    if (blockIdx.x == 0 && tid == 0) {
+        pararnn_info info;
+        info.iters = iters;
+        info.status = final_status;
+        info.delta = __uint_as_float(last_delta);
+        info.residual = __uint_as_float(last_resid);
+        *A.info_out = info;
+        hdr->info = info;
+    }
+    if (tid == 0)  // copies still in flight after a failed wait finish first
+        for (int q = 0; q < 2; ++q)
+            if ((fill_pending >> q) & 1u) mbar_drain(smem_u32(&bars[q]), (fill_par >> q) & 1u);
+}
+
+}  // namespace
+
+// The streaming path takes the diagonal cell with D a multiple of 64.
+bool diag2_supported(const pararnn_cell &cell, int B, int T) {
+    if (cell.kind != PARARNN_GRU_DIAG || cell.d % DL != 0) return false;
+    if (static_cast<long long>(B) * T >= (1ll << 31) - 1) return false;
+    return encode_fn() != nullptr;
+}
+
+// Look-back descriptors: tiles of 64 steps x 64 lanes, two words each.
+size_t diag2_desc_bytes(int B, int T, int D) {
+    const long long tiles = static_cast<long long>(B) * (D / DL) * ((T + TS - 1) / TS);
+    return static_cast<size_t>(tiles) * DL * 2 * 8;
+}
+
+cudaError_t launch_diag2(const DiagArgs &a, cudaStream_t s) {
+    Diag2Args S;
+    S.a = a;
+    S.ndg = a.D / DL;
+    S.ngroups = a.B * S.ndg;
+    S.n_tiles = static_cast<long long>(S.ngroups) * ((a.T + TS - 1) / TS);
+    CUtensorMap mp, m0, m1;
+    const long long rows = static_cast<long long>(a.B) * a.T;
+    if (!make_map(&mp, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.P, rows, 3 * a.D, HALF, TS) ||
+        !make_map(&m0, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.hbuf[0], rows, a.D, HALF, TS + 1) ||
+        !make_map(&m1, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.hbuf[1], rows, a.D, HALF, TS + 1))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(diag2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    int dev = 0, nsm = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, diag2_kernel, NT, SMEM_BYTES)) != cudaSuccess)
+        return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    long long grid = static_cast<long long>(per_sm) * nsm;
+    if (grid > S.n_tiles) grid = S.n_tiles;
+    void *params[] = {&mp, &m0, &m1, &S};
+    return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(diag2_kernel),
+                                       dim3(static_cast<unsigned>(grid)), dim3(NT), params, SMEM_BYTES, s);
+}
+
+}  // namespace pararnn

@@ -25,6 +25,9 @@ cudaError_t launch_dense_solver(const pararnn_cell &cell, int mode, const DiagAr
 size_t quasi_tc_desc_bytes(int B, int T, int D);
 bool quasi_tc_supported(const pararnn_cell &cell, int B, int T);
 cudaError_t launch_quasi_tc2(const DiagArgs &a, cudaStream_t s);
+bool diag2_supported(const pararnn_cell &cell, int B, int T);
+size_t diag2_desc_bytes(int B, int T, int D);
+cudaError_t launch_diag2(const DiagArgs &a, cudaStream_t s);
 cudaError_t launch_scan_dense(const float *A, const float *b, const float *h0, int B, int T,
                               int D, float *h, void *ws, cudaStream_t s);
 size_t scan_dense_ws_bytes(int B, int T, int D);
@@ -78,6 +81,11 @@ WsLayout ws_layout(const pararnn_cell &cell, int B, int T, int mode) {
             (cell.d == 32 || cell.d == 64)) {
             const size_t tc = quasi_tc_desc_bytes(B, T, cell.d);
             if (tc > desc) desc = tc;
+        }
+        // the streaming diagonal-cell path tiles by 64 steps x 64 lanes
+        if (cell.kind == PARARNN_GRU_DIAG && !is_elk(mode) && cell.d % 64 == 0) {
+            const size_t d2 = diag2_desc_bytes(B, T, cell.d);
+            if (d2 > desc) desc = d2;
         }
         off = align256(off + desc);
     }
@@ -167,6 +175,11 @@ static cudaError_t enqueue_iterate(const pararnn_cell *cell, const pararnn_param
         e = cudaMemsetAsync(a.hbuf[0], 0, states * sizeof(float), s);
         if (e != cudaSuccess) return e;
         return launch_quasi_tc2(a, s);
+    }
+    if (cell->kind == PARARNN_GRU_DIAG && !is_elk(mode) && diag2_supported(*cell, B, T)) {
+        e = cudaMemsetAsync(a.hbuf[0], 0, states * sizeof(float), s);
+        if (e != cudaSuccess) return e;
+        return launch_diag2(a, s);
     }
     return diag ? launch_diag_solver(*cell, mode, a, s)
                 : launch_dense_solver(*cell, mode, a, ws + L.dense, s);

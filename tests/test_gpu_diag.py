@@ -78,6 +78,7 @@ def test_affine_scan_closed_forms():
     ("tiny", dict(T=1000, bias_std=0.3, h0_std=0.5), "QUASI", 0.0),
     ("diag", dict(B=2, T=300, d=256, din=96, bias_std=0.3, h0_std=0.5), "QUASI", 0.0),
     ("diag", dict(B=2, T=130, d=100, din=40), "DEER", 0.0),
+    ("diag", dict(B=3, T=129, d=192, din=64, bias_std=0.3, h0_std=1.0), "DEER", 0.0),
     ("near_unstable", dict(B=2, T=600), "QUASI_ELK", 0.1),
     ("near_unstable", dict(B=2, T=333, d=32, din=16, h0_std=0.5), "QUASI_ELK", 1.0),
     ("diag", dict(B=2, T=260, d=64, din=64), "QUASI_ELK", 0.01),
@@ -109,6 +110,8 @@ def test_each_iteration_matches_oracle(name, over, mode, lam):
     ("untrained", dict(B=3, T=2049, bias_std=0.2, h0_std=0.5), "QUASI"),
     ("diag", dict(B=2, T=513, d=512, din=128), "QUASI"),
     ("diag", dict(B=1, T=100, d=68, din=20, h0_std=1.0), "DEER"),
+    ("diag", dict(B=5, T=1000, d=128, din=64, h0_std=1.0, bias_std=0.2), "DEER"),
+    ("diag", dict(B=2, T=1, d=64, din=32, h0_std=1.0), "QUASI"),
     ("near_unstable", dict(B=2, T=1000), "QUASI"),
 ])
 def test_converged_matches_rollout_and_counts(name, over, mode):
