@@ -8,14 +8,15 @@
 // recurrence h_t = a_t h_{t-1} + b_t is solved in one pass over time with
 // decoupled look-back between tiles.
 //
-// One cooperative launch runs every Newton iteration; one CTA of 512 threads
-// per SM walks tiles of (sequence b, 64 lanes, 64 steps), chunk-major.  A
-// tile's input pre-activations (3 gates) and guess rows h_{t0-1} .. h_{t0+63}
-// arrive by TMA in one of two shared-memory slots while the previous tile is
-// processed.  Thread (lane d, segment s) owns 8 consecutive steps of one lane:
-// it evaluates the cell and a_t, b_t (b_t = f_t - a_t h_{t-1}), composes its 8
-// maps, the 8 segments of a lane are chained through shared memory, the
-// tile's carry-in per lane comes from a cooperative look-back (8 threads per
+// One cooperative launch runs every Newton iteration; CTAs of 256 threads (two
+// or more per SM, so that one CTA's look-back wait overlaps another's cells)
+// walk tiles of (sequence b, 64 lanes, 32 steps), chunk-major.  A tile's input
+// pre-activations (3 gates) and guess rows h_{t0-1} .. h_{t0+31} arrive by TMA
+// in one of two shared-memory slots while the previous tile is processed.
+// Thread (lane d, segment s) owns 8 consecutive steps of one lane: it
+// evaluates the cell and a_t, b_t (b_t = f_t - a_t h_{t-1}), composes its 8
+// maps, the 4 segments of a lane are chained through shared memory, the
+// tile's carry-in per lane comes from a cooperative look-back (4 threads per
 // lane), and every state is swept and stored with the convergence maxima
 // max |h^(i+1) - h^(i)| and max |h_t - f_t|.
 // Traffic per state and iteration: P (12 B), the guess (4 B), h^(i+1) (4 B).
@@ -28,15 +29,15 @@ namespace pararnn {
 namespace {
 using namespace tc;
 
-constexpr int TS = 64;          // steps per tile
+constexpr int TS = 32;          // steps per tile
 constexpr int DL = 64;          // lanes per tile
-constexpr int NT = 512;         // threads: lane x 8 segments
-constexpr int SEGS = NT / DL;   // 8 segments of 8 steps
+constexpr int NT = 256;         // threads: lane x 4 segments
+constexpr int SEGS = NT / DL;   // 4 segments of 8 steps
 constexpr int SL = TS / SEGS;   // steps per thread
 constexpr int HALF = 32;        // lanes per 128-byte TMA box row
-constexpr int P_BOX = TS * 128;                // one (gate, half) box of P: 8 KB
-constexpr int H_BOX = 9 * 1024;                // one half of TS + 1 guess rows (8320 B), 1 KB aligned
-constexpr int SLOT = 6 * P_BOX + 2 * H_BOX;    // 66 KB
+constexpr int P_BOX = TS * 128;                // one (gate, half) box of P: 4 KB
+constexpr int H_BOX = ((TS + 1) * 128 + 1023) / 1024 * 1024;  // one half of TS + 1 guess rows, 1 KB aligned
+constexpr int SLOT = 6 * P_BOX + 2 * H_BOX;    // 34 KB
 constexpr int SLOT_TX = 6 * P_BOX + 2 * (TS + 1) * 128;
 constexpr int OFF_MISC = 2 * SLOT;
 // misc floats: segment maps 2 x SEGS x DL, carries DL, reduction 32
@@ -84,7 +85,7 @@ __device__ __forceinline__ void tile_pos(const Diag2Args &S, long long tile, int
     row0 = static_cast<long long>(b) * T + static_cast<long long>(chunk) * TS;
 }
 
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NT, 3)
 diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ CUtensorMap map_h0,
              const __grid_constant__ CUtensorMap map_h1, Diag2Args S) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -156,7 +157,7 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
             const int di = lane0 + d;
             const float ur = __ldg(A.w_hh + di), uz = __ldg(A.w_hh + D + di), un = __ldg(A.w_hh + 2 * D + di);
             const float br = __ldg(A.b_hh + di), bz = __ldg(A.b_hh + D + di), bn = __ldg(A.b_hh + 2 * D + di);
-            float av[SL], bv[SL], yv[SL];
+            float av[SL], bv[SL];
             float EA = 1.f, EB = 0.f;
 #pragma unroll
             for (int i = 0; i < SL; ++i) {
@@ -175,7 +176,6 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
                 }
                 av[i] = a_;
                 bv[i] = b_;
-                yv[i] = y;
                 EB = fmaf(a_, EB, b_);
                 EA = a_ * EA;
             }
@@ -211,7 +211,8 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
                     h = fmaf(av[i], h, bv[i]);
                     if (t0 + s < T) {
                         __stcg(out + static_cast<size_t>(s) * D, h);
-                        dmax = max(dmax, abs_bits(h - yv[i]));
+                        const float y = *reinterpret_cast<const float *>(Hs + sw_off(s + 1, d, H_BOX));
+                        dmax = max(dmax, abs_bits(h - y));
                     }
                 }
             }
@@ -271,7 +272,7 @@ bool diag2_supported(const pararnn_cell &cell, int B, int T) {
     return encode_fn() != nullptr;
 }
 
-// Look-back descriptors: tiles of 64 steps x 64 lanes, two words each.
+// Look-back descriptors: tiles of 32 steps x 64 lanes, two words each.
 size_t diag2_desc_bytes(int B, int T, int D) {
     const long long tiles = static_cast<long long>(B) * (D / DL) * ((T + TS - 1) / TS);
     return static_cast<size_t>(tiles) * DL * 2 * 8;

@@ -82,7 +82,7 @@ WsLayout ws_layout(const pararnn_cell &cell, int B, int T, int mode) {
             const size_t tc = quasi_tc_desc_bytes(B, T, cell.d);
             if (tc > desc) desc = tc;
         }
-        // the streaming diagonal-cell path tiles by 64 steps x 64 lanes
+        // the streaming diagonal-cell path tiles by 32 steps x 64 lanes
         if (cell.kind == PARARNN_GRU_DIAG && !is_elk(mode) && cell.d % 64 == 0) {
             const size_t d2 = diag2_desc_bytes(B, T, cell.d);
             if (d2 > desc) desc = d2;
