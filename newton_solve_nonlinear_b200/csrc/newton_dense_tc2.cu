@@ -208,9 +208,10 @@ __device__ __forceinline__ void issue_mma(unsigned tmem, unsigned acc, unsigned 
 // clamped to the sequence) into L2 ahead of use.
 template <int D>
 __device__ __forceinline__ void prefetch_p(const float *P, long long tile, int B, int T) {
-    const int t0 = static_cast<int>(tile / B) * TM;
+    const int c = static_cast<int>(static_cast<unsigned>(tile) / static_cast<unsigned>(B));
+    const int t0 = c * TM;
     const int n = min(TM, T - t0);
-    const float *src = P + (static_cast<size_t>(tile % B) * T + t0) * 3 * D;
+    const float *src = P + (static_cast<size_t>(static_cast<int>(tile) - c * B) * T + t0) * 3 * D;
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(n * 3 * D * 4) : "memory");
 }
 
@@ -297,7 +298,8 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
         blockIdx.x < S.n_tiles ? (S.n_tiles - blockIdx.x + nblocks - 1) / nblocks : 0;
     auto tile_of = [&](long long k) { return static_cast<long long>(blockIdx.x) + k * nblocks; };
     auto row0_of = [&](long long tile) {
-        return static_cast<long long>(tile % B) * T + static_cast<long long>(tile / B) * TM;
+        const int c = static_cast<int>(static_cast<unsigned>(tile) / static_cast<unsigned>(B));
+        return static_cast<long long>(static_cast<int>(tile) - c * B) * T + static_cast<long long>(c) * TM;
     };
 
     int iters = 0, final_status = PARARNN_NOT_CONVERGED;
@@ -325,7 +327,8 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
             fill_par ^= 1u;
             fill_pending &= ~1u;
             const long long t0t = tile_of(0);
-            write_a<D>(slots, tmem, A.h0 + static_cast<size_t>(t0t % B) * D, t0t / B == 0, warp, lane);
+            write_a<D>(slots, tmem, A.h0 + static_cast<size_t>(static_cast<int>(t0t) % B) * D,
+                       static_cast<int>(t0t) < B, warp, lane);
             asm volatile("tcgen05.fence::before_thread_sync;");
             __syncthreads();
             if (tid == 0) {
@@ -337,7 +340,9 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
 
         for (long long k = 0; k < my_n; ++k) {
             const long long tile = tile_of(k);
-            const int chunk = static_cast<int>(tile / B), b = static_cast<int>(tile % B);
+            // tile < 2^31 (B*T < 2^31 is required): 32-bit arithmetic
+            const int chunk = static_cast<int>(static_cast<unsigned>(tile) / static_cast<unsigned>(B));
+            const int b = static_cast<int>(tile) - chunk * B;
             const int t0 = chunk * TM;
             const long long row0 = static_cast<long long>(b) * T + t0;
             const int cur = static_cast<int>(k & 1);
@@ -373,8 +378,8 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
                 fill_par ^= 1u << nxt;
                 fill_pending &= ~(1u << nxt);
                 const long long tn = tile_of(k + 1);
-                write_a<D>(slots + nxt * G::SLOT_BYTES, tmem, A.h0 + static_cast<size_t>(tn % B) * D,
-                           tn / B == 0, warp, lane);
+                write_a<D>(slots + nxt * G::SLOT_BYTES, tmem, A.h0 + static_cast<size_t>(static_cast<int>(tn) % B) * D,
+                           static_cast<int>(tn) < B, warp, lane);
                 asm volatile("tcgen05.fence::before_thread_sync;");
             }
             __syncthreads();

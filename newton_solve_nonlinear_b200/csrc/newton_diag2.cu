@@ -76,12 +76,14 @@ __device__ __forceinline__ void issue_fill(const CUtensorMap *mp, const CUtensor
                     static_cast<int>(row0 - 1), bar);
 }
 
+// Tile indices stay below 2^31 (n_tiles <= B*T*D / 2048): 32-bit arithmetic.
 __device__ __forceinline__ void tile_pos(const Diag2Args &S, long long tile, int T, int &chunk, int &b,
                                          int &dg, long long &row0) {
-    chunk = static_cast<int>(tile / S.ngroups);
-    const int grp = static_cast<int>(tile % S.ngroups);
-    b = grp / S.ndg;
-    dg = grp % S.ndg;
+    const unsigned t32 = static_cast<unsigned>(tile), ng = static_cast<unsigned>(S.ngroups);
+    chunk = static_cast<int>(t32 / ng);
+    const unsigned grp = t32 - static_cast<unsigned>(chunk) * ng;
+    b = static_cast<int>(grp / static_cast<unsigned>(S.ndg));
+    dg = static_cast<int>(grp) - b * S.ndg;
     row0 = static_cast<long long>(b) * T + static_cast<long long>(chunk) * TS;
 }
 
@@ -107,6 +109,7 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
     const int tid = threadIdx.x;
     const int d = tid & (DL - 1), seg = tid / DL;  // sweep role: lane, segment
     const int ld = tid / SEGS, lq = tid % SEGS;     // look-back role: lane, rank
+    const int jq = (d & 31) >> 2;                   // 16-byte chunk of lane d in a 128-byte row
 
     if (tid == 0) {
         mbar_init(smem_u32(&bars[0]), 1);
@@ -157,19 +160,25 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
             const int di = lane0 + d;
             const float ur = __ldg(A.w_hh + di), uz = __ldg(A.w_hh + D + di), un = __ldg(A.w_hh + 2 * D + di);
             const float br = __ldg(A.b_hh + di), bz = __ldg(A.b_hh + D + di), bn = __ldg(A.b_hh + 2 * D + di);
+            // a thread's rows start at a multiple of 8, so the swizzle of row
+            // seg*SL + i is the constant i: lane offsets are hoisted out of the loop
+            const unsigned char *Pt = slot + (d >> 5) * P_BOX + seg * SL * 128 + (d & 3) * 4;
+            const unsigned char *Ht = Hs + (d >> 5) * H_BOX + seg * SL * 128 + (d & 3) * 4;
+            const bool full = t0 + TS <= T;
             float av[SL], bv[SL];
             float EA = 1.f, EB = 0.f;
+            float hp = *reinterpret_cast<const float *>(Ht + (jq << 4));
+            if (t0 == 0 && seg == 0) hp = __ldg(A.h0 + static_cast<size_t>(b) * D + di);
 #pragma unroll
             for (int i = 0; i < SL; ++i) {
-                const int s = seg * SL + i;
-                float hp = *reinterpret_cast<const float *>(Hs + sw_off(s, d, H_BOX));
-                if (t0 == 0 && s == 0) hp = __ldg(A.h0 + static_cast<size_t>(b) * D + di);
-                const float y = *reinterpret_cast<const float *>(Hs + sw_off(s + 1, d, H_BOX));
+                const int o = i * 128 + ((jq ^ i) << 4);
+                const int oy = (i + 1) * 128 + ((jq ^ ((i + 1) & 7)) << 4);
+                const float y = *reinterpret_cast<const float *>(Ht + oy);
                 float a_ = 1.f, b_ = 0.f;
-                if (t0 + s < T) {
-                    const float pr = *reinterpret_cast<const float *>(slot + 0 * P_BOX + sw_off(s, d, P_BOX));
-                    const float pz = *reinterpret_cast<const float *>(slot + 2 * P_BOX + sw_off(s, d, P_BOX));
-                    const float pn = *reinterpret_cast<const float *>(slot + 4 * P_BOX + sw_off(s, d, P_BOX));
+                if (full || t0 + seg * SL + i < T) {
+                    const float pr = *reinterpret_cast<const float *>(Pt + 0 * P_BOX + o);
+                    const float pz = *reinterpret_cast<const float *>(Pt + 2 * P_BOX + o);
+                    const float pn = *reinterpret_cast<const float *>(Pt + 4 * P_BOX + o);
                     float f;
                     gru_cell_diag(pr, pz, pn, ur * hp, uz * hp, un * hp, br, bz, bn, ur, uz, un, hp, f, a_, b_);
                     rmax = max(rmax, abs_bits(y - f));
@@ -178,6 +187,7 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
                 bv[i] = b_;
                 EB = fmaf(a_, EB, b_);
                 EA = a_ * EA;
+                hp = y;
             }
             seg_a[seg * DL + d] = EA;
             seg_b[seg * DL + d] = EB;
@@ -205,13 +215,14 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
                 float h = carry[d];
                 for (int q = 0; q < seg; ++q) h = fmaf(seg_a[q * DL + d], h, seg_b[q * DL + d]);
                 float *out = hnew + static_cast<size_t>(row0) * D + di;
+                out += static_cast<size_t>(seg) * SL * D;
 #pragma unroll
                 for (int i = 0; i < SL; ++i) {
-                    const int s = seg * SL + i;
                     h = fmaf(av[i], h, bv[i]);
-                    if (t0 + s < T) {
-                        __stcg(out + static_cast<size_t>(s) * D, h);
-                        const float y = *reinterpret_cast<const float *>(Hs + sw_off(s + 1, d, H_BOX));
+                    if (full || t0 + seg * SL + i < T) {
+                        __stcg(out + static_cast<size_t>(i) * D, h);
+                        const int oy = (i + 1) * 128 + ((jq ^ ((i + 1) & 7)) << 4);
+                        const float y = *reinterpret_cast<const float *>(Ht + oy);
                         dmax = max(dmax, abs_bits(h - y));
                     }
                 }
