@@ -127,12 +127,18 @@ __device__ __forceinline__ float lookback_affine(unsigned long long *desc, long 
 struct Mob {
     float m0, m1, m2, m3;
 };
-__device__ __forceinline__ Mob mob_mul(const Mob &x, const Mob &y) {  // x * y (apply y first)
+// x * y (apply y first).  A Moebius map does not change when its matrix is
+// scaled, so the product is rescaled by the power of two that brings its
+// largest entry into [1, 2): exact, and it keeps long products in range.
+__device__ __forceinline__ Mob mob_mul(const Mob &x, const Mob &y) {
     Mob r{x.m0 * y.m0 + x.m1 * y.m2, x.m0 * y.m1 + x.m1 * y.m3,
           x.m2 * y.m0 + x.m3 * y.m2, x.m2 * y.m1 + x.m3 * y.m3};
     const float s = fmaxf(fmaxf(fabsf(r.m0), fabsf(r.m1)), fmaxf(fabsf(r.m2), fabsf(r.m3)));
-    const float inv = s > 0.f ? 1.f / s : 1.f;
-    r.m0 *= inv; r.m1 *= inv; r.m2 *= inv; r.m3 *= inv;
+    const int e = (__float_as_int(s) >> 23) & 0xff;  // biased exponent of the largest entry
+    if (e > 0 && e < 255) {
+        const float sc = __int_as_float((254 - e) << 23);  // 2^(127 - e)
+        r.m0 *= sc; r.m1 *= sc; r.m2 *= sc; r.m3 *= sc;
+    }
     return r;
 }
 __device__ __forceinline__ float mob_apply(const Mob &x, float P) {
@@ -207,16 +213,16 @@ __device__ __forceinline__ float lookback_mobius(unsigned long long *desc, long 
 // Cooperative decoupled look-back for lane d, shared by G threads of one
 // lane group (G consecutive lanes of a warp, G a power of two <= 32; q = rank
 // in the group; every lane of the warp calls it).  Descriptors are laid out
-// [tile][DG lanes][2 words].  The
-// group reads the descriptors of G predecessors at once (thread q: the
-// (q+1)-th tile back), finds the nearest one that holds an inclusive value,
-// and composes the aggregates in front of it with an ordered shuffle
-// reduction; windows repeat until an inclusive value is reached (the chunk-0
-// tile always publishes one).  Thread q = 0 publishes the tile's aggregate
-// first and its inclusive value last.  Returns the carry into the tile
-// (carry0 for a sequence's first chunk).  Waits are bounded: a descriptor
-// that never arrives reads as an inclusive 0 and raises the timeout flag.
-template <int G>
+// [tile][DG lanes][2 words].  The group reads R x G predecessors per round
+// trip (thread q: tiles q R + 1 .. q R + R back), finds the nearest one that
+// holds an inclusive value, and composes the aggregates in front of it (first
+// serially inside a thread, then with an ordered shuffle reduction); windows
+// repeat until an inclusive value is reached (the chunk-0 tile always
+// publishes one).  Thread q = 0 publishes the tile's aggregate first and its
+// inclusive value last.  Returns the carry into the tile (carry0 when there
+// is no predecessor).  Waits are bounded: a descriptor that never arrives
+// reads as an inclusive 0 and raises the timeout flag.
+template <int G, int R = 1>
 __device__ __forceinline__ float coop_lookback(unsigned long long *desc, long long tile, long long step,
                                                int DG, int d, int q, unsigned epoch, float EA, float EB,
                                                int avail, float carry0, unsigned *status) {
@@ -233,33 +239,49 @@ __device__ __forceinline__ float coop_lookback(unsigned long long *desc, long lo
         }
         float accA = 1.f, accB = 0.f;
         bool done = false;
-        for (int base = 0;; base += G) {
-            const int p = base + q;
+        for (int base = 0;; base += G * R) {
+            // this thread's R predecessors, nearest first: map = m_0 o m_1 o ... up to
+            // (not including) the first inclusive value
+            unsigned long long wa[R], wb[R];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const int p = base + q * R + r;
+                wa[r] = wb[r] = 0ull;
+                if (!done && p < avail) {
+                    const unsigned long long *pp = desc + (static_cast<size_t>(tile - (p + 1) * step) * DG + d) * 2;
+                    wa[r] = ld_relaxed(pp);
+                    wb[r] = ld_relaxed(pp + 1);
+                }
+            }
             float ma = 1.f, mb = 0.f, iv = 0.f;
             bool inc = false;
-            if (!done && p < avail) {
-                const unsigned long long *pp = desc + (static_cast<size_t>(tile - (p + 1) * step) * DG + d) * 2;
-                unsigned long long a = ld_relaxed(pp);
-                if (!word_ready(a, epoch)) a = wait_ready(pp, epoch, status);
-                if (a == 0ull) {
-                    inc = true;
-                } else if ((word_tag(a) & 3u) == kStateInc) {
-                    inc = true;
-                    iv = word_val(a);
-                } else {
-                    unsigned long long bw = ld_relaxed(pp + 1);
-                    if (word_tag(bw) != word_tag(a)) bw = wait_tag(pp + 1, word_tag(a), status);
-                    if (bw == 0ull) {
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const int p = base + q * R + r;
+                if (!done && !inc && p < avail) {
+                    const unsigned long long *pp = desc + (static_cast<size_t>(tile - (p + 1) * step) * DG + d) * 2;
+                    unsigned long long a = wa[r];
+                    if (!word_ready(a, epoch)) a = wait_ready(pp, epoch, status);
+                    if (a == 0ull) {
                         inc = true;
+                    } else if ((word_tag(a) & 3u) == kStateInc) {
+                        inc = true;
+                        iv = word_val(a);
                     } else {
-                        ma = word_val(a);
-                        mb = word_val(bw);
+                        unsigned long long bw = wb[r];
+                        if (word_tag(bw) != word_tag(a)) bw = wait_tag(pp + 1, word_tag(a), status);
+                        if (bw == 0ull) {
+                            inc = true;
+                        } else {  // map := map o (a, b)
+                            mb = fmaf(ma, word_val(bw), mb);
+                            ma = ma * word_val(a);
+                        }
                     }
                 }
             }
             const unsigned incm = (__ballot_sync(0xffffffffu, inc) & gmask) >> gbase;
-            const int k = incm ? __ffs(incm) - 1 : G;  // nearest inclusive in this window
-            if (q >= k) {
+            const int k = incm ? __ffs(incm) - 1 : G;  // nearest thread holding an inclusive value
+            if (q > k) {
                 ma = 1.f;
                 mb = 0.f;
             }
@@ -290,5 +312,101 @@ __device__ __forceinline__ float coop_lookback(unsigned long long *desc, long lo
     return hin;
 }
 
+// The same for Moebius maps (descriptors [tile][DG lanes][4 words]); returns
+// the covariance entering the tile.
+template <int G, int R = 1>
+__device__ __forceinline__ float coop_lookback_mob(unsigned long long *desc, long long tile, long long step,
+                                                   int DG, int d, int q, unsigned epoch, const Mob &E,
+                                                   int avail, float carry0, unsigned *status) {
+    unsigned long long *mine = desc + (static_cast<size_t>(tile) * DG + d) * 4;
+    const int lane = threadIdx.x & 31;
+    const int gbase = lane & ~(G - 1);
+    const unsigned gmask = G == 32 ? 0xffffffffu : (((1u << G) - 1u) << gbase);
+    float pin = carry0;
+    if (avail > 0) {
+        if (q == 0) {
+            const unsigned tg = make_tag(epoch, kStateAgg);
+            st_relaxed(mine + 1, pack_word(tg, E.m1));
+            st_relaxed(mine + 2, pack_word(tg, E.m2));
+            st_relaxed(mine + 3, pack_word(tg, E.m3));
+            st_relaxed(mine, pack_word(tg, E.m0));
+        }
+        Mob acc{1.f, 0.f, 0.f, 1.f};
+        bool done = false;
+        for (int base = 0;; base += G * R) {
+            unsigned long long w[R][4];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const int p = base + q * R + r;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) w[r][e] = 0ull;
+                if (!done && p < avail) {
+                    const unsigned long long *pp = desc + (static_cast<size_t>(tile - (p + 1) * step) * DG + d) * 4;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) w[r][e] = ld_relaxed(pp + e);
+                }
+            }
+            Mob mm{1.f, 0.f, 0.f, 1.f};
+            float iv = 0.f;
+            bool inc = false;
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                const int p = base + q * R + r;
+                if (!done && !inc && p < avail) {
+                    const unsigned long long *pp = desc + (static_cast<size_t>(tile - (p + 1) * step) * DG + d) * 4;
+                    unsigned long long a = w[r][0];
+                    if (!word_ready(a, epoch)) a = wait_ready(pp, epoch, status);
+                    if (a == 0ull) {
+                        inc = true;
+                    } else if ((word_tag(a) & 3u) == kStateInc) {
+                        inc = true;
+                        iv = word_val(a);
+                    } else {
+                        float m[3];
+                        bool ok = true;
+#pragma unroll
+                        for (int e = 1; e < 4; ++e) {
+                            unsigned long long v = w[r][e];
+                            if (word_tag(v) != word_tag(a)) v = wait_tag(pp + e, word_tag(a), status);
+                            if (v == 0ull) ok = false;
+                            m[e - 1] = word_val(v);
+                        }
+                        if (!ok)
+                            inc = true;
+                        else
+                            mm = mob_mul(mm, Mob{word_val(a), m[0], m[1], m[2]});
+                    }
+                }
+            }
+            const unsigned incm = (__ballot_sync(0xffffffffu, inc) & gmask) >> gbase;
+            const int k = incm ? __ffs(incm) - 1 : G;
+            if (q > k) mm = Mob{1.f, 0.f, 0.f, 1.f};
+#pragma unroll
+            for (int o = 1; o < G; o <<= 1) {
+                Mob n;
+                n.m0 = __shfl_down_sync(0xffffffffu, mm.m0, o);
+                n.m1 = __shfl_down_sync(0xffffffffu, mm.m1, o);
+                n.m2 = __shfl_down_sync(0xffffffffu, mm.m2, o);
+                n.m3 = __shfl_down_sync(0xffffffffu, mm.m3, o);
+                if ((q & (2 * o - 1)) == 0) mm = mob_mul(mm, n);
+            }
+            mm.m0 = __shfl_sync(0xffffffffu, mm.m0, gbase);
+            mm.m1 = __shfl_sync(0xffffffffu, mm.m1, gbase);
+            mm.m2 = __shfl_sync(0xffffffffu, mm.m2, gbase);
+            mm.m3 = __shfl_sync(0xffffffffu, mm.m3, gbase);
+            const float kv = __shfl_sync(0xffffffffu, iv, gbase + (k < G ? k : 0));
+            if (!done) {
+                acc = mob_mul(acc, mm);
+                if (k < G) {
+                    pin = mob_apply(acc, kv);
+                    done = true;
+                }
+            }
+            if (__all_sync(0xffffffffu, done)) break;
+        }
+    }
+    if (q == 0) st_relaxed(mine, pack_word(make_tag(epoch, kStateInc), mob_apply(E, pin)));
+    return pin;
+}
 
 }  // namespace pararnn

@@ -73,8 +73,10 @@ struct Tc2Geom {
     static constexpr int OFF_BLO = B_BYTES;
     static constexpr int OFF_SLOT = 2 * B_BYTES;
     static constexpr int OFF_MISC = OFF_SLOT + 2 * SLOT_BYTES;
-    // misc floats: b_hh 3D, diag U 3D, warp-quarter totals 2 x 4D, carries D, reduction 32
-    static constexpr int MISC_FLOATS = 6 * D + 8 * D + D + 32;
+    // misc floats: b_hh 3D, diag U 3D, warp-quarter totals 2 x 4D, carries D, reduction 32,
+    // quasi-ELK segment maps (Moebius 4 + affine 2 per thread) and two carries per lane
+    static constexpr int ELK_FLOATS = 6 * NTHREADS + 2 * D;
+    static constexpr int MISC_FLOATS = 6 * D + 8 * D + D + 32 + 16 + ELK_FLOATS;  // 16: barriers, TMEM slot, flag
     static constexpr int SMEM_BYTES = OFF_MISC + MISC_FLOATS * 4 + 64 + 1024;
     static_assert(D == 32 || D == 64, "tensor-core cell path takes D = 32 or 64");
     static_assert(A_LO + 64 <= TMEM_COLS, "TMEM columns");
@@ -215,6 +217,222 @@ __device__ __forceinline__ void prefetch_p(const float *P, long long tile, int B
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(n * 3 * D * 4) : "memory");
 }
 
+// ---- quasi-ELK (the damped step as a scalar Kalman filter + RTS smoother per
+// lane; "Towards Scalable and Stable Parallelization of Nonlinear RNNs",
+// atlas summary "Approach": quasi-ELK) ------------------------------------------
+// With the linearisation a_t, b_t at the guess y = h^(i), process noise 1 and
+// observation noise 1 / lambda:
+//   filter   P-_t = a_t^2 P_{t-1} + 1,  K_t = lambda P-_t / (1 + lambda P-_t),
+//            P_t = P-_t / (1 + lambda P-_t)  (so K_t = lambda P_t),
+//            m_t = (1 - K_t)(a_t m_{t-1} + b_t) + K_t y_t,  m_0 = h0, P_0 = 0;
+//   smoother s_t = G_t s_{t+1} + (m_t - G_t (a_{t+1} m_t + b_{t+1})),
+//            G_t = P_t a_{t+1} / P-_{t+1},  s_T = m_T;  h^(i+1) = s.
+// The covariance step is the Moebius map [[a^2, 1], [lambda a^2, 1 + lambda]].
+// Inside a tile, thread (lane d, segment g) walks SLE consecutive steps; the
+// segments of a lane are chained through shared memory and tiles through
+// look-back (covariance, mean forward; smoother backward).
+
+constexpr int kElkWin = 3;  // predecessors each look-back thread reads per round trip
+
+struct ElkSmem {
+    float *mob;   // [SEGS][D][4] segment Moebius maps, then exclusive prefixes
+    float *aff;   // [SEGS][D][2] segment affine maps, then exclusive prefixes
+    float *cP;    // [D] covariance entering the tile
+    float *cM;    // [D] mean entering the tile (smoother: state after the tile)
+};
+
+// Forward scans of one tile: a_t, b_t of the tile are in A.elk_a / elk_b
+// (written by this CTA), the guess rows in `slot`.  Writes m_t and P_t.
+template <int D>
+__device__ void elk_forward_scans(const DiagArgs &A, const ElkSmem &E, const unsigned char *slot,
+                                  long long tile, int chunk, int b, int t0, long long row0,
+                                  unsigned epoch, unsigned long long *desc_cov,
+                                  unsigned long long *desc_mean, unsigned *status) {
+    using G = Tc2Geom<D>;
+    constexpr int SEGS = NTHREADS / D, SLE = TM / SEGS;
+    const int T = A.T, B = A.B;
+    const float lam = A.lambda;
+    const int tid = threadIdx.x, d = tid % D, g = tid / D, s0 = g * SLE;
+    // (i) covariance maps of the thread's steps
+    float ak[SLE];
+    Mob M{1.f, 0.f, 0.f, 1.f};
+#pragma unroll
+    for (int i = 0; i < SLE; ++i) {
+        const bool valid = t0 + s0 + i < T;
+        ak[i] = valid ? __ldcg(A.elk_a + (static_cast<size_t>(row0) + s0 + i) * D + d) : 1.f;
+        if (valid) {
+            const float a2 = ak[i] * ak[i];
+            M = mob_mul(Mob{a2, 1.f, lam * a2, 1.f + lam}, M);
+        }
+    }
+    {
+        float *mm = E.mob + (g * D + d) * 4;
+        mm[0] = M.m0; mm[1] = M.m1; mm[2] = M.m2; mm[3] = M.m3;
+    }
+    __syncthreads();
+    {  // covariance entering the tile: all threads, SEGS per lane
+        const int ld = tid / SEGS, lq = tid % SEGS;
+        Mob Ex{1.f, 0.f, 0.f, 1.f};
+        for (int q = 0; q < SEGS; ++q) {
+            const float *qm = E.mob + (q * D + ld) * 4;
+            Ex = mob_mul(Mob{qm[0], qm[1], qm[2], qm[3]}, Ex);
+        }
+        const float pin = coop_lookback_mob<SEGS, kElkWin>(desc_cov, tile, B, D, ld, lq, epoch, Ex, chunk,
+                                                           0.f, status);
+        if (lq == 0) E.cP[ld] = pin;
+    }
+    __syncthreads();
+    // (ii) covariances, gains and the mean's affine maps
+    float Pk[SLE];
+    {
+        Mob X{1.f, 0.f, 0.f, 1.f};  // this segment's exclusive prefix
+        for (int q = 0; q < g; ++q) {
+            const float *qm = E.mob + (q * D + d) * 4;
+            X = mob_mul(Mob{qm[0], qm[1], qm[2], qm[3]}, X);
+        }
+        float P = mob_apply(X, E.cP[d]);
+        float SA = 1.f, SB = 0.f;
+#pragma unroll
+        for (int i = 0; i < SLE; ++i) {
+            const int s = s0 + i;
+            float alpha = 1.f, beta = 0.f;
+            if (t0 + s < T) {
+                const float Pm = fmaf(ak[i] * ak[i], P, 1.f);
+                P = __fdividef(Pm, fmaf(lam, Pm, 1.f));
+                const float K = lam * P, omk = 1.f - K;
+                const float bt = __ldcg(A.elk_b + (static_cast<size_t>(row0) + s) * D + d);
+                const float y = *reinterpret_cast<const float *>(slot + sw_off(s + 1, d, G::SLOT_HALF));
+                alpha = omk * ak[i];
+                beta = fmaf(omk, bt, K * y);
+            }
+            Pk[i] = P;
+            SB = fmaf(alpha, SB, beta);
+            SA = alpha * SA;
+        }
+        float *fa = E.aff + (g * D + d) * 2;
+        fa[0] = SA;
+        fa[1] = SB;
+    }
+    __syncthreads();
+    {  // mean entering the tile
+        const int ld = tid / SEGS, lq = tid % SEGS;
+        float EA = 1.f, EB = 0.f;
+        for (int q = 0; q < SEGS; ++q) {
+            const float *qa = E.aff + (q * D + ld) * 2;
+            EB = fmaf(qa[0], EB, qa[1]);
+            EA = qa[0] * EA;
+        }
+        const float c0 = chunk == 0 ? __ldg(A.h0 + static_cast<size_t>(b) * D + ld) : 0.f;
+        const float min_ = coop_lookback<SEGS, kElkWin>(desc_mean, tile, B, D, ld, lq, epoch, EA, EB, chunk,
+                                                        c0, status);
+        if (lq == 0) E.cM[ld] = min_;
+    }
+    __syncthreads();
+    // (iii) filtered means and covariances of the thread's steps
+    {
+        float m = E.cM[d];
+        for (int q = 0; q < g; ++q) {
+            const float *qa = E.aff + (q * D + d) * 2;
+            m = fmaf(qa[0], m, qa[1]);
+        }
+#pragma unroll
+        for (int i = 0; i < SLE; ++i) {
+            const int s = s0 + i;
+            if (t0 + s < T) {  // the gain-weighted map again: K_t = lambda P_t
+                const size_t o = (static_cast<size_t>(row0) + s) * D + d;
+                const float K = lam * Pk[i], omk = 1.f - K;
+                const float bt = __ldcg(A.elk_b + o);
+                const float y = *reinterpret_cast<const float *>(slot + sw_off(s + 1, d, G::SLOT_HALF));
+                m = fmaf(omk * ak[i], m, fmaf(omk, bt, K * y));
+                __stcg(A.elk_m + o, m);
+                __stcg(A.elk_p + o, Pk[i]);
+            }
+        }
+    }
+}
+
+// Smoother over one tile (tiles visited in reverse chunk order): h^(i+1) and
+// max |h^(i+1) - h^(i)|.
+template <int D>
+__device__ void elk_backward_tile(const DiagArgs &A, const ElkSmem &E, long long tile, int chunk, int b,
+                                  int n_chunks, unsigned epoch, unsigned long long *desc_bwd,
+                                  const float *hold, float *hnew, unsigned &dmax, unsigned *status) {
+    constexpr int SEGS = NTHREADS / D, SLE = TM / SEGS;
+    const int T = A.T, B = A.B;
+    const int tid = threadIdx.x, d = tid % D, g = tid / D, s0 = g * SLE;
+    const int t0 = chunk * TM;
+    const long long row0 = static_cast<long long>(b) * T + t0;
+    float Gk[SLE], Ck[SLE], yk[SLE];
+#pragma unroll
+    for (int i0 = 0; i0 < SLE; i0 += 4) {  // loads in batches of 4 steps
+        float mv[4], pv[4], av[4], bv[4];
+#pragma unroll
+        for (int i = i0; i < i0 + 4; ++i) {
+            const int t = t0 + s0 + i;
+            const size_t o = (static_cast<size_t>(row0) + s0 + i) * D + d;
+            mv[i - i0] = t < T ? __ldcg(A.elk_m + o) : 0.f;
+            yk[i] = t < T ? __ldcg(hold + o) : 0.f;
+            pv[i - i0] = t + 1 < T ? __ldcg(A.elk_p + o) : 0.f;
+            av[i - i0] = t + 1 < T ? __ldcg(A.elk_a + o + D) : 0.f;
+            bv[i - i0] = t + 1 < T ? __ldcg(A.elk_b + o + D) : 0.f;
+        }
+#pragma unroll
+        for (int i = i0; i < i0 + 4; ++i) {
+            const int t = t0 + s0 + i;
+            float Gv = 1.f, Cv = 0.f;
+            if (t == T - 1) {
+                Gv = 0.f;
+                Cv = mv[i - i0];
+            } else if (t < T) {
+                const float P = pv[i - i0], an = av[i - i0], m = mv[i - i0];
+                Gv = __fdividef(P * an, fmaf(an * an, P, 1.f));
+                Cv = m - Gv * fmaf(an, m, bv[i - i0]);
+            }
+            Gk[i] = Gv;
+            Ck[i] = Cv;
+        }
+    }
+    float cG = 1.f, cC = 0.f;  // s at the segment's first step from s after its last
+#pragma unroll
+    for (int i = SLE - 1; i >= 0; --i) {
+        cC = fmaf(Gk[i], cC, Ck[i]);
+        cG = Gk[i] * cG;
+    }
+    {
+        float *fa = E.aff + (g * D + d) * 2;
+        fa[0] = cG;
+        fa[1] = cC;
+    }
+    __syncthreads();
+    {  // state after the tile (from the next chunk), all threads
+        const int ld = tid / SEGS, lq = tid % SEGS;
+        float EG = 1.f, EC = 0.f;
+        for (int q = SEGS - 1; q >= 0; --q) {
+            const float *qa = E.aff + (q * D + ld) * 2;
+            EC = fmaf(qa[0], EC, qa[1]);
+            EG = qa[0] * EG;
+        }
+        const float sin_ = coop_lookback<SEGS, kElkWin>(desc_bwd, tile, -static_cast<long long>(B), D, ld, lq,
+                                                        epoch, EG, EC, n_chunks - 1 - chunk, 0.f, status);
+        if (lq == 0) E.cM[ld] = sin_;
+    }
+    __syncthreads();
+    float sv = E.cM[d];
+    for (int q = SEGS - 1; q > g; --q) {
+        const float *qa = E.aff + (q * D + d) * 2;
+        sv = fmaf(qa[0], sv, qa[1]);
+    }
+#pragma unroll
+    for (int i = SLE - 1; i >= 0; --i) {
+        sv = fmaf(Gk[i], sv, Ck[i]);
+        if (t0 + s0 + i < T) {
+            __stcg(hnew + (static_cast<size_t>(row0) + s0 + i) * D + d, sv);
+            dmax = max(dmax, abs_bits(sv - yk[i]));
+        }
+    }
+    __syncthreads();  // the segment maps are rewritten by the next tile
+}
+
 template <int D>
 __device__ __forceinline__ void issue_fill(const CUtensorMap *map, unsigned char *slot, long long row0,
                                            unsigned bar) {
@@ -226,7 +444,7 @@ __device__ __forceinline__ void issue_fill(const CUtensorMap *map, unsigned char
         tma_load_2d(smem_u32(slot + hf * G::SLOT_HALF), map, hf * 32, static_cast<int>(row0 - 1), bar);
 }
 
-template <int D>
+template <int D, bool ELK>
 __global__ void __launch_bounds__(NTHREADS, 1)
 quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_constant__ CUtensorMap map_h1,
                  Tc2Args S) {
@@ -247,6 +465,11 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
     unsigned long long *bars = reinterpret_cast<unsigned long long *>(red + 32);  // fill[2], mma[2]
     unsigned *tmem_slot = reinterpret_cast<unsigned *>(bars + 4);
     volatile int *cta_err = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    ElkSmem es;
+    es.mob = reinterpret_cast<float *>(tmem_slot + 4);
+    es.aff = es.mob + 4 * NTHREADS;
+    es.cP = es.aff + 2 * NTHREADS;
+    es.cM = es.cP + D;
 
     const DiagArgs &A = S.a;
     const int T = A.T, B = A.B;
@@ -291,6 +514,10 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
     const unsigned tmem = *tmem_slot;
     constexpr unsigned idesc = make_idesc(2u, TM, G::N);  // kind::tf32, M=128, N=3D
     const unsigned b_hi = smem_u32(bhi), b_lo = smem_u32(blo);
+    // quasi-ELK look-back descriptors: covariance [tile][D][4], mean and smoother [tile][D][2]
+    unsigned long long *desc_cov = A.desc;
+    unsigned long long *desc_mean = A.desc + static_cast<size_t>(S.n_tiles) * D * 4;
+    unsigned long long *desc_bwd = A.desc + static_cast<size_t>(S.n_tiles) * D * 6;
 
     // bit q: mbarrier parity of fill slot q / accumulator q; an operation in flight
     unsigned fill_par = 0u, mma_par = 0u, fill_pending = 0u, mma_pending = 0u;
@@ -444,6 +671,32 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
             }
             asm volatile("tcgen05.fence::before_thread_sync;");
 
+            if constexpr (ELK) {
+                // 4'. quasi-ELK: a_t, b_t to memory (the smoother reads them too),
+                // then the filter's covariance and mean scans
+#pragma unroll
+                for (int rh = 0; rh < 2; ++rh)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int r = qd * 32 + rh * 16 + gid + 8 * e;
+                        if (t0 + r < T) {
+                            float va[V], vb[V];
+#pragma unroll
+                            for (int j = 0; j < NJ; ++j)
+#pragma unroll
+                                for (int x = 0; x < 2; ++x) {
+                                    va[2 * j + x] = av[rh][e][j][x];
+                                    vb[2 * j + x] = bv[rh][e][j][x];
+                                }
+                            const size_t o = (static_cast<size_t>(row0) + r) * D + dbase;
+                            stv<V>(A.elk_a + o, va);
+                            stv<V>(A.elk_b + o, vb);
+                        }
+                    }
+                __syncthreads();
+                elk_forward_scans<D>(A, es, slot, tile, chunk, b, t0, row0, epoch, desc_cov, desc_mean,
+                                     status);
+            } else {
             // 4. scan over the tile's steps, per lane d, in registers.  Inside a
             // warp the steps of lane d are s = 16 rh + 8 e + gid (gid across the
             // 8 lanes of one tq, (rh, e) inside the thread).
@@ -535,6 +788,8 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
                     }
             }
 
+            }  // quasi scan
+
             // 5. slot `cur` and accumulator `cur` are free: refill the slot with tile k+2
             asm volatile("tcgen05.fence::before_thread_sync;");
             __syncthreads();
@@ -543,6 +798,17 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
                     issue_fill<D>(map, slots + cur * G::SLOT_BYTES, row0_of(tile_of(k + 2)),
                                   smem_u32(&bars[cur]));
                 fill_pending |= 1u << cur;
+            }
+        }
+        if constexpr (ELK) {
+            // the smoother runs backward over time once every filter value is written
+            grid_barrier(hdr->barrier, nblocks, status);
+            const float *hold = A.hbuf[it & 1];
+            for (long long k = 0; k < my_n && !timed_out(status); ++k) {
+                const long long tr = S.n_tiles - 1 - tile_of(k);
+                const int c = static_cast<int>(static_cast<unsigned>(tr) / static_cast<unsigned>(B));
+                elk_backward_tile<D>(A, es, tr, c, static_cast<int>(tr) - c * B, S.n_chunks, epoch,
+                                     desc_bwd, hold, hnew, dmax, status);
             }
         }
         const unsigned bd = block_max_u32(dmax, red);
@@ -592,7 +858,7 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
     }
 }
 
-template <int D>
+template <int D, bool ELK>
 cudaError_t launch_tc2(const DiagArgs &a, cudaStream_t s) {
     using G = Tc2Geom<D>;
     Tc2Args S;
@@ -604,7 +870,7 @@ cudaError_t launch_tc2(const DiagArgs &a, cudaStream_t s) {
     if (!make_map(&m0, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.hbuf[0], rows, D, 32, ROWS) ||
         !make_map(&m1, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.hbuf[1], rows, D, 32, ROWS))
         return cudaErrorInvalidValue;
-    auto kern = quasi_tc2_kernel<D>;
+    auto kern = quasi_tc2_kernel<D, ELK>;
     // every CTA takes all 512 TMEM columns, so at most one may reside on an SM:
     // the shared-memory request alone guarantees it
     const int smem = G::SMEM_BYTES > 120 * 1024 ? G::SMEM_BYTES : 120 * 1024;
@@ -638,8 +904,9 @@ bool quasi_tc_supported(const pararnn_cell &cell, int B, int T) {
     return encode_fn() != nullptr;
 }
 
-cudaError_t launch_quasi_tc2(const DiagArgs &a, cudaStream_t s) {
-    return a.D == 32 ? launch_tc2<32>(a, s) : launch_tc2<64>(a, s);
+cudaError_t launch_quasi_tc2(const DiagArgs &a, bool elk, cudaStream_t s) {
+    if (elk) return a.D == 32 ? launch_tc2<32, true>(a, s) : launch_tc2<64, true>(a, s);
+    return a.D == 32 ? launch_tc2<32, false>(a, s) : launch_tc2<64, false>(a, s);
 }
 
 }  // namespace pararnn

@@ -24,7 +24,7 @@ cudaError_t launch_dense_solver(const pararnn_cell &cell, int mode, const DiagAr
                                 void *dense_ws, cudaStream_t s);
 size_t quasi_tc_desc_bytes(int B, int T, int D);
 bool quasi_tc_supported(const pararnn_cell &cell, int B, int T);
-cudaError_t launch_quasi_tc2(const DiagArgs &a, cudaStream_t s);
+cudaError_t launch_quasi_tc2(const DiagArgs &a, bool elk, cudaStream_t s);
 bool diag2_supported(const pararnn_cell &cell, int B, int T);
 size_t diag2_desc_bytes(int B, int T, int D);
 cudaError_t launch_diag2(const DiagArgs &a, cudaStream_t s);
@@ -76,10 +76,11 @@ WsLayout ws_layout(const pararnn_cell &cell, int B, int T, int mode) {
     L.desc = off;
     if (diag) {
         size_t desc = static_cast<size_t>(tl.n_tiles) * tl.DG * (is_elk(mode) ? 8 : 2) * 8;
-        // the tensor-core dense-cell path tiles by 128 steps x all lanes
-        if (cell.kind == PARARNN_GRU_DENSE && mode == PARARNN_QUASI &&
+        // the tensor-core dense-cell path tiles by 128 steps x all lanes (quasi-ELK:
+        // covariance, mean and smoother descriptors, 8 words per tile and lane)
+        if (cell.kind == PARARNN_GRU_DENSE && (mode == PARARNN_QUASI || mode == PARARNN_QUASI_ELK) &&
             (cell.d == 32 || cell.d == 64)) {
-            const size_t tc = quasi_tc_desc_bytes(B, T, cell.d);
+            const size_t tc = quasi_tc_desc_bytes(B, T, cell.d) * (is_elk(mode) ? 4 : 1);
             if (tc > desc) desc = tc;
         }
         // the streaming diagonal-cell path tiles by 32 steps x 64 lanes
@@ -170,11 +171,11 @@ static cudaError_t enqueue_iterate(const pararnn_cell *cell, const pararnn_param
     cudaError_t e = cudaMemsetAsync(ws + L.header, 0, 256, s);
     if (e == cudaSuccess && diag && L.elk > L.desc) e = cudaMemsetAsync(ws + L.desc, 0, L.elk - L.desc, s);
     if (e != cudaSuccess) return e;
-    if (mode == PARARNN_QUASI && quasi_tc_supported(*cell, B, T)) {
+    if ((mode == PARARNN_QUASI || mode == PARARNN_QUASI_ELK) && quasi_tc_supported(*cell, B, T)) {
         // the tensor-core path reads the initial guess (zero) from memory
         e = cudaMemsetAsync(a.hbuf[0], 0, states * sizeof(float), s);
         if (e != cudaSuccess) return e;
-        return launch_quasi_tc2(a, s);
+        return launch_quasi_tc2(a, mode == PARARNN_QUASI_ELK, s);
     }
     if (cell->kind == PARARNN_GRU_DIAG && !is_elk(mode) && diag2_supported(*cell, B, T)) {
         e = cudaMemsetAsync(a.hbuf[0], 0, states * sizeof(float), s);
