@@ -95,6 +95,23 @@ def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
 
+def max_over_ranks(ms: float, device) -> float:
+    """The slowest rank's time: device timings are combined with a MAX
+    all-reduce (a no-op without a process group)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(states_per_rank: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: the states every rank solved over the slowest
+    rank's time (weak scaling: each rank owns its own batch)."""
+    return world * steps * states_per_rank / (max_ms / 1e3)
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -279,11 +296,8 @@ def run_ours(args):
     total_ms = sum(e0.elapsed_time(e2) for e0, _, e2 in evs)
     solver_ms = [e1.elapsed_time(e2) for _, e1, e2 in evs]
     proj_ms = [e0.elapsed_time(e1) for e0, e1, _ in evs]
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
-    value = world * args.steps * states / (max_ms / 1e3)
+    max_ms = max_over_ranks(total_ms, dev)
+    value = job_value(states, args.steps, world, max_ms)
 
     # end to end through the public call: pinned host x in, host h out, each step
     x_host = w.x.pin_memory()
@@ -301,10 +315,7 @@ def run_ours(args):
         h_host.copy_(out, non_blocking=True)
     eb.record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([ea.elapsed_time(eb)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * e2e_steps * states / (float(te.item()) / 1e3)
+    e2e_value = job_value(states, e2e_steps, world, max_over_ranks(ea.elapsed_time(eb), dev))
 
     cpu = None
     if rank == 0 and world == 1:
