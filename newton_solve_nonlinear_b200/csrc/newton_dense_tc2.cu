@@ -283,7 +283,10 @@ __device__ void elk_forward_scans(const DiagArgs &A, const ElkSmem &E, const uns
     }
     __syncthreads();
     // (ii) covariances, gains and the mean's affine maps
-    float Pk[SLE];
+    float Pk[SLE], bk[SLE];
+#pragma unroll
+    for (int i = 0; i < SLE; ++i)  // all of the segment's b_t in flight at once
+        bk[i] = t0 + s0 + i < T ? __ldcg(A.elk_b + (static_cast<size_t>(row0) + s0 + i) * D + d) : 0.f;
     {
         Mob X{1.f, 0.f, 0.f, 1.f};  // this segment's exclusive prefix
         for (int q = 0; q < g; ++q) {
@@ -300,10 +303,9 @@ __device__ void elk_forward_scans(const DiagArgs &A, const ElkSmem &E, const uns
                 const float Pm = fmaf(ak[i] * ak[i], P, 1.f);
                 P = __fdividef(Pm, fmaf(lam, Pm, 1.f));
                 const float K = lam * P, omk = 1.f - K;
-                const float bt = __ldcg(A.elk_b + (static_cast<size_t>(row0) + s) * D + d);
                 const float y = *reinterpret_cast<const float *>(slot + sw_off(s + 1, d, G::SLOT_HALF));
                 alpha = omk * ak[i];
-                beta = fmaf(omk, bt, K * y);
+                beta = fmaf(omk, bk[i], K * y);
             }
             Pk[i] = P;
             SB = fmaf(alpha, SB, beta);
@@ -341,9 +343,8 @@ __device__ void elk_forward_scans(const DiagArgs &A, const ElkSmem &E, const uns
             if (t0 + s < T) {  // the gain-weighted map again: K_t = lambda P_t
                 const size_t o = (static_cast<size_t>(row0) + s) * D + d;
                 const float K = lam * Pk[i], omk = 1.f - K;
-                const float bt = __ldcg(A.elk_b + o);
                 const float y = *reinterpret_cast<const float *>(slot + sw_off(s + 1, d, G::SLOT_HALF));
-                m = fmaf(omk * ak[i], m, fmaf(omk, bt, K * y));
+                m = fmaf(omk * ak[i], m, fmaf(omk, bk[i], K * y));
                 __stcg(A.elk_m + o, m);
                 __stcg(A.elk_p + o, Pk[i]);
             }
@@ -363,30 +364,36 @@ __device__ void elk_backward_tile(const DiagArgs &A, const ElkSmem &E, long long
     const int t0 = chunk * TM;
     const long long row0 = static_cast<long long>(b) * T + t0;
     float Gk[SLE], Ck[SLE], yk[SLE];
-#pragma unroll
-    for (int i0 = 0; i0 < SLE; i0 += 4) {  // loads in batches of 4 steps
-        float mv[4], pv[4], av[4], bv[4];
+    // loads in batches of 4 steps, the next batch in flight while one is used
+    float mv[2][4], pv[2][4], av[2][4], bv[2][4];
+    auto load_batch = [&](int i0, int sl) {
 #pragma unroll
         for (int i = i0; i < i0 + 4; ++i) {
             const int t = t0 + s0 + i;
             const size_t o = (static_cast<size_t>(row0) + s0 + i) * D + d;
-            mv[i - i0] = t < T ? __ldcg(A.elk_m + o) : 0.f;
+            mv[sl][i - i0] = t < T ? __ldcg(A.elk_m + o) : 0.f;
             yk[i] = t < T ? __ldcg(hold + o) : 0.f;
-            pv[i - i0] = t + 1 < T ? __ldcg(A.elk_p + o) : 0.f;
-            av[i - i0] = t + 1 < T ? __ldcg(A.elk_a + o + D) : 0.f;
-            bv[i - i0] = t + 1 < T ? __ldcg(A.elk_b + o + D) : 0.f;
+            pv[sl][i - i0] = t + 1 < T ? __ldcg(A.elk_p + o) : 0.f;
+            av[sl][i - i0] = t + 1 < T ? __ldcg(A.elk_a + o + D) : 0.f;
+            bv[sl][i - i0] = t + 1 < T ? __ldcg(A.elk_b + o + D) : 0.f;
         }
+    };
+    load_batch(0, 0);
+#pragma unroll
+    for (int i0 = 0; i0 < SLE; i0 += 4) {
+        const int sl = (i0 / 4) & 1;
+        if (i0 + 4 < SLE) load_batch(i0 + 4, sl ^ 1);
 #pragma unroll
         for (int i = i0; i < i0 + 4; ++i) {
             const int t = t0 + s0 + i;
             float Gv = 1.f, Cv = 0.f;
             if (t == T - 1) {
                 Gv = 0.f;
-                Cv = mv[i - i0];
+                Cv = mv[sl][i - i0];
             } else if (t < T) {
-                const float P = pv[i - i0], an = av[i - i0], m = mv[i - i0];
+                const float P = pv[sl][i - i0], an = av[sl][i - i0], m = mv[sl][i - i0];
                 Gv = __fdividef(P * an, fmaf(an * an, P, 1.f));
-                Cv = m - Gv * fmaf(an, m, bv[i - i0]);
+                Cv = m - Gv * fmaf(an, m, bv[sl][i - i0]);
             }
             Gk[i] = Gv;
             Ck[i] = Cv;
