@@ -189,12 +189,14 @@ __device__ void stage_block(const DiagArgs &A, float *buf, int b, int tb, int n,
 __device__ void block_coefs(const float (&u)[3][4][4][2], const float *Pb, const float *Hb,
                             const float *bh, int D, const Lane &L, float *cf) {
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {  // rows 8 nt .. 8 nt + 7, all three gates
-        float acc[3][4];
+    for (int np = 0; np < 2; ++np) {  // row tiles in pairs: six independent accumulation chains
+        float acc[2][3][4];
 #pragma unroll
-        for (int g = 0; g < 3; ++g)
+        for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) acc[g][q] = 0.f;
+            for (int g = 0; g < 3; ++g)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[h][g][q] = 0.f;
 #pragma unroll
         for (int kt = 0; kt < 4; ++kt) {
             const float2 r0 = *reinterpret_cast<const float2 *>(Hb + L.gid * 32 + kt * 8 + 2 * L.tq);
@@ -208,36 +210,42 @@ __device__ void block_coefs(const float (&u)[3][4][4][2], const float *Pb, const
                 al[q] = __float_as_uint(av[q] - __uint_as_float(ah[q]));
             }
 #pragma unroll
-            for (int g = 0; g < 3; ++g) {
-                const unsigned bh0 = __float_as_uint(u[g][nt][kt][0]) & 0xffffe000u;
-                const unsigned bh1 = __float_as_uint(u[g][nt][kt][1]) & 0xffffe000u;
-                const unsigned bl0 = __float_as_uint(u[g][nt][kt][0] - __uint_as_float(bh0));
-                const unsigned bl1 = __float_as_uint(u[g][nt][kt][1] - __uint_as_float(bh1));
-                mma8(acc[g], al[0], al[1], al[2], al[3], bh0, bh1);
-                mma8(acc[g], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
-                mma8(acc[g], ah[0], ah[1], ah[2], ah[3], bh0, bh1);
-            }
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int g = 0; g < 3; ++g) {
+                    const int nt = 2 * np + h;
+                    const unsigned bh0 = __float_as_uint(u[g][nt][kt][0]) & 0xffffe000u;
+                    const unsigned bh1 = __float_as_uint(u[g][nt][kt][1]) & 0xffffe000u;
+                    const unsigned bl0 = __float_as_uint(u[g][nt][kt][0] - __uint_as_float(bh0));
+                    const unsigned bl1 = __float_as_uint(u[g][nt][kt][1] - __uint_as_float(bh1));
+                    mma8(acc[h][g], al[0], al[1], al[2], al[3], bh0, bh1);
+                    mma8(acc[h][g], ah[0], ah[1], ah[2], ah[3], bl0, bl1);
+                    mma8(acc[h][g], ah[0], ah[1], ah[2], ah[3], bh0, bh1);
+                }
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int s = L.gid + 8 * (q >> 1), i = nt * 8 + 2 * L.tq + (q & 1);
-            const float *Pt = Pb + s * 96;
-            const float r = sigmoidf_(Pt[i] + acc[0][q] + bh[i]);
-            const float z = sigmoidf_(Pt[32 + i] + acc[1][q] + bh[32 + i]);
-            const float gn = acc[2][q] + bh[64 + i];
-            const float nn = tanhf_(Pt[64 + i] + r * gn);
-            const float hprev = Hb[s * 32 + i];
-            const float f = nn + z * (hprev - nn);
-            const float omz = 1.f - z;
-            const float cn = omz * (1.f - nn * nn) * r;
-            const bool live = i < D;
-            float *o = cf + s * kCS + (2 * L.tq + (q & 1)) * 20 + nt;  // row i = 8 nt + gid'
-            o[0] = live ? z : 0.f;
-            o[4] = live ? (hprev - nn) * z * omz : 0.f;
-            o[8] = live ? cn : 0.f;
-            o[12] = live ? cn * gn * (1.f - r) : 0.f;
-            o[16] = live ? Hb[(s + 1) * 32 + i] - f : 0.f;
-        }
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int nt = 2 * np + h;
+                const int s = L.gid + 8 * (q >> 1), i = nt * 8 + 2 * L.tq + (q & 1);
+                const float *Pt = Pb + s * 96;
+                const float r = sigmoidf_(Pt[i] + acc[h][0][q] + bh[i]);
+                const float z = sigmoidf_(Pt[32 + i] + acc[h][1][q] + bh[32 + i]);
+                const float gn = acc[h][2][q] + bh[64 + i];
+                const float nn = tanhf_(Pt[64 + i] + r * gn);
+                const float hprev = Hb[s * 32 + i];
+                const float f = nn + z * (hprev - nn);
+                const float omz = 1.f - z;
+                const float cn = omz * (1.f - nn * nn) * r;
+                const bool live = i < D;
+                float *o = cf + s * kCS + (2 * L.tq + (q & 1)) * 20 + nt;  // row i = 8 nt + gid'
+                o[0] = live ? z : 0.f;
+                o[4] = live ? (hprev - nn) * z * omz : 0.f;
+                o[8] = live ? cn : 0.f;
+                o[12] = live ? cn * gn * (1.f - r) : 0.f;
+                o[16] = live ? Hb[(s + 1) * 32 + i] - f : 0.f;
+            }
     }
 }
 
