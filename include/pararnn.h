@@ -183,6 +183,44 @@ PARARNN_API int pararnn_newton_solve_async(const pararnn_cell *cell, const parar
                                pararnn_stream stream);
 
 /*
+ * pararnn_newton_solve_host -- the same evaluation from and to HOST memory,
+ * with the copies overlapped with the computation.
+ *
+ * The B sequences are independent, so the batch is solved in `parts`
+ * consecutive parts of ceil(B / parts) sequences (the last may be shorter;
+ * when that size leaves nothing for the last parts there are fewer parts,
+ * e.g. B = 4 asked in 3 parts runs as 2 + 2).
+ * While part p is solved on `stream`, part p+1's inputs are copied in and
+ * part p-1's states copied out on two streams the call creates and destroys;
+ * the device staging is double-buffered in the workspace.  Each part is an
+ * independent solve to `tol` (its own convergence test), so a part may take
+ * fewer iterations than the whole batch would.
+ *
+ * Arguments as for pararnn_newton_solve, except:
+ *   x_host     HOST [B, T, Din] of cell->x_dtype (page-locked memory lets the
+ *              copies run asynchronously; pageable memory is accepted).
+ *   h0_host    HOST [B, D] float.
+ *   h_host     HOST [B, T, D] float, output.
+ *   info       HOST, output, may be NULL: the worst part (largest iters,
+ *              status, delta and residual over the parts).
+ *   parts      1 <= parts <= B.
+ *   workspace  DEVICE, at least pararnn_host_workspace_size(cell, B, T, mode,
+ *              parts) bytes, 256-byte aligned.
+ *   stream     work on `stream` queued before the call runs first; on return
+ *              everything has completed (the call synchronises `stream`).
+ * Returns the worst part's status, or INVALID_ARG / CUDA_ERROR.
+ */
+PARARNN_API int pararnn_newton_solve_host(const pararnn_cell *cell, const pararnn_params *params,
+                              const void *x_host, const float *h0_host, int B, int T, int mode,
+                              float lambda, float tol, int max_iters, float *h_host,
+                              pararnn_info *info, int parts, void *workspace, size_t ws_bytes,
+                              pararnn_stream stream);
+
+/* Workspace bytes of pararnn_newton_solve_host; 0 if the arguments are rejected. */
+PARARNN_API size_t pararnn_host_workspace_size(const pararnn_cell *cell, int B, int T, int mode,
+                                               int parts);
+
+/*
  * pararnn_input_projection -- P = x W_ih^T + b_ih for every (b, t): the input
  * pre-activations, which do not depend on the state and so are computed once
  * per solve (as one GEMM [B*T, Din] x [Din, 3D]).  pararnn_newton_solve runs

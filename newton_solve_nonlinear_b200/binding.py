@@ -24,7 +24,8 @@ STATUS = {0: "OK", 1: "NOT_CONVERGED", 2: "DIVERGED", 3: "INVALID_ARG", 4: "CUDA
 EXPORTS = ("pararnn_workspace_size", "pararnn_newton_solve", "pararnn_newton_solve_async",
            "pararnn_input_projection", "pararnn_newton_iterate_async",
            "pararnn_affine_scan_workspace_size", "pararnn_affine_scan",
-           "pararnn_affine_scan_status", "pararnn_status_string")
+           "pararnn_affine_scan_status", "pararnn_status_string", "pararnn_newton_solve_host",
+           "pararnn_host_workspace_size")
 
 
 class Cell(ctypes.Structure):
@@ -73,6 +74,11 @@ def lib() -> ctypes.CDLL:
         L.pararnn_affine_scan.restype = ci
         L.pararnn_affine_scan_status.argtypes = [vp, vp]
         L.pararnn_affine_scan_status.restype = ci
+        L.pararnn_newton_solve_host.argtypes = [ctypes.POINTER(Cell), ctypes.POINTER(Params), vp, vp,
+                                                ci, ci, ci, cf, cf, ci, vp, vp, ci, vp, sz, vp]
+        L.pararnn_newton_solve_host.restype = ci
+        L.pararnn_host_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci, ci, ci]
+        L.pararnn_host_workspace_size.restype = sz
         L.pararnn_status_string.argtypes = [ci]
         L.pararnn_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -168,6 +174,52 @@ def newton_solve(w_ih, b_ih, w_hh, b_hh, x, h0, *, kind: str, mode: str, tol: fl
     if rc != 0:
         raise RuntimeError(f"pararnn_newton_solve_async: {L.pararnn_status_string(rc).decode()}")
     return out
+
+
+def _host(t: torch.Tensor, name: str) -> int:
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def host_workspace_size(kind: str, din: int, d: int, B: int, T: int, mode: str, parts: int,
+                        dtype: torch.dtype = torch.float32) -> int:
+    cell = make_cell(kind, din, d, dtype)
+    return int(lib().pararnn_host_workspace_size(ctypes.byref(cell), B, T, MODES[mode], parts))
+
+
+def newton_solve_host(w_ih, b_ih, w_hh, b_hh, x_host, h0_host, *, kind: str, mode: str, tol: float,
+                      lam: float = 0.0, max_iters: int = 0, parts: int = 4, out=None,
+                      workspace=None, device=None, stream=None) -> "SolveResult":
+    """The solve from and to HOST tensors (x_host [B,T,Din], h0_host [B,D];
+    ``out`` a host [B,T,D] fp32 tensor, page-locked for overlap).  The batch is
+    solved in ``parts`` parts with copies overlapped with compute; weights are
+    CUDA tensors.  Returns a SolveResult whose h is the host tensor and whose
+    report is the worst part's."""
+    B, T, din = x_host.shape
+    d = h0_host.shape[1]
+    parts = max(1, min(int(parts), B))
+    cell = make_cell(kind, din, d, x_host.dtype)
+    L = lib()
+    m = MODES[mode]
+    need = int(L.pararnn_host_workspace_size(ctypes.byref(cell), B, T, m, parts))
+    if need == 0:
+        raise ValueError("arguments rejected by pararnn_host_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, w_hh.device if device is None else device)
+    if out is None:
+        out = torch.empty(B, T, d, dtype=torch.float32).pin_memory()
+    params = Params(_dev(w_ih, "w_ih"), _dev(b_ih, "b_ih"), _dev(w_hh, "w_hh"), _dev(b_hh, "b_hh"))
+    info = Info()
+    rc = L.pararnn_newton_solve_host(ctypes.byref(cell), ctypes.byref(params), _host(x_host, "x_host"),
+                                     _host(h0_host, "h0_host"), B, T, m, float(lam), float(tol),
+                                     int(max_iters), _host(out, "out"), ctypes.byref(info), parts,
+                                     _dev(workspace, "workspace"), workspace.numel(), _stream(stream))
+    if rc in (3, 4):
+        raise RuntimeError(f"pararnn_newton_solve_host: {L.pararnn_status_string(rc).decode()}")
+    return SolveResult(out, info.iters, STATUS[info.status], info.delta, info.residual)
 
 
 def input_projection(x, w_ih, b_ih, *, d: int, kind: str = "dense", out=None, stream=None):

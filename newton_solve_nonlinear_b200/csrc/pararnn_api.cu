@@ -12,6 +12,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <vector>
 
 #include "common.cuh"
 #include "solver.cuh"
@@ -311,6 +312,121 @@ const char *pararnn_status_string(int status) {
         case PARARNN_TIMEOUT: return "PARARNN_TIMEOUT";
         default: return "PARARNN_UNKNOWN_STATUS";
     }
+}
+
+
+// ---- host-buffer solve: the batch in parts, copies overlapped with compute ----
+
+namespace {
+
+struct HostLayout {
+    int parts, bp;  // number of parts, sequences per part (the last may be shorter)
+    size_t solve, xs[2], hs[2], h0, infos, total;
+};
+
+HostLayout host_layout(const pararnn_cell &cell, int B, int T, int mode, int parts) {
+    HostLayout H{};
+    H.bp = (B + parts - 1) / parts;
+    H.parts = (B + H.bp - 1) / H.bp;  // e.g. B=4 in 3 parts is 2+2: no empty part
+    const size_t es = cell.x_dtype == PARARNN_BF16 ? 2 : 4;
+    const size_t xbytes = static_cast<size_t>(H.bp) * T * cell.din * es;
+    const size_t hbytes = static_cast<size_t>(H.bp) * T * cell.d * 4;
+    size_t off = 0;
+    H.solve = off; off = align256(off + ws_layout(cell, H.bp, T, mode).total);
+    for (int q = 0; q < 2; ++q) { H.xs[q] = off; off = align256(off + xbytes); }
+    for (int q = 0; q < 2; ++q) { H.hs[q] = off; off = align256(off + hbytes); }
+    H.h0 = off; off = align256(off + static_cast<size_t>(B) * cell.d * 4);
+    H.infos = off; off = align256(off + static_cast<size_t>(parts) * sizeof(pararnn_info));
+    H.total = off;
+    return H;
+}
+
+}  // namespace
+
+size_t pararnn_host_workspace_size(const pararnn_cell *cell, int B, int T, int mode, int parts) {
+    if (!cell_ok(cell, B, T, mode) || parts < 1 || parts > B) return 0;
+    return host_layout(*cell, B, T, mode, parts).total;
+}
+
+int pararnn_newton_solve_host(const pararnn_cell *cell, const pararnn_params *params, const void *x_host,
+                              const float *h0_host, int B, int T, int mode, float lambda, float tol,
+                              int max_iters, float *h_host, pararnn_info *info, int parts,
+                              void *workspace, size_t ws_bytes, pararnn_stream stream) {
+    if (!cell_ok(cell, B, T, mode) || parts < 1 || parts > B || !params || !x_host || !h0_host ||
+        !h_host || !workspace || !aligned(workspace, 256))
+        return PARARNN_INVALID_ARG;
+    const HostLayout H = host_layout(*cell, B, T, mode, parts);
+    if (ws_bytes < H.total) return PARARNN_INVALID_ARG;
+    char *ws = static_cast<char *>(workspace);
+    const size_t es = cell->x_dtype == PARARNN_BF16 ? 2 : 4;
+    const size_t xrow = static_cast<size_t>(T) * cell->din * es;  // bytes of one sequence's input
+    const size_t hrow = static_cast<size_t>(T) * cell->d * 4;      // bytes of one sequence's states
+    cudaStream_t sc = reinterpret_cast<cudaStream_t>(stream);
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev[7] = {};  // in[2], comp[2], out[2], h0
+    cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
+    for (int q = 0; q < 7 && e == cudaSuccess; ++q) e = cudaEventCreateWithFlags(&ev[q], cudaEventDisableTiming);
+    int rc = PARARNN_OK;
+    float *h0_dev = reinterpret_cast<float *>(ws + H.h0);
+    pararnn_info *infos = reinterpret_cast<pararnn_info *>(ws + H.infos);
+    if (e == cudaSuccess) {
+        // start only after the caller's earlier work on its stream
+        e = cudaEventRecord(ev[6], sc);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev[6], 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(h0_dev, h0_host, static_cast<size_t>(B) * cell->d * 4, cudaMemcpyHostToDevice, s_in);
+    }
+    for (int p = 0; p < H.parts && e == cudaSuccess && rc == PARARNN_OK; ++p) {
+        const int buf = p & 1;
+        const int b0 = p * H.bp, nb = (B - b0) < H.bp ? (B - b0) : H.bp;
+        if (p >= 2) e = cudaStreamWaitEvent(s_in, ev[4 + buf], 0);  // staging of part p-2 free
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(ws + H.xs[buf], static_cast<const char *>(x_host) + b0 * xrow, nb * xrow,
+                                cudaMemcpyHostToDevice, s_in);
+        if (e == cudaSuccess) e = cudaEventRecord(ev[buf], s_in);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(sc, ev[buf], 0);
+        if (e != cudaSuccess) break;
+        rc = solve_enqueue(cell, params, ws + H.xs[buf], h0_dev + static_cast<size_t>(b0) * cell->d, nb, T, mode,
+                           lambda, tol, max_iters, reinterpret_cast<float *>(ws + H.hs[buf]), infos + p,
+                           ws + H.solve, ws_layout(*cell, nb, T, mode).total, stream);
+        if (rc != PARARNN_OK) break;
+        e = cudaEventRecord(ev[2 + buf], sc);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev[2 + buf], 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(reinterpret_cast<char *>(h_host) + b0 * hrow, ws + H.hs[buf], nb * hrow,
+                                cudaMemcpyDeviceToHost, s_out);
+        if (e == cudaSuccess) e = cudaEventRecord(ev[4 + buf], s_out);
+    }
+    // the caller's stream continues after the last copy out
+    pararnn_info agg{};
+    if (e == cudaSuccess && rc == PARARNN_OK) {
+        e = cudaEventRecord(ev[6], s_out);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(sc, ev[6], 0);
+        std::vector<pararnn_info> host(H.parts);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(host.data(), infos, H.parts * sizeof(pararnn_info), cudaMemcpyDeviceToHost, sc);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(sc);
+        if (e == cudaSuccess) {
+            for (int p = 0; p < H.parts; ++p) {  // worst part: statuses are ordered by severity
+                agg.iters = host[p].iters > agg.iters ? host[p].iters : agg.iters;
+                agg.status = host[p].status > agg.status ? host[p].status : agg.status;
+                agg.delta = host[p].delta > agg.delta ? host[p].delta : agg.delta;
+                agg.residual = host[p].residual > agg.residual ? host[p].residual : agg.residual;
+            }
+            if (info) *info = agg;
+            rc = agg.status;
+        }
+    }
+    // leave nothing in flight before the helper streams go away
+    if (s_in) cudaStreamSynchronize(s_in);
+    if (s_out) cudaStreamSynchronize(s_out);
+    for (int q = 0; q < 7; ++q)
+        if (ev[q]) cudaEventDestroy(ev[q]);
+    if (s_in) cudaStreamDestroy(s_in);
+    if (s_out) cudaStreamDestroy(s_out);
+    if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
+    return rc;
 }
 
 }  // extern "C"

@@ -1,0 +1,99 @@
+"""GPU parity of the host-buffer solve (inputs and states in page-locked host
+memory, the batch solved in parts with the copies overlapped) vs the oracle.
+
+The parts are independent solves, so:
+  * with one part the call runs the device solve on the same batch and its
+    states equal the device call's bit for bit;
+  * with a fixed iteration count (tol 0) every sequence's iterate depends on
+    that sequence alone and matches the oracle's iterate within the family's
+    tolerance (5e-5 max-abs, as for the device path);
+  * converged states match the fp64 rollout within 1e-4 whatever the split.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle.cells import GRU, rollout
+from newton_solve_nonlinear_b200 import binding
+from newton_solve_nonlinear_b200.inputs import make_workload
+
+pytestmark = pytest.mark.gpu
+
+
+def _weights(w):
+    dev = lambda t: t.cuda().contiguous()
+    return dev(w.w_ih), dev(w.b_ih), dev(w.w_hh), dev(w.b_hh)
+
+
+def _host_solve(w, mode, parts, **kw):
+    x = w.x.contiguous().pin_memory()
+    h0 = w.h0.float().contiguous().pin_memory()
+    kw.setdefault("tol", w.tol)
+    return binding.newton_solve_host(*_weights(w), x, h0, kind=w.kind, mode=mode, parts=parts, **kw)
+
+
+def _oracle(w):
+    return GRU.from_workload(w), w.x.double().numpy(), w.h0.double().numpy()
+
+
+def test_one_part_equals_device_solve():
+    w = make_workload("untrained", B=3, T=2500, h0_std=0.5)
+    r_host = _host_solve(w, "QUASI", 1)
+    r_dev = binding.solve_workload(w, "QUASI")
+    assert r_host.status == r_dev.status == "OK"
+    assert r_host.iters == r_dev.iters
+    assert not r_host.h.is_cuda
+    assert torch.equal(r_host.h, r_dev.h.cpu())
+
+
+@pytest.mark.parametrize("name,over,mode,lam", [
+    ("untrained", dict(B=5, T=3000, h0_std=0.5), "QUASI", 0.0),
+    ("untrained", dict(B=4, T=1000, x_dtype=torch.bfloat16, w_dtype=torch.bfloat16), "DEER", 0.0),
+    ("dense_deer", dict(B=3, T=1500, bias_std=0.2), "DEER", 0.0),
+    ("near_unstable", dict(B=3, T=400), "QUASI_ELK", 0.5),
+    ("near_unstable", dict(B=3, T=200), "ELK", 0.3),
+])
+@pytest.mark.parametrize("parts", [2, 3])
+def test_fixed_iterations_match_oracle(name, over, mode, lam, parts):
+    w = make_workload(name, **over)
+    c, x, h0 = _oracle(w)
+    if mode in ("ELK", "QUASI_ELK"):
+        ref = oracle.elk_solve(c, x, h0, mode, lam, 0.0, max_iters=2, record=True)
+    else:
+        ref = oracle.newton_solve(c, x, h0, mode, 0.0, max_iters=2, record=True)
+    r = _host_solve(w, mode, parts, tol=0.0, max_iters=2, lam=lam)
+    assert r.iters == 2 and r.status == "NOT_CONVERGED"
+    err = np.max(np.abs(r.h.double().numpy() - ref["iterates"][1]))
+    assert err <= 5e-5, err
+
+
+@pytest.mark.parametrize("name,over,mode,parts", [
+    ("untrained", dict(B=5, T=3000, h0_std=0.5), "QUASI", 5),
+    ("untrained", dict(B=7, T=777, bias_std=0.3), "DEER", 3),
+    ("diag", dict(B=3, T=500, d=128, din=128), "DEER", 2),
+    ("diag", dict(B=2, T=300, d=256, din=256), "QUASI", 2),
+    ("dense_deer", dict(B=3, T=2000), "DEER", 3),
+])
+def test_converged_states_match_rollout(name, over, mode, parts):
+    w = make_workload(name, **over)
+    c, x, h0 = _oracle(w)
+    r = _host_solve(w, mode, parts)
+    assert r.status == "OK"
+    assert np.max(np.abs(r.h.double().numpy() - rollout(c, x, h0))) <= 1e-4
+
+
+def test_parts_clamped_and_caller_buffer_used():
+    w = make_workload("untrained", B=2, T=300)
+    out = torch.full((2, 300, 64), float("nan")).pin_memory()
+    r = _host_solve(w, "QUASI", 9, out=out)
+    assert r.h.data_ptr() == out.data_ptr() and r.status == "OK"
+    c, x, h0 = _oracle(w)
+    assert np.max(np.abs(out.double().numpy() - rollout(c, x, h0))) <= 1e-4
+
+
+def test_device_tensor_rejected():
+    w = make_workload("untrained", B=2, T=64)
+    with pytest.raises(ValueError):
+        binding.newton_solve_host(*_weights(w), w.x.cuda(), w.h0.float(), kind=w.kind,
+                                  mode="QUASI", tol=w.tol)
