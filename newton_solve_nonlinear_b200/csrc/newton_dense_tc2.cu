@@ -146,17 +146,26 @@ __device__ __forceinline__ void tmem_st(unsigned taddr, const unsigned (&v)[8]) 
                  : "memory");
 }
 
-// A operand of the tile staged in `slot`: rows r = 0..127 are h_{t0+r-1}
-// (staged row r; h0 replaces it for a sequence's first step).  Warp (quarter
-// qd, column group kq) writes TMEM lanes 32 qd .. 32 qd + 31 (its own lane
-// quarter), K columns kq KW .. kq KW + KW - 1, split into hi (A_HI) and lo (A_LO).
+// Time step held by TMEM lane 32 qd + l of the accumulator (and A row): the
+// 16x256b fragment hands thread (gid = l & 7) of a warp the lanes gid, gid + 8,
+// gid + 16, gid + 24 of its quarter; they hold the four consecutive steps
+// 32 qd + 4 gid .. + 3, so each thread scans its steps in registers.
+__device__ __forceinline__ int step_of_lane(int qd, int l) {
+    return qd * 32 + 4 * (l & 7) + 2 * (l >> 4) + ((l >> 3) & 1);
+}
+
+// A operand of the tile staged in `slot`: the row of TMEM lane L is h_{t0+s-1},
+// s = step_of_lane (staged row s; h0 replaces it for a sequence's first step).
+// Warp (quarter qd, column group kq) writes TMEM lanes 32 qd .. 32 qd + 31 (its
+// own lane quarter), K columns kq KW .. kq KW + KW - 1, split into hi (A_HI) and
+// lo (A_LO).
 template <int D>
 __device__ __forceinline__ void write_a(const unsigned char *slot, unsigned tmem, const float *h0row,
                                         bool first_chunk, int warp, int lane) {
     using G = Tc2Geom<D>;
     constexpr int KW = G::KW;
     const int qd = warp & 3, kq = warp >> 2;
-    const int r = qd * 32 + lane;
+    const int r = step_of_lane(qd, lane);
     const int k0 = kq * KW;
     float v[KW];
 #pragma unroll
@@ -584,13 +593,14 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
 
             if (tid == 0 && k + 2 < my_n) prefetch_p<D>(A.P, tile_of(k + 2), B, T);
             // 1. this tile's input pre-activations: thread (gid, tq) of warp (qd, lh)
-            // owns steps r = 32 qd + 16 rh + 8 e + gid and lanes dbase .. dbase + V - 1
+            // owns steps r = 32 qd + 4 gid + 2 rh + e (TMEM lanes 32 qd + 16 rh + 8 e
+            // + gid) and lanes dbase .. dbase + V - 1
             float pv[2][2][3][V];
 #pragma unroll
             for (int rh = 0; rh < 2; ++rh)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const int r = qd * 32 + rh * 16 + gid + 8 * e;
+                    const int r = qd * 32 + 4 * gid + 2 * rh + e;
                     const float *prow = A.P + (static_cast<size_t>(row0) + r) * 3 * D + dbase;
 #pragma unroll
                     for (int g = 0; g < 3; ++g) {
@@ -627,23 +637,34 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
             }
 
             // 3. epilogue: the cell at the guess, a_t and b_t per (step, lane);
-            // element (rh, e, j, x) is step r = 32 qd + 16 rh + 8 e + gid, lane
+            // element (rh, e, j, x) is step r = 32 qd + 4 gid + 2 rh + e, lane
             // dbase + 2 j + x
             float av[2][2][NJ][2], bv[2][2][NJ][2];
             const unsigned acc = cur ? G::ACC1 : 0u;
 #pragma unroll
             for (int rh = 0; rh < 2; ++rh) {
                 const unsigned trow = tmem + acc + (static_cast<unsigned>(qd * 32 + rh * 16) << 16);
+                // staged rows r, r + 1, r + 2 of the steps r, r + 1: h_{t-1} and h_t
                 float hp[2][V], y[2][V];
+                {
+                    const int r = qd * 32 + 4 * gid + 2 * rh;
+                    ldv<V>(reinterpret_cast<const float *>(slot + sw_off(r, dbase, G::SLOT_HALF)), hp[0]);
+                    if (t0 == 0 && r == 0) ldgv<V>(A.h0 + static_cast<size_t>(b) * D + dbase, hp[0]);
+                    ldv<V>(reinterpret_cast<const float *>(slot + sw_off(r + 1, dbase, G::SLOT_HALF)), y[0]);
+                    ldv<V>(reinterpret_cast<const float *>(slot + sw_off(r + 2, dbase, G::SLOT_HALF)), y[1]);
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int r = qd * 32 + rh * 16 + gid + 8 * e;
-                    ldv<V>(reinterpret_cast<const float *>(slot + sw_off(r, dbase, G::SLOT_HALF)), hp[e]);
-                    if (t0 == 0 && r == 0) ldgv<V>(A.h0 + static_cast<size_t>(b) * D + dbase, hp[e]);
-                    ldv<V>(reinterpret_cast<const float *>(slot + sw_off(r + 1, dbase, G::SLOT_HALF)), y[e]);
+                    for (int v = 0; v < V; ++v) hp[1][v] = y[0][v];
                 }
 #pragma unroll
                 for (int j = 0; j < NJ; ++j) {
+                    // the lane pair's recurrent biases and U diagonals, read once
+                    const int d2 = dbase + 2 * j;
+                    const float2 bhr = *reinterpret_cast<const float2 *>(c_bh + d2);
+                    const float2 bhz = *reinterpret_cast<const float2 *>(c_bh + D + d2);
+                    const float2 bhn = *reinterpret_cast<const float2 *>(c_bh + 2 * D + d2);
+                    const float2 udr = *reinterpret_cast<const float2 *>(c_ud + d2);
+                    const float2 udz = *reinterpret_cast<const float2 *>(c_ud + D + d2);
+                    const float2 udn = *reinterpret_cast<const float2 *>(c_ud + 2 * D + d2);
                     unsigned gv[3][4];
 #pragma unroll
                     for (int g = 0; g < 3; ++g)
@@ -653,7 +674,7 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
                     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int r = qd * 32 + rh * 16 + gid + 8 * e;
+                        const int r = qd * 32 + 4 * gid + 2 * rh + e;
                         const bool ok = t0 + r < T;
 #pragma unroll
                         for (int x = 0; x < 2; ++x) {
@@ -661,13 +682,12 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
                             float a_ = 1.f, b_ = 0.f;
                             if (ok) {
                                 float f;
-                                const int d = dbase + v;
                                 gru_cell_diag(pv[rh][e][0][v], pv[rh][e][1][v], pv[rh][e][2][v],
                                               __uint_as_float(gv[0][2 * e + x]),
                                               __uint_as_float(gv[1][2 * e + x]),
-                                              __uint_as_float(gv[2][2 * e + x]), c_bh[d], c_bh[D + d],
-                                              c_bh[2 * D + d], c_ud[d], c_ud[D + d], c_ud[2 * D + d],
-                                              hp[e][v], f, a_, b_);
+                                              __uint_as_float(gv[2][2 * e + x]), x ? bhr.y : bhr.x,
+                                              x ? bhz.y : bhz.x, x ? bhn.y : bhn.x, x ? udr.y : udr.x,
+                                              x ? udz.y : udz.x, x ? udn.y : udn.x, hp[e][v], f, a_, b_);
                                 rmax = max(rmax, abs_bits(y[e][v] - f));
                             }
                             av[rh][e][j][x] = a_;
@@ -685,7 +705,7 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
                 for (int rh = 0; rh < 2; ++rh)
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int r = qd * 32 + rh * 16 + gid + 8 * e;
+                        const int r = qd * 32 + 4 * gid + 2 * rh + e;
                         if (t0 + r < T) {
                             float va[V], vb[V];
 #pragma unroll
@@ -704,46 +724,38 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
                 elk_forward_scans<D>(A, es, slot, tile, chunk, b, t0, row0, epoch, desc_cov, desc_mean,
                                      status);
             } else {
-            // 4. scan over the tile's steps, per lane d, in registers.  Inside a
-            // warp the steps of lane d are s = 16 rh + 8 e + gid (gid across the
-            // 8 lanes of one tq, (rh, e) inside the thread).
-            // 4a. inclusive Kogge-Stone across gid within each 8-step group
-#pragma unroll
-            for (int o = 1; o < 8; o <<= 1) {
-#pragma unroll
-                for (int rh = 0; rh < 2; ++rh)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e)
-#pragma unroll
-                        for (int j = 0; j < NJ; ++j)
-#pragma unroll
-                            for (int x = 0; x < 2; ++x) {
-                                const float pa = __shfl_up_sync(0xffffffffu, av[rh][e][j][x], 4 * o);
-                                const float pb = __shfl_up_sync(0xffffffffu, bv[rh][e][j][x], 4 * o);
-                                if (gid >= o) compose(av[rh][e][j][x], bv[rh][e][j][x], pa, pb);
-                            }
-            }
-            // 4b. prefix over the four groups (group totals sit at gid = 7); the
-            // warp quarter's total goes to shared memory
+            // 4. scan over the tile's steps, per lane d, in registers.  Thread gid of
+            // a quad column holds the consecutive steps 32 qd + 4 gid + k, k = 2 rh + e.
 #pragma unroll
             for (int j = 0; j < NJ; ++j)
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
-                    float ea = 1.f, eb = 0.f;
+                    // 4a. inclusive prefix over the thread's four steps
+                    compose(av[0][1][j][x], bv[0][1][j][x], av[0][0][j][x], bv[0][0][j][x]);
+                    compose(av[1][0][j][x], bv[1][0][j][x], av[0][1][j][x], bv[0][1][j][x]);
+                    compose(av[1][1][j][x], bv[1][1][j][x], av[1][0][j][x], bv[1][0][j][x]);
+                    // 4b. Kogge-Stone over the eight threads' totals (gid = 0 .. 7)
+                    float ta = av[1][1][j][x], tb = bv[1][1][j][x];
 #pragma unroll
-                    for (int g4 = 0; g4 < 4; ++g4) {
-                        const int rh = g4 >> 1, e = g4 & 1;
-                        float ta = __shfl_sync(0xffffffffu, av[rh][e][j][x], 28 + tq);
-                        float tb = __shfl_sync(0xffffffffu, bv[rh][e][j][x], 28 + tq);
-                        if (g4 > 0) compose(av[rh][e][j][x], bv[rh][e][j][x], ea, eb);
-                        compose(ta, tb, ea, eb);
-                        ea = ta;
-                        eb = tb;
+                    for (int o = 1; o < 8; o <<= 1) {
+                        const float pa = __shfl_up_sync(0xffffffffu, ta, 4 * o);
+                        const float pb = __shfl_up_sync(0xffffffffu, tb, 4 * o);
+                        if (gid >= o) compose(ta, tb, pa, pb);
                     }
-                    if (gid == 0) {
+                    // the thread's exclusive prefix (gid - 1's inclusive) folded into its
+                    // steps: every (a, b) then maps the quarter's carry-in to the step
+                    float ea = __shfl_up_sync(0xffffffffu, ta, 4);
+                    float eb = __shfl_up_sync(0xffffffffu, tb, 4);
+                    if (gid > 0) {
+#pragma unroll
+                        for (int rh = 0; rh < 2; ++rh)
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) compose(av[rh][e][j][x], bv[rh][e][j][x], ea, eb);
+                    }
+                    if (gid == 7) {  // the warp quarter's total
                         const int d = dbase + 2 * j + x;
-                        wt_a[qd * D + d] = ea;
-                        wt_b[qd * D + d] = eb;
+                        wt_a[qd * D + d] = ta;
+                        wt_b[qd * D + d] = tb;
                     }
                 }
             __syncthreads();
@@ -778,7 +790,7 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
                 for (int rh = 0; rh < 2; ++rh)
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int r = qd * 32 + rh * 16 + gid + 8 * e;
+                        const int r = qd * 32 + 4 * gid + 2 * rh + e;
                         if (t0 + r < T) {
                             float y[V], h[V];
                             ldv<V>(reinterpret_cast<const float *>(slot + sw_off(r + 1, dbase, G::SLOT_HALF)), y);
