@@ -125,6 +125,80 @@ __device__ __forceinline__ void stv(float *p, const float (&v)[V]) {
         __stcg(reinterpret_cast<float2 *>(p), make_float2(v[0], v[1]));
 }
 
+// ---- two lanes of the GRU cell at once on the fp32x2 datapath (sm_100):
+// add / sub / mul / fma .f32x2 round each half exactly like the fp32
+// instruction, so results equal the one-lane form bit for bit up to the
+// order of operations; exp and reciprocal stay per lane (ex2.approx,
+// rcp.approx, as in the one-lane form).
+using u64 = unsigned long long;
+__device__ __forceinline__ u64 pk(float a, float b) {
+    u64 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void upk(u64 r, float &a, float &b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ u64 add2(u64 a, u64 b) {
+    u64 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ u64 sub2(u64 a, u64 b) {
+    u64 d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ u64 mul2(u64 a, u64 b) {
+    u64 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ u64 fma2(u64 a, u64 b, u64 c) {
+    u64 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ u64 ex2_2(u64 v) {  // 2^v per lane
+    float a, b;
+    upk(v, a, b);
+    asm("ex2.approx.ftz.f32 %0, %0;" : "+f"(a));
+    asm("ex2.approx.ftz.f32 %0, %0;" : "+f"(b));
+    return pk(a, b);
+}
+__device__ __forceinline__ u64 rcp2(u64 v) {  // 1 / v per lane
+    float a, b;
+    upk(v, a, b);
+    asm("rcp.approx.ftz.f32 %0, %0;" : "+f"(a));
+    asm("rcp.approx.ftz.f32 %0, %0;" : "+f"(b));
+    return pk(a, b);
+}
+__device__ __forceinline__ u64 splat(float v) { return pk(v, v); }
+
+// gru_cell_diag for two lanes: the gates r = 1 / (1 + 2^(-v log2 e)), likewise z,
+// n = tanh(u) = 1 - 2 / (2^(2 u log2 e) + 1); f = n + z (h - n); the Jacobian
+// diagonal a = z + (h - n) z (1 - z) U_z + (1 - z)(1 - n^2) r U_n
+// + (1 - z)(1 - n^2)(U_n h + b_hn) r (1 - r) U_r; bb = f - a h.
+__device__ __forceinline__ void gru_cell_diag_x2(u64 pr, u64 pz, u64 pn, u64 gr, u64 gz, u64 gnh,
+                                                 u64 bhr, u64 bhz, u64 bhn, u64 udr, u64 udz, u64 udn,
+                                                 u64 h, u64 &f, u64 &a, u64 &bb) {
+    constexpr float kLog2e = 1.4426950408889634f;
+    const u64 one = splat(1.f);
+    const u64 r = rcp2(add2(ex2_2(mul2(add2(add2(pr, gr), bhr), splat(-kLog2e))), one));
+    const u64 z = rcp2(add2(ex2_2(mul2(add2(add2(pz, gz), bhz), splat(-kLog2e))), one));
+    const u64 gn = add2(gnh, bhn);
+    const u64 en = ex2_2(mul2(fma2(r, gn, pn), splat(2.f * kLog2e)));
+    const u64 n = fma2(splat(-2.f), rcp2(add2(en, one)), one);
+    const u64 hmn = sub2(h, n);
+    f = fma2(z, hmn, n);
+    const u64 omz = sub2(one, z);
+    const u64 cz = mul2(mul2(hmn, z), omz);
+    const u64 m = mul2(mul2(omz, fma2(n, n, splat(-1.f))), r);  // -(1 - z)(1 - n^2) r
+    const u64 mr = mul2(mul2(m, gn), sub2(one, r));                // -(cell's U_r coefficient)
+    a = sub2(fma2(cz, udz, z), fma2(mr, udr, mul2(m, udn)));
+    bb = sub2(f, mul2(a, h));
+}
+
 // Affine map composition: apply (a1, b1) first, then (a2, b2).
 __device__ __forceinline__ void compose(float &a2, float &b2, float a1, float b1) {
     b2 = fmaf(a2, b1, b2);
@@ -676,23 +750,29 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
                     for (int e = 0; e < 2; ++e) {
                         const int r = qd * 32 + 4 * gid + 2 * rh + e;
                         const bool ok = t0 + r < T;
-#pragma unroll
-                        for (int x = 0; x < 2; ++x) {
-                            const int v = 2 * j + x;
-                            float a_ = 1.f, b_ = 0.f;
-                            if (ok) {
-                                float f;
-                                gru_cell_diag(pv[rh][e][0][v], pv[rh][e][1][v], pv[rh][e][2][v],
-                                              __uint_as_float(gv[0][2 * e + x]),
-                                              __uint_as_float(gv[1][2 * e + x]),
-                                              __uint_as_float(gv[2][2 * e + x]), x ? bhr.y : bhr.x,
-                                              x ? bhz.y : bhz.x, x ? bhn.y : bhn.x, x ? udr.y : udr.x,
-                                              x ? udz.y : udz.x, x ? udn.y : udn.x, hp[e][v], f, a_, b_);
-                                rmax = max(rmax, abs_bits(y[e][v] - f));
-                            }
-                            av[rh][e][j][x] = a_;
-                            bv[rh][e][j][x] = b_;
+                        float a0 = 1.f, a1 = 1.f, b0 = 0.f, b1 = 0.f;
+                        if (ok) {  // lanes 2j, 2j + 1 together
+                            const int v = 2 * j;
+                            u64 f2, a2, b2;
+                            gru_cell_diag_x2(pk(pv[rh][e][0][v], pv[rh][e][0][v + 1]),
+                                             pk(pv[rh][e][1][v], pv[rh][e][1][v + 1]),
+                                             pk(pv[rh][e][2][v], pv[rh][e][2][v + 1]),
+                                             pk(__uint_as_float(gv[0][2 * e]), __uint_as_float(gv[0][2 * e + 1])),
+                                             pk(__uint_as_float(gv[1][2 * e]), __uint_as_float(gv[1][2 * e + 1])),
+                                             pk(__uint_as_float(gv[2][2 * e]), __uint_as_float(gv[2][2 * e + 1])),
+                                             pk(bhr.x, bhr.y), pk(bhz.x, bhz.y), pk(bhn.x, bhn.y),
+                                             pk(udr.x, udr.y), pk(udz.x, udz.y), pk(udn.x, udn.y),
+                                             pk(hp[e][v], hp[e][v + 1]), f2, a2, b2);
+                            float r0, r1;
+                            upk(sub2(pk(y[e][v], y[e][v + 1]), f2), r0, r1);
+                            rmax = max(rmax, max(abs_bits(r0), abs_bits(r1)));
+                            upk(a2, a0, a1);
+                            upk(b2, b0, b1);
                         }
+                        av[rh][e][j][0] = a0;
+                        av[rh][e][j][1] = a1;
+                        bv[rh][e][j][0] = b0;
+                        bv[rh][e][j][1] = b1;
                     }
                 }
             }
