@@ -175,19 +175,21 @@ __device__ __forceinline__ u64 rcp2(u64 v) {  // 1 / v per lane
 }
 __device__ __forceinline__ u64 splat(float v) { return pk(v, v); }
 
+constexpr float kLog2eF = 1.4426950408889634f;
+
 // gru_cell_diag for two lanes: the gates r = 1 / (1 + 2^(-v log2 e)), likewise z,
 // n = tanh(u) = 1 - 2 / (2^(2 u log2 e) + 1); f = n + z (h - n); the Jacobian
 // diagonal a = z + (h - n) z (1 - z) U_z + (1 - z)(1 - n^2) r U_n
-// + (1 - z)(1 - n^2)(U_n h + b_hn) r (1 - r) U_r; bb = f - a h.
+// + (1 - z)(1 - n^2)(U_n h + b_hn) r (1 - r) U_r; bb = f - a h.  bhr and bhz
+// come premultiplied by -log2(e): -v log2 e = (p + g) (-log2 e) + bh (-log2 e).
 __device__ __forceinline__ void gru_cell_diag_x2(u64 pr, u64 pz, u64 pn, u64 gr, u64 gz, u64 gnh,
                                                  u64 bhr, u64 bhz, u64 bhn, u64 udr, u64 udz, u64 udn,
                                                  u64 h, u64 &f, u64 &a, u64 &bb) {
-    constexpr float kLog2e = 1.4426950408889634f;
     const u64 one = splat(1.f);
-    const u64 r = rcp2(add2(ex2_2(mul2(add2(add2(pr, gr), bhr), splat(-kLog2e))), one));
-    const u64 z = rcp2(add2(ex2_2(mul2(add2(add2(pz, gz), bhz), splat(-kLog2e))), one));
+    const u64 r = rcp2(add2(ex2_2(fma2(add2(pr, gr), splat(-kLog2eF), bhr)), one));
+    const u64 z = rcp2(add2(ex2_2(fma2(add2(pz, gz), splat(-kLog2eF), bhz)), one));
     const u64 gn = add2(gnh, bhn);
-    const u64 en = ex2_2(mul2(fma2(r, gn, pn), splat(2.f * kLog2e)));
+    const u64 en = ex2_2(mul2(fma2(r, gn, pn), splat(2.f * kLog2eF)));
     const u64 n = fma2(splat(-2.f), rcp2(add2(en, one)), one);
     const u64 hmn = sub2(h, n);
     f = fma2(z, hmn, n);
@@ -197,6 +199,17 @@ __device__ __forceinline__ void gru_cell_diag_x2(u64 pr, u64 pz, u64 pn, u64 gr,
     const u64 mr = mul2(mul2(m, gn), sub2(one, r));                // -(cell's U_r coefficient)
     a = sub2(fma2(cz, udz, z), fma2(mr, udr, mul2(m, udn)));
     bb = sub2(f, mul2(a, h));
+}
+
+// compose() for two lanes: (a2, b2) := (a2, b2) o (a1, b1).
+__device__ __forceinline__ void compose2(u64 &a2, u64 &b2, u64 a1, u64 b1) {
+    b2 = fma2(a2, b1, b2);
+    a2 = mul2(a2, a1);
+}
+__device__ __forceinline__ u64 shfl_up2(u64 v, int delta) {
+    float a, b;
+    upk(v, a, b);
+    return pk(__shfl_up_sync(0xffffffffu, a, delta), __shfl_up_sync(0xffffffffu, b, delta));
 }
 
 // Affine map composition: apply (a1, b1) first, then (a2, b2).
@@ -546,7 +559,7 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
     unsigned char *bhi = smem + G::OFF_BHI, *blo = smem + G::OFF_BLO;
     unsigned char *slots = smem + G::OFF_SLOT;
     float *misc = reinterpret_cast<float *>(smem + G::OFF_MISC);
-    float *c_bh = misc;                   // [3D] b_hh
+    float *c_bh = misc;                   // [3D] b_hh; the r and z parts times -log2(e)
     float *c_ud = c_bh + 3 * D;           // [3D] diagonal of U_g
     float *wt_a = c_ud + 3 * D;           // [4][D] affine total of each warp quarter's 32 steps
     float *wt_b = wt_a + 4 * D;
@@ -582,7 +595,7 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
         *reinterpret_cast<float *>(blo + off) = v - hi;
     }
     for (int i = tid; i < 3 * D; i += NTHREADS) {
-        c_bh[i] = __ldg(A.b_hh + i);
+        c_bh[i] = __ldg(A.b_hh + i) * (i < 2 * D ? -kLog2eF : 1.f);
         const int g = i / D, d = i % D;
         c_ud[i] = __ldg(A.w_hh + (static_cast<size_t>(g) * D + d) * D + d);
     }
@@ -807,37 +820,46 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
             // 4. scan over the tile's steps, per lane d, in registers.  Thread gid of
             // a quad column holds the consecutive steps 32 qd + 4 gid + k, k = 2 rh + e.
 #pragma unroll
-            for (int j = 0; j < NJ; ++j)
+            for (int j = 0; j < NJ; ++j) {  // lanes 2j, 2j + 1 as fp32x2 pairs
+                u64 pa_[2][2], pb_[2][2];
 #pragma unroll
-                for (int x = 0; x < 2; ++x) {
-                    // 4a. inclusive prefix over the thread's four steps
-                    compose(av[0][1][j][x], bv[0][1][j][x], av[0][0][j][x], bv[0][0][j][x]);
-                    compose(av[1][0][j][x], bv[1][0][j][x], av[0][1][j][x], bv[0][1][j][x]);
-                    compose(av[1][1][j][x], bv[1][1][j][x], av[1][0][j][x], bv[1][0][j][x]);
-                    // 4b. Kogge-Stone over the eight threads' totals (gid = 0 .. 7)
-                    float ta = av[1][1][j][x], tb = bv[1][1][j][x];
+                for (int rh = 0; rh < 2; ++rh)
 #pragma unroll
-                    for (int o = 1; o < 8; o <<= 1) {
-                        const float pa = __shfl_up_sync(0xffffffffu, ta, 4 * o);
-                        const float pb = __shfl_up_sync(0xffffffffu, tb, 4 * o);
-                        if (gid >= o) compose(ta, tb, pa, pb);
+                    for (int e = 0; e < 2; ++e) {
+                        pa_[rh][e] = pk(av[rh][e][j][0], av[rh][e][j][1]);
+                        pb_[rh][e] = pk(bv[rh][e][j][0], bv[rh][e][j][1]);
                     }
-                    // the thread's exclusive prefix (gid - 1's inclusive) folded into its
-                    // steps: every (a, b) then maps the quarter's carry-in to the step
-                    float ea = __shfl_up_sync(0xffffffffu, ta, 4);
-                    float eb = __shfl_up_sync(0xffffffffu, tb, 4);
-                    if (gid > 0) {
+                // 4a. inclusive prefix over the thread's four steps
+                compose2(pa_[0][1], pb_[0][1], pa_[0][0], pb_[0][0]);
+                compose2(pa_[1][0], pb_[1][0], pa_[0][1], pb_[0][1]);
+                compose2(pa_[1][1], pb_[1][1], pa_[1][0], pb_[1][0]);
+                // 4b. Kogge-Stone over the eight threads' totals (gid = 0 .. 7)
+                u64 ta = pa_[1][1], tb = pb_[1][1];
 #pragma unroll
-                        for (int rh = 0; rh < 2; ++rh)
-#pragma unroll
-                            for (int e = 0; e < 2; ++e) compose(av[rh][e][j][x], bv[rh][e][j][x], ea, eb);
-                    }
-                    if (gid == 7) {  // the warp quarter's total
-                        const int d = dbase + 2 * j + x;
-                        wt_a[qd * D + d] = ta;
-                        wt_b[qd * D + d] = tb;
-                    }
+                for (int o = 1; o < 8; o <<= 1) {
+                    const u64 qa = shfl_up2(ta, 4 * o), qb = shfl_up2(tb, 4 * o);
+                    if (gid >= o) compose2(ta, tb, qa, qb);
                 }
+                // the thread's exclusive prefix (gid - 1's inclusive) folded into its
+                // steps: every (a, b) then maps the quarter's carry-in to the step
+                const u64 ea = shfl_up2(ta, 4), eb = shfl_up2(tb, 4);
+#pragma unroll
+                for (int rh = 0; rh < 2; ++rh)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        if (gid > 0) compose2(pa_[rh][e], pb_[rh][e], ea, eb);
+                        upk(pa_[rh][e], av[rh][e][j][0], av[rh][e][j][1]);
+                        upk(pb_[rh][e], bv[rh][e][j][0], bv[rh][e][j][1]);
+                    }
+                if (gid == 7) {  // the warp quarter's total
+                    const int d = dbase + 2 * j;
+                    float a0, a1, b0, b1;
+                    upk(ta, a0, a1);
+                    upk(tb, b0, b1);
+                    *reinterpret_cast<float2 *>(wt_a + qd * D + d) = make_float2(a0, a1);
+                    *reinterpret_cast<float2 *>(wt_b + qd * D + d) = make_float2(b0, b1);
+                }
+            }
             __syncthreads();
             // 4c. the tile's carry-in per lane by look-back over earlier chunks;
             // every thread takes part (G per lane)
@@ -875,13 +897,15 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
                             float y[V], h[V];
                             ldv<V>(reinterpret_cast<const float *>(slot + sw_off(r + 1, dbase, G::SLOT_HALF)), y);
 #pragma unroll
-                            for (int j = 0; j < NJ; ++j)
-#pragma unroll
-                                for (int x = 0; x < 2; ++x) {
-                                    const int v = 2 * j + x;
-                                    h[v] = fmaf(av[rh][e][j][x], hin[v], bv[rh][e][j][x]);
-                                    dmax = max(dmax, abs_bits(h[v] - y[v]));
-                                }
+                            for (int j = 0; j < NJ; ++j) {
+                                const int v = 2 * j;
+                                const u64 h2 = fma2(pk(av[rh][e][j][0], av[rh][e][j][1]), pk(hin[v], hin[v + 1]),
+                                                    pk(bv[rh][e][j][0], bv[rh][e][j][1]));
+                                float d0, d1;
+                                upk(sub2(h2, pk(y[v], y[v + 1])), d0, d1);
+                                dmax = max(dmax, max(abs_bits(d0), abs_bits(d1)));
+                                upk(h2, h[v], h[v + 1]);
+                            }
                             stv<V>(hnew + (static_cast<size_t>(row0) + r) * D + dbase, h);
                         }
                     }
