@@ -155,6 +155,82 @@ __device__ __forceinline__ void gru_cell_diag(float pr, float pz, float pn, floa
     bb = f - a * h;
 }
 
+// ---- two cells at once on the fp32x2 datapath (sm_100):
+// add / sub / mul / fma .f32x2 round each half exactly like the fp32
+// instruction, so results equal the one-lane form bit for bit up to the
+// order of operations; exp and reciprocal stay per lane (ex2.approx,
+// rcp.approx, as in the one-lane form).
+using u64 = unsigned long long;
+__device__ __forceinline__ u64 pk(float a, float b) {
+    u64 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void upk(u64 r, float &a, float &b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ u64 add2(u64 a, u64 b) {
+    u64 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ u64 sub2(u64 a, u64 b) {
+    u64 d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ u64 mul2(u64 a, u64 b) {
+    u64 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ u64 fma2(u64 a, u64 b, u64 c) {
+    u64 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ u64 ex2_2(u64 v) {  // 2^v per lane
+    float a, b;
+    upk(v, a, b);
+    asm("ex2.approx.ftz.f32 %0, %0;" : "+f"(a));
+    asm("ex2.approx.ftz.f32 %0, %0;" : "+f"(b));
+    return pk(a, b);
+}
+__device__ __forceinline__ u64 rcp2(u64 v) {  // 1 / v per lane
+    float a, b;
+    upk(v, a, b);
+    asm("rcp.approx.ftz.f32 %0, %0;" : "+f"(a));
+    asm("rcp.approx.ftz.f32 %0, %0;" : "+f"(b));
+    return pk(a, b);
+}
+__device__ __forceinline__ u64 splat(float v) { return pk(v, v); }
+
+constexpr float kLog2eF = 1.4426950408889634f;
+
+// gru_cell_diag for two lanes: the gates r = 1 / (1 + 2^(-v log2 e)), likewise z,
+// n = tanh(u) = 1 - 2 / (2^(2 u log2 e) + 1); f = n + z (h - n); the Jacobian
+// diagonal a = z + (h - n) z (1 - z) U_z + (1 - z)(1 - n^2) r U_n
+// + (1 - z)(1 - n^2)(U_n h + b_hn) r (1 - r) U_r; bb = f - a h.  bhr and bhz
+// come premultiplied by -log2(e): -v log2 e = (p + g) (-log2 e) + bh (-log2 e).
+__device__ __forceinline__ void gru_cell_diag_x2(u64 pr, u64 pz, u64 pn, u64 gr, u64 gz, u64 gnh,
+                                                 u64 bhr, u64 bhz, u64 bhn, u64 udr, u64 udz, u64 udn,
+                                                 u64 h, u64 &f, u64 &a, u64 &bb) {
+    const u64 one = splat(1.f);
+    const u64 r = rcp2(add2(ex2_2(fma2(add2(pr, gr), splat(-kLog2eF), bhr)), one));
+    const u64 z = rcp2(add2(ex2_2(fma2(add2(pz, gz), splat(-kLog2eF), bhz)), one));
+    const u64 gn = add2(gnh, bhn);
+    const u64 en = ex2_2(mul2(fma2(r, gn, pn), splat(2.f * kLog2eF)));
+    const u64 n = fma2(splat(-2.f), rcp2(add2(en, one)), one);
+    const u64 hmn = sub2(h, n);
+    f = fma2(z, hmn, n);
+    const u64 omz = sub2(one, z);
+    const u64 cz = mul2(mul2(hmn, z), omz);
+    const u64 m = mul2(mul2(omz, fma2(n, n, splat(-1.f))), r);  // -(1 - z)(1 - n^2) r
+    const u64 mr = mul2(mul2(m, gn), sub2(one, r));                // -(cell's U_r coefficient)
+    a = sub2(fma2(cz, udz, z), fma2(mr, udr, mul2(m, udn)));
+    bb = sub2(f, mul2(a, h));
+}
+
 // |x| as an unsigned bit pattern: ordered like the float for x >= 0, and any
 // NaN or Inf maps above every finite value (0x7f800000 and up), so an integer
 // max over patterns both finds the largest |dh| and flags non-finite values.

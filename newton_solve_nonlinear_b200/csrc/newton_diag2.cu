@@ -159,7 +159,9 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
             // 1. cells of this thread's 8 steps
             const int di = lane0 + d;
             const float ur = __ldg(A.w_hh + di), uz = __ldg(A.w_hh + D + di), un = __ldg(A.w_hh + 2 * D + di);
-            const float br = __ldg(A.b_hh + di), bz = __ldg(A.b_hh + D + di), bn = __ldg(A.b_hh + 2 * D + di);
+            // r and z biases times -log2(e), as gru_cell_diag_x2 takes them
+            const float br = -kLog2eF * __ldg(A.b_hh + di), bz = -kLog2eF * __ldg(A.b_hh + D + di);
+            const float bn = __ldg(A.b_hh + 2 * D + di);
             // a thread's rows start at a multiple of 8, so the swizzle of row
             // seg*SL + i is the constant i: lane offsets are hoisted out of the loop
             const unsigned char *Pt = slot + (d >> 5) * P_BOX + seg * SL * 128 + (d & 3) * 4;
@@ -169,25 +171,46 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
             float EA = 1.f, EB = 0.f;
             float hp = *reinterpret_cast<const float *>(Ht + (jq << 4));
             if (t0 == 0 && seg == 0) hp = __ldg(A.h0 + static_cast<size_t>(b) * D + di);
+            const u64 ur2 = splat(ur), uz2 = splat(uz), un2 = splat(un);
 #pragma unroll
-            for (int i = 0; i < SL; ++i) {
-                const int o = i * 128 + ((jq ^ i) << 4);
-                const int oy = (i + 1) * 128 + ((jq ^ ((i + 1) & 7)) << 4);
-                const float y = *reinterpret_cast<const float *>(Ht + oy);
-                float a_ = 1.f, b_ = 0.f;
+            for (int i = 0; i < SL; i += 2) {  // steps i, i + 1 together on fp32x2
+                const int o0 = i * 128 + ((jq ^ i) << 4), o1 = (i + 1) * 128 + ((jq ^ (i + 1)) << 4);
+                const int oy = (i + 2) * 128 + ((jq ^ ((i + 2) & 7)) << 4);
+                const float y0 = *reinterpret_cast<const float *>(Ht + o1);  // h_{t}, then h_{t-1} of i + 1
+                const float y1 = *reinterpret_cast<const float *>(Ht + oy);
+                const u64 h2 = pk(hp, y0);
+                u64 f2, a2, b2;
+                gru_cell_diag_x2(pk(*reinterpret_cast<const float *>(Pt + 0 * P_BOX + o0),
+                                    *reinterpret_cast<const float *>(Pt + 0 * P_BOX + o1)),
+                                 pk(*reinterpret_cast<const float *>(Pt + 2 * P_BOX + o0),
+                                    *reinterpret_cast<const float *>(Pt + 2 * P_BOX + o1)),
+                                 pk(*reinterpret_cast<const float *>(Pt + 4 * P_BOX + o0),
+                                    *reinterpret_cast<const float *>(Pt + 4 * P_BOX + o1)),
+                                 mul2(ur2, h2), mul2(uz2, h2), mul2(un2, h2), splat(br), splat(bz), splat(bn), ur2,
+                                 uz2, un2, h2, f2, a2, b2);
+                float r0, r1;
+                upk(sub2(pk(y0, y1), f2), r0, r1);
+                upk(a2, av[i], av[i + 1]);
+                upk(b2, bv[i], bv[i + 1]);
+                // steps past the sequence's end (zero-filled rows) are the identity map
                 if (full || t0 + seg * SL + i < T) {
-                    const float pr = *reinterpret_cast<const float *>(Pt + 0 * P_BOX + o);
-                    const float pz = *reinterpret_cast<const float *>(Pt + 2 * P_BOX + o);
-                    const float pn = *reinterpret_cast<const float *>(Pt + 4 * P_BOX + o);
-                    float f;
-                    gru_cell_diag(pr, pz, pn, ur * hp, uz * hp, un * hp, br, bz, bn, ur, uz, un, hp, f, a_, b_);
-                    rmax = max(rmax, abs_bits(y - f));
+                    rmax = max(rmax, abs_bits(r0));
+                } else {
+                    av[i] = 1.f;
+                    bv[i] = 0.f;
                 }
-                av[i] = a_;
-                bv[i] = b_;
-                EB = fmaf(a_, EB, b_);
-                EA = a_ * EA;
-                hp = y;
+                if (full || t0 + seg * SL + i + 1 < T) {
+                    rmax = max(rmax, abs_bits(r1));
+                } else {
+                    av[i + 1] = 1.f;
+                    bv[i + 1] = 0.f;
+                }
+#pragma unroll
+                for (int u = i; u < i + 2; ++u) {
+                    EB = fmaf(av[u], EB, bv[u]);
+                    EA = av[u] * EA;
+                }
+                hp = y1;
             }
             seg_a[seg * DL + d] = EA;
             seg_b[seg * DL + d] = EB;
