@@ -53,12 +53,12 @@ E2E_PARTS = 4  # parts of the batch whose copies the host-buffer solve overlaps
 BENCHES = {
     "untrained": dict(
         workload="untrained", mode="QUASI", lam=0.0, bound="hbm", per_state=20,
-        kernel="quasi_tc2_kernel<64> (persistent, all iterations)",
+        kernel="quasi_tc2_kernel<64, quasi> (persistent, all iterations)",
         desc="untrained dense GRU Din=D=64, B={B}/GPU, T={T}, fp32, quasi-DEER tol 1e-5",
         cpu_sample=dict(B=16, T=1024), ref_sample=dict(B=4, T=256)),
     "diag": dict(
         workload="diag", mode="QUASI", lam=0.0, bound="hbm", per_state=20,
-        kernel="diag_solver_kernel<diag cell, quasi> (persistent, all iterations)",
+        kernel="diag2_kernel (persistent, all iterations)",
         desc="diagonal-recurrence GRU Din=D=2048, B={B}/GPU, T={T}, bf16 x and W_ih, fp32 state, "
              "quasi-DEER (exact Newton) tol 1e-4",
         cpu_sample=dict(B=1, T=1024), ref_sample=dict(B=1, T=128)),
@@ -69,7 +69,7 @@ BENCHES = {
         cpu_sample=dict(B=1, T=4096), ref_sample=dict(B=1, T=512)),
     "quasi_elk": dict(
         workload="near_unstable", mode="QUASI_ELK", lam=0.1, bound="hbm", per_state=56,
-        kernel="diag_solver_kernel<dense cell, quasi-ELK> (persistent, all iterations)",
+        kernel="quasi_tc2_kernel<64, quasi-ELK> (persistent, all iterations)",
         desc="near-unstable dense GRU Din=D=64 (spectral radius 1.5), B={B}/GPU, T={T}, fp32, "
              "quasi-ELK lambda 0.1, tol 1e-4",
         cpu_sample=dict(B=1, T=2000), ref_sample=dict(B=1, T=250)),
@@ -88,8 +88,8 @@ ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # hash of the kernel source it was measured on.  Traffic grows with states x
 # iterations, so the full launch's is scaled from it; reported only while the
 # source is unchanged.
-NCU_TRAFFIC = {"bytes_per_state_iter": (4.176904e9 + 0.991504e9) / (14 * 16 * 16384 * 64),
-               "source_sha1": "3333033a70cf"}
+NCU_TRAFFIC = {"bytes_per_state_iter": (4.052082e9 + 0.991486e9) / (14 * 16 * 16384 * 64),
+               "source_sha1": "f1412c7afeff"}
 
 
 def log(*a):
@@ -130,8 +130,12 @@ def tf32_peak():
 
 
 def kernel_sha():
-    src = os.path.join(ROOT, "newton_solve_nonlinear_b200", "csrc", "newton_dense_tc2.cu")
-    return hashlib.sha1(open(src, "rb").read()).hexdigest()[:12]
+    """Hash of the headline solver kernel's sources (the .cu and the headers it uses)."""
+    csrc = os.path.join(ROOT, "newton_solve_nonlinear_b200", "csrc")
+    h = hashlib.sha1()
+    for f in ("newton_dense_tc2.cu", "common.cuh", "lookback.cuh", "solver.cuh", "tc_utils.cuh"):
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:12]
 
 
 class Clocks:
