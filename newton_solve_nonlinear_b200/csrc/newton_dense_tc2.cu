@@ -277,10 +277,11 @@ __device__ void elk_forward_scans(const DiagArgs &A, const ElkSmem &E, const uns
     float ak[SLE];
     Mob M{1.f, 0.f, 0.f, 1.f};
 #pragma unroll
+    for (int i = 0; i < SLE; ++i)  // all of the segment's a_t in flight at once
+        ak[i] = t0 + s0 + i < T ? __ldcg(A.elk_a + (static_cast<size_t>(row0) + s0 + i) * D + d) : 1.f;
+#pragma unroll
     for (int i = 0; i < SLE; ++i) {
-        const bool valid = t0 + s0 + i < T;
-        ak[i] = valid ? __ldcg(A.elk_a + (static_cast<size_t>(row0) + s0 + i) * D + d) : 1.f;
-        if (valid) {
+        if (t0 + s0 + i < T) {
             const float a2 = ak[i] * ak[i];
             M = mob_mul(Mob{a2, 1.f, lam * a2, 1.f + lam}, M);
         }
