@@ -659,7 +659,8 @@ __global__ void __launch_bounds__(kThreads, 1) deer_mma_kernel(MmaArgs S) {
         last_delta = ld_acquire_u32(&hdr->delta_bits[it % 3]);
         last_resid = ld_acquire_u32(&hdr->resid_bits[it % 3]);
         iters = it + 1;
-        if (timed_out(status)) { final_status = PARARNN_TIMEOUT; break; }
+        // a timeout another CTA raises may land between two threads' reads: decide once per CTA
+        if (__syncthreads_or(timed_out(status))) { final_status = PARARNN_TIMEOUT; break; }
         if (last_delta >= 0x7f800000u) { final_status = PARARNN_DIVERGED; break; }
         if (__uint_as_float(last_delta) <= A.tol) { final_status = PARARNN_OK; break; }
     }

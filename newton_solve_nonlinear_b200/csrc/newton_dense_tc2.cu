@@ -852,7 +852,9 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
             // the smoother runs backward over time once every filter value is written
             grid_barrier(hdr->barrier, nblocks, status);
             const float *hold = A.hbuf[it & 1];
-            for (long long k = 0; k < my_n && !timed_out(status); ++k) {
+            for (long long k = 0; k < my_n; ++k) {
+                // leave on an error or a timeout seen by any thread (uniform decision)
+                if (__syncthreads_or(*cta_err != 0 || timed_out(status))) break;
                 const long long tr = S.n_tiles - 1 - tile_of(k);
                 const int c = static_cast<int>(static_cast<unsigned>(tr) / static_cast<unsigned>(B));
                 elk_backward_tile<D>(A, es, tr, c, static_cast<int>(tr) - c * B, S.n_chunks, epoch,
@@ -870,7 +872,8 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
         last_delta = ld_acquire_u32(&hdr->delta_bits[it % 3]);
         last_resid = ld_acquire_u32(&hdr->resid_bits[it % 3]);
         iters = it + 1;
-        if (*cta_err || timed_out(status)) { final_status = PARARNN_TIMEOUT; break; }
+        // a timeout another CTA raises may land between two threads' reads: decide once per CTA
+        if (__syncthreads_or(*cta_err || timed_out(status))) { final_status = PARARNN_TIMEOUT; break; }
         if (last_delta >= 0x7f800000u) { final_status = PARARNN_DIVERGED; break; }
         if (__uint_as_float(last_delta) <= A.tol) { final_status = PARARNN_OK; break; }
     }

@@ -272,7 +272,8 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
         last_delta = ld_acquire_u32(&hdr->delta_bits[it % 3]);
         last_resid = ld_acquire_u32(&hdr->resid_bits[it % 3]);
         iters = it + 1;
-        if (*cta_err || timed_out(status)) { final_status = PARARNN_TIMEOUT; break; }
+        // a timeout another CTA raises may land between two threads' reads: decide once per CTA
+        if (__syncthreads_or(*cta_err || timed_out(status))) { final_status = PARARNN_TIMEOUT; break; }
         if (last_delta >= 0x7f800000u) { final_status = PARARNN_DIVERGED; break; }
         if (__uint_as_float(last_delta) <= A.tol) { final_status = PARARNN_OK; break; }
     }
