@@ -222,10 +222,36 @@ __device__ __forceinline__ float lookback_mobius(unsigned long long *desc, long 
 // inclusive value last.  Returns the carry into the tile (carry0 when there
 // is no predecessor).  Waits are bounded: a descriptor that never arrives
 // reads as an inclusive 0 and raises the timeout flag.
+// The first window's descriptor words of coop_lookback, read ahead of time
+// (relaxed loads: words that are not ready yet are polled again as usual), so
+// that their round trip overlaps the caller's own work before the look-back.
+template <int R>
+struct LookbackWindow {
+    unsigned long long a[R], b[R];
+};
 template <int G, int R = 1>
+__device__ __forceinline__ LookbackWindow<R> coop_lookback_prefetch(const unsigned long long *desc, long long tile,
+                                                                    long long step, int DG, int d, int q,
+                                                                    int avail) {
+    LookbackWindow<R> w;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        const int p = q * R + r;
+        w.a[r] = w.b[r] = 0ull;
+        if (p < avail) {
+            const unsigned long long *pp = desc + (static_cast<size_t>(tile - (p + 1) * step) * DG + d) * 2;
+            w.a[r] = ld_relaxed(pp);
+            w.b[r] = ld_relaxed(pp + 1);
+        }
+    }
+    return w;
+}
+
+template <int G, int R = 1, bool kPrefetched = false>
 __device__ __forceinline__ float coop_lookback(unsigned long long *desc, long long tile, long long step,
                                                int DG, int d, int q, unsigned epoch, float EA, float EB,
-                                               int avail, float carry0, unsigned *status) {
+                                               int avail, float carry0, unsigned *status,
+                                               const LookbackWindow<R> *pre = nullptr) {
     unsigned long long *mine = desc + (static_cast<size_t>(tile) * DG + d) * 2;
     const int lane = threadIdx.x & 31;
     const int gbase = lane & ~(G - 1);
@@ -247,7 +273,10 @@ __device__ __forceinline__ float coop_lookback(unsigned long long *desc, long lo
             for (int r = 0; r < R; ++r) {
                 const int p = base + q * R + r;
                 wa[r] = wb[r] = 0ull;
-                if (!done && p < avail) {
+                if (kPrefetched && base == 0) {
+                    wa[r] = pre->a[r];
+                    wb[r] = pre->b[r];
+                } else if (!done && p < avail) {
                     const unsigned long long *pp = desc + (static_cast<size_t>(tile - (p + 1) * step) * DG + d) * 2;
                     wa[r] = ld_relaxed(pp);
                     wb[r] = ld_relaxed(pp + 1);

@@ -212,6 +212,8 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
                 }
                 hp = y1;
             }
+            // the predecessors' descriptors, on their way during the barrier
+            const LookbackWindow<1> lbw = coop_lookback_prefetch<SEGS>(A.desc, tile, S.ngroups, DL, ld, lq, chunk);
             seg_a[seg * DL + d] = EA;
             seg_b[seg * DL + d] = EB;
             __syncthreads();
@@ -228,7 +230,8 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
                 }
                 const float c0 = chunk == 0 ? __ldg(A.h0 + static_cast<size_t>(b) * D + lane0 + ld) : 0.f;
                 const float hin =
-                    coop_lookback<SEGS>(A.desc, tile, S.ngroups, DL, ld, lq, epoch, TA, TB, chunk, c0, status);
+                    coop_lookback<SEGS, 1, true>(A.desc, tile, S.ngroups, DL, ld, lq, epoch, TA, TB, chunk, c0,
+                                                 status, &lbw);
                 if (lq == 0) carry[ld] = hin;
             }
             __syncthreads();
