@@ -19,6 +19,9 @@ What it states, plainly and slowly, in float64:
                    and a sequential Kalman filter + RTS smoother.
   * ``brute``   -- dense (T*D) x (T*D) assemblies for tiny T, used only to pin
                    the structured solvers above.
+  * ``adjoint`` -- the backward pass: gradients of a loss through the evaluated
+                   states (reverse-time recurrence with J^T, exact or with the
+                   diagonal of J), and the parameter and input gradients.
 
 Pins (tests marked "not gpu") tie each part to something other than itself:
 ``torch.nn.GRUCell`` (a library routine), central finite differences, closed
@@ -27,7 +30,7 @@ dense solves, and invariants the pages state (Newton is exact on an affine
 cell; undamped Newton recovers one more exact state per iteration).  The pages
 print no worked numeric example, so nothing here is pinned to printed values.
 """
-from . import cells, scan, newton, elk, brute  # noqa: F401
+from . import cells, scan, newton, elk, brute, adjoint  # noqa: F401
 from .cells import GRU, rollout  # noqa: F401
 from .newton import newton_solve, STATUS_OK, STATUS_NOT_CONVERGED, STATUS_DIVERGED  # noqa: F401
 from .elk import elk_solve  # noqa: F401

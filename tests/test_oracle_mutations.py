@@ -75,3 +75,49 @@ def test_inverted_damping_convention(monkeypatch):
     orig = elk.lm_step_normal
     monkeypatch.setattr(elk, "lm_step_normal", lambda A, b, y, h0, lam: orig(A, b, y, h0, 1.0 / lam))
     _fails(pins.test_lm_limits, False)
+
+
+# ---------------------------------------------------------- backward pass --
+import oracle.adjoint as adj  # noqa: E402
+import tests.test_oracle_adjoint as adj_pins  # noqa: E402
+
+
+def test_adjoint_without_transpose(monkeypatch):
+    """J_t instead of J_t^T in the lam recurrence."""
+    orig = cells.GRU.jacobian
+
+    def bad(self, h, p):
+        f, J = orig(self, h, p)
+        return f, np.swapaxes(J, -1, -2)
+    monkeypatch.setattr(cells.GRU, "jacobian", bad)
+    _fails(adj_pins.test_exact_adjoint_equals_autograd, "dense")
+
+
+def test_adjoint_dropped_reset_factor(monkeypatch):
+    """The n gate's recurrent gradient without its reset-gate factor."""
+    orig = adj.step_partials
+
+    def bad(cell, h_prev, p):
+        fr, fz, fn, r, f = orig(cell, h_prev, p)
+        return fr, fz, fn, np.ones_like(r), f
+    monkeypatch.setattr(adj, "step_partials", bad)
+    _fails(adj_pins.test_exact_adjoint_equals_autograd, "diag")
+
+
+def test_adjoint_unshifted_previous_state(monkeypatch):
+    """Partials evaluated at h_t instead of h_{t-1}."""
+    def bad(cell, x, h0, h, g, jacobian="exact"):
+        B, T, _ = x.shape
+        P = cell.project(x)
+        lam = np.zeros_like(h)
+        carry = np.zeros((B, cell.d))
+        for t in range(T - 1, -1, -1):
+            lam[:, t] = g[:, t] + carry
+            _, a = cell.jacobian_diag(h[:, t], P[:, t])
+            carry = a * lam[:, t]
+        out = dict(lam=lam, dh0=carry)
+        for k in ("dx", "dw_ih", "db_ih", "dw_hh", "db_hh", "dP"):
+            out[k] = np.zeros(1)
+        return out
+    monkeypatch.setattr(adj_pins, "adjoint", bad)
+    _fails(adj_pins.test_diag_cell_quasi_backward_is_exact)
