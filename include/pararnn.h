@@ -318,6 +318,55 @@ PARARNN_API int pararnn_affine_scan_noalloc(const float *A, const float *b, cons
                                             int B, int T, int D, float *h,
                                             unsigned *status_dev, pararnn_stream stream);
 
+/*
+ * pararnn_adjoint -- the backward pass through an evaluated sequence of the
+ * diagonal-recurrence GRU (cell->kind == PARARNN_GRU_DIAG): the gradients of
+ * a loss L with respect to the input pre-activations, the initial state and
+ * the recurrent parameters, given the states and the upstream gradients.
+ *
+ * The pages train the evaluated RNN with the diagonal Jacobian in the backward
+ * pass ("Towards Scalable and Stable Parallelization of Nonlinear RNNs", atlas
+ * summary, table "Measured effects reported in the paper"); for this cell that
+ * Jacobian is exact, so the results are the exact gradients.  With
+ * a_t = df_t/dh_{t-1} (diagonal) and g_t = dh[t], the total derivatives
+ * lam_t = dL/dh_t solve lam_T = g_T, lam_t = g_t + a_{t+1} lam_{t+1} (one
+ * reverse pass with decoupled look-back), and then per (b, t, i):
+ *   dP[b,t,i]     = lam (1-z)(1-n^2) g r(1-r)      (reset-gate pre-activation)
+ *   dP[b,t,D+i]   = lam (h_{t-1} - n) z(1-z)       (update gate)
+ *   dP[b,t,2D+i]  = lam (1-z)(1-n^2)               (candidate), g = u_n h_{t-1} + b_hn
+ *   dh0[b,i]      = a_1 lam_1
+ *   dw_hh[k*D+i]  = sum_{b,t} (r: dP_r, z: dP_z, n: dP_n r) * h_{t-1}    (k = r, z, n)
+ *   db_hh[k*D+i]  = sum_{b,t} (dP_r, dP_z, dP_n r)
+ * The input projection's gradients follow from dP by plain GEMMs the caller
+ * runs (dx = dP W_ih, dW_ih = dP^T x, db_ih = sum dP); they are not computed
+ * here.  Sums are taken in a fixed order: results are deterministic.
+ *
+ *   cell, params  params->w_hh (the vectors u_r, u_z, u_n, [3D]) and
+ *                 params->b_hh [3D] are read; the input weights are not.
+ *   P   DEVICE [B, T, 3D] fp32 input pre-activations (pararnn_input_projection).
+ *   h0  DEVICE [B, D];  h DEVICE [B, T, D] the evaluated states (a converged
+ *       solve or a rollout);  dh DEVICE [B, T, D] the upstream gradients dL/dh.
+ *   dP  DEVICE [B, T, 3D] out;  dh0 DEVICE [B, D] out;  dw_hh, db_hh DEVICE [3D] out.
+ *   workspace  DEVICE, >= pararnn_adjoint_workspace_size bytes, 256-byte aligned.
+ * All device pointers 16-byte aligned; outputs must not overlap inputs or the
+ * workspace.  Asynchronous: enqueues on `stream` and returns PARARNN_OK,
+ * INVALID_ARG or CUDA_ERROR; pararnn_adjoint_status reports a device timeout.
+ */
+PARARNN_API int pararnn_adjoint(const pararnn_cell *cell, const pararnn_params *params, const float *P,
+                                const float *h0, const float *h, const float *dh, int B, int T, float *dP,
+                                float *dh0, float *dw_hh, float *db_hh, void *workspace, size_t ws_bytes,
+                                pararnn_stream stream);
+
+/* pararnn_adjoint_workspace_size -- bytes of workspace pararnn_adjoint needs
+ * (about 0.25 B + 0.02 B per state of B*T*D plus 256), or 0 when the
+ * arguments are rejected (not the diagonal cell, B, T or D < 1). */
+PARARNN_API size_t pararnn_adjoint_workspace_size(const pararnn_cell *cell, int B, int T);
+
+/* pararnn_adjoint_status -- wait for `stream` and read the status the last
+ * pararnn_adjoint using `workspace` left: PARARNN_OK, or PARARNN_TIMEOUT if a
+ * bounded device-side wait expired (results unreliable). */
+PARARNN_API int pararnn_adjoint_status(const void *workspace, pararnn_stream stream);
+
 /* pararnn_status_string -- a static, human-readable name of a status code. */
 PARARNN_API const char *pararnn_status_string(int status);
 

@@ -25,7 +25,8 @@ EXPORTS = ("pararnn_workspace_size", "pararnn_newton_solve", "pararnn_newton_sol
            "pararnn_input_projection", "pararnn_newton_iterate_async",
            "pararnn_affine_scan_workspace_size", "pararnn_affine_scan",
            "pararnn_affine_scan_status", "pararnn_status_string", "pararnn_newton_solve_host",
-           "pararnn_host_workspace_size")
+           "pararnn_host_workspace_size", "pararnn_adjoint", "pararnn_adjoint_workspace_size",
+           "pararnn_adjoint_status")
 
 
 class Cell(ctypes.Structure):
@@ -79,6 +80,13 @@ def lib() -> ctypes.CDLL:
         L.pararnn_newton_solve_host.restype = ci
         L.pararnn_host_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci, ci, ci]
         L.pararnn_host_workspace_size.restype = sz
+        L.pararnn_adjoint.argtypes = [ctypes.POINTER(Cell), ctypes.POINTER(Params), vp, vp, vp, vp, ci, ci,
+                                      vp, vp, vp, vp, vp, sz, vp]
+        L.pararnn_adjoint.restype = ci
+        L.pararnn_adjoint_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci]
+        L.pararnn_adjoint_workspace_size.restype = sz
+        L.pararnn_adjoint_status.argtypes = [vp, vp]
+        L.pararnn_adjoint_status.restype = ci
         L.pararnn_status_string.argtypes = [ci]
         L.pararnn_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -220,6 +228,42 @@ def newton_solve_host(w_ih, b_ih, w_hh, b_hh, x_host, h0_host, *, kind: str, mod
     if rc in (3, 4):
         raise RuntimeError(f"pararnn_newton_solve_host: {L.pararnn_status_string(rc).decode()}")
     return SolveResult(out, info.iters, STATUS[info.status], info.delta, info.residual)
+
+
+def adjoint_workspace_size(d: int, B: int, T: int, kind: str = "diag") -> int:
+    cell = make_cell(kind, 1, d, torch.float32)
+    return int(lib().pararnn_adjoint_workspace_size(ctypes.byref(cell), B, T))
+
+
+def adjoint(w_hh, b_hh, P, h0, h, dh, *, workspace=None, out=None, stream=None, check: bool = False) -> dict:
+    """Backward pass of the diagonal-recurrence GRU through the states h:
+    gradients w.r.t. the pre-activations P [B,T,3D], h0 [B,D], the recurrent
+    vectors w_hh [3D] and b_hh [3D], given dh = dL/dh [B,T,D] (all fp32 CUDA).
+    Returns dict(dP, dh0, dw_hh, db_hh)."""
+    B, T, d = h.shape
+    cell = make_cell("diag", 1, d, torch.float32)
+    L = lib()
+    need = int(L.pararnn_adjoint_workspace_size(ctypes.byref(cell), B, T))
+    if need == 0:
+        raise ValueError("arguments rejected by pararnn_adjoint_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, h.device)
+    o = out or {}
+    dP = o.get("dP", torch.empty_like(P))
+    dh0 = o.get("dh0", torch.empty_like(h0))
+    dw = o.get("dw_hh", torch.empty_like(w_hh))
+    db = o.get("db_hh", torch.empty_like(b_hh))
+    params = Params(None, None, _dev(w_hh, "w_hh"), _dev(b_hh, "b_hh"))
+    rc = L.pararnn_adjoint(ctypes.byref(cell), ctypes.byref(params), _dev(P, "P"), _dev(h0, "h0"), _dev(h, "h"),
+                           _dev(dh, "dh"), B, T, _dev(dP, "dP"), _dev(dh0, "dh0"), _dev(dw, "dw_hh"),
+                           _dev(db, "db_hh"), _dev(workspace, "workspace"), workspace.numel(), _stream(stream))
+    if rc != 0:
+        raise RuntimeError(f"pararnn_adjoint: {L.pararnn_status_string(rc).decode()}")
+    if check:
+        st = L.pararnn_adjoint_status(_dev(workspace, "workspace"), _stream(stream))
+        if st != 0:
+            raise RuntimeError(f"pararnn_adjoint: {STATUS.get(st, st)}")
+    return dict(dP=dP, dh0=dh0, dw_hh=dw, db_hh=db)
 
 
 def input_projection(x, w_ih, b_ih, *, d: int, kind: str = "dense", out=None, stream=None):

@@ -1,0 +1,249 @@
+// adjoint_diag.cu -- the backward pass through an evaluated sequence of the
+// diagonal-recurrence GRU: gradients of a loss with respect to the input
+// pre-activations, the initial state and the recurrent parameters.
+//
+// Method: the pages train the evaluated RNN with the diagonal Jacobian in the
+// backward pass ("Towards Scalable and Stable Parallelization of Nonlinear
+// RNNs", atlas summary, table "Measured effects reported in the paper"); for
+// the diagonal-recurrence cell (the "adapted" GRU of the ParaRNN talk page,
+// "Federico Danieli", Abstract) that Jacobian is exact.  The chain rule on the
+// unrolled system h_t = f(h_{t-1}, p_t) gives, backwards in time,
+//     lam_t = g_t + a_{t+1} lam_{t+1},   lam_T = g_T,
+// a_t = df_t/dh_{t-1} (diagonal), g_t = dL/dh_t the upstream gradient: a
+// reverse affine recurrence, solved in one pass with decoupled look-back over
+// the later chunks.  Then per state (lane i of step t, previous state hp):
+//     dL/dp_r = lam (1-z)(1-n^2) g r (1-r),  dL/dp_z = lam (hp - n) z (1-z),
+//     dL/dp_n = lam (1-z)(1-n^2),            dL/dh_0 = a_1 lam_1,
+//     dL/du_r = sum lam (1-z)(1-n^2) g r(1-r) hp,  dL/du_z = sum lam (hp-n) z(1-z) hp,
+//     dL/du_n = sum lam (1-z)(1-n^2) r hp,  dL/db_hh likewise without hp.
+//
+// One cooperative launch: CTAs of 256 threads walk tiles of (sequence, 64
+// lanes, 32 steps) from the last chunk to the first.  Thread (lane d, segment
+// s) evaluates the cell at its 8 steps and the next one (for a_{t+1}), folds
+// its steps' maps in reverse, the four segments of a lane chain through shared
+// memory, the tile takes lam at its end from a cooperative look-back over
+// later chunks, and the sweep writes dL/dP and the per-tile partial sums of
+// the parameter gradients.  After a grid barrier every warp reduces some of
+// those partials in a fixed order (deterministic results).
+// Traffic per state: P (12 B), h (4 B), dL/dh (4 B) read; dL/dP (12 B) written.
+#include "common.cuh"
+#include "lookback.cuh"
+#include "solver.cuh"
+
+namespace pararnn {
+namespace {
+
+constexpr int ATS = 32;            // steps per tile
+constexpr int ADL = 64;            // lanes per tile
+constexpr int ANT = 256;           // threads: lane x 4 segments
+constexpr int ASEGS = ANT / ADL;   // 4 segments
+constexpr int ASL = ATS / ASEGS;   // 8 steps per thread
+
+struct AdjArgs {
+    const float *P, *h0, *h, *dh, *u, *b_hh;  // u: [3D] recurrent vectors (r, z, n)
+    float *dP, *dh0, *du, *db_hh;
+    WsHeader *hdr;
+    unsigned long long *desc;  // [n_tiles][ADL][2] look-back words
+    float *part;               // [n_tiles][6][ADL] per-tile partial sums
+    int B, T, D, ndg, ngroups, n_chunks;
+    long long n_tiles;
+};
+
+// One step of the diagonal cell at (hp, p): the partials of f with respect to
+// the three pre-activations, r, and a = df/dh_{t-1}.
+__device__ __forceinline__ void adj_cell(float pr, float pz, float pn, float hp, float ur, float uz, float un,
+                                         float br, float bz, float bn, float &fr, float &fz, float &fn,
+                                         float &r, float &a) {
+    r = sigmoidf_(pr + ur * hp + br);
+    const float z = sigmoidf_(pz + uz * hp + bz);
+    const float g = un * hp + bn;
+    const float n = tanhf_(pn + r * g);
+    fn = (1.f - z) * (1.f - n * n);
+    fr = fn * g * r * (1.f - r);
+    fz = (hp - n) * z * (1.f - z);
+    a = z + fz * uz + fn * r * un + fr * ur;
+}
+
+__global__ void __launch_bounds__(ANT, 2) adjoint_diag_kernel(AdjArgs S) {
+    __shared__ float seg_a[ASEGS][ADL], seg_b[ASEGS][ADL];
+    __shared__ float carry[ADL];
+    __shared__ float red6[ASEGS][6][ADL];
+    const int T = S.T, D = S.D;
+    unsigned *status = &S.hdr->status;
+    const int tid = threadIdx.x;
+    const int d = tid & (ADL - 1), seg = tid / ADL;  // sweep role
+    const int ld = tid / ASEGS, lq = tid % ASEGS;    // look-back role
+    const unsigned nblocks = gridDim.x;
+    const unsigned epoch = 1u;
+
+    for (long long v = blockIdx.x; v < S.n_tiles; v += nblocks) {
+        // processing order: last chunk first; v - ngroups is the same lanes one chunk later
+        const unsigned v32 = static_cast<unsigned>(v), ng = static_cast<unsigned>(S.ngroups);
+        const int cidx = static_cast<int>(v32 / ng);
+        const int grp = static_cast<int>(v32 - static_cast<unsigned>(cidx) * ng);
+        const int chunk = S.n_chunks - 1 - cidx;
+        const int b = grp / S.ndg, dg = grp - (grp / S.ndg) * S.ndg;
+        const int t0 = chunk * ATS;
+        const int lane = dg * ADL + d;
+        const bool lane_ok = lane < D;
+        const size_t row0 = static_cast<size_t>(b) * T;
+
+        float ur = 0.f, uz = 0.f, un = 0.f, br = 0.f, bz = 0.f, bn = 0.f;
+        if (lane_ok) {
+            ur = __ldg(S.u + lane), uz = __ldg(S.u + D + lane), un = __ldg(S.u + 2 * D + lane);
+            br = __ldg(S.b_hh + lane), bz = __ldg(S.b_hh + D + lane), bn = __ldg(S.b_hh + 2 * D + lane);
+        }
+        // 1. the cell at the thread's 8 steps and the next one
+        float fr[ASL], fz[ASL], fn[ASL], rr[ASL], hp[ASL], gg[ASL], al[ASL];
+        float a_first = 0.f;
+        {
+            float pr[ASL + 1], pz[ASL + 1], pn[ASL + 1], hv[ASL + 1];
+#pragma unroll
+            for (int i = 0; i <= ASL; ++i) {  // all loads in flight together
+                const int t = t0 + seg * ASL + i;
+                const bool ok = lane_ok && t < T;
+                const size_t o = (row0 + t) * 3 * D + lane;
+                pr[i] = ok ? __ldcs(S.P + o) : 0.f;
+                pz[i] = ok ? __ldcs(S.P + o + D) : 0.f;
+                pn[i] = ok ? __ldcs(S.P + o + 2 * D) : 0.f;
+                hv[i] = ok ? (t == 0 ? __ldg(S.h0 + static_cast<size_t>(b) * D + lane)
+                                     : __ldcs(S.h + (row0 + t - 1) * D + lane))
+                           : 0.f;
+                if (i < ASL) gg[i] = ok ? __ldcs(S.dh + (row0 + t) * D + lane) : 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i <= ASL; ++i) {
+                const int t = t0 + seg * ASL + i;
+                float f_r, f_z, f_n, r_, a_;
+                adj_cell(pr[i], pz[i], pn[i], hv[i], ur, uz, un, br, bz, bn, f_r, f_z, f_n, r_, a_);
+                if (i < ASL) {
+                    fr[i] = f_r, fz[i] = f_z, fn[i] = f_n, rr[i] = r_, hp[i] = hv[i];
+                    if (i == 0) a_first = a_;
+                }
+                // a_{t} of step i is the coefficient of lam_i in lam_{i-1}
+                if (i > 0) al[i - 1] = (lane_ok && t < T) ? a_ : 0.f;
+            }
+        }
+        // 2. this segment's reverse map: lam_i = A_i lam_after + B_i
+        float Ai[ASL], Bi[ASL];
+        {
+            float A = 1.f, Bv = 0.f;
+#pragma unroll
+            for (int i = ASL - 1; i >= 0; --i) {
+                Bv = fmaf(al[i], Bv, gg[i]);
+                A = al[i] * A;
+                Ai[i] = A;
+                Bi[i] = Bv;
+            }
+        }
+        const LookbackWindow<1> lbw = coop_lookback_prefetch<ASEGS>(S.desc, v, S.ngroups, ADL, ld, lq, cidx);
+        seg_a[seg][d] = Ai[0];
+        seg_b[seg][d] = Bi[0];
+        __syncthreads();
+        // 3. lam at the tile's end (step t0 + 32) by look-back over later chunks
+        {
+            float TA = 1.f, TB = 0.f;  // the tile: lam_{t0} = TA lam_{t0+32} + TB
+#pragma unroll
+            for (int q = ASEGS - 1; q >= 0; --q) {
+                TB = fmaf(seg_a[q][ld], TB, seg_b[q][ld]);
+                TA = seg_a[q][ld] * TA;
+            }
+            const float lin =
+                coop_lookback<ASEGS, 1, true>(S.desc, v, S.ngroups, ADL, ld, lq, epoch, TA, TB, cidx, 0.f, status, &lbw);
+            if (lq == 0) carry[ld] = lin;
+        }
+        __syncthreads();
+        // 4. sweep: lam after this segment, then its steps; dL/dP and partial sums
+        float s_r = 0.f, s_z = 0.f, s_n = 0.f, q_r = 0.f, q_z = 0.f, q_n = 0.f;
+        {
+            float lam_after = carry[d];
+            for (int q = ASEGS - 1; q > seg; --q) lam_after = fmaf(seg_a[q][d], lam_after, seg_b[q][d]);
+#pragma unroll
+            for (int i = 0; i < ASL; ++i) {
+                const int t = t0 + seg * ASL + i;
+                if (lane_ok && t < T) {
+                    const float lam = fmaf(Ai[i], lam_after, Bi[i]);
+                    const float gr = fr[i] * lam, gz = fz[i] * lam, gn = fn[i] * lam, gnr = gn * rr[i];
+                    const size_t o = (row0 + t) * 3 * D + lane;
+                    __stcs(S.dP + o, gr);
+                    __stcs(S.dP + o + D, gz);
+                    __stcs(S.dP + o + 2 * D, gn);
+                    q_r += gr, q_z += gz, q_n += gnr;
+                    s_r = fmaf(gr, hp[i], s_r), s_z = fmaf(gz, hp[i], s_z), s_n = fmaf(gnr, hp[i], s_n);
+                    if (t == 0) S.dh0[static_cast<size_t>(b) * D + lane] = a_first * lam;
+                }
+            }
+        }
+        red6[seg][0][d] = s_r, red6[seg][1][d] = s_z, red6[seg][2][d] = s_n;
+        red6[seg][3][d] = q_r, red6[seg][4][d] = q_z, red6[seg][5][d] = q_n;
+        __syncthreads();
+        for (int i = tid; i < 6 * ADL; i += ANT) {  // per-tile partials, segments summed in order
+            const int k = i / ADL, dd = i % ADL;
+            S.part[(static_cast<size_t>(v) * 6 + k) * ADL + dd] =
+                ((red6[0][k][dd] + red6[1][k][dd]) + red6[2][k][dd]) + red6[3][k][dd];
+        }
+        __syncthreads();  // shared arrays are rewritten by the next tile
+    }
+
+    // 5. parameter gradients: each warp sums one (quantity, lane) over the tiles
+    // of that lane group, always in the same order
+    grid_barrier(S.hdr->barrier, nblocks, status);
+    const int warp = tid >> 5, wl = tid & 31;
+    const long long nwarps = static_cast<long long>(nblocks) * (ANT / 32);
+    const int per_group = S.n_chunks * S.B;  // tiles of one lane group
+    for (long long o = static_cast<long long>(blockIdx.x) * (ANT / 32) + warp; o < 6ll * D; o += nwarps) {
+        const int k = static_cast<int>(o / D), lane = static_cast<int>(o % D);
+        const int dg = lane / ADL, dd = lane % ADL;
+        float acc = 0.f;
+        for (int j = wl; j < per_group; j += 32) {
+            const int cidx = j / S.B, bb = j - cidx * S.B;
+            const long long v = static_cast<long long>(cidx) * S.ngroups + bb * S.ndg + dg;
+            acc += __ldcg(S.part + (static_cast<size_t>(v) * 6 + k) * ADL + dd);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (wl == 0) {
+            float *dst = k < 3 ? S.du : S.db_hh;
+            dst[(k % 3) * D + lane] = acc;
+        }
+    }
+}
+
+}  // namespace
+
+size_t adjoint_diag_desc_bytes(int B, int T, int D) {
+    const long long tiles = static_cast<long long>(B) * ((D + ADL - 1) / ADL) * ((T + ATS - 1) / ATS);
+    return static_cast<size_t>(tiles) * ADL * 2 * 8;
+}
+size_t adjoint_diag_part_bytes(int B, int T, int D) {
+    const long long tiles = static_cast<long long>(B) * ((D + ADL - 1) / ADL) * ((T + ATS - 1) / ATS);
+    return static_cast<size_t>(tiles) * 6 * ADL * 4;
+}
+
+cudaError_t launch_adjoint_diag(const float *P, const float *h0, const float *h, const float *dh, const float *u,
+                                const float *b_hh, float *dP, float *dh0, float *du, float *db_hh, int B, int T,
+                                int D, void *hdr, void *desc, void *part, cudaStream_t s) {
+    AdjArgs S;
+    S.P = P, S.h0 = h0, S.h = h, S.dh = dh, S.u = u, S.b_hh = b_hh;
+    S.dP = dP, S.dh0 = dh0, S.du = du, S.db_hh = db_hh;
+    S.hdr = static_cast<WsHeader *>(hdr);
+    S.desc = static_cast<unsigned long long *>(desc);
+    S.part = static_cast<float *>(part);
+    S.B = B, S.T = T, S.D = D;
+    S.ndg = (D + ADL - 1) / ADL;
+    S.ngroups = B * S.ndg;
+    S.n_chunks = (T + ATS - 1) / ATS;
+    S.n_tiles = static_cast<long long>(S.ngroups) * S.n_chunks;
+    int dev = 0, nsm = 0, per_sm = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adjoint_diag_kernel, ANT, 0);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    long long grid = static_cast<long long>(nsm) * per_sm;
+    void *params[] = {&S};
+    return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(adjoint_diag_kernel),
+                                       dim3(static_cast<unsigned>(grid)), dim3(ANT), params, 0, s);
+}
+
+}  // namespace pararnn

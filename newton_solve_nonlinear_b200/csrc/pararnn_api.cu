@@ -32,6 +32,11 @@ cudaError_t launch_diag2(const DiagArgs &a, cudaStream_t s);
 cudaError_t launch_scan_dense(const float *A, const float *b, const float *h0, int B, int T,
                               int D, float *h, void *ws, cudaStream_t s);
 size_t scan_dense_ws_bytes(int B, int T, int D);
+size_t adjoint_diag_desc_bytes(int B, int T, int D);
+size_t adjoint_diag_part_bytes(int B, int T, int D);
+cudaError_t launch_adjoint_diag(const float *P, const float *h0, const float *h, const float *dh, const float *u,
+                                const float *b_hh, float *dP, float *dh0, float *du, float *db_hh, int B, int T,
+                                int D, void *hdr, void *desc, void *part, cudaStream_t s);
 
 namespace {
 
@@ -300,6 +305,66 @@ int pararnn_affine_scan_status(const void *workspace, pararnn_stream stream) {
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
     return (st & kStatusTimeout) ? PARARNN_TIMEOUT : PARARNN_OK;
+}
+
+// ---- backward pass (diagonal cell) -------------------------------------------
+
+namespace {
+struct AdjLayout {
+    size_t header, desc, part, total;
+};
+AdjLayout adj_layout(int B, int T, int D) {
+    AdjLayout L{};
+    size_t off = 0;
+    L.header = off; off += 256;
+    L.desc = off; off = align256(off + adjoint_diag_desc_bytes(B, T, D));
+    L.part = off; off = align256(off + adjoint_diag_part_bytes(B, T, D));
+    L.total = off;
+    return L;
+}
+}  // namespace
+
+size_t pararnn_adjoint_workspace_size(const pararnn_cell *cell, int B, int T) {
+    if (!cell || cell->kind != PARARNN_GRU_DIAG || cell->d < 1 || B < 1 || T < 1) return 0;
+    if (static_cast<long long>(B) * T >= (1ll << 31) - 1) return 0;
+    return adj_layout(B, T, cell->d).total;
+}
+
+int pararnn_adjoint(const pararnn_cell *cell, const pararnn_params *params, const float *P, const float *h0,
+                    const float *h, const float *dh, int B, int T, float *dP, float *dh0, float *dw_hh,
+                    float *db_hh, void *workspace, size_t ws_bytes, pararnn_stream stream) {
+    const size_t need = pararnn_adjoint_workspace_size(cell, B, T);
+    if (need == 0 || ws_bytes < need || !params || !params->w_hh || !params->b_hh) return PARARNN_INVALID_ARG;
+    if (!P || !h0 || !h || !dh || !dP || !dh0 || !dw_hh || !db_hh || !workspace) return PARARNN_INVALID_ARG;
+    const void *ptrs[] = {P, h0, h, dh, dP, dh0, dw_hh, db_hh, params->w_hh, params->b_hh};
+    for (const void *q : ptrs)
+        if (!aligned(q, 16)) return PARARNN_INVALID_ARG;
+    if (!aligned(workspace, 256)) return PARARNN_INVALID_ARG;
+    const int D = cell->d;
+    const size_t st = static_cast<size_t>(B) * T * D * 4;
+    const size_t bd = static_cast<size_t>(B) * D * 4, pd = static_cast<size_t>(3) * D * 4;
+    const struct { const void *p; size_t n; } ins[] = {{P, 3 * st}, {h0, bd}, {h, st}, {dh, st},
+                                                       {params->w_hh, pd}, {params->b_hh, pd}, {workspace, need}};
+    const struct { const void *p; size_t n; } outs[] = {{dP, 3 * st}, {dh0, bd}, {dw_hh, pd}, {db_hh, pd}};
+    for (const auto &o : outs) {
+        for (const auto &i : ins)
+            if (overlaps(o.p, o.n, i.p, i.n)) return PARARNN_INVALID_ARG;
+        for (const auto &o2 : outs)
+            if (&o2 != &o && overlaps(o.p, o.n, o2.p, o2.n)) return PARARNN_INVALID_ARG;
+    }
+    const AdjLayout L = adj_layout(B, T, D);
+    char *ws = static_cast<char *>(workspace);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // header (status, grid barrier) and look-back words start at zero
+    cudaError_t e = cudaMemsetAsync(ws, 0, L.part, s);
+    if (e == cudaSuccess)
+        e = launch_adjoint_diag(P, h0, h, dh, params->w_hh, params->b_hh, dP, dh0, dw_hh, db_hh, B, T, D,
+                                ws + L.header, ws + L.desc, ws + L.part, s);
+    return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
+}
+
+int pararnn_adjoint_status(const void *workspace, pararnn_stream stream) {
+    return pararnn_affine_scan_status(workspace, stream);
 }
 
 const char *pararnn_status_string(int status) {

@@ -1,0 +1,128 @@
+"""GPU parity of the backward pass (diagonal-recurrence GRU) vs the fp64 oracle.
+
+Inputs: a random diagonal cell, synthetic fp32 pre-activations P, the fp64
+rollout of the cell from P (rounded to fp32), and random upstream gradients.
+The oracle sees exactly the same (fp32-valued) arrays: it runs with an
+identity input projection, so its x is P.
+
+Tolerance: normwise, ||got - want||_inf <= 1e-4 ||want||_inf for dP and dh0
+(lam accumulates T fp32 steps of a_t lam + g) and 1e-4 for the parameter sums
+over B*T terms; the kernel's exponentials carry ~1e-7 relative error.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle.adjoint import adjoint as oracle_adjoint
+from oracle.cells import GRU
+from newton_solve_nonlinear_b200 import binding
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(B, T, D, seed, u_range=0.9):
+    g = torch.Generator().manual_seed(seed)
+    u = (torch.rand(3 * D, generator=g) * 2 - 1) * u_range
+    b_hh = torch.randn(3 * D, generator=g) * 0.3
+    P = torch.randn(B, T, 3 * D, generator=g)
+    h0 = torch.randn(B, D, generator=g) * 0.5
+    dh = torch.randn(B, T, D, generator=g)
+    # the oracle's own cell, fed P directly (identity input projection)
+    cell = GRU(kind="diag", w_ih=np.zeros((3 * D, 0)), b_ih=np.zeros(3 * D), w_hh=u.double().numpy(),
+               b_hh=b_hh.double().numpy())
+    Pd = P.double().numpy()
+    hs, hv = [], h0.double().numpy()
+    for t in range(T):  # the rollout h_t = f(h_{t-1}, p_t) through the oracle's gates
+        hv = cell.gates(hv, Pd[:, t])[4]
+        hs.append(hv)
+    h = torch.from_numpy(np.stack(hs, 1)).float()
+    return cell, u, b_hh, P, h0, h, dh
+
+
+def _identity_cell(cell, idx3=None):
+    w = cell.w_hh if idx3 is None else cell.w_hh[idx3]
+    b = cell.b_hh if idx3 is None else cell.b_hh[idx3]
+    return GRU(kind="diag", w_ih=np.eye(len(w)), b_ih=np.zeros(len(w)), w_hh=w, b_hh=b)
+
+
+def _rel(got, want):
+    return float(np.max(np.abs(got - want)) / max(np.max(np.abs(want)), 1e-30))
+
+
+def _check(B, T, D, seed, lanes=None):
+    cell, u, b_hh, P, h0, h, dh = _case(B, T, D, seed)
+    r = binding.adjoint(u.cuda(), b_hh.cuda(), P.cuda(), h0.cuda(), h.cuda(), dh.cuda(), check=True)
+    f64 = lambda t: t.double().numpy()
+    if lanes is None:
+        ref = oracle_adjoint(_identity_cell(cell), f64(P), f64(h0), f64(h), f64(dh), jacobian="diag")
+        sel, sel3 = slice(None), slice(None)
+    else:  # the diagonal cell is separable by lane: the oracle on a subset of lanes
+        idx = np.asarray(lanes)
+        idx3 = np.concatenate([idx, D + idx, 2 * D + idx])
+        ref = oracle_adjoint(_identity_cell(cell, idx3), f64(P)[..., idx3], f64(h0)[:, idx], f64(h)[..., idx], f64(dh)[..., idx],
+                             jacobian="diag")
+        sel, sel3 = idx, idx3
+    got = {k: v.double().cpu().numpy() for k, v in r.items()}
+    assert _rel(got["dP"][..., sel3], ref["dP"]) <= 1e-4
+    assert _rel(got["dh0"][:, sel], ref["dh0"]) <= 1e-4
+    assert _rel(got["dw_hh"][sel3], ref["dw_hh"]) <= 1e-4
+    assert _rel(got["db_hh"][sel3], ref["db_hh"]) <= 1e-4
+
+
+@pytest.mark.parametrize("B,T,D", [(2, 100, 64), (3, 257, 96), (1, 1, 5), (2, 33, 130), (1, 64, 64),
+                                   (4, 1000, 128)])
+def test_adjoint_matches_oracle(B, T, D):
+    _check(B, T, D, seed=B * 1000 + T + D)
+
+
+def test_adjoint_full_size_sampled_lanes():
+    """The diagonal workload's size (B = 8, T = 4096, D = 2048), the oracle on 96 lanes."""
+    _check(8, 4096, 2048, seed=7, lanes=list(range(0, 2048, 64)) + list(range(1000, 1064)))
+
+
+def test_adjoint_deterministic_and_rejects_dense():
+    cell, u, b_hh, P, h0, h, dh = _case(2, 300, 64, seed=3)
+    args = [t.cuda() for t in (u, b_hh, P, h0, h, dh)]
+    r1 = binding.adjoint(*args)
+    r2 = binding.adjoint(*args)
+    for k in r1:
+        assert torch.equal(r1[k], r2[k]), k
+    assert binding.adjoint_workspace_size(64, 2, 300, kind="dense") == 0
+
+
+def test_adjoint_gives_autograd_gradients_of_a_solve():
+    """End to end on the GPU: solve the diagonal GRU with exact Newton, take the
+    backward pass, and form the input gradients with plain GEMMs; compare with
+    torch autograd of an fp64 rollout on the CPU (a library routine)."""
+    from newton_solve_nonlinear_b200.inputs import make_workload
+    w = make_workload("diag", B=2, T=300, d=64, din=48, x_dtype=torch.float32, w_dtype=torch.float32,
+                      bias_std=0.2, h0_std=0.5)
+    dev = lambda t: t.cuda().contiguous()
+    sol = binding.solve_workload(w, "QUASI", tol=1e-6)
+    assert sol.status == "OK"
+    P = binding.input_projection(dev(w.x), dev(w.w_ih), dev(w.b_ih), d=64, kind="diag")
+    gen = torch.Generator().manual_seed(5)
+    dh = torch.randn(2, 300, 64, generator=gen)
+    r = binding.adjoint(dev(w.w_hh), dev(w.b_hh), P, dev(w.h0), sol.h, dh.cuda())
+    dx = (r["dP"] @ dev(w.w_ih)).double().cpu()
+    # autograd reference: GRUCell with diagonal recurrent blocks, fp64
+    d = 64
+    m = torch.nn.GRUCell(48, d).double()
+    with torch.no_grad():
+        m.weight_ih.copy_(w.w_ih.double())
+        m.bias_ih.copy_(w.b_ih.double())
+        m.bias_hh.copy_(w.b_hh.double())
+        m.weight_hh.copy_(torch.cat([torch.diag(w.w_hh[k * d:(k + 1) * d].double()) for k in range(3)], 0))
+    x = w.x.double().requires_grad_(True)
+    h0 = w.h0.double().requires_grad_(True)
+    h, loss = h0, 0.0
+    for t in range(300):
+        h = m(x[:, t], h)
+        loss = loss + (h * dh[:, t].double()).sum()
+    loss.backward()
+    assert _rel(dx.numpy(), x.grad.numpy()) <= 1e-4
+    assert _rel(r["dh0"].double().cpu().numpy(), h0.grad.numpy()) <= 1e-4
+    gw = m.weight_hh.grad
+    du = torch.cat([torch.diagonal(gw[k * d:(k + 1) * d]) for k in range(3)])
+    assert _rel(r["dw_hh"].double().cpu().numpy(), du.numpy()) <= 1e-4
+    assert _rel(r["db_hh"].double().cpu().numpy(), m.bias_hh.grad.numpy()) <= 1e-4
