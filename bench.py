@@ -79,7 +79,16 @@ BENCHES = {
         desc="near-unstable dense GRU Din=D=64 (spectral radius 1.5), B={B}/GPU, T={T}, fp32, "
              "ELK lambda 0.01, tol 1e-4",
         cpu_sample=dict(B=1, T=1000), ref_sample=dict(B=1, T=150)),
+    # the backward pass through the evaluated diagonal-cell sequence (not a solve):
+    # reads P 12 + h 4 + dL/dh 4, writes dL/dP 12 = 32 B per state
+    "adjoint": dict(
+        workload="diag", mode="ADJOINT", lam=0.0, bound="hbm", per_state=32,
+        kernel="adjoint_diag_kernel (one reverse pass)",
+        desc="backward pass of the diagonal-recurrence GRU Din=D=2048, B={B}/GPU, T={T}: "
+             "dL/dP, dL/dh0, dL/du, dL/db_hh from the converged states and dL/dh",
+        cpu_sample=dict(B=1, T=512), ref_sample=dict(B=1, T=128)),
 }
+ADJ_METRIC = "backward states/sec (B*T*D per s, gradients through the evaluated sequence)"
 # fp32 FMA peak for the ALU-bound row: 148 SMs x 128 fp32 lanes x 2 flop x
 # 1965 MHz (the part's maximum SM clock), in TFLOP/s.
 ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
@@ -199,6 +208,19 @@ def cpu_baseline_oracle(spec: dict, sample: dict):
     c = GRU.from_workload(w)
     x, h0 = w.x.double().numpy(), w.h0.double().numpy()
     mode = spec["mode"]
+    if mode == "ADJOINT":
+        import numpy as np
+        from oracle.adjoint import adjoint
+        from oracle.cells import rollout
+        h = rollout(c, x, h0)
+        g = np.random.default_rng(0).normal(size=h.shape)
+        t0 = time.perf_counter()
+        adjoint(c, x, h0, h, g, jacobian="diag")
+        secs = time.perf_counter() - t0
+        states = w.B * w.T * w.d
+        return {"value": states / secs, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "sample": f"fp64 numpy oracle backward pass (reverse recurrence, dP, parameter and input "
+                          f"gradients) on B={w.B}, T={w.T}, D={w.d} ({secs:.1f} s); same distributions"}
     t0 = time.perf_counter()
     if mode in ("ELK", "QUASI_ELK"):
         r = oracle.elk_solve(c, x, h0, mode, spec["lam"], w.tol)
@@ -225,9 +247,10 @@ def run_reference(args):
         base = cb
     v = statistics.median(steps)
     from newton_solve_nonlinear_b200.inputs import WORKLOADS
+    metric = ADJ_METRIC if spec["mode"] == "ADJOINT" else METRIC
     full = WORKLOADS[spec["workload"]]
     T = args.T or full["T"]
-    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+    line = {"impl": "reference", "metric": metric, "value": v, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
@@ -236,6 +259,108 @@ def run_reference(args):
                              "sample": base["sample"]},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_adjoint(args):
+    """The backward pass through the converged diagonal-cell solve, timed alone."""
+    import torch
+    import torch.distributed as dist
+    from newton_solve_nonlinear_b200 import binding
+    from newton_solve_nonlinear_b200.inputs import make_workload
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    spec = BENCHES[args.workload]
+    over = {"T": args.T} if args.T else {}
+    w = make_workload(spec["workload"], seed=rank, **over)
+    B, T, D = w.B, w.T, w.d
+    states = B * T * D
+    g = lambda t: t.to(dev).contiguous()
+    # the forward solve gives the states; the upstream gradient is synthetic
+    sol = binding.solve_workload(w, "QUASI", device=dev)
+    P = binding.input_projection(g(w.x), g(w.w_ih), g(w.b_ih), d=D, kind=w.kind)
+    h, h0, u, bh = sol.h, g(w.h0), g(w.w_hh), g(w.b_hh)
+    dh = torch.randn(B, T, D, generator=torch.Generator().manual_seed(rank)).to(dev)
+    ws = binding.alloc_workspace(binding.adjoint_workspace_size(D, B, T), dev)
+    out = dict(dP=torch.empty_like(P), dh0=torch.empty_like(h0), dw_hh=torch.empty_like(u),
+               db_hh=torch.empty_like(bh))
+    stream = torch.cuda.current_stream(dev)
+    step = lambda: binding.adjoint(u, bh, P, h0, h, dh, workspace=ws, out=out)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with Clocks(local) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        for e0, e1 in evs:
+            e0.record(stream)
+            step()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    max_ms = max_over_ranks(sum(ms), dev)
+    value = job_value(states, args.steps, world, max_ms)
+    st = binding.lib().pararnn_adjoint_status(ws.data_ptr(), stream.cuda_stream)
+    # end to end: P, h and dL/dh from page-locked host memory, dL/dP back, each step
+    hP, hh, hdh = P.cpu().pin_memory(), h.cpu().pin_memory(), dh.cpu().pin_memory()
+    hdP = torch.empty(P.shape, dtype=torch.float32).pin_memory()
+    e2e_steps = max(1, min(args.steps, 3))
+    barrier()
+    torch.cuda.synchronize()
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record(stream)
+    for _ in range(e2e_steps):
+        P.copy_(hP, non_blocking=True)
+        h.copy_(hh, non_blocking=True)
+        dh.copy_(hdh, non_blocking=True)
+        step()
+        hdP.copy_(out["dP"], non_blocking=True)
+    eb.record(stream)
+    torch.cuda.synchronize()
+    e2e_value = job_value(states, e2e_steps, world, max_over_ranks(ea.elapsed_time(eb), dev))
+    cpu = cpu_baseline_oracle(spec, spec["cpu_sample"]) if rank == 0 and world == 1 else None
+    hbm_peak, peak_kind = peaks()
+    avg_s = statistics.mean(ms) / 1e3
+    achieved = states * spec["per_state"] / avg_s / 1e9
+    line = {
+        "metric": ADJ_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": spec["desc"].format(B=B, T=T), "name": args.workload, "B": B, "T": T, "D": D,
+                   "cell": w.kind, "status": binding.STATUS.get(st),
+                   "l2": f"inputs larger than L2 (126 MB): P {P.numel() * 4 / 1e6:.0f} MB, "
+                         f"h and dL/dh {h.numel() * 8 / 1e6:.0f} MB, dL/dP {P.numel() * 4 / 1e6:.0f} MB",
+                   "parallelism": f"replicas over sequences x{world}"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": None, "kernel": spec["kernel"],
+                     "algorithmic": f"{spec['per_state']} B/state x {states} states",
+                     "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"},
+        "e2e": {"value": e2e_value, "unit": UNIT,
+                "h2d_bytes_per_step": (P.numel() + h.numel() + dh.numel()) * 4,
+                "d2h_bytes_per_step": P.numel() * 4},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
     return 0
 
 
@@ -404,6 +529,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if BENCHES[args.workload]["mode"] == "ADJOINT":
+        return run_adjoint(args)
     return run_ours(args)
 
 

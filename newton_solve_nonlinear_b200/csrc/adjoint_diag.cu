@@ -17,10 +17,10 @@
 //     dL/du_r = sum lam (1-z)(1-n^2) g r(1-r) hp,  dL/du_z = sum lam (hp-n) z(1-z) hp,
 //     dL/du_n = sum lam (1-z)(1-n^2) r hp,  dL/db_hh likewise without hp.
 //
-// One cooperative launch: CTAs of 256 threads walk tiles of (sequence, 64
+// One cooperative launch: CTAs of 512 threads walk tiles of (sequence, 64
 // lanes, 32 steps) from the last chunk to the first.  Thread (lane d, segment
-// s) evaluates the cell at its 8 steps and the next one (for a_{t+1}), folds
-// its steps' maps in reverse, the four segments of a lane chain through shared
+// s) evaluates the cell at its 4 steps and the next one (for a_{t+1}), folds
+// its steps' maps in reverse, the eight segments of a lane chain through shared
 // memory, the tile takes lam at its end from a cooperative look-back over
 // later chunks, and the sweep writes dL/dP and the per-tile partial sums of
 // the parameter gradients.  After a grid barrier every warp reduces some of
@@ -35,9 +35,9 @@ namespace {
 
 constexpr int ATS = 32;            // steps per tile
 constexpr int ADL = 64;            // lanes per tile
-constexpr int ANT = 256;           // threads: lane x 4 segments
-constexpr int ASEGS = ANT / ADL;   // 4 segments
-constexpr int ASL = ATS / ASEGS;   // 8 steps per thread
+constexpr int ANT = 512;           // threads: lane x 8 segments
+constexpr int ASEGS = ANT / ADL;   // 8 segments
+constexpr int ASL = ATS / ASEGS;   // 4 steps per thread
 
 struct AdjArgs {
     const float *P, *h0, *h, *dh, *u, *b_hh;  // u: [3D] recurrent vectors (r, z, n)
@@ -65,6 +65,7 @@ __device__ __forceinline__ void adj_cell(float pr, float pz, float pn, float hp,
 }
 
 __global__ void __launch_bounds__(ANT, 2) adjoint_diag_kernel(AdjArgs S) {
+    static_assert(ASEGS == 8, "the per-tile partial sums below add eight segments");
     __shared__ float seg_a[ASEGS][ADL], seg_b[ASEGS][ADL];
     __shared__ float carry[ADL];
     __shared__ float red6[ASEGS][6][ADL];
@@ -180,7 +181,8 @@ __global__ void __launch_bounds__(ANT, 2) adjoint_diag_kernel(AdjArgs S) {
         for (int i = tid; i < 6 * ADL; i += ANT) {  // per-tile partials, segments summed in order
             const int k = i / ADL, dd = i % ADL;
             S.part[(static_cast<size_t>(v) * 6 + k) * ADL + dd] =
-                ((red6[0][k][dd] + red6[1][k][dd]) + red6[2][k][dd]) + red6[3][k][dd];
+                ((red6[0][k][dd] + red6[1][k][dd]) + (red6[2][k][dd] + red6[3][k][dd])) +
+                ((red6[4][k][dd] + red6[5][k][dd]) + (red6[6][k][dd] + red6[7][k][dd]));
         }
         __syncthreads();  // shared arrays are rewritten by the next tile
     }
