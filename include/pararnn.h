@@ -183,6 +183,49 @@ PARARNN_API int pararnn_newton_solve_async(const pararnn_cell *cell, const parar
                                pararnn_stream stream);
 
 /*
+ * pararnn_newton_solve_guess_async -- pararnn_newton_solve_async started from a
+ * caller's initial guess instead of zero (a warm start: the previous epoch's
+ * states, or a nearby solution).  The pages leave the starting guess open
+ * (the zero-start solve's choice is a reading); starting elsewhere changes only
+ * where the iteration begins: the fixed point, the convergence test and every
+ * other argument are those of the zero-start solve.
+ *   h_init  DEVICE float [B, T, D], 16-byte aligned, read once before the first
+ *           iteration; it may be `h` itself (the solve then updates h in place).
+ * Asynchronous; the report goes to info_dev.
+ */
+PARARNN_API int pararnn_newton_solve_guess_async(const pararnn_cell *cell, const pararnn_params *params,
+                                                 const void *x, const float *h0, const float *h_init, int B,
+                                                 int T, int mode, float lambda, float tol, int max_iters,
+                                                 float *h, pararnn_info *info_dev, void *workspace,
+                                                 size_t ws_bytes, pararnn_stream stream);
+
+/*
+ * pararnn_newton_solve_chunked -- the solve over consecutive time chunks of at
+ * most t_chunk steps, one after another, each started from the last state the
+ * previous chunk reached: device memory grows with t_chunk instead of T (for
+ * sequences too long for one solve's workspace; the ParaRNN summary page,
+ * "Experimental Results", names chunking as the remedy for the Newton
+ * iteration's hidden-state memory).  Each chunk is an independent
+ * solve to `tol`; for contractive cells the joined states match the
+ * one-shot solve to within the propagated tolerance.  Arguments as for
+ * pararnn_newton_solve, plus t_chunk >= 1 (max_iters <= 0 caps every chunk at
+ * T + 1 of the whole sequence); the workspace is
+ * pararnn_chunked_workspace_size bytes.  The report: iterations summed over
+ * the chunks, the worst status, the largest delta and residual.  Synchronises
+ * `stream` once, at the end.
+ */
+PARARNN_API int pararnn_newton_solve_chunked(const pararnn_cell *cell, const pararnn_params *params,
+                                             const void *x, const float *h0, int B, int T, int t_chunk,
+                                             int mode, float lambda, float tol, int max_iters, float *h,
+                                             pararnn_info *info, void *workspace, size_t ws_bytes,
+                                             pararnn_stream stream);
+
+/* pararnn_chunked_workspace_size -- bytes pararnn_newton_solve_chunked needs
+ * (one chunk's solve workspace plus staging for one chunk), or 0. */
+PARARNN_API size_t pararnn_chunked_workspace_size(const pararnn_cell *cell, int B, int T, int t_chunk,
+                                                  int mode);
+
+/*
  * pararnn_newton_solve_host -- the same evaluation from and to HOST memory,
  * with the copies overlapped with the computation.
  *

@@ -26,7 +26,8 @@ EXPORTS = ("pararnn_workspace_size", "pararnn_newton_solve", "pararnn_newton_sol
            "pararnn_affine_scan_workspace_size", "pararnn_affine_scan",
            "pararnn_affine_scan_status", "pararnn_status_string", "pararnn_newton_solve_host",
            "pararnn_host_workspace_size", "pararnn_adjoint", "pararnn_adjoint_workspace_size",
-           "pararnn_adjoint_status")
+           "pararnn_adjoint_status", "pararnn_newton_solve_guess_async", "pararnn_newton_solve_chunked",
+           "pararnn_chunked_workspace_size")
 
 
 class Cell(ctypes.Structure):
@@ -87,6 +88,14 @@ def lib() -> ctypes.CDLL:
         L.pararnn_adjoint_workspace_size.restype = sz
         L.pararnn_adjoint_status.argtypes = [vp, vp]
         L.pararnn_adjoint_status.restype = ci
+        L.pararnn_newton_solve_guess_async.argtypes = [ctypes.POINTER(Cell), ctypes.POINTER(Params), vp, vp, vp,
+                                                       ci, ci, ci, cf, cf, ci, vp, vp, vp, sz, vp]
+        L.pararnn_newton_solve_guess_async.restype = ci
+        L.pararnn_newton_solve_chunked.argtypes = [ctypes.POINTER(Cell), ctypes.POINTER(Params), vp, vp, ci, ci,
+                                                   ci, ci, cf, cf, ci, vp, ctypes.POINTER(Info), vp, sz, vp]
+        L.pararnn_newton_solve_chunked.restype = ci
+        L.pararnn_chunked_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci, ci, ci]
+        L.pararnn_chunked_workspace_size.restype = sz
         L.pararnn_status_string.argtypes = [ci]
         L.pararnn_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -143,13 +152,14 @@ class SolveResult:
 
 def newton_solve(w_ih, b_ih, w_hh, b_hh, x, h0, *, kind: str, mode: str, tol: float,
                  lam: float = 0.0, max_iters: int = 0, out=None, workspace=None,
-                 stream=None, sync: bool = True, info_dev=None):
+                 stream=None, sync: bool = True, info_dev=None, h_init=None):
     """Evaluate the GRU over x [B, T, Din] with the chosen Newton mode.
 
     All tensors must be contiguous CUDA tensors (x and w_ih fp32 or bf16, the
     rest fp32).  With ``sync`` the call waits and returns a SolveResult; with
     ``sync=False`` it only enqueues, writing the report into ``info_dev`` (an
-    int32 CUDA tensor of 4 elements) and returns ``out``."""
+    int32 CUDA tensor of 4 elements) and returns ``out``.  ``h_init`` [B, T, D]
+    (fp32 CUDA) starts the iteration from that guess instead of zero."""
     B, T, din = x.shape
     d = h0.shape[1]
     cell = make_cell(kind, din, d, x.dtype)
@@ -167,6 +177,22 @@ def newton_solve(w_ih, b_ih, w_hh, b_hh, x, h0, *, kind: str, mode: str, tol: fl
     params = Params(_dev(w_ih, "w_ih"), _dev(b_ih, "b_ih"), _dev(w_hh, "w_hh"), _dev(b_hh, "b_hh"))
     args = (ctypes.byref(cell), ctypes.byref(params), _dev(x, "x"), _dev(h0, "h0"), B, T, m,
             float(lam), float(tol), int(max_iters), _dev(out, "out"))
+    if h_init is not None:
+        own = info_dev is None
+        if own:
+            info_dev = torch.zeros(4, dtype=torch.int32, device=x.device)
+        rc = L.pararnn_newton_solve_guess_async(ctypes.byref(cell), ctypes.byref(params), _dev(x, "x"),
+                                                _dev(h0, "h0"), _dev(h_init, "h_init"), B, T, m, float(lam),
+                                                float(tol), int(max_iters), _dev(out, "out"),
+                                                _dev(info_dev, "info_dev"), _dev(workspace, "workspace"),
+                                                workspace.numel(), _stream(stream))
+        if rc != 0:
+            raise RuntimeError(f"pararnn_newton_solve_guess_async: {L.pararnn_status_string(rc).decode()}")
+        if not sync:
+            return out
+        rep = info_dev.cpu()  # waits for the solve
+        return SolveResult(out, int(rep[0]), STATUS[int(rep[1])], float(rep[2:3].view(torch.float32)),
+                           float(rep[3:4].view(torch.float32)))
     if sync:
         info = Info()
         rc = L.pararnn_newton_solve(*args, ctypes.byref(info), _dev(workspace, "workspace"),
@@ -190,6 +216,40 @@ def _host(t: torch.Tensor, name: str) -> int:
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return t.data_ptr()
+
+
+def newton_solve_chunked(w_ih, b_ih, w_hh, b_hh, x, h0, *, kind: str, mode: str, tol: float, t_chunk: int,
+                         lam: float = 0.0, max_iters: int = 0, out=None, workspace=None,
+                         stream=None) -> "SolveResult":
+    """The solve over consecutive time chunks of at most ``t_chunk`` steps (device
+    memory grows with t_chunk, not T); the report sums iterations over chunks."""
+    B, T, din = x.shape
+    d = h0.shape[1]
+    cell = make_cell(kind, din, d, x.dtype)
+    L = lib()
+    m = MODES[mode]
+    need = int(L.pararnn_chunked_workspace_size(ctypes.byref(cell), B, T, int(t_chunk), m))
+    if need == 0:
+        raise ValueError("arguments rejected by pararnn_chunked_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, x.device)
+    if out is None:
+        out = torch.empty(B, T, d, dtype=torch.float32, device=x.device)
+    params = Params(_dev(w_ih, "w_ih"), _dev(b_ih, "b_ih"), _dev(w_hh, "w_hh"), _dev(b_hh, "b_hh"))
+    info = Info()
+    rc = L.pararnn_newton_solve_chunked(ctypes.byref(cell), ctypes.byref(params), _dev(x, "x"), _dev(h0, "h0"),
+                                        B, T, int(t_chunk), m, float(lam), float(tol), int(max_iters),
+                                        _dev(out, "out"), ctypes.byref(info), _dev(workspace, "workspace"),
+                                        workspace.numel(), _stream(stream))
+    if rc in (3, 4):
+        raise RuntimeError(f"pararnn_newton_solve_chunked: {L.pararnn_status_string(rc).decode()}")
+    return SolveResult(out, info.iters, STATUS[info.status], info.delta, info.residual)
+
+
+def chunked_workspace_size(kind: str, din: int, d: int, B: int, T: int, t_chunk: int, mode: str,
+                           dtype: torch.dtype = torch.float32) -> int:
+    cell = make_cell(kind, din, d, dtype)
+    return int(lib().pararnn_chunked_workspace_size(ctypes.byref(cell), B, T, int(t_chunk), MODES[mode]))
 
 
 def host_workspace_size(kind: str, din: int, d: int, B: int, T: int, mode: str, parts: int,

@@ -436,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_deer_kernel(DenseArgs S) {
         }
         const float *hold = A.hbuf[it & 1];
         float *hnew = A.hbuf[(it + 1) & 1];
-        const bool zero_guess = it == 0;
+        const bool zero_guess = it == 0 && !A.warm;  // the first guess: zero, or the caller's
         unsigned dmax = 0u, rmax = 0u;
         for (long long tile = blockIdx.x; tile < S.g.n_tiles; tile += nblocks)
             phase_aggregate<DMAX>(S, sm, tile, hold, zero_guess, rmax);

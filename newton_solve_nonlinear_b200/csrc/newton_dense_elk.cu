@@ -565,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 2) dense_elk_kernel(ElkArgs S) {
         }
         const float *hold = A.hbuf[it & 1];
         float *hnew = A.hbuf[(it + 1) & 1];
-        const bool zero_guess = it == 0;
+        const bool zero_guess = it == 0 && !A.warm;  // the first guess: zero, or the caller's
         unsigned dmax = 0u, rmax = 0u;
         for (long long w = blockIdx.x; w < lin_items; w += nblocks) {
             const int b = static_cast<int>(w / n_chunks), c = static_cast<int>(w % n_chunks);

@@ -628,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1) deer_mma_kernel(MmaArgs S) {
         }
         const float *hold = A.hbuf[it & 1];
         float *hnew = A.hbuf[(it + 1) & 1];
-        const bool zero_guess = it == 0;
+        const bool zero_guess = it == 0 && !A.warm;  // the first guess: zero, or the caller's
         unsigned dmax = 0u, rmax = 0u;
         for (long long w = gw; w < n_chunks; w += nw)
             chunk_aggregate(S, W, static_cast<int>(w / S.NC), static_cast<int>(w % S.NC), hold,

@@ -756,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, ELK ? 1 : 2) diag_solver_kernel(Diag
         }
         const float *hold = A.hbuf[it & 1];
         float *hnew = A.hbuf[(it + 1) & 1];
-        const bool zero_guess = it == 0;
+        const bool zero_guess = it == 0 && !A.warm;  // the first guess: zero, or the caller's
         const unsigned epoch = static_cast<unsigned>(it + 1);
         unsigned dmax = 0u, rmax = 0u;
         if (!ELK) {

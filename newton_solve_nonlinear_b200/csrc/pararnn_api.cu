@@ -146,7 +146,8 @@ static int check_solve(const pararnn_cell *cell, const pararnn_params *params, c
 static cudaError_t enqueue_iterate(const pararnn_cell *cell, const pararnn_params *params,
                                    const float *P, const float *h0, int B, int T, int mode,
                                    float lambda, float tol, int max_iters, float *h,
-                                   pararnn_info *info_dev, void *workspace, cudaStream_t s) {
+                                   pararnn_info *info_dev, void *workspace, cudaStream_t s,
+                                   const float *h_init = nullptr) {
     const WsLayout L = ws_layout(*cell, B, T, mode);
     char *ws = static_cast<char *>(workspace);
     WsHeader *hdr = reinterpret_cast<WsHeader *>(ws + L.header);
@@ -173,18 +174,22 @@ static cudaError_t enqueue_iterate(const pararnn_cell *cell, const pararnn_param
     a.elk_b = reinterpret_cast<float *>(ws + L.elk + 3 * states4);
     a.hdr = hdr;
     a.info_out = info_dev ? info_dev : &hdr->info;
+    a.warm = h_init != nullptr;
 
     cudaError_t e = cudaMemsetAsync(ws + L.header, 0, 256, s);
     if (e == cudaSuccess && diag && L.elk > L.desc) e = cudaMemsetAsync(ws + L.desc, 0, L.elk - L.desc, s);
+    // the first guess: the caller's (copied first, so h_init may be h itself), else zero
+    if (e == cudaSuccess && h_init)
+        e = cudaMemcpyAsync(a.hbuf[0], h_init, states * sizeof(float), cudaMemcpyDeviceToDevice, s);
     if (e != cudaSuccess) return e;
     if ((mode == PARARNN_QUASI || mode == PARARNN_QUASI_ELK) && quasi_tc_supported(*cell, B, T)) {
-        // the tensor-core path reads the initial guess (zero) from memory
-        e = cudaMemsetAsync(a.hbuf[0], 0, states * sizeof(float), s);
+        // the tensor-core path reads the initial guess from memory
+        if (!h_init) e = cudaMemsetAsync(a.hbuf[0], 0, states * sizeof(float), s);
         if (e != cudaSuccess) return e;
         return launch_quasi_tc2(a, mode == PARARNN_QUASI_ELK, s);
     }
     if (cell->kind == PARARNN_GRU_DIAG && !is_elk(mode) && diag2_supported(*cell, B, T)) {
-        e = cudaMemsetAsync(a.hbuf[0], 0, states * sizeof(float), s);
+        if (!h_init) e = cudaMemsetAsync(a.hbuf[0], 0, states * sizeof(float), s);
         if (e != cudaSuccess) return e;
         return launch_diag2(a, s);
     }
@@ -226,10 +231,15 @@ int pararnn_newton_iterate_async(const pararnn_cell *cell, const pararnn_params 
 static int solve_enqueue(const pararnn_cell *cell, const pararnn_params *params, const void *x,
                          const float *h0, int B, int T, int mode, float lambda, float tol,
                          int max_iters, float *h, pararnn_info *info_dev, void *workspace,
-                         size_t ws_bytes, pararnn_stream stream) {
+                         size_t ws_bytes, pararnn_stream stream, const float *h_init = nullptr) {
     int rc = check_solve(cell, params, x, nullptr, h0, B, T, mode, lambda, tol, h, workspace,
                          ws_bytes);
     if (rc != PARARNN_OK) return rc;
+    if (h_init) {  // a guess of [B, T, D]: aligned, and clear of the workspace (it may be h)
+        const size_t nb = static_cast<size_t>(B) * T * cell->d * 4;
+        if (!aligned(h_init, 16) || overlaps(h_init, nb, workspace, ws_layout(*cell, B, T, mode).total))
+            return PARARNN_INVALID_ARG;
+    }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const WsLayout L = ws_layout(*cell, B, T, mode);
     float *P = reinterpret_cast<float *>(static_cast<char *>(workspace) + L.P);
@@ -237,7 +247,7 @@ static int solve_enqueue(const pararnn_cell *cell, const pararnn_params *params,
                                       static_cast<long long>(B) * T, s);
     if (e == cudaSuccess)
         e = enqueue_iterate(cell, params, P, h0, B, T, mode, lambda, tol, max_iters, h, info_dev,
-                            workspace, s);
+                            workspace, s, h_init);
     return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
 }
 
@@ -267,6 +277,101 @@ int pararnn_newton_solve(const pararnn_cell *cell, const pararnn_params *params,
     if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
     if (info) *info = host;
     return host.status;
+}
+
+int pararnn_newton_solve_guess_async(const pararnn_cell *cell, const pararnn_params *params, const void *x,
+                                     const float *h0, const float *h_init, int B, int T, int mode, float lambda,
+                                     float tol, int max_iters, float *h, pararnn_info *info_dev,
+                                     void *workspace, size_t ws_bytes, pararnn_stream stream) {
+    if (info_dev == nullptr || !aligned(info_dev, 4) || h_init == nullptr) return PARARNN_INVALID_ARG;
+    return solve_enqueue(cell, params, x, h0, B, T, mode, lambda, tol, max_iters, h, info_dev, workspace,
+                         ws_bytes, stream, h_init);
+}
+
+// ---- T-chunked solve: consecutive time chunks solved one after another ----
+
+namespace {
+struct ChunkLayout {
+    int tc, nchunks;
+    size_t solve, xs, hs, h0, infos, total;
+};
+ChunkLayout chunk_layout(const pararnn_cell &cell, int B, int T, int t_chunk, int mode) {
+    ChunkLayout C{};
+    C.tc = t_chunk < T ? t_chunk : T;
+    C.nchunks = (T + C.tc - 1) / C.tc;
+    const size_t es = cell.x_dtype == PARARNN_BF16 ? 2 : 4;
+    size_t off = 0;
+    C.solve = off; off = align256(off + ws_layout(cell, B, C.tc, mode).total);
+    C.xs = off; off = align256(off + static_cast<size_t>(B) * C.tc * cell.din * es);
+    C.hs = off; off = align256(off + static_cast<size_t>(B) * C.tc * cell.d * 4);
+    C.h0 = off; off = align256(off + static_cast<size_t>(B) * cell.d * 4);
+    C.infos = off; off = align256(off + static_cast<size_t>(C.nchunks) * sizeof(pararnn_info));
+    C.total = off;
+    return C;
+}
+}  // namespace
+
+size_t pararnn_chunked_workspace_size(const pararnn_cell *cell, int B, int T, int t_chunk, int mode) {
+    if (t_chunk < 1 || !cell_ok(cell, B, T, mode)) return 0;
+    const int tc = t_chunk < T ? t_chunk : T;
+    if (!cell_ok(cell, B, tc, mode)) return 0;
+    return chunk_layout(*cell, B, T, t_chunk, mode).total;
+}
+
+int pararnn_newton_solve_chunked(const pararnn_cell *cell, const pararnn_params *params, const void *x,
+                                 const float *h0, int B, int T, int t_chunk, int mode, float lambda, float tol,
+                                 int max_iters, float *h, pararnn_info *info, void *workspace, size_t ws_bytes,
+                                 pararnn_stream stream) {
+    const size_t need = pararnn_chunked_workspace_size(cell, B, T, t_chunk, mode);
+    if (need == 0 || ws_bytes < need || !params || !x || !h0 || !h || !workspace || !aligned(workspace, 256) ||
+        !aligned(x, 16) || !aligned(h0, 16) || !aligned(h, 16))
+        return PARARNN_INVALID_ARG;
+    const ChunkLayout C = chunk_layout(*cell, B, T, t_chunk, mode);
+    const size_t es = cell->x_dtype == PARARNN_BF16 ? 2 : 4;
+    const size_t xrow = static_cast<size_t>(T) * cell->din * es, hrow = static_cast<size_t>(T) * cell->d * 4;
+    if (overlaps(h, B * hrow, workspace, need) || overlaps(h, B * hrow, x, B * xrow) ||
+        overlaps(h, B * hrow, h0, static_cast<size_t>(B) * cell->d * 4))
+        return PARARNN_INVALID_ARG;
+    char *ws = static_cast<char *>(workspace);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    pararnn_info *infos = reinterpret_cast<pararnn_info *>(ws + C.infos);
+    cudaError_t e = cudaSuccess;
+    int rc = PARARNN_OK;
+    for (int c = 0; c < C.nchunks && e == cudaSuccess && rc == PARARNN_OK; ++c) {
+        const int t0 = c * C.tc, n = (T - t0) < C.tc ? (T - t0) : C.tc;
+        // this chunk's inputs of every sequence, packed [B, n, Din]
+        e = cudaMemcpy2DAsync(ws + C.xs, n * cell->din * es, static_cast<const char *>(x) + t0 * cell->din * es,
+                              xrow, n * cell->din * es, B, cudaMemcpyDeviceToDevice, s);
+        // the state entering the chunk: h0, or each sequence's last state of the previous chunk
+        if (e == cudaSuccess && c > 0)
+            e = cudaMemcpy2DAsync(ws + C.h0, cell->d * 4, reinterpret_cast<const char *>(h) + (t0 - 1) * cell->d * 4,
+                                  hrow, cell->d * 4, B, cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) break;
+        const float *hin = c == 0 ? h0 : reinterpret_cast<const float *>(ws + C.h0);
+        // the cap of the whole sequence's solve (T + 1 by default), not of the chunk:
+        // damped modes may need more iterations than a short chunk has steps
+        rc = solve_enqueue(cell, params, ws + C.xs, hin, B, n, mode, lambda, tol, max_iters > 0 ? max_iters : T + 1,
+                           reinterpret_cast<float *>(ws + C.hs), infos + c, ws + C.solve,
+                           ws_layout(*cell, B, n, mode).total, stream);
+        if (rc != PARARNN_OK) break;
+        e = cudaMemcpy2DAsync(reinterpret_cast<char *>(h) + t0 * cell->d * 4, hrow, ws + C.hs, n * cell->d * 4,
+                              n * cell->d * 4, B, cudaMemcpyDeviceToDevice, s);
+    }
+    if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
+    if (rc != PARARNN_OK) return rc;
+    std::vector<pararnn_info> host(C.nchunks);
+    e = cudaMemcpyAsync(host.data(), infos, C.nchunks * sizeof(pararnn_info), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
+    pararnn_info agg{};
+    for (const pararnn_info &q : host) {  // iterations summed over the chunks; the worst of the rest
+        agg.iters += q.iters;
+        agg.status = q.status > agg.status ? q.status : agg.status;
+        agg.delta = q.delta > agg.delta ? q.delta : agg.delta;
+        agg.residual = q.residual > agg.residual ? q.residual : agg.residual;
+    }
+    if (info) *info = agg;
+    return agg.status;
 }
 
 size_t pararnn_affine_scan_workspace_size(int B, int T, int D, int dense) {

@@ -57,6 +57,7 @@ struct DiagArgs {
     float *elk_m, *elk_p, *elk_a, *elk_b;  // quasi-ELK forward results [B, T, D]
     WsHeader *hdr;
     pararnn_info *info_out;  // device report destination
+    int warm;                // hbuf[0] holds a caller's initial guess (else the guess is zero)
 };
 
 // Workspace carve-up shared by the size query and the solver.

@@ -1,0 +1,88 @@
+"""GPU tests of the warm-started solve and the T-chunked solve against the
+fp64 rollout (the unique answer every solve must reach).
+
+Tolerances as for the zero-start solves: converged states within 1e-4 of the
+rollout (ELK modes at tol 1e-6, since damped steps converge linearly).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle.cells import GRU, rollout
+from newton_solve_nonlinear_b200 import binding
+from newton_solve_nonlinear_b200.inputs import make_workload
+
+pytestmark = pytest.mark.gpu
+
+# (workload, overrides, mode, lambda, tol) -- one per solver path
+PATHS = [
+    ("untrained", dict(B=3, T=1000), "QUASI", 0.0, None),                     # tensor-core quasi-DEER
+    ("diag", dict(B=2, T=600, d=128, din=128), "QUASI", 0.0, None),           # streaming diagonal cell
+    ("dense_deer", dict(B=2, T=800), "DEER", 0.0, None),                      # dense DEER (mma chains)
+    ("untrained", dict(B=2, T=500, d=48, din=48), "QUASI", 0.0, None),        # generic diagonal-Jacobian path
+    ("near_unstable", dict(B=2, T=400), "QUASI_ELK", 1.0, 1e-6),              # tensor-core quasi-ELK
+    ("near_unstable", dict(B=2, T=200), "ELK", 0.3, 1e-6),                    # dense ELK
+]
+
+
+def _rollout(w):
+    return rollout(GRU.from_workload(w), w.x.double().numpy(), w.h0.double().numpy())
+
+
+def _args(w):
+    dev = lambda t: t.cuda().contiguous()
+    return (dev(w.w_ih), dev(w.b_ih), dev(w.w_hh), dev(w.b_hh), dev(w.x), dev(w.h0))
+
+
+@pytest.mark.parametrize("name,over,mode,lam,tol", PATHS)
+def test_warm_start_from_solution_converges_at_once(name, over, mode, lam, tol):
+    w = make_workload(name, **over)
+    tol = w.tol if tol is None else tol
+    a = _args(w)
+    r0 = binding.newton_solve(*a, kind=w.kind, mode=mode, lam=lam, tol=tol)
+    assert r0.status == "OK"
+    r1 = binding.newton_solve(*a, kind=w.kind, mode=mode, lam=lam, tol=tol, h_init=r0.h.clone())
+    assert r1.status == "OK" and r1.iters <= 2, (r1.iters, r0.iters)
+    want = _rollout(w)
+    assert np.max(np.abs(r1.h.double().cpu().numpy() - want)) <= 1e-4
+
+
+def test_warm_start_from_perturbed_guess_in_place():
+    w = make_workload("untrained", B=2, T=2000)
+    a = _args(w)
+    r0 = binding.newton_solve(*a, kind=w.kind, mode="QUASI", tol=w.tol)
+    want = _rollout(w)
+    g = torch.Generator().manual_seed(1)
+    h = (torch.from_numpy(want).float() + 1e-3 * torch.randn(want.shape, generator=g)).cuda()
+    r1 = binding.newton_solve(*a, kind=w.kind, mode="QUASI", tol=w.tol, h_init=h, out=h)  # in place
+    assert r1.status == "OK" and r1.h.data_ptr() == h.data_ptr()
+    assert r1.iters < r0.iters, (r1.iters, r0.iters)
+    assert np.max(np.abs(h.double().cpu().numpy() - want)) <= 1e-4
+
+
+@pytest.mark.parametrize("name,over,mode,lam,tol,t_chunk", [
+    ("untrained", dict(B=3, T=1000), "QUASI", 0.0, None, 256),
+    ("diag", dict(B=2, T=700, d=128, din=128), "QUASI", 0.0, None, 300),
+    ("dense_deer", dict(B=2, T=1000), "DEER", 0.0, None, 333),
+    ("near_unstable", dict(B=2, T=500), "QUASI_ELK", 1.0, 1e-6, 128),
+    ("tiny", dict(T=100), "DEER", 0.0, None, 1),
+])
+def test_chunked_solve_matches_rollout(name, over, mode, lam, tol, t_chunk):
+    w = make_workload(name, **over)
+    tol = w.tol if tol is None else tol
+    r = binding.newton_solve_chunked(*_args(w), kind=w.kind, mode=mode, lam=lam, tol=tol, t_chunk=t_chunk)
+    assert r.status == "OK"
+    assert np.max(np.abs(r.h.double().cpu().numpy() - _rollout(w))) <= 1e-4
+
+
+def test_one_chunk_equals_one_solve_and_memory_shrinks():
+    w = make_workload("untrained", B=2, T=900)
+    a = _args(w)
+    r0 = binding.newton_solve(*a, kind=w.kind, mode="QUASI", tol=w.tol)
+    r1 = binding.newton_solve_chunked(*a, kind=w.kind, mode="QUASI", tol=w.tol, t_chunk=4096)
+    assert torch.equal(r0.h, r1.h) and r0.iters == r1.iters
+    full = binding.workspace_size("dense", 64, 64, 16, 65536, "QUASI")
+    part = binding.chunked_workspace_size("dense", 64, 64, 16, 65536, 4096, "QUASI")
+    assert 0 < part < full / 8
+    with pytest.raises(ValueError):
+        binding.newton_solve_chunked(*a, kind=w.kind, mode="QUASI", tol=w.tol, t_chunk=0)
