@@ -19,6 +19,8 @@ What it states, plainly and slowly, in float64:
                    and a sequential Kalman filter + RTS smoother.
   * ``brute``   -- dense (T*D) x (T*D) assemblies for tiny T, used only to pin
                    the structured solvers above.
+  * ``lstm``    -- the diagonal-recurrence LSTM: cell, 2x2-per-lane Jacobian,
+                   rollout and exact Newton on the unrolled system.
   * ``adjoint`` -- the backward pass: gradients of a loss through the evaluated
                    states (reverse-time recurrence with J^T, exact or with the
                    diagonal of J), and the parameter and input gradients.
@@ -30,7 +32,7 @@ dense solves, and invariants the pages state (Newton is exact on an affine
 cell; undamped Newton recovers one more exact state per iteration).  The pages
 print no worked numeric example, so nothing here is pinned to printed values.
 """
-from . import cells, scan, newton, elk, brute, adjoint  # noqa: F401
+from . import cells, scan, newton, elk, brute, adjoint, lstm  # noqa: F401
 from .cells import GRU, rollout  # noqa: F401
 from .newton import newton_solve, STATUS_OK, STATUS_NOT_CONVERGED, STATUS_DIVERGED  # noqa: F401
 from .elk import elk_solve  # noqa: F401

@@ -121,3 +121,40 @@ def test_adjoint_unshifted_previous_state(monkeypatch):
         return out
     monkeypatch.setattr(adj_pins, "adjoint", bad)
     _fails(adj_pins.test_diag_cell_quasi_backward_is_exact)
+
+
+# ------------------------------------------------------------------ LSTM --
+import oracle.lstm as lstm  # noqa: E402
+import tests.test_oracle_lstm as lstm_pins  # noqa: E402
+
+
+def test_lstm_dropped_candidate_term(monkeypatch):
+    """dc'/dh without its candidate-gate term."""
+    orig = lstm.LSTM.jacobian
+
+    def bad(self, c, h, p):
+        d = self.d
+        u = self.u.copy()
+        self.u = u.copy()
+        self.u[2 * d:3 * d] = 0.0
+        try:
+            _, _, A_wrong = orig(self, c, h, p)
+        finally:
+            self.u = u
+        c2, h2, A = orig(self, c, h, p)
+        A = A.copy()
+        A[..., 0, 1] = A_wrong[..., 0, 1]
+        return c2, h2, A
+    monkeypatch.setattr(lstm.LSTM, "jacobian", bad)
+    _fails(lstm_pins.test_jacobian_central_differences)
+
+
+def test_lstm_transposed_block(monkeypatch):
+    """The substitution with each 2x2 block transposed."""
+    orig = lstm.LSTM.jacobian
+
+    def bad(self, c, h, p):
+        c2, h2, A = orig(self, c, h, p)
+        return c2, h2, np.swapaxes(A, -1, -2)
+    monkeypatch.setattr(lstm.LSTM, "jacobian", bad)
+    _fails(lstm_pins.test_one_newton_iteration_equals_brute_force_step)
