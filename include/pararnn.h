@@ -63,7 +63,7 @@ typedef enum {
  * DIAG: the recurrent weights are elementwise vectors u_r, u_z, u_n, so the
  * Jacobian is exactly diagonal and QUASI is exact Newton (the "adapted" GRU of
  * the ParaRNN abstract). */
-typedef enum { PARARNN_GRU_DENSE = 0, PARARNN_GRU_DIAG = 1 } pararnn_cell_kind;
+typedef enum { PARARNN_GRU_DENSE = 0, PARARNN_GRU_DIAG = 1, PARARNN_LSTM_DIAG = 2 } pararnn_cell_kind;
 
 typedef enum { PARARNN_F32 = 0, PARARNN_BF16 = 1 } pararnn_dtype;
 
@@ -409,6 +409,39 @@ PARARNN_API size_t pararnn_adjoint_workspace_size(const pararnn_cell *cell, int 
  * pararnn_adjoint using `workspace` left: PARARNN_OK, or PARARNN_TIMEOUT if a
  * bounded device-side wait expired (results unreliable). */
 PARARNN_API int pararnn_adjoint_status(const void *workspace, pararnn_stream stream);
+
+/*
+ * pararnn_lstm_solve -- evaluate the diagonal-recurrence LSTM (cell->kind ==
+ * PARARNN_LSTM_DIAG; the pages' "adapted" LSTM, ParaLSTM: the ParaRNN talk
+ * page "Federico Danieli", Abstract; the ParaRNN summary page, "Experimental
+ * Results") over B sequences of length T by exact Newton (DEER), and wait.
+ *
+ * Cell (torch.nn.LSTMCell layout, gate rows i, f, g, o; u_k the recurrent
+ * vectors, p = W_ih x + b_ih, b = b_hh):
+ *   i = sig(p_i + u_i h + b_i), f = sig(p_f + u_f h + b_f), g = tanh(p_g + u_g h + b_g),
+ *   o = sig(p_o + u_o h + b_o), c' = f c + i g, h' = o tanh(c').
+ * Lane j of the state (c, h) depends only on lane j of the previous state, so
+ * the Jacobian is a 2x2 block per lane and each Newton step is the scan of
+ * s_t = A_t s_{t-1} + b_t over 2x2 affine maps (exact Newton).  The guess
+ * starts at zero; convergence: max |s^(i+1) - s^(i)| over c and h <= tol.
+ *
+ *   params  w_ih [4D, Din] of w_dtype, b_ih [4D], w_hh [4D] (u_i, u_f, u_g, u_o),
+ *           b_hh [4D] (float), all DEVICE.
+ *   x       DEVICE [B, T, Din];  c0, h0 DEVICE [B, D].
+ *   c, h    DEVICE [B, T, D] float, outputs (c[:, t], h[:, t] = state after step t+1).
+ *   info    HOST report (may be NULL);  workspace: pararnn_lstm_workspace_size bytes.
+ * d % 4 == 0 (as the GRU cells), x_dtype == w_dtype.  Synchronises `stream`
+ * once; returns the solve's status (OK / NOT_CONVERGED / DIVERGED / TIMEOUT)
+ * or INVALID_ARG / CUDA_ERROR.
+ */
+PARARNN_API int pararnn_lstm_solve(const pararnn_cell *cell, const pararnn_params *params, const void *x,
+                                   const float *c0, const float *h0, int B, int T, float tol, int max_iters,
+                                   float *c, float *h, pararnn_info *info, void *workspace, size_t ws_bytes,
+                                   pararnn_stream stream);
+
+/* pararnn_lstm_workspace_size -- bytes pararnn_lstm_solve needs (P, one
+ * iterate copy, look-back words), or 0 for rejected arguments. */
+PARARNN_API size_t pararnn_lstm_workspace_size(const pararnn_cell *cell, int B, int T);
 
 /* pararnn_status_string -- a static, human-readable name of a status code. */
 PARARNN_API const char *pararnn_status_string(int status);

@@ -17,7 +17,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpararnn
 
 DEER, QUASI, ELK, QUASI_ELK = 0, 1, 2, 3
 MODES = {"DEER": DEER, "QUASI": QUASI, "ELK": ELK, "QUASI_ELK": QUASI_ELK}
-GRU_DENSE, GRU_DIAG = 0, 1
+GRU_DENSE, GRU_DIAG, LSTM_DIAG = 0, 1, 2
 F32, BF16 = 0, 1
 STATUS = {0: "OK", 1: "NOT_CONVERGED", 2: "DIVERGED", 3: "INVALID_ARG", 4: "CUDA_ERROR",
           5: "TIMEOUT"}
@@ -27,7 +27,7 @@ EXPORTS = ("pararnn_workspace_size", "pararnn_newton_solve", "pararnn_newton_sol
            "pararnn_affine_scan_status", "pararnn_status_string", "pararnn_newton_solve_host",
            "pararnn_host_workspace_size", "pararnn_adjoint", "pararnn_adjoint_workspace_size",
            "pararnn_adjoint_status", "pararnn_newton_solve_guess_async", "pararnn_newton_solve_chunked",
-           "pararnn_chunked_workspace_size")
+           "pararnn_chunked_workspace_size", "pararnn_lstm_solve", "pararnn_lstm_workspace_size")
 
 
 class Cell(ctypes.Structure):
@@ -96,6 +96,11 @@ def lib() -> ctypes.CDLL:
         L.pararnn_newton_solve_chunked.restype = ci
         L.pararnn_chunked_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci, ci, ci]
         L.pararnn_chunked_workspace_size.restype = sz
+        L.pararnn_lstm_solve.argtypes = [ctypes.POINTER(Cell), ctypes.POINTER(Params), vp, vp, vp, ci, ci, cf, ci,
+                                         vp, vp, ctypes.POINTER(Info), vp, sz, vp]
+        L.pararnn_lstm_solve.restype = ci
+        L.pararnn_lstm_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci]
+        L.pararnn_lstm_workspace_size.restype = sz
         L.pararnn_status_string.argtypes = [ci]
         L.pararnn_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -124,8 +129,39 @@ def _stream(stream) -> int:
 
 
 def make_cell(kind: str, din: int, d: int, dtype: torch.dtype) -> Cell:
-    return Cell(GRU_DENSE if kind == "dense" else GRU_DIAG, din, d, _dtype_code(dtype),
-                _dtype_code(dtype))
+    code = {"dense": GRU_DENSE, "diag": GRU_DIAG, "lstm_diag": LSTM_DIAG}[kind]
+    return Cell(code, din, d, _dtype_code(dtype), _dtype_code(dtype))
+
+
+def lstm_workspace_size(din: int, d: int, B: int, T: int, dtype: torch.dtype = torch.float32) -> int:
+    cell = make_cell("lstm_diag", din, d, dtype)
+    return int(lib().pararnn_lstm_workspace_size(ctypes.byref(cell), B, T))
+
+
+def lstm_solve(w_ih, b_ih, u, b_hh, x, c0, h0, *, tol: float, max_iters: int = 0, out=None, workspace=None,
+               stream=None):
+    """Evaluate the diagonal-recurrence LSTM over x [B, T, Din] by exact Newton.
+    Weights: w_ih [4D, Din] (x's dtype), b_ih, u, b_hh [4D] fp32; c0, h0 [B, D].
+    Returns (c, h, SolveResult) with c, h [B, T, D] fp32 CUDA tensors."""
+    B, T, din = x.shape
+    d = h0.shape[1]
+    cell = make_cell("lstm_diag", din, d, x.dtype)
+    L = lib()
+    need = int(L.pararnn_lstm_workspace_size(ctypes.byref(cell), B, T))
+    if need == 0:
+        raise ValueError("arguments rejected by pararnn_lstm_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, x.device)
+    c, h = out if out is not None else (torch.empty(B, T, d, dtype=torch.float32, device=x.device),
+                                        torch.empty(B, T, d, dtype=torch.float32, device=x.device))
+    params = Params(_dev(w_ih, "w_ih"), _dev(b_ih, "b_ih"), _dev(u, "u"), _dev(b_hh, "b_hh"))
+    info = Info()
+    rc = L.pararnn_lstm_solve(ctypes.byref(cell), ctypes.byref(params), _dev(x, "x"), _dev(c0, "c0"), _dev(h0, "h0"),
+                              B, T, float(tol), int(max_iters), _dev(c, "c"), _dev(h, "h"), ctypes.byref(info),
+                              _dev(workspace, "workspace"), workspace.numel(), _stream(stream))
+    if rc in (3, 4):
+        raise RuntimeError(f"pararnn_lstm_solve: {L.pararnn_status_string(rc).decode()}")
+    return c, h, SolveResult(h, info.iters, STATUS[info.status], info.delta, info.residual)
 
 
 def workspace_size(kind: str, din: int, d: int, B: int, T: int, mode: str,

@@ -32,6 +32,10 @@ cudaError_t launch_diag2(const DiagArgs &a, cudaStream_t s);
 cudaError_t launch_scan_dense(const float *A, const float *b, const float *h0, int B, int T,
                               int D, float *h, void *ws, cudaStream_t s);
 size_t scan_dense_ws_bytes(int B, int T, int D);
+size_t lstm_diag_desc_bytes(int B, int T, int D);
+cudaError_t launch_lstm_diag(const float *P, const float *u, const float *b_hh, const float *c0, const float *h0,
+                             int B, int T, int D, float tol, int max_iters, float *c_ws, float *h_ws, float *c_out,
+                             float *h_out, void *hdr, void *desc, pararnn_info *info_out, cudaStream_t s);
 size_t adjoint_diag_desc_bytes(int B, int T, int D);
 size_t adjoint_diag_part_bytes(int B, int T, int D);
 cudaError_t launch_adjoint_diag(const float *P, const float *h0, const float *h, const float *dh, const float *u,
@@ -410,6 +414,76 @@ int pararnn_affine_scan_status(const void *workspace, pararnn_stream stream) {
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
     return (st & kStatusTimeout) ? PARARNN_TIMEOUT : PARARNN_OK;
+}
+
+// ---- diagonal-recurrence LSTM ------------------------------------------------
+
+namespace {
+struct LstmLayout {
+    size_t header, P, cws, hws, desc, total;
+};
+bool lstm_cell_ok(const pararnn_cell *cell, int B, int T) {
+    if (!cell || cell->kind != PARARNN_LSTM_DIAG || B < 1 || T < 1) return false;
+    if (cell->d < 4 || cell->d % 4 != 0 || cell->din < 1 || cell->x_dtype != cell->w_dtype) return false;
+    if (cell->x_dtype != PARARNN_F32 && cell->x_dtype != PARARNN_BF16) return false;
+    return static_cast<long long>(T) * 4 * cell->d <= (1ll << 31) && static_cast<long long>(B) * T < (1ll << 31);
+}
+LstmLayout lstm_layout(const pararnn_cell &cell, int B, int T) {
+    LstmLayout L{};
+    const size_t states = static_cast<size_t>(B) * T * cell.d;
+    size_t off = 0;
+    L.header = off; off += 256;
+    L.P = off; off = align256(off + states * 4 * sizeof(float));
+    L.cws = off; off = align256(off + states * sizeof(float));
+    L.hws = off; off = align256(off + states * sizeof(float));
+    L.desc = off; off = align256(off + lstm_diag_desc_bytes(B, T, cell.d));
+    L.total = off;
+    return L;
+}
+}  // namespace
+
+size_t pararnn_lstm_workspace_size(const pararnn_cell *cell, int B, int T) {
+    return lstm_cell_ok(cell, B, T) ? lstm_layout(*cell, B, T).total : 0;
+}
+
+int pararnn_lstm_solve(const pararnn_cell *cell, const pararnn_params *params, const void *x, const float *c0,
+                       const float *h0, int B, int T, float tol, int max_iters, float *c, float *h, pararnn_info *info,
+                       void *workspace, size_t ws_bytes, pararnn_stream stream) {
+    if (!lstm_cell_ok(cell, B, T) || !params || !params->w_ih || !params->b_ih || !params->w_hh || !params->b_hh)
+        return PARARNN_INVALID_ARG;
+    if (!x || !c0 || !h0 || !c || !h || !workspace || !(tol >= 0.f) || !std::isfinite(tol)) return PARARNN_INVALID_ARG;
+    const LstmLayout L = lstm_layout(*cell, B, T);
+    if (ws_bytes < L.total) return PARARNN_INVALID_ARG;
+    const void *ptrs[] = {x, c0, h0, c, h, params->w_ih, params->b_ih, params->w_hh, params->b_hh};
+    for (const void *q : ptrs)
+        if (!aligned(q, 16)) return PARARNN_INVALID_ARG;
+    if (!aligned(workspace, 256)) return PARARNN_INVALID_ARG;
+    const size_t sb = static_cast<size_t>(B) * T * cell->d * 4;
+    const size_t xb = static_cast<size_t>(B) * T * cell->din * (cell->x_dtype == PARARNN_BF16 ? 2 : 4);
+    const size_t bd = static_cast<size_t>(B) * cell->d * 4;
+    if (overlaps(c, sb, h, sb) || overlaps(c, sb, workspace, L.total) || overlaps(h, sb, workspace, L.total) ||
+        overlaps(c, sb, x, xb) || overlaps(h, sb, x, xb) || overlaps(c, sb, c0, bd) || overlaps(c, sb, h0, bd) ||
+        overlaps(h, sb, c0, bd) || overlaps(h, sb, h0, bd))
+        return PARARNN_INVALID_ARG;
+    char *ws = static_cast<char *>(workspace);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    float *P = reinterpret_cast<float *>(ws + L.P);
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws + L.header);
+    cudaError_t e = cudaMemsetAsync(ws + L.header, 0, 256, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.desc, 0, L.total - L.desc, s);
+    if (e == cudaSuccess)
+        e = launch_projection_n(cell->x_dtype, x, params->w_ih, params->b_ih, P, static_cast<long long>(B) * T,
+                                4 * cell->d, cell->din, s);
+    if (e == cudaSuccess)
+        e = launch_lstm_diag(P, params->w_hh, params->b_hh, c0, h0, B, T, cell->d, tol, max_iters,
+                             reinterpret_cast<float *>(ws + L.cws), reinterpret_cast<float *>(ws + L.hws), c, h, hdr,
+                             ws + L.desc, nullptr, s);
+    pararnn_info host{};
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&host, &hdr->info, sizeof(host), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
+    if (info) *info = host;
+    return host.status;
 }
 
 // ---- backward pass (diagonal cell) -------------------------------------------

@@ -189,14 +189,13 @@ proj_tcgen05_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_cons
 
 }  // namespace
 
-bool proj_tcgen05_supported(const pararnn_cell &cell) {
-    return cell.x_dtype == PARARNN_BF16 && cell.din % BK == 0 && (3 * cell.d) % BN == 0 &&
-           encode_fn() != nullptr;
+// N output columns (gate rows x lanes), K = Din.
+bool proj_tcgen05_supported(int x_dtype, int N, int K) {
+    return x_dtype == PARARNN_BF16 && K % BK == 0 && N % BN == 0 && encode_fn() != nullptr;
 }
 
-cudaError_t launch_proj_tcgen05(const pararnn_cell &cell, const void *x, const void *w_ih,
-                                const float *b_ih, float *P, long long M, cudaStream_t s) {
-    const int N = 3 * cell.d, K = cell.din;
+cudaError_t launch_proj_tcgen05(const void *x, const void *w_ih, const float *b_ih, float *P, long long M, int N,
+                                int K, cudaStream_t s) {
     CUtensorMap mx, mw, mp;
     if (!make_map(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, M, K, BK, BM) ||
         !make_map(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w_ih, N, K, BK, BN) ||

@@ -85,18 +85,18 @@ __global__ void __launch_bounds__(256) proj_gemm_kernel(const Tin *__restrict__ 
 
 }  // namespace
 
-bool proj_tcgen05_supported(const pararnn_cell &cell);
-cudaError_t launch_proj_tcgen05(const pararnn_cell &cell, const void *x, const void *w_ih,
-                                const float *b_ih, float *P, long long M, cudaStream_t s);
+bool proj_tcgen05_supported(int x_dtype, int N, int K);
+cudaError_t launch_proj_tcgen05(const void *x, const void *w_ih, const float *b_ih, float *P, long long M, int N,
+                                int K, cudaStream_t s);
 
 // bf16 operands with Din a multiple of 64 and 3D a multiple of 256 take the
 // tcgen05 kernel (proj_tcgen05.cu); everything else this CUDA-core kernel.
-cudaError_t launch_projection(const pararnn_cell &cell, const void *x, const void *w_ih,
-                              const float *b_ih, float *P, long long M, cudaStream_t s) {
-    if (proj_tcgen05_supported(cell)) return launch_proj_tcgen05(cell, x, w_ih, b_ih, P, M, s);
-    const int N = 3 * cell.d, K = cell.din;
+// P [M, N] = x [M, K] W^T + b, W [N, K] (x and W of dtype x_dtype).
+cudaError_t launch_projection_n(int x_dtype, const void *x, const void *w_ih, const float *b_ih, float *P,
+                                long long M, int N, int K, cudaStream_t s) {
+    if (proj_tcgen05_supported(x_dtype, N, K)) return launch_proj_tcgen05(x, w_ih, b_ih, P, M, N, K, s);
     const dim3 grid(static_cast<unsigned>((M + BM - 1) / BM), (N + BN - 1) / BN);
-    if (cell.x_dtype == PARARNN_BF16)
+    if (x_dtype == PARARNN_BF16)
         proj_gemm_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
             static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(w_ih), b_ih,
             P, M, N, K);
@@ -105,6 +105,12 @@ cudaError_t launch_projection(const pararnn_cell &cell, const void *x, const voi
                                                      static_cast<const float *>(w_ih), b_ih, P, M,
                                                      N, K);
     return cudaGetLastError();
+}
+
+// The GRU's projection: N = 3D gate rows.
+cudaError_t launch_projection(const pararnn_cell &cell, const void *x, const void *w_ih,
+                              const float *b_ih, float *P, long long M, cudaStream_t s) {
+    return launch_projection_n(cell.x_dtype, x, w_ih, b_ih, P, M, 3 * cell.d, cell.din, s);
 }
 
 }  // namespace pararnn

@@ -67,6 +67,8 @@ struct WsLayout {
 WsLayout ws_layout(const pararnn_cell &cell, int B, int T, int mode);
 
 // Kernel launchers (return a cudaError_t).
+cudaError_t launch_projection_n(int x_dtype, const void *x, const void *w_ih, const float *b_ih, float *P,
+                                long long M, int N, int K, cudaStream_t s);
 cudaError_t launch_projection(const pararnn_cell &cell, const void *x, const void *w_ih,
                               const float *b_ih, float *P, long long M, cudaStream_t s);
 cudaError_t launch_diag_solver(const pararnn_cell &cell, int mode, const DiagArgs &a,

@@ -198,3 +198,48 @@ def make_scan_input(B: int, T: int, D: int, *, dense: bool = False, seed: int = 
     h0 = _normal(g, (B, D), 1.0) * h0_std
     return ScanInput(A=A.contiguous(), b=b.contiguous(), h0=h0.contiguous(), dense=dense)
 
+
+
+@dataclass
+class LstmWorkload:
+    """A diagonal-recurrence LSTM problem (layouts row-major, contiguous):
+    w_ih [4D, Din] rows in gate order (i, f, g, o); b_ih [4D]; u [4D] the
+    recurrent vectors; b_hh [4D]; x [B, T, Din]; c0, h0 [B, D]."""
+
+    din: int
+    d: int
+    B: int
+    T: int
+    x_dtype: torch.dtype
+    w_ih: torch.Tensor
+    b_ih: torch.Tensor
+    u: torch.Tensor
+    b_hh: torch.Tensor
+    x: torch.Tensor
+    c0: torch.Tensor
+    h0: torch.Tensor
+    tol: float
+
+    @property
+    def states(self) -> int:
+        return self.B * self.T * self.d
+
+
+def make_lstm_workload(*, B: int = 8, T: int = 4096, d: int = 2048, din: int = 2048, seed: int = 0,
+                       x_dtype: torch.dtype = torch.bfloat16, tol: float = 1e-4, bias_std: float = 0.0,
+                       state_std: float = 0.0) -> LstmWorkload:
+    """The diagonal-recurrence LSTM with the diagonal GRU workload's
+    distributions: W_ih ~ N(0, 1/Din), u ~ U(-1, 1), x ~ N(0, 1), biases and
+    initial state 0 unless ``bias_std`` / ``state_std`` say otherwise; x and
+    W_ih in ``x_dtype`` (bf16 by default, as the diagonal GRU workload)."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    w_ih = _normal(g, (4 * d, din), 1.0 / din)
+    u = _uniform(g, (4 * d,), -1.0, 1.0)
+    b_ih = _normal(g, (4 * d,), 1.0) * bias_std
+    b_hh = _normal(g, (4 * d,), 1.0) * bias_std
+    x = _normal(g, (B, T, din), 1.0)
+    c0 = _normal(g, (B, d), 1.0) * state_std
+    h0 = _normal(g, (B, d), 1.0) * state_std
+    return LstmWorkload(din=din, d=d, B=B, T=T, x_dtype=x_dtype, w_ih=w_ih.to(x_dtype).contiguous(),
+                        b_ih=b_ih.contiguous(), u=u.contiguous(), b_hh=b_hh.contiguous(),
+                        x=x.to(x_dtype).contiguous(), c0=c0.contiguous(), h0=h0.contiguous(), tol=tol)
