@@ -89,6 +89,14 @@ BENCHES = {
         cpu_sample=dict(B=1, T=512), ref_sample=dict(B=1, T=128)),
 }
 ADJ_METRIC = "backward states/sec (B*T*D per s, gradients through the evaluated sequence)"
+# the diagonal-recurrence LSTM (state (c, h) per lane; exact Newton over 2x2 lane
+# blocks): reads P 16 + the guess (c, h) 8, writes (c, h) 8 = 32 B per lane-step
+BENCHES["lstm"] = dict(
+    workload="lstm", mode="LSTM", lam=0.0, bound="hbm", per_state=32,
+    kernel="lstm_diag_kernel (persistent, all iterations)",
+    desc="diagonal-recurrence LSTM Din=D=2048, B={B}/GPU, T={T}, bf16 x and W_ih, fp32 state (c, h), "
+         "exact Newton (2x2 lane Jacobians) tol 1e-4",
+    cpu_sample=dict(B=1, T=256), ref_sample=dict(B=1, T=64))
 # fp32 FMA peak for the ALU-bound row: 148 SMs x 128 fp32 lanes x 2 flop x
 # 1965 MHz (the part's maximum SM clock), in TFLOP/s.
 ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
@@ -204,10 +212,22 @@ def cpu_baseline_oracle(spec: dict, sample: dict):
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     except Exception:  # pragma: no cover
         cores = 1
+    mode = spec["mode"]
+    if mode == "LSTM":
+        from oracle.lstm import LSTM, lstm_newton_solve
+        from newton_solve_nonlinear_b200.inputs import make_lstm_workload
+        lw = make_lstm_workload(**sample)
+        lc = LSTM(w_ih=lw.w_ih.double().numpy(), b_ih=lw.b_ih.double().numpy(), u=lw.u.double().numpy(),
+                  b_hh=lw.b_hh.double().numpy())
+        t0 = time.perf_counter()
+        r = lstm_newton_solve(lc, lw.x.double().numpy(), lw.c0.double().numpy(), lw.h0.double().numpy(), lw.tol)
+        secs = time.perf_counter() - t0
+        return {"value": lw.states / secs, "unit": UNIT, "cores": cores, "kind": "oracle",
+                "sample": f"fp64 numpy oracle, exact Newton to tol {lw.tol:g} on B={lw.B}, T={lw.T}, D={lw.d} "
+                          f"({r['iters']} iterations, {secs:.1f} s); same distributions"}
     w = make_workload(spec["workload"], **sample)
     c = GRU.from_workload(w)
     x, h0 = w.x.double().numpy(), w.h0.double().numpy()
-    mode = spec["mode"]
     if mode == "ADJOINT":
         import numpy as np
         from oracle.adjoint import adjoint
@@ -248,7 +268,7 @@ def run_reference(args):
     v = statistics.median(steps)
     from newton_solve_nonlinear_b200.inputs import WORKLOADS
     metric = ADJ_METRIC if spec["mode"] == "ADJOINT" else METRIC
-    full = WORKLOADS[spec["workload"]]
+    full = WORKLOADS[spec["workload"]] if spec["workload"] in WORKLOADS else dict(B=8, T=4096)
     T = args.T or full["T"]
     line = {"impl": "reference", "metric": metric, "value": v, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
@@ -353,6 +373,103 @@ def run_adjoint(args):
                 "h2d_bytes_per_step": (P.numel() + h.numel() + dh.numel()) * 4,
                 "d2h_bytes_per_step": P.numel() * 4},
         "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def run_lstm(args):
+    """The diagonal-recurrence LSTM solve (projection + every Newton iteration)."""
+    import torch
+    import torch.distributed as dist
+    from newton_solve_nonlinear_b200 import binding
+    from newton_solve_nonlinear_b200.inputs import make_lstm_workload
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    spec = BENCHES[args.workload]
+    over = {"T": args.T} if args.T else {}
+    w = make_lstm_workload(seed=rank, **over)
+    B, T, D = w.B, w.T, w.d
+    states = B * T * D
+    g = lambda t: t.to(dev).contiguous()
+    w_ih, b_ih, u, b_hh, x, c0, h0 = map(g, (w.w_ih, w.b_ih, w.u, w.b_hh, w.x, w.c0, w.h0))
+    ws = binding.alloc_workspace(binding.lstm_workspace_size(w.din, D, B, T, w.x_dtype), dev)
+    out = (torch.empty(B, T, D, device=dev), torch.empty(B, T, D, device=dev))
+    stream = torch.cuda.current_stream(dev)
+    step = lambda: binding.lstm_solve(w_ih, b_ih, u, b_hh, x, c0, h0, tol=w.tol, out=out, workspace=ws)
+    res = None
+    for _ in range(args.warmup):
+        res = step()[2]
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with Clocks(local) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        for e0, e1 in evs:
+            e0.record(stream)
+            res = step()[2]
+            e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    max_ms = max_over_ranks(sum(ms), dev)
+    value = job_value(states, args.steps, world, max_ms)
+    # end to end: x from page-locked host memory, (c, h) back, each step
+    hx = w.x.pin_memory()
+    hc, hh = torch.empty(B, T, D).pin_memory(), torch.empty(B, T, D).pin_memory()
+    e2e_steps = max(1, min(args.steps, 3))
+    barrier()
+    torch.cuda.synchronize()
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record(stream)
+    for _ in range(e2e_steps):
+        x.copy_(hx, non_blocking=True)
+        step()
+        hc.copy_(out[0], non_blocking=True)
+        hh.copy_(out[1], non_blocking=True)
+    eb.record(stream)
+    torch.cuda.synchronize()
+    e2e_value = job_value(states, e2e_steps, world, max_over_ranks(ea.elapsed_time(eb), dev))
+    cpu = cpu_baseline_oracle(spec, spec["cpu_sample"]) if rank == 0 and world == 1 else None
+    hbm_peak, peak_kind = peaks()
+    avg_s = statistics.mean(ms) / 1e3
+    achieved = res.iters * states * spec["per_state"] / avg_s / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": spec["desc"].format(B=B, T=T), "name": args.workload, "B": B, "T": T, "D": D,
+                   "din": w.din, "cell": "lstm_diag", "mode": "DEER (exact, 2x2 lane blocks)", "tol": w.tol,
+                   "iters": res.iters, "status": res.status,
+                   "l2": f"inputs larger than L2 (126 MB): x {w.x.numel() * 2 / 1e6:.0f} MB, "
+                         f"P {states * 16 / 1e6:.0f} MB, (c, h) {states * 8 / 1e6:.0f} MB",
+                   "parallelism": f"replicas over sequences x{world}"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": None, "kernel": spec["kernel"],
+                     "algorithmic": f"{spec['per_state']} B/lane-step/iteration x {res.iters} iterations x "
+                                    f"{states} lane-steps (the solve's time includes the projection)",
+                     "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": w.x.numel() * w.x.element_size(),
+                "d2h_bytes_per_step": 2 * states * 4},
+        "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }
     if cpu is not None:
@@ -531,6 +648,8 @@ def main():
         return run_reference(args)
     if BENCHES[args.workload]["mode"] == "ADJOINT":
         return run_adjoint(args)
+    if BENCHES[args.workload]["mode"] == "LSTM":
+        return run_lstm(args)
     return run_ours(args)
 
 
