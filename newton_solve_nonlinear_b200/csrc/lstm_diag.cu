@@ -14,7 +14,7 @@
 //     g = tanh(p_g + u_g h + b_g), o = sig(p_o + u_o h + b_o),
 //     c' = f c + i g,  h' = o tanh(c').
 //
-// One cooperative launch runs every iteration.  CTAs of 512 threads walk tiles
+// One cooperative launch runs every iteration.  CTAs of 512 threads (two per SM) walk tiles
 // of (sequence, 64 lanes, 32 steps), chunk-major; thread (lane d, segment s)
 // owns 4 consecutive steps: it evaluates the cell and its 2x2 Jacobian at the
 // shifted guess, composes its steps' affine maps, the eight segments of a lane
@@ -218,7 +218,7 @@ __device__ __forceinline__ void lstm_cell(float pi, float pf, float pg, float po
     J.d = fmaf(tc * o * (1.f - o), uo, o * sech2 * dch);
 }
 
-__global__ void __launch_bounds__(LNT, 1) lstm_diag_kernel(LstmArgs S) {
+__global__ void __launch_bounds__(LNT, 2) lstm_diag_kernel(LstmArgs S) {
     __shared__ float seg_m[LSEGS][6][LDL];  // each segment's map
     __shared__ float carry[2][LDL];         // state entering the tile
     __shared__ unsigned red[32];
