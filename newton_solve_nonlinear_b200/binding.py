@@ -332,12 +332,13 @@ def adjoint_workspace_size(d: int, B: int, T: int, kind: str = "diag") -> int:
 
 
 def adjoint(w_hh, b_hh, P, h0, h, dh, *, workspace=None, out=None, stream=None, check: bool = False) -> dict:
-    """Backward pass of the diagonal-recurrence GRU through the states h:
-    gradients w.r.t. the pre-activations P [B,T,3D], h0 [B,D], the recurrent
-    vectors w_hh [3D] and b_hh [3D], given dh = dL/dh [B,T,D] (all fp32 CUDA).
-    Returns dict(dP, dh0, dw_hh, db_hh)."""
+    """Backward pass of the GRU through the states h: gradients w.r.t. the
+    pre-activations P [B,T,3D], h0 [B,D], w_hh and b_hh [3D], given
+    dh = dL/dh [B,T,D] (all fp32 CUDA).  w_hh [3D] is the diagonal cell (exact
+    gradients); w_hh [3D, D] the dense cell, whose adjoint runs with the
+    Jacobian's diagonal (D <= 64).  Returns dict(dP, dh0, dw_hh, db_hh)."""
     B, T, d = h.shape
-    cell = make_cell("diag", 1, d, torch.float32)
+    cell = make_cell("dense" if w_hh.dim() == 2 else "diag", 1, d, torch.float32)
     L = lib()
     need = int(L.pararnn_adjoint_workspace_size(ctypes.byref(cell), B, T))
     if need == 0:

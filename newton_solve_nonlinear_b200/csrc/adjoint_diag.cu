@@ -41,6 +41,11 @@ constexpr int ASL = ATS / ASEGS;   // 4 steps per thread
 
 struct AdjArgs {
     const float *P, *h0, *h, *dh, *u, *b_hh;  // u: [3D] recurrent vectors (r, z, n)
+    // dense cell (quasi backward): w_hh [3D, D] (the Jacobian's diagonal is read
+    // from it), G [B, T, 3D] = U h_{t-1} + b_hh, and grow [B, T, 3D] out: the
+    // gradient w.r.t. the recurrent pre-activations (dP with the n gate times r)
+    const float *w_hh, *G;
+    float *grow;
     float *dP, *dh0, *du, *db_hh;
     WsHeader *hdr;
     unsigned long long *desc;  // [n_tiles][ADL][2] look-back words
@@ -64,7 +69,22 @@ __device__ __forceinline__ void adj_cell(float pr, float pz, float pn, float hp,
     a = z + fz * uz + fn * r * un + fr * ur;
 }
 
-__global__ void __launch_bounds__(ANT, 2) adjoint_diag_kernel(AdjArgs S) {
+// The same for the dense cell at recurrent pre-activations q = U h_{t-1} + b_hh
+// (computed beforehand), with the Jacobian's diagonal entries ud of U.
+__device__ __forceinline__ void adj_cell_q(float pr, float pz, float pn, float qr, float qz, float qn, float hp,
+                                           float udr, float udz, float udn, float &fr, float &fz, float &fn,
+                                           float &r, float &a) {
+    r = sigmoidf_(pr + qr);
+    const float z = sigmoidf_(pz + qz);
+    const float n = tanhf_(pn + r * qn);
+    fn = (1.f - z) * (1.f - n * n);
+    fr = fn * qn * r * (1.f - r);
+    fz = (hp - n) * z * (1.f - z);
+    a = z + fz * udz + fn * r * udn + fr * udr;
+}
+
+template <bool DENSE>
+__global__ void __launch_bounds__(ANT, DENSE ? 1 : 2) adjoint_diag_kernel(AdjArgs S) {
     static_assert(ASEGS == 8, "the per-tile partial sums below add eight segments");
     __shared__ float seg_a[ASEGS][ADL], seg_b[ASEGS][ADL];
     __shared__ float carry[ADL];
@@ -91,14 +111,21 @@ __global__ void __launch_bounds__(ANT, 2) adjoint_diag_kernel(AdjArgs S) {
 
         float ur = 0.f, uz = 0.f, un = 0.f, br = 0.f, bz = 0.f, bn = 0.f;
         if (lane_ok) {
-            ur = __ldg(S.u + lane), uz = __ldg(S.u + D + lane), un = __ldg(S.u + 2 * D + lane);
-            br = __ldg(S.b_hh + lane), bz = __ldg(S.b_hh + D + lane), bn = __ldg(S.b_hh + 2 * D + lane);
+            if constexpr (DENSE) {  // the Jacobian's diagonal: U_g[lane][lane]
+                const size_t dd = static_cast<size_t>(lane) * D + lane;
+                ur = __ldg(S.w_hh + dd), uz = __ldg(S.w_hh + static_cast<size_t>(D) * D + dd);
+                un = __ldg(S.w_hh + 2 * static_cast<size_t>(D) * D + dd);
+            } else {
+                ur = __ldg(S.u + lane), uz = __ldg(S.u + D + lane), un = __ldg(S.u + 2 * D + lane);
+                br = __ldg(S.b_hh + lane), bz = __ldg(S.b_hh + D + lane), bn = __ldg(S.b_hh + 2 * D + lane);
+            }
         }
         // 1. the cell at the thread's 8 steps and the next one
         float fr[ASL], fz[ASL], fn[ASL], rr[ASL], hp[ASL], gg[ASL], al[ASL];
         float a_first = 0.f;
         {
             float pr[ASL + 1], pz[ASL + 1], pn[ASL + 1], hv[ASL + 1];
+            float qr[ASL + 1], qz[ASL + 1], qn[ASL + 1];  // dense: U h_{t-1} + b_hh
 #pragma unroll
             for (int i = 0; i <= ASL; ++i) {  // all loads in flight together
                 const int t = t0 + seg * ASL + i;
@@ -111,12 +138,20 @@ __global__ void __launch_bounds__(ANT, 2) adjoint_diag_kernel(AdjArgs S) {
                                      : __ldcs(S.h + (row0 + t - 1) * D + lane))
                            : 0.f;
                 if (i < ASL) gg[i] = ok ? __ldcs(S.dh + (row0 + t) * D + lane) : 0.f;
+                if constexpr (DENSE) {
+                    qr[i] = ok ? __ldcs(S.G + o) : 0.f;
+                    qz[i] = ok ? __ldcs(S.G + o + D) : 0.f;
+                    qn[i] = ok ? __ldcs(S.G + o + 2 * D) : 0.f;
+                }
             }
 #pragma unroll
             for (int i = 0; i <= ASL; ++i) {
                 const int t = t0 + seg * ASL + i;
                 float f_r, f_z, f_n, r_, a_;
-                adj_cell(pr[i], pz[i], pn[i], hv[i], ur, uz, un, br, bz, bn, f_r, f_z, f_n, r_, a_);
+                if constexpr (DENSE)
+                    adj_cell_q(pr[i], pz[i], pn[i], qr[i], qz[i], qn[i], hv[i], ur, uz, un, f_r, f_z, f_n, r_, a_);
+                else
+                    adj_cell(pr[i], pz[i], pn[i], hv[i], ur, uz, un, br, bz, bn, f_r, f_z, f_n, r_, a_);
                 if (i < ASL) {
                     fr[i] = f_r, fz[i] = f_z, fn[i] = f_n, rr[i] = r_, hp[i] = hv[i];
                     if (i == 0) a_first = a_;
@@ -169,6 +204,11 @@ __global__ void __launch_bounds__(ANT, 2) adjoint_diag_kernel(AdjArgs S) {
                     __stcs(S.dP + o, gr);
                     __stcs(S.dP + o + D, gz);
                     __stcs(S.dP + o + 2 * D, gn);
+                    if constexpr (DENSE) {  // for dW_hh = sum grow (outer) h_{t-1}, a GEMM after this pass
+                        __stcs(S.grow + o, gr);
+                        __stcs(S.grow + o + D, gz);
+                        __stcs(S.grow + o + 2 * D, gnr);
+                    }
                     q_r += gr, q_z += gz, q_n += gnr;
                     s_r = fmaf(gr, hp[i], s_r), s_z = fmaf(gz, hp[i], s_z), s_n = fmaf(gnr, hp[i], s_n);
                     if (t == 0) S.dh0[static_cast<size_t>(b) * D + lane] = a_first * lam;
@@ -204,7 +244,7 @@ __global__ void __launch_bounds__(ANT, 2) adjoint_diag_kernel(AdjArgs S) {
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (wl == 0) {
+        if (wl == 0 && (k >= 3 || !DENSE)) {  // dense: dW_hh comes from the GEMM after this pass
             float *dst = k < 3 ? S.du : S.db_hh;
             dst[(k % 3) * D + lane] = acc;
         }
@@ -222,11 +262,104 @@ size_t adjoint_diag_part_bytes(int B, int T, int D) {
     return static_cast<size_t>(tiles) * 6 * ADL * 4;
 }
 
+namespace {
+
+// dW_hh [N, K] = sum over the M rows m of grow[m, :N] (outer) hp[m, :K]
+// (grow [M, 3D], hp [M, D]): each CTA sums a chunk of OSR rows into its own
+// partial (no atomics), a second pass adds the partials in chunk order, so the
+// result does not depend on scheduling.
+constexpr int OSR = 512;   // rows per chunk
+constexpr int OSM = 32;    // rows per shared-memory stage
+constexpr int OST = 256;   // threads: 32 row groups x 8 column groups
+constexpr int ONI = 6, OKJ = 8;  // outputs per thread: n = nb + 32 i (i < 6), k = kb + 8 j (j < 8)
+__global__ void __launch_bounds__(OST) outer_sum_partial_kernel(const float *grow, const float *hp, long long M,
+                                                                int N, int K, float *part) {
+    extern __shared__ float osm[];  // [OSM][N] grow rows, then [OSM][K] hp rows
+    float *sg = osm, *sh = osm + OSM * N;
+    const long long m0 = static_cast<long long>(blockIdx.x) * OSR;
+    const int tid = threadIdx.x;
+    const int kb = tid % OKJ, nb = tid / OKJ;  // N <= 32 * 6, K <= 8 * 8
+    float acc[ONI][OKJ];
+#pragma unroll
+    for (int i = 0; i < ONI; ++i)
+#pragma unroll
+        for (int j = 0; j < OKJ; ++j) acc[i][j] = 0.f;
+    for (long long mb = m0; mb < m0 + OSR && mb < M; mb += OSM) {
+        const int rows = M - mb < OSM ? static_cast<int>(M - mb) : OSM;
+        __syncthreads();
+        for (int i = tid; i < OSM * N; i += OST) {
+            const int r = i / N;
+            sg[i] = r < rows ? __ldcs(grow + (mb + r) * N + i % N) : 0.f;
+        }
+        for (int i = tid; i < OSM * K; i += OST) {
+            const int r = i / K;
+            sh[i] = r < rows ? __ldcs(hp + (mb + r) * K + i % K) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int r = 0; r < OSM; ++r) {
+            float gv[ONI], hv[OKJ];
+#pragma unroll
+            for (int i = 0; i < ONI; ++i) {
+                const int n = nb + 32 * i;
+                gv[i] = n < N ? sg[r * N + n] : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < OKJ; ++j) {
+                const int k = kb + OKJ * j;
+                hv[j] = k < K ? sh[r * K + k] : 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < ONI; ++i)
+#pragma unroll
+                for (int j = 0; j < OKJ; ++j) acc[i][j] = fmaf(gv[i], hv[j], acc[i][j]);
+        }
+    }
+    float *dst = part + static_cast<size_t>(blockIdx.x) * N * K;
+#pragma unroll
+    for (int i = 0; i < ONI; ++i)
+#pragma unroll
+        for (int j = 0; j < OKJ; ++j) {
+            const int n = nb + 32 * i, k = kb + OKJ * j;
+            if (n < N && k < K) dst[n * K + k] = acc[i][j];
+        }
+}
+__global__ void outer_sum_reduce_kernel(const float *part, int nchunks, int NK, float *out) {
+    const int o = blockIdx.x * blockDim.x + threadIdx.x;
+    if (o >= NK) return;
+    float a = 0.f;
+    for (int c = 0; c < nchunks; ++c) a += __ldcg(part + static_cast<size_t>(c) * NK + o);
+    out[o] = a;
+}
+
+}  // namespace
+
+size_t adjoint_outer_part_bytes(long long M, int N, int K) {
+    return static_cast<size_t>((M + OSR - 1) / OSR) * N * K * 4;
+}
+
+cudaError_t launch_outer_sum(const float *grow, const float *hp, long long M, int N, int K, float *part, float *out,
+                             cudaStream_t s) {
+    if (N > 32 * ONI || K > OKJ * OKJ) return cudaErrorInvalidValue;
+    const long long nchunks = (M + OSR - 1) / OSR;
+    const size_t smem = static_cast<size_t>(OSM) * (N + K) * 4;
+    cudaError_t e = cudaFuncSetAttribute(outer_sum_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    outer_sum_partial_kernel<<<static_cast<unsigned>(nchunks), OST, smem, s>>>(grow, hp, M, N, K, part);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int NK = N * K;
+    outer_sum_reduce_kernel<<<(NK + 255) / 256, 256, 0, s>>>(part, static_cast<int>(nchunks), NK, out);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_adjoint_diag(const float *P, const float *h0, const float *h, const float *dh, const float *u,
                                 const float *b_hh, float *dP, float *dh0, float *du, float *db_hh, int B, int T,
-                                int D, void *hdr, void *desc, void *part, cudaStream_t s) {
+                                int D, void *hdr, void *desc, void *part, cudaStream_t s, const float *w_hh_dense,
+                                const float *G, float *grow) {
     AdjArgs S;
     S.P = P, S.h0 = h0, S.h = h, S.dh = dh, S.u = u, S.b_hh = b_hh;
+    S.w_hh = w_hh_dense, S.G = G, S.grow = grow;
     S.dP = dP, S.dh0 = dh0, S.du = du, S.db_hh = db_hh;
     S.hdr = static_cast<WsHeader *>(hdr);
     S.desc = static_cast<unsigned long long *>(desc);
@@ -236,16 +369,18 @@ cudaError_t launch_adjoint_diag(const float *P, const float *h0, const float *h,
     S.ngroups = B * S.ndg;
     S.n_chunks = (T + ATS - 1) / ATS;
     S.n_tiles = static_cast<long long>(S.ngroups) * S.n_chunks;
+    const bool dense = G != nullptr;
+    const void *kern = dense ? reinterpret_cast<const void *>(adjoint_diag_kernel<true>)
+                             : reinterpret_cast<const void *>(adjoint_diag_kernel<false>);
     int dev = 0, nsm = 0, per_sm = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adjoint_diag_kernel, ANT, 0);
+    if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, ANT, 0);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     long long grid = static_cast<long long>(nsm) * per_sm;
     void *params[] = {&S};
-    return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(adjoint_diag_kernel),
-                                       dim3(static_cast<unsigned>(grid)), dim3(ANT), params, 0, s);
+    return cudaLaunchCooperativeKernel(kern, dim3(static_cast<unsigned>(grid)), dim3(ANT), params, 0, s);
 }
 
 }  // namespace pararnn

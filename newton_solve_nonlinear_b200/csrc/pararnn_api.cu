@@ -40,7 +40,11 @@ size_t adjoint_diag_desc_bytes(int B, int T, int D);
 size_t adjoint_diag_part_bytes(int B, int T, int D);
 cudaError_t launch_adjoint_diag(const float *P, const float *h0, const float *h, const float *dh, const float *u,
                                 const float *b_hh, float *dP, float *dh0, float *du, float *db_hh, int B, int T,
-                                int D, void *hdr, void *desc, void *part, cudaStream_t s);
+                                int D, void *hdr, void *desc, void *part, cudaStream_t s, const float *w_hh_dense,
+                                const float *G, float *grow);
+size_t adjoint_outer_part_bytes(long long M, int N, int K);
+cudaError_t launch_outer_sum(const float *grow, const float *hp, long long M, int N, int K, float *part, float *out,
+                             cudaStream_t s);
 
 namespace {
 
@@ -490,23 +494,33 @@ int pararnn_lstm_solve(const pararnn_cell *cell, const pararnn_params *params, c
 
 namespace {
 struct AdjLayout {
-    size_t header, desc, part, total;
+    size_t header, desc, part, hprev, G, grow, opart, total;
 };
-AdjLayout adj_layout(int B, int T, int D) {
+// dense: + h_{t-1} [B, T, D], U h_{t-1} + b_hh [B, T, 3D], grow [B, T, 3D] and
+// the dW_hh GEMM's per-chunk partials
+AdjLayout adj_layout(int B, int T, int D, bool dense) {
     AdjLayout L{};
     size_t off = 0;
     L.header = off; off += 256;
     L.desc = off; off = align256(off + adjoint_diag_desc_bytes(B, T, D));
     L.part = off; off = align256(off + adjoint_diag_part_bytes(B, T, D));
+    if (dense) {
+        const size_t st = static_cast<size_t>(B) * T * D * 4;
+        L.hprev = off; off = align256(off + st);
+        L.G = off; off = align256(off + 3 * st);
+        L.grow = off; off = align256(off + 3 * st);
+        L.opart = off; off = align256(off + adjoint_outer_part_bytes(static_cast<long long>(B) * T, 3 * D, D));
+    }
     L.total = off;
     return L;
 }
 }  // namespace
 
 size_t pararnn_adjoint_workspace_size(const pararnn_cell *cell, int B, int T) {
-    if (!cell || cell->kind != PARARNN_GRU_DIAG || cell->d < 1 || B < 1 || T < 1) return 0;
+    if (!cell || cell->d < 1 || B < 1 || T < 1) return 0;
+    if (cell->kind != PARARNN_GRU_DIAG && !(cell->kind == PARARNN_GRU_DENSE && cell->d <= 64)) return 0;
     if (static_cast<long long>(B) * T >= (1ll << 31) - 1) return 0;
-    return adj_layout(B, T, cell->d).total;
+    return adj_layout(B, T, cell->d, cell->kind == PARARNN_GRU_DENSE).total;
 }
 
 int pararnn_adjoint(const pararnn_cell *cell, const pararnn_params *params, const float *P, const float *h0,
@@ -520,25 +534,50 @@ int pararnn_adjoint(const pararnn_cell *cell, const pararnn_params *params, cons
         if (!aligned(q, 16)) return PARARNN_INVALID_ARG;
     if (!aligned(workspace, 256)) return PARARNN_INVALID_ARG;
     const int D = cell->d;
+    const bool dense = cell->kind == PARARNN_GRU_DENSE;
     const size_t st = static_cast<size_t>(B) * T * D * 4;
-    const size_t bd = static_cast<size_t>(B) * D * 4, pd = static_cast<size_t>(3) * D * 4;
+    const size_t bd = static_cast<size_t>(B) * D * 4, pd = static_cast<size_t>(3) * D * 4 * (dense ? D : 1);
+    const size_t bb = static_cast<size_t>(3) * D * 4;  // b_hh and db_hh
     const struct { const void *p; size_t n; } ins[] = {{P, 3 * st}, {h0, bd}, {h, st}, {dh, st},
-                                                       {params->w_hh, pd}, {params->b_hh, pd}, {workspace, need}};
-    const struct { const void *p; size_t n; } outs[] = {{dP, 3 * st}, {dh0, bd}, {dw_hh, pd}, {db_hh, pd}};
+                                                       {params->w_hh, pd}, {params->b_hh, bb}, {workspace, need}};
+    const struct { const void *p; size_t n; } outs[] = {{dP, 3 * st}, {dh0, bd}, {dw_hh, pd}, {db_hh, bb}};
     for (const auto &o : outs) {
         for (const auto &i : ins)
             if (overlaps(o.p, o.n, i.p, i.n)) return PARARNN_INVALID_ARG;
         for (const auto &o2 : outs)
             if (&o2 != &o && overlaps(o.p, o.n, o2.p, o2.n)) return PARARNN_INVALID_ARG;
     }
-    const AdjLayout L = adj_layout(B, T, D);
+    const AdjLayout L = adj_layout(B, T, D, dense);
     char *ws = static_cast<char *>(workspace);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // header (status, grid barrier) and look-back words start at zero
     cudaError_t e = cudaMemsetAsync(ws, 0, L.part, s);
+    if (!dense) {
+        if (e == cudaSuccess)
+            e = launch_adjoint_diag(P, h0, h, dh, params->w_hh, params->b_hh, dP, dh0, dw_hh, db_hh, B, T, D,
+                                    ws + L.header, ws + L.desc, ws + L.part, s, nullptr, nullptr, nullptr);
+        return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
+    }
+    // dense cell: h_{t-1} packed [B, T, D] (h0, then the states shifted by one step)
+    float *hp = reinterpret_cast<float *>(ws + L.hprev);
+    const size_t row = static_cast<size_t>(D) * 4, seq = static_cast<size_t>(T) * D * 4;
+    if (e == cudaSuccess) e = cudaMemcpy2DAsync(hp, seq, h0, row, row, B, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess && T > 1)
+        e = cudaMemcpy2DAsync(reinterpret_cast<char *>(hp) + row, seq, h, seq, seq - row, B, cudaMemcpyDeviceToDevice, s);
+    // U h_{t-1} + b_hh for every step: one fp32 GEMM
+    float *G = reinterpret_cast<float *>(ws + L.G);
     if (e == cudaSuccess)
-        e = launch_adjoint_diag(P, h0, h, dh, params->w_hh, params->b_hh, dP, dh0, dw_hh, db_hh, B, T, D,
-                                ws + L.header, ws + L.desc, ws + L.part, s);
+        e = launch_projection_n(PARARNN_F32, hp, params->w_hh, params->b_hh, G, static_cast<long long>(B) * T, 3 * D,
+                                D, s);
+    // the reverse scan with the Jacobian's diagonal; dP, dh0, db_hh and grow
+    float *grow = reinterpret_cast<float *>(ws + L.grow);
+    if (e == cudaSuccess)
+        e = launch_adjoint_diag(P, h0, h, dh, nullptr, params->b_hh, dP, dh0, nullptr, db_hh, B, T, D, ws + L.header,
+                                ws + L.desc, ws + L.part, s, params->w_hh, G, grow);
+    // dW_hh = sum over steps of grow (outer) h_{t-1}
+    if (e == cudaSuccess)
+        e = launch_outer_sum(grow, hp, static_cast<long long>(B) * T, 3 * D, D,
+                             reinterpret_cast<float *>(ws + L.opart), dw_hh, s);
     return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
 }
 

@@ -1,4 +1,5 @@
-"""GPU parity of the backward pass (diagonal-recurrence GRU) vs the fp64 oracle.
+"""GPU parity of the backward pass vs the fp64 oracle: the diagonal-recurrence
+GRU (exact) and the dense GRU with the Jacobian's diagonal (the quasi backward).
 
 Inputs: a random diagonal cell, synthetic fp32 pre-activations P, the fp64
 rollout of the cell from P (rounded to fp32), and random upstream gradients.
@@ -80,14 +81,112 @@ def test_adjoint_full_size_sampled_lanes():
     _check(8, 4096, 2048, seed=7, lanes=list(range(0, 2048, 64)) + list(range(1000, 1064)))
 
 
-def test_adjoint_deterministic_and_rejects_dense():
+def test_adjoint_deterministic_and_rejects_wide_dense():
     cell, u, b_hh, P, h0, h, dh = _case(2, 300, 64, seed=3)
     args = [t.cuda() for t in (u, b_hh, P, h0, h, dh)]
     r1 = binding.adjoint(*args)
     r2 = binding.adjoint(*args)
     for k in r1:
         assert torch.equal(r1[k], r2[k]), k
-    assert binding.adjoint_workspace_size(64, 2, 300, kind="dense") == 0
+    assert binding.adjoint_workspace_size(64, 2, 300, kind="dense") > 0
+    assert binding.adjoint_workspace_size(65, 2, 300, kind="dense") == 0
+
+
+def _dense_case(B, T, D, seed, scale=0.9):
+    """A random dense GRU (U [3D, D] with entries of std scale/sqrt(D)), P, h0,
+    the fp64 rollout from P (rounded to fp32) and upstream gradients."""
+    g = torch.Generator().manual_seed(seed)
+    w_hh = torch.randn(3 * D, D, generator=g) * (scale / D ** 0.5)
+    b_hh = torch.randn(3 * D, generator=g) * 0.3
+    P = torch.randn(B, T, 3 * D, generator=g)
+    h0 = torch.randn(B, D, generator=g) * 0.5
+    dh = torch.randn(B, T, D, generator=g)
+    cell = GRU(kind="dense", w_ih=np.eye(3 * D), b_ih=np.zeros(3 * D), w_hh=w_hh.double().numpy(),
+               b_hh=b_hh.double().numpy())
+    Pd = P.double().numpy()
+    hs, hv = [], h0.double().numpy()
+    for t in range(T):
+        hv = cell.gates(hv, Pd[:, t])[4]
+        hs.append(hv)
+    h = torch.from_numpy(np.stack(hs, 1)).float()
+    return cell, w_hh, b_hh, P, h0, h, dh
+
+
+@pytest.mark.parametrize("B,T,D", [(2, 100, 64), (3, 257, 32), (1, 1, 5), (2, 1030, 64), (1, 64, 48),
+                                   (4, 700, 12)])
+def test_dense_adjoint_matches_oracle_diag_jacobian(B, T, D):
+    """The dense cell's backward with the Jacobian's diagonal in the lam
+    recurrence, against the oracle's jacobian='diag' pass; dW_hh [3D, D] is
+    a sum over B*T outer products (normwise 1e-4 as above)."""
+    cell, w_hh, b_hh, P, h0, h, dh = _dense_case(B, T, D, seed=B * 7 + T + D)
+    r = binding.adjoint(w_hh.cuda(), b_hh.cuda(), P.cuda(), h0.cuda(), h.cuda(), dh.cuda(), check=True)
+    f64 = lambda t: t.double().numpy()
+    ref = oracle_adjoint(cell, f64(P), f64(h0), f64(h), f64(dh), jacobian="diag")
+    got = {k: v.double().cpu().numpy() for k, v in r.items()}
+    assert got["dw_hh"].shape == (3 * D, D)
+    for k in ("dP", "dh0", "dw_hh", "db_hh"):
+        assert _rel(got[k], ref[k]) <= 1e-4, k
+
+
+def test_dense_adjoint_full_size_deterministic():
+    """The dense workloads' size (B = 16, T = 65536, D = 64): two runs are
+    bitwise equal; dP and dh0 of sequence 0 match the oracle run on that
+    sequence alone (sequences are independent); db_hh and dW_hh match fp64
+    sums formed from the returned dP over all sequences."""
+    B, T, D = 16, 65536, 64
+    g = torch.Generator().manual_seed(11)
+    w_hh = torch.randn(3 * D, D, generator=g) * (0.9 / D ** 0.5)
+    b_hh = torch.randn(3 * D, generator=g) * 0.3
+    P = torch.randn(B, T, 3 * D, generator=g)
+    h0 = torch.randn(B, D, generator=g) * 0.5
+    dh = torch.randn(B, T, D, generator=g)
+    cell = GRU(kind="dense", w_ih=np.eye(3 * D), b_ih=np.zeros(3 * D), w_hh=w_hh.double().numpy(),
+               b_hh=b_hh.double().numpy())
+    # states: an fp32 rollout on the CPU (torch ops); the oracle reads the same h
+    h = torch.empty(B, T, D)
+    hv = h0.clone()
+    Pc = P
+    for t in range(T):
+        q = hv @ w_hh.T + b_hh
+        r_ = torch.sigmoid(Pc[:, t, :D] + q[:, :D])
+        z_ = torch.sigmoid(Pc[:, t, D:2 * D] + q[:, D:2 * D])
+        n_ = torch.tanh(Pc[:, t, 2 * D:] + r_ * q[:, 2 * D:])
+        hv = (1 - z_) * n_ + z_ * hv
+        h[:, t] = hv
+    args = [t.cuda() for t in (w_hh, b_hh, P, h0, h, dh)]
+    r1 = binding.adjoint(*args, check=True)
+    r2 = binding.adjoint(*args)
+    for k in r1:
+        assert torch.equal(r1[k], r2[k]), k
+    f64 = lambda t: t.double().numpy()
+    ref = oracle_adjoint(cell, f64(P[:1]), f64(h0[:1]), f64(h[:1]), f64(dh[:1]), jacobian="diag")
+    got = {k: v.double().cpu().numpy() for k, v in r1.items()}
+    assert _rel(got["dP"][:1], ref["dP"]) <= 1e-4
+    assert _rel(got["dh0"][:1], ref["dh0"]) <= 1e-4
+    # the parameter sums from the kernel's own dP, in fp64: db_hh exactly
+    # from dP and r; dW_hh from grow (outer) h_{t-1}
+    Pd, hd = f64(P), f64(h)
+    hp = np.concatenate([f64(h0)[:, None], hd[:, :-1]], 1)
+    q = hp @ f64(w_hh).T + f64(b_hh)
+    rg = 1 / (1 + np.exp(-(Pd[..., :D] + q[..., :D])))
+    dP = got["dP"]
+    grow = np.concatenate([dP[..., :2 * D], dP[..., 2 * D:] * rg], -1)
+    assert _rel(got["db_hh"], grow.sum((0, 1))) <= 1e-4
+    assert _rel(got["dw_hh"], np.einsum("btk,btj->kj", grow, hp)) <= 1e-4
+
+
+def test_dense_adjoint_with_diagonal_u_equals_diagonal_cell():
+    """A dense U that is diagonal per gate is the diagonal cell: the two paths
+    give the same dP, dh0, db_hh, and dW_hh's diagonal blocks equal du."""
+    B, T, D = 2, 500, 64
+    cell, u, b_hh, P, h0, h, dh = _case(B, T, D, seed=21)
+    U = torch.cat([torch.diag(u[k * D:(k + 1) * D]) for k in range(3)], 0)
+    rd = binding.adjoint(u.cuda(), b_hh.cuda(), P.cuda(), h0.cuda(), h.cuda(), dh.cuda())
+    rD = binding.adjoint(U.cuda(), b_hh.cuda(), P.cuda(), h0.cuda(), h.cuda(), dh.cuda())
+    for k in ("dP", "dh0", "db_hh"):
+        assert _rel(rD[k].double().cpu().numpy(), rd[k].double().cpu().numpy()) <= 1e-5, k
+    diag = torch.cat([torch.diagonal(rD["dw_hh"][k * D:(k + 1) * D]) for k in range(3)])
+    assert _rel(diag.double().cpu().numpy(), rd["dw_hh"].double().cpu().numpy()) <= 1e-5
 
 
 def test_adjoint_gives_autograd_gradients_of_a_solve():
