@@ -26,6 +26,13 @@ Readings of what the pages leave open (also listed in the design notes):
     DIVERGED; otherwise NOT_CONVERGED after max_iters iterations.  The default
     cap is T + 1: undamped Newton is exact after T iterations (each iteration
     fixes one more leading state), and one more iteration observes delta = 0.
+
+Jacobian reuse (approximate Newton: the Jacobian recomputed only every few
+steps, "ParaRNN" summary, "Newton's Iteration").  Reading: with period k,
+iteration i keeps the A_t of iteration k floor(i / k) and forms b_t from the
+new guess, b_t = f(h^(i)_{t-1}, x_t) - A_t h^(i)_{t-1} (the chord method in
+between refreshes).  The fixed point is unchanged, and since h_0 is fixed the
+first i states are still exact after i iterations.
 """
 from __future__ import annotations
 
@@ -59,19 +66,29 @@ def linearise(cell: GRU, h: np.ndarray, p: np.ndarray, h0: np.ndarray, dense: bo
     return A, b, f
 
 
+def kept_operands(A_kept: np.ndarray, f: np.ndarray, hp: np.ndarray, dense: bool):
+    """Scan operands with a kept Jacobian: A_t = A_kept_t and
+    b_t = f_t - A_kept_t h_{t-1}, f and h_{t-1} from the current guess."""
+    b = f - (np.einsum("btij,btj->bti", A_kept, hp) if dense else A_kept * hp)
+    return A_kept, b
+
+
 def newton_solve(cell: GRU, x: np.ndarray, h0: np.ndarray, mode: str, tol: float,
                  max_iters: int | None = None, h_init: np.ndarray | None = None,
-                 record: bool = False) -> dict:
+                 record: bool = False, jac_every: int = 1) -> dict:
     """Solve the unrolled system with DEER (mode 'DEER') or quasi-DEER ('QUASI').
 
     For the diagonal cell the Jacobian is diagonal, so both modes are exact
-    Newton and produce identical iterates.
+    Newton and produce identical iterates.  jac_every = k > 1 recomputes the
+    Jacobian only at iterations 0, k, 2k, ... (see the module notes).
 
     Returns a dict: h [B,T,D], iters, status, delta (last max |dh|),
     deltas (every iteration's delta) and, when ``record``, the list of iterates.
     """
     if mode not in ("DEER", "QUASI"):
         raise ValueError(mode)
+    if jac_every < 1:
+        raise ValueError(jac_every)
     x = np.asarray(x, np.float64)
     h0 = np.asarray(h0, np.float64)
     B, T, _ = x.shape
@@ -82,9 +99,14 @@ def newton_solve(cell: GRU, x: np.ndarray, h0: np.ndarray, mode: str, tol: float
     h = np.zeros((B, T, D)) if h_init is None else np.array(h_init, np.float64, copy=True)
     deltas, iterates = [], []
     status, iters = STATUS_NOT_CONVERGED, max_iters
+    A_kept = None
     for i in range(max_iters):
         with np.errstate(all="ignore"):
-            A, b, _ = linearise(cell, h, p, h0, dense)
+            A, b, f = linearise(cell, h, p, h0, dense)
+            if i % jac_every == 0:
+                A_kept = A
+            else:
+                A, b = kept_operands(A_kept, f, shifted(h, h0), dense)
             h_new = affine_scan(A, b, h0)
             delta = float(np.max(np.abs(h_new - h)))
         h = h_new

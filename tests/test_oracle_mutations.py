@@ -9,6 +9,7 @@ import pytest
 
 from oracle import cells, elk, newton, scan
 import tests.test_oracle_pins as pins
+import tests.test_oracle_reuse as reuse_pins
 
 
 def _fails(fn, *args):
@@ -158,3 +159,31 @@ def test_lstm_transposed_block(monkeypatch):
         return c2, h2, np.swapaxes(A, -1, -2)
     monkeypatch.setattr(lstm.LSTM, "jacobian", bad)
     _fails(lstm_pins.test_one_newton_iteration_equals_brute_force_step)
+
+
+def test_reuse_with_offset_from_the_new_jacobian(monkeypatch):
+    """Jacobian reuse that keeps A but forms b_t with the new guess's Jacobian."""
+    def bad(A_kept, f, hp, dense):
+        return A_kept, f - (np.einsum("btij,btj->bti", A_kept, hp) * 0.0 if dense else 0.0 * hp)
+    monkeypatch.setattr(newton, "kept_operands", bad)
+    _fails(reuse_pins.test_reuse_iterates_equal_chord_method, "DEER", 2)
+    _fails(reuse_pins.test_reuse_iterates_equal_chord_method, "QUASI", 2)
+
+
+def test_reuse_ignored(monkeypatch):
+    """Jacobian reuse that silently recomputes the Jacobian every iteration."""
+    orig = newton.linearise
+    latest = {}
+
+    def lin(cell, h, p, h0, dense):
+        A, b, f = orig(cell, h, p, h0, dense)
+        latest["A"] = A
+        return A, b, f
+
+    def fresh(A_kept, f, hp, dense):
+        A = latest["A"]
+        return A, f - (np.einsum("btij,btj->bti", A, hp) if dense else A * hp)
+    monkeypatch.setattr(newton, "linearise", lin)
+    monkeypatch.setattr(newton, "kept_operands", fresh)
+    _fails(reuse_pins.test_reuse_iterates_equal_chord_method, "DEER", 3)
+    _fails(reuse_pins.test_reuse_iterates_equal_chord_method, "QUASI", 100)
