@@ -86,8 +86,19 @@ BENCHES = {
         kernel="adjoint_diag_kernel (one reverse pass)",
         desc="backward pass of the diagonal-recurrence GRU Din=D=2048, B={B}/GPU, T={T}: "
              "dL/dP, dL/dh0, dL/du, dL/db_hh from the converged states and dL/dh",
-        cpu_sample=dict(B=1, T=512), ref_sample=dict(B=1, T=128)),
+        cpu_sample=dict(B=1, T=1024), ref_sample=dict(B=1, T=128)),
 }
+# the dense cell's backward pass with the Jacobian's diagonal: the step is four
+# kernels; algorithmic bytes per state over all of them: h_{t-1} copy 8, GEMM
+# U h_{t-1} (reads h 4, writes 12), reverse scan (reads P 12, U h 12, h 4,
+# dL/dh 4; writes dL/dP 12, grow 12), dW_hh GEMM (reads grow 12, h 4) = 96 B
+BENCHES["adjoint_dense"] = dict(
+    workload="untrained", mode="ADJOINT", lam=0.0, bound="hbm", per_state=96,
+    kernel="the backward step: h_{t-1} copy, proj_gemm_kernel (U h), adjoint_diag_kernel<dense>, "
+           "outer_sum_partial_kernel + outer_sum_reduce_kernel",
+    desc="backward pass of the dense GRU Din=D=64, B={B}/GPU, T={T}, with the Jacobian's diagonal: "
+         "dL/dP, dL/dh0, dL/dW_hh [3D, D], dL/db_hh from the converged states and dL/dh",
+    cpu_sample=dict(B=16, T=32768), ref_sample=dict(B=4, T=4096))
 ADJ_METRIC = "backward states/sec (B*T*D per s, gradients through the evaluated sequence)"
 # the diagonal-recurrence LSTM (state (c, h) per lane; exact Newton over 2x2 lane
 # blocks): reads P 16 + the guess (c, h) 8, writes (c, h) 8 = 32 B per lane-step
@@ -201,7 +212,7 @@ class Clocks:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def cpu_baseline_oracle(spec: dict, sample: dict):
+def cpu_baseline_oracle(spec: dict, sample: dict, jac_every: int = 1):
     """Time the fp64 oracle (as it stands) on a bounded sample of the workload:
     the same generator and distributions, fewer sequences and steps."""
     import oracle
@@ -245,12 +256,14 @@ def cpu_baseline_oracle(spec: dict, sample: dict):
     if mode in ("ELK", "QUASI_ELK"):
         r = oracle.elk_solve(c, x, h0, mode, spec["lam"], w.tol)
     else:
-        r = oracle.newton_solve(c, x, h0, mode, w.tol)
+        r = oracle.newton_solve(c, x, h0, mode, w.tol, jac_every=jac_every)
     secs = time.perf_counter() - t0
     states = w.B * w.T * w.d
     return {"value": states / secs, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"fp64 numpy oracle, {mode} to tol {w.tol:g} on B={w.B}, T={w.T}, "
-                      f"D={w.d} ({r['iters']} iterations, {secs:.1f} s); same distributions"}
+                      f"D={w.d} ({r['iters']} iterations, {secs:.1f} s"
+                      + (f", Jacobian every {jac_every} iterations" if jac_every != 1 else "")
+                      + "); same distributions"}
 
 
 def run_reference(args):
@@ -261,7 +274,7 @@ def run_reference(args):
     steps = []
     base = None
     for i in range(args.warmup + args.steps):
-        cb = cpu_baseline_oracle(spec, spec["ref_sample"])
+        cb = cpu_baseline_oracle(spec, spec["ref_sample"], args.jac_every)
         if i >= args.warmup:
             steps.append(cb["value"])
         base = cb
@@ -283,7 +296,7 @@ def run_reference(args):
 
 
 def run_adjoint(args):
-    """The backward pass through the converged diagonal-cell solve, timed alone."""
+    """The backward pass through the converged solve (diagonal or dense cell), timed alone."""
     import torch
     import torch.distributed as dist
     from newton_solve_nonlinear_b200 import binding
@@ -313,7 +326,7 @@ def run_adjoint(args):
     P = binding.input_projection(g(w.x), g(w.w_ih), g(w.b_ih), d=D, kind=w.kind)
     h, h0, u, bh = sol.h, g(w.h0), g(w.w_hh), g(w.b_hh)
     dh = torch.randn(B, T, D, generator=torch.Generator().manual_seed(rank)).to(dev)
-    ws = binding.alloc_workspace(binding.adjoint_workspace_size(D, B, T), dev)
+    ws = binding.alloc_workspace(binding.adjoint_workspace_size(D, B, T, kind=w.kind), dev)
     out = dict(dP=torch.empty_like(P), dh0=torch.empty_like(h0), dw_hh=torch.empty_like(u),
                db_hh=torch.empty_like(bh))
     stream = torch.cuda.current_stream(dev)
@@ -372,7 +385,7 @@ def run_adjoint(args):
         "e2e": {"value": e2e_value, "unit": UNIT,
                 "h2d_bytes_per_step": (P.numel() + h.numel() + dh.numel()) * 4,
                 "d2h_bytes_per_step": P.numel() * 4},
-        "gpu_launches": args.steps,
+        "gpu_launches": (4 if w.kind == "dense" else 1) * args.steps,
         "clocks": clk.summary(),
     }
     if cpu is not None:
@@ -515,7 +528,21 @@ def run_ours(args):
     info = torch.zeros(4, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    k = args.jac_every
+    if k != 1:
+        if mode != "DEER":
+            raise SystemExit("--jac-every needs a DEER workload")
+        ws = binding.alloc_workspace(binding.lib().pararnn_reuse_workspace_size(
+            binding.make_cell(kind, din, D, w.x_dtype), B, T), dev)
+
     def step(ev_mid=None):
+        if k != 1:  # one synchronous call: projection and the solve with the Jacobian reused
+            if ev_mid is not None:
+                ev_mid.record(stream)
+            r = binding.newton_solve(w_ih, b_ih, w_hh, b_hh, x, h0, kind=kind, mode=mode, tol=w.tol,
+                                     jac_every=k, out=out, workspace=ws, stream=stream)
+            info[0], info[1] = r.iters, {v: c for c, v in binding.STATUS.items()}[r.status]
+            return
         binding.input_projection(x, w_ih, b_ih, d=D, kind=kind, out=P)
         if ev_mid is not None:
             ev_mid.record(stream)
@@ -552,11 +579,20 @@ def run_ours(args):
     h0_host = w.h0.float().contiguous().pin_memory()
     h_host = torch.empty(B, T, D, dtype=torch.float32).pin_memory()
     parts = max(1, min(E2E_PARTS, B))
+    if k != 1:
+        parts = 1
     ws_host = binding.alloc_workspace(
         binding.host_workspace_size(kind, din, D, B, T, mode, parts, w.x_dtype), dev)
     e2e_steps = max(1, min(args.steps, 5))
 
     def e2e_step():
+        if k != 1:  # copies around the reuse solve (no host-buffer variant of it)
+            x.copy_(x_host, non_blocking=True)
+            h0.copy_(h0_host, non_blocking=True)
+            binding.newton_solve(w_ih, b_ih, w_hh, b_hh, x, h0, kind=kind, mode=mode, tol=w.tol,
+                                 jac_every=k, out=out, workspace=ws, stream=stream)
+            h_host.copy_(out, non_blocking=True)
+            return
         return binding.newton_solve_host(w_ih, b_ih, w_hh, b_hh, x_host, h0_host, kind=kind,
                                          mode=mode, lam=lam, tol=w.tol, parts=parts, out=h_host,
                                          workspace=ws_host, stream=stream)
@@ -574,7 +610,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1:
-        cpu = cpu_baseline_oracle(spec, spec["cpu_sample"])
+        cpu = cpu_baseline_oracle(spec, spec["cpu_sample"], k)
 
     hbm_peak, peak_kind = peaks()
     solver_avg_s = statistics.mean(solver_ms) / 1e3
@@ -589,9 +625,12 @@ def run_ours(args):
             traffic = NCU_TRAFFIC["bytes_per_state_iter"] * iters * states
     elif spec["bound"] == "tensor":
         per_state = 2 * D * D
-        achieved = iters * states * per_state / solver_avg_s / 1e12
+        fresh = (iters + k - 1) // k  # iterations that form new Jacobian products
+        achieved = fresh * states * per_state / solver_avg_s / 1e12
         peak, unit = tf32_peak(), "TFLOP/s"
-        algo = f"2 D^3 flop/step = {per_state} flop/state/iteration x {iters} x {states} states"
+        algo = f"2 D^3 flop/step = {per_state} flop/state/iteration x {fresh} x {states} states"
+        if k != 1:
+            algo += f" (Jacobian every {k} iterations: {fresh} of {iters} form products; time includes the projection)"
         pk = "TF32 dense = MEASURED_PEAKS.json bf16_tflops x 1/2 (nominal TF32:bf16 ratio)"
     else:
         per_state = 14 * D * D
@@ -606,6 +645,7 @@ def run_ours(args):
         "config": {"workload": spec["desc"].format(B=B, T=T), "name": args.workload,
                    "B": B, "T": T, "D": D, "din": din, "cell": kind, "mode": mode,
                    "lambda": lam if mode in ("ELK", "QUASI_ELK") else None,
+                   "jac_every": k,
                    "tol": w.tol, "iters": iters, "status": binding.STATUS.get(status),
                    "l2": (f"inputs larger than L2 (126 MB) summed per solve: "
                           f"x {x.numel() * x.element_size() / 1e6:.0f} MB, "
@@ -640,6 +680,8 @@ def main():
     ap.add_argument("--workload", default="untrained", choices=sorted(BENCHES),
                     help="which solve to time (default: the untrained dense GRU headline)")
     ap.add_argument("--T", type=int, default=0, help="override the sequence length")
+    ap.add_argument("--jac-every", type=int, default=1,
+                    help="DEER workloads: recompute the Jacobian only every k iterations")
     args = ap.parse_args()
     if args.warmup < 3:
         log("warmup raised to 3 (timing rule)")

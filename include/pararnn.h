@@ -200,6 +200,34 @@ PARARNN_API int pararnn_newton_solve_guess_async(const pararnn_cell *cell, const
                                                  size_t ws_bytes, pararnn_stream stream);
 
 /*
+ * pararnn_newton_solve_reuse -- DEER on the dense cell with the Jacobian reused:
+ * recomputed only every jac_every iterations, an approximate Newton strategy
+ * the pages name for cost at scale ("ParaRNN" summary, "Newton's Iteration").
+ * Iteration i linearises with the J_t of iteration jac_every * floor(i /
+ * jac_every) and the residual of its own guess:
+ *   h^(i+1)_t = J^(i0)_t h^(i+1)_{t-1} + f(h^(i)_{t-1}, x_t) - J^(i0)_t h^(i)_{t-1},
+ * so the fixed point is the one of DEER, and after i iterations the first i
+ * states are exact (the T + 1 cap holds); in between refreshes convergence is
+ * linear instead of quadratic.  On this path an iteration that reuses the
+ * Jacobian also reuses the scan's matrix products (the chunk and group
+ * aggregates of J), so it costs O(D^2) per step instead of O(D^3).
+ *   jac_every  >= 1 (1: plain DEER).  Other arguments as pararnn_newton_solve
+ *              with mode DEER; the cell: PARARNN_GRU_DENSE, d <= 32.
+ *   workspace  pararnn_reuse_workspace_size bytes (the DEER workspace plus
+ *              512 bytes per step of B*T for the frozen coefficients).
+ * Synchronises `stream` once; returns the solve's status, or INVALID_ARG /
+ * CUDA_ERROR.
+ */
+PARARNN_API int pararnn_newton_solve_reuse(const pararnn_cell *cell, const pararnn_params *params,
+                                           const void *x, const float *h0, int B, int T, int jac_every,
+                                           float tol, int max_iters, float *h, pararnn_info *info,
+                                           void *workspace, size_t ws_bytes, pararnn_stream stream);
+
+/* pararnn_reuse_workspace_size -- bytes pararnn_newton_solve_reuse needs, or 0
+ * for arguments it rejects (not the dense cell with d <= 32). */
+PARARNN_API size_t pararnn_reuse_workspace_size(const pararnn_cell *cell, int B, int T);
+
+/*
  * pararnn_newton_solve_chunked -- the solve over consecutive time chunks of at
  * most t_chunk steps, one after another, each started from the last state the
  * previous chunk reached: device memory grows with t_chunk instead of T (for

@@ -27,7 +27,8 @@ EXPORTS = ("pararnn_workspace_size", "pararnn_newton_solve", "pararnn_newton_sol
            "pararnn_affine_scan_status", "pararnn_status_string", "pararnn_newton_solve_host",
            "pararnn_host_workspace_size", "pararnn_adjoint", "pararnn_adjoint_workspace_size",
            "pararnn_adjoint_status", "pararnn_newton_solve_guess_async", "pararnn_newton_solve_chunked",
-           "pararnn_chunked_workspace_size", "pararnn_lstm_solve", "pararnn_lstm_workspace_size")
+           "pararnn_chunked_workspace_size", "pararnn_lstm_solve", "pararnn_lstm_workspace_size",
+           "pararnn_newton_solve_reuse", "pararnn_reuse_workspace_size")
 
 
 class Cell(ctypes.Structure):
@@ -101,6 +102,11 @@ def lib() -> ctypes.CDLL:
         L.pararnn_lstm_solve.restype = ci
         L.pararnn_lstm_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci]
         L.pararnn_lstm_workspace_size.restype = sz
+        L.pararnn_newton_solve_reuse.argtypes = [ctypes.POINTER(Cell), ctypes.POINTER(Params), vp, vp, ci, ci, ci,
+                                                 cf, ci, vp, ctypes.POINTER(Info), vp, sz, vp]
+        L.pararnn_newton_solve_reuse.restype = ci
+        L.pararnn_reuse_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci]
+        L.pararnn_reuse_workspace_size.restype = sz
         L.pararnn_status_string.argtypes = [ci]
         L.pararnn_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -188,20 +194,41 @@ class SolveResult:
 
 def newton_solve(w_ih, b_ih, w_hh, b_hh, x, h0, *, kind: str, mode: str, tol: float,
                  lam: float = 0.0, max_iters: int = 0, out=None, workspace=None,
-                 stream=None, sync: bool = True, info_dev=None, h_init=None):
+                 stream=None, sync: bool = True, info_dev=None, h_init=None, jac_every: int = 1):
     """Evaluate the GRU over x [B, T, Din] with the chosen Newton mode.
 
     All tensors must be contiguous CUDA tensors (x and w_ih fp32 or bf16, the
     rest fp32).  With ``sync`` the call waits and returns a SolveResult; with
     ``sync=False`` it only enqueues, writing the report into ``info_dev`` (an
     int32 CUDA tensor of 4 elements) and returns ``out``.  ``h_init`` [B, T, D]
-    (fp32 CUDA) starts the iteration from that guess instead of zero."""
+    (fp32 CUDA) starts the iteration from that guess instead of zero.
+    ``jac_every`` > 1 (mode DEER, dense cell, d <= 32) recomputes the Jacobian
+    only every jac_every iterations (synchronous; no h_init)."""
     B, T, din = x.shape
     d = h0.shape[1]
     cell = make_cell(kind, din, d, x.dtype)
     if w_ih.dtype != x.dtype:
         raise TypeError("x and w_ih must have the same dtype")
     L = lib()
+    if jac_every != 1:
+        if mode != "DEER" or h_init is not None or not sync:
+            raise ValueError("jac_every > 1 takes mode DEER, sync=True and no h_init")
+        need = int(L.pararnn_reuse_workspace_size(ctypes.byref(cell), B, T))
+        if need == 0:
+            raise ValueError("arguments rejected by pararnn_reuse_workspace_size")
+        if workspace is None:
+            workspace = alloc_workspace(need, x.device)
+        if out is None:
+            out = torch.empty(B, T, d, dtype=torch.float32, device=x.device)
+        params = Params(_dev(w_ih, "w_ih"), _dev(b_ih, "b_ih"), _dev(w_hh, "w_hh"), _dev(b_hh, "b_hh"))
+        info = Info()
+        rc = L.pararnn_newton_solve_reuse(ctypes.byref(cell), ctypes.byref(params), _dev(x, "x"), _dev(h0, "h0"),
+                                          B, T, int(jac_every), float(tol), int(max_iters), _dev(out, "out"),
+                                          ctypes.byref(info), _dev(workspace, "workspace"), workspace.numel(),
+                                          _stream(stream))
+        if rc in (3, 4):
+            raise RuntimeError(f"pararnn_newton_solve_reuse: {L.pararnn_status_string(rc).decode()}")
+        return SolveResult(out, info.iters, STATUS[info.status], info.delta, info.residual)
     m = MODES[mode]
     need = int(L.pararnn_workspace_size(ctypes.byref(cell), B, T, m))
     if need == 0:

@@ -84,7 +84,7 @@ __device__ __forceinline__ void adj_cell_q(float pr, float pz, float pn, float q
 }
 
 template <bool DENSE>
-__global__ void __launch_bounds__(ANT, DENSE ? 1 : 2) adjoint_diag_kernel(AdjArgs S) {
+__global__ void __launch_bounds__(ANT, 2) adjoint_diag_kernel(AdjArgs S) {
     static_assert(ASEGS == 8, "the per-tile partial sums below add eight segments");
     __shared__ float seg_a[ASEGS][ADL], seg_b[ASEGS][ADL];
     __shared__ float carry[ADL];
@@ -267,62 +267,95 @@ namespace {
 // dW_hh [N, K] = sum over the M rows m of grow[m, :N] (outer) hp[m, :K]
 // (grow [M, 3D], hp [M, D]): each CTA sums a chunk of OSR rows into its own
 // partial (no atomics), a second pass adds the partials in chunk order, so the
-// result does not depend on scheduling.
+// result does not depend on scheduling.  Rows are staged 32 at a time into
+// shared memory, zero-padded to 192 x 64 columns (cp.async, double-buffered);
+// each thread keeps a 6 x 8 block of the outputs in registers (n = 6 nb + i,
+// k = 8 kb + j) and adds 48 products per row from five vector loads, as
+// packed fp32x2 FMAs.
 constexpr int OSR = 512;   // rows per chunk
 constexpr int OSM = 32;    // rows per shared-memory stage
-constexpr int OST = 256;   // threads: 32 row groups x 8 column groups
-constexpr int ONI = 6, OKJ = 8;  // outputs per thread: n = nb + 32 i (i < 6), k = kb + 8 j (j < 8)
+constexpr int OST = 256;   // threads: 32 row blocks x 8 column blocks
+constexpr int ONI = 6, OKJ = 8;
+constexpr int ONP = 32 * ONI, OKP = 8 * OKJ;  // padded widths: N <= 192, K <= 64
+constexpr int OSTAGE = OSM * (ONP + OKP);     // floats per stage
+constexpr size_t OS_SMEM = 2 * OSTAGE * sizeof(float);
+
+// 4-byte asynchronous copy to shared memory; zero-fills when !ok (the source
+// is then not read).
+__device__ __forceinline__ void cp4z(float *dst, const float *src, bool ok) {
+    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(d), "l"(src), "r"(ok ? 4 : 0) : "memory");
+}
+
+__device__ __forceinline__ void os_stage(float *st, const float *grow, const float *hp, long long mb, long long M,
+                                         int N, int K) {
+    for (int i = threadIdx.x; i < OSM * ONP; i += OST) {
+        const int r = i / ONP, n = i - r * ONP;
+        const bool ok = mb + r < M && n < N;
+        cp4z(st + i, ok ? grow + (mb + r) * N + n : grow, ok);
+    }
+    for (int i = threadIdx.x; i < OSM * OKP; i += OST) {
+        const int r = i / OKP, k = i - r * OKP;
+        const bool ok = mb + r < M && k < K;
+        cp4z(st + OSM * ONP + i, ok ? hp + (mb + r) * K + k : hp, ok);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
 __global__ void __launch_bounds__(OST) outer_sum_partial_kernel(const float *grow, const float *hp, long long M,
                                                                 int N, int K, float *part) {
-    extern __shared__ float osm[];  // [OSM][N] grow rows, then [OSM][K] hp rows
-    float *sg = osm, *sh = osm + OSM * N;
+    extern __shared__ float4 os_raw[];
+    float *buf = reinterpret_cast<float *>(os_raw);
     const long long m0 = static_cast<long long>(blockIdx.x) * OSR;
-    const int tid = threadIdx.x;
-    const int kb = tid % OKJ, nb = tid / OKJ;  // N <= 32 * 6, K <= 8 * 8
-    float acc[ONI][OKJ];
+    const long long m1 = m0 + OSR < M ? m0 + OSR : M;
+    const int nst = static_cast<int>((m1 - m0 + OSM - 1) / OSM);
+    const int kb = threadIdx.x % OKJ, nb = threadIdx.x / OKJ;
+    u64 acc[ONI][OKJ / 2];
 #pragma unroll
     for (int i = 0; i < ONI; ++i)
 #pragma unroll
-        for (int j = 0; j < OKJ; ++j) acc[i][j] = 0.f;
-    for (long long mb = m0; mb < m0 + OSR && mb < M; mb += OSM) {
-        const int rows = M - mb < OSM ? static_cast<int>(M - mb) : OSM;
-        __syncthreads();
-        for (int i = tid; i < OSM * N; i += OST) {
-            const int r = i / N;
-            sg[i] = r < rows ? __ldcs(grow + (mb + r) * N + i % N) : 0.f;
-        }
-        for (int i = tid; i < OSM * K; i += OST) {
-            const int r = i / K;
-            sh[i] = r < rows ? __ldcs(hp + (mb + r) * K + i % K) : 0.f;
+        for (int j = 0; j < OKJ / 2; ++j) acc[i][j] = 0ull;
+    os_stage(buf, grow, hp, m0, m1, N, K);
+    for (int st = 0; st < nst; ++st) {
+        if (st + 1 < nst) {
+            os_stage(buf + ((st + 1) & 1) * OSTAGE, grow, hp, m0 + (st + 1) * OSM, m1, N, K);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
         __syncthreads();
+        const float *sg = buf + (st & 1) * OSTAGE, *sh = sg + OSM * ONP;
 #pragma unroll 4
         for (int r = 0; r < OSM; ++r) {
-            float gv[ONI], hv[OKJ];
+            const float2 g0 = *reinterpret_cast<const float2 *>(sg + r * ONP + ONI * nb);
+            const float2 g1 = *reinterpret_cast<const float2 *>(sg + r * ONP + ONI * nb + 2);
+            const float2 g2 = *reinterpret_cast<const float2 *>(sg + r * ONP + ONI * nb + 4);
+            const float4 h0 = *reinterpret_cast<const float4 *>(sh + r * OKP + OKJ * kb);
+            const float4 h1 = *reinterpret_cast<const float4 *>(sh + r * OKP + OKJ * kb + 4);
+            const float gv[ONI] = {g0.x, g0.y, g1.x, g1.y, g2.x, g2.y};
+            const u64 hv[OKJ / 2] = {pk(h0.x, h0.y), pk(h0.z, h0.w), pk(h1.x, h1.y), pk(h1.z, h1.w)};
 #pragma unroll
             for (int i = 0; i < ONI; ++i) {
-                const int n = nb + 32 * i;
-                gv[i] = n < N ? sg[r * N + n] : 0.f;
+                const u64 g = splat(gv[i]);
+#pragma unroll
+                for (int j = 0; j < OKJ / 2; ++j) acc[i][j] = fma2(g, hv[j], acc[i][j]);
             }
-#pragma unroll
-            for (int j = 0; j < OKJ; ++j) {
-                const int k = kb + OKJ * j;
-                hv[j] = k < K ? sh[r * K + k] : 0.f;
-            }
-#pragma unroll
-            for (int i = 0; i < ONI; ++i)
-#pragma unroll
-                for (int j = 0; j < OKJ; ++j) acc[i][j] = fmaf(gv[i], hv[j], acc[i][j]);
         }
+        __syncthreads();  // the buffer is refilled next
     }
     float *dst = part + static_cast<size_t>(blockIdx.x) * N * K;
 #pragma unroll
-    for (int i = 0; i < ONI; ++i)
+    for (int i = 0; i < ONI; ++i) {
+        const int n = ONI * nb + i;
 #pragma unroll
-        for (int j = 0; j < OKJ; ++j) {
-            const int n = nb + 32 * i, k = kb + OKJ * j;
-            if (n < N && k < K) dst[n * K + k] = acc[i][j];
+        for (int j = 0; j < OKJ / 2; ++j) {
+            float a, b;
+            upk(acc[i][j], a, b);
+            const int k = OKJ * kb + 2 * j;
+            if (n < N && k < K) dst[n * K + k] = a;
+            if (n < N && k + 1 < K) dst[n * K + k + 1] = b;
         }
+    }
 }
 __global__ void outer_sum_reduce_kernel(const float *part, int nchunks, int NK, float *out) {
     const int o = blockIdx.x * blockDim.x + threadIdx.x;
@@ -340,13 +373,12 @@ size_t adjoint_outer_part_bytes(long long M, int N, int K) {
 
 cudaError_t launch_outer_sum(const float *grow, const float *hp, long long M, int N, int K, float *part, float *out,
                              cudaStream_t s) {
-    if (N > 32 * ONI || K > OKJ * OKJ) return cudaErrorInvalidValue;
+    if (N > ONP || K > OKP) return cudaErrorInvalidValue;
     const long long nchunks = (M + OSR - 1) / OSR;
-    const size_t smem = static_cast<size_t>(OSM) * (N + K) * 4;
     cudaError_t e = cudaFuncSetAttribute(outer_sum_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+                                         static_cast<int>(OS_SMEM));
     if (e != cudaSuccess) return e;
-    outer_sum_partial_kernel<<<static_cast<unsigned>(nchunks), OST, smem, s>>>(grow, hp, M, N, K, part);
+    outer_sum_partial_kernel<<<static_cast<unsigned>(nchunks), OST, OS_SMEM, s>>>(grow, hp, M, N, K, part);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int NK = N * K;
     outer_sum_reduce_kernel<<<(NK + 255) / 256, 256, 0, s>>>(part, static_cast<int>(nchunks), NK, out);

@@ -32,6 +32,18 @@
 // the fp32 re-sweep, so the fixed point (r = 0) is exact in fp32 and a
 // rounded product only perturbs the step, not where the iteration ends.
 //
+// Jacobian reuse (approximate Newton: the Jacobian recomputed only every few
+// iterations, "ParaRNN" summary, "Newton's Iteration").  With jac_every = k > 1
+// the J_t of iteration i are those of iteration k floor(i / k): a refreshing
+// iteration runs as above and also stores the per-row coefficients
+// (z, cz, cn, cr) of every step, 512 bytes per step; the k - 1 iterations after
+// it reload them instead of taking them from the new guess.  Their chunk and
+// group products Phi are then still the refreshed ones, so those iterations
+// skip every matrix-matrix product: P1 and P2a shrink to the matrix-vector
+// recurrences of the particular solutions, and each step of the iteration
+// costs O(D^2) instead of O(D^3).  The residual r_t always comes from the
+// current guess, so the fixed point is unchanged.
+//
 // Lane layout (lane = 4 gid + tq): rows R(nt) = 8 nt + gid, columns
 // C(kt, e) = 8 kt + 2 tq + e, nt, kt in 0..3, e in 0..1.  Each lane keeps
 // U_g[R(nt)][C(kt, e)] for the three gates (96 registers): they serve both
@@ -61,6 +73,13 @@ struct MmaArgs {
     int G, NG;   // chunks per group, groups per sequence
     float *PhiC, *pC, *PhiG, *pG, *carryC;
 };
+
+// The frozen coefficients: step t of sequence b is 128 floats, [gid][z, cz, cn,
+// cr][nt] (the coefficient block's layout without the residual), one float4
+// per lane.
+__device__ __forceinline__ float *coef_step(const DiagArgs &A, int b, int t) {
+    return A.coef + (static_cast<size_t>(b) * A.T + t) * 128;
+}
 
 // mma.sync with .tf32 operands reads the top 19 bits of each 32-bit register
 // (the low 13 mantissa bits are ignored: truncation), so fp32 values are passed
@@ -187,7 +206,7 @@ __device__ void stage_block(const DiagArgs &A, float *buf, int b, int tb, int n,
 // [s][i mod 8][coefficient][i / 8] so that a lane reads its rows R(nt) as
 // five float4.
 __device__ void block_coefs(const float (&u)[3][4][4][2], const float *Pb, const float *Hb,
-                            const float *bh, int D, const Lane &L, float *cf) {
+                            const float *bh, int D, const Lane &L, float *cf, bool coefs = true) {
 #pragma unroll
     for (int np = 0; np < 2; ++np) {  // row tiles in pairs: six independent accumulation chains
         float acc[2][3][4];
@@ -240,10 +259,12 @@ __device__ void block_coefs(const float (&u)[3][4][4][2], const float *Pb, const
                 const float cn = omz * (1.f - nn * nn) * r;
                 const bool live = i < D;
                 float *o = cf + s * kCS + (2 * L.tq + (q & 1)) * 20 + nt;  // row i = 8 nt + gid'
-                o[0] = live ? z : 0.f;
-                o[4] = live ? (hprev - nn) * z * omz : 0.f;
-                o[8] = live ? cn : 0.f;
-                o[12] = live ? cn * gn * (1.f - r) : 0.f;
+                if (coefs) {  // else they come from the frozen copy
+                    o[0] = live ? z : 0.f;
+                    o[4] = live ? (hprev - nn) * z * omz : 0.f;
+                    o[8] = live ? cn : 0.f;
+                    o[12] = live ? cn * gn * (1.f - r) : 0.f;
+                }
                 o[16] = live ? Hb[(s + 1) * 32 + i] - f : 0.f;
             }
     }
@@ -262,6 +283,18 @@ __device__ __forceinline__ void read_coefs(const float *cf, int s, const Lane &L
     C.cn[0] = cn.x; C.cn[1] = cn.y; C.cn[2] = cn.z; C.cn[3] = cn.w;
     C.cr[0] = cr.x; C.cr[1] = cr.y; C.cr[2] = cr.z; C.cr[3] = cr.w;
     C.res[0] = res.x; C.res[1] = res.y; C.res[2] = res.z; C.res[3] = res.w;
+}
+
+// Frozen coefficients of the block's steps tb .. tb+n-1: store from, or
+// fetch (cp.async, one commit group) into, the coefficient block.
+__device__ __forceinline__ void coefs_store(const DiagArgs &A, const float *cf, int b, int tb, int n, const Lane &L) {
+    for (int s = 0; s < n; ++s)
+        __stcg(reinterpret_cast<float4 *>(coef_step(A, b, tb + s)) + L.lane,
+               *reinterpret_cast<const float4 *>(cf + s * kCS + L.gid * 20 + L.tq * 4));
+}
+__device__ __forceinline__ void coefs_fetch(const DiagArgs &A, float *cf, int b, int tb, int n, const Lane &L) {
+    for (int s = 0; s < n; ++s) cp16(cf + s * kCS + L.gid * 20 + L.tq * 4, coef_step(A, b, tb + s) + 4 * L.lane);
+    cp_commit();
 }
 
 // J[R(nt)][C(kt, e)] for one kt (pairs e = 0, 1 as packed FMAs).  dz0, dz1:
@@ -363,7 +396,8 @@ struct WarpCtx {
     float *cf;   // this warp's coefficient block
 };
 
-// One step of the chunk chain: pout = pin J_t^T, p <- J_t p - r_t.
+// One step of the chunk chain: pout = pin J_t^T (kChain), p <- J_t p - r_t.
+template <bool kChain = true>
 __device__ __forceinline__ void chain_step(const float (&u)[3][4][4][2], const float *cf, int s,
                                            const Lane &L, float dz0, float dz1,
                                            const float (&pin)[2][4][4], float (&pout)[2][4][4],
@@ -377,16 +411,19 @@ __device__ __forceinline__ void chain_step(const float (&u)[3][4][4][2], const f
         jac_slice(u, C, kt, dz0, dz1, bj);
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) ffma2v(q0[nt], q1[nt], bj[nt][0], bj[nt][1], pcol[kt][0], pcol[kt][1]);
-        chain_slice(pin, pout, bj, kt);
+        if constexpr (kChain) chain_slice(pin, pout, bj, kt);
     }
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) prow[nt] = quad_sum(q0[nt] + q1[nt]) - C.res[nt];
     rows_to_cols(prow, pcol, L.tq);
 }
 
-// P1: aggregate (Phi_c, p_c) of chunk c of sequence b.
+// P1: aggregate (Phi_c, p_c) of chunk c of sequence b.  fresh: the Jacobian
+// is taken at this guess (stored when it is to be reused); else the frozen
+// one is reloaded and only p_c is formed (Phi_c is the refreshed one).
 __device__ void chunk_aggregate(const MmaArgs &S, const WarpCtx &W, int b, int c, const float *hold,
-                                bool zero_guess) {
+                                bool zero_guess, bool fresh) {
+    const bool reuse = S.a.jac_every > 1;
     const DiagArgs &A = S.a;
     const Lane L = lane_ids();
     const int t0 = c * S.L, n = min(S.L, A.T - t0), nb = (n + kBlk - 1) / kBlk;
@@ -408,8 +445,16 @@ __device__ void chunk_aggregate(const MmaArgs &S, const WarpCtx &W, int b, int c
         }
         __syncwarp();
         const float *Pb = W.buf + (blk & 1) * (kPB + kHB), *Hb = Pb + kPB;
-        block_coefs(u, Pb, Hb, W.bh, A.D, L, W.cf);
+        if (!fresh) coefs_fetch(A, W.cf, b, tb, nblk, L);
+        block_coefs(u, Pb, Hb, W.bh, A.D, L, W.cf, fresh);
+        if (!fresh) cp_wait<0>();
         __syncwarp();
+        if (!fresh) {
+            for (int s = 0; s < nblk; ++s) chain_step<false>(u, W.cf, s, L, dz0, dz1, psi, tmp, pcol, prow);
+            __syncwarp();
+            continue;
+        }
+        if (reuse) coefs_store(A, W.cf, b, tb, nblk, L);
         int s = 0;
         for (; s + 1 < nblk; s += 2) {
             chain_step(u, W.cf, s, L, dz0, dz1, psi, tmp, pcol, prow);
@@ -427,7 +472,7 @@ __device__ void chunk_aggregate(const MmaArgs &S, const WarpCtx &W, int b, int c
         __syncwarp();
     }
     const size_t idx = static_cast<size_t>(b) * S.NC + c;
-    store_phi(S.PhiC + idx * 1024, psi, L);
+    if (fresh) store_phi(S.PhiC + idx * 1024, psi, L);
     if (L.tq == 0)
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) __stcg(S.pC + idx * 32 + nt * 8 + L.gid, prow[nt]);
@@ -455,8 +500,9 @@ __device__ __forceinline__ void read_agg(const float *slot, const Lane &L, float
     }
 }
 
-// P2a: aggregate of group g of sequence b (chunks g G .. g G + G - 1).
-__device__ void group_aggregate(const MmaArgs &S, const WarpCtx &W, int b, int g) {
+// P2a: aggregate of group g of sequence b (chunks g G .. g G + G - 1); with a
+// frozen Jacobian (not fresh) only p_g: Phi_g is the refreshed one.
+__device__ void group_aggregate(const MmaArgs &S, const WarpCtx &W, int b, int g, bool fresh) {
     const Lane L = lane_ids();
     const int c0 = g * S.G, c1 = min(S.NC, c0 + S.G);
     float psi[2][4][4];
@@ -476,29 +522,31 @@ __device__ void group_aggregate(const MmaArgs &S, const WarpCtx &W, int b, int g
         __syncwarp();
         float ph[4][4][2], pc[4];
         read_agg(W.buf + slot * 1056, L, ph, pc);
-        float acc[2][4][4];
+        if (fresh) {
+            float acc[2][4][4];
 #pragma unroll
-        for (int kt = 0; kt < 4; ++kt) {
-            float bj[4][2];
+            for (int kt = 0; kt < 4; ++kt) {
+                float bj[4][2];
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                bj[nt][0] = ph[nt][kt][0];
-                bj[nt][1] = ph[nt][kt][1];
+                for (int nt = 0; nt < 4; ++nt) {
+                    bj[nt][0] = ph[nt][kt][0];
+                    bj[nt][1] = ph[nt][kt][1];
+                }
+                chain_slice(psi, acc, bj, kt);
             }
-            chain_slice(psi, acc, bj, kt);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) psi[mt][nt][q] = acc[mt][nt][q];
         }
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) psi[mt][nt][q] = acc[mt][nt][q];
         matvec(ph, pcol, pc, prow);
         rows_to_cols(prow, pcol, L.tq);
         __syncwarp();
     }
     const size_t idx = static_cast<size_t>(b) * S.NG + g;
-    store_phi(S.PhiG + idx * 1024, psi, L);
+    if (fresh) store_phi(S.PhiG + idx * 1024, psi, L);
     if (L.tq == 0)
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) __stcg(S.pG + idx * 32 + nt * 8 + L.gid, prow[nt]);
@@ -536,7 +584,7 @@ __device__ void carry_chain(const WarpCtx &W, const float *Phi, const float *p, 
 
 // P3: re-sweep chunk c of sequence b from its carry-in.
 __device__ void chunk_sweep(const MmaArgs &S, const WarpCtx &W, int b, int c, const float *hold,
-                            float *hnew, bool zero_guess, unsigned &dmax, unsigned &rmax) {
+                            float *hnew, bool zero_guess, bool fresh, unsigned &dmax, unsigned &rmax) {
     const DiagArgs &A = S.a;
     const Lane L = lane_ids();
     const int D = A.D, T = A.T;
@@ -561,7 +609,9 @@ __device__ void chunk_sweep(const MmaArgs &S, const WarpCtx &W, int b, int c, co
         }
         __syncwarp();
         const float *Pb = W.buf + (blk & 1) * (kPB + kHB), *Hb = Pb + kPB;
-        block_coefs(u, Pb, Hb, W.bh, D, L, W.cf);
+        if (!fresh) coefs_fetch(A, W.cf, b, tb, nblk, L);
+        block_coefs(u, Pb, Hb, W.bh, D, L, W.cf, fresh);
+        if (!fresh) cp_wait<0>();
         __syncwarp();
         for (int s = 0; s < nblk; ++s) {
             Coef C;
@@ -629,13 +679,14 @@ __global__ void __launch_bounds__(kThreads, 1) deer_mma_kernel(MmaArgs S) {
         const float *hold = A.hbuf[it & 1];
         float *hnew = A.hbuf[(it + 1) & 1];
         const bool zero_guess = it == 0 && !A.warm;  // the first guess: zero, or the caller's
+        const bool fresh = A.jac_every <= 1 || it % A.jac_every == 0;  // Jacobian taken at this guess
         unsigned dmax = 0u, rmax = 0u;
         for (long long w = gw; w < n_chunks; w += nw)
             chunk_aggregate(S, W, static_cast<int>(w / S.NC), static_cast<int>(w % S.NC), hold,
-                            zero_guess);
+                            zero_guess, fresh);
         grid_barrier(hdr->barrier, nblocks, status);
         for (long long w = gw; w < n_groups; w += nw)
-            group_aggregate(S, W, static_cast<int>(w / S.NG), static_cast<int>(w % S.NG));
+            group_aggregate(S, W, static_cast<int>(w / S.NG), static_cast<int>(w % S.NG), fresh);
         grid_barrier(hdr->barrier, nblocks, status);
         for (long long w = gw; w < n_groups; w += nw) {
             const int b = static_cast<int>(w / S.NG), g = static_cast<int>(w % S.NG);
@@ -648,7 +699,7 @@ __global__ void __launch_bounds__(kThreads, 1) deer_mma_kernel(MmaArgs S) {
         grid_barrier(hdr->barrier, nblocks, status);
         for (long long w = gw; w < n_chunks; w += nw)
             chunk_sweep(S, W, static_cast<int>(w / S.NC), static_cast<int>(w % S.NC), hold, hnew,
-                        zero_guess, dmax, rmax);
+                        zero_guess, fresh, dmax, rmax);
         const unsigned bd = block_max_u32(dmax, red);
         const unsigned br = block_max_u32(rmax, red);
         if (threadIdx.x == 0) {

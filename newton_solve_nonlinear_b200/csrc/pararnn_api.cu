@@ -43,6 +43,7 @@ cudaError_t launch_adjoint_diag(const float *P, const float *h0, const float *h,
                                 int D, void *hdr, void *desc, void *part, cudaStream_t s, const float *w_hh_dense,
                                 const float *G, float *grow);
 size_t adjoint_outer_part_bytes(long long M, int N, int K);
+bool deer_mma_supported(const pararnn_cell &cell);
 cudaError_t launch_outer_sum(const float *grow, const float *hp, long long M, int N, int K, float *part, float *out,
                              cudaStream_t s);
 
@@ -155,7 +156,7 @@ static cudaError_t enqueue_iterate(const pararnn_cell *cell, const pararnn_param
                                    const float *P, const float *h0, int B, int T, int mode,
                                    float lambda, float tol, int max_iters, float *h,
                                    pararnn_info *info_dev, void *workspace, cudaStream_t s,
-                                   const float *h_init = nullptr) {
+                                   const float *h_init = nullptr, int jac_every = 1) {
     const WsLayout L = ws_layout(*cell, B, T, mode);
     char *ws = static_cast<char *>(workspace);
     WsHeader *hdr = reinterpret_cast<WsHeader *>(ws + L.header);
@@ -183,6 +184,9 @@ static cudaError_t enqueue_iterate(const pararnn_cell *cell, const pararnn_param
     a.hdr = hdr;
     a.info_out = info_dev ? info_dev : &hdr->info;
     a.warm = h_init != nullptr;
+    a.jac_every = jac_every;
+    // the frozen Jacobian coefficients sit after the solve's own workspace
+    a.coef = jac_every > 1 ? reinterpret_cast<float *>(ws + L.total) : nullptr;
 
     cudaError_t e = cudaMemsetAsync(ws + L.header, 0, 256, s);
     if (e == cudaSuccess && diag && L.elk > L.desc) e = cudaMemsetAsync(ws + L.desc, 0, L.elk - L.desc, s);
@@ -239,7 +243,8 @@ int pararnn_newton_iterate_async(const pararnn_cell *cell, const pararnn_params 
 static int solve_enqueue(const pararnn_cell *cell, const pararnn_params *params, const void *x,
                          const float *h0, int B, int T, int mode, float lambda, float tol,
                          int max_iters, float *h, pararnn_info *info_dev, void *workspace,
-                         size_t ws_bytes, pararnn_stream stream, const float *h_init = nullptr) {
+                         size_t ws_bytes, pararnn_stream stream, const float *h_init = nullptr,
+                         int jac_every = 1) {
     int rc = check_solve(cell, params, x, nullptr, h0, B, T, mode, lambda, tol, h, workspace,
                          ws_bytes);
     if (rc != PARARNN_OK) return rc;
@@ -255,7 +260,7 @@ static int solve_enqueue(const pararnn_cell *cell, const pararnn_params *params,
                                       static_cast<long long>(B) * T, s);
     if (e == cudaSuccess)
         e = enqueue_iterate(cell, params, P, h0, B, T, mode, lambda, tol, max_iters, h, info_dev,
-                            workspace, s, h_init);
+                            workspace, s, h_init, jac_every);
     return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
 }
 
@@ -294,6 +299,38 @@ int pararnn_newton_solve_guess_async(const pararnn_cell *cell, const pararnn_par
     if (info_dev == nullptr || !aligned(info_dev, 4) || h_init == nullptr) return PARARNN_INVALID_ARG;
     return solve_enqueue(cell, params, x, h0, B, T, mode, lambda, tol, max_iters, h, info_dev, workspace,
                          ws_bytes, stream, h_init);
+}
+
+// ---- DEER with the Jacobian reused for several iterations ----
+
+// Frozen coefficients: 128 floats per step (z, cz, cn, cr for 32 rows).
+static size_t reuse_coef_bytes(int B, int T) { return align256(static_cast<size_t>(B) * T * 512); }
+
+size_t pararnn_reuse_workspace_size(const pararnn_cell *cell, int B, int T) {
+    if (!cell || cell->kind != PARARNN_GRU_DENSE || !cell_ok(cell, B, T, PARARNN_DEER) ||
+        !deer_mma_supported(*cell))
+        return 0;
+    return ws_layout(*cell, B, T, PARARNN_DEER).total + reuse_coef_bytes(B, T);
+}
+
+int pararnn_newton_solve_reuse(const pararnn_cell *cell, const pararnn_params *params, const void *x,
+                               const float *h0, int B, int T, int jac_every, float tol, int max_iters, float *h,
+                               pararnn_info *info, void *workspace, size_t ws_bytes, pararnn_stream stream) {
+    const size_t need = pararnn_reuse_workspace_size(cell, B, T);
+    if (need == 0 || jac_every < 1 || ws_bytes < need || !h || !workspace) return PARARNN_INVALID_ARG;
+    if (overlaps(h, static_cast<size_t>(B) * T * cell->d * 4, workspace, need)) return PARARNN_INVALID_ARG;
+    const int rc = solve_enqueue(cell, params, x, h0, B, T, PARARNN_DEER, 0.f, tol, max_iters, h, nullptr,
+                                 workspace, ws_bytes, stream, nullptr, jac_every);
+    if (rc != PARARNN_OK) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const WsLayout L = ws_layout(*cell, B, T, PARARNN_DEER);
+    pararnn_info host{};
+    const WsHeader *hdr = reinterpret_cast<const WsHeader *>(static_cast<char *>(workspace) + L.header);
+    cudaError_t e = cudaMemcpyAsync(&host, &hdr->info, sizeof(host), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
+    if (info) *info = host;
+    return host.status;
 }
 
 // ---- T-chunked solve: consecutive time chunks solved one after another ----

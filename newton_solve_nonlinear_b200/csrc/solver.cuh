@@ -58,6 +58,8 @@ struct DiagArgs {
     WsHeader *hdr;
     pararnn_info *info_out;  // device report destination
     int warm;                // hbuf[0] holds a caller's initial guess (else the guess is zero)
+    int jac_every;           // Jacobian refreshed every jac_every iterations (<= 1: every one)
+    float *coef;             // frozen Jacobian coefficients while jac_every > 1
 };
 
 // Workspace carve-up shared by the size query and the solver.

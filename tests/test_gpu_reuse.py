@@ -1,0 +1,87 @@
+"""GPU parity of DEER with the Jacobian reused for k iterations vs the oracle.
+
+The dense-cell DEER kernel (d <= 32) refreshes the Jacobian every k-th
+iteration and, in between, reuses it together with the chunk and group
+products built from it.  Tolerances as for plain DEER: single iterations
+within 5e-5 of the oracle's iterates (the carries pass through TF32 chunk
+products), converged states within 1e-4 of the fp64 rollout, iteration counts
+within +-1 of the oracle's with the same k.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle.cells import GRU, rollout
+from newton_solve_nonlinear_b200 import binding
+from newton_solve_nonlinear_b200.inputs import make_workload
+
+pytestmark = pytest.mark.gpu
+
+
+def _make(name, over):
+    kw = {k: over[k] for k in ("bias_std", "h0_std") if k in over}
+    return make_workload(name, **{k: v for k, v in over.items() if k not in kw}, **kw)
+
+
+def _oracle(w):
+    return GRU.from_workload(w), w.x.double().numpy(), w.h0.double().numpy()
+
+
+@pytest.mark.parametrize("k", [2, 3])
+@pytest.mark.parametrize("name,over", [
+    ("tiny", dict(T=1000, bias_std=0.3, h0_std=0.5)),
+    ("dense_deer", dict(B=2, T=700, bias_std=0.2)),
+    ("dense_deer", dict(B=3, T=257, d=12, din=5, h0_std=0.5)),
+])
+def test_each_reuse_iteration_matches_oracle(name, over, k):
+    w = _make(name, over)
+    c, x, h0 = _oracle(w)
+    ref = oracle.newton_solve(c, x, h0, "DEER", 0.0, max_iters=5, record=True, jac_every=k)
+    for n in range(1, 6):
+        r = binding.solve_workload(w, "DEER", tol=0.0, max_iters=n, jac_every=k)
+        assert r.iters == n
+        err = np.max(np.abs(r.h.double().cpu().numpy() - ref["iterates"][n - 1]))
+        assert err <= 5e-5, (n, err)
+
+
+@pytest.mark.parametrize("k", [2, 4])
+@pytest.mark.parametrize("name,over", [
+    ("tiny", {}),
+    ("dense_deer", dict(B=2, T=4096)),
+    ("dense_deer", dict(B=1, T=999, d=20, din=7, h0_std=1.0, bias_std=0.3)),
+])
+def test_reuse_converges_to_rollout(name, over, k):
+    w = _make(name, over)
+    c, x, h0 = _oracle(w)
+    r = binding.solve_workload(w, "DEER", jac_every=k)
+    assert r.status == "OK"
+    assert np.max(np.abs(r.h.double().cpu().numpy() - rollout(c, x, h0))) <= 1e-4
+    ref = oracle.newton_solve(c, x, h0, "DEER", w.tol, jac_every=k)
+    assert abs(r.iters - ref["iters"]) <= 1, (r.iters, ref["iters"])
+
+
+def test_reuse_full_size_sampled():
+    """The dense DEER workload's full size (B = 4, T = 65536, D = 32), k = 3."""
+    w = make_workload("dense_deer")
+    r = binding.solve_workload(w, "DEER", jac_every=3)
+    assert r.status == "OK"
+    c = GRU.from_workload(w)
+    h = r.h.cpu()
+    for b in (0, 3):
+        want = rollout(c, w.x[b:b + 1].double().numpy(), w.h0[b:b + 1].double().numpy())
+        assert np.max(np.abs(h[b:b + 1].double().numpy() - want)) <= 1e-4
+
+
+def test_period_one_is_plain_deer_and_arguments_checked():
+    w = make_workload("dense_deer", B=2, T=1500)
+    r0 = binding.solve_workload(w, "DEER")
+    r1 = binding.solve_workload(w, "DEER", jac_every=1)
+    r2 = binding.solve_workload(w, "DEER", jac_every=2)
+    r3 = binding.solve_workload(w, "DEER", jac_every=2)
+    assert torch.equal(r0.h, r1.h) and r0.iters == r1.iters
+    assert torch.equal(r2.h, r3.h) and r2.iters == r3.iters  # deterministic
+    with pytest.raises(ValueError):
+        binding.solve_workload(w, "QUASI", jac_every=2)
+    cell = binding.make_cell("dense", 64, 64, torch.float32)
+    assert binding.lib().pararnn_reuse_workspace_size(cell, 2, 100) == 0
