@@ -357,12 +357,26 @@ __global__ void __launch_bounds__(OST) outer_sum_partial_kernel(const float *gro
         }
     }
 }
-__global__ void outer_sum_reduce_kernel(const float *part, int nchunks, int NK, float *out) {
-    const int o = blockIdx.x * blockDim.x + threadIdx.x;
-    if (o >= NK) return;
+// out[o] = sum over chunks of part[c][o]: a CTA owns 32 consecutive outputs
+// (coalesced rows of the partials); its 8 warps take the chunks c = w, w + 8,
+// ... and the 8 warp sums are added in warp order, so the order is fixed.
+constexpr int ORW = 8;
+__global__ void __launch_bounds__(32 * ORW) outer_sum_reduce_kernel(const float *part, int nchunks, int NK,
+                                                                    float *out) {
+    __shared__ float red[ORW][32];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int o = blockIdx.x * 32 + lane;
     float a = 0.f;
-    for (int c = 0; c < nchunks; ++c) a += __ldcg(part + static_cast<size_t>(c) * NK + o);
-    out[o] = a;
+    if (o < NK)
+        for (int c = w; c < nchunks; c += ORW) a += __ldcs(part + static_cast<size_t>(c) * NK + o);
+    red[w][lane] = a;
+    __syncthreads();
+    if (w == 0 && o < NK) {
+        float t = red[0][lane];
+#pragma unroll
+        for (int q = 1; q < ORW; ++q) t += red[q][lane];
+        out[o] = t;
+    }
 }
 
 }  // namespace
@@ -381,7 +395,7 @@ cudaError_t launch_outer_sum(const float *grow, const float *hp, long long M, in
     outer_sum_partial_kernel<<<static_cast<unsigned>(nchunks), OST, OS_SMEM, s>>>(grow, hp, M, N, K, part);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int NK = N * K;
-    outer_sum_reduce_kernel<<<(NK + 255) / 256, 256, 0, s>>>(part, static_cast<int>(nchunks), NK, out);
+    outer_sum_reduce_kernel<<<(NK + 31) / 32, 32 * ORW, 0, s>>>(part, static_cast<int>(nchunks), NK, out);
     return cudaGetLastError();
 }
 
