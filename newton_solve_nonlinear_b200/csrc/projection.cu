@@ -170,6 +170,9 @@ __global__ void __launch_bounds__(256, VEC ? 3 : 2) proj_gemm_kernel(const Tin *
 }  // namespace
 
 bool proj_tcgen05_supported(int x_dtype, int N, int K);
+bool proj_tf32_supported(int x_dtype, long long M, int N, int K, const void *x, const void *P);
+cudaError_t launch_proj_tf32(const float *x, const float *w, const float *b, float *P, long long M, int N, int K,
+                             cudaStream_t s);
 cudaError_t launch_proj_tcgen05(const void *x, const void *w_ih, const float *b_ih, float *P, long long M, int N,
                                 int K, cudaStream_t s);
 
@@ -179,6 +182,8 @@ cudaError_t launch_proj_tcgen05(const void *x, const void *w_ih, const float *b_
 cudaError_t launch_projection_n(int x_dtype, const void *x, const void *w_ih, const float *b_ih, float *P,
                                 long long M, int N, int K, cudaStream_t s) {
     if (proj_tcgen05_supported(x_dtype, N, K)) return launch_proj_tcgen05(x, w_ih, b_ih, P, M, N, K, s);
+    if (proj_tf32_supported(x_dtype, M, N, K, x, P))
+        return launch_proj_tf32(static_cast<const float *>(x), static_cast<const float *>(w_ih), b_ih, P, M, N, K, s);
     const dim3 grid(static_cast<unsigned>((M + BM - 1) / BM), (N + BN - 1) / BN);
     const bool vec = K % 4 == 0 && reinterpret_cast<uintptr_t>(x) % 16 == 0 &&
                      reinterpret_cast<uintptr_t>(w_ih) % 16 == 0;
