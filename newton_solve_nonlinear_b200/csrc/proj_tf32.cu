@@ -17,7 +17,8 @@
 //     instruction) for lo*W_hi + hi*W_lo + hi*W_hi into one of two TMEM
 //     accumulators (W_hi, W_lo stay in shared memory for the whole launch);
 //   * while those products run, the warps read the other accumulator (the
-//     previous tile), add the bias and store the rows of P.
+//     previous tile) in the 16x256b layout, add the bias and store the rows of
+//     P in whole 32-byte sectors.
 // The dropped lo*lo term is below 2^-22 of each product, so P agrees with an
 // fp32 FMA evaluation to within fp32 rounding of the sum.  Every wait is
 // bounded; a wait that runs out makes the CTA drain what it started and write
@@ -238,29 +239,39 @@ proj_tf32_kernel(const __grid_constant__ CUtensorMap map_x, const float *__restr
             mma_pending |= 1u << nxt;
             if (k + 3 < my_n) load_pending |= 1u << nxt;
         }
-        // epilogue of tile k: thread = row, columns ch N/2 .. + N/2 - 1, 16 at a time
-        const long long m = row0_of(k) + qd * 32 + lane;
+        // epilogue of tile k: warp (qd, ch) takes rows 32 qd .. + 31 and columns
+        // ch N/2 .. + N/2 - 1 in the 16x256b layout (thread (gid, tq): rows gid and
+        // gid + 8 of a 16-row half, columns 2 tq, 2 tq + 1 of each 8), so the four
+        // threads of a row store 32 contiguous bytes: whole sectors
+        const int gid = lane >> 2, tq = lane & 3;
         const unsigned tbase = tmem + (cur ? G::ACC1 : 0u) + (static_cast<unsigned>(qd * 32) << 16);
 #pragma unroll
-        for (int c = 0; c < N / 2; c += 16) {
-            const int col = ch * (N / 2) + c;
-            unsigned v[16];
-            asm volatile(
-                "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-                "%15}, [%16];"
-                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-                  "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-                  "=r"(v[14]), "=r"(v[15])
-                : "r"(tbase + col));
-            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-            if (m < M) {
-                float4 *dst = reinterpret_cast<float4 *>(P + m * N + col);
+        for (int rh = 0; rh < 2; ++rh) {
+            const unsigned trow = tbase + (static_cast<unsigned>(rh * 16) << 16);
+            const long long ma = row0_of(k) + qd * 32 + rh * 16 + gid, mb = ma + 8;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float4 b4 = *reinterpret_cast<const float4 *>(c_b + col + 4 * q);
-                    __stcs(dst + q, make_float4(__uint_as_float(v[4 * q]) + b4.x, __uint_as_float(v[4 * q + 1]) + b4.y,
-                                                __uint_as_float(v[4 * q + 2]) + b4.z,
-                                                __uint_as_float(v[4 * q + 3]) + b4.w));
+            for (int c = 0; c < N / 2; c += 32) {
+                constexpr int NQ_FULL = 4;
+                const int nq = (N / 2 - c) / 8 < NQ_FULL ? (N / 2 - c) / 8 : NQ_FULL;
+                unsigned v[NQ_FULL][4];
+#pragma unroll
+                for (int q = 0; q < NQ_FULL; ++q)
+                    if (q < nq)
+                        asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];"
+                                     : "=r"(v[q][0]), "=r"(v[q][1]), "=r"(v[q][2]), "=r"(v[q][3])
+                                     : "r"(trow + ch * (N / 2) + c + 8 * q));
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                for (int q = 0; q < NQ_FULL; ++q) {
+                    if (q >= nq) continue;
+                    const int col = ch * (N / 2) + c + 8 * q + 2 * tq;
+                    const float2 b2 = *reinterpret_cast<const float2 *>(c_b + col);
+                    if (ma < M)
+                        __stcs(reinterpret_cast<float2 *>(P + ma * N + col),
+                               make_float2(__uint_as_float(v[q][0]) + b2.x, __uint_as_float(v[q][1]) + b2.y));
+                    if (mb < M)
+                        __stcs(reinterpret_cast<float2 *>(P + mb * N + col),
+                               make_float2(__uint_as_float(v[q][2]) + b2.x, __uint_as_float(v[q][3]) + b2.y));
                 }
             }
         }
