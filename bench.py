@@ -38,7 +38,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "converged states/sec (B*T*D per s, Newton to tol)"
 UNIT = "states/s"
-E2E_PARTS = 4  # parts of the batch whose copies the host-buffer solve overlaps
+E2E_PARTS = 7  # parts of the batch whose copies the host-buffer solve overlaps (ramped sizes)
 # The benchmarked solves, one per row family of the hot path.  "untrained"
 # (the default) is the headline; the others measure the other solver kernels
 # with the same JSON line.  Roofline units per state and Newton iteration:

@@ -258,12 +258,16 @@ PARARNN_API size_t pararnn_chunked_workspace_size(const pararnn_cell *cell, int 
  * with the copies overlapped with the computation.
  *
  * The B sequences are independent, so the batch is solved in `parts`
- * consecutive parts of ceil(B / parts) sequences (the last may be shorter;
- * when that size leaves nothing for the last parts there are fewer parts,
- * e.g. B = 4 asked in 3 parts runs as 2 + 2).
+ * consecutive parts.  Their sizes ramp, because the first part's copy in and
+ * the last part's copy out overlap no solve while a solve's cost per sequence
+ * falls as the part grows: part p has weight min(p + 1, parts - p, 4)
+ * (1, 2, 3, 4, ..., 4, 3, 2, 1), rounded by largest remainder, at least one
+ * sequence each (B = 16 in 7 parts: 1, 2, 3, 4, 3, 2, 1).
  * While part p is solved on `stream`, part p+1's inputs are copied in and
  * part p-1's states copied out on two streams the call creates and destroys;
- * the device staging is double-buffered in the workspace.  Each part is an
+ * the device staging holds three parts' inputs and outputs in the workspace
+ * (with two, a part's input copy would wait for the output copy two parts
+ * earlier, and copies slower than the solve would set the pace).  Each part is an
  * independent solve to `tol` (its own convergence test), so a part may take
  * fewer iterations than the whole batch would.
  *

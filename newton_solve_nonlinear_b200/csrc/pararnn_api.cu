@@ -9,6 +9,7 @@
 //   desc    look-back descriptors: tiles x lanes x (2 words, or 8 for quasi-ELK)
 //   elk     quasi-ELK forward results m, P, a, b: 4 x [B, T, D] fp32
 //   dense   block-scan scratch of the dense-Jacobian modes
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -639,22 +640,64 @@ const char *pararnn_status_string(int status) {
 
 namespace {
 
+// Staging buffers for the parts' inputs and outputs.  With two, part p+2's
+// input copy would wait for part p's output copy, so whenever both copies of a
+// part take longer than one part's solve (PCIe: ~10 ms of copies against ~7 ms
+// of solve on the dense workload) the copies would set the pace; three keep
+// the solve busy.
+constexpr int kHostBufs = 3;
+
+// Sequences per part.  The first part's copy in and the last part's copy out
+// overlap no solve, while a solve's cost per sequence falls as its part grows
+// (fewer, shorter look-back chains per iteration), so the parts ramp up and
+// down: weight min(p + 1, parts - p, 4) for part p (1, 2, 3, 4, ..., 4, 3, 2,
+// 1), rounded by largest remainder with at least one sequence per part
+// (parts <= B).  Each next part's copy in then fits under the solve before it.
+std::vector<int> part_sizes(int B, int parts) {
+    std::vector<int> w(parts);
+    for (int p = 0; p < parts; ++p) w[p] = std::min(std::min(p + 1, parts - p), 4);
+    long long W = 0;
+    for (int v : w) W += v;
+    std::vector<int> n(parts);
+    std::vector<std::pair<long long, int>> rem(parts);
+    int used = 0;
+    for (int i = 0; i < parts; ++i) {
+        const long long num = static_cast<long long>(B) * w[i];
+        n[i] = static_cast<int>(num / W);
+        rem[i] = {num % W, -i};
+        used += n[i];
+    }
+    std::sort(rem.begin(), rem.end(), [](const auto &a, const auto &b) { return a > b; });
+    for (int r = 0; used < B; ++r, ++used) ++n[-rem[r % parts].second];
+    for (int i = 0; i < parts; ++i)  // at least one each: from the largest part
+        while (n[i] == 0) {
+            int j = 0;
+            for (int q = 1; q < parts; ++q)
+                if (n[q] > n[j]) j = q;
+            --n[j];
+            ++n[i];
+        }
+    return n;
+}
+
 struct HostLayout {
-    int parts, bp;  // number of parts, sequences per part (the last may be shorter)
-    size_t solve, xs[2], hs[2], h0, infos, total;
+    int parts, bp, nbuf;  // number of parts, sequences of the largest part, buffers
+    size_t solve, xs[kHostBufs], hs[kHostBufs], h0, infos, total;
 };
 
 HostLayout host_layout(const pararnn_cell &cell, int B, int T, int mode, int parts) {
     HostLayout H{};
-    H.bp = (B + parts - 1) / parts;
-    H.parts = (B + H.bp - 1) / H.bp;  // e.g. B=4 in 3 parts is 2+2: no empty part
+    H.parts = parts;
+    H.bp = 0;
+    for (int v : part_sizes(B, parts)) H.bp = v > H.bp ? v : H.bp;
+    H.nbuf = H.parts < kHostBufs ? H.parts : kHostBufs;
     const size_t es = cell.x_dtype == PARARNN_BF16 ? 2 : 4;
     const size_t xbytes = static_cast<size_t>(H.bp) * T * cell.din * es;
     const size_t hbytes = static_cast<size_t>(H.bp) * T * cell.d * 4;
     size_t off = 0;
     H.solve = off; off = align256(off + ws_layout(cell, H.bp, T, mode).total);
-    for (int q = 0; q < 2; ++q) { H.xs[q] = off; off = align256(off + xbytes); }
-    for (int q = 0; q < 2; ++q) { H.hs[q] = off; off = align256(off + hbytes); }
+    for (int q = 0; q < H.nbuf; ++q) { H.xs[q] = off; off = align256(off + xbytes); }
+    for (int q = 0; q < H.nbuf; ++q) { H.hs[q] = off; off = align256(off + hbytes); }
     H.h0 = off; off = align256(off + static_cast<size_t>(B) * cell.d * 4);
     H.infos = off; off = align256(off + static_cast<size_t>(parts) * sizeof(pararnn_info));
     H.total = off;
@@ -683,46 +726,51 @@ int pararnn_newton_solve_host(const pararnn_cell *cell, const pararnn_params *pa
     const size_t hrow = static_cast<size_t>(T) * cell->d * 4;      // bytes of one sequence's states
     cudaStream_t sc = reinterpret_cast<cudaStream_t>(stream);
     cudaStream_t s_in = nullptr, s_out = nullptr;
-    cudaEvent_t ev[7] = {};  // in[2], comp[2], out[2], h0
+    constexpr int NB = kHostBufs;
+    cudaEvent_t ev[3 * NB + 1] = {};  // in[NB], comp[NB], out[NB], start / end
+    cudaEvent_t *ev_in = ev, *ev_comp = ev + NB, *ev_out = ev + 2 * NB, &ev_edge = ev[3 * NB];
     cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
-    for (int q = 0; q < 7 && e == cudaSuccess; ++q) e = cudaEventCreateWithFlags(&ev[q], cudaEventDisableTiming);
+    for (int q = 0; q < 3 * NB + 1 && e == cudaSuccess; ++q)
+        e = cudaEventCreateWithFlags(&ev[q], cudaEventDisableTiming);
     int rc = PARARNN_OK;
     float *h0_dev = reinterpret_cast<float *>(ws + H.h0);
     pararnn_info *infos = reinterpret_cast<pararnn_info *>(ws + H.infos);
     if (e == cudaSuccess) {
         // start only after the caller's earlier work on its stream
-        e = cudaEventRecord(ev[6], sc);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev[6], 0);
+        e = cudaEventRecord(ev_edge, sc);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev_edge, 0);
         if (e == cudaSuccess)
             e = cudaMemcpyAsync(h0_dev, h0_host, static_cast<size_t>(B) * cell->d * 4, cudaMemcpyHostToDevice, s_in);
     }
-    for (int p = 0; p < H.parts && e == cudaSuccess && rc == PARARNN_OK; ++p) {
-        const int buf = p & 1;
-        const int b0 = p * H.bp, nb = (B - b0) < H.bp ? (B - b0) : H.bp;
-        if (p >= 2) e = cudaStreamWaitEvent(s_in, ev[4 + buf], 0);  // staging of part p-2 free
+    const std::vector<int> sizes = part_sizes(B, H.parts);
+    int b0 = 0;
+    for (int p = 0; p < H.parts && e == cudaSuccess && rc == PARARNN_OK; b0 += sizes[p], ++p) {
+        const int buf = p % H.nbuf;
+        const int nb = sizes[p];
+        if (p >= H.nbuf) e = cudaStreamWaitEvent(s_in, ev_out[buf], 0);  // staging of part p-nbuf free
         if (e == cudaSuccess)
             e = cudaMemcpyAsync(ws + H.xs[buf], static_cast<const char *>(x_host) + b0 * xrow, nb * xrow,
                                 cudaMemcpyHostToDevice, s_in);
-        if (e == cudaSuccess) e = cudaEventRecord(ev[buf], s_in);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(sc, ev[buf], 0);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_in[buf], s_in);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(sc, ev_in[buf], 0);
         if (e != cudaSuccess) break;
         rc = solve_enqueue(cell, params, ws + H.xs[buf], h0_dev + static_cast<size_t>(b0) * cell->d, nb, T, mode,
                            lambda, tol, max_iters, reinterpret_cast<float *>(ws + H.hs[buf]), infos + p,
                            ws + H.solve, ws_layout(*cell, nb, T, mode).total, stream);
         if (rc != PARARNN_OK) break;
-        e = cudaEventRecord(ev[2 + buf], sc);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev[2 + buf], 0);
+        e = cudaEventRecord(ev_comp[buf], sc);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_comp[buf], 0);
         if (e == cudaSuccess)
             e = cudaMemcpyAsync(reinterpret_cast<char *>(h_host) + b0 * hrow, ws + H.hs[buf], nb * hrow,
                                 cudaMemcpyDeviceToHost, s_out);
-        if (e == cudaSuccess) e = cudaEventRecord(ev[4 + buf], s_out);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_out[buf], s_out);
     }
     // the caller's stream continues after the last copy out
     pararnn_info agg{};
     if (e == cudaSuccess && rc == PARARNN_OK) {
-        e = cudaEventRecord(ev[6], s_out);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(sc, ev[6], 0);
+        e = cudaEventRecord(ev_edge, s_out);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(sc, ev_edge, 0);
         std::vector<pararnn_info> host(H.parts);
         if (e == cudaSuccess)
             e = cudaMemcpyAsync(host.data(), infos, H.parts * sizeof(pararnn_info), cudaMemcpyDeviceToHost, sc);
@@ -741,7 +789,7 @@ int pararnn_newton_solve_host(const pararnn_cell *cell, const pararnn_params *pa
     // leave nothing in flight before the helper streams go away
     if (s_in) cudaStreamSynchronize(s_in);
     if (s_out) cudaStreamSynchronize(s_out);
-    for (int q = 0; q < 7; ++q)
+    for (int q = 0; q < 3 * NB + 1; ++q)
         if (ev[q]) cudaEventDestroy(ev[q]);
     if (s_in) cudaStreamDestroy(s_in);
     if (s_out) cudaStreamDestroy(s_out);
