@@ -83,6 +83,8 @@ __device__ __forceinline__ void adj_cell_q(float pr, float pz, float pn, float q
     a = z + fz * udz + fn * r * udn + fr * udr;
 }
 
+__device__ __forceinline__ void prefetch_l2(const float *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
 template <bool DENSE>
 __global__ void __launch_bounds__(ANT, 2) adjoint_diag_kernel(AdjArgs S) {
     static_assert(ASEGS == 8, "the per-tile partial sums below add eight segments");
@@ -143,6 +145,35 @@ __global__ void __launch_bounds__(ANT, 2) adjoint_diag_kernel(AdjArgs S) {
                     qz[i] = ok ? __ldcs(S.G + o + D) : 0.f;
                     qn[i] = ok ? __ldcs(S.G + o + 2 * D) : 0.f;
                 }
+            }
+            // dense cell: the CTA's next tile (its rows are whole, contiguous state
+            // rows) into L2 while this one is computed; on the diagonal cell's
+            // 64-lane slices of wide rows this measured slower, so it is not done there
+            const long long vn = v + nblocks;
+            if (DENSE && vn < S.n_tiles) {
+                const unsigned vn32 = static_cast<unsigned>(vn);
+                const int cn = static_cast<int>(vn32 / ng);
+                const int gn = static_cast<int>(vn32 - static_cast<unsigned>(cn) * ng);
+                const int tn0 = (S.n_chunks - 1 - cn) * ATS;
+                const int bn = gn / S.ndg, lanen = (gn - bn * S.ndg) * ADL + d;
+                const size_t rown = static_cast<size_t>(bn) * T;
+                if (lanen < D)
+#pragma unroll
+                    for (int i = 0; i < ASL; ++i) {
+                        const int t = tn0 + seg * ASL + i;
+                        if (t >= T) break;
+                        const size_t o = (rown + t) * 3 * D + lanen;
+                        prefetch_l2(S.P + o);
+                        prefetch_l2(S.P + o + D);
+                        prefetch_l2(S.P + o + 2 * D);
+                        if constexpr (DENSE) {
+                            prefetch_l2(S.G + o);
+                            prefetch_l2(S.G + o + D);
+                            prefetch_l2(S.G + o + 2 * D);
+                        }
+                        prefetch_l2(S.dh + (rown + t) * D + lanen);
+                        if (t > 0) prefetch_l2(S.h + (rown + t - 1) * D + lanen);
+                    }
             }
 #pragma unroll
             for (int i = 0; i <= ASL; ++i) {
