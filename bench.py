@@ -55,30 +55,30 @@ BENCHES = {
         workload="untrained", mode="QUASI", lam=0.0, bound="hbm", per_state=20,
         kernel="quasi_tc2_kernel<64, quasi> (persistent, all iterations)",
         desc="untrained dense GRU Din=D=64, B={B}/GPU, T={T}, fp32, quasi-DEER tol 1e-5",
-        cpu_sample=dict(B=16, T=12288), ref_sample=dict(B=4, T=256)),
+        cpu_sample=dict(B=16, T=12288), ref_sample=dict(B=4, T=256), roll_sample=dict()),
     "diag": dict(
         workload="diag", mode="QUASI", lam=0.0, bound="hbm", per_state=20,
         kernel="diag2_kernel (persistent, all iterations)",
         desc="diagonal-recurrence GRU Din=D=2048, B={B}/GPU, T={T}, bf16 x and W_ih, fp32 state, "
              "quasi-DEER (exact Newton) tol 1e-4",
-        cpu_sample=dict(B=1, T=16384), ref_sample=dict(B=1, T=128)),
+        cpu_sample=dict(B=1, T=16384), ref_sample=dict(B=1, T=128), roll_sample=dict(T=256)),
     "dense_deer": dict(
         workload="dense_deer", mode="DEER", lam=0.0, bound="tensor", per_state=None,
         kernel="deer_mma_kernel (persistent, all iterations)",
         desc="dense GRU Din=16, D=32, B={B}/GPU, T={T}, fp32 cell, TF32 Jacobian products, DEER tol 1e-5",
-        cpu_sample=dict(B=4, T=32768), ref_sample=dict(B=1, T=512)),
+        cpu_sample=dict(B=4, T=32768), ref_sample=dict(B=1, T=512), roll_sample=dict()),
     "quasi_elk": dict(
         workload="near_unstable", mode="QUASI_ELK", lam=0.1, bound="hbm", per_state=56,
         kernel="quasi_tc2_kernel<64, quasi-ELK> (persistent, all iterations)",
         desc="near-unstable dense GRU Din=D=64 (spectral radius 1.5), B={B}/GPU, T={T}, fp32, "
              "quasi-ELK lambda 0.1, tol 1e-4",
-        cpu_sample=dict(B=8, T=8000), ref_sample=dict(B=1, T=250)),
+        cpu_sample=dict(B=8, T=8000), ref_sample=dict(B=1, T=250), roll_sample=dict()),
     "elk": dict(
         workload="near_unstable", mode="ELK", lam=0.01, bound="alu", per_state=None,
         kernel="dense_elk_kernel<64> (persistent, all iterations)",
         desc="near-unstable dense GRU Din=D=64 (spectral radius 1.5), B={B}/GPU, T={T}, fp32, "
              "ELK lambda 0.01, tol 1e-4",
-        cpu_sample=dict(B=1, T=5000), ref_sample=dict(B=1, T=150)),
+        cpu_sample=dict(B=1, T=5000), ref_sample=dict(B=1, T=150), roll_sample=dict()),
     # the backward pass through the evaluated diagonal-cell sequence (not a solve):
     # reads P 12 + h 4 + dL/dh 4, writes dL/dP 12 = 32 B per state
     "adjoint": dict(
@@ -264,6 +264,46 @@ def cpu_baseline_oracle(spec: dict, sample: dict, jac_every: int = 1):
                       f"D={w.d} ({r['iters']} iterations, {secs:.1f} s"
                       + (f", Jacobian every {jac_every} iterations" if jac_every != 1 else "")
                       + "); same distributions"}
+
+
+def cpu_rollout_baseline(spec: dict) -> dict | None:
+    """The plain sequential evaluation on the host (oracle/rollout.c: fp64 and
+    fp32, one thread and OpenMP over the batch's sequences), on the sample
+    `roll_sample` of the workload (the whole workload where it fits in seconds).
+    Reported beside the GPU solve: what a CPU does without the parallel method."""
+    import numpy as np
+    from oracle import crollout
+    from oracle.cells import GRU
+    from newton_solve_nonlinear_b200.inputs import make_workload
+    sample = spec.get("roll_sample")
+    if sample is None:
+        return None
+    w = make_workload(spec["workload"], **sample)
+    c = GRU.from_workload(w)
+    x, h0 = w.x.double().numpy(), w.h0.double().numpy()
+    states = w.B * w.T * w.d
+    nthr = min(crollout.max_threads(), w.B)
+    out = {"unit": UNIT, "cores": os.cpu_count(), "threads": nthr, "cpu": cpu_model(),
+           "sample": f"B={w.B}, T={w.T}, D={w.d}, Din={w.din} on {nthr} threads, the first sequence alone "
+                     f"on one thread (sequential rollout, gcc -O3 -fopenmp)"}
+    for name, dt in (("fp64", np.float64), ("fp32", np.float32)):
+        t0 = time.perf_counter()
+        crollout.rollout(c, x, h0, dt, threads=nthr)
+        out[name] = states / (time.perf_counter() - t0)
+        t0 = time.perf_counter()
+        crollout.rollout(c, x[:1], h0[:1], dt, threads=1)
+        out[name + "_1thread"] = states / w.B / (time.perf_counter() - t0)
+    return out
+
+
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def run_reference(args):
@@ -608,9 +648,10 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_value = job_value(states, e2e_steps, world, max_over_ranks(ea.elapsed_time(eb), dev))
 
-    cpu = None
+    cpu = roll = None
     if rank == 0 and world == 1:
         cpu = cpu_baseline_oracle(spec, spec["cpu_sample"], k)
+        roll = cpu_rollout_baseline(spec)
 
     hbm_peak, peak_kind = peaks()
     solver_avg_s = statistics.mean(solver_ms) / 1e3
@@ -664,6 +705,8 @@ def run_ours(args):
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
+    if roll is not None:
+        line["cpu_rollout"] = roll
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
