@@ -475,6 +475,30 @@ PARARNN_API int pararnn_lstm_solve(const pararnn_cell *cell, const pararnn_param
  * iterate copy, look-back words), or 0 for rejected arguments. */
 PARARNN_API size_t pararnn_lstm_workspace_size(const pararnn_cell *cell, int B, int T);
 
+/*
+ * pararnn_lstm_solve_host -- pararnn_lstm_solve from and to HOST memory, with
+ * the copies overlapped with the computation as in pararnn_newton_solve_host:
+ * the batch in `parts` ramped parts (same sizes), three staging buffers, part
+ * p's x copied in and its (c, h) copied out on two streams the call creates,
+ * while part p's neighbours are solved on `stream`.  Each part is an
+ * independent solve to `tol`; the report is the worst part's.
+ *   x_host     HOST [B, T, Din] of cell->x_dtype;  c0_host, h0_host HOST [B, D].
+ *   c_host, h_host  HOST [B, T, D] float outputs.  Page-locked memory lets the
+ *              copies run asynchronously.
+ *   parts      1 <= parts <= B.
+ *   workspace  DEVICE, >= pararnn_lstm_host_workspace_size bytes, 256-byte aligned.
+ * Synchronises `stream` once, at the end; returns the worst part's status, or
+ * INVALID_ARG / CUDA_ERROR.
+ */
+PARARNN_API int pararnn_lstm_solve_host(const pararnn_cell *cell, const pararnn_params *params, const void *x_host,
+                                        const float *c0_host, const float *h0_host, int B, int T, float tol,
+                                        int max_iters, float *c_host, float *h_host, pararnn_info *info, int parts,
+                                        void *workspace, size_t ws_bytes, pararnn_stream stream);
+
+/* pararnn_lstm_host_workspace_size -- bytes pararnn_lstm_solve_host needs (one
+ * part's solve workspace, three parts' staging, the initial states), or 0. */
+PARARNN_API size_t pararnn_lstm_host_workspace_size(const pararnn_cell *cell, int B, int T, int parts);
+
 /* pararnn_status_string -- a static, human-readable name of a status code. */
 PARARNN_API const char *pararnn_status_string(int status);
 

@@ -28,7 +28,8 @@ EXPORTS = ("pararnn_workspace_size", "pararnn_newton_solve", "pararnn_newton_sol
            "pararnn_host_workspace_size", "pararnn_adjoint", "pararnn_adjoint_workspace_size",
            "pararnn_adjoint_status", "pararnn_newton_solve_guess_async", "pararnn_newton_solve_chunked",
            "pararnn_chunked_workspace_size", "pararnn_lstm_solve", "pararnn_lstm_workspace_size",
-           "pararnn_newton_solve_reuse", "pararnn_reuse_workspace_size")
+           "pararnn_newton_solve_reuse", "pararnn_reuse_workspace_size", "pararnn_lstm_solve_host",
+           "pararnn_lstm_host_workspace_size")
 
 
 class Cell(ctypes.Structure):
@@ -107,6 +108,11 @@ def lib() -> ctypes.CDLL:
         L.pararnn_newton_solve_reuse.restype = ci
         L.pararnn_reuse_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci]
         L.pararnn_reuse_workspace_size.restype = sz
+        L.pararnn_lstm_solve_host.argtypes = [ctypes.POINTER(Cell), ctypes.POINTER(Params), vp, vp, vp, ci, ci, cf, ci,
+                                              vp, vp, ctypes.POINTER(Info), ci, vp, sz, vp]
+        L.pararnn_lstm_solve_host.restype = ci
+        L.pararnn_lstm_host_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci, ci]
+        L.pararnn_lstm_host_workspace_size.restype = sz
         L.pararnn_status_string.argtypes = [ci]
         L.pararnn_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -351,6 +357,35 @@ def newton_solve_host(w_ih, b_ih, w_hh, b_hh, x_host, h0_host, *, kind: str, mod
     if rc in (3, 4):
         raise RuntimeError(f"pararnn_newton_solve_host: {L.pararnn_status_string(rc).decode()}")
     return SolveResult(out, info.iters, STATUS[info.status], info.delta, info.residual)
+
+
+def lstm_solve_host(w_ih, b_ih, u, b_hh, x_host, c0_host, h0_host, *, tol: float, max_iters: int = 0,
+                    parts: int = 4, out=None, workspace=None, device=None, stream=None):
+    """The LSTM solve from and to HOST tensors (x_host [B,T,Din], c0_host and
+    h0_host [B,D]; ``out`` a pair of host [B,T,D] fp32 tensors, page-locked for
+    overlap), in ``parts`` parts with the copies overlapped with compute;
+    weights are CUDA tensors.  Returns (c, h, SolveResult) with host c, h."""
+    B, T, din = x_host.shape
+    d = h0_host.shape[1]
+    parts = max(1, min(int(parts), B))
+    cell = make_cell("lstm_diag", din, d, x_host.dtype)
+    L = lib()
+    need = int(L.pararnn_lstm_host_workspace_size(ctypes.byref(cell), B, T, parts))
+    if need == 0:
+        raise ValueError("arguments rejected by pararnn_lstm_host_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, u.device if device is None else device)
+    c, h = out if out is not None else (torch.empty(B, T, d, dtype=torch.float32).pin_memory(),
+                                        torch.empty(B, T, d, dtype=torch.float32).pin_memory())
+    params = Params(_dev(w_ih, "w_ih"), _dev(b_ih, "b_ih"), _dev(u, "u"), _dev(b_hh, "b_hh"))
+    info = Info()
+    rc = L.pararnn_lstm_solve_host(ctypes.byref(cell), ctypes.byref(params), _host(x_host, "x_host"),
+                                   _host(c0_host, "c0_host"), _host(h0_host, "h0_host"), B, T, float(tol),
+                                   int(max_iters), _host(c, "c"), _host(h, "h"), ctypes.byref(info), parts,
+                                   _dev(workspace, "workspace"), workspace.numel(), _stream(stream))
+    if rc in (3, 4):
+        raise RuntimeError(f"pararnn_lstm_solve_host: {L.pararnn_status_string(rc).decode()}")
+    return c, h, SolveResult(h, info.iters, STATUS[info.status], info.delta, info.residual)
 
 
 def adjoint_workspace_size(d: int, B: int, T: int, kind: str = "diag") -> int:

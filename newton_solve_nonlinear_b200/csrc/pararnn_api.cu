@@ -482,6 +482,27 @@ LstmLayout lstm_layout(const pararnn_cell &cell, int B, int T) {
     L.total = off;
     return L;
 }
+
+// Enqueue the projection (4D gate rows) and the solve on `s`; the report goes
+// to info_dev (nullptr: the workspace header).  Arguments already checked.
+cudaError_t lstm_enqueue(const pararnn_cell *cell, const pararnn_params *params, const void *x, const float *c0,
+                         const float *h0, int B, int T, float tol, int max_iters, float *c, float *h,
+                         pararnn_info *info_dev, void *workspace, cudaStream_t s) {
+    const LstmLayout L = lstm_layout(*cell, B, T);
+    char *ws = static_cast<char *>(workspace);
+    float *P = reinterpret_cast<float *>(ws + L.P);
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws + L.header);
+    cudaError_t e = cudaMemsetAsync(ws + L.header, 0, 256, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.desc, 0, L.total - L.desc, s);
+    if (e == cudaSuccess)
+        e = launch_projection_n(cell->x_dtype, x, params->w_ih, params->b_ih, P, static_cast<long long>(B) * T,
+                                4 * cell->d, cell->din, s);
+    if (e == cudaSuccess)
+        e = launch_lstm_diag(P, params->w_hh, params->b_hh, c0, h0, B, T, cell->d, tol, max_iters,
+                             reinterpret_cast<float *>(ws + L.cws), reinterpret_cast<float *>(ws + L.hws), c, h, hdr,
+                             ws + L.desc, info_dev, s);
+    return e;
+}
 }  // namespace
 
 size_t pararnn_lstm_workspace_size(const pararnn_cell *cell, int B, int T) {
@@ -507,19 +528,9 @@ int pararnn_lstm_solve(const pararnn_cell *cell, const pararnn_params *params, c
         overlaps(c, sb, x, xb) || overlaps(h, sb, x, xb) || overlaps(c, sb, c0, bd) || overlaps(c, sb, h0, bd) ||
         overlaps(h, sb, c0, bd) || overlaps(h, sb, h0, bd))
         return PARARNN_INVALID_ARG;
-    char *ws = static_cast<char *>(workspace);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    float *P = reinterpret_cast<float *>(ws + L.P);
-    WsHeader *hdr = reinterpret_cast<WsHeader *>(ws + L.header);
-    cudaError_t e = cudaMemsetAsync(ws + L.header, 0, 256, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(ws + L.desc, 0, L.total - L.desc, s);
-    if (e == cudaSuccess)
-        e = launch_projection_n(cell->x_dtype, x, params->w_ih, params->b_ih, P, static_cast<long long>(B) * T,
-                                4 * cell->d, cell->din, s);
-    if (e == cudaSuccess)
-        e = launch_lstm_diag(P, params->w_hh, params->b_hh, c0, h0, B, T, cell->d, tol, max_iters,
-                             reinterpret_cast<float *>(ws + L.cws), reinterpret_cast<float *>(ws + L.hws), c, h, hdr,
-                             ws + L.desc, nullptr, s);
+    const WsHeader *hdr = reinterpret_cast<const WsHeader *>(static_cast<char *>(workspace) + L.header);
+    cudaError_t e = lstm_enqueue(cell, params, x, c0, h0, B, T, tol, max_iters, c, h, nullptr, workspace, s);
     pararnn_info host{};
     if (e == cudaSuccess) e = cudaMemcpyAsync(&host, &hdr->info, sizeof(host), cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
@@ -704,6 +715,117 @@ HostLayout host_layout(const pararnn_cell &cell, int B, int T, int mode, int par
     return H;
 }
 
+// The host arrays one pipeline moves per part: up to two inputs and two
+// outputs, [B, ...] with `row` bytes per sequence, staged in the workspace at
+// off[q] for buffer q.
+struct PipeIo {
+    int nin = 0, nout = 0;
+    const char *in[2] = {};
+    char *out[2] = {};
+    size_t in_row[2] = {}, out_row[2] = {};
+    size_t in_off[2][kHostBufs] = {}, out_off[2][kHostBufs] = {};
+};
+
+// The batch in ramped parts (part_sizes) through `nbuf` staging buffers: part
+// p's inputs are copied in on one helper stream, solved on `sc` by
+// enq(p, b0, nb, buf) (returns a pararnn status), and its outputs copied out
+// on a second helper stream; pre(s_in) enqueues the copies made once per call
+// (initial states).  On return `sc` is ordered after the last copy out.
+extern "C++" {  // a template: C++ linkage inside the exported block
+template <class Pre, class Enq>
+int run_pipeline(int B, int parts, int nbuf, const PipeIo &io, char *ws, cudaStream_t sc, Pre pre, Enq enq) {
+    constexpr int NB = kHostBufs;
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev[3 * NB + 1] = {};  // in[NB], comp[NB], out[NB], start / end
+    cudaEvent_t *ev_in = ev, *ev_comp = ev + NB, *ev_out = ev + 2 * NB, &ev_edge = ev[3 * NB];
+    cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
+    for (int q = 0; q < 3 * NB + 1 && e == cudaSuccess; ++q)
+        e = cudaEventCreateWithFlags(&ev[q], cudaEventDisableTiming);
+    int rc = PARARNN_OK;
+    if (e == cudaSuccess) {  // start only after the caller's earlier work on its stream
+        e = cudaEventRecord(ev_edge, sc);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev_edge, 0);
+        if (e == cudaSuccess) e = pre(s_in);
+    }
+    const std::vector<int> sizes = part_sizes(B, parts);
+    int b0 = 0;
+    for (int p = 0; p < parts && e == cudaSuccess && rc == PARARNN_OK; b0 += sizes[p], ++p) {
+        const int buf = p % nbuf, nb = sizes[p];
+        if (p >= nbuf) e = cudaStreamWaitEvent(s_in, ev_out[buf], 0);  // staging of part p-nbuf free
+        for (int a = 0; a < io.nin && e == cudaSuccess; ++a)
+            e = cudaMemcpyAsync(ws + io.in_off[a][buf], io.in[a] + b0 * io.in_row[a], nb * io.in_row[a],
+                                cudaMemcpyHostToDevice, s_in);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_in[buf], s_in);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(sc, ev_in[buf], 0);
+        if (e != cudaSuccess) break;
+        rc = enq(p, b0, nb, buf);
+        if (rc != PARARNN_OK) break;
+        e = cudaEventRecord(ev_comp[buf], sc);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_comp[buf], 0);
+        for (int a = 0; a < io.nout && e == cudaSuccess; ++a)
+            e = cudaMemcpyAsync(io.out[a] + b0 * io.out_row[a], ws + io.out_off[a][buf], nb * io.out_row[a],
+                                cudaMemcpyDeviceToHost, s_out);
+        if (e == cudaSuccess) e = cudaEventRecord(ev_out[buf], s_out);
+    }
+    if (e == cudaSuccess && rc == PARARNN_OK) {  // the caller's stream continues after the last copy out
+        e = cudaEventRecord(ev_edge, s_out);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(sc, ev_edge, 0);
+    }
+    // leave nothing in flight before the helper streams go away
+    if (s_in) cudaStreamSynchronize(s_in);
+    if (s_out) cudaStreamSynchronize(s_out);
+    for (int q = 0; q < 3 * NB + 1; ++q)
+        if (ev[q]) cudaEventDestroy(ev[q]);
+    if (s_in) cudaStreamDestroy(s_in);
+    if (s_out) cudaStreamDestroy(s_out);
+    if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
+    return rc;
+}
+}  // extern "C++"
+
+// Wait for `sc`, read the parts' reports and fold them: the worst part
+// (statuses are ordered by severity), the largest count, delta and residual.
+int fold_reports(const pararnn_info *infos_dev, int parts, cudaStream_t sc, pararnn_info *info) {
+    std::vector<pararnn_info> host(parts);
+    cudaError_t e = cudaMemcpyAsync(host.data(), infos_dev, parts * sizeof(pararnn_info), cudaMemcpyDeviceToHost, sc);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(sc);
+    if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
+    pararnn_info agg{};
+    for (int p = 0; p < parts; ++p) {
+        agg.iters = host[p].iters > agg.iters ? host[p].iters : agg.iters;
+        agg.status = host[p].status > agg.status ? host[p].status : agg.status;
+        agg.delta = host[p].delta > agg.delta ? host[p].delta : agg.delta;
+        agg.residual = host[p].residual > agg.residual ? host[p].residual : agg.residual;
+    }
+    if (info) *info = agg;
+    return agg.status;
+}
+
+struct LstmHostLayout {
+    int bp, nbuf;
+    size_t solve, xs[kHostBufs], cs[kHostBufs], hs[kHostBufs], c0, h0, infos, total;
+};
+
+LstmHostLayout lstm_host_layout(const pararnn_cell &cell, int B, int T, int parts) {
+    LstmHostLayout H{};
+    for (int v : part_sizes(B, parts)) H.bp = v > H.bp ? v : H.bp;
+    H.nbuf = parts < kHostBufs ? parts : kHostBufs;
+    const size_t es = cell.x_dtype == PARARNN_BF16 ? 2 : 4;
+    const size_t xbytes = static_cast<size_t>(H.bp) * T * cell.din * es;
+    const size_t sbytes = static_cast<size_t>(H.bp) * T * cell.d * 4;
+    size_t off = 0;
+    H.solve = off; off = align256(off + lstm_layout(cell, H.bp, T).total);
+    for (int q = 0; q < H.nbuf; ++q) { H.xs[q] = off; off = align256(off + xbytes); }
+    for (int q = 0; q < H.nbuf; ++q) { H.cs[q] = off; off = align256(off + sbytes); }
+    for (int q = 0; q < H.nbuf; ++q) { H.hs[q] = off; off = align256(off + sbytes); }
+    H.c0 = off; off = align256(off + static_cast<size_t>(B) * cell.d * 4);
+    H.h0 = off; off = align256(off + static_cast<size_t>(B) * cell.d * 4);
+    H.infos = off; off = align256(off + static_cast<size_t>(parts) * sizeof(pararnn_info));
+    H.total = off;
+    return H;
+}
+
 }  // namespace
 
 size_t pararnn_host_workspace_size(const pararnn_cell *cell, int B, int T, int mode, int parts) {
@@ -722,79 +844,78 @@ int pararnn_newton_solve_host(const pararnn_cell *cell, const pararnn_params *pa
     if (ws_bytes < H.total) return PARARNN_INVALID_ARG;
     char *ws = static_cast<char *>(workspace);
     const size_t es = cell->x_dtype == PARARNN_BF16 ? 2 : 4;
-    const size_t xrow = static_cast<size_t>(T) * cell->din * es;  // bytes of one sequence's input
-    const size_t hrow = static_cast<size_t>(T) * cell->d * 4;      // bytes of one sequence's states
+    PipeIo io;
+    io.nin = io.nout = 1;
+    io.in[0] = static_cast<const char *>(x_host);
+    io.in_row[0] = static_cast<size_t>(T) * cell->din * es;  // bytes of one sequence's input
+    io.out[0] = reinterpret_cast<char *>(h_host);
+    io.out_row[0] = static_cast<size_t>(T) * cell->d * 4;    // bytes of one sequence's states
+    for (int q = 0; q < H.nbuf; ++q) io.in_off[0][q] = H.xs[q], io.out_off[0][q] = H.hs[q];
     cudaStream_t sc = reinterpret_cast<cudaStream_t>(stream);
-    cudaStream_t s_in = nullptr, s_out = nullptr;
-    constexpr int NB = kHostBufs;
-    cudaEvent_t ev[3 * NB + 1] = {};  // in[NB], comp[NB], out[NB], start / end
-    cudaEvent_t *ev_in = ev, *ev_comp = ev + NB, *ev_out = ev + 2 * NB, &ev_edge = ev[3 * NB];
-    cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
-    for (int q = 0; q < 3 * NB + 1 && e == cudaSuccess; ++q)
-        e = cudaEventCreateWithFlags(&ev[q], cudaEventDisableTiming);
-    int rc = PARARNN_OK;
     float *h0_dev = reinterpret_cast<float *>(ws + H.h0);
     pararnn_info *infos = reinterpret_cast<pararnn_info *>(ws + H.infos);
-    if (e == cudaSuccess) {
-        // start only after the caller's earlier work on its stream
-        e = cudaEventRecord(ev_edge, sc);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev_edge, 0);
-        if (e == cudaSuccess)
-            e = cudaMemcpyAsync(h0_dev, h0_host, static_cast<size_t>(B) * cell->d * 4, cudaMemcpyHostToDevice, s_in);
-    }
-    const std::vector<int> sizes = part_sizes(B, H.parts);
-    int b0 = 0;
-    for (int p = 0; p < H.parts && e == cudaSuccess && rc == PARARNN_OK; b0 += sizes[p], ++p) {
-        const int buf = p % H.nbuf;
-        const int nb = sizes[p];
-        if (p >= H.nbuf) e = cudaStreamWaitEvent(s_in, ev_out[buf], 0);  // staging of part p-nbuf free
-        if (e == cudaSuccess)
-            e = cudaMemcpyAsync(ws + H.xs[buf], static_cast<const char *>(x_host) + b0 * xrow, nb * xrow,
-                                cudaMemcpyHostToDevice, s_in);
-        if (e == cudaSuccess) e = cudaEventRecord(ev_in[buf], s_in);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(sc, ev_in[buf], 0);
-        if (e != cudaSuccess) break;
-        rc = solve_enqueue(cell, params, ws + H.xs[buf], h0_dev + static_cast<size_t>(b0) * cell->d, nb, T, mode,
-                           lambda, tol, max_iters, reinterpret_cast<float *>(ws + H.hs[buf]), infos + p,
-                           ws + H.solve, ws_layout(*cell, nb, T, mode).total, stream);
-        if (rc != PARARNN_OK) break;
-        e = cudaEventRecord(ev_comp[buf], sc);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_comp[buf], 0);
-        if (e == cudaSuccess)
-            e = cudaMemcpyAsync(reinterpret_cast<char *>(h_host) + b0 * hrow, ws + H.hs[buf], nb * hrow,
-                                cudaMemcpyDeviceToHost, s_out);
-        if (e == cudaSuccess) e = cudaEventRecord(ev_out[buf], s_out);
-    }
-    // the caller's stream continues after the last copy out
-    pararnn_info agg{};
-    if (e == cudaSuccess && rc == PARARNN_OK) {
-        e = cudaEventRecord(ev_edge, s_out);
-        if (e == cudaSuccess) e = cudaStreamWaitEvent(sc, ev_edge, 0);
-        std::vector<pararnn_info> host(H.parts);
-        if (e == cudaSuccess)
-            e = cudaMemcpyAsync(host.data(), infos, H.parts * sizeof(pararnn_info), cudaMemcpyDeviceToHost, sc);
-        if (e == cudaSuccess) e = cudaStreamSynchronize(sc);
-        if (e == cudaSuccess) {
-            for (int p = 0; p < H.parts; ++p) {  // worst part: statuses are ordered by severity
-                agg.iters = host[p].iters > agg.iters ? host[p].iters : agg.iters;
-                agg.status = host[p].status > agg.status ? host[p].status : agg.status;
-                agg.delta = host[p].delta > agg.delta ? host[p].delta : agg.delta;
-                agg.residual = host[p].residual > agg.residual ? host[p].residual : agg.residual;
-            }
-            if (info) *info = agg;
-            rc = agg.status;
-        }
-    }
-    // leave nothing in flight before the helper streams go away
-    if (s_in) cudaStreamSynchronize(s_in);
-    if (s_out) cudaStreamSynchronize(s_out);
-    for (int q = 0; q < 3 * NB + 1; ++q)
-        if (ev[q]) cudaEventDestroy(ev[q]);
-    if (s_in) cudaStreamDestroy(s_in);
-    if (s_out) cudaStreamDestroy(s_out);
-    if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
-    return rc;
+    auto pre = [&](cudaStream_t s_in) {
+        return cudaMemcpyAsync(h0_dev, h0_host, static_cast<size_t>(B) * cell->d * 4, cudaMemcpyHostToDevice, s_in);
+    };
+    auto enq = [&](int p, int b0, int nb, int buf) {
+        return solve_enqueue(cell, params, ws + H.xs[buf], h0_dev + static_cast<size_t>(b0) * cell->d, nb, T, mode,
+                             lambda, tol, max_iters, reinterpret_cast<float *>(ws + H.hs[buf]), infos + p,
+                             ws + H.solve, ws_layout(*cell, nb, T, mode).total, stream);
+    };
+    const int rc = run_pipeline(B, parts, H.nbuf, io, ws, sc, pre, enq);
+    if (rc != PARARNN_OK) return rc;
+    return fold_reports(infos, parts, sc, info);
+}
+
+size_t pararnn_lstm_host_workspace_size(const pararnn_cell *cell, int B, int T, int parts) {
+    if (!lstm_cell_ok(cell, B, T) || parts < 1 || parts > B) return 0;
+    return lstm_host_layout(*cell, B, T, parts).total;
+}
+
+int pararnn_lstm_solve_host(const pararnn_cell *cell, const pararnn_params *params, const void *x_host,
+                            const float *c0_host, const float *h0_host, int B, int T, float tol, int max_iters,
+                            float *c_host, float *h_host, pararnn_info *info, int parts, void *workspace,
+                            size_t ws_bytes, pararnn_stream stream) {
+    if (!lstm_cell_ok(cell, B, T) || parts < 1 || parts > B || !params || !params->w_ih || !params->b_ih ||
+        !params->w_hh || !params->b_hh || !x_host || !c0_host || !h0_host || !c_host || !h_host || !workspace ||
+        !aligned(workspace, 256) || !(tol >= 0.f) || !std::isfinite(tol))
+        return PARARNN_INVALID_ARG;
+    const void *ptrs[] = {params->w_ih, params->b_ih, params->w_hh, params->b_hh};
+    for (const void *q : ptrs)
+        if (!aligned(q, 16)) return PARARNN_INVALID_ARG;
+    const LstmHostLayout H = lstm_host_layout(*cell, B, T, parts);
+    if (ws_bytes < H.total) return PARARNN_INVALID_ARG;
+    char *ws = static_cast<char *>(workspace);
+    const size_t es = cell->x_dtype == PARARNN_BF16 ? 2 : 4;
+    const size_t srow = static_cast<size_t>(T) * cell->d * 4;
+    PipeIo io;
+    io.nin = 1;
+    io.nout = 2;
+    io.in[0] = static_cast<const char *>(x_host);
+    io.in_row[0] = static_cast<size_t>(T) * cell->din * es;
+    io.out[0] = reinterpret_cast<char *>(c_host);
+    io.out[1] = reinterpret_cast<char *>(h_host);
+    io.out_row[0] = io.out_row[1] = srow;
+    for (int q = 0; q < H.nbuf; ++q) io.in_off[0][q] = H.xs[q], io.out_off[0][q] = H.cs[q], io.out_off[1][q] = H.hs[q];
+    cudaStream_t sc = reinterpret_cast<cudaStream_t>(stream);
+    float *c0_dev = reinterpret_cast<float *>(ws + H.c0), *h0_dev = reinterpret_cast<float *>(ws + H.h0);
+    pararnn_info *infos = reinterpret_cast<pararnn_info *>(ws + H.infos);
+    const size_t bd = static_cast<size_t>(B) * cell->d * 4;
+    auto pre = [&](cudaStream_t s_in) {
+        cudaError_t e = cudaMemcpyAsync(c0_dev, c0_host, bd, cudaMemcpyHostToDevice, s_in);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(h0_dev, h0_host, bd, cudaMemcpyHostToDevice, s_in);
+        return e;
+    };
+    auto enq = [&](int p, int b0, int nb, int buf) {
+        const size_t o = static_cast<size_t>(b0) * cell->d;
+        const cudaError_t e = lstm_enqueue(cell, params, ws + H.xs[buf], c0_dev + o, h0_dev + o, nb, T, tol,
+                                           max_iters, reinterpret_cast<float *>(ws + H.cs[buf]),
+                                           reinterpret_cast<float *>(ws + H.hs[buf]), infos + p, ws + H.solve, sc);
+        return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
+    };
+    const int rc = run_pipeline(B, parts, H.nbuf, io, ws, sc, pre, enq);
+    if (rc != PARARNN_OK) return rc;
+    return fold_reports(infos, parts, sc, info);
 }
 
 }  // extern "C"

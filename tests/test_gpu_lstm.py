@@ -82,3 +82,23 @@ def test_statuses_and_rejections():
     c, h, r = _solve(w, tol=0.0, max_iters=2)
     assert r.status == "NOT_CONVERGED" and r.iters == 2
     assert binding.lstm_workspace_size(4, 6, 1, 50) == 0  # d % 4 != 0
+
+
+@pytest.mark.parametrize("B,T,d,din,parts", [(5, 400, 64, 32, 3), (4, 300, 128, 64, 4), (3, 200, 64, 16, 1)])
+def test_host_buffer_solve(B, T, d, din, parts):
+    """From and to host memory in ramped parts: with one part the states equal
+    the device solve's bit for bit; in any split the parts are independent
+    solves, so the converged (c, h) match the fp64 rollout within 1e-4."""
+    w = make_lstm_workload(B=B, T=T, d=d, din=din, x_dtype=torch.float32, bias_std=0.3, state_std=0.5, seed=B * T)
+    dev = lambda t: t.cuda().contiguous()
+    pin = lambda t: t.contiguous().pin_memory()
+    c, h, r = binding.lstm_solve_host(dev(w.w_ih), dev(w.b_ih), dev(w.u), dev(w.b_hh), pin(w.x), pin(w.c0),
+                                      pin(w.h0), tol=w.tol, parts=parts)
+    assert r.status == "OK" and not c.is_cuda and not h.is_cuda
+    cell, x, c0, h0 = _oracle(w)
+    cr, hr = lstm_rollout(cell, x, c0, h0)
+    assert np.max(np.abs(c.double().numpy() - cr)) <= 1e-4
+    assert np.max(np.abs(h.double().numpy() - hr)) <= 1e-4
+    if parts == 1:
+        cd, hd, rd = _solve(w)
+        assert torch.equal(cd.cpu(), c) and torch.equal(hd.cpu(), h) and rd.iters == r.iters
