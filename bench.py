@@ -388,20 +388,25 @@ def run_adjoint(args):
     max_ms = max_over_ranks(sum(ms), dev)
     value = job_value(states, args.steps, world, max_ms)
     st = binding.lib().pararnn_adjoint_status(ws.data_ptr(), stream.cuda_stream)
-    # end to end: P, h and dL/dh from page-locked host memory, dL/dP back, each step
-    hP, hh, hdh = P.cpu().pin_memory(), h.cpu().pin_memory(), dh.cpu().pin_memory()
-    hdP = torch.empty(P.shape, dtype=torch.float32).pin_memory()
+    # end to end through the public host-buffer call: P, h0, h and dL/dh from
+    # page-locked host memory; dL/dP, dL/dh0 and the parameter gradients back;
+    # the library overlaps the copies with the parts' passes
+    hP, hh, hdh, hh0 = (t.cpu().pin_memory() for t in (P, h, dh, h0))
+    parts = max(1, min(E2E_PARTS, B))
+    hout = dict(dP=torch.empty(P.shape).pin_memory(), dh0=torch.empty(h0.shape).pin_memory(),
+                dw_hh=torch.empty(u.shape).pin_memory(), db_hh=torch.empty(bh.shape).pin_memory())
+    ws_host = binding.alloc_workspace(int(binding.lib().pararnn_adjoint_host_workspace_size(
+        binding.make_cell(w.kind if w.kind == "dense" else "diag", 1, D, torch.float32), B, T, parts)), dev)
+    e2e_step = lambda: binding.adjoint_host(u, bh, hP, hh0, hh, hdh, parts=parts, out=hout, workspace=ws_host,
+                                            stream=stream)
+    e2e_step()
     e2e_steps = max(1, min(args.steps, 3))
     barrier()
     torch.cuda.synchronize()
     ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ea.record(stream)
     for _ in range(e2e_steps):
-        P.copy_(hP, non_blocking=True)
-        h.copy_(hh, non_blocking=True)
-        dh.copy_(hdh, non_blocking=True)
-        step()
-        hdP.copy_(out["dP"], non_blocking=True)
+        e2e_step()
     eb.record(stream)
     torch.cuda.synchronize()
     e2e_value = job_value(states, e2e_steps, world, max_over_ranks(ea.elapsed_time(eb), dev))
@@ -423,8 +428,8 @@ def run_adjoint(args):
                      "algorithmic": f"{spec['per_state']} B/state x {states} states",
                      "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"},
         "e2e": {"value": e2e_value, "unit": UNIT,
-                "h2d_bytes_per_step": (P.numel() + h.numel() + dh.numel()) * 4,
-                "d2h_bytes_per_step": P.numel() * 4},
+                "h2d_bytes_per_step": (P.numel() + h.numel() + dh.numel() + h0.numel()) * 4,
+                "d2h_bytes_per_step": (P.numel() + h0.numel() + u.numel() + bh.numel()) * 4, "parts": parts},
         "gpu_launches": (4 if w.kind == "dense" else 1) * args.steps,
         "clocks": clk.summary(),
     }

@@ -476,6 +476,30 @@ PARARNN_API int pararnn_lstm_solve(const pararnn_cell *cell, const pararnn_param
 PARARNN_API size_t pararnn_lstm_workspace_size(const pararnn_cell *cell, int B, int T);
 
 /*
+ * pararnn_adjoint_host -- pararnn_adjoint from and to HOST memory, the copies
+ * overlapped with the computation through the host-buffer pipeline (ramped
+ * parts, three staging buffers, copy streams the call creates): part p's P,
+ * h and dL/dh are copied in while its neighbours are computed, its dL/dP
+ * copied out.  Each part's dW_hh and db_hh partial sums stay on the device and
+ * are added in part order at the end (deterministic for a given `parts`).
+ *   P_host [B, T, 3D], h0_host [B, D], h_host, dh_host [B, T, D]: HOST float.
+ *   dP_host [B, T, 3D], dh0_host [B, D], dw_hh_host (the cell's w_hh shape),
+ *   db_hh_host [3D]: HOST float outputs.  Page-locked memory lets the copies
+ *   run asynchronously.  params->w_hh, b_hh: DEVICE, as for pararnn_adjoint.
+ *   parts      1 <= parts <= B.
+ *   workspace  DEVICE, >= pararnn_adjoint_host_workspace_size bytes.
+ * Synchronises `stream` once, at the end; returns PARARNN_OK, PARARNN_TIMEOUT
+ * (a bounded device-side wait expired in some part), INVALID_ARG or CUDA_ERROR.
+ */
+PARARNN_API int pararnn_adjoint_host(const pararnn_cell *cell, const pararnn_params *params, const float *P_host,
+                                     const float *h0_host, const float *h_host, const float *dh_host, int B, int T,
+                                     float *dP_host, float *dh0_host, float *dw_hh_host, float *db_hh_host,
+                                     int parts, void *workspace, size_t ws_bytes, pararnn_stream stream);
+
+/* pararnn_adjoint_host_workspace_size -- bytes pararnn_adjoint_host needs, or 0. */
+PARARNN_API size_t pararnn_adjoint_host_workspace_size(const pararnn_cell *cell, int B, int T, int parts);
+
+/*
  * pararnn_lstm_solve_host -- pararnn_lstm_solve from and to HOST memory, with
  * the copies overlapped with the computation as in pararnn_newton_solve_host:
  * the batch in `parts` ramped parts (same sizes), three staging buffers, part

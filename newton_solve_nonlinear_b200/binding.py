@@ -29,7 +29,7 @@ EXPORTS = ("pararnn_workspace_size", "pararnn_newton_solve", "pararnn_newton_sol
            "pararnn_adjoint_status", "pararnn_newton_solve_guess_async", "pararnn_newton_solve_chunked",
            "pararnn_chunked_workspace_size", "pararnn_lstm_solve", "pararnn_lstm_workspace_size",
            "pararnn_newton_solve_reuse", "pararnn_reuse_workspace_size", "pararnn_lstm_solve_host",
-           "pararnn_lstm_host_workspace_size")
+           "pararnn_lstm_host_workspace_size", "pararnn_adjoint_host", "pararnn_adjoint_host_workspace_size")
 
 
 class Cell(ctypes.Structure):
@@ -113,6 +113,11 @@ def lib() -> ctypes.CDLL:
         L.pararnn_lstm_solve_host.restype = ci
         L.pararnn_lstm_host_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci, ci]
         L.pararnn_lstm_host_workspace_size.restype = sz
+        L.pararnn_adjoint_host.argtypes = [ctypes.POINTER(Cell), ctypes.POINTER(Params), vp, vp, vp, vp, ci, ci,
+                                           vp, vp, vp, vp, ci, vp, sz, vp]
+        L.pararnn_adjoint_host.restype = ci
+        L.pararnn_adjoint_host_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci, ci]
+        L.pararnn_adjoint_host_workspace_size.restype = sz
         L.pararnn_status_string.argtypes = [ci]
         L.pararnn_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -408,10 +413,10 @@ def adjoint(w_hh, b_hh, P, h0, h, dh, *, workspace=None, out=None, stream=None, 
     if workspace is None:
         workspace = alloc_workspace(need, h.device)
     o = out or {}
-    dP = o.get("dP", torch.empty_like(P))
-    dh0 = o.get("dh0", torch.empty_like(h0))
-    dw = o.get("dw_hh", torch.empty_like(w_hh))
-    db = o.get("db_hh", torch.empty_like(b_hh))
+    dP = o["dP"] if "dP" in o else torch.empty_like(P)
+    dh0 = o["dh0"] if "dh0" in o else torch.empty_like(h0)
+    dw = o["dw_hh"] if "dw_hh" in o else torch.empty_like(w_hh)
+    db = o["db_hh"] if "db_hh" in o else torch.empty_like(b_hh)
     params = Params(None, None, _dev(w_hh, "w_hh"), _dev(b_hh, "b_hh"))
     rc = L.pararnn_adjoint(ctypes.byref(cell), ctypes.byref(params), _dev(P, "P"), _dev(h0, "h0"), _dev(h, "h"),
                            _dev(dh, "dh"), B, T, _dev(dP, "dP"), _dev(dh0, "dh0"), _dev(dw, "dw_hh"),
@@ -422,6 +427,38 @@ def adjoint(w_hh, b_hh, P, h0, h, dh, *, workspace=None, out=None, stream=None, 
         st = L.pararnn_adjoint_status(_dev(workspace, "workspace"), _stream(stream))
         if st != 0:
             raise RuntimeError(f"pararnn_adjoint: {STATUS.get(st, st)}")
+    return dict(dP=dP, dh0=dh0, dw_hh=dw, db_hh=db)
+
+
+def adjoint_host(w_hh, b_hh, P_host, h0_host, h_host, dh_host, *, parts: int = 4, out=None, workspace=None,
+                 stream=None) -> dict:
+    """The backward pass from and to HOST tensors (P_host [B,T,3D], h0_host
+    [B,D], h_host and dh_host [B,T,D], page-locked for overlap), in ``parts``
+    parts with the copies overlapped with compute; w_hh, b_hh CUDA tensors
+    (w_hh [3D]: diagonal cell, [3D, D]: dense cell).  Returns dict(dP, dh0,
+    dw_hh, db_hh) of host tensors."""
+    B, T, d = h_host.shape
+    parts = max(1, min(int(parts), B))
+    cell = make_cell("dense" if w_hh.dim() == 2 else "diag", 1, d, torch.float32)
+    L = lib()
+    need = int(L.pararnn_adjoint_host_workspace_size(ctypes.byref(cell), B, T, parts))
+    if need == 0:
+        raise ValueError("arguments rejected by pararnn_adjoint_host_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, w_hh.device)
+    o = out or {}
+    pinned = lambda key, shape: o[key] if key in o else torch.empty(shape, dtype=torch.float32).pin_memory()
+    dP = pinned("dP", P_host.shape)
+    dh0 = pinned("dh0", h0_host.shape)
+    dw = pinned("dw_hh", w_hh.shape)
+    db = pinned("db_hh", b_hh.shape)
+    params = Params(None, None, _dev(w_hh, "w_hh"), _dev(b_hh, "b_hh"))
+    rc = L.pararnn_adjoint_host(ctypes.byref(cell), ctypes.byref(params), _host(P_host, "P_host"),
+                                _host(h0_host, "h0_host"), _host(h_host, "h_host"), _host(dh_host, "dh_host"), B, T,
+                                _host(dP, "dP"), _host(dh0, "dh0"), _host(dw, "dw_hh"), _host(db, "db_hh"), parts,
+                                _dev(workspace, "workspace"), workspace.numel(), _stream(stream))
+    if rc != 0:
+        raise RuntimeError(f"pararnn_adjoint_host: {L.pararnn_status_string(rc).decode()}")
     return dict(dP=dP, dh0=dh0, dw_hh=dw, db_hh=db)
 
 

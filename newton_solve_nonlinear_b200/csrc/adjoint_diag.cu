@@ -430,6 +430,12 @@ cudaError_t launch_outer_sum(const float *grow, const float *hp, long long M, in
     return cudaGetLastError();
 }
 
+// out[o] = sum over r < rows of in[r][o] (o < n), added in row order.
+cudaError_t launch_sum_rows(const float *in, int rows, int n, float *out, cudaStream_t s) {
+    outer_sum_reduce_kernel<<<(n + 31) / 32, 32 * ORW, 0, s>>>(in, rows, n, out);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_adjoint_diag(const float *P, const float *h0, const float *h, const float *dh, const float *u,
                                 const float *b_hh, float *dP, float *dh0, float *du, float *db_hh, int B, int T,
                                 int D, void *hdr, void *desc, void *part, cudaStream_t s, const float *w_hh_dense,

@@ -45,6 +45,10 @@ cudaError_t launch_adjoint_diag(const float *P, const float *h0, const float *h,
                                 const float *G, float *grow);
 size_t adjoint_outer_part_bytes(long long M, int N, int K);
 bool deer_mma_supported(const pararnn_cell &cell);
+cudaError_t launch_sum_rows(const float *in, int rows, int n, float *out, cudaStream_t s);
+cudaError_t adjoint_enqueue(const pararnn_cell *cell, const pararnn_params *params, const float *P, const float *h0,
+                            const float *h, const float *dh, int B, int T, float *dP, float *dh0, float *dw_hh,
+                            float *db_hh, void *workspace, cudaStream_t s);
 cudaError_t launch_outer_sum(const float *grow, const float *hp, long long M, int N, int K, float *part, float *out,
                              cudaStream_t s);
 
@@ -596,16 +600,33 @@ int pararnn_adjoint(const pararnn_cell *cell, const pararnn_params *params, cons
         for (const auto &o2 : outs)
             if (&o2 != &o && overlaps(o.p, o.n, o2.p, o2.n)) return PARARNN_INVALID_ARG;
     }
+    const cudaError_t e = adjoint_enqueue(cell, params, P, h0, h, dh, B, T, dP, dh0, dw_hh, db_hh, workspace,
+                                          reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
+}
+
+int pararnn_adjoint_status(const void *workspace, pararnn_stream stream) {
+    return pararnn_affine_scan_status(workspace, stream);
+}
+
+}  // extern "C"
+
+namespace pararnn {
+// The backward pass enqueued on `s` (arguments already checked).
+cudaError_t adjoint_enqueue(const pararnn_cell *cell, const pararnn_params *params, const float *P, const float *h0,
+                            const float *h, const float *dh, int B, int T, float *dP, float *dh0, float *dw_hh,
+                            float *db_hh, void *workspace, cudaStream_t s) {
+    const int D = cell->d;
+    const bool dense = cell->kind == PARARNN_GRU_DENSE;
     const AdjLayout L = adj_layout(B, T, D, dense);
     char *ws = static_cast<char *>(workspace);
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // header (status, grid barrier) and look-back words start at zero
     cudaError_t e = cudaMemsetAsync(ws, 0, L.part, s);
     if (!dense) {
         if (e == cudaSuccess)
             e = launch_adjoint_diag(P, h0, h, dh, params->w_hh, params->b_hh, dP, dh0, dw_hh, db_hh, B, T, D,
                                     ws + L.header, ws + L.desc, ws + L.part, s, nullptr, nullptr, nullptr);
-        return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
+        return e;
     }
     // dense cell: h_{t-1} packed [B, T, D] (h0, then the states shifted by one step)
     float *hp = reinterpret_cast<float *>(ws + L.hprev);
@@ -627,12 +648,11 @@ int pararnn_adjoint(const pararnn_cell *cell, const pararnn_params *params, cons
     if (e == cudaSuccess)
         e = launch_outer_sum(grow, hp, static_cast<long long>(B) * T, 3 * D, D,
                              reinterpret_cast<float *>(ws + L.opart), dw_hh, s);
-    return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
+    return e;
 }
+}  // namespace pararnn
 
-int pararnn_adjoint_status(const void *workspace, pararnn_stream stream) {
-    return pararnn_affine_scan_status(workspace, stream);
-}
+extern "C" {
 
 const char *pararnn_status_string(int status) {
     switch (status) {
@@ -715,15 +735,15 @@ HostLayout host_layout(const pararnn_cell &cell, int B, int T, int mode, int par
     return H;
 }
 
-// The host arrays one pipeline moves per part: up to two inputs and two
+// The host arrays one pipeline moves per part: up to three inputs and two
 // outputs, [B, ...] with `row` bytes per sequence, staged in the workspace at
 // off[q] for buffer q.
 struct PipeIo {
     int nin = 0, nout = 0;
-    const char *in[2] = {};
+    const char *in[3] = {};
     char *out[2] = {};
-    size_t in_row[2] = {}, out_row[2] = {};
-    size_t in_off[2][kHostBufs] = {}, out_off[2][kHostBufs] = {};
+    size_t in_row[3] = {}, out_row[2] = {};
+    size_t in_off[3][kHostBufs] = {}, out_off[2][kHostBufs] = {};
 };
 
 // The batch in ramped parts (part_sizes) through `nbuf` staging buffers: part
@@ -826,7 +846,109 @@ LstmHostLayout lstm_host_layout(const pararnn_cell &cell, int B, int T, int part
     return H;
 }
 
+struct AdjHostLayout {
+    int bp, nbuf;
+    size_t solve, Ps[kHostBufs], hs[kHostBufs], dhs[kHostBufs], dPs[kHostBufs], h0, dh0, dwp, dbp, dw, db, stat,
+        total;
+};
+
+// dW_hh per part: 3D (diagonal cell) or 3D x D (dense) floats.
+size_t adj_param_floats(const pararnn_cell &cell) {
+    return static_cast<size_t>(3) * cell.d * (cell.kind == PARARNN_GRU_DENSE ? cell.d : 1);
+}
+
+AdjHostLayout adj_host_layout(const pararnn_cell &cell, int B, int T, int parts) {
+    AdjHostLayout H{};
+    for (int v : part_sizes(B, parts)) H.bp = v > H.bp ? v : H.bp;
+    H.nbuf = parts < kHostBufs ? parts : kHostBufs;
+    const size_t st = static_cast<size_t>(H.bp) * T * cell.d * 4, bd = static_cast<size_t>(B) * cell.d * 4;
+    size_t off = 0;
+    H.solve = off; off = align256(off + pararnn_adjoint_workspace_size(&cell, H.bp, T));
+    for (int q = 0; q < H.nbuf; ++q) { H.Ps[q] = off; off = align256(off + 3 * st); }
+    for (int q = 0; q < H.nbuf; ++q) { H.hs[q] = off; off = align256(off + st); }
+    for (int q = 0; q < H.nbuf; ++q) { H.dhs[q] = off; off = align256(off + st); }
+    for (int q = 0; q < H.nbuf; ++q) { H.dPs[q] = off; off = align256(off + 3 * st); }
+    H.h0 = off; off = align256(off + bd);
+    H.dh0 = off; off = align256(off + bd);
+    H.dwp = off; off = align256(off + static_cast<size_t>(parts) * adj_param_floats(cell) * 4);
+    H.dbp = off; off = align256(off + static_cast<size_t>(parts) * 3 * cell.d * 4);
+    H.dw = off; off = align256(off + adj_param_floats(cell) * 4);
+    H.db = off; off = align256(off + static_cast<size_t>(3) * cell.d * 4);
+    H.stat = off; off = align256(off + static_cast<size_t>(parts) * 4);
+    H.total = off;
+    return H;
+}
+
 }  // namespace
+
+size_t pararnn_adjoint_host_workspace_size(const pararnn_cell *cell, int B, int T, int parts) {
+    if (pararnn_adjoint_workspace_size(cell, B, T) == 0 || parts < 1 || parts > B) return 0;
+    return adj_host_layout(*cell, B, T, parts).total;
+}
+
+int pararnn_adjoint_host(const pararnn_cell *cell, const pararnn_params *params, const float *P_host,
+                         const float *h0_host, const float *h_host, const float *dh_host, int B, int T, float *dP_host,
+                         float *dh0_host, float *dw_hh_host, float *db_hh_host, int parts, void *workspace,
+                         size_t ws_bytes, pararnn_stream stream) {
+    if (pararnn_adjoint_workspace_size(cell, B, T) == 0 || parts < 1 || parts > B || !params || !params->w_hh ||
+        !params->b_hh || !P_host || !h0_host || !h_host || !dh_host || !dP_host || !dh0_host || !dw_hh_host ||
+        !db_hh_host || !workspace || !aligned(workspace, 256) || !aligned(params->w_hh, 16) ||
+        !aligned(params->b_hh, 16))
+        return PARARNN_INVALID_ARG;
+    const AdjHostLayout H = adj_host_layout(*cell, B, T, parts);
+    if (ws_bytes < H.total) return PARARNN_INVALID_ARG;
+    char *ws = static_cast<char *>(workspace);
+    const int D = cell->d;
+    const size_t srow = static_cast<size_t>(T) * D * 4, pf = adj_param_floats(*cell);
+    PipeIo io;  // in: P, h, dL/dh; out: dL/dP
+    io.nin = 3;
+    io.nout = 1;
+    io.in[0] = reinterpret_cast<const char *>(P_host);
+    io.in[1] = reinterpret_cast<const char *>(h_host);
+    io.in[2] = reinterpret_cast<const char *>(dh_host);
+    io.in_row[0] = 3 * srow;
+    io.in_row[1] = io.in_row[2] = srow;
+    io.out[0] = reinterpret_cast<char *>(dP_host);
+    io.out_row[0] = 3 * srow;
+    for (int q = 0; q < H.nbuf; ++q)
+        io.in_off[0][q] = H.Ps[q], io.in_off[1][q] = H.hs[q], io.in_off[2][q] = H.dhs[q], io.out_off[0][q] = H.dPs[q];
+    cudaStream_t sc = reinterpret_cast<cudaStream_t>(stream);
+    float *h0_dev = reinterpret_cast<float *>(ws + H.h0), *dh0_dev = reinterpret_cast<float *>(ws + H.dh0);
+    float *dwp = reinterpret_cast<float *>(ws + H.dwp), *dbp = reinterpret_cast<float *>(ws + H.dbp);
+    unsigned *stat = reinterpret_cast<unsigned *>(ws + H.stat);
+    const WsHeader *shdr = reinterpret_cast<const WsHeader *>(ws + H.solve);
+    const size_t bd = static_cast<size_t>(B) * D * 4;
+    auto pre = [&](cudaStream_t s_in) {
+        return cudaMemcpyAsync(h0_dev, h0_host, bd, cudaMemcpyHostToDevice, s_in);
+    };
+    auto enq = [&](int p, int b0, int nb, int buf) {
+        const size_t o = static_cast<size_t>(b0) * D;
+        cudaError_t e = adjoint_enqueue(cell, params, reinterpret_cast<const float *>(ws + H.Ps[buf]), h0_dev + o,
+                                reinterpret_cast<const float *>(ws + H.hs[buf]),
+                                reinterpret_cast<const float *>(ws + H.dhs[buf]), nb, T,
+                                reinterpret_cast<float *>(ws + H.dPs[buf]), dh0_dev + o, dwp + p * pf,
+                                dbp + static_cast<size_t>(p) * 3 * D, ws + H.solve, sc);
+        if (e == cudaSuccess)  // the part's bounded-wait status, before the next part clears it
+            e = cudaMemcpyAsync(stat + p, &shdr->status, sizeof(unsigned), cudaMemcpyDeviceToDevice, sc);
+        return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
+    };
+    int rc = run_pipeline(B, parts, H.nbuf, io, ws, sc, pre, enq);
+    if (rc != PARARNN_OK) return rc;
+    // the parameter gradients: the parts' sums added in part order
+    float *dw = reinterpret_cast<float *>(ws + H.dw), *db = reinterpret_cast<float *>(ws + H.db);
+    std::vector<unsigned> hstat(parts);
+    cudaError_t e = launch_sum_rows(dwp, parts, static_cast<int>(pf), dw, sc);
+    if (e == cudaSuccess) e = launch_sum_rows(dbp, parts, 3 * D, db, sc);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(dw_hh_host, dw, pf * 4, cudaMemcpyDeviceToHost, sc);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(db_hh_host, db, static_cast<size_t>(3) * D * 4, cudaMemcpyDeviceToHost, sc);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(dh0_host, dh0_dev, bd, cudaMemcpyDeviceToHost, sc);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(hstat.data(), stat, parts * sizeof(unsigned), cudaMemcpyDeviceToHost, sc);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(sc);
+    if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
+    for (unsigned v : hstat)
+        if (v != 0u) return PARARNN_TIMEOUT;
+    return PARARNN_OK;
+}
 
 size_t pararnn_host_workspace_size(const pararnn_cell *cell, int B, int T, int mode, int parts) {
     if (!cell_ok(cell, B, T, mode) || parts < 1 || parts > B) return 0;

@@ -225,3 +225,22 @@ def test_adjoint_gives_autograd_gradients_of_a_solve():
     du = torch.cat([torch.diagonal(gw[k * d:(k + 1) * d]) for k in range(3)])
     assert _rel(r["dw_hh"].double().cpu().numpy(), du.numpy()) <= 1e-4
     assert _rel(r["db_hh"].double().cpu().numpy(), m.bias_hh.grad.numpy()) <= 1e-4
+
+
+@pytest.mark.parametrize("kind,B,T,D,parts", [("diag", 5, 300, 64, 3), ("diag", 3, 100, 130, 1),
+                                              ("dense", 4, 500, 64, 4), ("dense", 2, 77, 12, 2)])
+def test_host_buffer_adjoint_matches_device(kind, B, T, D, parts):
+    """From and to host memory in ramped parts: dL/dP and dL/dh0 are per
+    sequence, so they equal the device pass's bit for bit; dW_hh and db_hh
+    are the parts' sums added in part order (the device pass adds the same
+    terms in another order): normwise within 1e-5."""
+    if kind == "diag":
+        cell, w, b_hh, P, h0, h, dh = _case(B, T, D, seed=B + T)
+    else:
+        cell, w, b_hh, P, h0, h, dh = _dense_case(B, T, D, seed=B + T)
+    ref = binding.adjoint(w.cuda(), b_hh.cuda(), P.cuda(), h0.cuda(), h.cuda(), dh.cuda())
+    pin = lambda t: t.contiguous().pin_memory()
+    got = binding.adjoint_host(w.cuda(), b_hh.cuda(), pin(P), pin(h0), pin(h), pin(dh), parts=parts)
+    assert torch.equal(got["dP"], ref["dP"].cpu()) and torch.equal(got["dh0"], ref["dh0"].cpu())
+    for k in ("dw_hh", "db_hh"):
+        assert _rel(got[k].double().numpy(), ref[k].double().cpu().numpy()) <= 1e-5, k
