@@ -366,18 +366,6 @@ __device__ __forceinline__ void store_phi(float *dst, const float (&psi)[2][4][4
             }
 }
 
-__device__ __forceinline__ void load_phi(float (&ph)[4][4][2], const float *src, const Lane &L) {
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-        for (int kt = 0; kt < 4; ++kt) {
-            const float2 v = __ldcg(reinterpret_cast<const float2 *>(
-                src + (nt * 8 + L.gid) * 32 + kt * 8 + 2 * L.tq));
-            ph[nt][kt][0] = v.x;
-            ph[nt][kt][1] = v.y;
-        }
-}
-
 // y[R(nt)] = sum_k M[R(nt)][k] x[k] + add[R(nt)] from the lane's entries of M.
 __device__ __forceinline__ void matvec(const float (&m)[4][4][2], const float (&xc)[4][2],
                                        const float (&add)[4], float (&row)[4]) {

@@ -52,13 +52,6 @@ struct Diag2Args {
     long long n_tiles;
 };
 
-// Byte offset of (row, lane k < 64) in a pair of 128-byte-swizzled boxes of
-// `box` bytes each (lanes 0..31 in the first, 32..63 in the second).
-__device__ __forceinline__ int sw_off(int row, int k, int box) {
-    const int hf = k >> 5, j = (k & 31) >> 2;
-    return hf * box + row * 128 + ((j ^ (row & 7)) << 4) + ((k & 3) << 2);
-}
-
 __device__ __forceinline__ void issue_fill(const CUtensorMap *mp, const CUtensorMap *mh,
                                            unsigned char *slot, int D, long long row0, int lane0,
                                            unsigned bar) {

@@ -50,7 +50,7 @@ proj_tcgen05_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_cons
     volatile int *issued = reinterpret_cast<volatile int *>(tmem_slot + 2);    // TMA k-blocks issued
     volatile int *consumed = reinterpret_cast<volatile int *>(tmem_slot + 3);  // k-blocks given to MMA
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
     const int m0 = blockIdx.x * BM, n0 = blockIdx.y * BN;
     const int nk = K / BK;
 
