@@ -867,6 +867,8 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
             atomicMax(&hdr->delta_bits[it % 3], bd);
             atomicMax(&hdr->resid_bits[it % 3], br);
             if (*cta_err) flag_timeout(status);
+            // P of the next iteration's first two tiles into L2 while the grid meets
+            for (int q = 0; q < 2 && q < my_n; ++q) prefetch_p<D>(A.P, tile_of(q), B, T);
         }
         grid_barrier(hdr->barrier, nblocks, status);
         last_delta = ld_acquire_u32(&hdr->delta_bits[it % 3]);
