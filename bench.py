@@ -55,30 +55,30 @@ BENCHES = {
         workload="untrained", mode="QUASI", lam=0.0, bound="hbm", per_state=20,
         kernel="quasi_tc2_kernel<64, quasi> (persistent, all iterations)",
         desc="untrained dense GRU Din=D=64, B={B}/GPU, T={T}, fp32, quasi-DEER tol 1e-5",
-        cpu_sample=dict(B=16, T=12288), ref_sample=dict(B=4, T=256), roll_sample=dict()),
+        cpu_sample=dict(B=16, T=12288), ref_sample=dict(B=16, T=4096), roll_sample=dict()),
     "diag": dict(
         workload="diag", mode="QUASI", lam=0.0, bound="hbm", per_state=20,
         kernel="diag2_kernel (persistent, all iterations)",
         desc="diagonal-recurrence GRU Din=D=2048, B={B}/GPU, T={T}, bf16 x and W_ih, fp32 state, "
              "quasi-DEER (exact Newton) tol 1e-4",
-        cpu_sample=dict(B=1, T=16384), ref_sample=dict(B=1, T=128), roll_sample=dict(T=256)),
+        cpu_sample=dict(B=1, T=16384), ref_sample=dict(B=1, T=2048), roll_sample=dict(T=256)),
     "dense_deer": dict(
         workload="dense_deer", mode="DEER", lam=0.0, bound="tensor", per_state=None,
         kernel="deer_mma_kernel (persistent, all iterations)",
         desc="dense GRU Din=16, D=32, B={B}/GPU, T={T}, fp32 cell, TF32 Jacobian products, DEER tol 1e-5",
-        cpu_sample=dict(B=4, T=32768), ref_sample=dict(B=1, T=512), roll_sample=dict()),
+        cpu_sample=dict(B=4, T=32768), ref_sample=dict(B=4, T=4096), roll_sample=dict()),
     "quasi_elk": dict(
         workload="near_unstable", mode="QUASI_ELK", lam=0.1, bound="hbm", per_state=56,
         kernel="quasi_tc2_kernel<64, quasi-ELK> (persistent, all iterations)",
         desc="near-unstable dense GRU Din=D=64 (spectral radius 1.5), B={B}/GPU, T={T}, fp32, "
              "quasi-ELK lambda 0.1, tol 1e-4",
-        cpu_sample=dict(B=8, T=8000), ref_sample=dict(B=1, T=250), roll_sample=dict()),
+        cpu_sample=dict(B=8, T=8000), ref_sample=dict(B=2, T=2000), roll_sample=dict()),
     "elk": dict(
         workload="near_unstable", mode="ELK", lam=0.01, bound="alu", per_state=None,
         kernel="dense_elk_kernel<64> (persistent, all iterations)",
         desc="near-unstable dense GRU Din=D=64 (spectral radius 1.5), B={B}/GPU, T={T}, fp32, "
              "ELK lambda 0.01, tol 1e-4",
-        cpu_sample=dict(B=1, T=5000), ref_sample=dict(B=1, T=150), roll_sample=dict()),
+        cpu_sample=dict(B=1, T=5000), ref_sample=dict(B=1, T=1000), roll_sample=dict()),
     # the backward pass through the evaluated diagonal-cell sequence (not a solve):
     # reads P 12 + h 4 + dL/dh 4, writes dL/dP 12 = 32 B per state
     "adjoint": dict(
@@ -86,7 +86,7 @@ BENCHES = {
         kernel="adjoint_diag_kernel (one reverse pass)",
         desc="backward pass of the diagonal-recurrence GRU Din=D=2048, B={B}/GPU, T={T}: "
              "dL/dP, dL/dh0, dL/du, dL/db_hh from the converged states and dL/dh",
-        cpu_sample=dict(B=1, T=1024), ref_sample=dict(B=1, T=128)),
+        cpu_sample=dict(B=1, T=1024), ref_sample=dict(B=1, T=512)),
 }
 # the dense cell's backward pass with the Jacobian's diagonal: the step is four
 # kernels; algorithmic bytes per state over all of them: h_{t-1} copy 8, GEMM
@@ -98,7 +98,7 @@ BENCHES["adjoint_dense"] = dict(
            "outer_sum_partial_kernel + outer_sum_reduce_kernel",
     desc="backward pass of the dense GRU Din=D=64, B={B}/GPU, T={T}, with the Jacobian's diagonal: "
          "dL/dP, dL/dh0, dL/dW_hh [3D, D], dL/db_hh from the converged states and dL/dh",
-    cpu_sample=dict(B=16, T=32768), ref_sample=dict(B=4, T=4096))
+    cpu_sample=dict(B=16, T=32768), ref_sample=dict(B=4, T=16384))
 ADJ_METRIC = "backward states/sec (B*T*D per s, gradients through the evaluated sequence)"
 # the diagonal-recurrence LSTM (state (c, h) per lane; exact Newton over 2x2 lane
 # blocks): reads P 16 + the guess (c, h) 8, writes (c, h) 8 = 32 B per lane-step
@@ -107,7 +107,7 @@ BENCHES["lstm"] = dict(
     kernel="lstm_diag_kernel (persistent, all iterations)",
     desc="diagonal-recurrence LSTM Din=D=2048, B={B}/GPU, T={T}, bf16 x and W_ih, fp32 state (c, h), "
          "exact Newton (2x2 lane Jacobians) tol 1e-4",
-    cpu_sample=dict(B=1, T=8192), ref_sample=dict(B=1, T=64))
+    cpu_sample=dict(B=1, T=8192), ref_sample=dict(B=1, T=1024))
 # fp32 FMA peak for the ALU-bound row: 148 SMs x 128 fp32 lanes x 2 flop x
 # 1965 MHz (the part's maximum SM clock), in TFLOP/s.
 ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
@@ -116,8 +116,8 @@ ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 # hash of the kernel source it was measured on.  Traffic grows with states x
 # iterations, so the full launch's is scaled from it; reported only while the
 # source is unchanged.
-NCU_TRAFFIC = {"bytes_per_state_iter": (4.053384e9 + 0.990802e9) / (14 * 16 * 16384 * 64),
-               "source_sha1": "e48aa98c7598"}
+NCU_TRAFFIC = {"bytes_per_state_iter": (4.193761e9 + 0.992682e9) / (14 * 16 * 16384 * 64),
+               "source_sha1": "93248604af25"}
 
 
 def log(*a):
