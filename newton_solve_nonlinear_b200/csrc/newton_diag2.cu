@@ -264,6 +264,20 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
             atomicMax(&hdr->resid_bits[it % 3], br);
             if (*cta_err) flag_timeout(status);
         }
+        // P of the next iteration's first two tiles into L2 while the grid meets:
+        // one 256-byte row segment (gate, step) per thread
+        if (tid < 2 * 3 * TS) {
+            const int q = tid / (3 * TS), g = (tid / TS) % 3, r = tid % TS;
+            if (q < my_n) {
+                int chunk, b, dg;
+                long long row0;
+                tile_pos(S, blockIdx.x + static_cast<long long>(q) * nblocks, T, chunk, b, dg, row0);
+                if (chunk * TS + r < T) {
+                    const float *src = A.P + (row0 + r) * 3 * D + g * D + dg * DL;
+                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], 256;" ::"l"(src) : "memory");
+                }
+            }
+        }
         grid_barrier(hdr->barrier, nblocks, status);
         last_delta = ld_acquire_u32(&hdr->delta_bits[it % 3]);
         last_resid = ld_acquire_u32(&hdr->resid_bits[it % 3]);
