@@ -80,3 +80,38 @@ def test_invalid_arguments_are_rejected_without_a_gpu(L):
     assert rc == 3
     rc = L.pararnn_affine_scan(None, None, None, 1, 10, 8, 0, None, None, 0, None)
     assert rc == 3
+
+
+def _al(n):
+    return (n + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("B,parts,largest", [(16, 7, 4), (16, 6, 4), (16, 1, 16), (8, 7, 2), (5, 5, 1), (4, 3, 2)])
+def test_host_pipeline_part_sizes(L, B, parts, largest):
+    """The host-buffer solve ramps its parts (weights 1, 2, 3, 4, ..., 4, 3, 2, 1,
+    largest remainder, at least one sequence each); its workspace is one solve
+    workspace for the largest part, three staging buffers (fewer when there are
+    fewer parts) of that part's x and h, h0 for the batch and one report per part."""
+    T, din, d = 1000, 64, 64
+    cell = binding.make_cell("dense", din, d, binding.torch.float32)
+    m = binding.MODES["QUASI"]
+    solve = L.pararnn_workspace_size(ctypes.byref(cell), largest, T, m)
+    nbuf = min(parts, 3)
+    want = (_al(solve) + nbuf * _al(largest * T * din * 4) + nbuf * _al(largest * T * d * 4) + _al(B * d * 4)
+            + _al(parts * 16))
+    assert L.pararnn_host_workspace_size(ctypes.byref(cell), B, T, m, parts) == want
+    assert L.pararnn_host_workspace_size(ctypes.byref(cell), B, T, m, B + 1) == 0
+
+
+def test_reuse_and_adjoint_size_queries(L):
+    dense32 = binding.make_cell("dense", 16, 32, binding.torch.float32)
+    dense64 = binding.make_cell("dense", 64, 64, binding.torch.float32)
+    m = binding.MODES["DEER"]
+    assert L.pararnn_reuse_workspace_size(ctypes.byref(dense32), 4, 1000) == \
+        L.pararnn_workspace_size(ctypes.byref(dense32), 4, 1000, m) + _al(4 * 1000 * 512)
+    assert L.pararnn_reuse_workspace_size(ctypes.byref(dense64), 4, 1000) == 0
+    assert L.pararnn_adjoint_workspace_size(ctypes.byref(dense64), 2, 100) > 0
+    assert L.pararnn_adjoint_workspace_size(ctypes.byref(binding.make_cell("dense", 65, 65, binding.torch.float32)),
+                                            2, 100) == 0
+    assert L.pararnn_adjoint_host_workspace_size(ctypes.byref(dense64), 4, 100, 3) > 0
+    assert L.pararnn_adjoint_host_workspace_size(ctypes.byref(dense64), 4, 100, 5) == 0
