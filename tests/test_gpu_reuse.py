@@ -19,6 +19,14 @@ from newton_solve_nonlinear_b200.inputs import make_workload
 pytestmark = pytest.mark.gpu
 
 
+def _same_run(a, b, atol=1e-6):
+    """Two launches of the same solve agree to within fp32 rounding: the
+    decoupled look-back composes the later tiles' maps in an order set by
+    timing (how far back the first finished prefix lies), so the last bits
+    may differ from one launch to the next."""
+    return float((a.double().cpu() - b.double().cpu()).abs().max()) <= atol
+
+
 def _make(name, over):
     kw = {k: over[k] for k in ("bias_std", "h0_std") if k in over}
     return make_workload(name, **{k: v for k, v in over.items() if k not in kw}, **kw)
@@ -79,8 +87,8 @@ def test_period_one_is_plain_deer_and_arguments_checked():
     r1 = binding.solve_workload(w, "DEER", jac_every=1)
     r2 = binding.solve_workload(w, "DEER", jac_every=2)
     r3 = binding.solve_workload(w, "DEER", jac_every=2)
-    assert torch.equal(r0.h, r1.h) and r0.iters == r1.iters
-    assert torch.equal(r2.h, r3.h) and r2.iters == r3.iters  # deterministic
+    assert r0.iters == r1.iters and _same_run(r0.h, r1.h)
+    assert r2.iters == r3.iters and _same_run(r2.h, r3.h)  # repeatable
     with pytest.raises(ValueError):
         binding.solve_workload(w, "QUASI", jac_every=2)
     cell = binding.make_cell("dense", 64, 64, torch.float32)
