@@ -107,7 +107,7 @@ BENCHES["lstm"] = dict(
     kernel="lstm_diag_kernel (persistent, all iterations)",
     desc="diagonal-recurrence LSTM Din=D=2048, B={B}/GPU, T={T}, bf16 x and W_ih, fp32 state (c, h), "
          "exact Newton (2x2 lane Jacobians) tol 1e-4",
-    cpu_sample=dict(B=1, T=8192), ref_sample=dict(B=1, T=1024))
+    cpu_sample=dict(B=1, T=8192), ref_sample=dict(B=1, T=1024), roll_sample=dict(T=256))
 # fp32 FMA peak for the ALU-bound row: 148 SMs x 128 fp32 lanes x 2 flop x
 # 1965 MHz (the part's maximum SM clock), in TFLOP/s.
 ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
@@ -278,9 +278,20 @@ def cpu_rollout_baseline(spec: dict) -> dict | None:
     sample = spec.get("roll_sample")
     if sample is None:
         return None
-    w = make_workload(spec["workload"], **sample)
-    c = GRU.from_workload(w)
-    x, h0 = w.x.double().numpy(), w.h0.double().numpy()
+    if spec["mode"] == "LSTM":  # the diagonal LSTM: (c, h) per lane
+        from oracle.lstm import LSTM
+        from newton_solve_nonlinear_b200.inputs import make_lstm_workload
+        w = make_lstm_workload(**sample)
+        c = LSTM(w_ih=w.w_ih.double().numpy(), b_ih=w.b_ih.double().numpy(), u=w.u.double().numpy(),
+                 b_hh=w.b_hh.double().numpy())
+        x, c0, h0 = w.x.double().numpy(), w.c0.double().numpy(), w.h0.double().numpy()
+        roll = lambda xx, cc, hh, dt, thr: crollout.lstm_rollout(c, xx, cc, hh, dt, threads=thr)
+    else:
+        w = make_workload(spec["workload"], **sample)
+        c = GRU.from_workload(w)
+        x, h0 = w.x.double().numpy(), w.h0.double().numpy()
+        c0 = h0
+        roll = lambda xx, cc, hh, dt, thr: crollout.rollout(c, xx, hh, dt, threads=thr)
     states = w.B * w.T * w.d
     nthr = min(crollout.max_threads(), w.B)
     out = {"unit": UNIT, "cores": os.cpu_count(), "threads": nthr, "cpu": cpu_model(),
@@ -288,10 +299,10 @@ def cpu_rollout_baseline(spec: dict) -> dict | None:
                      f"on one thread (sequential rollout, gcc -O3 -fopenmp)"}
     for name, dt in (("fp64", np.float64), ("fp32", np.float32)):
         t0 = time.perf_counter()
-        crollout.rollout(c, x, h0, dt, threads=nthr)
+        roll(x, c0, h0, dt, nthr)
         out[name] = states / (time.perf_counter() - t0)
         t0 = time.perf_counter()
-        crollout.rollout(c, x[:1], h0[:1], dt, threads=1)
+        roll(x[:1], c0[:1], h0[:1], dt, 1)
         out[name + "_1thread"] = states / w.B / (time.perf_counter() - t0)
     return out
 
@@ -511,6 +522,7 @@ def run_lstm(args):
     torch.cuda.synchronize()
     e2e_value = job_value(states, e2e_steps, world, max_over_ranks(ea.elapsed_time(eb), dev))
     cpu = cpu_baseline_oracle(spec, spec["cpu_sample"]) if rank == 0 and world == 1 else None
+    roll = cpu_rollout_baseline(spec) if rank == 0 and world == 1 else None
     hbm_peak, peak_kind = peaks()
     avg_s = statistics.mean(ms) / 1e3
     achieved = res.iters * states * spec["per_state"] / avg_s / 1e9
@@ -537,6 +549,8 @@ def run_lstm(args):
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
+    if roll is not None:
+        line["cpu_rollout"] = roll
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -40,6 +40,11 @@ def lib() -> ctypes.CDLL:
             p = ctypes.POINTER(real)
             f.argtypes = [p, p, p, p, p, p] + [ctypes.c_int] * 5 + [p, ctypes.c_int]
             f.restype = ctypes.c_int
+        for name, real in (("lstm_rollout_f64", ctypes.c_double), ("lstm_rollout_f32", ctypes.c_float)):
+            f = getattr(L, name)
+            p = ctypes.POINTER(real)
+            f.argtypes = [p] * 7 + [ctypes.c_int] * 4 + [p, p, ctypes.c_int]
+            f.restype = ctypes.c_int
         L.rollout_max_threads.restype = ctypes.c_int
         _lib = L
     return _lib
@@ -66,3 +71,23 @@ def rollout(cell: GRU, x: np.ndarray, h0: np.ndarray, dtype=np.float64, threads:
     if rc != 0:
         raise RuntimeError("gru_rollout failed")
     return h
+
+
+def lstm_rollout(cell, x: np.ndarray, c0: np.ndarray, h0: np.ndarray, dtype=np.float64, threads: int = 0):
+    """(c, h) [B, T, D] of the diagonal LSTM's sequential evaluation in `dtype`
+    (``cell``: oracle.lstm.LSTM)."""
+    dtype = np.dtype(dtype)
+    real = ctypes.c_double if dtype == np.float64 else ctypes.c_float
+    fn = lib().lstm_rollout_f64 if dtype == np.float64 else lib().lstm_rollout_f32
+    arr = lambda a: np.ascontiguousarray(a, dtype=dtype)
+    x_, wi, bi, u, bh, c0_, h0_ = map(arr, (x, cell.w_ih, cell.b_ih, cell.u, cell.b_hh, c0, h0))
+    B, T, din = x_.shape
+    d = cell.d
+    c = np.empty((B, T, d), dtype=dtype)
+    h = np.empty((B, T, d), dtype=dtype)
+    ptr = lambda a: a.ctypes.data_as(ctypes.POINTER(real))
+    rc = fn(ptr(x_), ptr(wi), ptr(bi), ptr(u), ptr(bh), ptr(c0_), ptr(h0_), B, T, din, d, ptr(c), ptr(h),
+            int(threads))
+    if rc != 0:
+        raise RuntimeError("lstm_rollout failed")
+    return c, h

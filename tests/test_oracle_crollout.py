@@ -26,3 +26,19 @@ def test_c_rollout_equals_oracle(kind, B, T, din, d):
     assert got32.dtype == np.float32
     assert np.max(np.abs(got32 - want)) <= 1e-4
     assert crollout.max_threads() >= 1
+
+
+def test_c_lstm_rollout_equals_oracle():
+    from oracle.lstm import LSTM, lstm_rollout
+    rng = np.random.default_rng(3)
+    din, d, B, T = 5, 6, 3, 150
+    cell = LSTM(w_ih=rng.normal(0, 0.5, (4 * d, din)), b_ih=rng.normal(0, 0.3, 4 * d), u=rng.uniform(-1, 1, 4 * d),
+                b_hh=rng.normal(0, 0.3, 4 * d))
+    x = rng.normal(size=(B, T, din))
+    c0, h0 = rng.normal(0, 0.5, (B, d)), rng.normal(0, 0.5, (B, d))
+    cw, hw = lstm_rollout(cell, x, c0, h0)
+    c, h = crollout.lstm_rollout(cell, x, c0, h0, np.float64, threads=2)
+    np.testing.assert_allclose(c, cw, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(h, hw, rtol=0, atol=1e-12)
+    c32, h32 = crollout.lstm_rollout(cell, x, c0, h0, np.float32, threads=1)
+    assert max(np.max(np.abs(c32 - cw)), np.max(np.abs(h32 - hw))) <= 1e-4
