@@ -100,6 +100,7 @@ BENCHES["adjoint_dense"] = dict(
          "dL/dP, dL/dh0, dL/dW_hh [3D, D], dL/db_hh from the converged states and dL/dh",
     cpu_sample=dict(B=16, T=32768), ref_sample=dict(B=4, T=16384))
 ADJ_METRIC = "backward states/sec (B*T*D per s, gradients through the evaluated sequence)"
+SCAN_METRIC = "affine-scan elements/sec (B*T*D per s, h_t = a_t h_(t-1) + b_t)"
 # the diagonal-recurrence LSTM (state (c, h) per lane; exact Newton over 2x2 lane
 # blocks): reads P 16 + the guess (c, h) 8, writes (c, h) 8 = 32 B per lane-step
 BENCHES["lstm"] = dict(
@@ -321,6 +322,8 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
+    if args.workload == "scan":
+        return run_reference_scan(args)
     spec = BENCHES[args.workload]
     steps = []
     base = None
@@ -342,6 +345,33 @@ def run_reference(args):
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": base["cores"], "kind": "oracle",
                              "sample": base["sample"]},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_reference_scan(args):
+    """The oracle's serial fp64 scan on a bounded sample of the scan workload."""
+    import numpy as np
+    from oracle.scan import affine_scan
+    from newton_solve_nonlinear_b200.inputs import make_scan_input
+    B, T, D = 2, (args.T or 65536), 64
+    s = make_scan_input(B, T, D, seed=0)
+    A, b, h0 = s.A.double().numpy(), s.b.double().numpy(), s.h0.double().numpy()
+    vals = []
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        affine_scan(A, b, h0)
+        if i >= args.warmup:
+            vals.append(B * T * D / (time.perf_counter() - t0))
+    v = statistics.median(vals)
+    sample = f"fp64 numpy serial recurrence on B={B}, T={T}, D={D} (same distributions, one thread over t)"
+    line = {"impl": "reference", "metric": SCAN_METRIC, "value": v, "unit": "elements/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"affine scan alone h_t = a_t h_(t-1) + b_t, [B=16, T={T}, D=64], "
+                                   f"a ~ U(0.5, 1), b ~ N(0, 1), h0 = 0", "sample": sample},
+            "cpu_baseline": {"value": v, "unit": "elements/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": "elements/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -558,28 +588,40 @@ def run_lstm(args):
     return 0
 
 
-def run_ours(args):
+def _dist_setup():
+    """(world, rank, local rank, device, barrier) of this process; NCCL only when
+    launched as several ranks."""
     import torch
     import torch.distributed as dist
-    from newton_solve_nonlinear_b200 import binding
-    from newton_solve_nonlinear_b200.inputs import make_workload
-
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
+    if world > 1 and not dist.is_initialized():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
 
     def barrier():
         if world > 1:
             dist.barrier()
+    return world, rank, local, dev, barrier
 
-    spec = BENCHES[args.workload]
+
+def bench_solve(args, name: str, *, full: bool = True, steps: int | None = None):
+    """Time one solver family (projection + the whole Newton loop per step) and
+    return its JSON line.  ``full`` adds the end-to-end (host buffers) number,
+    the CPU baselines and the clock record; the per-family entries of the
+    default run's ``workloads`` key leave those out."""
+    import torch
+    from newton_solve_nonlinear_b200 import binding
+    from newton_solve_nonlinear_b200.inputs import make_workload
+
+    world, rank, local, dev, barrier = _dist_setup()
+    steps = args.steps if steps is None else steps
+    spec = BENCHES[name]
     mode, lam = spec["mode"], spec["lam"]
-    over = {"T": args.T} if args.T else {}
+    over = {"T": args.T} if (args.T and name == args.workload) else {}
     w = make_workload(spec["workload"], seed=rank, **over)
     B, T, D, din, kind = w.B, w.T, w.d, w.din, w.kind
     states = B * T * D
@@ -589,17 +631,18 @@ def run_ours(args):
         binding.workspace_size(kind, din, D, B, T, mode, w.x_dtype), dev)
     P = torch.empty(B, T, 3 * D, dtype=torch.float32, device=dev)
     out = torch.empty(B, T, D, dtype=torch.float32, device=dev)
-    info = torch.zeros(4, dtype=torch.int32, device=dev)
+    # one report per timed step, read after the timed region
+    infos = torch.zeros(max(steps, 1) + 1, 4, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    k = args.jac_every
+    k = args.jac_every if name == args.workload else 1
     if k != 1:
         if mode != "DEER":
             raise SystemExit("--jac-every needs a DEER workload")
         ws = binding.alloc_workspace(binding.lib().pararnn_reuse_workspace_size(
             binding.make_cell(kind, din, D, w.x_dtype), B, T), dev)
 
-    def step(ev_mid=None):
+    def step(info, ev_mid=None):
         if k != 1:  # one synchronous call: projection and the solve with the Jacobian reused
             if ev_mid is not None:
                 ev_mid.record(stream)
@@ -614,66 +657,82 @@ def run_ours(args):
                                tol=w.tol, info_dev=info, out=out, workspace=ws, dtype=w.x_dtype)
 
     for _ in range(args.warmup):
-        step()
+        step(infos[-1])
     torch.cuda.synchronize()
-    iters, status = int(info[0]), int(info[1])
-    if status != 0:
-        log(f"warning: solve status {binding.STATUS.get(status)} after {iters} iterations")
 
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    with Clocks(local) as clk:
-        barrier()
-        torch.cuda.synchronize()
-        for e0, e1, e2 in evs:
-            e0.record(stream)
-            step(e1)
-            e2.record(stream)
-        torch.cuda.synchronize()
-        barrier()
+            torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    clk = Clocks(local) if full else None
+    if clk is not None:
+        clk.__enter__()
+    barrier()
+    torch.cuda.synchronize()
+    for i, (e0, e1, e2) in enumerate(evs):
+        e0.record(stream)
+        step(infos[i], e1)
+        e2.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    if clk is not None:
+        clk.__exit__(None, None, None)
     total_ms = sum(e0.elapsed_time(e2) for e0, _, e2 in evs)
     solver_ms = [e1.elapsed_time(e2) for _, e1, e2 in evs]
     proj_ms = [e0.elapsed_time(e1) for e0, e1, _ in evs]
     max_ms = max_over_ranks(total_ms, dev)
-    value = job_value(states, args.steps, world, max_ms)
+    value = job_value(states, steps, world, max_ms)
+    # the timed solves' own reports: every one must have converged, and the
+    # iteration count the roofline uses is theirs
+    rep = infos[:steps].cpu()
+    step_iters = [int(v) for v in rep[:, 0]]
+    step_status = [binding.STATUS.get(int(v), str(int(v))) for v in rep[:, 1]]
+    if any(st != "OK" for st in step_status):
+        raise SystemExit(f"{name}: a timed solve did not converge: iterations {step_iters}, "
+                         f"statuses {step_status}")
+    iters = max(step_iters)
 
-    # end to end through the public host-buffer call: page-locked x and h0 in,
-    # h out; the library splits the batch into parts and overlaps the copies
-    x_host = w.x.contiguous().pin_memory()
-    h0_host = w.h0.float().contiguous().pin_memory()
-    h_host = torch.empty(B, T, D, dtype=torch.float32).pin_memory()
-    parts = max(1, min(E2E_PARTS, B))
-    if k != 1:
-        parts = 1
-    ws_host = binding.alloc_workspace(
-        binding.host_workspace_size(kind, din, D, B, T, mode, parts, w.x_dtype), dev)
-    e2e_steps = max(1, min(args.steps, 5))
+    e2e = None
+    parts = max(1, min(E2E_PARTS, B)) if k == 1 else 1
+    if full:
+        # end to end through the public host-buffer call: page-locked x and h0 in,
+        # h out; the library splits the batch into parts and overlaps the copies
+        x_host = w.x.contiguous().pin_memory()
+        h0_host = w.h0.float().contiguous().pin_memory()
+        h_host = torch.empty(B, T, D, dtype=torch.float32).pin_memory()
+        ws_host = binding.alloc_workspace(
+            binding.host_workspace_size(kind, din, D, B, T, mode, parts, w.x_dtype), dev)
+        e2e_steps = max(1, min(steps, 5))
 
-    def e2e_step():
-        if k != 1:  # copies around the reuse solve (no host-buffer variant of it)
-            x.copy_(x_host, non_blocking=True)
-            h0.copy_(h0_host, non_blocking=True)
-            binding.newton_solve(w_ih, b_ih, w_hh, b_hh, x, h0, kind=kind, mode=mode, tol=w.tol,
-                                 jac_every=k, out=out, workspace=ws, stream=stream)
-            h_host.copy_(out, non_blocking=True)
-            return
-        return binding.newton_solve_host(w_ih, b_ih, w_hh, b_hh, x_host, h0_host, kind=kind,
-                                         mode=mode, lam=lam, tol=w.tol, parts=parts, out=h_host,
-                                         workspace=ws_host, stream=stream)
+        def e2e_step():
+            if k != 1:  # copies around the reuse solve (no host-buffer variant of it)
+                x.copy_(x_host, non_blocking=True)
+                h0.copy_(h0_host, non_blocking=True)
+                binding.newton_solve(w_ih, b_ih, w_hh, b_hh, x, h0, kind=kind, mode=mode, tol=w.tol,
+                                     jac_every=k, out=out, workspace=ws, stream=stream)
+                h_host.copy_(out, non_blocking=True)
+                return None
+            return binding.newton_solve_host(w_ih, b_ih, w_hh, b_hh, x_host, h0_host, kind=kind,
+                                             mode=mode, lam=lam, tol=w.tol, parts=parts, out=h_host,
+                                             workspace=ws_host, stream=stream)
 
-    e2e_step()
-    barrier()
-    torch.cuda.synchronize()
-    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ea.record(stream)
-    for _ in range(e2e_steps):
         e2e_step()
-    eb.record(stream)
-    torch.cuda.synchronize()
-    e2e_value = job_value(states, e2e_steps, world, max_over_ranks(ea.elapsed_time(eb), dev))
+        barrier()
+        torch.cuda.synchronize()
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ea.record(stream)
+        for _ in range(e2e_steps):
+            r = e2e_step()
+            if r is not None and r.status != "OK":
+                raise SystemExit(f"{name}: end-to-end solve status {r.status}")
+        eb.record(stream)
+        torch.cuda.synchronize()
+        e2e = {"value": job_value(states, e2e_steps, world, max_over_ranks(ea.elapsed_time(eb), dev)),
+               "unit": UNIT,
+               "h2d_bytes_per_step": x_host.numel() * x_host.element_size() + h0_host.numel() * 4,
+               "d2h_bytes_per_step": h_host.numel() * 4 + 16 * parts, "parts": parts}
+        del ws_host
 
     cpu = roll = None
-    if rank == 0 and world == 1:
+    if full and rank == 0 and world == 1:
         cpu = cpu_baseline_oracle(spec, spec["cpu_sample"], k)
         roll = cpu_rollout_baseline(spec)
 
@@ -686,7 +745,7 @@ def run_ours(args):
         peak, unit = hbm_peak, "GB/s"
         algo = f"{per_state} B/state/iteration x {iters} iterations x {states} states"
         pk = f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
-        if args.workload == "untrained" and NCU_TRAFFIC["source_sha1"] == kernel_sha():
+        if name == "untrained" and NCU_TRAFFIC["source_sha1"] == kernel_sha():
             traffic = NCU_TRAFFIC["bytes_per_state_iter"] * iters * states
     elif spec["bound"] == "tensor":
         per_state = 2 * D * D
@@ -704,14 +763,14 @@ def run_ours(args):
         algo = f"14 D^3 flop/step = {per_state} flop/state/iteration x {iters} x {states} states"
         pk = "fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1965 MHz"
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": spec["desc"].format(B=B, T=T), "name": args.workload,
+        "config": {"workload": spec["desc"].format(B=B, T=T), "name": name,
                    "B": B, "T": T, "D": D, "din": din, "cell": kind, "mode": mode,
                    "lambda": lam if mode in ("ELK", "QUASI_ELK") else None,
                    "jac_every": k,
-                   "tol": w.tol, "iters": iters, "status": binding.STATUS.get(status),
+                   "tol": w.tol, "iters": iters, "status": "OK", "iters_per_step": step_iters,
                    "l2": (f"inputs larger than L2 (126 MB) summed per solve: "
                           f"x {x.numel() * x.element_size() / 1e6:.0f} MB, "
                           f"P {P.numel() * 4 / 1e6:.0f} MB, h {out.numel() * 4 / 1e6:.0f} MB"),
@@ -721,21 +780,152 @@ def run_ours(args):
         "roofline": {"bound": spec["bound"], "achieved": achieved, "peak": peak, "unit": unit,
                      "frac": achieved / peak, "traffic": traffic, "kernel": spec["kernel"],
                      "algorithmic": algo, "peak_kind": pk},
-        "e2e": {"value": e2e_value, "unit": UNIT,
-                "h2d_bytes_per_step": x_host.numel() * x_host.element_size() + h0_host.numel() * 4,
-                "d2h_bytes_per_step": h_host.numel() * 4 + 16 * parts, "parts": parts},
-        "gpu_launches": 2 * args.steps,
-        "clocks": clk.summary(),
+        "gpu_launches": 2 * steps,
     }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if clk is not None:
+        line["clocks"] = clk.summary()
     if cpu is not None:
         line["cpu_baseline"] = cpu
     if roll is not None:
         line["cpu_rollout"] = roll
+    del ws, P, out
+    torch.cuda.empty_cache()
+    return line
+
+
+def bench_scan(args, *, steps: int | None = None, full: bool = False):
+    """The affine scan alone (pararnn_affine_scan, diagonal): [16, 65536, 64],
+    a ~ U(0.5, 1), b ~ N(0, 1), h0 = 0; 12 B per element (a, b in, h out)."""
+    import torch
+    from newton_solve_nonlinear_b200 import binding
+    from newton_solve_nonlinear_b200.inputs import make_scan_input
+
+    world, rank, local, dev, barrier = _dist_setup()
+    steps = args.steps if steps is None else steps
+    B, T, D = 16, (args.T if (args.T and args.workload == "scan") else 65536), 64
+    s = make_scan_input(B, T, D, seed=rank)
+    A, b, h0 = s.A.to(dev), s.b.to(dev), s.h0.to(dev)
+    ws = binding.alloc_workspace(int(binding.lib().pararnn_affine_scan_workspace_size(B, T, D, 0)), dev)
+    h = torch.empty_like(b)
+    stream = torch.cuda.current_stream(dev)
+    run = lambda: binding.affine_scan(A, b, h0, out=h, workspace=ws, stream=stream)
+    for _ in range(args.warmup):
+        run()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    clk = Clocks(local) if full else None
+    if clk is not None:
+        clk.__enter__()
+    barrier()
+    torch.cuda.synchronize()
+    for e0, e1 in evs:
+        e0.record(stream)
+        run()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    if clk is not None:
+        clk.__exit__(None, None, None)
+    st = binding.lib().pararnn_affine_scan_status(ws.data_ptr(), stream.cuda_stream)
+    if st != 0:
+        raise SystemExit(f"scan: status {binding.STATUS.get(st, st)}")
+    ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    max_ms = max_over_ranks(sum(ms), dev)
+    n = B * T * D
+    value = job_value(n, steps, world, max_ms)
+    hbm_peak, peak_kind = peaks()
+    achieved = n * 12 / (statistics.mean(ms) / 1e3) / 1e9
+    line = {
+        "metric": SCAN_METRIC, "value": value, "unit": "elements/s", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"affine scan alone h_t = a_t h_(t-1) + b_t, [B={B}, T={T}, D={D}], "
+                               f"a ~ U(0.5, 1), b ~ N(0, 1), h0 = 0", "name": "scan", "B": B, "T": T, "D": D,
+                   "l2": f"inputs larger than L2 (126 MB): a, b {2 * n * 4 / 1e6:.0f} MB, h {n * 4 / 1e6:.0f} MB",
+                   "parallelism": f"replicas over sequences x{world}"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "traffic": None, "kernel": "scan_diag_kernel (one pass)",
+                     "algorithmic": f"12 B/element x {n} elements",
+                     "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"},
+        "gpu_launches": steps,
+    }
+    if full:
+        # end to end: a, b, h0 from page-locked host memory, h back, around the same call
+        hA, hb, hh0 = s.A.pin_memory(), s.b.pin_memory(), s.h0.pin_memory()
+        hh = torch.empty(B, T, D).pin_memory()
+        e2e_steps = max(1, min(steps, 5))
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        ea.record(stream)
+        for _ in range(e2e_steps):
+            A.copy_(hA, non_blocking=True)
+            b.copy_(hb, non_blocking=True)
+            h0.copy_(hh0, non_blocking=True)
+            run()
+            hh.copy_(h, non_blocking=True)
+        eb.record(stream)
+        torch.cuda.synchronize()
+        line["e2e"] = {"value": job_value(n, e2e_steps, world, max_over_ranks(ea.elapsed_time(eb), dev)),
+                       "unit": "elements/s", "h2d_bytes_per_step": (2 * n + B * D) * 4, "d2h_bytes_per_step": n * 4}
+        line["clocks"] = clk.summary()
+    del ws, h, A, b
+    torch.cuda.empty_cache()
+    return line
+
+
+# The default run also times these families on the same box, a few steps each,
+# and reports them under "workloads" (value, roofline, iterations).
+SIDE_FAMILIES = ("diag", "dense_deer", "quasi_elk", "elk")
+
+
+def _summary(line: dict) -> dict:
+    rf = line["roofline"]
+    c = line["config"]
+    return {"value": line["value"], "unit": line["unit"], "ms_per_step": line["ms_per_step"],
+            "steps": line["steps"], "iters": c.get("iters"), "status": c.get("status", "OK"),
+            "workload": c["workload"],
+            "roofline": {"bound": rf["bound"], "achieved": rf["achieved"], "peak": rf["peak"], "unit": rf["unit"],
+                         "frac": rf["frac"], "kernel": rf["kernel"], "algorithmic": rf["algorithmic"]}}
+
+
+def run_ours(args):
+    import torch.distributed as dist
+    world, rank = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0"))
+    if args.workload == "scan":
+        line = bench_scan(args, full=True)
+    else:
+        line = bench_solve(args, args.workload)
+    if args.workload == "untrained" and not args.no_side and args.jac_every == 1 and not args.T:
+        side = {}
+        for name in SIDE_FAMILIES:
+            side[name] = _summary(bench_solve(args, name, full=False, steps=min(args.steps, 5)))
+        side["scan"] = _summary(bench_scan(args, steps=min(args.steps, 10)))
+        line["workloads"] = side
+        line["gpu_launches"] += sum(2 * v["steps"] for k, v in side.items() if k != "scan") + side["scan"]["steps"]
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
+    if world > 1 and dist.is_initialized():
         dist.destroy_process_group()
     return 0
+
+
+def plan_launch(gpus: int, env: dict, argv: list[str]):
+    """How bench.py runs for --gpus N: ("run", None) in this process,
+    ("exec", cmd) re-launched under torchrun with one rank per GPU, or
+    ("error", why) when an outer launcher started a different rank count."""
+    world = env.get("WORLD_SIZE")
+    if world is None:
+        if gpus <= 1:
+            return "run", None
+        port = env.get("MASTER_PORT") or "29517"
+        cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+               "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+        return "exec", cmd
+    if int(world) != gpus:
+        return "error", f"--gpus {gpus} but WORLD_SIZE={world}"
+    return "run", None
 
 
 def main():
@@ -744,20 +934,29 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="untrained", choices=sorted(BENCHES),
+    ap.add_argument("--workload", default="untrained", choices=sorted(BENCHES) + ["scan"],
                     help="which solve to time (default: the untrained dense GRU headline)")
     ap.add_argument("--T", type=int, default=0, help="override the sequence length")
     ap.add_argument("--jac-every", type=int, default=1,
                     help="DEER workloads: recompute the Jacobian only every k iterations")
+    ap.add_argument("--no-side", action="store_true",
+                    help="default workload: skip the other families' entries under \"workloads\"")
     args = ap.parse_args()
+    how, what = plan_launch(args.gpus, dict(os.environ), sys.argv[1:])
+    if how == "error":
+        log(what)
+        return 2
+    if how == "exec":
+        log("launching: " + " ".join(what))
+        return subprocess.call(what)
     if args.warmup < 3:
         log("warmup raised to 3 (timing rule)")
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
-    if BENCHES[args.workload]["mode"] == "ADJOINT":
+    if args.workload != "scan" and BENCHES[args.workload]["mode"] == "ADJOINT":
         return run_adjoint(args)
-    if BENCHES[args.workload]["mode"] == "LSTM":
+    if args.workload != "scan" and BENCHES[args.workload]["mode"] == "LSTM":
         return run_lstm(args)
     return run_ours(args)
 

@@ -200,6 +200,49 @@ PARARNN_API int pararnn_newton_solve_guess_async(const pararnn_cell *cell, const
                                                  size_t ws_bytes, pararnn_stream stream);
 
 /*
+ * pararnn_newton_solve_trace -- pararnn_newton_solve that also records every
+ * iteration's convergence maxima, so a caller can follow the whole trajectory
+ * of the stopping test rather than its last value: the per-iteration max|dh|
+ * whose first value <= tol ends the solve ("ParaRNN" summary, "Newton's
+ * Iteration"; "Towards Scalable and Stable Parallelization of Nonlinear RNNs",
+ * atlas summary "Limitations": the quasi methods take more iterations).
+ *   trace      DEVICE float [trace_len][2], 8-byte aligned, not overlapping h
+ *              or the workspace: trace[i][0] = max_{b,t,d} |h^(i+1) - h^(i)|,
+ *              trace[i][1] = max |h^(i)_t - f(h^(i)_{t-1}, x_t)| at iteration
+ *              i's linearisation point, for i < min(iters, trace_len); later
+ *              entries are left untouched.
+ *   trace_len  >= 1.
+ * Other arguments, the stopping rule and the return value as
+ * pararnn_newton_solve (synchronises `stream` once).
+ */
+PARARNN_API int pararnn_newton_solve_trace(const pararnn_cell *cell, const pararnn_params *params,
+                                           const void *x, const float *h0, int B, int T, int mode,
+                                           float lambda, float tol, int max_iters, float *h,
+                                           pararnn_info *info, float *trace, int trace_len,
+                                           void *workspace, size_t ws_bytes, pararnn_stream stream);
+
+/*
+ * pararnn_test_withheld_publish -- a testing hook for the bounded device-side
+ * waits (no counterpart on the pages).  It runs pararnn_newton_solve (tol,
+ * max_iters = T + 1) with one change: in the first iteration, look-back tile
+ * `tile` of the single-pass scan never publishes its descriptors, so every
+ * later tile of its lanes waits for a value that never arrives.  Those waits
+ * give up after their fixed spin budget (seconds), raise the workspace's
+ * timeout flag, and every CTA then leaves its waits and the grid barrier: the
+ * call returns PARARNN_TIMEOUT, h is unreliable, and the workspace is fit for
+ * the next solve (its header is rewritten by every solve).
+ * Taken by two paths only: the dense cell with d = 32 or 64 in mode QUASI (the
+ * tensor-core kernel; tiles of 128 steps x all lanes, chunk-major: tile =
+ * chunk * B + b), and the diagonal cell with d % 64 == 0 in mode DEER or QUASI
+ * (tiles of 32 steps x 64 lanes).  Other arguments, or a tile beyond the
+ * path's tile count, give PARARNN_INVALID_ARG.  Synchronises `stream`.
+ */
+PARARNN_API int pararnn_test_withheld_publish(const pararnn_cell *cell, const pararnn_params *params,
+                                              const void *x, const float *h0, int B, int T, int mode,
+                                              float tol, float *h, pararnn_info *info, long long tile,
+                                              void *workspace, size_t ws_bytes, pararnn_stream stream);
+
+/*
  * pararnn_newton_solve_reuse -- DEER on the dense cell with the Jacobian reused:
  * recomputed only every jac_every iterations, an approximate Newton strategy
  * the pages name for cost at scale ("ParaRNN" summary, "Newton's Iteration").
@@ -346,7 +389,8 @@ PARARNN_API size_t pararnn_affine_scan_workspace_size(int B, int T, int D, int d
  *                         dense != 0: [B, T, D, D], row-major matrices.
  *   b      DEVICE float [B, T, D].
  *   h0     DEVICE float [B, D].
- *   h      DEVICE float [B, T, D], output.  May alias b (not A or h0).
+ *   h      DEVICE float [B, T, D], output.  May be b itself; must not
+ *          overlap b otherwise, nor A or h0.
  *   workspace  DEVICE, >= pararnn_affine_scan_workspace_size(B, T, D, dense)
  *              bytes, 256-byte aligned.  Contents on entry do not matter.
  *   D must be a multiple of 4; dense needs D <= 64.
@@ -376,14 +420,22 @@ PARARNN_API int pararnn_affine_scan_status(const void *workspace, pararnn_stream
  * file-scope device array of 16 MiB inside this library, created when the
  * library's device code is loaded and held by every GPU that loads it until
  * the process exits.  No call allocates or frees anything.
- *   A, b, h0, h   as pararnn_affine_scan with dense == 0 (h may alias b).
+ *   A, b, h0, h   as pararnn_affine_scan with dense == 0, except that h may
+ *                 also be A itself (h may equal A or b exactly; any other
+ *                 overlap with A, b or h0 is rejected).
  *   status_dev    DEVICE unsigned, may be NULL: receives 0, or 1 if a bounded
  *                 device-side wait expired (result unreliable).
- * Limits: sizes whose scratch exceeds the array, i.e. 256 + 16 * L bytes with
- * L = (number of 64-lane, 64-step tiles) * min(D, 64) > 16 MiB (about 2^24
- * elements of B*T*D for D >= 64), are rejected with PARARNN_INVALID_ARG.
- * The first call on each device looks the array's device address up with
- * that device current; make that first call before any stream capture.
+ * Limits: the scratch a size needs is pararnn_affine_scan_workspace_size(B, T,
+ * D, 0) bytes (a 256-byte header plus 16 bytes per lane of every look-back
+ * tile; a tile spans min(D, 64) lanes and 4 * 256 / (min(D, 64) / 4) steps,
+ * i.e. 64 steps for D >= 64).  Sizes needing more than 16 MiB -- about 2^24
+ * elements of B*T*D for D >= 64, e.g. [15, 65536, 64] is accepted and
+ * [16, 65536, 64] is not -- are rejected with PARARNN_INVALID_ARG.
+ * Every call made outside stream capture looks the array's device address up
+ * with the current device (so a device reset, which reloads the library's
+ * device code, is followed correctly); a call inside a capture reuses the
+ * address the last uncaptured call on that device found, so make one call on
+ * each device before capturing it (a captured first call returns CUDA_ERROR).
  * Every call shares the one array and overwrites it (the parts that must
  * start at zero are cleared on the stream first), so calls that overlap on
  * the GPU -- on different streams, or from different host threads -- race.

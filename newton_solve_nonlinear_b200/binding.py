@@ -29,7 +29,8 @@ EXPORTS = ("pararnn_workspace_size", "pararnn_newton_solve", "pararnn_newton_sol
            "pararnn_adjoint_status", "pararnn_newton_solve_guess_async", "pararnn_newton_solve_chunked",
            "pararnn_chunked_workspace_size", "pararnn_lstm_solve", "pararnn_lstm_workspace_size",
            "pararnn_newton_solve_reuse", "pararnn_reuse_workspace_size", "pararnn_lstm_solve_host",
-           "pararnn_lstm_host_workspace_size", "pararnn_adjoint_host", "pararnn_adjoint_host_workspace_size")
+           "pararnn_lstm_host_workspace_size", "pararnn_adjoint_host", "pararnn_adjoint_host_workspace_size",
+           "pararnn_newton_solve_trace", "pararnn_test_withheld_publish")
 
 
 class Cell(ctypes.Structure):
@@ -118,6 +119,12 @@ def lib() -> ctypes.CDLL:
         L.pararnn_adjoint_host.restype = ci
         L.pararnn_adjoint_host_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci, ci]
         L.pararnn_adjoint_host_workspace_size.restype = sz
+        L.pararnn_newton_solve_trace.argtypes = [ctypes.POINTER(Cell), ctypes.POINTER(Params), vp, vp, ci, ci, ci,
+                                                 cf, cf, ci, vp, ctypes.POINTER(Info), vp, ci, vp, sz, vp]
+        L.pararnn_newton_solve_trace.restype = ci
+        L.pararnn_test_withheld_publish.argtypes = [ctypes.POINTER(Cell), ctypes.POINTER(Params), vp, vp, ci, ci,
+                                                    ci, cf, vp, ctypes.POINTER(Info), ctypes.c_longlong, vp, sz, vp]
+        L.pararnn_test_withheld_publish.restype = ci
         L.pararnn_status_string.argtypes = [ci]
         L.pararnn_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -201,11 +208,13 @@ class SolveResult:
     status: str
     delta: float
     residual: float
+    trace: object = None  # [iters, 2] host tensor: max |dh| and max |r| per iteration (trace=True)
 
 
 def newton_solve(w_ih, b_ih, w_hh, b_hh, x, h0, *, kind: str, mode: str, tol: float,
                  lam: float = 0.0, max_iters: int = 0, out=None, workspace=None,
-                 stream=None, sync: bool = True, info_dev=None, h_init=None, jac_every: int = 1):
+                 stream=None, sync: bool = True, info_dev=None, h_init=None, jac_every: int = 1,
+                 trace: bool = False):
     """Evaluate the GRU over x [B, T, Din] with the chosen Newton mode.
 
     All tensors must be contiguous CUDA tensors (x and w_ih fp32 or bf16, the
@@ -214,7 +223,8 @@ def newton_solve(w_ih, b_ih, w_hh, b_hh, x, h0, *, kind: str, mode: str, tol: fl
     int32 CUDA tensor of 4 elements) and returns ``out``.  ``h_init`` [B, T, D]
     (fp32 CUDA) starts the iteration from that guess instead of zero.
     ``jac_every`` > 1 (mode DEER, dense cell, d <= 32) recomputes the Jacobian
-    only every jac_every iterations (synchronous; no h_init)."""
+    only every jac_every iterations (synchronous; no h_init).  ``trace`` (sync
+    only) also returns every iteration's max |dh| and max |r| (SolveResult.trace)."""
     B, T, din = x.shape
     d = h0.shape[1]
     cell = make_cell(kind, din, d, x.dtype)
@@ -267,6 +277,16 @@ def newton_solve(w_ih, b_ih, w_hh, b_hh, x, h0, *, kind: str, mode: str, tol: fl
         rep = info_dev.cpu()  # waits for the solve
         return SolveResult(out, int(rep[0]), STATUS[int(rep[1])], float(rep[2:3].view(torch.float32)),
                            float(rep[3:4].view(torch.float32)))
+    if sync and trace:
+        cap = int(max_iters) if max_iters > 0 else T + 1
+        tr = torch.full((cap, 2), float("nan"), dtype=torch.float32, device=x.device)
+        info = Info()
+        rc = L.pararnn_newton_solve_trace(*args, ctypes.byref(info), _dev(tr, "trace"), cap,
+                                          _dev(workspace, "workspace"), workspace.numel(), _stream(stream))
+        if rc in (3, 4):
+            raise RuntimeError(f"pararnn_newton_solve_trace: {L.pararnn_status_string(rc).decode()}")
+        return SolveResult(out, info.iters, STATUS[info.status], info.delta, info.residual,
+                           tr[:info.iters].cpu())
     if sync:
         info = Info()
         rc = L.pararnn_newton_solve(*args, ctypes.byref(info), _dev(workspace, "workspace"),
@@ -508,6 +528,33 @@ def solve_workload(w, mode: str, *, lam: float = 0.0, tol=None, max_iters: int =
     return newton_solve(dev(w.w_ih), dev(w.b_ih), dev(w.w_hh), dev(w.b_hh), dev(w.x), dev(w.h0),
                         kind=w.kind, mode=mode, tol=w.tol if tol is None else tol, lam=lam,
                         max_iters=max_iters, **kw)
+
+
+def withheld_publish(w, mode: str, tile: int, *, out=None, workspace=None, device="cuda",
+                     stream=None) -> SolveResult:
+    """The testing hook pararnn_test_withheld_publish on a ``inputs.Workload``:
+    the solve with look-back tile ``tile`` silent in the first iteration."""
+    dev = lambda t: t.to(device).contiguous()
+    x, h0 = dev(w.x), dev(w.h0)
+    B, T, din = x.shape
+    d = h0.shape[1]
+    cell = make_cell(w.kind, din, d, x.dtype)
+    L = lib()
+    m = MODES[mode]
+    need = int(L.pararnn_workspace_size(ctypes.byref(cell), B, T, m))
+    if workspace is None:
+        workspace = alloc_workspace(need, x.device)
+    if out is None:
+        out = torch.empty(B, T, d, dtype=torch.float32, device=x.device)
+    w_ih, b_ih, w_hh, b_hh = dev(w.w_ih), dev(w.b_ih), dev(w.w_hh), dev(w.b_hh)
+    params = Params(_dev(w_ih, "w_ih"), _dev(b_ih, "b_ih"), _dev(w_hh, "w_hh"), _dev(b_hh, "b_hh"))
+    info = Info()
+    rc = L.pararnn_test_withheld_publish(ctypes.byref(cell), ctypes.byref(params), _dev(x, "x"), _dev(h0, "h0"),
+                                         B, T, m, float(w.tol), _dev(out, "out"), ctypes.byref(info), int(tile),
+                                         _dev(workspace, "workspace"), workspace.numel(), _stream(stream))
+    if rc in (3, 4):
+        raise RuntimeError(f"pararnn_test_withheld_publish: {L.pararnn_status_string(rc).decode()}")
+    return SolveResult(out, info.iters, STATUS[info.status], info.delta, info.residual)
 
 
 def affine_scan(A, b, h0, *, out=None, workspace=None, stream=None, check: bool = False):

@@ -221,7 +221,8 @@ __device__ __forceinline__ float lookback_mobius(unsigned long long *desc, long 
 // publishes one).  Thread q = 0 publishes the tile's aggregate first and its
 // inclusive value last.  Returns the carry into the tile (carry0 when there
 // is no predecessor).  Waits are bounded: a descriptor that never arrives
-// reads as an inclusive 0 and raises the timeout flag.
+// reads as an inclusive 0 and raises the timeout flag.  `publish` false keeps
+// the tile's descriptors unwritten (a testing hook for those bounded waits).
 // The first window's descriptor words of coop_lookback, read ahead of time
 // (relaxed loads: words that are not ready yet are polled again as usual), so
 // that their round trip overlaps the caller's own work before the look-back.
@@ -251,14 +252,14 @@ template <int G, int R = 1, bool kPrefetched = false>
 __device__ __forceinline__ float coop_lookback(unsigned long long *desc, long long tile, long long step,
                                                int DG, int d, int q, unsigned epoch, float EA, float EB,
                                                int avail, float carry0, unsigned *status,
-                                               const LookbackWindow<R> *pre = nullptr) {
+                                               const LookbackWindow<R> *pre = nullptr, bool publish = true) {
     unsigned long long *mine = desc + (static_cast<size_t>(tile) * DG + d) * 2;
     const int lane = threadIdx.x & 31;
     const int gbase = lane & ~(G - 1);
     const unsigned gmask = G == 32 ? 0xffffffffu : (((1u << G) - 1u) << gbase);
     float hin = carry0;
     if (avail > 0) {  // the same for every thread of the CTA
-        if (q == 0) {
+        if (q == 0 && publish) {
             const unsigned tag = make_tag(epoch, kStateAgg);
             st_relaxed(mine + 1, pack_word(tag, EB));
             st_relaxed(mine, pack_word(tag, EA));
@@ -337,7 +338,7 @@ __device__ __forceinline__ float coop_lookback(unsigned long long *desc, long lo
             if (__all_sync(0xffffffffu, done)) break;
         }
     }
-    if (q == 0) st_relaxed(mine, pack_word(make_tag(epoch, kStateInc), fmaf(EA, hin, EB)));
+    if (q == 0 && publish) st_relaxed(mine, pack_word(make_tag(epoch, kStateInc), fmaf(EA, hin, EB)));
     return hin;
 }
 

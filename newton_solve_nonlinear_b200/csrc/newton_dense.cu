@@ -454,6 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_deer_kernel(DenseArgs S) {
         grid_barrier(hdr->barrier, nblocks, status);
         last_delta = ld_acquire_u32(&hdr->delta_bits[it % 3]);
         last_resid = ld_acquire_u32(&hdr->resid_bits[it % 3]);
+        record_trace(A, it, last_delta, last_resid);
         iters = it + 1;
         // a timeout another CTA raises may land between two threads' reads: decide once per CTA
         if (__syncthreads_or(timed_out(status))) { final_status = PARARNN_TIMEOUT; break; }

@@ -800,7 +800,8 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
                     EB = qb;
                 }
                 const float c0 = chunk == 0 ? __ldg(A.h0 + static_cast<size_t>(b) * D + d) : 0.f;
-                const float hin = coop_lookback<GL>(A.desc, tile, B, D, d, q, epoch, EA, EB, chunk, c0, status);
+                const float hin = coop_lookback<GL, 1, false>(A.desc, tile, B, D, d, q, epoch, EA, EB, chunk, c0, status,
+                                                    nullptr, publishes(A, tile, epoch));
                 if (q == 0) carry[d] = hin;
             }
             __syncthreads();
@@ -873,6 +874,7 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
         grid_barrier(hdr->barrier, nblocks, status);
         last_delta = ld_acquire_u32(&hdr->delta_bits[it % 3]);
         last_resid = ld_acquire_u32(&hdr->resid_bits[it % 3]);
+        record_trace(A, it, last_delta, last_resid);
         iters = it + 1;
         // a timeout another CTA raises may land between two threads' reads: decide once per CTA
         if (__syncthreads_or(*cta_err || timed_out(status))) { final_status = PARARNN_TIMEOUT; break; }

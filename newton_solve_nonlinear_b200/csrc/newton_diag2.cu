@@ -224,7 +224,7 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
                 const float c0 = chunk == 0 ? __ldg(A.h0 + static_cast<size_t>(b) * D + lane0 + ld) : 0.f;
                 const float hin =
                     coop_lookback<SEGS, 1, true>(A.desc, tile, S.ngroups, DL, ld, lq, epoch, TA, TB, chunk, c0,
-                                                 status, &lbw);
+                                                 status, &lbw, publishes(A, tile, epoch));
                 if (lq == 0) carry[ld] = hin;
             }
             __syncthreads();
@@ -281,6 +281,7 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
         grid_barrier(hdr->barrier, nblocks, status);
         last_delta = ld_acquire_u32(&hdr->delta_bits[it % 3]);
         last_resid = ld_acquire_u32(&hdr->resid_bits[it % 3]);
+        record_trace(A, it, last_delta, last_resid);
         iters = it + 1;
         // a timeout another CTA raises may land between two threads' reads: decide once per CTA
         if (__syncthreads_or(*cta_err || timed_out(status))) { final_status = PARARNN_TIMEOUT; break; }

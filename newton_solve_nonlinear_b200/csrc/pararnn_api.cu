@@ -161,7 +161,8 @@ static cudaError_t enqueue_iterate(const pararnn_cell *cell, const pararnn_param
                                    const float *P, const float *h0, int B, int T, int mode,
                                    float lambda, float tol, int max_iters, float *h,
                                    pararnn_info *info_dev, void *workspace, cudaStream_t s,
-                                   const float *h_init = nullptr, int jac_every = 1) {
+                                   const float *h_init = nullptr, int jac_every = 1,
+                                   float *trace = nullptr, int trace_len = 0, long long withhold = -1) {
     const WsLayout L = ws_layout(*cell, B, T, mode);
     char *ws = static_cast<char *>(workspace);
     WsHeader *hdr = reinterpret_cast<WsHeader *>(ws + L.header);
@@ -192,6 +193,9 @@ static cudaError_t enqueue_iterate(const pararnn_cell *cell, const pararnn_param
     a.jac_every = jac_every;
     // the frozen Jacobian coefficients sit after the solve's own workspace
     a.coef = jac_every > 1 ? reinterpret_cast<float *>(ws + L.total) : nullptr;
+    a.trace = trace;
+    a.trace_len = trace ? trace_len : 0;
+    a.withhold = withhold;
 
     cudaError_t e = cudaMemsetAsync(ws + L.header, 0, 256, s);
     if (e == cudaSuccess && diag && L.elk > L.desc) e = cudaMemsetAsync(ws + L.desc, 0, L.elk - L.desc, s);
@@ -249,7 +253,8 @@ static int solve_enqueue(const pararnn_cell *cell, const pararnn_params *params,
                          const float *h0, int B, int T, int mode, float lambda, float tol,
                          int max_iters, float *h, pararnn_info *info_dev, void *workspace,
                          size_t ws_bytes, pararnn_stream stream, const float *h_init = nullptr,
-                         int jac_every = 1) {
+                         int jac_every = 1, float *trace = nullptr, int trace_len = 0,
+                         long long withhold = -1) {
     int rc = check_solve(cell, params, x, nullptr, h0, B, T, mode, lambda, tol, h, workspace,
                          ws_bytes);
     if (rc != PARARNN_OK) return rc;
@@ -265,7 +270,7 @@ static int solve_enqueue(const pararnn_cell *cell, const pararnn_params *params,
                                       static_cast<long long>(B) * T, s);
     if (e == cudaSuccess)
         e = enqueue_iterate(cell, params, P, h0, B, T, mode, lambda, tol, max_iters, h, info_dev,
-                            workspace, s, h_init, jac_every);
+                            workspace, s, h_init, jac_every, trace, trace_len, withhold);
     return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
 }
 
@@ -304,6 +309,53 @@ int pararnn_newton_solve_guess_async(const pararnn_cell *cell, const pararnn_par
     if (info_dev == nullptr || !aligned(info_dev, 4) || h_init == nullptr) return PARARNN_INVALID_ARG;
     return solve_enqueue(cell, params, x, h0, B, T, mode, lambda, tol, max_iters, h, info_dev, workspace,
                          ws_bytes, stream, h_init);
+}
+
+// Wait for `stream` and read the report the last solve on `workspace` left.
+static int read_report(const pararnn_cell *cell, int B, int T, int mode, void *workspace, cudaStream_t s,
+                       pararnn_info *info) {
+    const WsLayout L = ws_layout(*cell, B, T, mode);
+    pararnn_info host{};
+    const WsHeader *hdr = reinterpret_cast<const WsHeader *>(static_cast<char *>(workspace) + L.header);
+    cudaError_t e = cudaMemcpyAsync(&host, &hdr->info, sizeof(host), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
+    if (info) *info = host;
+    return host.status;
+}
+
+int pararnn_newton_solve_trace(const pararnn_cell *cell, const pararnn_params *params, const void *x,
+                               const float *h0, int B, int T, int mode, float lambda, float tol, int max_iters,
+                               float *h, pararnn_info *info, float *trace, int trace_len, void *workspace,
+                               size_t ws_bytes, pararnn_stream stream) {
+    if (trace == nullptr || trace_len < 1 || !aligned(trace, 8)) return PARARNN_INVALID_ARG;
+    if (cell_ok(cell, B, T, mode)) {
+        const size_t tb = static_cast<size_t>(trace_len) * 8;
+        const size_t hb = static_cast<size_t>(B) * T * cell->d * 4;
+        if (overlaps(trace, tb, workspace, ws_layout(*cell, B, T, mode).total) || overlaps(trace, tb, h, hb))
+            return PARARNN_INVALID_ARG;
+    }
+    const int rc = solve_enqueue(cell, params, x, h0, B, T, mode, lambda, tol, max_iters, h, nullptr, workspace,
+                                 ws_bytes, stream, nullptr, 1, trace, trace_len);
+    if (rc != PARARNN_OK) return rc;
+    return read_report(cell, B, T, mode, workspace, reinterpret_cast<cudaStream_t>(stream), info);
+}
+
+int pararnn_test_withheld_publish(const pararnn_cell *cell, const pararnn_params *params, const void *x,
+                                  const float *h0, int B, int T, int mode, float tol, float *h, pararnn_info *info,
+                                  long long tile, void *workspace, size_t ws_bytes, pararnn_stream stream) {
+    if (!cell_ok(cell, B, T, mode) || tile < 0) return PARARNN_INVALID_ARG;
+    long long tiles = 0;  // tiles of the look-back the solve will take
+    if (mode == PARARNN_QUASI && quasi_tc_supported(*cell, B, T))
+        tiles = static_cast<long long>(quasi_tc_desc_bytes(B, T, cell->d) / (static_cast<size_t>(cell->d) * 16));
+    else if (cell->kind == PARARNN_GRU_DIAG && (mode == PARARNN_DEER || mode == PARARNN_QUASI) &&
+             diag2_supported(*cell, B, T))
+        tiles = static_cast<long long>(diag2_desc_bytes(B, T, cell->d) / (64 * 16));
+    if (tile >= tiles) return PARARNN_INVALID_ARG;
+    const int rc = solve_enqueue(cell, params, x, h0, B, T, mode, 0.f, tol, 0, h, nullptr, workspace, ws_bytes,
+                                 stream, nullptr, 1, nullptr, 0, tile);
+    if (rc != PARARNN_OK) return rc;
+    return read_report(cell, B, T, mode, workspace, reinterpret_cast<cudaStream_t>(stream), info);
 }
 
 // ---- DEER with the Jacobian reused for several iterations ----
@@ -442,8 +494,9 @@ int pararnn_affine_scan(const float *A, const float *b, const float *h0, int B, 
         return PARARNN_INVALID_ARG;
     const size_t nA = static_cast<size_t>(B) * T * D * (dense ? D : 1) * 4;
     const size_t nh = static_cast<size_t>(B) * T * D * 4;
+    // h may be b itself (each b_t is read before its h_t is written), not a part of it
     if (overlaps(h, nh, A, nA) || overlaps(h, nh, h0, static_cast<size_t>(B) * D * 4) ||
-        overlaps(h, nh, workspace, need))
+        overlaps(h, nh, workspace, need) || (h != b && overlaps(h, nh, b, nh)))
         return PARARNN_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const cudaError_t e = dense ? launch_scan_dense(A, b, h0, B, T, D, h, workspace, s)

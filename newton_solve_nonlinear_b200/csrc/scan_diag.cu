@@ -162,19 +162,26 @@ std::mutex g_noalloc_mutex;
 void *g_noalloc_ptr[kNoAllocMaxDevices] = {};
 
 // Device address of the scratch array on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device (with that device current) and cached.
-cudaError_t noalloc_scratch(void **out) {
+// array's name is only a host-side stand-in, so the address is looked up with
+// the device current.  It is looked up again on every call made outside stream
+// capture: a device reset (or a primary context released and retained again)
+// reloads the library's device code, and the array may then live elsewhere.
+// Inside a capture the address the last uncaptured call on this device found
+// is used (the lookup itself may load device code, which a capture forbids).
+cudaError_t noalloc_scratch(cudaStream_t s, void **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if ((e = cudaStreamIsCapturing(s, &cap)) != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (g_noalloc_ptr[dev] == nullptr) {
+    if (cap == cudaStreamCaptureStatusNone) {
         void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) return e;
+        if ((e = cudaGetSymbolAddress(&p, g_noalloc_scratch)) != cudaSuccess) return e;
         g_noalloc_ptr[dev] = p;
+    } else if (g_noalloc_ptr[dev] == nullptr) {
+        return cudaErrorStreamCaptureUnsupported;
     }
     *out = g_noalloc_ptr[dev];
     return cudaSuccess;
@@ -200,10 +207,14 @@ extern "C" PARARNN_API int pararnn_affine_scan_noalloc(const float *A, const flo
         const auto px = reinterpret_cast<uintptr_t>(x), py = reinterpret_cast<uintptr_t>(y);
         return px < py + ny && py < px + nx;
     };
-    if (over(h, nh, A, nh) || over(h, nh, h0, static_cast<size_t>(B) * D * 4)) return PARARNN_INVALID_ARG;
-    void *scratch = nullptr;
-    if (noalloc_scratch(&scratch) != cudaSuccess) return PARARNN_CUDA_ERROR;
+    // h may be A or b exactly (each element is read before the thread that owns
+    // it writes h), but must not overlap them partly, nor h0
+    if ((h != A && over(h, nh, A, nh)) || (h != b && over(h, nh, b, nh)) ||
+        over(h, nh, h0, static_cast<size_t>(B) * D * 4))
+        return PARARNN_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    void *scratch = nullptr;
+    if (noalloc_scratch(s, &scratch) != cudaSuccess) return PARARNN_CUDA_ERROR;
     // launch_scan_diag first clears the header and the descriptors it will use
     cudaError_t e = launch_scan_diag(A, b, h0, B, T, D, h, scratch, s);
     if (e == cudaSuccess && status_dev)

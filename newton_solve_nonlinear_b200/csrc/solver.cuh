@@ -60,7 +60,23 @@ struct DiagArgs {
     int warm;                // hbuf[0] holds a caller's initial guess (else the guess is zero)
     int jac_every;           // Jacobian refreshed every jac_every iterations (<= 1: every one)
     float *coef;             // frozen Jacobian coefficients while jac_every > 1
+    float *trace;            // optional [trace_len][2]: max |dh| and max |r| of every iteration
+    int trace_len;
+    long long withhold;      // testing hook: this tile never publishes in the first iteration (-1: none)
 };
+
+// Iteration `it`'s convergence maxima into the optional trace (one thread).
+__device__ __forceinline__ void record_trace(const DiagArgs &A, int it, unsigned dbits, unsigned rbits) {
+    if (A.trace != nullptr && it < A.trace_len && blockIdx.x == 0 && threadIdx.x == 0) {
+        A.trace[2 * it] = __uint_as_float(dbits);
+        A.trace[2 * it + 1] = __uint_as_float(rbits);
+    }
+}
+
+// Whether a tile publishes its look-back descriptors in iteration epoch - 1.
+__device__ __forceinline__ bool publishes(const DiagArgs &A, long long tile, unsigned epoch) {
+    return epoch != 1u || tile != A.withhold;
+}
 
 // Workspace carve-up shared by the size query and the solver.
 struct WsLayout {
