@@ -21,7 +21,10 @@
  *   - Arrays are dense, row-major and contiguous; device arrays start on a
  *     16-byte boundary.
  *   - The caller owns all memory, including the workspace.  The library
- *     allocates no device or host memory and keeps no state between calls.
+ *     allocates no device or host memory.  The host-buffer calls (the
+ *     *_host entry points) keep two helper streams and their events per device
+ *     (one set per call running at a time), created on first use and reused
+ *     until the process exits; nothing else persists between calls.
  *   - Work is enqueued on `stream` (NULL means the legacy default stream).
  *   - Return value: a pararnn_status code; pararnn_status_string() names it.
  *     On PARARNN_INVALID_ARG nothing was enqueued.
@@ -307,7 +310,8 @@ PARARNN_API size_t pararnn_chunked_workspace_size(const pararnn_cell *cell, int 
  * (1, 2, 3, 4, ..., 4, 3, 2, 1), rounded by largest remainder, at least one
  * sequence each (B = 16 in 7 parts: 1, 2, 3, 4, 3, 2, 1).
  * While part p is solved on `stream`, part p+1's inputs are copied in and
- * part p-1's states copied out on two streams the call creates and destroys;
+ * part p-1's states copied out on two helper streams (kept per device and
+ * reused by later calls);
  * the device staging holds three parts' inputs and outputs in the workspace
  * (with two, a part's input copy would wait for the output copy two parts
  * earlier, and copies slower than the solve would set the pace).  Each part is an
@@ -532,7 +536,7 @@ PARARNN_API size_t pararnn_lstm_workspace_size(const pararnn_cell *cell, int B, 
 /*
  * pararnn_adjoint_host -- pararnn_adjoint from and to HOST memory, the copies
  * overlapped with the computation through the host-buffer pipeline (ramped
- * parts, three staging buffers, copy streams the call creates): part p's P,
+ * parts, three staging buffers, the helper copy streams): part p's P,
  * h and dL/dh are copied in while its neighbours are computed, its dL/dP
  * copied out.  Each part's dW_hh and db_hh partial sums stay on the device and
  * are added in part order at the end.
@@ -557,7 +561,7 @@ PARARNN_API size_t pararnn_adjoint_host_workspace_size(const pararnn_cell *cell,
  * pararnn_lstm_solve_host -- pararnn_lstm_solve from and to HOST memory, with
  * the copies overlapped with the computation as in pararnn_newton_solve_host:
  * the batch in `parts` ramped parts (same sizes), three staging buffers, part
- * p's x copied in and its (c, h) copied out on two streams the call creates,
+ * p's x copied in and its (c, h) copied out on the two helper streams,
  * while part p's neighbours are solved on `stream`.  Each part is an
  * independent solve to `tol`; the report is the worst part's.
  *   x_host     HOST [B, T, Din] of cell->x_dtype;  c0_host, h0_host HOST [B, D].

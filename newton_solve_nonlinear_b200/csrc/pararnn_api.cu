@@ -13,7 +13,10 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <vector>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "common.cuh"
 #include "solver.cuh"
@@ -53,6 +56,17 @@ cudaError_t launch_outer_sum(const float *grow, const float *hp, long long M, in
                              cudaStream_t s);
 
 namespace {
+
+// NVTX range around a host-side phase of a call (projection, Newton loop,
+// host-buffer part, backward pass, report wait): Nsight Systems shows the
+// phases and the launches they enqueue; with no tool attached a push/pop is a
+// few nanoseconds.
+struct Range {
+    explicit Range(const char *name) { nvtxRangePushA(name); }
+    ~Range() { nvtxRangePop(); }
+    Range(const Range &) = delete;
+    Range &operator=(const Range &) = delete;
+};
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -163,6 +177,7 @@ static cudaError_t enqueue_iterate(const pararnn_cell *cell, const pararnn_param
                                    pararnn_info *info_dev, void *workspace, cudaStream_t s,
                                    const float *h_init = nullptr, int jac_every = 1,
                                    float *trace = nullptr, int trace_len = 0, long long withhold = -1) {
+    const Range range("pararnn: Newton loop");
     const WsLayout L = ws_layout(*cell, B, T, mode);
     char *ws = static_cast<char *>(workspace);
     WsHeader *hdr = reinterpret_cast<WsHeader *>(ws + L.header);
@@ -228,6 +243,7 @@ int pararnn_input_projection(const pararnn_cell *cell, const pararnn_params *par
     if (!params || !x || !P || !params->w_ih || !params->b_ih) return PARARNN_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(P, 16) || !aligned(params->w_ih, 16) || !aligned(params->b_ih, 16))
         return PARARNN_INVALID_ARG;
+    const Range range("pararnn: input projection");
     const cudaError_t e = launch_projection(*cell, x, params->w_ih, params->b_ih, P,
                                             static_cast<long long>(B) * T,
                                             reinterpret_cast<cudaStream_t>(stream));
@@ -266,8 +282,11 @@ static int solve_enqueue(const pararnn_cell *cell, const pararnn_params *params,
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const WsLayout L = ws_layout(*cell, B, T, mode);
     float *P = reinterpret_cast<float *>(static_cast<char *>(workspace) + L.P);
-    cudaError_t e = launch_projection(*cell, x, params->w_ih, params->b_ih, P,
-                                      static_cast<long long>(B) * T, s);
+    cudaError_t e;
+    {
+        const Range range("pararnn: input projection");
+        e = launch_projection(*cell, x, params->w_ih, params->b_ih, P, static_cast<long long>(B) * T, s);
+    }
     if (e == cudaSuccess)
         e = enqueue_iterate(cell, params, P, h0, B, T, mode, lambda, tol, max_iters, h, info_dev,
                             workspace, s, h_init, jac_every, trace, trace_len, withhold);
@@ -314,6 +333,7 @@ int pararnn_newton_solve_guess_async(const pararnn_cell *cell, const pararnn_par
 // Wait for `stream` and read the report the last solve on `workspace` left.
 static int read_report(const pararnn_cell *cell, int B, int T, int mode, void *workspace, cudaStream_t s,
                        pararnn_info *info) {
+    const Range range("pararnn: wait for the report");
     const WsLayout L = ws_layout(*cell, B, T, mode);
     pararnn_info host{};
     const WsHeader *hdr = reinterpret_cast<const WsHeader *>(static_cast<char *>(workspace) + L.header);
@@ -653,6 +673,7 @@ int pararnn_adjoint(const pararnn_cell *cell, const pararnn_params *params, cons
         for (const auto &o2 : outs)
             if (&o2 != &o && overlaps(o.p, o.n, o2.p, o2.n)) return PARARNN_INVALID_ARG;
     }
+    const Range range("pararnn: backward pass");
     const cudaError_t e = adjoint_enqueue(cell, params, P, h0, h, dh, B, T, dP, dh0, dw_hh, db_hh, workspace,
                                           reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
@@ -804,17 +825,85 @@ struct PipeIo {
 // enq(p, b0, nb, buf) (returns a pararnn status), and its outputs copied out
 // on a second helper stream; pre(s_in) enqueues the copies made once per call
 // (initial states).  On return `sc` is ordered after the last copy out.
+// The pipeline's two helper streams and their events, created on a device's
+// first host-buffer call and reused by later calls on that device (creating
+// and destroying them cost a visible fraction of a short call).  A set is
+// held by one call at a time; concurrent calls on one device take separate
+// sets.  A set whose stream no longer answers (its context was reset) is
+// dropped and a new one made.
+struct PipeRes {
+    int dev = -1;
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev[3 * kHostBufs + 1] = {};  // in[NB], comp[NB], out[NB], start / end
+};
+std::mutex g_pipe_mutex;
+std::vector<PipeRes *> g_pipe_free;
+
+void pipe_destroy(PipeRes *r) {
+    for (cudaEvent_t &v : r->ev)
+        if (v) cudaEventDestroy(v);
+    if (r->s_in) cudaStreamDestroy(r->s_in);
+    if (r->s_out) cudaStreamDestroy(r->s_out);
+    delete r;
+}
+
+cudaError_t pipe_acquire(PipeRes **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    PipeRes *r = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_pipe_mutex);
+        for (size_t i = 0; i < g_pipe_free.size(); ++i)
+            if (g_pipe_free[i]->dev == dev) {
+                r = g_pipe_free[i];
+                g_pipe_free.erase(g_pipe_free.begin() + static_cast<long>(i));
+                break;
+            }
+    }
+    if (r != nullptr) {
+        const cudaError_t q = cudaStreamQuery(r->s_in);
+        if (q != cudaSuccess && q != cudaErrorNotReady) {  // stale: drop it without touching it
+            cudaGetLastError();
+            delete r;
+            r = nullptr;
+        }
+    }
+    if (r == nullptr) {
+        r = new PipeRes;
+        r->dev = dev;
+        e = cudaStreamCreateWithFlags(&r->s_in, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&r->s_out, cudaStreamNonBlocking);
+        for (int q = 0; q < 3 * kHostBufs + 1 && e == cudaSuccess; ++q)
+            e = cudaEventCreateWithFlags(&r->ev[q], cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            pipe_destroy(r);
+            return e;
+        }
+    }
+    *out = r;
+    return cudaSuccess;
+}
+
+void pipe_release(PipeRes *r, bool reuse) {
+    if (!reuse) {
+        pipe_destroy(r);
+        return;
+    }
+    std::lock_guard<std::mutex> lock(g_pipe_mutex);
+    g_pipe_free.push_back(r);
+}
+
 extern "C++" {  // a template: C++ linkage inside the exported block
 template <class Pre, class Enq>
 int run_pipeline(int B, int parts, int nbuf, const PipeIo &io, char *ws, cudaStream_t sc, Pre pre, Enq enq) {
     constexpr int NB = kHostBufs;
-    cudaStream_t s_in = nullptr, s_out = nullptr;
-    cudaEvent_t ev[3 * NB + 1] = {};  // in[NB], comp[NB], out[NB], start / end
+    PipeRes *res = nullptr;
+    cudaError_t e = pipe_acquire(&res);
+    if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
+    cudaStream_t s_in = res->s_in, s_out = res->s_out;
+    cudaEvent_t *ev = res->ev;
     cudaEvent_t *ev_in = ev, *ev_comp = ev + NB, *ev_out = ev + 2 * NB, &ev_edge = ev[3 * NB];
-    cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
-    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
-    for (int q = 0; q < 3 * NB + 1 && e == cudaSuccess; ++q)
-        e = cudaEventCreateWithFlags(&ev[q], cudaEventDisableTiming);
     int rc = PARARNN_OK;
     if (e == cudaSuccess) {  // start only after the caller's earlier work on its stream
         e = cudaEventRecord(ev_edge, sc);
@@ -832,7 +921,10 @@ int run_pipeline(int B, int parts, int nbuf, const PipeIo &io, char *ws, cudaStr
         if (e == cudaSuccess) e = cudaEventRecord(ev_in[buf], s_in);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(sc, ev_in[buf], 0);
         if (e != cudaSuccess) break;
-        rc = enq(p, b0, nb, buf);
+        {
+            const Range range("pararnn: host-buffer part");
+            rc = enq(p, b0, nb, buf);
+        }
         if (rc != PARARNN_OK) break;
         e = cudaEventRecord(ev_comp[buf], sc);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_comp[buf], 0);
@@ -845,13 +937,10 @@ int run_pipeline(int B, int parts, int nbuf, const PipeIo &io, char *ws, cudaStr
         e = cudaEventRecord(ev_edge, s_out);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(sc, ev_edge, 0);
     }
-    // leave nothing in flight before the helper streams go away
-    if (s_in) cudaStreamSynchronize(s_in);
-    if (s_out) cudaStreamSynchronize(s_out);
-    for (int q = 0; q < 3 * NB + 1; ++q)
-        if (ev[q]) cudaEventDestroy(ev[q]);
-    if (s_in) cudaStreamDestroy(s_in);
-    if (s_out) cudaStreamDestroy(s_out);
+    // leave nothing in flight on the helper streams before the set is handed on
+    const cudaError_t e1 = cudaStreamSynchronize(s_in);
+    const cudaError_t e2 = cudaStreamSynchronize(s_out);
+    pipe_release(res, e == cudaSuccess && e1 == cudaSuccess && e2 == cudaSuccess);
     if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
     return rc;
 }

@@ -100,32 +100,27 @@ def test_elk_full_size_sampled():
         assert abs(r.iters - g["iters"]) <= 1, (r.iters, g["iters"])
 
 
-@pytest.mark.parametrize("lam,slack", [(0.1, 1), (1.0, 2)])
-def test_elk_full_size_stronger_damping_iterations(lam, slack):
-    """The full near-unstable workload at lambda 0.1 and 1 (39 and 221 oracle
-    iterations).  Damped steps converge linearly, so the solve stops far from
-    the fixed point (the oracle's own final iterate is 5.6e-3 from the rollout
-    at lambda 1): the gates are the iteration count against the stored oracle
-    count (lambda 1: its delta at the stopping iteration is 0.02% below tol
-    and shrinks by ~1.7% per iteration, so fp32 rounding may move the stop by
-    two) and the fp64 residual of sampled sequences, max |h_t - f(h_{t-1})|,
-    at most 20 tol (the oracle's at lambda 1 on a B = 1, T = 1000 sample of
-    the same distribution is 7 tol)."""
+def test_elk_full_size_lambda_01_iterations():
+    """The full near-unstable workload at lambda 0.1 (39 oracle iterations).
+    Damped steps converge linearly, so the solve stops away from the fixed
+    point (the oracle's own final iterate is 5.6e-4 from the rollout): the
+    gates are the iteration count against the stored oracle count (+-1) and
+    the fp64 residual of sampled sequences, max |h_t - f(h_{t-1})| <= 10 tol.
+    Lambda 1 (221 iterations) is gated with its whole delta trajectory in
+    test_gpu_trace_timeout.py."""
     w = make_workload("near_unstable")
-    r = binding.solve_workload(w, "ELK", lam=lam)
+    r = binding.solve_workload(w, "ELK", lam=0.1)
     assert r.status == "OK"
     p = os.path.join(os.path.dirname(__file__), "golden", "oracle_iters.json")
-    key = f"near_unstable/ELK/{lam:g}"
-    g = json.load(open(p)).get(key) if os.path.exists(p) else None
-    assert g is not None, key
-    assert abs(r.iters - g["iters"]) <= slack, (r.iters, g["iters"])
+    g = json.load(open(p))["near_unstable/ELK/0.1"]
+    assert abs(r.iters - g["iters"]) <= 1, (r.iters, g["iters"])
     c = GRU.from_workload(w)
     h = r.h.cpu().double().numpy()
     for b in (0, 7):
         x = w.x[b:b + 1].double().numpy()
         hp = np.concatenate([w.h0[b:b + 1].double().numpy()[:, None], h[b:b + 1, :-1]], 1)
         f = c.gates(hp, c.project(x))[4]
-        assert np.max(np.abs(h[b:b + 1] - f)) <= 20 * w.tol
+        assert np.max(np.abs(h[b:b + 1] - f)) <= 10 * w.tol
 
 
 def test_elk_nan_input_diverges_and_bad_lambda_rejected():

@@ -204,8 +204,12 @@ def _golden():
 
 @pytest.mark.parametrize("key,name,over,mode,lam,samples", [
     ("untrained/T65536/QUASI", "untrained", dict(T=65536), "QUASI", 0.0, (0, 15)),
+    ("untrained/T16384/QUASI", "untrained", dict(T=16384), "QUASI", 0.0, (0, 15)),
+    ("untrained/T4096/QUASI", "untrained", dict(T=4096), "QUASI", 0.0, (0, 9)),
+    ("untrained/T1024/QUASI", "untrained", dict(T=1024), "QUASI", 0.0, (2,)),
     ("diag/QUASI", "diag", {}, "QUASI", 0.0, (3,)),
     ("near_unstable/QUASI_ELK/0.1", "near_unstable", {}, "QUASI_ELK", 0.1, (0, 7)),
+    ("near_unstable/QUASI_ELK/0.01", "near_unstable", {}, "QUASI_ELK", 0.01, (1, 6)),
     ("tiny/QUASI", "tiny", {}, "QUASI", 0.0, (0,)),
 ])
 def test_full_size_sampled(key, name, over, mode, lam, samples):

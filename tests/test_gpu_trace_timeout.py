@@ -153,3 +153,27 @@ def test_full_size_heavy_damping_trajectory(key, name, over, mode, lam):
         hp = np.concatenate([w.h0[b:b + 1].double().numpy()[:, None], h[b:b + 1, :-1]], 1)
         f = c.gates(hp, c.project(x))[4]
         assert np.max(np.abs(h[b:b + 1] - f)) <= 10 * w.tol
+
+
+_KEYS = [k for k in json.load(open(GOLDEN)) if not k.startswith("_") and not k.endswith("/1")]
+
+
+@pytest.mark.parametrize("key", _KEYS)
+def test_full_size_trajectory_against_stored_oracle(key):
+    """Every stored full-size oracle solve: the GPU's count within +-1 and its
+    recorded delta trajectory against the oracle's at every iteration."""
+    g = _golden()[key]
+    parts = key.split("/")
+    name, over = parts[0], {}
+    if name == "untrained":
+        over["T"] = int(parts[1][1:])
+        mode = parts[2]
+    else:
+        mode = parts[1]
+    lam = float(parts[2]) if mode in ("ELK", "QUASI_ELK") else 0.0
+    w = make_workload(name, **over)
+    r = binding.solve_workload(w, mode, lam=lam, trace=True)
+    assert r.status == g["status"] == "OK"
+    assert abs(r.iters - g["iters"]) <= 1, (r.iters, g["iters"])
+    ok = _close(r.trace[:, 0].numpy(), g["deltas"])
+    assert np.all(ok), (np.nonzero(~ok)[0][:10], r.trace[:, 0].numpy(), g["deltas"])
