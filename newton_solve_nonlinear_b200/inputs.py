@@ -137,6 +137,17 @@ WORKLOADS = {
                           w_dtype=torch.float32, tol=1e-4,
                           modes=("ELK", "QUASI_ELK", "DEER"),
                           lambdas=(1e-2, 1e-1, 1.0)),
+    # The near-unstable GRU with each recurrent block at spectral radius 3:
+    # the setting in which undamped Newton (DEER) actually fails -- its steps
+    # overshoot by many orders of magnitude and it does not converge -- while
+    # the damped methods (ELK, quasi-ELK) and quasi-DEER do.  At radius 1.5
+    # the GRU's gates keep the Jacobians contractive enough that DEER converges.
+    "unstable": dict(kind="dense", din=64, d=64, B=2, T=1000,
+                     w_var=lambda din, d: 1.0 / din, whh_var=None,
+                     radius=3.0, x_dtype=torch.float32,
+                     w_dtype=torch.float32, tol=1e-4,
+                     modes=("ELK", "QUASI_ELK", "QUASI", "DEER"),
+                     lambdas=(1e-2, 1e-1, 1.0)),
 }
 
 

@@ -48,24 +48,36 @@ CASES = [
     ("near_unstable/ELK/0.01", "near_unstable", {}, "ELK", 0.01),
     ("near_unstable/ELK/0.1", "near_unstable", {}, "ELK", 0.1),
     ("near_unstable/ELK/1", "near_unstable", {}, "ELK", 1.0),
+    # radius 3: undamped DEER fails (capped at 40 iterations), the others converge
+    ("unstable/DEER", "unstable", {}, "DEER", None, 40),
+    ("unstable/QUASI", "unstable", {}, "QUASI", None),
+    ("unstable/QUASI_ELK/0.01", "unstable", {}, "QUASI_ELK", 0.01),
+    ("unstable/QUASI_ELK/0.1", "unstable", {}, "QUASI_ELK", 0.1),
+    ("unstable/QUASI_ELK/1", "unstable", {}, "QUASI_ELK", 1.0),
+    # full-Jacobian ELK stalls on it (max |dh| levels off near 7e-3 at lambda 1):
+    # the first 100 damped steps are stored, capped
+    ("unstable/ELK/1", "unstable", {}, "ELK", 1.0, 100),
 ]
 
 
-def run_case(name, over, mode, lam):
+def run_case(name, over, mode, lam, max_iters=None):
     w = make_workload(name, **over)
     c = GRU.from_workload(w)
     x = w.x.double().numpy()
     h0 = w.h0.double().numpy()
     t0 = time.time()
     if mode in ("DEER", "QUASI"):
-        r = oracle.newton_solve(c, x, h0, mode, w.tol)
+        r = oracle.newton_solve(c, x, h0, mode, w.tol, max_iters=max_iters)
     else:
-        r = oracle.elk_solve(c, x, h0, mode, lam, w.tol)
+        r = oracle.elk_solve(c, x, h0, mode, lam, w.tol, max_iters=max_iters)
     secs = time.time() - t0
     ref = rollout(c, x, h0)
     err = float(np.max(np.abs(r["h"] - ref))) if np.all(np.isfinite(r["h"])) else float("nan")
-    return dict(iters=r["iters"], status=r["status"], tol=w.tol, deltas=r["deltas"],
-                max_abs_vs_rollout=err, B=w.B, T=w.T, D=w.d, din=w.din, seconds=round(secs, 1))
+    out = dict(iters=r["iters"], status=r["status"], tol=w.tol, deltas=r["deltas"],
+               max_abs_vs_rollout=err, B=w.B, T=w.T, D=w.d, din=w.din, seconds=round(secs, 1))
+    if max_iters is not None:
+        out["max_iters"] = max_iters
+    return out
 
 
 def main():
@@ -81,10 +93,10 @@ def main():
     data = json.load(open(OUT)) if os.path.exists(OUT) else {}
     data.setdefault("_about", "fp64 oracle iteration counts at full workload sizes; written by "
                     "tests/golden/make_golden.py (oracle only)")
-    for key, name, over, mode, lam in CASES:
+    for key, name, over, mode, lam, *cap in CASES:
         if args.only and not key.startswith(args.only):
             continue
-        res = run_case(name, over, mode, lam)
+        res = run_case(name, over, mode, lam, *cap)
         data[key] = res
         print(key, res["iters"], res["status"], res["max_abs_vs_rollout"], res["seconds"], flush=True)
         with open(OUT, "w") as f:

@@ -155,7 +155,10 @@ def test_full_size_heavy_damping_trajectory(key, name, over, mode, lam):
         assert np.max(np.abs(h[b:b + 1] - f)) <= 10 * w.tol
 
 
-_KEYS = [k for k in json.load(open(GOLDEN)) if not k.startswith("_") and not k.endswith("/1")]
+# the lambda 1 solves have their own test above; the radius-3 workload (whose
+# DEER does not converge) is covered by test_gpu_unstable.py
+_KEYS = [k for k in json.load(open(GOLDEN))
+         if not k.startswith("_") and not k.endswith("/1") and not k.startswith("unstable/")]
 
 
 @pytest.mark.parametrize("key", _KEYS)
