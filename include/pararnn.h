@@ -431,10 +431,10 @@ PARARNN_API int pararnn_affine_scan_status(const void *workspace, pararnn_stream
  *                 device-side wait expired (result unreliable).
  * Limits: the scratch a size needs is pararnn_affine_scan_workspace_size(B, T,
  * D, 0) bytes (a 256-byte header plus 16 bytes per lane of every look-back
- * tile; a tile spans min(D, 64) lanes and 4 * 256 / (min(D, 64) / 4) steps,
- * i.e. 64 steps for D >= 64).  Sizes needing more than 16 MiB -- about 2^24
- * elements of B*T*D for D >= 64, e.g. [15, 65536, 64] is accepted and
- * [16, 65536, 64] is not -- are rejected with PARARNN_INVALID_ARG.
+ * tile; a tile spans min(D, 64) lanes and 8 * 256 / (min(D, 64) / 4) steps,
+ * i.e. 128 steps for D >= 64).  Sizes needing more than 16 MiB -- about 2^25
+ * elements of B*T*D for D >= 64, e.g. [31, 65536, 64] is accepted and
+ * [32, 65536, 64] is not -- are rejected with PARARNN_INVALID_ARG.
  * Every call made outside stream capture looks the array's device address up
  * with the current device (so a device reset, which reloads the library's
  * device code, is followed correctly); a call inside a capture reuses the

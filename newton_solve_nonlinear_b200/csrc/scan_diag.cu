@@ -7,7 +7,7 @@
 // system).  Single pass over HBM (12 bytes per element: a, b in, h out):
 // tiles of (sequence, 64 lanes, L steps) are taken in order from a ticket
 // counter, so every tile's predecessor has already started; each thread
-// composes 4 steps x 4 lanes in registers, a shared-memory pass forms the
+// composes 8 steps x 4 lanes in registers, a shared-memory pass forms the
 // tile-local exclusive prefixes, one thread per lane resolves the carry with a
 // decoupled look-back, and the tile is re-swept and written with float4 stores.
 #include <mutex>
@@ -19,7 +19,7 @@
 namespace pararnn {
 namespace {
 
-constexpr int TK = 4;
+constexpr int TK = 8;  // steps per thread, 128-step tiles (measured: 4 steps 0.61 of HBM, 8 0.72, 12 0.67, 16 0.69)
 
 struct ScanArgs {
     const float *A, *b, *h0;
