@@ -490,6 +490,35 @@ PARARNN_API int pararnn_adjoint(const pararnn_cell *cell, const pararnn_params *
                                 float *dh0, float *dw_hh, float *db_hh, void *workspace, size_t ws_bytes,
                                 pararnn_stream stream);
 
+/*
+ * pararnn_adjoint_exact -- the exact backward pass of the dense GRU
+ * (cell->kind == PARARNN_GRU_DENSE): pararnn_adjoint with the full transposed
+ * Jacobian in the reverse recurrence, lam_T = g_T, lam_t = g_t + J_{t+1}^T
+ * lam_{t+1}, instead of its diagonal (the pages train with the diagonal --
+ * "Towards Scalable and Stable Parallelization of Nonlinear RNNs", atlas
+ * summary, table "Measured effects reported in the paper" -- so this is the
+ * reference those gradients approximate).  J_t is the dense-cell Jacobian of
+ * pararnn_newton_solve (mode DEER) at the evaluated states.  The recurrence is
+ * solved as the library's dense affine scan over reversed time on the
+ * materialised matrices J_{t+1}^T, so the workspace holds B * T * D^2 floats
+ * besides the pass's vectors.  Outputs and formulas otherwise as
+ * pararnn_adjoint (dw_hh [3D, D]; dh0 = J_1^T lam_1).
+ *   cell      PARARNN_GRU_DENSE, d a multiple of 4, d <= 64.
+ *   workspace DEVICE, >= pararnn_adjoint_exact_workspace_size bytes, 256-byte aligned.
+ * All device pointers 16-byte aligned; outputs must not overlap inputs or the
+ * workspace.  Asynchronous: returns PARARNN_OK, INVALID_ARG or CUDA_ERROR.
+ * The parameter sums are taken in a fixed order.
+ */
+PARARNN_API int pararnn_adjoint_exact(const pararnn_cell *cell, const pararnn_params *params, const float *P,
+                                      const float *h0, const float *h, const float *dh, int B, int T, float *dP,
+                                      float *dh0, float *dw_hh, float *db_hh, void *workspace, size_t ws_bytes,
+                                      pararnn_stream stream);
+
+/* pararnn_adjoint_exact_workspace_size -- bytes pararnn_adjoint_exact needs
+ * (about (D + 12) floats per state of B*T*D, plus the scan's and the sums'
+ * scratch), or 0 for rejected arguments. */
+PARARNN_API size_t pararnn_adjoint_exact_workspace_size(const pararnn_cell *cell, int B, int T);
+
 /* pararnn_adjoint_workspace_size -- bytes of workspace pararnn_adjoint needs
  * (about 0.25 B + 0.02 B per state of B*T*D plus 256), or 0 when the
  * arguments are rejected (not the diagonal cell, B, T or D < 1). */

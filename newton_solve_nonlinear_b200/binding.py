@@ -30,7 +30,8 @@ EXPORTS = ("pararnn_workspace_size", "pararnn_newton_solve", "pararnn_newton_sol
            "pararnn_chunked_workspace_size", "pararnn_lstm_solve", "pararnn_lstm_workspace_size",
            "pararnn_newton_solve_reuse", "pararnn_reuse_workspace_size", "pararnn_lstm_solve_host",
            "pararnn_lstm_host_workspace_size", "pararnn_adjoint_host", "pararnn_adjoint_host_workspace_size",
-           "pararnn_newton_solve_trace", "pararnn_test_withheld_publish")
+           "pararnn_newton_solve_trace", "pararnn_test_withheld_publish", "pararnn_adjoint_exact",
+           "pararnn_adjoint_exact_workspace_size")
 
 
 class Cell(ctypes.Structure):
@@ -125,6 +126,11 @@ def lib() -> ctypes.CDLL:
         L.pararnn_test_withheld_publish.argtypes = [ctypes.POINTER(Cell), ctypes.POINTER(Params), vp, vp, ci, ci,
                                                     ci, cf, vp, ctypes.POINTER(Info), ctypes.c_longlong, vp, sz, vp]
         L.pararnn_test_withheld_publish.restype = ci
+        L.pararnn_adjoint_exact.argtypes = [ctypes.POINTER(Cell), ctypes.POINTER(Params), vp, vp, vp, vp, ci, ci,
+                                            vp, vp, vp, vp, vp, sz, vp]
+        L.pararnn_adjoint_exact.restype = ci
+        L.pararnn_adjoint_exact_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci]
+        L.pararnn_adjoint_exact_workspace_size.restype = sz
         L.pararnn_status_string.argtypes = [ci]
         L.pararnn_status_string.restype = ctypes.c_char_p
         _lib = L
@@ -416,6 +422,33 @@ def lstm_solve_host(w_ih, b_ih, u, b_hh, x_host, c0_host, h0_host, *, tol: float
 def adjoint_workspace_size(d: int, B: int, T: int, kind: str = "diag") -> int:
     cell = make_cell(kind, 1, d, torch.float32)
     return int(lib().pararnn_adjoint_workspace_size(ctypes.byref(cell), B, T))
+
+
+def adjoint_exact(w_hh, b_hh, P, h0, h, dh, *, workspace=None, out=None, stream=None) -> dict:
+    """The exact backward pass of the dense GRU (full transposed Jacobian):
+    w_hh [3D, D], b_hh [3D], P [B,T,3D], h0 [B,D], h and dh [B,T,D], all fp32
+    CUDA.  Returns dict(dP, dh0, dw_hh, db_hh)."""
+    B, T, d = h.shape
+    cell = make_cell("dense", 1, d, torch.float32)
+    L = lib()
+    need = int(L.pararnn_adjoint_exact_workspace_size(ctypes.byref(cell), B, T))
+    if need == 0:
+        raise ValueError("arguments rejected by pararnn_adjoint_exact_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, h.device)
+    o = out or {}
+    dP = o["dP"] if "dP" in o else torch.empty_like(P)
+    dh0 = o["dh0"] if "dh0" in o else torch.empty_like(h0)
+    dw = o["dw_hh"] if "dw_hh" in o else torch.empty_like(w_hh)
+    db = o["db_hh"] if "db_hh" in o else torch.empty_like(b_hh)
+    params = Params(None, None, _dev(w_hh, "w_hh"), _dev(b_hh, "b_hh"))
+    rc = L.pararnn_adjoint_exact(ctypes.byref(cell), ctypes.byref(params), _dev(P, "P"), _dev(h0, "h0"),
+                                 _dev(h, "h"), _dev(dh, "dh"), B, T, _dev(dP, "dP"), _dev(dh0, "dh0"),
+                                 _dev(dw, "dw_hh"), _dev(db, "db_hh"), _dev(workspace, "workspace"),
+                                 workspace.numel(), _stream(stream))
+    if rc != 0:
+        raise RuntimeError(f"pararnn_adjoint_exact: {L.pararnn_status_string(rc).decode()}")
+    return dict(dP=dP, dh0=dh0, dw_hh=dw, db_hh=db)
 
 
 def adjoint(w_hh, b_hh, P, h0, h, dh, *, workspace=None, out=None, stream=None, check: bool = False) -> dict:

@@ -54,6 +54,10 @@ cudaError_t adjoint_enqueue(const pararnn_cell *cell, const pararnn_params *para
                             float *db_hh, void *workspace, cudaStream_t s);
 cudaError_t launch_outer_sum(const float *grow, const float *hp, long long M, int N, int K, float *part, float *out,
                              cudaStream_t s);
+size_t adjoint_exact_ws_bytes(int B, int T, int D);
+cudaError_t adjoint_exact_enqueue(const float *w_hh, const float *b_hh, const float *P, const float *h0,
+                                  const float *h, const float *dh, int B, int T, int D, float *dP, float *dh0,
+                                  float *dw_hh, float *db_hh, void *workspace, cudaStream_t s);
 
 namespace {
 
@@ -676,6 +680,42 @@ int pararnn_adjoint(const pararnn_cell *cell, const pararnn_params *params, cons
     const Range range("pararnn: backward pass");
     const cudaError_t e = adjoint_enqueue(cell, params, P, h0, h, dh, B, T, dP, dh0, dw_hh, db_hh, workspace,
                                           reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
+}
+
+size_t pararnn_adjoint_exact_workspace_size(const pararnn_cell *cell, int B, int T) {
+    if (!cell || cell->kind != PARARNN_GRU_DENSE || B < 1 || T < 1) return 0;
+    if (cell->d < 4 || cell->d > 64 || cell->d % 4 != 0) return 0;
+    if (static_cast<long long>(B) * T >= (1ll << 31) - 1) return 0;
+    return adjoint_exact_ws_bytes(B, T, cell->d);
+}
+
+int pararnn_adjoint_exact(const pararnn_cell *cell, const pararnn_params *params, const float *P, const float *h0,
+                          const float *h, const float *dh, int B, int T, float *dP, float *dh0, float *dw_hh,
+                          float *db_hh, void *workspace, size_t ws_bytes, pararnn_stream stream) {
+    const size_t need = pararnn_adjoint_exact_workspace_size(cell, B, T);
+    if (need == 0 || ws_bytes < need || !params || !params->w_hh || !params->b_hh) return PARARNN_INVALID_ARG;
+    if (!P || !h0 || !h || !dh || !dP || !dh0 || !dw_hh || !db_hh || !workspace) return PARARNN_INVALID_ARG;
+    const void *ptrs[] = {P, h0, h, dh, dP, dh0, dw_hh, db_hh, params->w_hh, params->b_hh};
+    for (const void *q : ptrs)
+        if (!aligned(q, 16)) return PARARNN_INVALID_ARG;
+    if (!aligned(workspace, 256)) return PARARNN_INVALID_ARG;
+    const int D = cell->d;
+    const size_t st = static_cast<size_t>(B) * T * D * 4;
+    const size_t bd = static_cast<size_t>(B) * D * 4, pd = static_cast<size_t>(3) * D * D * 4;
+    const size_t bb = static_cast<size_t>(3) * D * 4;
+    const struct { const void *p; size_t n; } ins[] = {{P, 3 * st}, {h0, bd}, {h, st}, {dh, st},
+                                                       {params->w_hh, pd}, {params->b_hh, bb}, {workspace, need}};
+    const struct { const void *p; size_t n; } outs[] = {{dP, 3 * st}, {dh0, bd}, {dw_hh, pd}, {db_hh, bb}};
+    for (const auto &o : outs) {
+        for (const auto &i : ins)
+            if (overlaps(o.p, o.n, i.p, i.n)) return PARARNN_INVALID_ARG;
+        for (const auto &o2 : outs)
+            if (&o2 != &o && overlaps(o.p, o.n, o2.p, o2.n)) return PARARNN_INVALID_ARG;
+    }
+    const Range range("pararnn: exact backward pass");
+    const cudaError_t e = adjoint_exact_enqueue(params->w_hh, params->b_hh, P, h0, h, dh, B, T, D, dP, dh0, dw_hh,
+                                                db_hh, workspace, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
 }
 

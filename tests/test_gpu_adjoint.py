@@ -10,6 +10,8 @@ Tolerance: normwise, ||got - want||_inf <= 1e-4 ||want||_inf for dP and dh0
 (lam accumulates T fp32 steps of a_t lam + g) and 1e-4 for the parameter sums
 over B*T terms; the kernel's exponentials carry ~1e-7 relative error.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -252,3 +254,47 @@ def test_host_buffer_adjoint_matches_device(kind, B, T, D, parts):
     assert _same_run(got["dP"], ref["dP"]) and _same_run(got["dh0"], ref["dh0"])
     for k in ("dw_hh", "db_hh"):
         assert _rel(got[k].double().numpy(), ref[k].double().cpu().numpy()) <= 1e-5, k
+
+
+# ---- the dense cell's exact backward pass (full transposed Jacobian) ----
+
+@pytest.mark.parametrize("B,T,D", [(2, 100, 64), (3, 257, 32), (1, 1, 8), (2, 300, 12), (1, 64, 48)])
+def test_exact_dense_adjoint_matches_oracle(B, T, D):
+    """pararnn_adjoint_exact against the oracle's jacobian='exact' pass (whose
+    reverse recurrence is J_{t+1}^T lam_{t+1} with the full Jacobian; the
+    oracle itself equals torch autograd through an fp64 GRUCell rollout):
+    normwise 1e-4 as the other backward passes.  The diagonal pass differs from
+    it (checked too), so the test tells the two apart."""
+    cell, w_hh, b_hh, P, h0, h, dh = _dense_case(B, T, D, seed=B * 5 + T + D)
+    r = binding.adjoint_exact(w_hh.cuda(), b_hh.cuda(), P.cuda(), h0.cuda(), h.cuda(), dh.cuda())
+    f64 = lambda t: t.double().numpy()
+    ref = oracle_adjoint(cell, f64(P), f64(h0), f64(h), f64(dh), jacobian="exact")
+    got = {k: v.double().cpu().numpy() for k, v in r.items()}
+    for k in ("dP", "dh0", "dw_hh", "db_hh"):
+        assert _rel(got[k], ref[k]) <= 1e-4, k
+    if T > 1:
+        quasi = oracle_adjoint(cell, f64(P), f64(h0), f64(h), f64(dh), jacobian="diag")
+        assert _rel(got["dP"], quasi["dP"]) > 1e-3
+
+
+def test_exact_dense_adjoint_with_diagonal_u_equals_diagonal_pass():
+    """With every recurrent block diagonal the Jacobian is diagonal, so the
+    exact pass equals the diagonal-Jacobian pass."""
+    B, T, D = 2, 400, 32
+    cell, u, b_hh, P, h0, h, dh = _case(B, T, D, seed=33)
+    U = torch.cat([torch.diag(u[k * D:(k + 1) * D]) for k in range(3)], 0)
+    args = [U.cuda(), b_hh.cuda(), P.cuda(), h0.cuda(), h.cuda(), dh.cuda()]
+    rx = binding.adjoint_exact(*args)
+    rq = binding.adjoint(*args)
+    for k in ("dP", "dh0", "dw_hh", "db_hh"):
+        assert _rel(rx[k].double().cpu().numpy(), rq[k].double().cpu().numpy()) <= 1e-5, k
+
+
+def test_exact_dense_adjoint_rejects_other_cells():
+    L = binding.lib()
+    assert L.pararnn_adjoint_exact_workspace_size(ctypes.byref(binding.make_cell("diag", 1, 64, torch.float32)),
+                                                  2, 10) == 0
+    assert L.pararnn_adjoint_exact_workspace_size(ctypes.byref(binding.make_cell("dense", 1, 68, torch.float32)),
+                                                  2, 10) == 0
+    assert L.pararnn_adjoint_exact_workspace_size(ctypes.byref(binding.make_cell("dense", 1, 30, torch.float32)),
+                                                  2, 10) == 0
