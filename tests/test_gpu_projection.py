@@ -21,6 +21,7 @@ pytestmark = pytest.mark.gpu
     (4096, 2048, 2048, torch.bfloat16),   # tcgen05, the diagonal-layer shape (reduced M)
     (1000, 128, 256, torch.bfloat16),     # tcgen05, ragged M (not a multiple of 128)
     (77, 64, 512, torch.bfloat16),        # tcgen05, a single partial row tile
+    (33001, 128, 256, torch.bfloat16),    # tcgen05, several tiles per CTA (both accumulators), ragged M
     (333, 96, 256, torch.bfloat16),       # CUDA-core (Din not a multiple of 64)
     (2000, 64, 64, torch.float32),        # tcgen05 3 x TF32 (N = 192, K = 64)
     (1000, 32, 32, torch.float32),        # tcgen05 3 x TF32 (N = 96, K = 32), ragged M
