@@ -36,7 +36,7 @@ namespace pararnn {
 namespace {
 using namespace tc;
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 3;
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;        // 16 KB
 constexpr int B_BYTES = BN * BK * 2;        // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
