@@ -608,6 +608,37 @@ def _dist_setup():
     return world, rank, local, dev, barrier
 
 
+def copy_bandwidth(dev, nbytes: int = 256 << 20) -> dict:
+    """Pinned host <-> device copy bandwidth of this machine, GB/s (the ceiling of
+    every end-to-end number that moves its inputs and results over the host
+    link): one copy each way, then both at once, timed with CUDA events."""
+    import torch
+    n = nbytes // 4
+    hsrc, hdst = torch.empty(n).pin_memory(), torch.empty(n).pin_memory()
+    d1, d2 = torch.empty(n, device=dev), torch.empty(n, device=dev)
+    s1, s2 = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    out = {}
+    for name in ("h2d", "d2h", "both"):
+        for rep in range(2):  # the first pass warms the link
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            if name in ("h2d", "both"):
+                with torch.cuda.stream(s1):
+                    d1.copy_(hsrc, non_blocking=True)
+            if name in ("d2h", "both"):
+                with torch.cuda.stream(s2):
+                    hdst.copy_(d2, non_blocking=True)
+            cur = torch.cuda.current_stream(dev)
+            cur.wait_stream(s1)
+            cur.wait_stream(s2)
+            e1.record()
+            torch.cuda.synchronize()
+        moved = nbytes * (2 if name == "both" else 1)
+        out[name] = moved / (e0.elapsed_time(e1) / 1e3) / 1e9
+    return out
+
+
 def bench_solve(args, name: str, *, full: bool = True, steps: int | None = None):
     """Time one solver family (projection + the whole Newton loop per step) and
     return its JSON line.  ``full`` adds the end-to-end (host buffers) number,
@@ -728,7 +759,8 @@ def bench_solve(args, name: str, *, full: bool = True, steps: int | None = None)
         e2e = {"value": job_value(states, e2e_steps, world, max_over_ranks(ea.elapsed_time(eb), dev)),
                "unit": UNIT,
                "h2d_bytes_per_step": x_host.numel() * x_host.element_size() + h0_host.numel() * 4,
-               "d2h_bytes_per_step": h_host.numel() * 4 + 16 * parts, "parts": parts}
+               "d2h_bytes_per_step": h_host.numel() * 4 + 16 * parts, "parts": parts,
+               "copy_gbs": copy_bandwidth(dev)}
         del ws_host
 
     cpu = roll = None
