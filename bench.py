@@ -38,7 +38,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "converged states/sec (B*T*D per s, Newton to tol)"
 UNIT = "states/s"
-E2E_PARTS = 7  # parts of the batch whose copies the host-buffer solve overlaps (ramped sizes)
+E2E_PARTS = 7  # parts (ramped sizes) whose copies the host-buffer calls overlap with the solves
 # The benchmarked solves, one per row family of the hot path.  "untrained"
 # (the default) is the headline; the others measure the other solver kernels
 # with the same JSON line.  Roofline units per state and Newton iteration:
@@ -722,15 +722,16 @@ def bench_solve(args, name: str, *, full: bool = True, steps: int | None = None)
     iters = max(step_iters)
 
     e2e = None
-    parts = max(1, min(E2E_PARTS, B)) if k == 1 else 1
+    parts = max(1, min(E2E_PARTS, (T + 127) // 128)) if k == 1 else 1
     if full:
         # end to end through the public host-buffer call: page-locked x and h0 in,
-        # h out; the library splits the batch into parts and overlaps the copies
+        # h out; the library streams the sequence through the device in time
+        # parts (the whole batch in each) and overlaps the copies with the solves
         x_host = w.x.contiguous().pin_memory()
         h0_host = w.h0.float().contiguous().pin_memory()
         h_host = torch.empty(B, T, D, dtype=torch.float32).pin_memory()
         ws_host = binding.alloc_workspace(
-            binding.host_workspace_size(kind, din, D, B, T, mode, parts, w.x_dtype), dev)
+            binding.host_streamed_workspace_size(kind, din, D, B, T, mode, parts, w.x_dtype), dev)
         e2e_steps = max(1, min(steps, 5))
 
         def e2e_step():
@@ -741,25 +742,30 @@ def bench_solve(args, name: str, *, full: bool = True, steps: int | None = None)
                                      jac_every=k, out=out, workspace=ws, stream=stream)
                 h_host.copy_(out, non_blocking=True)
                 return None
-            return binding.newton_solve_host(w_ih, b_ih, w_hh, b_hh, x_host, h0_host, kind=kind,
-                                             mode=mode, lam=lam, tol=w.tol, parts=parts, out=h_host,
-                                             workspace=ws_host, stream=stream)
+            return binding.newton_solve_host_streamed(w_ih, b_ih, w_hh, b_hh, x_host, h0_host, kind=kind,
+                                                      mode=mode, lam=lam, tol=w.tol, parts=parts, out=h_host,
+                                                      workspace=ws_host, stream=stream)
 
         e2e_step()
         barrier()
         torch.cuda.synchronize()
         ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ea.record(stream)
+        e2e_iters = []
         for _ in range(e2e_steps):
             r = e2e_step()
             if r is not None and r.status != "OK":
                 raise SystemExit(f"{name}: end-to-end solve status {r.status}")
+            if r is not None:
+                e2e_iters.append(r.iters)
         eb.record(stream)
         torch.cuda.synchronize()
         e2e = {"value": job_value(states, e2e_steps, world, max_over_ranks(ea.elapsed_time(eb), dev)),
                "unit": UNIT,
                "h2d_bytes_per_step": x_host.numel() * x_host.element_size() + h0_host.numel() * 4,
                "d2h_bytes_per_step": h_host.numel() * 4 + 16 * parts, "parts": parts,
+               "split": "time" if k == 1 else "none",
+               "iters_summed_over_parts": e2e_iters,
                "copy_gbs": copy_bandwidth(dev)}
         del ws_host
 

@@ -343,6 +343,46 @@ PARARNN_API size_t pararnn_host_workspace_size(const pararnn_cell *cell, int B, 
                                                int parts);
 
 /*
+ * pararnn_newton_solve_host_streamed -- the evaluation from and to HOST memory
+ * with the sequence streamed through the device in `parts` consecutive time
+ * parts, every sequence of the batch in each part.  Part p starts from each
+ * sequence's last state of part p-1 (h0 for the first) and is solved to `tol`
+ * on its own: the solve over time chunks of pararnn_newton_solve_chunked (the
+ * ParaRNN summary page, "Experimental Results", names chunking for the Newton
+ * iteration's state memory), here with the copies overlapped: while part p is
+ * solved on `stream`, part p+1's inputs are copied in and part p-1's states
+ * out on two helper streams.  Unlike batch
+ * parts, every part keeps the whole batch, so each solve keeps its full width;
+ * the parts ramp (128-step units weighted min(p + 1, parts - p, 4), rounded
+ * by largest remainder with at least one unit each, as in
+ * pararnn_newton_solve_host; the last part gives up the steps past T) so that
+ * the exposed first copy in and last copy out are short (T = 65536 in 7 parts:
+ * 4096, 8192, 12288, 16384, 12288, 8192, 4096 steps).  The states differ from the single solve's within the
+ * convergence tolerance (each part meets it on its own).
+ *
+ * Arguments as for pararnn_newton_solve_host, except:
+ *   parts      1 <= parts <= ceil(T / 128).
+ *   max_iters  the cap of each part's solve; <= 0 means T + 1.
+ *   info       HOST, output, may be NULL: iterations summed over the parts
+ *              (as pararnn_newton_solve_chunked reports them), the worst
+ *              status, the largest delta and residual.
+ *   workspace  DEVICE, at least pararnn_host_streamed_workspace_size(cell, B,
+ *              T, mode, parts) bytes, 256-byte aligned.
+ * The copies are strided (each sequence's rows of a part): x_host, h_host
+ * are [B, T, .] as for pararnn_newton_solve_host.
+ * Returns the worst part's status, or INVALID_ARG / CUDA_ERROR.
+ */
+PARARNN_API int pararnn_newton_solve_host_streamed(const pararnn_cell *cell, const pararnn_params *params,
+                                                   const void *x_host, const float *h0_host, int B, int T,
+                                                   int mode, float lambda, float tol, int max_iters,
+                                                   float *h_host, pararnn_info *info, int parts,
+                                                   void *workspace, size_t ws_bytes, pararnn_stream stream);
+
+/* Workspace bytes of pararnn_newton_solve_host_streamed; 0 if the arguments are rejected. */
+PARARNN_API size_t pararnn_host_streamed_workspace_size(const pararnn_cell *cell, int B, int T, int mode,
+                                                        int parts);
+
+/*
  * pararnn_input_projection -- P = x W_ih^T + b_ih for every (b, t): the input
  * pre-activations, which do not depend on the state and so are computed once
  * per solve (as one GEMM [B*T, Din] x [Din, 3D]).  pararnn_newton_solve runs

@@ -31,7 +31,8 @@ EXPORTS = ("pararnn_workspace_size", "pararnn_newton_solve", "pararnn_newton_sol
            "pararnn_newton_solve_reuse", "pararnn_reuse_workspace_size", "pararnn_lstm_solve_host",
            "pararnn_lstm_host_workspace_size", "pararnn_adjoint_host", "pararnn_adjoint_host_workspace_size",
            "pararnn_newton_solve_trace", "pararnn_test_withheld_publish", "pararnn_adjoint_exact",
-           "pararnn_adjoint_exact_workspace_size")
+           "pararnn_adjoint_exact_workspace_size", "pararnn_newton_solve_host_streamed",
+           "pararnn_host_streamed_workspace_size")
 
 
 class Cell(ctypes.Structure):
@@ -85,6 +86,10 @@ def lib() -> ctypes.CDLL:
         L.pararnn_newton_solve_host.restype = ci
         L.pararnn_host_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci, ci, ci]
         L.pararnn_host_workspace_size.restype = sz
+        L.pararnn_newton_solve_host_streamed.argtypes = L.pararnn_newton_solve_host.argtypes
+        L.pararnn_newton_solve_host_streamed.restype = ci
+        L.pararnn_host_streamed_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci, ci, ci]
+        L.pararnn_host_streamed_workspace_size.restype = sz
         L.pararnn_adjoint.argtypes = [ctypes.POINTER(Cell), ctypes.POINTER(Params), vp, vp, vp, vp, ci, ci,
                                       vp, vp, vp, vp, vp, sz, vp]
         L.pararnn_adjoint.restype = ci
@@ -387,6 +392,44 @@ def newton_solve_host(w_ih, b_ih, w_hh, b_hh, x_host, h0_host, *, kind: str, mod
                                      _dev(workspace, "workspace"), workspace.numel(), _stream(stream))
     if rc in (3, 4):
         raise RuntimeError(f"pararnn_newton_solve_host: {L.pararnn_status_string(rc).decode()}")
+    return SolveResult(out, info.iters, STATUS[info.status], info.delta, info.residual)
+
+
+def host_streamed_workspace_size(kind: str, din: int, d: int, B: int, T: int, mode: str, parts: int,
+                                 dtype: torch.dtype = torch.float32) -> int:
+    cell = make_cell(kind, din, d, dtype)
+    return int(lib().pararnn_host_streamed_workspace_size(ctypes.byref(cell), B, T, MODES[mode], parts))
+
+
+def newton_solve_host_streamed(w_ih, b_ih, w_hh, b_hh, x_host, h0_host, *, kind: str, mode: str, tol: float,
+                               lam: float = 0.0, max_iters: int = 0, parts: int = 7, out=None,
+                               workspace=None, device=None, stream=None) -> "SolveResult":
+    """The solve from and to HOST tensors with the sequence streamed through
+    the device in ``parts`` time parts (whole batch in each; clamped to
+    1 .. ceil(T / 128)), each part solved from the previous part's last states
+    while the next part's inputs are copied in and the previous part's states
+    out.  The report sums iterations over the parts."""
+    B, T, din = x_host.shape
+    d = h0_host.shape[1]
+    parts = max(1, min(int(parts), (T + 127) // 128))
+    cell = make_cell(kind, din, d, x_host.dtype)
+    L = lib()
+    m = MODES[mode]
+    need = int(L.pararnn_host_streamed_workspace_size(ctypes.byref(cell), B, T, m, parts))
+    if need == 0:
+        raise ValueError("arguments rejected by pararnn_host_streamed_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, w_hh.device if device is None else device)
+    if out is None:
+        out = torch.empty(B, T, d, dtype=torch.float32).pin_memory()
+    params = Params(_dev(w_ih, "w_ih"), _dev(b_ih, "b_ih"), _dev(w_hh, "w_hh"), _dev(b_hh, "b_hh"))
+    info = Info()
+    rc = L.pararnn_newton_solve_host_streamed(ctypes.byref(cell), ctypes.byref(params), _host(x_host, "x_host"),
+                                              _host(h0_host, "h0_host"), B, T, m, float(lam), float(tol),
+                                              int(max_iters), _host(out, "out"), ctypes.byref(info), parts,
+                                              _dev(workspace, "workspace"), workspace.numel(), _stream(stream))
+    if rc in (3, 4):
+        raise RuntimeError(f"pararnn_newton_solve_host_streamed: {L.pararnn_status_string(rc).decode()}")
     return SolveResult(out, info.iters, STATUS[info.status], info.delta, info.residual)
 
 

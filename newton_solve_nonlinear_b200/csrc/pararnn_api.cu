@@ -860,11 +860,6 @@ struct PipeIo {
     size_t in_off[3][kHostBufs] = {}, out_off[2][kHostBufs] = {};
 };
 
-// The batch in ramped parts (part_sizes) through `nbuf` staging buffers: part
-// p's inputs are copied in on one helper stream, solved on `sc` by
-// enq(p, b0, nb, buf) (returns a pararnn status), and its outputs copied out
-// on a second helper stream; pre(s_in) enqueues the copies made once per call
-// (initial states).  On return `sc` is ordered after the last copy out.
 // The pipeline's two helper streams and their events, created on a device's
 // first host-buffer call and reused by later calls on that device (creating
 // and destroying them cost a visible fraction of a short call).  A set is
@@ -934,9 +929,16 @@ void pipe_release(PipeRes *r, bool reuse) {
     g_pipe_free.push_back(r);
 }
 
-extern "C++" {  // a template: C++ linkage inside the exported block
-template <class Pre, class Enq>
-int run_pipeline(int B, int parts, int nbuf, const PipeIo &io, char *ws, cudaStream_t sc, Pre pre, Enq enq) {
+extern "C++" {  // templates: C++ linkage inside the exported block
+// The parts of `sizes` through `nbuf` staging buffers: part p's inputs are
+// copied in by cin(p, first, n, buf, s_in) on one helper stream, solved on `sc`
+// by enq(p, first, n, buf) (returns a pararnn status), and its outputs copied
+// out by cout(p, first, n, buf, s_out) on a second helper stream; `first` is
+// the part's first sequence (batch parts) or step (time parts), n its count.
+// pre(s_in) enqueues the copies made once per call (initial states).  On
+// return `sc` is ordered after the last copy out.
+template <class Pre, class In, class Enq, class Out>
+int run_parts(const std::vector<int> &sizes, int nbuf, cudaStream_t sc, Pre pre, In cin, Enq enq, Out cout) {
     constexpr int NB = kHostBufs;
     PipeRes *res = nullptr;
     cudaError_t e = pipe_acquire(&res);
@@ -950,27 +952,23 @@ int run_pipeline(int B, int parts, int nbuf, const PipeIo &io, char *ws, cudaStr
         if (e == cudaSuccess) e = cudaStreamWaitEvent(s_in, ev_edge, 0);
         if (e == cudaSuccess) e = pre(s_in);
     }
-    const std::vector<int> sizes = part_sizes(B, parts);
-    int b0 = 0;
-    for (int p = 0; p < parts && e == cudaSuccess && rc == PARARNN_OK; b0 += sizes[p], ++p) {
-        const int buf = p % nbuf, nb = sizes[p];
+    const int parts = static_cast<int>(sizes.size());
+    int first = 0;
+    for (int p = 0; p < parts && e == cudaSuccess && rc == PARARNN_OK; first += sizes[p], ++p) {
+        const int buf = p % nbuf, n = sizes[p];
         if (p >= nbuf) e = cudaStreamWaitEvent(s_in, ev_out[buf], 0);  // staging of part p-nbuf free
-        for (int a = 0; a < io.nin && e == cudaSuccess; ++a)
-            e = cudaMemcpyAsync(ws + io.in_off[a][buf], io.in[a] + b0 * io.in_row[a], nb * io.in_row[a],
-                                cudaMemcpyHostToDevice, s_in);
+        if (e == cudaSuccess) e = cin(p, first, n, buf, s_in);
         if (e == cudaSuccess) e = cudaEventRecord(ev_in[buf], s_in);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(sc, ev_in[buf], 0);
         if (e != cudaSuccess) break;
         {
             const Range range("pararnn: host-buffer part");
-            rc = enq(p, b0, nb, buf);
+            rc = enq(p, first, n, buf);
         }
         if (rc != PARARNN_OK) break;
         e = cudaEventRecord(ev_comp[buf], sc);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(s_out, ev_comp[buf], 0);
-        for (int a = 0; a < io.nout && e == cudaSuccess; ++a)
-            e = cudaMemcpyAsync(io.out[a] + b0 * io.out_row[a], ws + io.out_off[a][buf], nb * io.out_row[a],
-                                cudaMemcpyDeviceToHost, s_out);
+        if (e == cudaSuccess) e = cout(p, first, n, buf, s_out);
         if (e == cudaSuccess) e = cudaEventRecord(ev_out[buf], s_out);
     }
     if (e == cudaSuccess && rc == PARARNN_OK) {  // the caller's stream continues after the last copy out
@@ -984,18 +982,40 @@ int run_pipeline(int B, int parts, int nbuf, const PipeIo &io, char *ws, cudaStr
     if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
     return rc;
 }
+
+// The batch in ramped parts (part_sizes): whole sequences of every array in `io`.
+template <class Pre, class Enq>
+int run_pipeline(int B, int parts, int nbuf, const PipeIo &io, char *ws, cudaStream_t sc, Pre pre, Enq enq) {
+    auto cin = [&](int, int b0, int nb, int buf, cudaStream_t s) {
+        cudaError_t e = cudaSuccess;
+        for (int a = 0; a < io.nin && e == cudaSuccess; ++a)
+            e = cudaMemcpyAsync(ws + io.in_off[a][buf], io.in[a] + b0 * io.in_row[a], nb * io.in_row[a],
+                                cudaMemcpyHostToDevice, s);
+        return e;
+    };
+    auto cout = [&](int, int b0, int nb, int buf, cudaStream_t s) {
+        cudaError_t e = cudaSuccess;
+        for (int a = 0; a < io.nout && e == cudaSuccess; ++a)
+            e = cudaMemcpyAsync(io.out[a] + b0 * io.out_row[a], ws + io.out_off[a][buf], nb * io.out_row[a],
+                                cudaMemcpyDeviceToHost, s);
+        return e;
+    };
+    return run_parts(part_sizes(B, parts), nbuf, sc, pre, cin, enq, cout);
+}
 }  // extern "C++"
 
 // Wait for `sc`, read the parts' reports and fold them: the worst part
-// (statuses are ordered by severity), the largest count, delta and residual.
-int fold_reports(const pararnn_info *infos_dev, int parts, cudaStream_t sc, pararnn_info *info) {
+// (statuses are ordered by severity), the largest count (or, with sum_iters,
+// the total over parts), delta and residual.
+int fold_reports(const pararnn_info *infos_dev, int parts, cudaStream_t sc, pararnn_info *info,
+                 bool sum_iters = false) {
     std::vector<pararnn_info> host(parts);
     cudaError_t e = cudaMemcpyAsync(host.data(), infos_dev, parts * sizeof(pararnn_info), cudaMemcpyDeviceToHost, sc);
     if (e == cudaSuccess) e = cudaStreamSynchronize(sc);
     if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
     pararnn_info agg{};
     for (int p = 0; p < parts; ++p) {
-        agg.iters = host[p].iters > agg.iters ? host[p].iters : agg.iters;
+        agg.iters = sum_iters ? agg.iters + host[p].iters : (host[p].iters > agg.iters ? host[p].iters : agg.iters);
         agg.status = host[p].status > agg.status ? host[p].status : agg.status;
         agg.delta = host[p].delta > agg.delta ? host[p].delta : agg.delta;
         agg.residual = host[p].residual > agg.residual ? host[p].residual : agg.residual;
@@ -1169,6 +1189,98 @@ int pararnn_newton_solve_host(const pararnn_cell *cell, const pararnn_params *pa
     const int rc = run_pipeline(B, parts, H.nbuf, io, ws, sc, pre, enq);
     if (rc != PARARNN_OK) return rc;
     return fold_reports(infos, parts, sc, info);
+}
+
+namespace {
+
+// Steps per time part: whole 128-step units (the solvers' tile length) with the
+// ramped weights of part_sizes; the last part ends at T.  parts <= ceil(T / 128).
+std::vector<int> time_part_sizes(int T, int parts) {
+    const int units = (T + 127) / 128;
+    std::vector<int> n = part_sizes(units, parts);
+    for (int &v : n) v *= 128;
+    n.back() -= units * 128 - T;
+    return n;
+}
+
+struct StreamLayout {
+    int tmax, nbuf;  // steps of the longest part, staging buffers
+    size_t solve, xs[kHostBufs], hs[kHostBufs], h0, carry, infos, total;
+};
+
+StreamLayout stream_layout(const pararnn_cell &cell, int B, int T, int mode, int parts) {
+    StreamLayout H{};
+    for (int v : time_part_sizes(T, parts)) H.tmax = v > H.tmax ? v : H.tmax;
+    H.nbuf = parts < kHostBufs ? parts : kHostBufs;
+    const size_t es = cell.x_dtype == PARARNN_BF16 ? 2 : 4;
+    const size_t xbytes = static_cast<size_t>(B) * H.tmax * cell.din * es;
+    const size_t hbytes = static_cast<size_t>(B) * H.tmax * cell.d * 4;
+    size_t off = 0;
+    H.solve = off; off = align256(off + ws_layout(cell, B, H.tmax, mode).total);
+    for (int q = 0; q < H.nbuf; ++q) { H.xs[q] = off; off = align256(off + xbytes); }
+    for (int q = 0; q < H.nbuf; ++q) { H.hs[q] = off; off = align256(off + hbytes); }
+    H.h0 = off; off = align256(off + static_cast<size_t>(B) * cell.d * 4);
+    H.carry = off; off = align256(off + static_cast<size_t>(B) * cell.d * 4);
+    H.infos = off; off = align256(off + static_cast<size_t>(parts) * sizeof(pararnn_info));
+    H.total = off;
+    return H;
+}
+
+}  // namespace
+
+size_t pararnn_host_streamed_workspace_size(const pararnn_cell *cell, int B, int T, int mode, int parts) {
+    if (!cell_ok(cell, B, T, mode) || parts < 1 || parts > (T + 127) / 128) return 0;
+    return stream_layout(*cell, B, T, mode, parts).total;
+}
+
+int pararnn_newton_solve_host_streamed(const pararnn_cell *cell, const pararnn_params *params,
+                                       const void *x_host, const float *h0_host, int B, int T, int mode,
+                                       float lambda, float tol, int max_iters, float *h_host, pararnn_info *info,
+                                       int parts, void *workspace, size_t ws_bytes, pararnn_stream stream) {
+    if (!cell_ok(cell, B, T, mode) || parts < 1 || parts > (T + 127) / 128 || !params || !x_host ||
+        !h0_host || !h_host || !workspace || !aligned(workspace, 256))
+        return PARARNN_INVALID_ARG;
+    const StreamLayout H = stream_layout(*cell, B, T, mode, parts);
+    if (ws_bytes < H.total) return PARARNN_INVALID_ARG;
+    char *ws = static_cast<char *>(workspace);
+    const size_t es = cell->x_dtype == PARARNN_BF16 ? 2 : 4;
+    const size_t xstep = static_cast<size_t>(cell->din) * es, hstep = static_cast<size_t>(cell->d) * 4;
+    const std::vector<int> sizes = time_part_sizes(T, parts);
+    cudaStream_t sc = reinterpret_cast<cudaStream_t>(stream);
+    float *h0_dev = reinterpret_cast<float *>(ws + H.h0), *carry = reinterpret_cast<float *>(ws + H.carry);
+    pararnn_info *infos = reinterpret_cast<pararnn_info *>(ws + H.infos);
+    const char *xh = static_cast<const char *>(x_host);
+    char *hh = reinterpret_cast<char *>(h_host);
+    // the cap of the whole sequence's solve (T + 1 by default), as for the chunked solve
+    const int cap = max_iters > 0 ? max_iters : T + 1;
+    auto pre = [&](cudaStream_t s_in) {
+        return cudaMemcpyAsync(h0_dev, h0_host, B * hstep, cudaMemcpyHostToDevice, s_in);
+    };
+    // steps [t0, t0 + n) of every sequence: rows of the host arrays, packed [B, n, .] in staging
+    auto cin = [&](int, int t0, int n, int buf, cudaStream_t s) {
+        return cudaMemcpy2DAsync(ws + H.xs[buf], n * xstep, xh + t0 * xstep, T * xstep, n * xstep, B,
+                                 cudaMemcpyHostToDevice, s);
+    };
+    auto enq = [&](int p, int, int n, int buf) {
+        const float *hin = h0_dev;
+        if (p > 0) {  // the state entering the part: each sequence's last state of the part before
+            const int pb = (p - 1) % H.nbuf, pn = sizes[p - 1];
+            if (cudaMemcpy2DAsync(carry, hstep, ws + H.hs[pb] + (pn - 1) * hstep, pn * hstep, hstep, B,
+                                  cudaMemcpyDeviceToDevice, sc) != cudaSuccess)
+                return static_cast<int>(PARARNN_CUDA_ERROR);
+            hin = carry;
+        }
+        return solve_enqueue(cell, params, ws + H.xs[buf], hin, B, n, mode, lambda, tol, cap,
+                             reinterpret_cast<float *>(ws + H.hs[buf]), infos + p, ws + H.solve,
+                             ws_layout(*cell, B, n, mode).total, stream);
+    };
+    auto cout = [&](int, int t0, int n, int buf, cudaStream_t s) {
+        return cudaMemcpy2DAsync(hh + t0 * hstep, T * hstep, ws + H.hs[buf], n * hstep, n * hstep, B,
+                                 cudaMemcpyDeviceToHost, s);
+    };
+    const int rc = run_parts(sizes, H.nbuf, sc, pre, cin, enq, cout);
+    if (rc != PARARNN_OK) return rc;
+    return fold_reports(infos, parts, sc, info, true);
 }
 
 size_t pararnn_lstm_host_workspace_size(const pararnn_cell *cell, int B, int T, int parts) {

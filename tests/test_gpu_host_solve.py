@@ -106,3 +106,96 @@ def test_device_tensor_rejected():
     with pytest.raises(ValueError):
         binding.newton_solve_host(*_weights(w), w.x.cuda(), w.h0.float(), kind=w.kind,
                                   mode="QUASI", tol=w.tol)
+
+
+# ---- the streamed solve: time parts, every sequence in each part ----------
+
+def _time_parts(T, parts):
+    """The documented split: 128-step units weighted min(p + 1, parts - p, 4),
+    largest remainder (ties to the earlier part), at least one unit each, the
+    last part ending at T."""
+    units = (T + 127) // 128
+    w = [min(p + 1, parts - p, 4) for p in range(parts)]
+    W = sum(w)
+    n = [units * v // W for v in w]
+    rem = sorted(range(parts), key=lambda i: (-(units * w[i] % W), i))
+    for r in range(units - sum(n)):
+        n[rem[r % parts]] += 1
+    for i in range(parts):
+        while n[i] == 0:
+            j = max(range(parts), key=lambda q: (n[q], -q))
+            n[j] -= 1
+            n[i] += 1
+    n = [v * 128 for v in n]
+    n[-1] -= units * 128 - T
+    return n
+
+
+def _streamed(w, mode, parts, **kw):
+    x = w.x.contiguous().pin_memory()
+    h0 = w.h0.float().contiguous().pin_memory()
+    kw.setdefault("tol", w.tol)
+    return binding.newton_solve_host_streamed(*_weights(w), x, h0, kind=w.kind, mode=mode, parts=parts, **kw)
+
+
+def test_streamed_one_part_equals_device_solve():
+    w = make_workload("untrained", B=3, T=2500, h0_std=0.5)
+    r = _streamed(w, "QUASI", 1)
+    r_dev = binding.solve_workload(w, "QUASI")
+    assert r.status == r_dev.status == "OK" and abs(r.iters - r_dev.iters) <= 1
+    assert _same_run(r.h, r_dev.h, atol=1e-6 if r.iters == r_dev.iters else w.tol)
+
+
+@pytest.mark.parametrize("name,over,mode,lam,parts", [
+    ("untrained", dict(B=3, T=1000, h0_std=0.5), "QUASI", 0.0, 3),
+    ("dense_deer", dict(B=2, T=1500, bias_std=0.2), "DEER", 0.0, 4),
+    ("near_unstable", dict(B=2, T=700), "QUASI_ELK", 0.5, 3),
+    ("diag", dict(B=2, T=900, d=128, din=128), "QUASI", 0.0, 5),
+])
+def test_streamed_fixed_iterations_match_oracle_per_part(name, over, mode, lam, parts):
+    """tol 0, two iterations: each part is the oracle's two-iteration solve of
+    its window, started from the state the part before it left (read from the
+    result, so that each part is checked on its own)."""
+    w = make_workload(name, **over)
+    c, x, h0 = _oracle(w)
+    r = _streamed(w, mode, parts, tol=0.0, max_iters=2, lam=lam)
+    sizes = _time_parts(w.T, parts)
+    assert sum(sizes) == w.T and r.iters == 2 * parts and r.status == "NOT_CONVERGED"
+    got = r.h.double().numpy()
+    t0, hin = 0, h0
+    for n in sizes:
+        if mode in ("ELK", "QUASI_ELK"):
+            ref = oracle.elk_solve(c, x[:, t0:t0 + n], hin, mode, lam, 0.0, max_iters=2, record=True)
+        else:
+            ref = oracle.newton_solve(c, x[:, t0:t0 + n], hin, mode, 0.0, max_iters=2, record=True)
+        err = np.max(np.abs(got[:, t0:t0 + n] - ref["iterates"][1]))
+        assert err <= 5e-5, (t0, n, err)
+        hin = got[:, t0 + n - 1]
+        t0 += n
+
+
+@pytest.mark.parametrize("name,over,mode,lam,parts", [
+    ("untrained", dict(B=5, T=3000, h0_std=0.5), "QUASI", 0.0, 7),
+    ("untrained", dict(B=4, T=1000, x_dtype=torch.bfloat16, w_dtype=torch.bfloat16), "DEER", 0.0, 3),
+    ("diag", dict(B=3, T=777, d=128, din=128), "DEER", 0.0, 4),
+    ("dense_deer", dict(B=3, T=2000), "DEER", 0.0, 6),
+    ("near_unstable", dict(B=2, T=600), "ELK", 0.3, 2),
+])
+def test_streamed_converged_states_match_rollout(name, over, mode, lam, parts):
+    w = make_workload(name, **over)
+    c, x, h0 = _oracle(w)
+    tol = 1e-6 if mode in ("ELK", "QUASI_ELK") else w.tol
+    r = _streamed(w, mode, parts, lam=lam, tol=tol)
+    assert r.status == "OK"
+    assert np.max(np.abs(r.h.double().numpy() - rollout(c, x, h0))) <= 1e-4
+
+
+def test_streamed_parts_bounds():
+    w = make_workload("untrained", B=2, T=300)
+    out = torch.full((2, 300, 64), float("nan")).pin_memory()
+    r = _streamed(w, "QUASI", 99, out=out)  # clamped to ceil(300 / 128) = 3 parts
+    assert r.h.data_ptr() == out.data_ptr() and r.status == "OK"
+    c, x, h0 = _oracle(w)
+    assert np.max(np.abs(out.double().numpy() - rollout(c, x, h0))) <= 1e-4
+    assert binding.host_streamed_workspace_size("dense", 64, 64, 2, 300, "QUASI", 4) == 0
+    assert binding.host_streamed_workspace_size("dense", 64, 64, 2, 300, "QUASI", 3) > 0
