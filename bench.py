@@ -532,22 +532,28 @@ def run_lstm(args):
     max_ms = max_over_ranks(sum(ms), dev)
     value = job_value(states, args.steps, world, max_ms)
     # end to end through the public host-buffer call: x, c0, h0 from page-locked
-    # host memory, (c, h) back; the library overlaps the copies with the parts' solves
+    # host memory, (c, h) back; the library streams the sequence through the
+    # device in time parts and overlaps the copies with the parts' solves
     hx, hc0, hh0 = w.x.pin_memory(), w.c0.float().pin_memory(), w.h0.float().pin_memory()
     hc, hh = torch.empty(B, T, D).pin_memory(), torch.empty(B, T, D).pin_memory()
-    parts = max(1, min(E2E_PARTS, B))
-    ws_host = binding.alloc_workspace(int(binding.lib().pararnn_lstm_host_workspace_size(
-        binding.make_cell("lstm_diag", w.din, D, w.x.dtype), B, T, parts)), dev)
-    e2e_step = lambda: binding.lstm_solve_host(g(w.w_ih), g(w.b_ih), g(w.u), g(w.b_hh), hx, hc0, hh0, tol=w.tol,
-                                               parts=parts, out=(hc, hh), workspace=ws_host, stream=stream)
+    parts = max(1, min(E2E_PARTS, (T + 127) // 128))
+    ws_host = binding.alloc_workspace(binding.lstm_host_streamed_workspace_size(w.din, D, B, T, parts, w.x.dtype),
+                                      dev)
+    e2e_step = lambda: binding.lstm_solve_host_streamed(g(w.w_ih), g(w.b_ih), g(w.u), g(w.b_hh), hx, hc0, hh0,
+                                                        tol=w.tol, parts=parts, out=(hc, hh), workspace=ws_host,
+                                                        stream=stream)
     e2e_step()
     e2e_steps = max(1, min(args.steps, 3))
     barrier()
     torch.cuda.synchronize()
     ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ea.record(stream)
+    e2e_iters = []
     for _ in range(e2e_steps):
-        e2e_step()
+        _, _, r_e2e = e2e_step()
+        if r_e2e.status != "OK":
+            raise SystemExit(f"lstm: end-to-end solve status {r_e2e.status}")
+        e2e_iters.append(r_e2e.iters)
     eb.record(stream)
     torch.cuda.synchronize()
     e2e_value = job_value(states, e2e_steps, world, max_over_ranks(ea.elapsed_time(eb), dev))
@@ -573,7 +579,8 @@ def run_lstm(args):
                      "peak_kind": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"},
         "e2e": {"value": e2e_value, "unit": UNIT,
                 "h2d_bytes_per_step": w.x.numel() * w.x.element_size() + 2 * B * D * 4,
-                "d2h_bytes_per_step": 2 * states * 4 + 16 * parts, "parts": parts},
+                "d2h_bytes_per_step": 2 * states * 4 + 16 * parts, "parts": parts, "split": "time",
+                "iters_summed_over_parts": e2e_iters, "copy_gbs": copy_bandwidth(dev)},
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
     }

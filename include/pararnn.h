@@ -650,6 +650,27 @@ PARARNN_API int pararnn_lstm_solve_host(const pararnn_cell *cell, const pararnn_
  * part's solve workspace, three parts' staging, the initial states), or 0. */
 PARARNN_API size_t pararnn_lstm_host_workspace_size(const pararnn_cell *cell, int B, int T, int parts);
 
+/*
+ * pararnn_lstm_solve_host_streamed -- the LSTM solve from and to HOST memory
+ * with the sequence streamed through the device in `parts` consecutive time
+ * parts (every sequence in each), as pararnn_newton_solve_host_streamed: part
+ * p starts from each sequence's last (c, h) of part p-1 ((c0, h0) for the
+ * first) and is solved to `tol` on its own while part p+1's inputs are copied
+ * in and part p-1's (c, h) out.  Same ramped split in 128-step units.
+ * Arguments as for pararnn_lstm_solve_host, except 1 <= parts <= ceil(T / 128),
+ * max_iters caps each part (<= 0: T + 1), the workspace is
+ * pararnn_lstm_host_streamed_workspace_size bytes, and the report sums
+ * iterations over the parts (worst status, largest delta and residual).
+ */
+PARARNN_API int pararnn_lstm_solve_host_streamed(const pararnn_cell *cell, const pararnn_params *params,
+                                                 const void *x_host, const float *c0_host, const float *h0_host,
+                                                 int B, int T, float tol, int max_iters, float *c_host,
+                                                 float *h_host, pararnn_info *info, int parts, void *workspace,
+                                                 size_t ws_bytes, pararnn_stream stream);
+
+/* Workspace bytes of pararnn_lstm_solve_host_streamed; 0 if the arguments are rejected. */
+PARARNN_API size_t pararnn_lstm_host_streamed_workspace_size(const pararnn_cell *cell, int B, int T, int parts);
+
 /* pararnn_status_string -- a static, human-readable name of a status code. */
 PARARNN_API const char *pararnn_status_string(int status);
 

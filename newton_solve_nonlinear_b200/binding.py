@@ -32,7 +32,8 @@ EXPORTS = ("pararnn_workspace_size", "pararnn_newton_solve", "pararnn_newton_sol
            "pararnn_lstm_host_workspace_size", "pararnn_adjoint_host", "pararnn_adjoint_host_workspace_size",
            "pararnn_newton_solve_trace", "pararnn_test_withheld_publish", "pararnn_adjoint_exact",
            "pararnn_adjoint_exact_workspace_size", "pararnn_newton_solve_host_streamed",
-           "pararnn_host_streamed_workspace_size")
+           "pararnn_host_streamed_workspace_size", "pararnn_lstm_solve_host_streamed",
+           "pararnn_lstm_host_streamed_workspace_size")
 
 
 class Cell(ctypes.Structure):
@@ -120,6 +121,10 @@ def lib() -> ctypes.CDLL:
         L.pararnn_lstm_solve_host.restype = ci
         L.pararnn_lstm_host_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci, ci]
         L.pararnn_lstm_host_workspace_size.restype = sz
+        L.pararnn_lstm_solve_host_streamed.argtypes = L.pararnn_lstm_solve_host.argtypes
+        L.pararnn_lstm_solve_host_streamed.restype = ci
+        L.pararnn_lstm_host_streamed_workspace_size.argtypes = [ctypes.POINTER(Cell), ci, ci, ci]
+        L.pararnn_lstm_host_streamed_workspace_size.restype = sz
         L.pararnn_adjoint_host.argtypes = [ctypes.POINTER(Cell), ctypes.POINTER(Params), vp, vp, vp, vp, ci, ci,
                                            vp, vp, vp, vp, ci, vp, sz, vp]
         L.pararnn_adjoint_host.restype = ci
@@ -460,6 +465,40 @@ def lstm_solve_host(w_ih, b_ih, u, b_hh, x_host, c0_host, h0_host, *, tol: float
     if rc in (3, 4):
         raise RuntimeError(f"pararnn_lstm_solve_host: {L.pararnn_status_string(rc).decode()}")
     return c, h, SolveResult(h, info.iters, STATUS[info.status], info.delta, info.residual)
+
+
+def lstm_solve_host_streamed(w_ih, b_ih, u, b_hh, x_host, c0_host, h0_host, *, tol: float, max_iters: int = 0,
+                             parts: int = 7, out=None, workspace=None, device=None, stream=None):
+    """The LSTM solve from and to HOST tensors with the sequence streamed
+    through the device in ``parts`` time parts (clamped to 1 .. ceil(T / 128));
+    the report sums iterations over the parts.  Returns (c, h, SolveResult)."""
+    B, T, din = x_host.shape
+    d = h0_host.shape[1]
+    parts = max(1, min(int(parts), (T + 127) // 128))
+    cell = make_cell("lstm_diag", din, d, x_host.dtype)
+    L = lib()
+    need = int(L.pararnn_lstm_host_streamed_workspace_size(ctypes.byref(cell), B, T, parts))
+    if need == 0:
+        raise ValueError("arguments rejected by pararnn_lstm_host_streamed_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, u.device if device is None else device)
+    c, h = out if out is not None else (torch.empty(B, T, d, dtype=torch.float32).pin_memory(),
+                                        torch.empty(B, T, d, dtype=torch.float32).pin_memory())
+    params = Params(_dev(w_ih, "w_ih"), _dev(b_ih, "b_ih"), _dev(u, "u"), _dev(b_hh, "b_hh"))
+    info = Info()
+    rc = L.pararnn_lstm_solve_host_streamed(ctypes.byref(cell), ctypes.byref(params), _host(x_host, "x_host"),
+                                            _host(c0_host, "c0_host"), _host(h0_host, "h0_host"), B, T, float(tol),
+                                            int(max_iters), _host(c, "c"), _host(h, "h"), ctypes.byref(info), parts,
+                                            _dev(workspace, "workspace"), workspace.numel(), _stream(stream))
+    if rc in (3, 4):
+        raise RuntimeError(f"pararnn_lstm_solve_host_streamed: {L.pararnn_status_string(rc).decode()}")
+    return c, h, SolveResult(h, info.iters, STATUS[info.status], info.delta, info.residual)
+
+
+def lstm_host_streamed_workspace_size(din: int, d: int, B: int, T: int, parts: int,
+                                      dtype: torch.dtype = torch.bfloat16) -> int:
+    cell = make_cell("lstm_diag", din, d, dtype)
+    return int(lib().pararnn_lstm_host_streamed_workspace_size(ctypes.byref(cell), B, T, parts))
 
 
 def adjoint_workspace_size(d: int, B: int, T: int, kind: str = "diag") -> int:

@@ -1283,6 +1283,107 @@ int pararnn_newton_solve_host_streamed(const pararnn_cell *cell, const pararnn_p
     return fold_reports(infos, parts, sc, info, true);
 }
 
+namespace {
+
+struct LstmStreamLayout {
+    int tmax, nbuf;
+    size_t solve, xs[kHostBufs], cs[kHostBufs], hs[kHostBufs], c0, h0, cc, hc, infos, total;
+};
+
+LstmStreamLayout lstm_stream_layout(const pararnn_cell &cell, int B, int T, int parts) {
+    LstmStreamLayout H{};
+    for (int v : time_part_sizes(T, parts)) H.tmax = v > H.tmax ? v : H.tmax;
+    H.nbuf = parts < kHostBufs ? parts : kHostBufs;
+    const size_t es = cell.x_dtype == PARARNN_BF16 ? 2 : 4;
+    const size_t xbytes = static_cast<size_t>(B) * H.tmax * cell.din * es;
+    const size_t sbytes = static_cast<size_t>(B) * H.tmax * cell.d * 4;
+    const size_t bd = static_cast<size_t>(B) * cell.d * 4;
+    size_t off = 0;
+    H.solve = off; off = align256(off + lstm_layout(cell, B, H.tmax).total);
+    for (int q = 0; q < H.nbuf; ++q) { H.xs[q] = off; off = align256(off + xbytes); }
+    for (int q = 0; q < H.nbuf; ++q) { H.cs[q] = off; off = align256(off + sbytes); }
+    for (int q = 0; q < H.nbuf; ++q) { H.hs[q] = off; off = align256(off + sbytes); }
+    H.c0 = off; off = align256(off + bd);
+    H.h0 = off; off = align256(off + bd);
+    H.cc = off; off = align256(off + bd);
+    H.hc = off; off = align256(off + bd);
+    H.infos = off; off = align256(off + static_cast<size_t>(parts) * sizeof(pararnn_info));
+    H.total = off;
+    return H;
+}
+
+}  // namespace
+
+size_t pararnn_lstm_host_streamed_workspace_size(const pararnn_cell *cell, int B, int T, int parts) {
+    if (!lstm_cell_ok(cell, B, T) || parts < 1 || parts > (T + 127) / 128) return 0;
+    return lstm_stream_layout(*cell, B, T, parts).total;
+}
+
+int pararnn_lstm_solve_host_streamed(const pararnn_cell *cell, const pararnn_params *params, const void *x_host,
+                                     const float *c0_host, const float *h0_host, int B, int T, float tol,
+                                     int max_iters, float *c_host, float *h_host, pararnn_info *info, int parts,
+                                     void *workspace, size_t ws_bytes, pararnn_stream stream) {
+    if (!lstm_cell_ok(cell, B, T) || parts < 1 || parts > (T + 127) / 128 || !params || !params->w_ih ||
+        !params->b_ih || !params->w_hh || !params->b_hh || !x_host || !c0_host || !h0_host || !c_host || !h_host ||
+        !workspace || !aligned(workspace, 256) || !(tol >= 0.f) || !std::isfinite(tol))
+        return PARARNN_INVALID_ARG;
+    const void *ptrs[] = {params->w_ih, params->b_ih, params->w_hh, params->b_hh};
+    for (const void *q : ptrs)
+        if (!aligned(q, 16)) return PARARNN_INVALID_ARG;
+    const LstmStreamLayout H = lstm_stream_layout(*cell, B, T, parts);
+    if (ws_bytes < H.total) return PARARNN_INVALID_ARG;
+    char *ws = static_cast<char *>(workspace);
+    const size_t es = cell->x_dtype == PARARNN_BF16 ? 2 : 4;
+    const size_t xstep = static_cast<size_t>(cell->din) * es, sstep = static_cast<size_t>(cell->d) * 4;
+    const std::vector<int> sizes = time_part_sizes(T, parts);
+    cudaStream_t sc = reinterpret_cast<cudaStream_t>(stream);
+    float *c0_dev = reinterpret_cast<float *>(ws + H.c0), *h0_dev = reinterpret_cast<float *>(ws + H.h0);
+    float *cc = reinterpret_cast<float *>(ws + H.cc), *hc = reinterpret_cast<float *>(ws + H.hc);
+    pararnn_info *infos = reinterpret_cast<pararnn_info *>(ws + H.infos);
+    const char *xh = static_cast<const char *>(x_host);
+    char *ch = reinterpret_cast<char *>(c_host), *hh = reinterpret_cast<char *>(h_host);
+    const int cap = max_iters > 0 ? max_iters : T + 1;  // the whole sequence's cap
+    auto pre = [&](cudaStream_t s_in) {
+        cudaError_t e = cudaMemcpyAsync(c0_dev, c0_host, B * sstep, cudaMemcpyHostToDevice, s_in);
+        if (e == cudaSuccess) e = cudaMemcpyAsync(h0_dev, h0_host, B * sstep, cudaMemcpyHostToDevice, s_in);
+        return e;
+    };
+    auto cin = [&](int, int t0, int n, int buf, cudaStream_t s) {
+        return cudaMemcpy2DAsync(ws + H.xs[buf], n * xstep, xh + t0 * xstep, T * xstep, n * xstep, B,
+                                 cudaMemcpyHostToDevice, s);
+    };
+    auto enq = [&](int p, int, int n, int buf) {
+        const float *cin0 = c0_dev, *hin0 = h0_dev;
+        cudaError_t e = cudaSuccess;
+        if (p > 0) {  // (c, h) entering the part: each sequence's last state of the part before
+            const int pb = (p - 1) % H.nbuf, pn = sizes[p - 1];
+            e = cudaMemcpy2DAsync(cc, sstep, ws + H.cs[pb] + (pn - 1) * sstep, pn * sstep, sstep, B,
+                                  cudaMemcpyDeviceToDevice, sc);
+            if (e == cudaSuccess)
+                e = cudaMemcpy2DAsync(hc, sstep, ws + H.hs[pb] + (pn - 1) * sstep, pn * sstep, sstep, B,
+                                      cudaMemcpyDeviceToDevice, sc);
+            cin0 = cc;
+            hin0 = hc;
+        }
+        if (e == cudaSuccess)
+            e = lstm_enqueue(cell, params, ws + H.xs[buf], cin0, hin0, B, n, tol, cap,
+                             reinterpret_cast<float *>(ws + H.cs[buf]), reinterpret_cast<float *>(ws + H.hs[buf]),
+                             infos + p, ws + H.solve, sc);
+        return e == cudaSuccess ? PARARNN_OK : PARARNN_CUDA_ERROR;
+    };
+    auto cout = [&](int, int t0, int n, int buf, cudaStream_t s) {
+        cudaError_t e = cudaMemcpy2DAsync(ch + t0 * sstep, T * sstep, ws + H.cs[buf], n * sstep, n * sstep, B,
+                                          cudaMemcpyDeviceToHost, s);
+        if (e == cudaSuccess)
+            e = cudaMemcpy2DAsync(hh + t0 * sstep, T * sstep, ws + H.hs[buf], n * sstep, n * sstep, B,
+                                  cudaMemcpyDeviceToHost, s);
+        return e;
+    };
+    const int rc = run_parts(sizes, H.nbuf, sc, pre, cin, enq, cout);
+    if (rc != PARARNN_OK) return rc;
+    return fold_reports(infos, parts, sc, info, true);
+}
+
 size_t pararnn_lstm_host_workspace_size(const pararnn_cell *cell, int B, int T, int parts) {
     if (!lstm_cell_ok(cell, B, T) || parts < 1 || parts > B) return 0;
     return lstm_host_layout(*cell, B, T, parts).total;

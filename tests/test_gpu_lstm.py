@@ -112,3 +112,66 @@ def test_host_buffer_solve(B, T, d, din, parts):
         assert abs(rd.iters - r.iters) <= 1
         tol = 1e-6 if rd.iters == r.iters else w.tol
         assert _same_run(cd, c, tol) and _same_run(hd, h, tol)
+
+
+def _time_parts(T, parts):
+    """The documented split of the streamed calls: 128-step units weighted
+    min(p + 1, parts - p, 4), largest remainder (ties to the earlier part), at
+    least one unit each, the last part ending at T."""
+    units = (T + 127) // 128
+    w = [min(p + 1, parts - p, 4) for p in range(parts)]
+    W = sum(w)
+    n = [units * v // W for v in w]
+    rem = sorted(range(parts), key=lambda i: (-(units * w[i] % W), i))
+    for r in range(units - sum(n)):
+        n[rem[r % parts]] += 1
+    n = [v * 128 for v in n]
+    n[-1] -= units * 128 - T
+    return n
+
+
+def _streamed(w, parts, **kw):
+    dev = lambda t: t.cuda().contiguous()
+    pin = lambda t: t.contiguous().pin_memory()
+    return binding.lstm_solve_host_streamed(dev(w.w_ih), dev(w.b_ih), dev(w.u), dev(w.b_hh), pin(w.x), pin(w.c0),
+                                            pin(w.h0), tol=kw.pop("tol", w.tol), parts=parts, **kw)
+
+
+@pytest.mark.parametrize("B,T,d,din,dtype,parts", [(3, 1000, 64, 32, torch.float32, 3),
+                                                   (2, 777, 128, 128, torch.bfloat16, 5),
+                                                   (4, 300, 68, 12, torch.float32, 1)])
+def test_streamed_host_solve_converges_to_rollout(B, T, d, din, dtype, parts):
+    """Time parts, every sequence in each, each part started from the (c, h)
+    the part before it left: converged (c, h) within 1e-4 of the fp64 rollout;
+    with one part the call is the device solve (fp32 rounding)."""
+    w = make_lstm_workload(B=B, T=T, d=d, din=din, x_dtype=dtype, bias_std=0.3, state_std=0.5, seed=T + parts)
+    c, h, r = _streamed(w, parts)
+    assert r.status == "OK" and not c.is_cuda
+    cell, x, c0, h0 = _oracle(w)
+    cr, hr = lstm_rollout(cell, x, c0, h0)
+    assert np.max(np.abs(c.double().numpy() - cr)) <= 1e-4
+    assert np.max(np.abs(h.double().numpy() - hr)) <= 1e-4
+    if parts == 1:
+        cd, hd, rd = _solve(w)
+        assert abs(rd.iters - r.iters) <= 1
+        tol = 1e-6 if rd.iters == r.iters else w.tol
+        assert _same_run(cd, c, tol) and _same_run(hd, h, tol)
+
+
+def test_streamed_host_solve_fixed_iterations_per_part():
+    """tol 0, two iterations: each part equals the oracle's two-iteration solve
+    of its window from the (c, h) the result holds at the part's start."""
+    w = make_lstm_workload(B=2, T=600, d=64, din=16, x_dtype=torch.float32, bias_std=0.3, state_std=0.5, seed=9)
+    parts = 4
+    c, h, r = _streamed(w, parts, tol=0.0, max_iters=2)
+    assert r.iters == 2 * parts and r.status == "NOT_CONVERGED"
+    cell, x, c0, h0 = _oracle(w)
+    gc, gh = c.double().numpy(), h.double().numpy()
+    t0, cin, hin = 0, c0, h0
+    for n in _time_parts(w.T, parts):
+        ref = lstm_newton_solve(cell, x[:, t0:t0 + n], cin, hin, 0.0, max_iters=2, record=True)
+        rc, rh = ref["iterates"][1]
+        assert np.max(np.abs(gc[:, t0:t0 + n] - rc)) <= 2e-5
+        assert np.max(np.abs(gh[:, t0:t0 + n] - rh)) <= 2e-5
+        cin, hin = gc[:, t0 + n - 1], gh[:, t0 + n - 1]
+        t0 += n
