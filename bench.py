@@ -539,7 +539,8 @@ def run_lstm(args):
     parts = max(1, min(E2E_PARTS, (T + 127) // 128))
     ws_host = binding.alloc_workspace(binding.lstm_host_streamed_workspace_size(w.din, D, B, T, parts, w.x.dtype),
                                       dev)
-    e2e_step = lambda: binding.lstm_solve_host_streamed(g(w.w_ih), g(w.b_ih), g(w.u), g(w.b_hh), hx, hc0, hh0,
+    # the weights stay resident on the device, as in the device-timed steps
+    e2e_step = lambda: binding.lstm_solve_host_streamed(w_ih, b_ih, u, b_hh, hx, hc0, hh0,
                                                         tol=w.tol, parts=parts, out=(hc, hh), workspace=ws_host,
                                                         stream=stream)
     e2e_step()
