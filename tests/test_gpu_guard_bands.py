@@ -247,3 +247,49 @@ def test_chunked_and_host_guard_bands():
     assert r.status == "OK" and _finite(oh2.t) and _close(oh2.t, ref.h, 1e-4)
     for g in (xh, h0h, oh2, wss):
         assert g.bands_intact()
+
+
+def test_host_lstm_and_adjoint_guard_bands():
+    """The host-buffer LSTM calls (batch parts and time parts) and the
+    host-buffer backward pass, with banded host and device arrays."""
+    w = make_lstm_workload(B=3, T=300, d=64, din=16, seed=13, x_dtype=torch.float32, bias_std=0.3, state_std=0.5)
+    dev = [getattr(w, k).cuda().contiguous() for k in ("w_ih", "b_ih", "u", "b_hh")]
+    hin = {k: Guarded(tuple(getattr(w, k).shape), torch.float32, device="cpu", init=getattr(w, k), pinned=True)
+           for k in ("x", "c0", "h0")}
+    rc, rh, _ = binding.lstm_solve(*dev, w.x.cuda(), w.c0.cuda(), w.h0.cuda(), tol=w.tol)
+    for streamed in (False, True):
+        c = Guarded((w.B, w.T, w.d), torch.float32, device="cpu", pinned=True)
+        h = Guarded((w.B, w.T, w.d), torch.float32, device="cpu", pinned=True)
+        if streamed:
+            ws = _ws(binding.lstm_host_streamed_workspace_size(w.din, w.d, w.B, w.T, 3, torch.float32))
+            _, _, r = binding.lstm_solve_host_streamed(*dev, hin["x"].t, hin["c0"].t, hin["h0"].t, tol=w.tol,
+                                                       parts=3, out=(c.t, h.t), workspace=ws.t)
+        else:
+            cell = binding.make_cell("lstm_diag", w.din, w.d, torch.float32)
+            ws = _ws(int(binding.lib().pararnn_lstm_host_workspace_size(ctypes.byref(cell), w.B, w.T, 2)))
+            _, _, r = binding.lstm_solve_host(*dev, hin["x"].t, hin["c0"].t, hin["h0"].t, tol=w.tol, parts=2,
+                                              out=(c.t, h.t), workspace=ws.t)
+        assert r.status == "OK" and _finite(c.t, h.t)
+        assert _close(c.t, rc, 1e-4) and _close(h.t, rh, 1e-4)
+        for g in (*hin.values(), c, h, ws):
+            assert g.bands_intact()
+
+    B, T, D = 3, 200, 48
+    arrs = _adjoint_inputs(B, T, D, True, seed=21)
+    w_hh, b_hh = arrs[0].cuda(), arrs[1].cuda()
+    hP, hh0, hh, hdh = (Guarded(tuple(a.shape), torch.float32, device="cpu", init=a, pinned=True)
+                        for a in (arrs[2], arrs[3], arrs[4], arrs[5]))
+    outs = {"dP": Guarded(tuple(arrs[2].shape), torch.float32, device="cpu", pinned=True),
+            "dh0": Guarded(tuple(arrs[3].shape), torch.float32, device="cpu", pinned=True),
+            "dw_hh": Guarded(tuple(arrs[0].shape), torch.float32, device="cpu", pinned=True),
+            "db_hh": Guarded(tuple(arrs[1].shape), torch.float32, device="cpu", pinned=True)}
+    cell = binding.make_cell("dense", 1, D, torch.float32)
+    ws = _ws(int(binding.lib().pararnn_adjoint_host_workspace_size(ctypes.byref(cell), B, T, 2)))
+    binding.adjoint_host(w_hh, b_hh, hP.t, hh0.t, hh.t, hdh.t, parts=2, out={k: g.t for k, g in outs.items()},
+                         workspace=ws.t)
+    ref = binding.adjoint(*(a.cuda() for a in arrs), check=True)
+    for k, g in outs.items():
+        assert _finite(g.t), k
+        assert _close(g.t, ref[k], 1e-5), k
+    for g in (hP, hh0, hh, hdh, *outs.values(), ws):
+        assert g.bands_intact()
