@@ -199,3 +199,18 @@ def test_streamed_parts_bounds():
     assert np.max(np.abs(out.double().numpy() - rollout(c, x, h0))) <= 1e-4
     assert binding.host_streamed_workspace_size("dense", 64, 64, 2, 300, "QUASI", 4) == 0
     assert binding.host_streamed_workspace_size("dense", 64, 64, 2, 300, "QUASI", 3) > 0
+
+
+@pytest.mark.parametrize("name,over,mode,parts", [("untrained", {}, "QUASI", 7),
+                                                  ("diag", {}, "QUASI", 7)])
+def test_streamed_full_size_sampled(name, over, mode, parts):
+    """The streamed host-buffer solve at the benchmark's full size and part
+    count (the call the end-to-end number goes through): every part converged,
+    whole sampled sequences within 1e-4 of the fp64 rollout."""
+    w = make_workload(name, **over)
+    r = _streamed(w, mode, parts)
+    assert r.status == "OK"
+    c = GRU.from_workload(w)
+    for b in (0, w.B - 1):
+        want = rollout(c, w.x[b:b + 1].double().numpy(), w.h0[b:b + 1].double().numpy())
+        assert np.max(np.abs(r.h[b:b + 1].double().numpy() - want)) <= 1e-4
