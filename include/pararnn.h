@@ -454,6 +454,36 @@ PARARNN_API int pararnn_affine_scan(const float *A, const float *b, const float 
 PARARNN_API int pararnn_affine_scan_status(const void *workspace, pararnn_stream stream);
 
 /*
+ * pararnn_affine_scan_host -- the same scan from and to HOST memory, streamed
+ * through the device in `parts` consecutive time parts (every sequence in
+ * each): part p is scanned from each sequence's last state of part p-1 (h0 for
+ * the first), which is exact, since the scan's carry across a part boundary is
+ * that state (ParaRNN summary, "Newton's Iteration": forward substitution
+ * over the time steps).  While part p is scanned on `stream`, part p+1's A and
+ * b are copied in and part p-1's h out on two helper streams (as in
+ * pararnn_newton_solve_host_streamed, with the same ramped split in 128-step
+ * units).  The results equal pararnn_affine_scan's up to the association order
+ * of fp32 products.
+ *   A_host     HOST [B, T, D] (dense = 0) or [B, T, D, D] (dense = 1) float.
+ *   b_host     HOST [B, T, D] float.   h0_host  HOST [B, D] float.
+ *   h_host     HOST [B, T, D] float, output.  Page-locked host memory lets the
+ *              copies overlap; pageable memory is accepted.
+ *   parts      1 <= parts <= ceil(T / 128).
+ *   workspace  DEVICE, >= pararnn_affine_scan_host_workspace_size(B, T, D,
+ *              dense, parts) bytes, 256-byte aligned.
+ *   stream     work queued on it before the call runs first; on return
+ *              everything has completed (the call synchronises `stream`).
+ * Returns PARARNN_OK, PARARNN_TIMEOUT (a part's bounded look-back gave up;
+ * h_host unreliable), INVALID_ARG or CUDA_ERROR.
+ */
+PARARNN_API int pararnn_affine_scan_host(const float *A_host, const float *b_host, const float *h0_host, int B,
+                                         int T, int D, int dense, float *h_host, int parts, void *workspace,
+                                         size_t ws_bytes, pararnn_stream stream);
+
+/* Workspace bytes of pararnn_affine_scan_host; 0 if the arguments are rejected. */
+PARARNN_API size_t pararnn_affine_scan_host_workspace_size(int B, int T, int D, int dense, int parts);
+
+/*
  * pararnn_affine_scan_noalloc -- the diagonal scan of pararnn_affine_scan
  * (dense == 0) for callers that cannot allocate device memory: plugins handed
  * only their input and output buffers, code running where an allocator must

@@ -33,7 +33,8 @@ EXPORTS = ("pararnn_workspace_size", "pararnn_newton_solve", "pararnn_newton_sol
            "pararnn_newton_solve_trace", "pararnn_test_withheld_publish", "pararnn_adjoint_exact",
            "pararnn_adjoint_exact_workspace_size", "pararnn_newton_solve_host_streamed",
            "pararnn_host_streamed_workspace_size", "pararnn_lstm_solve_host_streamed",
-           "pararnn_lstm_host_streamed_workspace_size")
+           "pararnn_lstm_host_streamed_workspace_size", "pararnn_affine_scan_host",
+           "pararnn_affine_scan_host_workspace_size")
 
 
 class Cell(ctypes.Structure):
@@ -82,6 +83,10 @@ def lib() -> ctypes.CDLL:
         L.pararnn_affine_scan.restype = ci
         L.pararnn_affine_scan_status.argtypes = [vp, vp]
         L.pararnn_affine_scan_status.restype = ci
+        L.pararnn_affine_scan_host.argtypes = [vp, vp, vp, ci, ci, ci, ci, vp, ci, vp, sz, vp]
+        L.pararnn_affine_scan_host.restype = ci
+        L.pararnn_affine_scan_host_workspace_size.argtypes = [ci, ci, ci, ci, ci]
+        L.pararnn_affine_scan_host_workspace_size.restype = sz
         L.pararnn_newton_solve_host.argtypes = [ctypes.POINTER(Cell), ctypes.POINTER(Params), vp, vp,
                                                 ci, ci, ci, cf, cf, ci, vp, vp, ci, vp, sz, vp]
         L.pararnn_newton_solve_host.restype = ci
@@ -694,4 +699,29 @@ def affine_scan(A, b, h0, *, out=None, workspace=None, stream=None, check: bool 
         st = L.pararnn_affine_scan_status(_dev(workspace, "workspace"), _stream(stream))
         if st != 0:
             raise RuntimeError(f"pararnn_affine_scan: {STATUS.get(st, st)}")
+    return out
+
+
+def affine_scan_host(A_host, b_host, h0_host, *, parts: int = 7, out=None, workspace=None, device=None,
+                     stream=None):
+    """The affine scan from and to HOST tensors (A [B,T,D] or [B,T,D,D], b
+    [B,T,D], h0 [B,D], fp32; page-locked for overlap), streamed through the
+    device in ``parts`` time parts (clamped to 1 .. ceil(T / 128)), each part
+    started from the previous part's last states.  Returns the host h."""
+    B, T, D = b_host.shape
+    dense = 1 if A_host.dim() == 4 else 0
+    parts = max(1, min(int(parts), (T + 127) // 128))
+    L = lib()
+    need = int(L.pararnn_affine_scan_host_workspace_size(B, T, D, dense, parts))
+    if need == 0:
+        raise ValueError("arguments rejected by pararnn_affine_scan_host_workspace_size")
+    if workspace is None:
+        workspace = alloc_workspace(need, device or "cuda")
+    if out is None:
+        out = torch.empty(B, T, D, dtype=torch.float32).pin_memory()
+    rc = L.pararnn_affine_scan_host(_host(A_host, "A_host"), _host(b_host, "b_host"), _host(h0_host, "h0_host"),
+                                    B, T, D, dense, _host(out, "out"), parts, _dev(workspace, "workspace"),
+                                    workspace.numel(), _stream(stream))
+    if rc != 0:
+        raise RuntimeError(f"pararnn_affine_scan_host: {L.pararnn_status_string(rc).decode()}")
     return out

@@ -1384,6 +1384,104 @@ int pararnn_lstm_solve_host_streamed(const pararnn_cell *cell, const pararnn_par
     return fold_reports(infos, parts, sc, info, true);
 }
 
+namespace {
+
+struct ScanStreamLayout {
+    int tmax, nbuf;
+    size_t scan, As[kHostBufs], bs[kHostBufs], hs[kHostBufs], h0, carry, stat, total;
+};
+
+ScanStreamLayout scan_stream_layout(int B, int T, int D, int dense, int parts) {
+    ScanStreamLayout H{};
+    for (int v : time_part_sizes(T, parts)) H.tmax = v > H.tmax ? v : H.tmax;
+    H.nbuf = parts < kHostBufs ? parts : kHostBufs;
+    const size_t n = static_cast<size_t>(B) * H.tmax * D * 4;
+    const size_t nA = n * (dense ? D : 1);
+    const size_t bd = static_cast<size_t>(B) * D * 4;
+    size_t off = 0;
+    H.scan = off; off = align256(off + pararnn_affine_scan_workspace_size(B, H.tmax, D, dense));
+    for (int q = 0; q < H.nbuf; ++q) { H.As[q] = off; off = align256(off + nA); }
+    for (int q = 0; q < H.nbuf; ++q) { H.bs[q] = off; off = align256(off + n); }
+    for (int q = 0; q < H.nbuf; ++q) { H.hs[q] = off; off = align256(off + n); }
+    H.h0 = off; off = align256(off + bd);
+    H.carry = off; off = align256(off + bd);
+    H.stat = off; off = align256(off + static_cast<size_t>(parts) * 4);
+    H.total = off;
+    return H;
+}
+
+}  // namespace
+
+size_t pararnn_affine_scan_host_workspace_size(int B, int T, int D, int dense, int parts) {
+    if (pararnn_affine_scan_workspace_size(B, T, D, dense) == 0 || parts < 1 || parts > (T + 127) / 128) return 0;
+    return scan_stream_layout(B, T, D, dense, parts).total;
+}
+
+int pararnn_affine_scan_host(const float *A_host, const float *b_host, const float *h0_host, int B, int T, int D,
+                             int dense, float *h_host, int parts, void *workspace, size_t ws_bytes,
+                             pararnn_stream stream) {
+    if (pararnn_affine_scan_workspace_size(B, T, D, dense) == 0 || parts < 1 || parts > (T + 127) / 128 ||
+        !A_host || !b_host || !h0_host || !h_host || !workspace || !aligned(workspace, 256))
+        return PARARNN_INVALID_ARG;
+    const ScanStreamLayout H = scan_stream_layout(B, T, D, dense, parts);
+    if (ws_bytes < H.total) return PARARNN_INVALID_ARG;
+    char *ws = static_cast<char *>(workspace);
+    const size_t hstep = static_cast<size_t>(D) * 4, astep = hstep * (dense ? D : 1);
+    const std::vector<int> sizes = time_part_sizes(T, parts);
+    cudaStream_t sc = reinterpret_cast<cudaStream_t>(stream);
+    float *h0_dev = reinterpret_cast<float *>(ws + H.h0), *carry = reinterpret_cast<float *>(ws + H.carry);
+    unsigned *stat = reinterpret_cast<unsigned *>(ws + H.stat);
+    const char *Ah = reinterpret_cast<const char *>(A_host), *bh = reinterpret_cast<const char *>(b_host);
+    char *hh = reinterpret_cast<char *>(h_host);
+    auto pre = [&](cudaStream_t s_in) {
+        return cudaMemcpyAsync(h0_dev, h0_host, B * hstep, cudaMemcpyHostToDevice, s_in);
+    };
+    // steps [t0, t0 + n) of every sequence, packed [B, n, .] in staging
+    auto cin = [&](int, int t0, int n, int buf, cudaStream_t s) {
+        cudaError_t e = cudaMemcpy2DAsync(ws + H.As[buf], n * astep, Ah + t0 * astep, T * astep, n * astep, B,
+                                          cudaMemcpyHostToDevice, s);
+        if (e == cudaSuccess)
+            e = cudaMemcpy2DAsync(ws + H.bs[buf], n * hstep, bh + t0 * hstep, T * hstep, n * hstep, B,
+                                  cudaMemcpyHostToDevice, s);
+        return e;
+    };
+    auto enq = [&](int p, int, int n, int buf) {
+        const float *hin = h0_dev;
+        cudaError_t e = cudaSuccess;
+        if (p > 0) {  // the state entering the part: each sequence's last state of the part before
+            const int pb = (p - 1) % H.nbuf, pn = sizes[p - 1];
+            e = cudaMemcpy2DAsync(carry, hstep, ws + H.hs[pb] + (pn - 1) * hstep, pn * hstep, hstep, B,
+                                  cudaMemcpyDeviceToDevice, sc);
+            hin = carry;
+        }
+        const Range range("pararnn: affine scan");
+        const float *Ap = reinterpret_cast<const float *>(ws + H.As[buf]);
+        const float *bp = reinterpret_cast<const float *>(ws + H.bs[buf]);
+        float *hp = reinterpret_cast<float *>(ws + H.hs[buf]);
+        if (e == cudaSuccess)
+            e = dense ? launch_scan_dense(Ap, bp, hin, B, n, D, hp, ws + H.scan, sc)
+                      : launch_scan_diag(Ap, bp, hin, B, n, D, hp, ws + H.scan, sc);
+        // the part's status word, kept before the next part's scan clears it
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(stat + p, &reinterpret_cast<const WsHeader *>(ws + H.scan)->status, 4,
+                                cudaMemcpyDeviceToDevice, sc);
+        return e == cudaSuccess ? static_cast<int>(PARARNN_OK) : static_cast<int>(PARARNN_CUDA_ERROR);
+    };
+    auto cout = [&](int, int t0, int n, int buf, cudaStream_t s) {
+        return cudaMemcpy2DAsync(hh + t0 * hstep, T * hstep, ws + H.hs[buf], n * hstep, n * hstep, B,
+                                 cudaMemcpyDeviceToHost, s);
+    };
+    const int rc = run_parts(sizes, H.nbuf, sc, pre, cin, enq, cout);
+    if (rc != PARARNN_OK) return rc;
+    std::vector<unsigned> host(parts);
+    cudaError_t e = cudaMemcpyAsync(host.data(), stat, parts * 4, cudaMemcpyDeviceToHost, sc);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(sc);
+    if (e != cudaSuccess) return PARARNN_CUDA_ERROR;
+    for (unsigned v : host)
+        if (v & kStatusTimeout) return PARARNN_TIMEOUT;
+    return PARARNN_OK;
+}
+
 size_t pararnn_lstm_host_workspace_size(const pararnn_cell *cell, int B, int T, int parts) {
     if (!lstm_cell_ok(cell, B, T) || parts < 1 || parts > B) return 0;
     return lstm_host_layout(*cell, B, T, parts).total;

@@ -143,6 +143,18 @@ def test_affine_scan_guard_bands(B, T, D, dense):
     for g in (A, b, h0, h, ws):
         assert g.bands_intact()
 
+    # the same from and to host memory, streamed in time parts
+    parts = min(3, (T + 127) // 128)
+    hA = Guarded(tuple(s.A.shape), torch.float32, device="cpu", init=s.A, pinned=True)
+    hb = Guarded(tuple(s.b.shape), torch.float32, device="cpu", init=s.b, pinned=True)
+    hh0 = Guarded(tuple(s.h0.shape), torch.float32, device="cpu", init=s.h0, pinned=True)
+    hh = Guarded((B, T, D), torch.float32, device="cpu", pinned=True)
+    wsh = _ws(int(binding.lib().pararnn_affine_scan_host_workspace_size(B, T, D, int(dense), parts)))
+    binding.affine_scan_host(hA.t, hb.t, hh0.t, parts=parts, out=hh.t, workspace=wsh.t)
+    assert _finite(hh.t) and _close(hh.t, ref)
+    for g in (hA, hb, hh0, hh, wsh):
+        assert g.bands_intact()
+
 
 def _adjoint_inputs(B, T, D, dense, seed):
     g = torch.Generator().manual_seed(seed)
