@@ -214,3 +214,32 @@ def test_streamed_full_size_sampled(name, over, mode, parts):
     for b in (0, w.B - 1):
         want = rollout(c, w.x[b:b + 1].double().numpy(), w.h0[b:b + 1].double().numpy())
         assert np.max(np.abs(r.h[b:b + 1].double().numpy() - want)) <= 1e-4
+
+
+def test_concurrent_host_calls_on_two_streams():
+    """Two host-buffer solves running at once from two host threads on two
+    streams: each call takes its own set of helper streams (the per-device
+    cache hands a set to one call at a time) and both results are right."""
+    import threading
+    ws_ = [make_workload("untrained", B=2, T=1500, h0_std=0.5, seed=s) for s in (1, 2)]
+    outs, errs = [None, None], []
+
+    def run(i):
+        try:
+            with torch.cuda.stream(torch.cuda.Stream()):
+                s = torch.cuda.current_stream()
+                outs[i] = _streamed(ws_[i], "QUASI", 3, stream=s) if i == 0 else _host_solve(ws_[i], "QUASI", 2,
+                                                                                           stream=s)
+        except Exception as e:  # reported on the main thread
+            errs.append(e)
+
+    th = [threading.Thread(target=run, args=(i,)) for i in (0, 1)]
+    for t in th:
+        t.start()
+    for t in th:
+        t.join()
+    assert not errs, errs
+    for w, r in zip(ws_, outs):
+        assert r.status == "OK"
+        c, x, h0 = _oracle(w)
+        assert np.max(np.abs(r.h.double().numpy() - rollout(c, x, h0))) <= 1e-4
