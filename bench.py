@@ -38,7 +38,15 @@ sys.path.insert(0, ROOT)
 
 METRIC = "converged states/sec (B*T*D per s, Newton to tol)"
 UNIT = "states/s"
-E2E_PARTS = 7  # parts (ramped sizes) whose copies the host-buffer calls overlap with the solves
+# Parts (ramped sizes) whose copies the host-buffer calls overlap with the solves.
+# Every part costs a solve's fixed overhead (a launch, and per iteration a grid
+# barrier and a pipeline refill), while the first part's copy in and the last
+# part's copy out overlap nothing: large copies against a short solve want
+# more parts, a short sequence with many iterations fewer.  Measured on the
+# streamed call (one B200): untrained GRU best at 7 (9.26 ms; 5: 9.54, 9: 9.53);
+# quasi-ELK (28 iterations, 5.1 M states) at 2 (4.52 ms; 7: 6.38); dense DEER
+# at 2 (3.20 ms; 7: 4.71).
+E2E_PARTS = 7
 # The benchmarked solves, one per row family of the hot path.  "untrained"
 # (the default) is the headline; the others measure the other solver kernels
 # with the same JSON line.  Roofline units per state and Newton iteration:
@@ -66,19 +74,19 @@ BENCHES = {
         workload="dense_deer", mode="DEER", lam=0.0, bound="tensor", per_state=None,
         kernel="deer_mma_kernel (persistent, all iterations)",
         desc="dense GRU Din=16, D=32, B={B}/GPU, T={T}, fp32 cell, TF32 Jacobian products, DEER tol 1e-5",
-        cpu_sample=dict(B=4, T=32768), ref_sample=dict(B=4, T=4096), roll_sample=dict()),
+        cpu_sample=dict(B=4, T=32768), ref_sample=dict(B=4, T=4096), roll_sample=dict(), e2e_parts=2),
     "quasi_elk": dict(
         workload="near_unstable", mode="QUASI_ELK", lam=0.1, bound="hbm", per_state=56,
         kernel="quasi_tc2_kernel<64, quasi-ELK> (persistent, all iterations)",
         desc="near-unstable dense GRU Din=D=64 (spectral radius 1.5), B={B}/GPU, T={T}, fp32, "
              "quasi-ELK lambda 0.1, tol 1e-4",
-        cpu_sample=dict(B=8, T=8000), ref_sample=dict(B=2, T=2000), roll_sample=dict()),
+        cpu_sample=dict(B=8, T=8000), ref_sample=dict(B=2, T=2000), roll_sample=dict(), e2e_parts=2),
     "elk": dict(
         workload="near_unstable", mode="ELK", lam=0.01, bound="alu", per_state=None,
         kernel="dense_elk_kernel<64> (persistent, all iterations)",
         desc="near-unstable dense GRU Din=D=64 (spectral radius 1.5), B={B}/GPU, T={T}, fp32, "
              "ELK lambda 0.01, tol 1e-4",
-        cpu_sample=dict(B=1, T=5000), ref_sample=dict(B=1, T=1000), roll_sample=dict()),
+        cpu_sample=dict(B=1, T=5000), ref_sample=dict(B=1, T=1000), roll_sample=dict(), e2e_parts=2),
     # the backward pass through the evaluated diagonal-cell sequence (not a solve):
     # reads P 12 + h 4 + dL/dh 4, writes dL/dP 12 = 32 B per state
     "adjoint": dict(
@@ -730,7 +738,7 @@ def bench_solve(args, name: str, *, full: bool = True, steps: int | None = None)
     iters = max(step_iters)
 
     e2e = None
-    parts = max(1, min(E2E_PARTS, (T + 127) // 128)) if k == 1 else 1
+    parts = max(1, min(spec.get("e2e_parts", E2E_PARTS), (T + 127) // 128)) if k == 1 else 1
     if full:
         # end to end through the public host-buffer call: page-locked x and h0 in,
         # h out; the library streams the sequence through the device in time
