@@ -252,7 +252,9 @@ __device__ __forceinline__ void prefetch_p(const float *P, long long tile, int B
 // segments of a lane are chained through shared memory and tiles through
 // look-back (covariance, mean forward; smoother backward).
 
-constexpr int kElkWin = 3;  // predecessors each look-back thread reads per round trip
+// predecessors each look-back thread reads per round trip (near-unstable GRU,
+// B = 8, T = 10000: 1 -> 3.54 ms per solve, 2 -> 3.77, 3 -> 3.87, 5 -> 4.49, 8 -> 4.90)
+constexpr int kElkWin = 1;
 
 struct ElkSmem {
     float *mob;   // [SEGS][D][4] segment Moebius maps, then exclusive prefixes
