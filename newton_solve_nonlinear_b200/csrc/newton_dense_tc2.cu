@@ -26,7 +26,7 @@
 // without leaving registers: Kogge-Stone over the 8 steps a quad column holds
 // (warp shuffles), a 4-group prefix inside the thread, a 4-warp prefix through
 // shared memory, and the tile's carry-in by decoupled look-back over earlier
-// chunks of the sequence.  Every state is then final and is stored with the
+// chunks of the sequence (one thread per lane).  Every state is then final and is stored with the
 // convergence maxima max |h^(i+1) - h^(i)| and max |h_t - f_t|.
 // Traffic per state and iteration: P (12 B), the guess (4 B, by TMA),
 // h^(i+1) (4 B).  A bounded grid barrier ends each iteration.
@@ -788,11 +788,14 @@ quasi_tc2_kernel(const __grid_constant__ CUtensorMap map_h0, const __grid_consta
                 }
             }
             __syncthreads();
-            // 4c. the tile's carry-in per lane by look-back over earlier chunks;
-            // every thread takes part (G per lane)
-            {
-                constexpr int GL = NTHREADS / D;
-                const int d = tid / GL, q = tid % GL;
+            // 4c. the tile's carry-in per lane by look-back over earlier chunks: one
+            // thread per lane (threads 0 .. D-1; the rest go on to the barrier).
+            // Threads per lane, measured on the untrained workload (ms per solve):
+            // 8 (all 512 threads) 7.19, 4 6.74, 2 6.68, 1 6.65 -- the wider groups'
+            // shuffles and ballots cost more issue slots than their reads save
+            if (tid < D) {
+                constexpr int GL = 1;
+                const int d = tid, q = 0;
                 float EA = wt_a[d], EB = wt_b[d];
 #pragma unroll
                 for (int qq = 1; qq < 4; ++qq) {
