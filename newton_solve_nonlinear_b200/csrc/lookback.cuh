@@ -17,9 +17,11 @@ namespace pararnn {
 // value in one 64-bit word, and each (epoch, state) value is written once, so a
 // word whose tag matches *is* the value: no acquire/release ordering is needed
 // between words.  The look-back therefore reads predecessors with relaxed
-// loads in batches of up to kWin tiles, which resolves a chain of aggregates in
-// about one L2 round trip per batch instead of one per tile.
-constexpr int kWin = 4;
+// loads, kWin tiles per L2 round trip.  One per round trip measured fastest
+// (standalone scan [16, 65536, 64], us per scan: 4 -> 170, 2 -> 166, 1 -> 162):
+// the predecessors in one wave publish within about a round trip of each other,
+// so a wider batch rarely saves a round trip and costs instructions.
+constexpr int kWin = 1;
 
 __device__ __forceinline__ bool word_ready(unsigned long long w, unsigned epoch) {
     const unsigned t = word_tag(w);

@@ -18,8 +18,8 @@
 // of (sequence, 64 lanes, 32 steps), chunk-major; thread (lane d, segment s)
 // owns 8 consecutive steps: it evaluates the cell and its 2x2 Jacobian at the
 // shifted guess, composes its steps' affine maps, the four segments of a lane
-// chain through shared memory, and a cooperative look-back over earlier
-// chunks (2x2 maps, four threads per lane) gives the tile's entering state.
+// chain through shared memory, and a decoupled look-back over earlier
+// chunks (2x2 maps, one thread per lane) gives the tile's entering state.
 // The sweep writes the new iterate and the convergence maxima
 // max |s^(i+1) - s^(i)| (both halves of the state) and max |s^(i) - F|.
 // Traffic per lane-step and iteration: P (16 B), the guess (c, h: 8 B read,
@@ -227,7 +227,9 @@ __global__ void __launch_bounds__(LNT, 2) lstm_diag_kernel(LstmArgs S) {
     unsigned *status = &hdr->status;
     const int tid = threadIdx.x;
     const int d = tid & (LDL - 1), seg = tid / LDL;   // sweep role
-    const int ld = tid / LSEGS, lq = tid % LSEGS;     // look-back role
+    // look-back threads per lane (diagonal LSTM workload, ms per solve: 4 -> 6.78, 2 -> 6.53, 1 -> 6.42)
+    constexpr int LLB = 1;
+    const int ld = tid / LLB, lq = tid % LLB;         // look-back role (tid < LDL * LLB)
     const unsigned nblocks = gridDim.x;
 
     int iters = 0, final_status = PARARNN_NOT_CONVERGED;
@@ -309,7 +311,7 @@ __global__ void __launch_bounds__(LNT, 2) lstm_diag_kernel(LstmArgs S) {
                 break;
             }
             // 2. the state entering the tile, by look-back over earlier chunks
-            {
+            if (tid < LDL * LLB) {
                 M2 E = m2_identity();
 #pragma unroll
                 for (int q = 0; q < LSEGS; ++q)
@@ -321,7 +323,7 @@ __global__ void __launch_bounds__(LNT, 2) lstm_diag_kernel(LstmArgs S) {
                 if (chunk == 0 && ln < D)
                     s0 = make_float2(__ldg(S.c0 + static_cast<size_t>(b) * D + ln),
                                      __ldg(S.h0 + static_cast<size_t>(b) * D + ln));
-                const float2 sin = coop_lookback_m2<LSEGS, LWIN>(S.desc, v, S.ngroups, LDL, ld, lq, epoch, E, chunk,
+                const float2 sin = coop_lookback_m2<LLB, LWIN>(S.desc, v, S.ngroups, LDL, ld, lq, epoch, E, chunk,
                                                                  s0, status);
                 if (lq == 0) carry[0][ld] = sin.x, carry[1][ld] = sin.y;
             }

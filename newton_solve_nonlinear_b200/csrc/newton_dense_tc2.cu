@@ -250,10 +250,12 @@ __device__ __forceinline__ void prefetch_p(const float *P, long long tile, int B
 // The covariance step is the Moebius map [[a^2, 1], [lambda a^2, 1 + lambda]].
 // Inside a tile, thread (lane d, segment g) walks SLE consecutive steps; the
 // segments of a lane are chained through shared memory and tiles through
-// look-back (covariance, mean forward; smoother backward).
+// look-back (covariance, mean forward; smoother backward), one thread per lane
+// (near-unstable GRU, B = 8, T = 10000, ms per solve: 8 threads per lane 3.62,
+// one 3.18).
 
-// predecessors each look-back thread reads per round trip (near-unstable GRU,
-// B = 8, T = 10000: 1 -> 3.54 ms per solve, 2 -> 3.77, 3 -> 3.87, 5 -> 4.49, 8 -> 4.90)
+// predecessors each look-back thread reads per round trip (same workload, with
+// 8 threads per lane: 1 -> 3.54 ms per solve, 2 -> 3.77, 3 -> 3.87, 5 -> 4.49, 8 -> 4.90)
 constexpr int kElkWin = 1;
 
 struct ElkSmem {
@@ -293,15 +295,15 @@ __device__ void elk_forward_scans(const DiagArgs &A, const ElkSmem &E, const uns
         mm[0] = M.m0; mm[1] = M.m1; mm[2] = M.m2; mm[3] = M.m3;
     }
     __syncthreads();
-    {  // covariance entering the tile: all threads, SEGS per lane
-        const int ld = tid / SEGS, lq = tid % SEGS;
+    if (tid < D) {  // covariance entering the tile: one thread per lane
+        const int ld = tid, lq = 0;
         Mob Ex{1.f, 0.f, 0.f, 1.f};
         for (int q = 0; q < SEGS; ++q) {
             const float *qm = E.mob + (q * D + ld) * 4;
             Ex = mob_mul(Mob{qm[0], qm[1], qm[2], qm[3]}, Ex);
         }
-        const float pin = coop_lookback_mob<SEGS, kElkWin>(desc_cov, tile, B, D, ld, lq, epoch, Ex, chunk,
-                                                           0.f, status);
+        const float pin = coop_lookback_mob<1, kElkWin>(desc_cov, tile, B, D, ld, lq, epoch, Ex, chunk,
+                                                        0.f, status);
         if (lq == 0) E.cP[ld] = pin;
     }
     __syncthreads();
@@ -339,8 +341,8 @@ __device__ void elk_forward_scans(const DiagArgs &A, const ElkSmem &E, const uns
         fa[1] = SB;
     }
     __syncthreads();
-    {  // mean entering the tile
-        const int ld = tid / SEGS, lq = tid % SEGS;
+    if (tid < D) {  // mean entering the tile: one thread per lane
+        const int ld = tid, lq = 0;
         float EA = 1.f, EB = 0.f;
         for (int q = 0; q < SEGS; ++q) {
             const float *qa = E.aff + (q * D + ld) * 2;
@@ -348,8 +350,8 @@ __device__ void elk_forward_scans(const DiagArgs &A, const ElkSmem &E, const uns
             EA = qa[0] * EA;
         }
         const float c0 = chunk == 0 ? __ldg(A.h0 + static_cast<size_t>(b) * D + ld) : 0.f;
-        const float min_ = coop_lookback<SEGS, kElkWin>(desc_mean, tile, B, D, ld, lq, epoch, EA, EB, chunk,
-                                                        c0, status);
+        const float min_ = coop_lookback<1, kElkWin>(desc_mean, tile, B, D, ld, lq, epoch, EA, EB, chunk,
+                                                     c0, status);
         if (lq == 0) E.cM[ld] = min_;
     }
     __syncthreads();
@@ -434,16 +436,16 @@ __device__ void elk_backward_tile(const DiagArgs &A, const ElkSmem &E, long long
         fa[1] = cC;
     }
     __syncthreads();
-    {  // state after the tile (from the next chunk), all threads
-        const int ld = tid / SEGS, lq = tid % SEGS;
+    if (tid < D) {  // state after the tile (from the next chunk): one thread per lane
+        const int ld = tid, lq = 0;
         float EG = 1.f, EC = 0.f;
         for (int q = SEGS - 1; q >= 0; --q) {
             const float *qa = E.aff + (q * D + ld) * 2;
             EC = fmaf(qa[0], EC, qa[1]);
             EG = qa[0] * EG;
         }
-        const float sin_ = coop_lookback<SEGS, kElkWin>(desc_bwd, tile, -static_cast<long long>(B), D, ld, lq,
-                                                        epoch, EG, EC, n_chunks - 1 - chunk, 0.f, status);
+        const float sin_ = coop_lookback<1, kElkWin>(desc_bwd, tile, -static_cast<long long>(B), D, ld, lq,
+                                                     epoch, EG, EC, n_chunks - 1 - chunk, 0.f, status);
         if (lq == 0) E.cM[ld] = sin_;
     }
     __syncthreads();

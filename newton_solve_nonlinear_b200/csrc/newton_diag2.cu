@@ -16,7 +16,7 @@
 // Thread (lane d, segment s) owns 8 consecutive steps of one lane: it
 // evaluates the cell and a_t, b_t (b_t = f_t - a_t h_{t-1}), composes its 8
 // maps, the 4 segments of a lane are chained through shared memory, the
-// tile's carry-in per lane comes from a cooperative look-back (4 threads per
+// tile's carry-in per lane comes from a decoupled look-back (one thread per
 // lane), and every state is swept and stored with the convergence maxima
 // max |h^(i+1) - h^(i)| and max |h_t - f_t|.
 // Traffic per state and iteration: P (12 B), the guess (4 B), h^(i+1) (4 B).
@@ -101,7 +101,9 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
     const unsigned nblocks = gridDim.x;
     const int tid = threadIdx.x;
     const int d = tid & (DL - 1), seg = tid / DL;  // sweep role: lane, segment
-    const int ld = tid / SEGS, lq = tid % SEGS;     // look-back role: lane, rank
+    // look-back threads per lane (diagonal workload, us per iteration: 4 -> 362, 2 -> 339, 1 -> 325)
+    constexpr int LBG = 1;
+    const int ld = tid / LBG, lq = tid % LBG;       // look-back role: lane, rank (tid < DL * LBG)
     const int jq = (d & 31) >> 2;                   // 16-byte chunk of lane d in a 128-byte row
 
     if (tid == 0) {
@@ -206,14 +208,15 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
                 hp = y1;
             }
             // the predecessors' descriptors, on their way during the barrier
-            const LookbackWindow<1> lbw = coop_lookback_prefetch<SEGS>(A.desc, tile, S.ngroups, DL, ld, lq, chunk);
+            LookbackWindow<1> lbw{};
+            if (tid < DL * LBG) lbw = coop_lookback_prefetch<LBG>(A.desc, tile, S.ngroups, DL, ld, lq, chunk);
             seg_a[seg * DL + d] = EA;
             seg_b[seg * DL + d] = EB;
             __syncthreads();
             if (*cta_err != 0) break;  // uniform: read after the barrier
 
-            // 2. tile carry-in per lane (8 threads per lane)
-            {
+            // 2. tile carry-in per lane (LBG threads per lane)
+            if (tid < DL * LBG) {
                 float TA = 1.f, TB = 0.f;
 #pragma unroll
                 for (int q = 0; q < SEGS; ++q) {
@@ -223,7 +226,7 @@ diag2_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ 
                 }
                 const float c0 = chunk == 0 ? __ldg(A.h0 + static_cast<size_t>(b) * D + lane0 + ld) : 0.f;
                 const float hin =
-                    coop_lookback<SEGS, 1, true>(A.desc, tile, S.ngroups, DL, ld, lq, epoch, TA, TB, chunk, c0,
+                    coop_lookback<LBG, 1, true>(A.desc, tile, S.ngroups, DL, ld, lq, epoch, TA, TB, chunk, c0,
                                                  status, &lbw, publishes(A, tile, epoch));
                 if (lq == 0) carry[ld] = hin;
             }
