@@ -115,3 +115,31 @@ def test_reuse_and_adjoint_size_queries(L):
                                             2, 100) == 0
     assert L.pararnn_adjoint_host_workspace_size(ctypes.byref(dense64), 4, 100, 3) > 0
     assert L.pararnn_adjoint_host_workspace_size(ctypes.byref(dense64), 4, 100, 5) == 0
+
+
+@pytest.mark.parametrize("T,parts,largest", [(65536, 7, 16384), (1000, 3, 512), (300, 3, 128), (129, 2, 128),
+                                             (4096, 7, 1024), (1, 1, 1)])
+def test_streamed_host_part_sizes(L, T, parts, largest):
+    """The streamed calls split T in 128-step units with the ramped weights
+    (T = 65536 in 7 parts: 4096, 8192, 12288, 16384, ...); their workspace is
+    one solve (or scan) workspace for the longest part, three staging buffers
+    (fewer when there are fewer parts) of that part for every sequence, h0 and
+    the carry for the batch, and one report per part.  parts > ceil(T / 128)
+    is rejected."""
+    B, din, d = 4, 64, 64
+    cell = binding.make_cell("dense", din, d, binding.torch.float32)
+    m = binding.MODES["QUASI"]
+    solve = L.pararnn_workspace_size(ctypes.byref(cell), B, largest, m)
+    nbuf = min(parts, 3)
+    want = (_al(solve) + nbuf * _al(B * largest * din * 4) + nbuf * _al(B * largest * d * 4) + 2 * _al(B * d * 4)
+            + _al(parts * 16))
+    assert L.pararnn_host_streamed_workspace_size(ctypes.byref(cell), B, T, m, parts) == want
+    assert L.pararnn_host_streamed_workspace_size(ctypes.byref(cell), B, T, m, (T + 127) // 128 + 1) == 0
+    # the scan from host memory: A, b and h staged per part, h0 and the carry, a status word per part
+    scan = L.pararnn_affine_scan_workspace_size(B, largest, d, 0)
+    want_scan = (_al(scan) + 3 * nbuf * _al(B * largest * d * 4) + 2 * _al(B * d * 4) + _al(parts * 4))
+    assert L.pararnn_affine_scan_host_workspace_size(B, T, d, 0, parts) == want_scan
+    assert L.pararnn_affine_scan_host_workspace_size(B, T, d, 0, (T + 127) // 128 + 1) == 0
+    lstm = binding.make_cell("lstm_diag", din, d, binding.torch.float32)
+    assert L.pararnn_lstm_host_streamed_workspace_size(ctypes.byref(lstm), B, T, parts) > 0
+    assert L.pararnn_lstm_host_streamed_workspace_size(ctypes.byref(lstm), B, T, (T + 127) // 128 + 1) == 0
